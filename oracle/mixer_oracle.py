@@ -1,0 +1,144 @@
+"""ctypes wrapper around the plain C oracle (mixer_oracle.c).  TEST INFRASTRUCTURE ONLY.
+
+``build()`` compiles the C file with gcc; ``mixer()`` runs the oracle on numpy arrays.
+The arithmetic lives entirely in mixer_oracle_impl.h (a sequential restatement of the
+calm-mamba 0.1.4 "Mamba operator" steps 2, 4, 5 and 6); this module only converts
+arrays and passes pointers.
+
+Parity status: pinned.  tests/test_oracle_pins.py checks this oracle against closed
+forms, library routines (numpy.convolve, numpy.logaddexp, scipy.special.expit,
+numpy.cumsum) and an O(L^2) brute-force unrolled sum.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mixer_oracle.c")
+_IMPL = os.path.join(_HERE, "mixer_oracle_impl.h")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_BUILD, "liboracle_mixer.so")
+
+GCC_FLAGS = ["-O2", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+             "-Wall", "-Wextra"]
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc into oracle/_build/liboracle_mixer.so."""
+    os.makedirs(_BUILD, exist_ok=True)
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_IMPL))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+        for name in ("oracle_mixer_f64", "oracle_mixer_f32"):
+            fn = getattr(lib, name)
+            fn.restype = ci
+            fn.argtypes = [i64] * 5 + [vp] * 15 + [ci]
+        lib.oracle_max_threads.restype = ci
+        lib.oracle_max_threads.argtypes = []
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _arr(a, dt):
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
+          h_in=None, conv_state_in=None, precision: str = "f64",
+          nthreads: int = 1) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Run the oracle.
+
+    Arrays are numeric numpy arrays (already widened from bf16 where that applies) in
+    the layouts of mixer_oracle.c.  ``conv_b``, ``h_in`` and ``conv_state_in`` may be
+    None (zero bias; zero initial state).  Returns (y [Bt,L,Di], h_out [Bt,Di,N],
+    conv_state_out [Bt,Di,K-1]) in the requested precision ("f64" or "f32").
+    """
+    dt = {"f64": np.float64, "f32": np.float32}[precision]
+    fn = getattr(_load(), f"oracle_mixer_{precision}")
+    xp, z, dt_raw = _arr(xp, dt), _arr(z, dt), _arr(dt_raw, dt)
+    B, C = _arr(B, dt), _arr(C, dt)
+    A_log, D, conv_w = _arr(A_log, dt), _arr(D, dt), _arr(conv_w, dt)
+    conv_b, dt_bias = _arr(conv_b, dt), _arr(dt_bias, dt)
+    h_in, conv_state_in = _arr(h_in, dt), _arr(conv_state_in, dt)
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    assert z.shape == xp.shape and dt_raw.shape == xp.shape
+    assert B.shape == (Bt, L, N) and C.shape == (Bt, L, N)
+    assert A_log.shape == (Di, N) and D.shape == (Di,) and dt_bias.shape == (Di,)
+    assert conv_b is None or conv_b.shape == (Di,)
+    assert h_in is None or h_in.shape == (Bt, Di, N)
+    assert conv_state_in is None or conv_state_in.shape == (Bt, Di, K - 1)
+    y = np.empty((Bt, L, Di), dtype=dt)
+    h_out = np.empty((Bt, Di, N), dtype=dt)
+    cs_out = np.empty((Bt, Di, K - 1), dtype=dt)
+    rc = fn(Bt, L, Di, N, K, _ptr(xp), _ptr(z), _ptr(dt_raw), _ptr(B), _ptr(C), _ptr(A_log),
+            _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(h_in),
+            _ptr(conv_state_in), _ptr(y), _ptr(h_out), _ptr(cs_out), int(nthreads))
+    if rc != 0:
+        raise RuntimeError(f"oracle failed with code {rc}")
+    return y, h_out, cs_out
+
+
+def mixer_channels(inp: dict, batch_idx, chan_idx, precision: str = "f64",
+                   nthreads: int = 1, widen=None):
+    """Oracle over a subset of channels of one workload's inputs.
+
+    Every channel (b, d) of the mixer is independent given B[b], C[b] and the
+    parameters of d, so the selected channels form a smaller problem: batch rows
+    ``batch_idx`` and channels ``chan_idx`` (all pairs).  ``widen`` maps a stored
+    activation to float64 (bf16 bit patterns are widened exactly).  Returns the outputs
+    of the sub-problem with shapes [len(batch_idx), L, len(chan_idx)] etc.
+    """
+    bi = np.asarray(batch_idx)
+    di = np.asarray(chan_idx)
+    w = widen or (lambda a: np.asarray(a, dtype=np.float64))
+    sub = {
+        "xp": w(inp["xp"][bi][:, :, di]),
+        "z": w(inp["z"][bi][:, :, di]),
+        "dt_raw": w(inp["dt_raw"][bi][:, :, di]),
+        "B": w(inp["B"][bi]),
+        "C": w(inp["C"][bi]),
+        "A_log": inp["A_log"][di],
+        "D": inp["D"][di],
+        "conv_w": inp["conv_w"][di],
+        "conv_b": None if inp.get("conv_b") is None else inp["conv_b"][di],
+        "dt_bias": inp["dt_bias"][di],
+    }
+    h_in = inp.get("h")
+    cs_in = inp.get("conv_state")
+    if h_in is not None:
+        h_in = h_in[bi][:, di]
+    if cs_in is not None:
+        cs_in = w(cs_in[bi][:, di])
+    return mixer(sub["xp"], sub["z"], sub["dt_raw"], sub["B"], sub["C"], sub["A_log"],
+                 sub["D"], sub["conv_w"], sub["conv_b"], sub["dt_bias"], h_in, cs_in,
+                 precision=precision, nthreads=nthreads)
