@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the fused selective-SSM mixer core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload m130|long|decode|stress|tiny]
+
+One step = one pass of the whole hot path over one batch: the fused forward
+(conv+SiLU, softplus, selective scan with the chunk carry, gate, state out) over the
+workload's prompt, then one decode step per sequence on the state the forward left
+(in place).  ``--workload decode`` times the decode step alone on its own shapes.
+
+Prints ONE JSON line (rank 0).  ``value`` is achieved algorithmic HBM GB/s over all
+ranks: algorithmic bytes (each input read once, each output written once) divided by
+the device time of the K timed steps (CUDA events on the launching stream, L2 flushed
+between steps, max over ranks).  ``--impl reference`` times the CPU oracle instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_state_space_silu_b200 import inputs as I  # noqa: E402
+
+METRIC = "fused conv+selective-scan+gate: achieved HBM GB/s and % of B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- bytes
+def fwd_bytes(w: I.Workload) -> int:
+    s = w.io_bytes
+    Bt, L, Di, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    return (4 * Bt * L * Di * s            # x', z, dt_raw in; y out
+            + 2 * Bt * L * N * s           # B, C
+            + Di * (4 * N + 28)            # A_log, D, conv_w, conv_b, dt_bias
+            + Bt * Di * N * 4              # h out
+            + Bt * Di * 3 * s)             # conv state out
+
+
+def step_bytes(w: I.Workload) -> int:
+    s = w.io_bytes
+    Bt, Di, N = w.batch, w.d_inner, w.d_state
+    return (Bt * Di * (2 * N * 4 + 2 * 3 * s + 4 * s)   # h in/out, conv state in/out, x' z dt y
+            + 2 * Bt * N * s                          # B, C of the token
+            + Di * (4 * N + 28))
+
+
+def workload_bytes(w: I.Workload) -> dict:
+    if w.decode:
+        return {"fwd": 0, "step": step_bytes(w)}
+    return {"fwd": fwd_bytes(w), "step": step_bytes(w.with_(seqlen=1))}
+
+
+# ----------------------------------------------------------------------------- misc
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "selective_state_space_silu_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per forward launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"fwd_{workload}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if ":" in line:
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    try:
+        return int(float(kv["dram_bytes_per_fwd_call"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self) -> dict:
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                             "hw": parts[5], "hwt": parts[6], "swt": parts[7], "pc": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        load = [r for r in rows if r["sm"] > 0.5 * r["max"]] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pc", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- ours
+def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_silu_b200 import mixer as M
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M.load_library()
+    inp = I.make_inputs(w)
+    tok_w = w.with_(seqlen=1, decode=True, seed=w.seed + 7919)
+    tok = I.make_inputs(tok_w)     # the decode token (its h / conv_state are unused)
+
+    def td(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    P = {k: td(inp[k]) for k in ("A_log", "D", "conv_w", "conv_b", "dt_bias")}
+    X = {k: td(inp[k]) for k in ("xp", "z", "dt_raw", "B", "C")}
+    T = {k: td(tok[k]) for k in ("xp", "z", "dt_raw", "B", "C")}
+    Bt, L, Di, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    iot = X["xp"].dtype
+    stream = torch.cuda.current_stream(dev)
+    if w.decode:
+        h = td(inp["h"])
+        cs = td(inp["conv_state"])
+        y = torch.empty((Bt, 1, Di), dtype=iot, device=dev)
+        ws = None
+        X = T = {k: td(inp[k]) for k in ("xp", "z", "dt_raw", "B", "C")}
+    else:
+        y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
+        h = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+        cs = torch.empty((Bt, Di, 3), dtype=iot, device=dev)
+        need = M.mamba_mixer_fwd_workspace_bytes(M.make_dims(Bt, L, Di, N, 4, M._io_code(X["xp"])))
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    yt = torch.empty((Bt, 1, Di), dtype=iot, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def fwd():
+        M.mamba_mixer_fwd(X["xp"], X["z"], X["dt_raw"], X["B"], X["C"], P["A_log"], P["D"],
+                          P["conv_w"], P["conv_b"], P["dt_bias"], y=y, h_out=h,
+                          conv_state_out=cs, workspace=ws, stream=stream)
+
+    def step():
+        M.mamba_mixer_step(T["xp"], T["z"], T["dt_raw"], T["B"], T["C"], P["A_log"], P["D"],
+                           P["conv_w"], P["conv_b"], P["dt_bias"], h, cs, y=yt, h_out=h,
+                           conv_state_out=cs, stream=stream)
+
+    launches_fwd = 0 if w.decode else M.launches_per_fwd(M.make_dims(Bt, L, Di, N, 4, M._io_code(X["xp"])))
+    launches_per_step = launches_fwd + 1
+
+    def one_step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        if not w.decode:
+            fwd()
+        if ev is not None:
+            ev[1].record(stream)
+        step()
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        one_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(1.0)        # L2 flush (not timed)
+            one_step(evs[i])
+        torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+
+    # end to end through the public API: pinned host inputs -> device -> mixer -> host
+    e2e = None
+    if rank == 0 or world > 1:
+        hx = {k: v.cpu().pin_memory() for k, v in X.items()}
+        ht = {k: v.cpu().pin_memory() for k, v in T.items()}
+        hy = torch.empty(y.shape, dtype=iot).pin_memory()
+        hyt = torch.empty(yt.shape, dtype=iot).pin_memory()
+        hh = torch.empty(h.shape, dtype=torch.float32).pin_memory()
+        hcs = torch.empty(cs.shape, dtype=iot).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hx.values())
+        if not w.decode:
+            h2d += sum(v.numel() * v.element_size() for v in ht.values())
+        d2h = (0 if w.decode else hy.numel() * hy.element_size()) + hyt.numel() * hyt.element_size() \
+            + hh.numel() * 4 + hcs.numel() * hcs.element_size()
+        if w.decode:
+            h2d += hh.numel() * 4 + hcs.numel() * hcs.element_size()
+            hh0, hcs0 = h.cpu().pin_memory(), cs.cpu().pin_memory()
+        e2e_steps = max(3, min(args.steps, 50))
+        ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+        for i in range(e2e_steps + 2):
+            flush.fill_(1.0)
+            if i >= 2:
+                ev0[i - 2].record(stream)
+            for k in X:
+                X[k].copy_(hx[k], non_blocking=True)
+            if not w.decode:
+                for k in T:
+                    T[k].copy_(ht[k], non_blocking=True)
+            else:
+                h.copy_(hh0, non_blocking=True)
+                cs.copy_(hcs0, non_blocking=True)
+            one_step()
+            if not w.decode:
+                hy.copy_(y, non_blocking=True)
+            hyt.copy_(yt, non_blocking=True)
+            hh.copy_(h, non_blocking=True)
+            hcs.copy_(cs, non_blocking=True)
+            if i >= 2:
+                ev1[i - 2].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"ms_per_step": e2e_ms / e2e_steps, "h2d": h2d, "d2h": d2h}
+
+    bytes_ = workload_bytes(w)
+    step_total = bytes_["fwd"] + bytes_["step"]
+    if rank != 0:
+        return None
+    peaks = measured_peaks()
+    value = world * step_total * args.steps / (total_ms * 1e-3) / 1e9
+    # dominant kernel: the forward call (the decode step when timing decode alone)
+    if w.decode:
+        dom_ms = statistics.mean(dec_ms)
+        dom_bytes = bytes_["step"]
+        dom = "mamba_mixer_step"
+    else:
+        dom_ms = statistics.mean(fwd_ms)
+        dom_bytes = bytes_["fwd"]
+        dom = "mamba_mixer_fwd"
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    clocks = clk.summary()
+    e2e_val = world * step_total / (e2e["ms_per_step"] * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name) if not w.decode else None
+    return {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.io_dtype == I.BF16 else "f32",
+        "data": "synthetic (seeded; shapes and distributions of the pages' workloads)",
+        "config": {
+            "workload": w.name,
+            "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.d_inner, "d_state": w.d_state,
+            "d_conv": w.d_conv, "io": w.io_dtype, "state": "f32",
+            "step": "decode step only" if w.decode else "fused forward over the prompt + one decode step (state in place)",
+            "global_batch": w.batch * world,
+            "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
+            "l2": "flushed between timed steps (256 MiB write, outside the timed events)",
+            "algorithmic_bytes_per_step": step_total,
+        },
+        "tokens_channels_per_s": round(world * w.batch * w.seqlen * w.d_inner * args.steps
+                                        / (total_ms * 1e-3), 1),
+        "fwd_ms_mean": round(statistics.mean(fwd_ms), 5) if not w.decode else None,
+        "decode_ms_mean": round(statistics.mean(dec_ms), 5),
+        "roofline": {
+            "kernel": dom,
+            "bound": "hbm",
+            "achieved": round(achieved, 2),
+            "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured" else "fallback",
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic,
+            "algorithmic_bytes_per_launch": dom_bytes,
+            "avg_launch_ms": round(dom_ms, 5),
+        },
+        "e2e": {"value": round(e2e_val, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": round(e2e["ms_per_step"], 4)},
+        "gpu_launches": launches_per_step * args.steps if not w.decode else args.steps,
+        "clocks": clocks,
+    }
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample(w: I.Workload, target_s: float):
+    """Times the CPU oracle, as it stands, on a bounded sample of the workload: all batch
+    rows, a subset of channels, the full sequence.  Returns (GB/s, cores, description)."""
+    from oracle import mixer_oracle as O
+    O.build()
+    cores = O.max_threads()
+    inp = I.make_inputs(w)
+    Bt, L, Di = w.batch, w.seqlen, w.d_inner
+    per = workload_bytes(w)
+    bytes_per_tc = (per["fwd"] + per["step"]) / (Bt * L * Di)
+    # size the sample from a quick probe so one pass takes about target_s
+    probe = np.arange(min(Di, 8))
+    t0 = time.perf_counter()
+    O.mixer_channels(inp, np.arange(Bt), probe, widen=I.as_f64, nthreads=0)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    nch = int(min(Di, max(8, len(probe) * target_s / dt)))
+    chans = np.linspace(0, Di - 1, nch).astype(np.int64)
+    t0 = time.perf_counter()
+    O.mixer_channels(inp, np.arange(Bt), chans, widen=I.as_f64, nthreads=0)
+    el = time.perf_counter() - t0
+    tc = Bt * L * nch
+    gbs = tc / el * bytes_per_tc / 1e9
+    desc = (f"{w.name}: all {Bt} batch rows x {nch} of {Di} channels x L={L} "
+            f"({tc} token-channels, fp64 oracle, {el:.2f} s)")
+    return gbs, cores, desc, el
+
+
+def run_reference(args, w: I.Workload, rank: int):
+    if rank != 0:
+        return None
+    vals = []
+    desc = ""
+    cores = 1
+    for _ in range(max(1, args.warmup and 1)):
+        oracle_sample(w, 1.0)
+    for _ in range(args.steps):
+        gbs, cores, desc, _ = oracle_sample(w, max(2.0, 20.0 / max(args.steps, 1)))
+        vals.append(gbs)
+    v = statistics.mean(vals)
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                   "d_inner": w.d_inner, "d_state": w.d_state},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="m130", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    w = I.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        res = run_reference(args, w, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, w, rank, world, local_rank)
+        if res is not None:
+            if not args.no_cpu_baseline:
+                gbs, cores, desc, _ = oracle_sample(w, 10.0)
+                res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                       "kind": "oracle", "sample": desc}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

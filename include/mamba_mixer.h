@@ -1,0 +1,147 @@
+/*
+ * mamba_mixer.h -- C ABI of the B200 (sm_100a) fused Mamba-1 selective-SSM mixer core.
+ *
+ * The operator is the "Mamba operator" of calm-mamba 0.1.4 (PyPI PKG-INFO), steps 2 and
+ * 4-6; the projections of steps 1, 3, 4 (matmul) and 7 stay outside this library and
+ * their outputs (x', z, dt_raw, B, C) are its inputs:
+ *
+ *   u[t]   = SiLU(conv_b + sum_{k<4} conv_w[k] * xpad[t+k])     step 2 (causal, left-padded)
+ *   D[t]   = softplus(dt_raw[t] + dt_bias)                       step 4
+ *   h[t]   = exp(D[t]*A) * h[t-1] + D[t]*B[t]*u[t],  A = -exp(A_log)
+ *   y[t]   = C[t] . h[t] + D*u[t]                                 step 5 (selective scan)
+ *   out[t] = y[t] * SiLU(z[t])                                    step 6 (gate)
+ *
+ * with xpad = [conv state (3 values, oldest first) or zeros ; x'[0..L-1]].  The decode
+ * step is the same computation for one token on a cached (h, conv state) pair: calm-mamba
+ * 0.1.4 (introduction: O(1) per-token state-cached generation) and niverel-mamba 0.1.0
+ * (section "Autoregressive decoding": step returns a new state and mutates nothing).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.    Every array argument is a DEVICE pointer owned by the caller.  The library
+ *            allocates no device memory and keeps no state besides a thread-local error
+ *            message.  Work is enqueued on `cuda_stream` (a cudaStream_t; NULL = the
+ *            legacy default stream); calls return once the work is enqueued.
+ * Layouts.   Row-major, channel-contiguous ("BLD"):
+ *              x', z, dt_raw, y         [batch, seqlen, d_inner]   io dtype
+ *              B, C                     [batch, seqlen, d_state]   io dtype (shared by all
+ *                                                                  channels of a (b, t))
+ *              A_log                    [d_inner, d_state]         fp32
+ *              D, conv_b, dt_bias       [d_inner]                  fp32
+ *              conv_w                   [d_inner, d_conv]          fp32
+ *              h (SSM state)            [batch, d_inner, d_state]  fp32
+ *              conv state               [batch, d_inner, d_conv-1] io dtype, oldest first
+ * Types.     io dtype MAMBA_F32 or MAMBA_BF16; all arithmetic is fp32; outputs in the io
+ *            dtype are rounded to nearest even.
+ * Support.   d_conv == 4, d_state in {8, 16}, d_inner a multiple of 8; batch, seqlen and
+ *            d_inner may be 0 (nothing to do beyond writing the states).
+ * Errors.    Every check is made on the host before anything is enqueued; a call that
+ *            returns non-OK has enqueued nothing.  There is no fallback path.
+ *              MAMBA_ERR_INVALID_ARGUMENT  NULL required pointer, negative size, bad
+ *                                          overlap between an output and another array
+ *              MAMBA_ERR_UNSUPPORTED       d_conv, d_state, d_inner or dtype outside the
+ *                                          supported set
+ *              MAMBA_ERR_ALIGNMENT         an activation, state or output pointer not
+ *                                          16-byte aligned, or a parameter pointer not
+ *                                          4-byte aligned
+ *              MAMBA_ERR_WORKSPACE         workspace smaller than
+ *                                          mamba_mixer_fwd_workspace_bytes() or not
+ *                                          16-byte aligned
+ *              MAMBA_ERR_CUDA              a CUDA launch or query failed
+ *            mamba_last_error() gives a one-line message for the last non-OK return on
+ *            the calling thread.
+ */
+#ifndef MAMBA_MIXER_H_
+#define MAMBA_MIXER_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MAMBA_MIXER_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define MAMBA_API __attribute__((visibility("default")))
+#else
+#define MAMBA_API
+#endif
+
+typedef enum { MAMBA_F32 = 0, MAMBA_BF16 = 1 } mamba_dtype;
+
+typedef enum {
+  MAMBA_OK = 0,
+  MAMBA_ERR_INVALID_ARGUMENT = 1,
+  MAMBA_ERR_UNSUPPORTED = 2,
+  MAMBA_ERR_ALIGNMENT = 3,
+  MAMBA_ERR_WORKSPACE = 4,
+  MAMBA_ERR_CUDA = 5
+} mamba_status;
+
+/* Problem sizes.  io_dtype holds a mamba_dtype value. */
+typedef struct {
+  int64_t batch;
+  int64_t seqlen;
+  int64_t d_inner;
+  int64_t d_state;
+  int64_t d_conv;
+  int32_t io_dtype;
+  int32_t reserved; /* must be 0 */
+} mamba_dims;
+
+/*
+ * Device workspace, in bytes, that mamba_mixer_fwd needs for `dims` (0 when the sequence
+ * is short enough to need no carry between time chunks).  Long sequences are split into
+ * time chunks that run in parallel; the workspace holds each chunk's end-of-chunk
+ * aggregate (decay product and local end state, fp32 [batch, chunks-1, d_inner, d_state]
+ * each) for the carry between chunks.  Returns 0 for dims the library does not support
+ * (mamba_mixer_fwd then reports why).
+ */
+MAMBA_API size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims);
+
+/*
+ * Fused forward over a whole sequence from a zero state (no initial state: the
+ * niverel-mamba weight contract, section "The weight contract", has no init_states).
+ * Inputs: xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b (may be NULL = zero bias),
+ * dt_bias.  Outputs: y [batch, seqlen, d_inner]; h_out, the SSM state after the last
+ * token (may be NULL = not written); conv_state_out, the last d_conv-1 inputs of xpad
+ * (zeros included when seqlen < d_conv-1; may be NULL = not written).
+ * Outputs must not overlap any input or each other.  `workspace` may be NULL only when
+ * mamba_mixer_fwd_workspace_bytes(dims) is 0.  Calls that share a workspace must not
+ * overlap on the GPU.
+ */
+MAMBA_API int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z,
+                    const void* dt_raw, const void* B, const void* C, const float* A_log,
+                    const float* D, const float* conv_w, const float* conv_b,
+                    const float* dt_bias, void* y, float* h_out, void* conv_state_out,
+                    void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * One decode step: one token for each of `batch` sequences (dims->seqlen must be 1) on a
+ * cached state.  Inputs: xp, z, dt_raw [batch, 1, d_inner]; B, C [batch, 1, d_state];
+ * the parameters as for mamba_mixer_fwd; h_in [batch, d_inner, d_state] fp32 and
+ * conv_state_in [batch, d_inner, 3] io dtype.  Outputs: y [batch, 1, d_inner], h_out,
+ * conv_state_out (the new state; both required).
+ * Functional by default (distinct output buffers leave the inputs untouched).  In-place
+ * update is allowed: h_out == h_in and/or conv_state_out == conv_state_in exactly; any
+ * other overlap is MAMBA_ERR_INVALID_ARGUMENT.
+ */
+MAMBA_API int mamba_mixer_step(const mamba_dims* dims, const void* xp, const void* z,
+                     const void* dt_raw, const void* B, const void* C, const float* A_log,
+                     const float* D, const float* conv_w, const float* conv_b,
+                     const float* dt_bias, const float* h_in, const void* conv_state_in,
+                     void* y, float* h_out, void* conv_state_out, void* cuda_stream);
+
+/* Message for the last non-OK return on this thread ("" if none). Never NULL. */
+MAMBA_API const char* mamba_last_error(void);
+
+/* Library version string, e.g. "mamba_mixer 0.1.0 (abi 1, sm_100a)". */
+MAMBA_API const char* mamba_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_MIXER_H_ */

@@ -1,0 +1,312 @@
+// Host side of the C ABI declared in include/mamba_mixer.h: argument checks, the
+// time-chunk plan, and kernel launches on the caller's stream.
+//
+// Every check happens before the first CUDA call; a failing call enqueues nothing.
+
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "mamba_mixer.h"
+#include "fwd_simple.cuh"
+#include "step.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return MAMBA_OK;
+}
+
+struct Span {
+  const void* p;
+  size_t bytes;
+  const char* name;
+};
+
+bool overlaps(const Span& a, const Span& b) {
+  if (!a.p || !b.p || a.bytes == 0 || b.bytes == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), a1 = a0 + a.bytes;
+  const uintptr_t b0 = reinterpret_cast<uintptr_t>(b.p), b1 = b0 + b.bytes;
+  return a0 < b1 && b0 < a1;
+}
+
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > INT64_MAX / a) return false;
+  *out = a * b;
+  return true;
+}
+
+// Validates sizes and support.  Fills element counts.
+struct Sizes {
+  int64_t act;     // batch*L*Di
+  int64_t bc;      // batch*L*N
+  int64_t state;   // batch*Di*N
+  int64_t cstate;  // batch*Di*(K-1)
+  int esize;       // bytes per io element
+};
+
+int check_dims(const mamba_dims* d, Sizes* s) {
+  if (!d) return fail(MAMBA_ERR_INVALID_ARGUMENT, "dims is NULL");
+  if (d->batch < 0 || d->seqlen < 0 || d->d_inner < 0 || d->d_state < 0 || d->d_conv < 0)
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "negative size in dims");
+  if (d->reserved != 0) return fail(MAMBA_ERR_INVALID_ARGUMENT, "dims.reserved must be 0");
+  if (d->io_dtype != MAMBA_F32 && d->io_dtype != MAMBA_BF16)
+    return fail(MAMBA_ERR_UNSUPPORTED, "io_dtype %d is not MAMBA_F32 or MAMBA_BF16",
+                int(d->io_dtype));
+  if (d->d_conv != 4) return fail(MAMBA_ERR_UNSUPPORTED, "d_conv %lld unsupported (only 4)",
+                                  (long long)d->d_conv);
+  if (d->d_state != 8 && d->d_state != 16)
+    return fail(MAMBA_ERR_UNSUPPORTED, "d_state %lld unsupported (8 or 16)",
+                (long long)d->d_state);
+  if (d->d_inner % 8 != 0)
+    return fail(MAMBA_ERR_UNSUPPORTED, "d_inner %lld is not a multiple of 8",
+                (long long)d->d_inner);
+  int64_t bl = 0;
+  if (!mul_ok(d->batch, d->seqlen, &bl) || !mul_ok(bl, d->d_inner, &s->act) ||
+      !mul_ok(bl, d->d_state, &s->bc) || !mul_ok(d->batch * d->d_inner, d->d_state, &s->state) ||
+      !mul_ok(d->batch * d->d_inner, d->d_conv - 1, &s->cstate) || s->act > (INT64_MAX >> 3))
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "sizes overflow");
+  if (d->batch > 65535) return fail(MAMBA_ERR_UNSUPPORTED, "batch > 65535");
+  s->esize = d->io_dtype == MAMBA_F32 ? 4 : 2;
+  return MAMBA_OK;
+}
+
+int check_ptr(const void* p, const char* name, bool required, size_t align) {
+  if (!p) {
+    if (required) return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s is NULL", name);
+    return MAMBA_OK;
+  }
+  if (reinterpret_cast<uintptr_t>(p) % align != 0)
+    return fail(MAMBA_ERR_ALIGNMENT, "%s is not %zu-byte aligned", name, align);
+  return MAMBA_OK;
+}
+
+// ---- time-chunk plan ---------------------------------------------------------------
+// Enough (channel, chunk) threads to fill the GPU, chunks no shorter than 512 steps.
+struct Plan {
+  int nchunks;
+  int64_t chunk_len;
+};
+
+Plan make_plan(const mamba_dims* d) {
+  Plan p{1, d->seqlen > 0 ? d->seqlen : 1};
+  const int64_t channels = d->batch * d->d_inner;
+  if (channels <= 0 || d->seqlen < 1024) return p;
+  const int64_t want_threads = 148 * 512;
+  int64_t c = (want_threads + channels - 1) / channels;
+  const int64_t cmax = d->seqlen / 512;
+  if (c > cmax) c = cmax;
+  if (c > 64) c = 64;
+  if (c <= 1) return p;
+  int64_t len = (d->seqlen + c - 1) / c;
+  len = (len + 63) / 64 * 64;
+  p.nchunks = int((d->seqlen + len - 1) / len);
+  p.chunk_len = len;
+  return p;
+}
+
+size_t workspace_bytes_for(const mamba_dims* d, const Plan& p) {
+  if (p.nchunks <= 1) return 0;
+  return size_t(2) * size_t(d->batch) * size_t(p.nchunks - 1) * size_t(d->d_inner) *
+         size_t(d->d_state) * sizeof(float);
+}
+
+template <int N, typename IO, bool P>
+cudaError_t launch_fwd(const mm::FwdArgs& a, cudaStream_t st) {
+  const dim3 block(mm::kSimpleThreads);
+  const unsigned gx = unsigned((a.Di + mm::kSimpleThreads - 1) / mm::kSimpleThreads);
+  if (a.nchunks > 1) {
+    mm::fwd_chunk_state<N, IO, P><<<dim3(gx, unsigned(a.batch), unsigned(a.nchunks - 1)),
+                                    block, 0, st>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  mm::fwd_chunk_main<N, IO, P><<<dim3(gx, unsigned(a.batch), unsigned(a.nchunks)), block, 0,
+                                 st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int N, typename IO, bool P>
+cudaError_t launch_step(const mm::StepArgs& a, cudaStream_t st) {
+  const int64_t threads = a.batch * a.Di * mm::kStepLanes;
+  const int64_t blocks = (threads + mm::kStepThreads - 1) / mm::kStepThreads;
+  mm::step_kernel<N, IO, P><<<unsigned(blocks), mm::kStepThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* mamba_last_error(void) { return g_last_error.c_str(); }
+
+const char* mamba_version(void) { return "mamba_mixer 0.1.0 (abi 1, sm_100a)"; }
+
+size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims) {
+  Sizes s;
+  if (check_dims(dims, &s) != MAMBA_OK) return 0;
+  return workspace_bytes_for(dims, make_plan(dims));
+}
+
+int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+                    const void* B, const void* C, const float* A_log, const float* D,
+                    const float* conv_w, const float* conv_b, const float* dt_bias, void* y,
+                    float* h_out, void* conv_state_out, void* workspace,
+                    size_t workspace_bytes, void* cuda_stream) {
+  Sizes s;
+  int rc = check_dims(dims, &s);
+  if (rc) return rc;
+  const bool act = s.act > 0, bc = s.bc > 0;
+  if ((rc = check_ptr(xp, "xp", act, 16)) || (rc = check_ptr(z, "z", act, 16)) ||
+      (rc = check_ptr(dt_raw, "dt_raw", act, 16)) || (rc = check_ptr(B, "B", bc, 16)) ||
+      (rc = check_ptr(C, "C", bc, 16)) || (rc = check_ptr(y, "y", act, 16)) ||
+      (rc = check_ptr(A_log, "A_log", dims->d_inner > 0, 16)) ||
+      (rc = check_ptr(D, "D", dims->d_inner > 0, 4)) ||
+      (rc = check_ptr(conv_w, "conv_w", dims->d_inner > 0, 16)) ||
+      (rc = check_ptr(conv_b, "conv_b", false, 4)) ||
+      (rc = check_ptr(dt_bias, "dt_bias", dims->d_inner > 0, 4)) ||
+      (rc = check_ptr(h_out, "h_out", false, 16)) ||
+      (rc = check_ptr(conv_state_out, "conv_state_out", false, 2)))
+    return rc;
+  const int64_t Di = dims->d_inner, N = dims->d_state;
+  const Span ins[] = {{xp, size_t(s.act) * s.esize, "xp"},   {z, size_t(s.act) * s.esize, "z"},
+                      {dt_raw, size_t(s.act) * s.esize, "dt_raw"},
+                      {B, size_t(s.bc) * s.esize, "B"},     {C, size_t(s.bc) * s.esize, "C"},
+                      {A_log, size_t(Di * N) * 4, "A_log"}, {D, size_t(Di) * 4, "D"},
+                      {conv_w, size_t(Di) * 16, "conv_w"},  {conv_b, size_t(Di) * 4, "conv_b"},
+                      {dt_bias, size_t(Di) * 4, "dt_bias"}};
+  const Span outs[] = {{y, size_t(s.act) * s.esize, "y"},
+                       {h_out, size_t(s.state) * 4, "h_out"},
+                       {conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"}};
+  const Plan plan = make_plan(dims);
+  const size_t need = workspace_bytes_for(dims, plan);
+  const Span wsp{workspace, need, "workspace"};
+  for (const Span& o : outs) {
+    for (const Span& i : ins)
+      if (overlaps(o, i)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, i.name);
+    for (const Span& o2 : outs)
+      if (&o2 != &o && overlaps(o, o2))
+        return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, o2.name);
+    if (overlaps(o, wsp)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps workspace", o.name);
+  }
+  for (const Span& i : ins)
+    if (overlaps(i, wsp)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "workspace overlaps %s", i.name);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need)
+      return fail(MAMBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                  workspace ? workspace_bytes : size_t(0), need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+      return fail(MAMBA_ERR_WORKSPACE, "workspace is not 16-byte aligned");
+  }
+  if (dims->batch == 0 || Di == 0) return ok();
+
+  mm::FwdArgs a{};
+  a.xp = xp; a.z = z; a.dt = dt_raw; a.B = B; a.C = C;
+  a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
+  a.y = y; a.h_out = h_out; a.cs_out = conv_state_out;
+  a.batch = dims->batch; a.L = dims->seqlen; a.Di = Di;
+  a.nchunks = plan.nchunks; a.chunk_len = plan.chunk_len;
+  if (need > 0) {
+    a.ws_P = static_cast<float*>(workspace);
+    a.ws_H = a.ws_P + need / sizeof(float) / 2;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e;
+  const bool f32 = dims->io_dtype == MAMBA_F32;
+  if (N == 16)
+    e = f32 ? launch_fwd<16, float, true>(a, st) : launch_fwd<16, __nv_bfloat16, false>(a, st);
+  else
+    e = f32 ? launch_fwd<8, float, true>(a, st) : launch_fwd<8, __nv_bfloat16, false>(a, st);
+  if (e != cudaSuccess)
+    return fail(MAMBA_ERR_CUDA, "forward launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int mamba_mixer_step(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+                     const void* B, const void* C, const float* A_log, const float* D,
+                     const float* conv_w, const float* conv_b, const float* dt_bias,
+                     const float* h_in, const void* conv_state_in, void* y, float* h_out,
+                     void* conv_state_out, void* cuda_stream) {
+  Sizes s;
+  int rc = check_dims(dims, &s);
+  if (rc) return rc;
+  if (dims->seqlen != 1)
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "step needs seqlen == 1 (got %lld)",
+                (long long)dims->seqlen);
+  const bool act = s.act > 0;
+  const bool st_ = s.state > 0;
+  if ((rc = check_ptr(xp, "xp", act, 16)) || (rc = check_ptr(z, "z", act, 16)) ||
+      (rc = check_ptr(dt_raw, "dt_raw", act, 16)) || (rc = check_ptr(B, "B", act, 16)) ||
+      (rc = check_ptr(C, "C", act, 16)) || (rc = check_ptr(y, "y", act, 16)) ||
+      (rc = check_ptr(A_log, "A_log", dims->d_inner > 0, 16)) ||
+      (rc = check_ptr(D, "D", dims->d_inner > 0, 4)) ||
+      (rc = check_ptr(conv_w, "conv_w", dims->d_inner > 0, 16)) ||
+      (rc = check_ptr(conv_b, "conv_b", false, 4)) ||
+      (rc = check_ptr(dt_bias, "dt_bias", dims->d_inner > 0, 4)) ||
+      (rc = check_ptr(h_in, "h_in", st_, 16)) || (rc = check_ptr(h_out, "h_out", st_, 16)) ||
+      (rc = check_ptr(conv_state_in, "conv_state_in", st_, 2)) ||
+      (rc = check_ptr(conv_state_out, "conv_state_out", st_, 2)))
+    return rc;
+  const int64_t Di = dims->d_inner, N = dims->d_state;
+  const Span ins[] = {{xp, size_t(s.act) * s.esize, "xp"},   {z, size_t(s.act) * s.esize, "z"},
+                      {dt_raw, size_t(s.act) * s.esize, "dt_raw"},
+                      {B, size_t(s.bc) * s.esize, "B"},     {C, size_t(s.bc) * s.esize, "C"},
+                      {A_log, size_t(Di * N) * 4, "A_log"}, {D, size_t(Di) * 4, "D"},
+                      {conv_w, size_t(Di) * 16, "conv_w"},  {conv_b, size_t(Di) * 4, "conv_b"},
+                      {dt_bias, size_t(Di) * 4, "dt_bias"}};
+  const Span h_in_s{h_in, size_t(s.state) * 4, "h_in"};
+  const Span cs_in_s{conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"};
+  const Span y_s{y, size_t(s.act) * s.esize, "y"};
+  const Span h_out_s{h_out, size_t(s.state) * 4, "h_out"};
+  const Span cs_out_s{conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"};
+  const Span outs[] = {y_s, h_out_s, cs_out_s};
+  for (const Span& o : outs)
+    for (const Span& i : ins)
+      if (overlaps(o, i)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, i.name);
+  if (overlaps(y_s, h_out_s) || overlaps(y_s, cs_out_s) || overlaps(h_out_s, cs_out_s) ||
+      overlaps(y_s, h_in_s) || overlaps(y_s, cs_in_s))
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "output buffers overlap");
+  // in place is allowed only as exact aliasing
+  if (overlaps(h_out_s, h_in_s) && h_out != h_in)
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "h_out partially overlaps h_in");
+  if (overlaps(cs_out_s, cs_in_s) && conv_state_out != conv_state_in)
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "conv_state_out partially overlaps conv_state_in");
+  if (overlaps(h_out_s, cs_in_s) || overlaps(cs_out_s, h_in_s))
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "state outputs overlap the other state input");
+  if (dims->batch == 0 || Di == 0) return ok();
+
+  mm::StepArgs a{};
+  a.xp = xp; a.z = z; a.dt = dt_raw; a.B = B; a.C = C;
+  a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
+  a.h_in = h_in; a.cs_in = conv_state_in; a.y = y; a.h_out = h_out; a.cs_out = conv_state_out;
+  a.batch = dims->batch; a.Di = Di;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e;
+  const bool f32 = dims->io_dtype == MAMBA_F32;
+  if (N == 16)
+    e = f32 ? launch_step<16, float, true>(a, st) : launch_step<16, __nv_bfloat16, false>(a, st);
+  else
+    e = f32 ? launch_step<8, float, true>(a, st) : launch_step<8, __nv_bfloat16, false>(a, st);
+  if (e != cudaSuccess)
+    return fail(MAMBA_ERR_CUDA, "step launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+}  // extern "C"

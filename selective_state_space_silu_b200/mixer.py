@@ -1,0 +1,200 @@
+"""Python binding of libmamba_mixer.so (include/mamba_mixer.h), by ctypes.
+
+Argument marshalling only: torch tensors are checked for device, dtype and contiguity,
+their data pointers and the current CUDA stream are passed to the C entry points of the
+same names, and a non-OK status becomes a ``MambaError``.  Every step of the mixer runs
+in the library's CUDA kernels; there is no other implementation behind these calls.
+Missing outputs (and the forward's workspace) are allocated with ``torch.empty``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmamba_mixer.so")
+
+MAMBA_F32 = 0
+MAMBA_BF16 = 1
+STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPORTED",
+          3: "MAMBA_ERR_ALIGNMENT", 4: "MAMBA_ERR_WORKSPACE", 5: "MAMBA_ERR_CUDA"}
+EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd", "mamba_mixer_step",
+           "mamba_last_error", "mamba_version")
+
+
+class MambaError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+class mamba_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
+                ("d_conv", ctypes.c_int64), ("io_dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library; raises if it is missing (build it first)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m selective_state_space_silu_b200.build` "
+            "(there is no fallback implementation)")
+    lib = ctypes.CDLL(path)
+    vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    P = ctypes.POINTER(mamba_dims)
+    lib.mamba_mixer_fwd_workspace_bytes.restype = sz
+    lib.mamba_mixer_fwd_workspace_bytes.argtypes = [P]
+    lib.mamba_mixer_fwd.restype = i
+    lib.mamba_mixer_fwd.argtypes = [P] + [vp] * 13 + [vp, sz, vp]
+    lib.mamba_mixer_step.restype = i
+    lib.mamba_mixer_step.argtypes = [P] + [vp] * 15 + [vp]
+    lib.mamba_last_error.restype = ctypes.c_char_p
+    lib.mamba_last_error.argtypes = []
+    lib.mamba_version.restype = ctypes.c_char_p
+    lib.mamba_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def mamba_version() -> str:
+    return load_library().mamba_version().decode()
+
+
+def mamba_last_error() -> str:
+    return load_library().mamba_last_error().decode()
+
+
+def make_dims(batch, seqlen, d_inner, d_state, d_conv=4, io_dtype=MAMBA_BF16) -> mamba_dims:
+    return mamba_dims(int(batch), int(seqlen), int(d_inner), int(d_state), int(d_conv),
+                      int(io_dtype), 0)
+
+
+def _io_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MAMBA_F32
+    if t.dtype == torch.bfloat16:
+        return MAMBA_BF16
+    raise TypeError(f"activations must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor], name: str, dtype=None, device=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream_handle(stream, device) -> Optional[int]:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise MambaError(rc, mamba_last_error())
+
+
+def mamba_mixer_fwd_workspace_bytes(dims: mamba_dims) -> int:
+    return int(load_library().mamba_mixer_fwd_workspace_bytes(ctypes.byref(dims)))
+
+
+def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
+                    y=None, h_out=None, conv_state_out=None, workspace=None,
+                    stream=None, want_states: bool = True
+                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
+    """Fused forward (conv + SiLU, softplus, selective scan, gate) from a zero state.
+
+    Shapes: xp, z, dt_raw [batch, L, d_inner]; B, C [batch, L, d_state]; A_log
+    [d_inner, d_state]; D, dt_bias, conv_b [d_inner]; conv_w [d_inner, 4].  Returns
+    (y, h_out, conv_state_out).
+    """
+    lib = load_library()
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    dims = make_dims(Bt, L, Di, N, K, io)
+    if y is None:
+        y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
+    if want_states and h_out is None:
+        h_out = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+    if want_states and conv_state_out is None:
+        conv_state_out = torch.empty((Bt, Di, K - 1), dtype=iot, device=dev)
+    need = mamba_mixer_fwd_workspace_bytes(dims)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    f32 = torch.float32
+    rc = lib.mamba_mixer_fwd(
+        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
+        _ptr(conv_state_out, "conv_state_out", iot, dev),
+        _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
+    _check(rc)
+    return y, h_out, conv_state_out
+
+
+def mamba_mixer_step(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, h_in,
+                     conv_state_in, *, y=None, h_out=None, conv_state_out=None,
+                     stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """One decode step on a cached state; functional unless outputs alias the inputs.
+
+    Shapes: xp, z, dt_raw [batch, 1, d_inner] (or [batch, d_inner]); B, C [batch, 1,
+    d_state] (or [batch, d_state]); h_in [batch, d_inner, d_state] fp32; conv_state_in
+    [batch, d_inner, 3].  Returns (y, h_out, conv_state_out); pass h_out=h_in and
+    conv_state_out=conv_state_in for an in-place update.
+    """
+    lib = load_library()
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, Di, N = h_in.shape
+    K = conv_w.shape[1]
+    dims = make_dims(Bt, 1, Di, N, K, io)
+    if y is None:
+        y = torch.empty(xp.shape, dtype=iot, device=dev)
+    if h_out is None:
+        h_out = torch.empty_like(h_in)
+    if conv_state_out is None:
+        conv_state_out = torch.empty_like(conv_state_in)
+    f32 = torch.float32
+    rc = lib.mamba_mixer_step(
+        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(h_in, "h_in", f32, dev), _ptr(conv_state_in, "conv_state_in", iot, dev),
+        _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
+        _ptr(conv_state_out, "conv_state_out", iot, dev), _stream_handle(stream, dev))
+    _check(rc)
+    return y, h_out, conv_state_out
+
+
+def launches_per_fwd(dims: mamba_dims) -> int:
+    """Kernel launches one mamba_mixer_fwd call makes: the main fused kernel, plus the
+    chunk-state kernel when the sequence is split into time chunks (workspace > 0)."""
+    return 2 if mamba_mixer_fwd_workspace_bytes(dims) > 0 else 1

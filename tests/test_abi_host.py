@@ -1,0 +1,152 @@
+"""Host-side checks of the C ABI: the library loads, exports what include/*.h declares,
+links no vendor math library, and rejects bad arguments before touching CUDA.
+
+Nothing here launches a kernel: every call either fails validation (which happens before
+the first CUDA call) or has nothing to do (batch 0).
+"""
+
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from selective_state_space_silu_b200 import build as B
+from selective_state_space_silu_b200 import mixer as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return M.load_library()
+
+
+def declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names |= set(re.findall(r"MAMBA_API\s+[\w\s\*]+?\b(mamba_\w+)\s*\(", src))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert {"mamba_mixer_fwd", "mamba_mixer_step", "mamba_mixer_fwd_workspace_bytes",
+            "mamba_last_error", "mamba_version"} <= names
+    out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s(mamba_\w+)", out))
+    assert names <= exported, names - exported
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_linkage_has_no_vendor_math_or_torch(lib):
+    """No cuBLAS / cuDNN / libtorch, and the CUDA runtime is linked statically."""
+    out = subprocess.run(["ldd", M.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    for bad in ("cublas", "cudnn", "torch", "c10", "cudart", "nccl", "cufft", "curand"):
+        assert bad not in out.lower(), out
+
+
+def test_version(lib):
+    assert M.mamba_version().startswith("mamba_mixer ")
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def _fwd(lib, dims, ptrs=None, ws=None, ws_bytes=0):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(
+        ["xp", "z", "dt", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias", "y", "h", "cs"])}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba_mixer_fwd(ctypes.byref(dims), p["xp"], p["z"], p["dt"], p["B"], p["C"],
+                               p["A_log"], p["D"], p["conv_w"], p["conv_b"], p["dt_bias"],
+                               p["y"], p["h"], p["cs"], ws, ws_bytes, None)
+
+
+def _step(lib, dims, ptrs=None):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(
+        ["xp", "z", "dt", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias", "h_in", "cs_in",
+         "y", "h", "cs"])}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba_mixer_step(ctypes.byref(dims), p["xp"], p["z"], p["dt"], p["B"], p["C"],
+                                p["A_log"], p["D"], p["conv_w"], p["conv_b"], p["dt_bias"],
+                                p["h_in"], p["cs_in"], p["y"], p["h"], p["cs"], None)
+
+
+def test_unsupported_dims(lib):
+    for kw, code in [(dict(d_conv=3), 2), (dict(d_state=32), 2), (dict(d_state=12), 2),
+                     (dict(d_inner=12), 2), (dict(io_dtype=7), 2), (dict(batch=-1), 1),
+                     (dict(seqlen=-5), 1)]:
+        args = dict(batch=2, seqlen=16, d_inner=128, d_state=16, d_conv=4, io_dtype=M.MAMBA_BF16)
+        args.update(kw)
+        dims = M.make_dims(**args)
+        rc = _fwd(lib, dims)
+        assert rc == code, (kw, rc, M.mamba_last_error())
+        assert M.mamba_last_error()
+        assert lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(dims)) == 0
+
+
+def test_reserved_and_null_dims(lib):
+    d = M.make_dims(2, 16, 128, 16)
+    d.reserved = 1
+    assert _fwd(lib, d) == 1
+    assert lib.mamba_mixer_fwd(None, *([None] * 13), None, 0, None) == 1
+    assert "dims" in M.mamba_last_error()
+
+
+def test_null_required_pointers(lib):
+    dims = M.make_dims(2, 16, 128, 16)
+    for k in ("xp", "z", "dt", "B", "C", "A_log", "D", "conv_w", "dt_bias", "y"):
+        assert _fwd(lib, dims, {k: None}) == 1, k
+    sd = M.make_dims(4, 1, 64, 16)
+    for k in ("xp", "h_in", "cs_in", "h", "cs", "y"):
+        assert _step(lib, sd, {k: None}) == 1, k
+
+
+def test_misaligned_pointers(lib):
+    dims = M.make_dims(2, 16, 128, 16)
+    assert _fwd(lib, dims, {"xp": _fake(0x10000008)}) == 3
+    assert "xp" in M.mamba_last_error()
+    assert _fwd(lib, dims, {"D": _fake(0x6010000002)}) == 3
+    sd = M.make_dims(4, 1, 64, 16)
+    assert _step(lib, sd, {"h_in": _fake(0xa010000004)}) == 3
+
+
+def test_overlaps_rejected(lib):
+    dims = M.make_dims(2, 16, 128, 16)
+    assert _fwd(lib, dims, {"y": _fake(0x10000000)}) == 1          # y on top of xp
+    assert _fwd(lib, dims, {"h": _fake(0xa010000010)}) == 1          # h_out inside y
+    sd = M.make_dims(4, 1, 64, 16)
+    # exact in-place aliasing of the states is fine at validation; partial overlap is not
+    assert _step(lib, sd, {"h": _fake(0xa010000040)}) == 1
+    assert "partially" in M.mamba_last_error()
+    assert _step(lib, sd, {"cs": _fake(0xb010000006)}) == 1
+    assert _step(lib, M.make_dims(4, 2, 64, 16)) == 1               # step needs seqlen 1
+
+
+def test_workspace_rules(lib):
+    short = M.make_dims(8, 512, 1536, 16)
+    assert lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(short)) == 0
+    long = M.make_dims(2, 65536, 2560, 16)
+    need = lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(long))
+    assert need > 0 and need % 16 == 0
+    assert _fwd(lib, long) == 4
+    assert "workspace" in M.mamba_last_error()
+    assert _fwd(lib, long, ws=_fake(0x14010000000), ws_bytes=need - 16) == 4
+    assert _fwd(lib, long, ws=_fake(0x14010000008), ws_bytes=need) == 4
+
+
+def test_empty_batch_is_a_no_op(lib):
+    d = M.make_dims(0, 16, 128, 16)
+    assert _fwd(lib, d, {k: None for k in ("xp", "z", "dt", "B", "C", "y", "h", "cs")}) == 0
+    assert M.mamba_last_error() == ""
