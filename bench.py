@@ -193,8 +193,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
         y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
         h = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
         cs = torch.empty((Bt, Di, 3), dtype=iot, device=dev)
-        need = M.mamba_mixer_fwd_workspace_bytes(M.make_dims(Bt, L, Di, N, 4, M._io_code(X["xp"])))
-        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        ws = M.new_workspace(M.make_dims(Bt, L, Di, N, 4, M._io_code(X["xp"])), dev)
     yt = torch.empty((Bt, 1, Di), dtype=iot, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
 
@@ -208,7 +207,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
                            P["conv_w"], P["conv_b"], P["dt_bias"], h, cs, y=yt, h_out=h,
                            conv_state_out=cs, stream=stream)
 
-    launches_fwd = 0 if w.decode else M.launches_per_fwd(M.make_dims(Bt, L, Di, N, 4, M._io_code(X["xp"])))
+    launches_fwd = 0 if w.decode else M.mamba_mixer_fwd_launches(M.make_dims(Bt, L, Di, N, 4, M._io_code(X["xp"])))
     launches_per_step = launches_fwd + 1
 
     def one_step(ev=None):

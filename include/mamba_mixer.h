@@ -48,8 +48,13 @@
  *                                          mamba_mixer_fwd_workspace_bytes() or not
  *                                          16-byte aligned
  *              MAMBA_ERR_CUDA              a CUDA launch or query failed
+ *              MAMBA_ERR_TIMEOUT           (mamba_mixer_check only) a forward kernel gave
+ *                                          up on a bounded wait; see mamba_mixer_check
  *            mamba_last_error() gives a one-line message for the last non-OK return on
  *            the calling thread.
+ * Waits.     The forward kernels wait on their own asynchronous copies (TMA into shared
+ *            memory).  Every such wait gives up after one second, stops the CTA cleanly
+ *            and records MAMBA_ERR_TIMEOUT in the workspace status word; no call hangs.
  */
 #ifndef MAMBA_MIXER_H_
 #define MAMBA_MIXER_H_
@@ -77,7 +82,8 @@ typedef enum {
   MAMBA_ERR_UNSUPPORTED = 2,
   MAMBA_ERR_ALIGNMENT = 3,
   MAMBA_ERR_WORKSPACE = 4,
-  MAMBA_ERR_CUDA = 5
+  MAMBA_ERR_CUDA = 5,
+  MAMBA_ERR_TIMEOUT = 6
 } mamba_status;
 
 /* Problem sizes.  io_dtype holds a mamba_dtype value. */
@@ -92,14 +98,22 @@ typedef struct {
 } mamba_dims;
 
 /*
- * Device workspace, in bytes, that mamba_mixer_fwd needs for `dims` (0 when the sequence
- * is short enough to need no carry between time chunks).  Long sequences are split into
- * time chunks that run in parallel; the workspace holds each chunk's end-of-chunk
- * aggregate (decay product and local end state, fp32 [batch, chunks-1, d_inner, d_state]
- * each) for the carry between chunks.  Returns 0 for dims the library does not support
- * (mamba_mixer_fwd then reports why).
+ * Device workspace, in bytes, that mamba_mixer_fwd needs for `dims`: a 256-byte header
+ * whose first 4 bytes are the status word, then -- when the sequence is split into time
+ * chunks that run in parallel -- each chunk's carry aggregate (decay product and local end
+ * state, fp32 [batch, chunks-1, d_inner, d_state] each).  The status word must be zero
+ * before the first forward that uses the workspace (clear the header once after
+ * allocating it); the library only sets it on a timeout and mamba_mixer_check clears it.
+ * Returns 0 for dims the library does not support (mamba_mixer_fwd then reports why).
  */
 MAMBA_API size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims);
+
+/*
+ * Number of kernels one mamba_mixer_fwd call with `dims` launches (1, or 2 when the
+ * sequence is split into time chunks: the chunk-state pass, then the main pass); 0 when
+ * there is nothing to compute; -1 for unsupported dims.
+ */
+MAMBA_API int mamba_mixer_fwd_launches(const mamba_dims* dims);
 
 /*
  * Fused forward over a whole sequence from a zero state (no initial state: the
@@ -108,9 +122,9 @@ MAMBA_API size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims);
  * dt_bias.  Outputs: y [batch, seqlen, d_inner]; h_out, the SSM state after the last
  * token (may be NULL = not written); conv_state_out, the last d_conv-1 inputs of xpad
  * (zeros included when seqlen < d_conv-1; may be NULL = not written).
- * Outputs must not overlap any input or each other.  `workspace` may be NULL only when
- * mamba_mixer_fwd_workspace_bytes(dims) is 0.  Calls that share a workspace must not
- * overlap on the GPU.
+ * Outputs must not overlap any input or each other.  `workspace` (device, 16-byte
+ * aligned, at least mamba_mixer_fwd_workspace_bytes(dims) bytes) is required.  Calls that
+ * share a workspace must not overlap on the GPU.
  */
 MAMBA_API int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z,
                     const void* dt_raw, const void* B, const void* C, const float* A_log,
@@ -133,6 +147,13 @@ MAMBA_API int mamba_mixer_step(const mamba_dims* dims, const void* xp, const voi
                      const float* D, const float* conv_w, const float* conv_b,
                      const float* dt_bias, const float* h_in, const void* conv_state_in,
                      void* y, float* h_out, void* conv_state_out, void* cuda_stream);
+
+/*
+ * Waits for `cuda_stream`, then reads and clears the status word of `workspace`.
+ * Returns MAMBA_ERR_TIMEOUT if a forward that used this workspace since the last check
+ * gave up on a bounded wait (its outputs are then incomplete), MAMBA_OK otherwise.
+ */
+MAMBA_API int mamba_mixer_check(void* workspace, void* cuda_stream);
 
 /* Message for the last non-OK return on this thread ("" if none). Never NULL. */
 MAMBA_API const char* mamba_last_error(void);

@@ -3,15 +3,17 @@
 //
 // Every check happens before the first CUDA call; a failing call enqueues nothing.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "mamba_mixer.h"
-#include "fwd_simple.cuh"
+#include "fwd_kernel.cuh"
 #include "step.cuh"
 
 namespace {
@@ -99,7 +101,12 @@ int check_ptr(const void* p, const char* name, bool required, size_t align) {
 }
 
 // ---- time-chunk plan ---------------------------------------------------------------
-// Enough (channel, chunk) threads to fill the GPU, chunks no shorter than 512 steps.
+// A CTA covers one batch row and 32 channels.  When there are too few such tiles to give
+// every SM about four CTAs, the sequence is cut into time chunks (multiples of the tile
+// length, at least 256 steps) that run in parallel with a carried state between them.
+constexpr int kResidentCtas = 148 * 4;
+constexpr size_t kWsHeader = 256;  // status word + padding
+
 struct Plan {
   int nchunks;
   int64_t chunk_len;
@@ -107,40 +114,89 @@ struct Plan {
 
 Plan make_plan(const mamba_dims* d) {
   Plan p{1, d->seqlen > 0 ? d->seqlen : 1};
-  const int64_t channels = d->batch * d->d_inner;
-  if (channels <= 0 || d->seqlen < 1024) return p;
-  const int64_t want_threads = 148 * 512;
-  int64_t c = (want_threads + channels - 1) / channels;
-  const int64_t cmax = d->seqlen / 512;
+  const int64_t tiles = d->batch * ((d->d_inner + mm::kCh - 1) / mm::kCh);
+  if (tiles <= 0 || d->seqlen < 512 || tiles * 2 >= kResidentCtas) return p;
+  int64_t c = (kResidentCtas + tiles / 2) / tiles;
+  const int64_t cmax = d->seqlen / 256;
   if (c > cmax) c = cmax;
-  if (c > 64) c = 64;
+  if (c > 256) c = 256;
   if (c <= 1) return p;
   int64_t len = (d->seqlen + c - 1) / c;
-  len = (len + 63) / 64 * 64;
+  len = (len + mm::kTileT - 1) / mm::kTileT * mm::kTileT;
   p.nchunks = int((d->seqlen + len - 1) / len);
   p.chunk_len = len;
   return p;
 }
 
 size_t workspace_bytes_for(const mamba_dims* d, const Plan& p) {
-  if (p.nchunks <= 1) return 0;
-  return size_t(2) * size_t(d->batch) * size_t(p.nchunks - 1) * size_t(d->d_inner) *
-         size_t(d->d_state) * sizeof(float);
+  size_t agg = 0;
+  if (p.nchunks > 1)
+    agg = size_t(2) * size_t(d->batch) * size_t(p.nchunks - 1) * size_t(d->d_inner) *
+          size_t(d->d_state) * sizeof(float);
+  return kWsHeader + agg;
+}
+
+// ---- TMA descriptors ---------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over a row-major [d2][d1][d0] tensor, box (b0, b1, 1).
+bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t d0, uint64_t d1,
+              uint64_t d2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t es = bf16 ? 2 : 4;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * es, d0 * d1 * es};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct FwdMaps {
+  CUtensorMap x, z, dt, B, C;
+};
+
+template <int N, typename IO, bool P, bool kPre>
+cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdParams& a, dim3 grid,
+                              cudaStream_t st) {
+  using S = mm::FwdSmem<IO, N>;
+  auto kern = mm::fwd_kernel<N, IO, P, kPre>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       S::kDynamic);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, mm::kFwdThreads, S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, a);
+  return cudaGetLastError();
 }
 
 template <int N, typename IO, bool P>
-cudaError_t launch_fwd(const mm::FwdArgs& a, cudaStream_t st) {
-  const dim3 block(mm::kSimpleThreads);
-  const unsigned gx = unsigned((a.Di + mm::kSimpleThreads - 1) / mm::kSimpleThreads);
+cudaError_t launch_fwd(const FwdMaps& m, const mm::FwdParams& a, int64_t batch, cudaStream_t st) {
+  const unsigned gx = unsigned((a.Di + mm::kCh - 1) / mm::kCh);
   if (a.nchunks > 1) {
-    mm::fwd_chunk_state<N, IO, P><<<dim3(gx, unsigned(a.batch), unsigned(a.nchunks - 1)),
-                                    block, 0, st>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_fwd_kernel<N, IO, P, true>(
+        m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), st);
     if (e != cudaSuccess) return e;
   }
-  mm::fwd_chunk_main<N, IO, P><<<dim3(gx, unsigned(a.batch), unsigned(a.nchunks)), block, 0,
-                                 st>>>(a);
-  return cudaGetLastError();
+  return launch_fwd_kernel<N, IO, P, false>(m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks)),
+                                            st);
 }
 
 template <int N, typename IO, bool P>
@@ -208,34 +264,79 @@ int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const
   }
   for (const Span& i : ins)
     if (overlaps(i, wsp)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "workspace overlaps %s", i.name);
-  if (need > 0) {
-    if (!workspace || workspace_bytes < need)
-      return fail(MAMBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
-                  workspace ? workspace_bytes : size_t(0), need);
-    if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
-      return fail(MAMBA_ERR_WORKSPACE, "workspace is not 16-byte aligned");
-  }
+  if (!workspace || workspace_bytes < need)
+    return fail(MAMBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                workspace ? workspace_bytes : size_t(0), need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+    return fail(MAMBA_ERR_WORKSPACE, "workspace is not 16-byte aligned");
   if (dims->batch == 0 || Di == 0) return ok();
 
-  mm::FwdArgs a{};
-  a.xp = xp; a.z = z; a.dt = dt_raw; a.B = B; a.C = C;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const bool f32 = dims->io_dtype == MAMBA_F32;
+  if (dims->seqlen == 0) {
+    // empty sequence: the states are the zero initial state and zero padding
+    cudaError_t e = cudaSuccess;
+    if (h_out) e = cudaMemsetAsync(h_out, 0, size_t(s.state) * 4, st);
+    if (e == cudaSuccess && conv_state_out)
+      e = cudaMemsetAsync(conv_state_out, 0, size_t(s.cstate) * s.esize, st);
+    if (e != cudaSuccess)
+      return fail(MAMBA_ERR_CUDA, "state reset failed: %s", cudaGetErrorString(e));
+    return ok();
+  }
+
+  FwdMaps m;
+  const uint64_t Bt = uint64_t(dims->batch), L = uint64_t(dims->seqlen);
+  const CUtensorMapSwizzle swz = f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const uint32_t nrow = uint32_t(mm::kTileT);
+  if (!make_map(&m.x, xp, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow + mm::kHalo, swz) ||
+      !make_map(&m.z, z, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) ||
+      !make_map(&m.dt, dt_raw, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) ||
+      !make_map(&m.B, B, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&m.C, C, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return fail(MAMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
+
+  mm::FwdParams a{};
   a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
   a.y = y; a.h_out = h_out; a.cs_out = conv_state_out;
-  a.batch = dims->batch; a.L = dims->seqlen; a.Di = Di;
+  a.status = static_cast<int*>(workspace);
+  a.L = dims->seqlen; a.Di = Di;
   a.nchunks = plan.nchunks; a.chunk_len = plan.chunk_len;
-  if (need > 0) {
-    a.ws_P = static_cast<float*>(workspace);
-    a.ws_H = a.ws_P + need / sizeof(float) / 2;
+  if (plan.nchunks > 1) {
+    const size_t agg = (need - kWsHeader) / sizeof(float) / 2;
+    a.ws_P = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + kWsHeader);
+    a.ws_H = a.ws_P + agg;
   }
-  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e;
-  const bool f32 = dims->io_dtype == MAMBA_F32;
   if (N == 16)
-    e = f32 ? launch_fwd<16, float, true>(a, st) : launch_fwd<16, __nv_bfloat16, false>(a, st);
+    e = f32 ? launch_fwd<16, float, true>(m, a, dims->batch, st)
+            : launch_fwd<16, __nv_bfloat16, false>(m, a, dims->batch, st);
   else
-    e = f32 ? launch_fwd<8, float, true>(a, st) : launch_fwd<8, __nv_bfloat16, false>(a, st);
+    e = f32 ? launch_fwd<8, float, true>(m, a, dims->batch, st)
+            : launch_fwd<8, __nv_bfloat16, false>(m, a, dims->batch, st);
   if (e != cudaSuccess)
     return fail(MAMBA_ERR_CUDA, "forward launch failed: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+int mamba_mixer_fwd_launches(const mamba_dims* dims) {
+  Sizes s;
+  if (check_dims(dims, &s) != MAMBA_OK) return -1;
+  if (dims->batch == 0 || dims->d_inner == 0 || dims->seqlen == 0) return 0;
+  return make_plan(dims).nchunks > 1 ? 2 : 1;
+}
+
+int mamba_mixer_check(void* workspace, void* cuda_stream) {
+  if (!workspace) return fail(MAMBA_ERR_INVALID_ARGUMENT, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  int status = 0;
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e == cudaSuccess) e = cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail(MAMBA_ERR_CUDA, "status read failed: %s", cudaGetErrorString(e));
+  if (status != 0) {
+    const int zero = 0;
+    cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    return fail(MAMBA_ERR_TIMEOUT, "a forward kernel gave up on a bounded wait (status %d)", status);
+  }
   return ok();
 }
 

@@ -21,9 +21,10 @@ LIB_PATH = os.path.join(_PKG, "libmamba_mixer.so")
 MAMBA_F32 = 0
 MAMBA_BF16 = 1
 STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPORTED",
-          3: "MAMBA_ERR_ALIGNMENT", 4: "MAMBA_ERR_WORKSPACE", 5: "MAMBA_ERR_CUDA"}
-EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd", "mamba_mixer_step",
-           "mamba_last_error", "mamba_version")
+          3: "MAMBA_ERR_ALIGNMENT", 4: "MAMBA_ERR_WORKSPACE", 5: "MAMBA_ERR_CUDA",
+          6: "MAMBA_ERR_TIMEOUT"}
+EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba_mixer_fwd",
+           "mamba_mixer_step", "mamba_mixer_check", "mamba_last_error", "mamba_version")
 
 
 class MambaError(RuntimeError):
@@ -56,6 +57,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P = ctypes.POINTER(mamba_dims)
     lib.mamba_mixer_fwd_workspace_bytes.restype = sz
     lib.mamba_mixer_fwd_workspace_bytes.argtypes = [P]
+    lib.mamba_mixer_fwd_launches.restype = i
+    lib.mamba_mixer_fwd_launches.argtypes = [P]
+    lib.mamba_mixer_check.restype = i
+    lib.mamba_mixer_check.argtypes = [vp, vp]
     lib.mamba_mixer_fwd.restype = i
     lib.mamba_mixer_fwd.argtypes = [P] + [vp] * 13 + [vp, sz, vp]
     lib.mamba_mixer_step.restype = i
@@ -117,6 +122,22 @@ def mamba_mixer_fwd_workspace_bytes(dims: mamba_dims) -> int:
     return int(load_library().mamba_mixer_fwd_workspace_bytes(ctypes.byref(dims)))
 
 
+def new_workspace(dims: mamba_dims, device) -> torch.Tensor:
+    """A zeroed workspace of the size mamba_mixer_fwd needs for ``dims``."""
+    need = mamba_mixer_fwd_workspace_bytes(dims)
+    if need == 0:
+        raise MambaError(2, "unsupported dims: " + mamba_last_error())
+    return torch.zeros(need, dtype=torch.uint8, device=device)
+
+
+def mamba_mixer_check(workspace: torch.Tensor, stream=None) -> None:
+    """Wait for the stream; raise MambaError(MAMBA_ERR_TIMEOUT) if a forward that used
+    ``workspace`` gave up on a bounded wait since the last check (clears the status)."""
+    rc = load_library().mamba_mixer_check(workspace.data_ptr(),
+                                          _stream_handle(stream, workspace.device))
+    _check(rc)
+
+
 def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
                     y=None, h_out=None, conv_state_out=None, workspace=None,
                     stream=None, want_states: bool = True
@@ -141,9 +162,8 @@ def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
         h_out = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
     if want_states and conv_state_out is None:
         conv_state_out = torch.empty((Bt, Di, K - 1), dtype=iot, device=dev)
-    need = mamba_mixer_fwd_workspace_bytes(dims)
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        workspace = new_workspace(dims, dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     f32 = torch.float32
     rc = lib.mamba_mixer_fwd(
@@ -194,7 +214,6 @@ def mamba_mixer_step(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, h_i
     return y, h_out, conv_state_out
 
 
-def launches_per_fwd(dims: mamba_dims) -> int:
-    """Kernel launches one mamba_mixer_fwd call makes: the main fused kernel, plus the
-    chunk-state kernel when the sequence is split into time chunks (workspace > 0)."""
-    return 2 if mamba_mixer_fwd_workspace_bytes(dims) > 0 else 1
+def mamba_mixer_fwd_launches(dims: mamba_dims) -> int:
+    """Kernel launches one mamba_mixer_fwd call with ``dims`` makes."""
+    return int(load_library().mamba_mixer_fwd_launches(ctypes.byref(dims)))

@@ -35,8 +35,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(lib):
     names = declared_symbols()
-    assert {"mamba_mixer_fwd", "mamba_mixer_step", "mamba_mixer_fwd_workspace_bytes",
-            "mamba_last_error", "mamba_version"} <= names
+    assert set(M.EXPORTS) <= names
     out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
     exported = set(re.findall(r"\sT\s(mamba_\w+)", out))
@@ -136,8 +135,11 @@ def test_overlaps_rejected(lib):
 
 def test_workspace_rules(lib):
     short = M.make_dims(8, 512, 1536, 16)
-    assert lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(short)) == 0
+    assert lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(short)) == 256   # status header only
+    assert lib.mamba_mixer_fwd_launches(ctypes.byref(short)) == 1
+    assert _fwd(lib, short) == 4                                          # workspace required
     long = M.make_dims(2, 65536, 2560, 16)
+    assert lib.mamba_mixer_fwd_launches(ctypes.byref(long)) == 2
     need = lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(long))
     assert need > 0 and need % 16 == 0
     assert _fwd(lib, long) == 4
@@ -148,5 +150,12 @@ def test_workspace_rules(lib):
 
 def test_empty_batch_is_a_no_op(lib):
     d = M.make_dims(0, 16, 128, 16)
-    assert _fwd(lib, d, {k: None for k in ("xp", "z", "dt", "B", "C", "y", "h", "cs")}) == 0
+    ws = _fake(0x10000000 + 30 * (1 << 36))
+    assert _fwd(lib, d, {k: None for k in ("xp", "z", "dt", "B", "C", "y", "h", "cs")},
+                ws=ws, ws_bytes=256) == 0
     assert M.mamba_last_error() == ""
+    assert lib.mamba_mixer_fwd_launches(ctypes.byref(d)) == 0
+
+
+def test_check_rejects_null_workspace(lib):
+    assert lib.mamba_mixer_check(None, None) == 1
