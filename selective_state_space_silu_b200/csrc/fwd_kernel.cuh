@@ -73,8 +73,8 @@ struct FwdSmem {
   static constexpr int kZOff = align1k(kXBytes);
   static constexpr int kDtOff = kZOff + align1k(kZBytes);
   static constexpr int kBOff = kDtOff + align1k(kZBytes);
-  static constexpr int kCOff = kBOff + kBBytes;
-  static constexpr int kBCfOff = align1k(kCOff + kBBytes);
+  static constexpr int kCOff = kBOff + align1k(kBBytes);
+  static constexpr int kBCfOff = kCOff + align1k(kBBytes);
   static constexpr int kStageBytes = align1k(kBCfOff + kBCfBytes);
   static constexpr int kBarOff = kStages * kStageBytes;
   static constexpr int kTotal = kBarOff + 2 * kStages * 8 + 16;
@@ -133,7 +133,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     }
     *abort_flag = 0;
     *prod_abort = 0;
-    fence_mbar_init();
   }
   __syncthreads();
 
@@ -142,33 +141,37 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 
   if (tid >= kConsumers) {
     // ------------------------------------------------------------ producer warp
+    // The whole warp walks the tiles together; lane 0 issues the copies.
+    const bool leader = tid == kConsumers;
+    constexpr uint32_t kSwzAlign = 1024, kPlainAlign = 128;
     int issued = 0;
-    if (tid == kConsumers) {
-      prefetch_tmap(&tm_x); prefetch_tmap(&tm_dt); prefetch_tmap(&tm_B);
-      if constexpr (!kPrepass) { prefetch_tmap(&tm_z); prefetch_tmap(&tm_C); }
-      for (int k = 0; k < ntiles; ++k) {
-        const int s = k % kStages;
-        if (k >= kStages && !mbar_wait(&empty[s], uint32_t((k / kStages) - 1) & 1u, p.status)) {
-          *reinterpret_cast<volatile int*>(prod_abort) = 1;
-          break;
-        }
+    for (int k = 0; k < ntiles; ++k) {
+      const int s = k % kStages;
+      bool got = k < kStages || mbar_wait(&empty[s], uint32_t((k / kStages) - 1) & 1u, p.status);
+      got = __all_sync(0xffffffffu, got);   // the warp decides together
+      if (!got) {
+        *reinterpret_cast<volatile int*>(prod_abort) = 1;
+        break;
+      }
+      if (leader) {
         unsigned char* st = smem + s * S::kStageBytes;
         const int tt = int(t_begin) + k * kTileT;
         mbar_arrive_expect_tx(&full[s], kTxBytes);
-        tma_load_3d(st + S::kXOff, &tm_x, &full[s], d0, tt - kHalo, b);
-        tma_load_3d(st + S::kDtOff, &tm_dt, &full[s], d0, tt, b);
-        tma_load_3d(st + S::kBOff, &tm_B, &full[s], 0, tt, b);
+        tma_load_3d(st + S::kXOff, &tm_x, &full[s], d0, tt - kHalo, b, kSwzAlign, kEs, p.status);
+        tma_load_3d(st + S::kDtOff, &tm_dt, &full[s], d0, tt, b, kSwzAlign, kEs, p.status);
+        tma_load_3d(st + S::kBOff, &tm_B, &full[s], 0, tt, b, kPlainAlign, kEs, p.status);
         if constexpr (!kPrepass) {
-          tma_load_3d(st + S::kZOff, &tm_z, &full[s], d0, tt, b);
-          tma_load_3d(st + S::kCOff, &tm_C, &full[s], 0, tt, b);
+          tma_load_3d(st + S::kZOff, &tm_z, &full[s], d0, tt, b, kSwzAlign, kEs, p.status);
+          tma_load_3d(st + S::kCOff, &tm_C, &full[s], 0, tt, b, kPlainAlign, kEs, p.status);
         }
-        issued = k + 1;
       }
+      __syncwarp();
+      issued = k + 1;
     }
-    __syncthreads();
+    named_bar_sync(0, kFwdThreads);
     // drain: every copy this CTA started must land before the CTA exits
-    if (tid == kConsumers && (*reinterpret_cast<volatile int*>(abort_flag) ||
-                              *reinterpret_cast<volatile int*>(prod_abort))) {
+    if (leader && (*reinterpret_cast<volatile int*>(abort_flag) ||
+                   *reinterpret_cast<volatile int*>(prod_abort))) {
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         mbar_wait(&full[k % kStages], uint32_t(k / kStages) & 1u, nullptr);
     }
@@ -324,7 +327,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     if (lane == 0) mbar_arrive(&empty[s]);
   }
 
-  named_bar_sync(0, kFwdThreads);  // pairs with the producer's __syncthreads()
+  named_bar_sync(0, kFwdThreads);  // pairs with the producer warp's barrier
   if (!ok) return;
 
   if constexpr (kPrepass) {

@@ -335,6 +335,9 @@ int mamba_mixer_check(void* workspace, void* cuda_stream) {
   if (status != 0) {
     const int zero = 0;
     cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (status == mm::kStatusBadCopy)
+      return fail(MAMBA_ERR_CUDA, "a forward kernel refused a TMA copy that failed its "
+                  "alignment self-check (outputs incomplete)");
     return fail(MAMBA_ERR_TIMEOUT, "a forward kernel gave up on a bounded wait (status %d)", status);
   }
   return ok();

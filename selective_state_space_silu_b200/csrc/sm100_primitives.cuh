@@ -12,6 +12,7 @@ namespace mm {
 
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 constexpr int kStatusTimeout = 6;                               // MAMBA_ERR_TIMEOUT
+constexpr int kStatusBadCopy = 7;  // a TMA copy failed its alignment self-check (not issued)
 
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
@@ -27,26 +28,20 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));
 }
 
-__device__ __forceinline__ void fence_mbar_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.release.cta.shared::cta.b64 st, [%0];\n\t}"
-               ::"r"(smem_addr(bar)) : "memory");
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.release.cta.shared::cta.b64 st, [%0], %1;\n\t}"
-      ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+               ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok) : "r"(smem_addr(bar)), "r"(parity) : "memory");
   return ok != 0;
@@ -66,23 +61,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
-__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
-  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
-}
-
-// 3-D tiled TMA load (no multicast): coordinates innermost first.
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int c0, int c1, int c2) {
+// 3-D tiled TMA load (no multicast): coordinates innermost first.  Self-checked: the
+// tensor map must be 64-byte aligned, the destination `dst_align`-byte aligned (1024 for
+// swizzled tiles, 128 otherwise) and the innermost coordinate times the element size a
+// multiple of 16 bytes; a copy that fails a check is not issued and *status records
+// kStatusBadCopy (its barrier then times out and the CTA stops cleanly).
+__device__ __forceinline__ bool tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, uint32_t dst_align,
+                                            int elem_bytes, int* status) {
+  const uint32_t sdst = smem_addr(dst);
+  const uint64_t gmap = reinterpret_cast<uint64_t>(map);
+  if ((sdst & (dst_align - 1)) != 0 || (gmap & 63u) != 0 || ((c0 * elem_bytes) & 15) != 0) {
+    atomicExch(status, kStatusBadCopy);
+    return false;
+  }
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];"
-      ::"r"(smem_addr(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)),
-        "r"(c0), "r"(c1), "r"(c2)
+      ::"r"(sdst), "l"(gmap), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
+  return true;
 }
 
+// Named barrier that tolerates divergent arrival (non-.aligned form).
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 }  // namespace mm
