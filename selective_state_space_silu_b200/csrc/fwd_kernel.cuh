@@ -57,7 +57,7 @@ struct FwdParams {
 constexpr int kCh = 32;          // channels per CTA
 constexpr int kTileT = 32;       // time steps per tile
 constexpr int kHalo = 4;         // x' rows loaded before each tile (3 needed)
-constexpr int kStages = 4;       // shared-memory ring depth
+constexpr int kStages = 3;       // shared-memory ring depth
 constexpr int kConsumers = 128;  // 4 warps
 constexpr int kFwdThreads = kConsumers + 32;
 
@@ -77,11 +77,12 @@ struct FwdSmem {
   static constexpr int kBCfOff = kCOff + align1k(kBBytes);
   static constexpr int kStageBytes = align1k(kBCfOff + kBCfBytes);
   static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kTotal = kBarOff + 2 * kStages * 8 + 16;
+  static constexpr int kTotal = kBarOff + 3 * kStages * 8 + 16;
   static constexpr int kDynamic = kTotal + 1024;  // slack to align the base to 1 KiB
 };
 
-// Byte offset of (row, col) in a swizzled tile with kRow-byte rows (64B or 128B swizzle).
+// Byte offset of (row, col) in a swizzled tile with kRow-byte rows (64B or 128B swizzle:
+// the 16-byte unit index is XORed with address bits 7.. of the row start).
 template <int kRow>
 __device__ __forceinline__ uint32_t swz(int row, int col_bytes) {
   const uint32_t a = uint32_t(row) * kRow + uint32_t(col_bytes);
@@ -89,14 +90,14 @@ __device__ __forceinline__ uint32_t swz(int row, int col_bytes) {
 }
 
 template <typename IO>
-__device__ __forceinline__ float lds_io(const unsigned char* base, uint32_t off);
+__device__ __forceinline__ float lds_io(uint32_t a);
 template <>
-__device__ __forceinline__ float lds_io<float>(const unsigned char* base, uint32_t off) {
-  return *reinterpret_cast<const float*>(base + off);
+__device__ __forceinline__ float lds_io<float>(uint32_t a) {
+  return lds_f32(a);
 }
 template <>
-__device__ __forceinline__ float lds_io<__nv_bfloat16>(const unsigned char* base, uint32_t off) {
-  return __uint_as_float(uint32_t(*reinterpret_cast<const unsigned short*>(base + off)) << 16);
+__device__ __forceinline__ float lds_io<__nv_bfloat16>(uint32_t a) {
+  return __uint_as_float(lds_u16(a) << 16);
 }
 
 template <int N, typename IO, bool kPrecise, bool kPrepass>
@@ -111,14 +112,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   constexpr int kEs = int(sizeof(IO));
 
   extern __shared__ unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);
-  uint64_t* empty = full + kStages;
-  int* abort_flag = reinterpret_cast<int*>(empty + kStages);   // consumers' decision
-  int* prod_abort = abort_flag + 1;                              // producer gave up
+  const uint32_t raw = smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sb = smem_addr(smem);                 // 1 KiB-aligned shared address
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // TMA landed
+  uint64_t* ready = full + kStages;                                  // B/C widened
+  uint64_t* empty = ready + kStages;                                 // consumers done
+  int* prod_abort = reinterpret_cast<int*>(empty + kStages);
 
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   const int d0 = blockIdx.x * kCh;
   const int b = blockIdx.y;
   const int c = blockIdx.z;
@@ -129,9 +132,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
+      mbar_init(&ready[s], 1);
       mbar_init(&empty[s], kConsumers / 32);
     }
-    *abort_flag = 0;
     *prod_abort = 0;
   }
   __syncthreads();
@@ -141,21 +144,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 
   if (tid >= kConsumers) {
     // ------------------------------------------------------------ producer warp
-    // The whole warp walks the tiles together; lane 0 issues the copies.
-    const bool leader = tid == kConsumers;
-    constexpr uint32_t kSwzAlign = 1024, kPlainAlign = 128;
+    // The warp walks the tiles together: lane 0 issues the copies, all lanes widen B/C.
+    const bool leader = lane == 0;
     int issued = 0;
-    for (int k = 0; k < ntiles; ++k) {
+    auto issue = [&](int k) {
       const int s = k % kStages;
-      bool got = k < kStages || mbar_wait(&empty[s], uint32_t((k / kStages) - 1) & 1u, p.status);
-      got = __all_sync(0xffffffffu, got);   // the warp decides together
-      if (!got) {
-        *reinterpret_cast<volatile int*>(prod_abort) = 1;
-        break;
-      }
       if (leader) {
-        unsigned char* st = smem + s * S::kStageBytes;
+        const uint32_t st = sb + uint32_t(s * S::kStageBytes);
         const int tt = int(t_begin) + k * kTileT;
+        constexpr uint32_t kSwzAlign = 1024, kPlainAlign = 128;
         mbar_arrive_expect_tx(&full[s], kTxBytes);
         tma_load_3d(st + S::kXOff, &tm_x, &full[s], d0, tt - kHalo, b, kSwzAlign, kEs, p.status);
         tma_load_3d(st + S::kDtOff, &tm_dt, &full[s], d0, tt, b, kSwzAlign, kEs, p.status);
@@ -167,11 +164,37 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       }
       __syncwarp();
       issued = k + 1;
+    };
+    for (int k = 0; k < ntiles && k < kStages; ++k) issue(k);
+    bool good = true;
+    for (int k = 0; k < ntiles && good; ++k) {
+      const int s = k % kStages;
+      good = __all_sync(0xffffffffu, mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status));
+      if (!good) break;
+      // widen this tile's B (and C) to fp32, interleaved as [t][j]{B[kS], C[kS]}
+      const uint32_t st = sb + uint32_t(s * S::kStageBytes);
+      for (int idx = lane; idx < kTileT * N; idx += 32) {
+        const int t = idx / N, n = idx - t * N;
+        const int jj = n / kS, ss = n - jj * kS;
+        const uint32_t dst = st + S::kBCfOff + uint32_t(((t * 4 + jj) * (2 * kS) + ss) * 4);
+        sts_f32(dst, lds_io<IO>(st + S::kBOff + idx * kEs));
+        if constexpr (!kPrepass) sts_f32(dst + kS * 4, lds_io<IO>(st + S::kCOff + idx * kEs));
+      }
+      __syncwarp();
+      if (leader) mbar_arrive(&ready[s]);
+      // refill the stage of tile k-1 once the consumers have released it
+      const int kn = k - 1 + kStages;
+      if (k >= 1 && kn < ntiles) {
+        const int sp = (k - 1) % kStages;
+        good = __all_sync(0xffffffffu,
+                          mbar_wait(&empty[sp], uint32_t((k - 1) / kStages) & 1u, p.status));
+        if (good) issue(kn);
+      }
     }
+    if (!good) *reinterpret_cast<volatile int*>(prod_abort) = 1;
     named_bar_sync(0, kFwdThreads);
     // drain: every copy this CTA started must land before the CTA exits
-    if (leader && (*reinterpret_cast<volatile int*>(abort_flag) ||
-                   *reinterpret_cast<volatile int*>(prod_abort))) {
+    if (leader && *reinterpret_cast<volatile int*>(prod_abort)) {
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         mbar_wait(&full[k % kStages], uint32_t(k / kStages) & 1u, nullptr);
     }
@@ -179,14 +202,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   }
 
   // -------------------------------------------------------------- consumer warps
-  const int lane = tid & 31;
   const int warp = tid >> 5;
   const int chl = lane & 7;
   const int j = lane >> 3;
   const int cl = warp * 8 + chl;  // channel within the CTA tile
   // d_inner % 8 == 0, so a warp's 8 channels are all in range or all out of range; an
-  // out-of-range warp still takes part in every barrier but reads channel 0's parameters
-  // and stores nothing.
+  // out-of-range warp still walks the tiles (it releases every stage) but reads channel
+  // 0's parameters and stores nothing.
   const bool active = d0 + cl < p.Di;
   const int64_t d = active ? d0 + cl : 0;
 
@@ -214,49 +236,33 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   IO* y = static_cast<IO*>(p.y);
   const int col_bytes = cl * kEs;
   bool ok = true;
-  int k = 0;
-  for (; k < ntiles; ++k) {
+  for (int k = 0; k < ntiles; ++k) {
     const int s = k % kStages;
-    const unsigned char* st = smem + s * S::kStageBytes;
+    const uint32_t st = sb + uint32_t(s * S::kStageBytes);
     const int64_t tt = t_begin + int64_t(k) * kTileT;
-    if (!mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status))
-      *reinterpret_cast<volatile int*>(abort_flag) = 1;
-    // widen this tile's B (and C) to fp32, interleaved as [t][j]{B[kS], C[kS]}
-    float* bcf = reinterpret_cast<float*>(const_cast<unsigned char*>(st) + S::kBCfOff);
-    if (!*reinterpret_cast<volatile int*>(abort_flag)) {
-      for (int idx = tid; idx < kTileT * N; idx += kConsumers) {
-        const int t = idx / N, n = idx - t * N;
-        const int jj = n / kS, ss = n - jj * kS;
-        float* dst = bcf + (t * 4 + jj) * (2 * kS);
-        dst[ss] = lds_io<IO>(st, S::kBOff + idx * kEs);
-        if constexpr (!kPrepass) dst[kS + ss] = lds_io<IO>(st, S::kCOff + idx * kEs);
-      }
-    }
-    named_bar_sync(1, kConsumers);
-    if (*reinterpret_cast<volatile int*>(abort_flag)) { ok = false; break; }
+    ok = __all_sync(0xffffffffu, mbar_wait(&ready[s], uint32_t(k / kStages) & 1u, p.status) &&
+                                     mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status));
+    if (!ok) break;
 
-    const unsigned char* X = st + S::kXOff;
-    const unsigned char* Z = st + S::kZOff;
-    const unsigned char* DT = st + S::kDtOff;
+    const uint32_t X = st + S::kXOff, Z = st + S::kZOff, DT = st + S::kDtOff;
+    const uint32_t BCF = st + S::kBCfOff + uint32_t(j * 2 * kS * 4);
 
     // scalar work of step (4q + j) of this tile
-    auto scalar = [&](int q, float& dl, float& dul, float& du_skip, float& szl) {
+    auto scalar = [&](int q, float& dl, float& dul, float& skip, float& szl) {
       const int r = 4 * q + j;                        // tile row of this lane's step
-      const bool valid = tt + r < t_end;
-      const float x0 = lds_io<IO>(X, swz<kRow>(r + 1, col_bytes));
-      const float x1 = lds_io<IO>(X, swz<kRow>(r + 2, col_bytes));
-      const float x2 = lds_io<IO>(X, swz<kRow>(r + 3, col_bytes));
-      const float x3 = lds_io<IO>(X, swz<kRow>(r + 4, col_bytes));
+      const float x0 = lds_io<IO>(X + swz<kRow>(r + 1, col_bytes));
+      const float x1 = lds_io<IO>(X + swz<kRow>(r + 2, col_bytes));
+      const float x2 = lds_io<IO>(X + swz<kRow>(r + 3, col_bytes));
+      const float x3 = lds_io<IO>(X + swz<kRow>(r + 4, col_bytes));
       const float pre = cb + w0 * x0 + w1 * x1 + w2 * x2 + w3 * x3;
       const float u = M::silu(pre);
-      const float dv = M::softplus(lds_io<IO>(DT, swz<kRow>(r, col_bytes)) + dtb);
-      dl = valid ? dv : 0.0f;
-      dul = valid ? dv * u : 0.0f;
+      dl = M::softplus(lds_io<IO>(DT + swz<kRow>(r, col_bytes)) + dtb);
+      dul = dl * u;
       if constexpr (!kPrepass) {
-        du_skip = Dd * u;
-        szl = M::silu(lds_io<IO>(Z, swz<kRow>(r, col_bytes)));
+        skip = Dd * u;
+        szl = M::silu(lds_io<IO>(Z + swz<kRow>(r, col_bytes)));
       } else {
-        du_skip = 0.0f;
+        skip = 0.0f;
         szl = 0.0f;
       }
     };
@@ -272,7 +278,6 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         dui[i] = __shfl_sync(0xffffffffu, dul, (i << 3) | chl);
       }
       const float cur_skip = dsk, cur_sz = sz;
-      const bool cur_valid = tt + 4 * q + j < t_end;
       if (q + 1 < kTileT / 4) scalar(q + 1, dl, dul, dsk, sz);
 
       // steps past the chunk end (ragged last tile) leave the state untouched
@@ -283,17 +288,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       for (int i = 0; i < 4; ++i) {
         yp[i] = 0.0f;
         if (i >= nvalid) continue;
-        const float* row = bcf + ((4 * q + i) * 4 + j) * (2 * kS);
+        const uint32_t row = BCF + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
         float Bv[kS], Cv[kS];
         if constexpr (kS == 4) {
-          const float4 bv = *reinterpret_cast<const float4*>(row);
+          const float4 bv = lds_f32x4(row);
           Bv[0] = bv.x; Bv[1] = bv.y; Bv[2] = bv.z; Bv[3] = bv.w;
           if constexpr (!kPrepass) {
-            const float4 cv = *reinterpret_cast<const float4*>(row + 4);
+            const float4 cv = lds_f32x4(row + 16);
             Cv[0] = cv.x; Cv[1] = cv.y; Cv[2] = cv.z; Cv[3] = cv.w;
           }
         } else {
-          const float4 v = *reinterpret_cast<const float4*>(row);
+          const float4 v = lds_f32x4(row);
           Bv[0] = v.x; Bv[1] = v.y; Cv[0] = v.z; Cv[1] = v.w;
         }
         float acc = 0.0f;
@@ -317,7 +322,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         float kp = odd ? k1 : k0;
         const float sp = odd ? k0 : k1;
         kp += __shfl_xor_sync(0xffffffffu, sp, 8);
-        if (cur_valid && active) {
+        if (j < nvalid && active) {
           const float out = (kp + cur_skip) * cur_sz;
           y[(int64_t(b) * p.L + tt + 4 * q + j) * p.Di + d] = IOT<IO>::from_f(out);
         }
@@ -328,17 +333,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   }
 
   named_bar_sync(0, kFwdThreads);  // pairs with the producer warp's barrier
-  if (!ok) return;
+  if (!ok || !active) return;
 
   if constexpr (kPrepass) {
-    if (!active) return;
     const int64_t o = ((int64_t(b) * (p.nchunks - 1) + c) * p.Di + d) * N + j * kS;
 #pragma unroll
     for (int s = 0; s < kS; ++s) {
       p.ws_P[o + s] = P[s];
       p.ws_H[o + s] = h[s];
     }
-  } else if (c == p.nchunks - 1 && active) {
+  } else if (c == p.nchunks - 1) {
     if (p.h_out) {
       float* ho = p.h_out + (int64_t(b) * p.Di + d) * N + j * kS;
       if constexpr (kS == 4) {
@@ -350,11 +354,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     if (p.cs_out && j < 3) {
       // last 3 entries of xpad: x'[L-3+j] (zeros for negative t) from the last x tile
       const int kl = ntiles - 1;
-      const unsigned char* X = smem + (kl % kStages) * S::kStageBytes + S::kXOff;
+      const uint32_t X = sb + uint32_t((kl % kStages) * S::kStageBytes) + S::kXOff;
       const int64_t tt = t_begin + int64_t(kl) * kTileT;
       const int r = int(p.L - 3 + j - (tt - kHalo));
       IO* cs = static_cast<IO*>(p.cs_out) + (int64_t(b) * p.Di + d) * 3;
-      cs[j] = IOT<IO>::from_f(lds_io<IO>(X, swz<kRow>(r, col_bytes)));
+      cs[j] = IOT<IO>::from_f(lds_io<IO>(X + swz<kRow>(r, col_bytes)));
     }
   }
 }

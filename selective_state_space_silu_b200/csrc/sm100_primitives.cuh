@@ -66,10 +66,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
 // swizzled tiles, 128 otherwise) and the innermost coordinate times the element size a
 // multiple of 16 bytes; a copy that fails a check is not issued and *status records
 // kStatusBadCopy (its barrier then times out and the CTA stops cleanly).
-__device__ __forceinline__ bool tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+__device__ __forceinline__ bool tma_load_3d(uint32_t sdst, const CUtensorMap* map, uint64_t* bar,
                                             int c0, int c1, int c2, uint32_t dst_align,
                                             int elem_bytes, int* status) {
-  const uint32_t sdst = smem_addr(dst);
   const uint64_t gmap = reinterpret_cast<uint64_t>(map);
   if ((sdst & (dst_align - 1)) != 0 || (gmap & 63u) != 0 || ((c0 * elem_bytes) & 15) != 0) {
     atomicExch(status, kStatusBadCopy);
@@ -81,6 +80,27 @@ __device__ __forceinline__ bool tma_load_3d(void* dst, const CUtensorMap* map, u
       ::"r"(sdst), "l"(gmap), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
   return true;
+}
+
+// Shared-memory accesses by 32-bit shared-window address (always LDS/STS, never generic).
+__device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t a) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
 
 // Named barrier that tolerates divergent arrival (non-.aligned form).
