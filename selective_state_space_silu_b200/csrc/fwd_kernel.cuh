@@ -1,36 +1,41 @@
 // Fused forward of the selective-SSM mixer core for sm_100a.
 //
-// Work decomposition
-//   CTA   = one batch row b, a tile of kCh = 32 channels, one time chunk.
-//   warp  = 8 channels x 4 lanes.  Lane (chl = lane & 7, j = lane >> 3) owns states
-//           n in [j*kS, (j+1)*kS), kS = d_state / 4, of channel chl.  Keeping j uniform
-//           within each 8-lane phase makes the B/C shared-memory reads phase broadcasts.
-//   quad  = 4 consecutive time steps.  Lane j computes the per-(t, d) scalar work of step
-//           t0 + j (conv + SiLU, softplus, SiLU(z)); the step sizes are exchanged with
-//           shuffles, every lane advances its states through the 4 steps, and the partial
-//           readouts C.h are reduce-scattered so that lane j finishes step t0 + j.
+// Work decomposition (warp-specialised CTA: 2 prep warps + 4 scan warps)
+//   CTA        = one batch row b, a tile of kCh = 32 channels, one time chunk.
+//   prep warps = lane c is channel c.  Prep warp 0 also issues the TMA copies.  For each
+//                32-step tile, prep warp w handles steps [16w, 16w+16): it widens B and C
+//                to fp32 and computes the per-(t, d) scalars of the operator -- causal
+//                conv + SiLU (u), Delta = softplus(dt_raw + dt_bias), Delta*u, D*u and
+//                SiLU(z) -- once per (t, d), keeping the conv window in registers.
+//   scan warps = 8 channels x 4 lanes.  Lane (chl = lane & 7, j = lane >> 3) owns states
+//                n in [j*kS, (j+1)*kS), kS = d_state / 4, of channel chl; j is uniform in
+//                each 8-lane phase so the B/C reads are phase broadcasts.  Per group of 4
+//                steps ("quad") every lane reads Delta and Delta*u of the 4 steps, advances
+//                its states, and the partial readouts C.h are reduce-scattered over the 4
+//                lanes of the channel so that lane j finishes step 4q + j (gate, store).
 //
 // Data movement
-//   A producer warp streams 32-step tiles of x' (with a 4-row halo for the causal conv),
-//   z, dt_raw, B and C into a ring of shared-memory stages with TMA (3-D tensor maps,
-//   no multicast); x'/z/dt tiles use the 64/128-byte swizzle so that the lanes of a warp
-//   (4 rows x 8 channels) read without bank conflicts.  Negative or past-the-end time
-//   coordinates read zeros, which is the causal left padding at t < 0.  The consumer
-//   warps widen each B/C tile to fp32 once (shared by the 32 channels), then run the
-//   scan from registers.  y is stored directly (8 channels x 2 bytes per lane phase).
+//   Raw tiles of x' (with a 4-row halo for the causal conv), z, dt_raw, B and C stream
+//   into a 3-deep ring with TMA (3-D tensor maps, no multicast).  Negative or past-the-end
+//   time coordinates read zeros (the causal left padding at t < 0).  Prepared tiles (fp32
+//   B/C and the scalars) go through a 2-deep ring between prep and scan warps; the scalar
+//   records are 64 bytes per (quad, channel) with their 16-byte units XOR-swizzled by
+//   channel so that both sides access shared memory without bank conflicts.
 //
 // Time chunks (long sequences)
 //   A chunk c > 0 starts from the state carried out of chunks 0..c-1.  The chunk-state
 //   pass (kPrepass = true) runs the same recurrence over chunks 0..nchunks-2 and writes
 //   each chunk's pair (P, H): decay product prod_t exp(Delta_t A) and end state from zero.
 //   The main pass folds h = P*h + H over the earlier chunks to get its initial state.
+//   Steps past the chunk end get Delta = Delta*u = 0, which leaves the state unchanged.
 //
-// Every mbarrier wait is bounded (see sm100_primitives.cuh); on a timeout the CTA stops
-// issuing work, waits (bounded) for the copies it started, records MAMBA_ERR_TIMEOUT in
-// the status word and returns.
+// Every mbarrier wait is bounded (sm100_primitives.cuh): a warp that gives up leaves its
+// loop, the CTA meets at a final barrier, waits (bounded) for the copies it started,
+// records MAMBA_ERR_TIMEOUT in the status word and returns without writing states.
 #pragma once
 
 #include <cuda.h>
+#include <float.h>
 
 #include "device_math.cuh"
 #include "sm100_primitives.cuh"
@@ -56,10 +61,15 @@ struct FwdParams {
 
 constexpr int kCh = 32;          // channels per CTA
 constexpr int kTileT = 32;       // time steps per tile
+constexpr int kQuads = kTileT / 4;
 constexpr int kHalo = 4;         // x' rows loaded before each tile (3 needed)
-constexpr int kStages = 3;       // shared-memory ring depth
-constexpr int kConsumers = 128;  // 4 warps
-constexpr int kFwdThreads = kConsumers + 32;
+constexpr int kStages = 3;       // raw TMA ring depth
+constexpr int kPrepBufs = 2;     // prepared-tile ring depth
+constexpr int kScanWarps = 4;
+constexpr int kPrepWarps = 2;
+constexpr int kScanThreads = 32 * kScanWarps;
+constexpr int kFwdThreads = 32 * (kScanWarps + kPrepWarps);
+constexpr int kScRec = 64;       // bytes per (quad, channel) scalar record
 
 template <typename IO, int N>
 struct FwdSmem {
@@ -67,17 +77,21 @@ struct FwdSmem {
   static constexpr int kXBytes = (kTileT + kHalo) * kRow;
   static constexpr int kZBytes = kTileT * kRow;
   static constexpr int kBBytes = kTileT * N * int(sizeof(IO));
-  static constexpr int kBCfBytes = kTileT * 2 * N * 4;
   static constexpr int align1k(int v) { return (v + 1023) / 1024 * 1024; }
+  // raw stage (TMA destinations)
   static constexpr int kXOff = 0;
   static constexpr int kZOff = align1k(kXBytes);
   static constexpr int kDtOff = kZOff + align1k(kZBytes);
   static constexpr int kBOff = kDtOff + align1k(kZBytes);
   static constexpr int kCOff = kBOff + align1k(kBBytes);
-  static constexpr int kBCfOff = kCOff + align1k(kBBytes);
-  static constexpr int kStageBytes = align1k(kBCfOff + kBCfBytes);
-  static constexpr int kBarOff = kStages * kStageBytes;
-  static constexpr int kTotal = kBarOff + 3 * kStages * 8 + 16;
+  static constexpr int kRawStage = kCOff + align1k(kBBytes);
+  // prepared tile: fp32 B/C as [t][j]{B[kS], C[kS]}, then scalar records [q][c]
+  static constexpr int kBCfBytes = kTileT * 2 * N * 4;
+  static constexpr int kScOff = align1k(kBCfBytes);
+  static constexpr int kPrepBytes = kScOff + kQuads * kCh * kScRec;
+  static constexpr int kPrepBase = kStages * kRawStage;
+  static constexpr int kBarOff = kPrepBase + kPrepBufs * kPrepBytes;
+  static constexpr int kTotal = kBarOff + 8 * (2 * kStages + 2 * kPrepBufs) + 16;
   static constexpr int kDynamic = kTotal + 1024;  // slack to align the base to 1 KiB
 };
 
@@ -89,6 +103,11 @@ __device__ __forceinline__ uint32_t swz(int row, int col_bytes) {
   return a ^ (((a >> 7) & uint32_t(kRow / 16 - 1)) << 4);
 }
 
+// Offset of 16-byte unit u of the scalar record of (quad q, channel c).
+__device__ __forceinline__ uint32_t sc_unit(int q, int c, int u) {
+  return uint32_t((q * kCh + c) * kScRec + ((u ^ ((c >> 1) & 3)) << 4));
+}
+
 template <typename IO>
 __device__ __forceinline__ float lds_io(uint32_t a);
 template <>
@@ -98,6 +117,11 @@ __device__ __forceinline__ float lds_io<float>(uint32_t a) {
 template <>
 __device__ __forceinline__ float lds_io<__nv_bfloat16>(uint32_t a) {
   return __uint_as_float(lds_u16(a) << 16);
+}
+
+__device__ __forceinline__ void sts_f32x4(uint32_t a, float x, float y, float z, float w) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x), "f"(y), "f"(z),
+               "f"(w) : "memory");
 }
 
 template <int N, typename IO, bool kPrecise, bool kPrepass>
@@ -115,13 +139,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   const uint32_t raw = smem_addr(smem_raw);
   unsigned char* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const uint32_t sb = smem_addr(smem);                 // 1 KiB-aligned shared address
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);   // TMA landed
-  uint64_t* ready = full + kStages;                                  // B/C widened
-  uint64_t* empty = ready + kStages;                                 // consumers done
-  int* prod_abort = reinterpret_cast<int*>(empty + kStages);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::kBarOff);  // raw tile landed
+  uint64_t* raw_free = full + kStages;                              // prep warps done with it
+  uint64_t* prep_ready = raw_free + kStages;                        // prepared tile written
+  uint64_t* prep_free = prep_ready + kPrepBufs;                     // scan warps done with it
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  const int warp = tid >> 5;
   const int d0 = blockIdx.x * kCh;
   const int b = blockIdx.y;
   const int c = blockIdx.z;
@@ -132,25 +157,37 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&ready[s], 1);
-      mbar_init(&empty[s], kConsumers / 32);
+      mbar_init(&raw_free[s], kPrepWarps);
     }
-    *prod_abort = 0;
+    for (int r = 0; r < kPrepBufs; ++r) {
+      mbar_init(&prep_ready[r], kPrepWarps);
+      mbar_init(&prep_free[r], kScanWarps);
+    }
   }
   __syncthreads();
 
   constexpr uint32_t kTxBytes =
       uint32_t(S::kXBytes + (kPrepass ? 1 : 2) * S::kZBytes + (kPrepass ? 1 : 2) * S::kBBytes);
 
-  if (tid >= kConsumers) {
-    // ------------------------------------------------------------ producer warp
-    // The warp walks the tiles together: lane 0 issues the copies, all lanes widen B/C.
-    const bool leader = lane == 0;
+  if (warp >= kScanWarps) {
+    // ============================================================ prep warps
+    const int w = warp - kScanWarps;  // 0 or 1: steps [16w, 16w + 16) of each tile
+    const bool issuer = (w == 0);
+    const int cl = lane;               // channel within the CTA tile
+    const bool active = d0 + cl < p.Di;
+    const int64_t d = active ? d0 + cl : 0;
+    const float w0 = __ldg(p.conv_w + d * 4 + 0), w1 = __ldg(p.conv_w + d * 4 + 1);
+    const float w2 = __ldg(p.conv_w + d * 4 + 2), w3 = __ldg(p.conv_w + d * 4 + 3);
+    const float cb = p.conv_b ? __ldg(p.conv_b + d) : 0.0f;
+    const float dtb = __ldg(p.dt_bias + d);
+    const float Dd = kPrepass ? 0.0f : __ldg(p.D + d);
+    const int col = cl * kEs;
+
     int issued = 0;
     auto issue = [&](int k) {
       const int s = k % kStages;
-      if (leader) {
-        const uint32_t st = sb + uint32_t(s * S::kStageBytes);
+      if (lane == 0) {
+        const uint32_t st = sb + uint32_t(s * S::kRawStage);
         const int tt = int(t_begin) + k * kTileT;
         constexpr uint32_t kSwzAlign = 1024, kPlainAlign = 128;
         mbar_arrive_expect_tx(&full[s], kTxBytes);
@@ -165,67 +202,111 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       __syncwarp();
       issued = k + 1;
     };
-    for (int k = 0; k < ntiles && k < kStages; ++k) issue(k);
+    if (issuer)
+      for (int k = 0; k < ntiles && k < kStages; ++k) issue(k);
+
     bool good = true;
-    for (int k = 0; k < ntiles && good; ++k) {
-      const int s = k % kStages;
-      good = __all_sync(0xffffffffu, mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status));
+    for (int k = 0; k < ntiles; ++k) {
+      const int s = k % kStages, r = k % kPrepBufs;
+      bool got = mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status);
+      if (k >= kPrepBufs)
+        got = got && mbar_wait(&prep_free[r], uint32_t(k / kPrepBufs - 1) & 1u, p.status);
+      good = __all_sync(0xffffffffu, got);
       if (!good) break;
-      // widen this tile's B (and C) to fp32, interleaved as [t][j]{B[kS], C[kS]}
-      const uint32_t st = sb + uint32_t(s * S::kStageBytes);
-      for (int idx = lane; idx < kTileT * N; idx += 32) {
-        const int t = idx / N, n = idx - t * N;
-        const int jj = n / kS, ss = n - jj * kS;
-        const uint32_t dst = st + S::kBCfOff + uint32_t(((t * 4 + jj) * (2 * kS) + ss) * 4);
-        sts_f32(dst, lds_io<IO>(st + S::kBOff + idx * kEs));
-        if constexpr (!kPrepass) sts_f32(dst + kS * 4, lds_io<IO>(st + S::kCOff + idx * kEs));
+      const uint32_t st = sb + uint32_t(s * S::kRawStage);
+      const uint32_t pr = sb + uint32_t(S::kPrepBase + r * S::kPrepBytes);
+      const int64_t tt = t_begin + int64_t(k) * kTileT;
+
+      // B (and C) to fp32 for steps [16w, 16w + 16): [t][j]{B[kS], C[kS]}
+      for (int idx = lane; idx < (kTileT / 2) * N; idx += 32) {
+        const int t = (kTileT / 2) * w + idx / N, n = idx % N;
+        const int jj = n / kS, ss = n % kS;
+        const uint32_t dst = pr + uint32_t(((t * 4 + jj) * (2 * kS) + ss) * 4);
+        sts_f32(dst, lds_io<IO>(st + S::kBOff + (t * N + n) * kEs));
+        if constexpr (!kPrepass) sts_f32(dst + kS * 4, lds_io<IO>(st + S::kCOff + (t * N + n) * kEs));
+      }
+
+      // scalars of steps [16w, 16w + 16) of channel cl; x' tile row r holds t = tt - 4 + r
+      const int t0 = (kTileT / 2) * w;
+      float xa = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 1, col));
+      float xb = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 2, col));
+      float xc = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 3, col));
+#pragma unroll 1
+      for (int q = t0 / 4; q < t0 / 4 + kQuads / 2; ++q) {
+        float dv[4], duv[4], skv[4], szv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = 4 * q + i;
+          const float xt = lds_io<IO>(st + S::kXOff + swz<kRow>(t + 4, col));
+          const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          xa = xb; xb = xc; xc = xt;
+          const float u = M::silu(pre);
+          const bool valid = tt + t < t_end;
+          const float dl = M::softplus(lds_io<IO>(st + S::kDtOff + swz<kRow>(t, col)) + dtb);
+          dv[i] = valid ? dl : 0.0f;
+          duv[i] = valid ? dl * u : 0.0f;
+          if constexpr (!kPrepass) {
+            skv[i] = Dd * u;
+            szv[i] = M::silu(lds_io<IO>(st + S::kZOff + swz<kRow>(t, col)));
+          }
+        }
+        const uint32_t rec = pr + S::kScOff;
+        sts_f32x4(rec + sc_unit(q, cl, 0), dv[0], dv[1], dv[2], dv[3]);
+        sts_f32x4(rec + sc_unit(q, cl, 1), duv[0], duv[1], duv[2], duv[3]);
+        if constexpr (!kPrepass) {
+          sts_f32x4(rec + sc_unit(q, cl, 2), skv[0], skv[1], skv[2], skv[3]);
+          sts_f32x4(rec + sc_unit(q, cl, 3), szv[0], szv[1], szv[2], szv[3]);
+        }
       }
       __syncwarp();
-      if (leader) mbar_arrive(&ready[s]);
-      // refill the stage of tile k-1 once the consumers have released it
-      const int kn = k - 1 + kStages;
-      if (k >= 1 && kn < ntiles) {
-        const int sp = (k - 1) % kStages;
+      if (lane == 0) {
+        mbar_arrive(&prep_ready[r]);
+        mbar_arrive(&raw_free[s]);
+      }
+      // new conv state: last 3 entries of xpad, x'[L-3+i] (zeros for negative t)
+      if (!kPrepass && w == 1 && k == ntiles - 1 && c == p.nchunks - 1 && p.cs_out && active) {
+        IO* cs = static_cast<IO*>(p.cs_out) + (int64_t(b) * p.Di + d) * 3;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+          const int rr = int(p.L - 3 + i - (tt - kHalo));
+          cs[i] = IOT<IO>::from_f(lds_io<IO>(st + S::kXOff + swz<kRow>(rr, col)));
+        }
+      }
+      // refill this raw stage with tile k + kStages once both prep warps are done with it
+      if (issuer && k + kStages < ntiles) {
         good = __all_sync(0xffffffffu,
-                          mbar_wait(&empty[sp], uint32_t((k - 1) / kStages) & 1u, p.status));
-        if (good) issue(kn);
+                          mbar_wait(&raw_free[s], uint32_t(k / kStages) & 1u, p.status));
+        if (!good) break;
+        issue(k + kStages);
       }
     }
-    if (!good) *reinterpret_cast<volatile int*>(prod_abort) = 1;
     named_bar_sync(0, kFwdThreads);
     // drain: every copy this CTA started must land before the CTA exits
-    if (leader && *reinterpret_cast<volatile int*>(prod_abort)) {
+    if (issuer && lane == 0 && !good) {
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         mbar_wait(&full[k % kStages], uint32_t(k / kStages) & 1u, nullptr);
     }
     return;
   }
 
-  // -------------------------------------------------------------- consumer warps
-  const int warp = tid >> 5;
+  // ============================================================== scan warps
   const int chl = lane & 7;
   const int j = lane >> 3;
   const int cl = warp * 8 + chl;  // channel within the CTA tile
-  // d_inner % 8 == 0, so a warp's 8 channels are all in range or all out of range; an
-  // out-of-range warp still walks the tiles (it releases every stage) but reads channel
-  // 0's parameters and stores nothing.
+  // d_inner % 8 == 0: a warp's 8 channels are all in range or all out of range; an
+  // out-of-range warp still walks the tiles (it releases every buffer) but stores nothing.
   const bool active = d0 + cl < p.Di;
   const int64_t d = active ? d0 + cl : 0;
-
-  const float w0 = __ldg(p.conv_w + d * 4 + 0), w1 = __ldg(p.conv_w + d * 4 + 1);
-  const float w2 = __ldg(p.conv_w + d * 4 + 2), w3 = __ldg(p.conv_w + d * 4 + 3);
-  const float cb = p.conv_b ? __ldg(p.conv_b + d) : 0.0f;
-  const float dtb = __ldg(p.dt_bias + d);
-  const float Dd = kPrepass ? 0.0f : __ldg(p.D + d);
   float A2[kS], h[kS], P[kS];
 #pragma unroll
   for (int s = 0; s < kS; ++s) {
-    A2[s] = M::neg_exp(__ldg(p.A_log + d * N + j * kS + s)) * M::a_scale();
+    // A = -exp(A_log) (held times log2 e on the fast path); clamped finite so that a
+    // masked step (Delta = 0) multiplies to exactly 0 and decays by exactly 1.
+    A2[s] = fmaxf(M::neg_exp(__ldg(p.A_log + d * N + j * kS + s)) * M::a_scale(), -FLT_MAX);
     h[s] = 0.0f;
     P[s] = 1.0f;
   }
   if constexpr (!kPrepass) {
-    // carried prefix: fold the (P, H) pairs of chunks 0..c-1
     for (int cc = 0; cc < c; ++cc) {
       const int64_t o = ((int64_t(b) * (p.nchunks - 1) + cc) * p.Di + d) * N + j * kS;
 #pragma unroll
@@ -233,62 +314,28 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     }
   }
 
-  IO* y = static_cast<IO*>(p.y);
-  const int col_bytes = cl * kEs;
+  IO* yrow = static_cast<IO*>(p.y) + (int64_t(b) * p.L + t_begin + j) * p.Di + d;
   bool ok = true;
   for (int k = 0; k < ntiles; ++k) {
-    const int s = k % kStages;
-    const uint32_t st = sb + uint32_t(s * S::kStageBytes);
-    const int64_t tt = t_begin + int64_t(k) * kTileT;
-    ok = __all_sync(0xffffffffu, mbar_wait(&ready[s], uint32_t(k / kStages) & 1u, p.status) &&
-                                     mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status));
+    const int r = k % kPrepBufs;
+    ok = __all_sync(0xffffffffu,
+                    mbar_wait(&prep_ready[r], uint32_t(k / kPrepBufs) & 1u, p.status));
     if (!ok) break;
+    const uint32_t pr = sb + uint32_t(S::kPrepBase + r * S::kPrepBytes);
+    const uint32_t bcf = pr + uint32_t(j * 2 * kS * 4);
+    const uint32_t rec = pr + S::kScOff;
+    const int64_t rem = t_end - (t_begin + int64_t(k) * kTileT) - j;  // my step valid if 4q < rem
 
-    const uint32_t X = st + S::kXOff, Z = st + S::kZOff, DT = st + S::kDtOff;
-    const uint32_t BCF = st + S::kBCfOff + uint32_t(j * 2 * kS * 4);
-
-    // scalar work of step (4q + j) of this tile
-    auto scalar = [&](int q, float& dl, float& dul, float& skip, float& szl) {
-      const int r = 4 * q + j;                        // tile row of this lane's step
-      const float x0 = lds_io<IO>(X + swz<kRow>(r + 1, col_bytes));
-      const float x1 = lds_io<IO>(X + swz<kRow>(r + 2, col_bytes));
-      const float x2 = lds_io<IO>(X + swz<kRow>(r + 3, col_bytes));
-      const float x3 = lds_io<IO>(X + swz<kRow>(r + 4, col_bytes));
-      const float pre = cb + w0 * x0 + w1 * x1 + w2 * x2 + w3 * x3;
-      const float u = M::silu(pre);
-      dl = M::softplus(lds_io<IO>(DT + swz<kRow>(r, col_bytes)) + dtb);
-      dul = dl * u;
-      if constexpr (!kPrepass) {
-        skip = Dd * u;
-        szl = M::silu(lds_io<IO>(Z + swz<kRow>(r, col_bytes)));
-      } else {
-        skip = 0.0f;
-        szl = 0.0f;
-      }
-    };
-
-    float dl, dul, dsk, sz;
-    scalar(0, dl, dul, dsk, sz);
-#pragma unroll 1
-    for (int q = 0; q < kTileT / 4; ++q) {
-      float di[4], dui[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        di[i] = __shfl_sync(0xffffffffu, dl, (i << 3) | chl);
-        dui[i] = __shfl_sync(0xffffffffu, dul, (i << 3) | chl);
-      }
-      const float cur_skip = dsk, cur_sz = sz;
-      if (q + 1 < kTileT / 4) scalar(q + 1, dl, dul, dsk, sz);
-
-      // steps past the chunk end (ragged last tile) leave the state untouched
-      const int64_t left = t_end - (tt + 4 * q);
-      const int nvalid = left >= 4 ? 4 : int(left);
+#pragma unroll 2
+    for (int q = 0; q < kQuads; ++q) {
+      const float4 dv = lds_f32x4(rec + sc_unit(q, cl, 0));
+      const float4 duv = lds_f32x4(rec + sc_unit(q, cl, 1));
+      const float di[4] = {dv.x, dv.y, dv.z, dv.w};
+      const float dui[4] = {duv.x, duv.y, duv.z, duv.w};
       float yp[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        yp[i] = 0.0f;
-        if (i >= nvalid) continue;
-        const uint32_t row = BCF + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
+        const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
         float Bv[kS], Cv[kS];
         if constexpr (kS == 4) {
           const float4 bv = lds_f32x4(row);
@@ -312,7 +359,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         yp[i] = acc;
       }
       if constexpr (!kPrepass) {
-        // reduce-scatter over j (lane bits 4 then 3): lane j ends with step j's sum
+        // reduce-scatter over j (lane bits 4 then 3): lane j ends with step 4q+j's sum
         const bool hi = (j & 2) != 0;
         float k0 = hi ? yp[2] : yp[0], k1 = hi ? yp[3] : yp[1];
         const float s0 = hi ? yp[0] : yp[2], s1 = hi ? yp[1] : yp[3];
@@ -322,17 +369,17 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         float kp = odd ? k1 : k0;
         const float sp = odd ? k0 : k1;
         kp += __shfl_xor_sync(0xffffffffu, sp, 8);
-        if (j < nvalid && active) {
-          const float out = (kp + cur_skip) * cur_sz;
-          y[(int64_t(b) * p.L + tt + 4 * q + j) * p.Di + d] = IOT<IO>::from_f(out);
-        }
+        const float skip = lds_f32(rec + sc_unit(q, cl, 2) + 4 * j);
+        const float sz = lds_f32(rec + sc_unit(q, cl, 3) + 4 * j);
+        if (4 * q < rem && active) yrow[int64_t(4 * q) * p.Di] = IOT<IO>::from_f((kp + skip) * sz);
       }
     }
+    yrow += int64_t(kTileT) * p.Di;
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (lane == 0) mbar_arrive(&prep_free[r]);
   }
 
-  named_bar_sync(0, kFwdThreads);  // pairs with the producer warp's barrier
+  named_bar_sync(0, kFwdThreads);  // pairs with the prep warps' barrier
   if (!ok || !active) return;
 
   if constexpr (kPrepass) {
@@ -342,23 +389,12 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       p.ws_P[o + s] = P[s];
       p.ws_H[o + s] = h[s];
     }
-  } else if (c == p.nchunks - 1) {
-    if (p.h_out) {
-      float* ho = p.h_out + (int64_t(b) * p.Di + d) * N + j * kS;
-      if constexpr (kS == 4) {
-        *reinterpret_cast<float4*>(ho) = make_float4(h[0], h[1], h[2], h[3]);
-      } else {
-        *reinterpret_cast<float2*>(ho) = make_float2(h[0], h[1]);
-      }
-    }
-    if (p.cs_out && j < 3) {
-      // last 3 entries of xpad: x'[L-3+j] (zeros for negative t) from the last x tile
-      const int kl = ntiles - 1;
-      const uint32_t X = sb + uint32_t((kl % kStages) * S::kStageBytes) + S::kXOff;
-      const int64_t tt = t_begin + int64_t(kl) * kTileT;
-      const int r = int(p.L - 3 + j - (tt - kHalo));
-      IO* cs = static_cast<IO*>(p.cs_out) + (int64_t(b) * p.Di + d) * 3;
-      cs[j] = IOT<IO>::from_f(lds_io<IO>(X + swz<kRow>(r, col_bytes)));
+  } else if (c == p.nchunks - 1 && p.h_out) {
+    float* ho = p.h_out + (int64_t(b) * p.Di + d) * N + j * kS;
+    if constexpr (kS == 4) {
+      *reinterpret_cast<float4*>(ho) = make_float4(h[0], h[1], h[2], h[3]);
+    } else {
+      *reinterpret_cast<float2*>(ho) = make_float2(h[0], h[1]);
     }
   }
 }
