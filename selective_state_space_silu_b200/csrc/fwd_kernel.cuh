@@ -1,9 +1,10 @@
 // Fused forward of the selective-SSM mixer core for sm_100a.
 //
-// Work decomposition (warp-specialised CTA: 2 prep warps + 4 scan warps)
-//   CTA        = one batch row b, a tile of kCh = 32 channels, one time chunk.
+// Work decomposition (warp-specialised CTA)
+//   CTA        = one batch row b, a tile of kCh = 32 channels, one time chunk; 4 prep
+//                warps and 4 scan warps.
 //   prep warps = lane c is channel c.  Prep warp 0 also issues the TMA copies.  For each
-//                32-step tile, prep warp w handles steps [16w, 16w+16): it widens B and C
+//                32-step tile, prep warp w handles steps [8w, 8w+8): it widens B and C
 //                to fp32 and computes the per-(t, d) scalars of the operator -- causal
 //                conv + SiLU (u), Delta = softplus(dt_raw + dt_bias), Delta*u, D*u and
 //                SiLU(z) -- once per (t, d), keeping the conv window in registers.
@@ -66,7 +67,8 @@ constexpr int kHalo = 4;         // x' rows loaded before each tile (3 needed)
 constexpr int kStages = 3;       // raw TMA ring depth
 constexpr int kPrepBufs = 2;     // prepared-tile ring depth
 constexpr int kScanWarps = 4;
-constexpr int kPrepWarps = 2;
+constexpr int kPrepWarps = 4;
+constexpr int kPrepSteps = kTileT / kPrepWarps;  // steps per prep warp per tile
 constexpr int kScanThreads = 32 * kScanWarps;
 constexpr int kFwdThreads = 32 * (kScanWarps + kPrepWarps);
 constexpr int kScRec = 64;       // bytes per (quad, channel) scalar record
@@ -171,7 +173,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 
   if (warp >= kScanWarps) {
     // ============================================================ prep warps
-    const int w = warp - kScanWarps;  // 0 or 1: steps [16w, 16w + 16) of each tile
+    const int w = warp - kScanWarps;  // steps [kPrepSteps*w, kPrepSteps*(w+1)) of each tile
     const bool issuer = (w == 0);
     const int cl = lane;               // channel within the CTA tile
     const bool active = d0 + cl < p.Di;
@@ -217,22 +219,22 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       const uint32_t pr = sb + uint32_t(S::kPrepBase + r * S::kPrepBytes);
       const int64_t tt = t_begin + int64_t(k) * kTileT;
 
-      // B (and C) to fp32 for steps [16w, 16w + 16): [t][j]{B[kS], C[kS]}
-      for (int idx = lane; idx < (kTileT / 2) * N; idx += 32) {
-        const int t = (kTileT / 2) * w + idx / N, n = idx % N;
+      // B (and C) to fp32 for this warp's steps: [t][j]{B[kS], C[kS]}
+      for (int idx = lane; idx < kPrepSteps * N; idx += 32) {
+        const int t = kPrepSteps * w + idx / N, n = idx % N;
         const int jj = n / kS, ss = n % kS;
         const uint32_t dst = pr + uint32_t(((t * 4 + jj) * (2 * kS) + ss) * 4);
         sts_f32(dst, lds_io<IO>(st + S::kBOff + (t * N + n) * kEs));
         if constexpr (!kPrepass) sts_f32(dst + kS * 4, lds_io<IO>(st + S::kCOff + (t * N + n) * kEs));
       }
 
-      // scalars of steps [16w, 16w + 16) of channel cl; x' tile row r holds t = tt - 4 + r
-      const int t0 = (kTileT / 2) * w;
+      // scalars of this warp's steps for channel cl; x' tile row r holds t = tt - 4 + r
+      const int t0 = kPrepSteps * w;
       float xa = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 1, col));
       float xb = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 2, col));
       float xc = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 3, col));
 #pragma unroll 1
-      for (int q = t0 / 4; q < t0 / 4 + kQuads / 2; ++q) {
+      for (int q = t0 / 4; q < (t0 + kPrepSteps) / 4; ++q) {
         float dv[4], duv[4], skv[4], szv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -264,7 +266,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         mbar_arrive(&raw_free[s]);
       }
       // new conv state: last 3 entries of xpad, x'[L-3+i] (zeros for negative t)
-      if (!kPrepass && w == 1 && k == ntiles - 1 && c == p.nchunks - 1 && p.cs_out && active) {
+      if (!kPrepass && w == kPrepWarps - 1 && k == ntiles - 1 && c == p.nchunks - 1 && p.cs_out && active) {
         IO* cs = static_cast<IO*>(p.cs_out) + (int64_t(b) * p.Di + d) * 3;
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
@@ -313,6 +315,14 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       for (int s = 0; s < kS; ++s) h[s] = p.ws_P[o + s] * h[s] + p.ws_H[o + s];
     }
   }
+  // packed copies for the fast path (pairs of states)
+  f32x2 A2p[kS / 2], hp[kS / 2], Pp[kS / 2];
+#pragma unroll
+  for (int pp = 0; pp < kS / 2; ++pp) {
+    A2p[pp] = pk2(A2[2 * pp], A2[2 * pp + 1]);
+    hp[pp] = pk2(h[2 * pp], h[2 * pp + 1]);
+    Pp[pp] = pk2(1.0f, 1.0f);
+  }
 
   IO* yrow = static_cast<IO*>(p.y) + (int64_t(b) * p.L + t_begin + j) * p.Di + d;
   bool ok = true;
@@ -333,6 +343,40 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       const float di[4] = {dv.x, dv.y, dv.z, dv.w};
       const float dui[4] = {duv.x, duv.y, duv.z, duv.w};
       float yp[4];
+      if constexpr (!kPrecise) {
+        // fast path: states in packed pairs; per step and pair one f32x2 multiply for
+        // Delta*A, two ex2, one f32x2 multiply for Delta*u*B and f32x2 FMAs for h and C.h
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
+          const f32x2 d2 = pk2(di[i], di[i]), du2 = pk2(dui[i], dui[i]);
+          f32x2 Bp[kS / 2], Cp[kS / 2];
+          if constexpr (kS == 4) {
+            const float4 bv = lds_f32x4(row);
+            Bp[0] = pk2(bv.x, bv.y); Bp[1] = pk2(bv.z, bv.w);
+            if constexpr (!kPrepass) {
+              const float4 cv = lds_f32x4(row + 16);
+              Cp[0] = pk2(cv.x, cv.y); Cp[1] = pk2(cv.z, cv.w);
+            }
+          } else {
+            const float4 v = lds_f32x4(row);
+            Bp[0] = pk2(v.x, v.y); Cp[0] = pk2(v.z, v.w);
+          }
+          f32x2 acc2 = pk2(0.0f, 0.0f);
+#pragma unroll
+          for (int pp = 0; pp < kS / 2; ++pp) {
+            float xl, xh;
+            upk2(mul2(d2, A2p[pp]), xl, xh);
+            const f32x2 a2 = pk2(ex2_approx(xl), ex2_approx(xh));
+            hp[pp] = fma2(a2, hp[pp], mul2(du2, Bp[pp]));
+            if constexpr (kPrepass) Pp[pp] = mul2(Pp[pp], a2);
+            else acc2 = fma2(Cp[pp], hp[pp], acc2);
+          }
+          float al, ah;
+          upk2(acc2, al, ah);
+          yp[i] = al + ah;
+        }
+      } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
@@ -358,6 +402,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         }
         yp[i] = acc;
       }
+      }
       if constexpr (!kPrepass) {
         // reduce-scatter over j (lane bits 4 then 3): lane j ends with step 4q+j's sum
         const bool hi = (j & 2) != 0;
@@ -381,6 +426,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
 
   named_bar_sync(0, kFwdThreads);  // pairs with the prep warps' barrier
   if (!ok || !active) return;
+  if constexpr (!kPrecise) {
+#pragma unroll
+    for (int pp = 0; pp < kS / 2; ++pp) {
+      upk2(hp[pp], h[2 * pp], h[2 * pp + 1]);
+      upk2(Pp[pp], P[2 * pp], P[2 * pp + 1]);
+    }
+  }
 
   if constexpr (kPrepass) {
     const int64_t o = ((int64_t(b) * (p.nchunks - 1) + c) * p.Di + d) * N + j * kS;
