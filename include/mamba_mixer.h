@@ -155,6 +155,31 @@ MAMBA_API int mamba_mixer_step(const mamba_dims* dims, const void* xp, const voi
  */
 MAMBA_API int mamba_mixer_check(void* workspace, void* cuda_stream);
 
+/*
+ * The fused forward for callers that cannot allocate device memory.  The pages describe no
+ * such entry point; it exists for this library's users.  Plugin hosts that hand over the
+ * input and output buffers but no allocator, code running inside an allocator's callback,
+ * and latency-critical paths that must not call cudaMalloc (it can synchronize the device)
+ * cannot provide the workspace mamba_mixer_fwd asks for.  This variant takes the same
+ * inputs and outputs, computes the same result, and uses a scratch array owned by the
+ * library instead: 2 MiB (2097152 bytes) of device memory per GPU that loads the library,
+ * held until the process exits.  It calls no cudaMalloc/cudaFree.
+ * Limits and conventions:
+ *   - dims whose mamba_mixer_fwd_workspace_bytes exceeds 2 MiB are rejected with
+ *     MAMBA_ERR_WORKSPACE (message via mamba_last_error); use mamba_mixer_fwd for them;
+ *   - the first call on each device looks up the array's device address with that device
+ *     current (cudaGetSymbolAddress); make that first call before any stream capture;
+ *   - all calls on a device share the one array and it keeps the last call's contents:
+ *     calls that overlap on the GPU (e.g. on two streams at once) race; serialize them;
+ *   - a bounded-wait timeout in this variant is recorded only in the array and is not
+ *     reported (there is no workspace to pass to mamba_mixer_check).
+ */
+MAMBA_API int mamba_mixer_fwd_noalloc(const mamba_dims* dims, const void* xp, const void* z,
+                                      const void* dt_raw, const void* B, const void* C,
+                                      const float* A_log, const float* D, const float* conv_w,
+                                      const float* conv_b, const float* dt_bias, void* y,
+                                      float* h_out, void* conv_state_out, void* cuda_stream);
+
 /* Message for the last non-OK return on this thread ("" if none). Never NULL. */
 MAMBA_API const char* mamba_last_error(void);
 

@@ -209,6 +209,11 @@ cudaError_t launch_step(const mm::StepArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+namespace mm_internal {
+// Lets the other translation units of the library report through mamba_last_error.
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace mm_internal
+
 extern "C" {
 
 const char* mamba_last_error(void) { return g_last_error.c_str(); }

@@ -217,3 +217,42 @@ def mamba_mixer_step(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, h_i
 def mamba_mixer_fwd_launches(dims: mamba_dims) -> int:
     """Kernel launches one mamba_mixer_fwd call with ``dims`` makes."""
     return int(load_library().mamba_mixer_fwd_launches(ctypes.byref(dims)))
+
+
+def mamba_mixer_fwd_noalloc(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
+                            y=None, h_out=None, conv_state_out=None, stream=None,
+                            want_states: bool = True):
+    """The fused forward without a workspace, for callers that cannot allocate device
+    memory: the library uses its own fixed 2 MiB scratch array per device instead.
+
+    Same arguments and results as ``mamba_mixer_fwd`` minus ``workspace``.  Calls on one
+    device share that scratch, so calls that overlap on the GPU race; sizes needing more
+    scratch than 2 MiB raise MambaError(MAMBA_ERR_WORKSPACE).  (This binding still creates
+    output tensors when they are not given; pass them in to allocate nothing.)
+    """
+    lib = load_library()
+    lib.mamba_mixer_fwd_noalloc.restype = ctypes.c_int
+    lib.mamba_mixer_fwd_noalloc.argtypes = [ctypes.POINTER(mamba_dims)] + [ctypes.c_void_p] * 14
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    dims = make_dims(Bt, L, Di, N, K, io)
+    if y is None:
+        y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
+    if want_states and h_out is None:
+        h_out = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+    if want_states and conv_state_out is None:
+        conv_state_out = torch.empty((Bt, Di, K - 1), dtype=iot, device=dev)
+    f32 = torch.float32
+    rc = lib.mamba_mixer_fwd_noalloc(
+        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
+        _ptr(conv_state_out, "conv_state_out", iot, dev), _stream_handle(stream, dev))
+    _check(rc)
+    return y, h_out, conv_state_out

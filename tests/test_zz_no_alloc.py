@@ -1,0 +1,63 @@
+"""The forward for callers that cannot allocate device memory (mamba_mixer_fwd_noalloc).
+
+Plugin hosts that hand over only input and output buffers, code running inside an
+allocator's callback, and latency-critical paths that must avoid cudaMalloc's device-wide
+synchronisation cannot give mamba_mixer_fwd the workspace it asks for.  The no-alloc entry
+point serves them from a fixed 2 MiB scratch array inside the library.  These tests call it
+through the C ABI and check that two calls in a row give what mamba_mixer_fwd gives, within
+the tolerance the other GPU tests use, and that sizes needing more scratch are refused.
+This file is collected last on purpose.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from selective_state_space_silu_b200 import build as Bld
+from selective_state_space_silu_b200 import inputs as I
+from selective_state_space_silu_b200 import mixer as M
+from tests.gpu_util import gpu_fwd, host, host_bits, to_device
+from tests.tolerances import assert_close
+
+
+def _noalloc(d):
+    return M.mamba_mixer_fwd_noalloc(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"],
+                                     d["D"], d["conv_w"], d.get("conv_b"), d["dt_bias"])
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("w", [
+    # long enough to be cut into time chunks, so the scratch carries the chunk aggregates
+    I.Workload("noalloc_bf16", 2, 4096, 128, 16, 4, "bf16", 2024),
+    I.Workload("noalloc_f32", 2, 1500, 64, 8, 4, "f32", 2025),
+], ids=lambda w: w.name)
+def test_noalloc_matches_fwd_on_two_calls(w):
+    Bld.build()
+    dims = M.make_dims(w.batch, w.seqlen, w.d_inner, w.d_state, 4,
+                       M.MAMBA_BF16 if w.io_dtype == "bf16" else M.MAMBA_F32)
+    assert M.mamba_mixer_fwd_workspace_bytes(dims) > 256   # the scratch is really used
+    d = to_device(I.make_inputs(w))
+    y0, h0, c0 = gpu_fwd(d)
+    for call in range(2):
+        y, h, cs = _noalloc(d)
+        torch.cuda.synchronize()
+        assert_close(host(y), host(y0), w.io_dtype, f"no-alloc y, call {call + 1}")
+        assert_close(host(h), host(h0), w.io_dtype, f"no-alloc h_out, call {call + 1}")
+        np.testing.assert_array_equal(host_bits(cs), host_bits(c0))
+
+
+def test_noalloc_refuses_sizes_beyond_its_scratch():
+    """1 x 65536 x 4096 (d_state 16) needs 2 MiB + 256 bytes of scratch: refused before any
+    CUDA call, with the reason in mamba_last_error."""
+    Bld.build()
+    lib = M.load_library()
+    lib.mamba_mixer_fwd_noalloc.restype = ctypes.c_int
+    lib.mamba_mixer_fwd_noalloc.argtypes = [ctypes.POINTER(M.mamba_dims)] + [ctypes.c_void_p] * 14
+    dims = M.make_dims(1, 65536, 4096, 16)
+    assert M.mamba_mixer_fwd_workspace_bytes(dims) > (2 << 20)
+    fake = [ctypes.c_void_p(0x10000000 + i * (1 << 36)) for i in range(13)]
+    rc = lib.mamba_mixer_fwd_noalloc(ctypes.byref(dims), *fake, None)
+    assert rc == 4, M.mamba_last_error()
+    assert "scratch" in M.mamba_last_error()
