@@ -87,8 +87,10 @@ struct FwdSmem {
   static constexpr int kBOff = kDtOff + align1k(kZBytes);
   static constexpr int kCOff = kBOff + align1k(kBBytes);
   static constexpr int kRawStage = kCOff + align1k(kBBytes);
-  // prepared tile: fp32 B/C as [t][j]{B[kS], C[kS]}, then scalar records [q][c]
-  static constexpr int kBCfBytes = kTileT * 2 * N * 4;
+  // prepared tile: B/C records [t][j]{B[kS], C[kS]} in the I/O type (fp32 or bf16),
+  // then the scalar records [q][c]
+  static constexpr int kBCRec = 2 * (N / 4) * int(sizeof(IO));   // 16 or 32 (N=16), 8/16 (N=8)
+  static constexpr int kBCfBytes = kTileT * 4 * kBCRec;
   static constexpr int kScOff = align1k(kBCfBytes);
   static constexpr int kPrepBytes = kScOff + kQuads * kCh * kScRec;
   static constexpr int kPrepBase = kStages * kRawStage;
@@ -121,6 +123,34 @@ __device__ __forceinline__ float lds_io<__nv_bfloat16>(uint32_t a) {
   return __uint_as_float(lds_u16(a) << 16);
 }
 
+// Copies kHalf bytes of B and kHalf bytes of C into one B/C record.
+template <int kHalf>
+__device__ __forceinline__ void copy_record(uint32_t dst, uint32_t b, uint32_t c, bool b_only) {
+  if constexpr (kHalf == 8) {
+    uint32_t b0, b1, c0 = 0, c1 = 0;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(b));
+    if (!b_only) asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(c0), "=r"(c1) : "r"(c));
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(b0), "r"(b1), "r"(c0),
+                 "r"(c1) : "memory");
+  } else if constexpr (kHalf == 4) {
+    uint32_t b0, c0 = 0;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b0) : "r"(b));
+    if (!b_only) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(c0) : "r"(c));
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(b0), "r"(c0) : "memory");
+  } else {  // 16 bytes each (fp32, 4 states)
+    const float4 bv = lds_f32x4(b);
+    const float4 cv = b_only ? make_float4(0.f, 0.f, 0.f, 0.f) : lds_f32x4(c);
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(bv.x), "f"(bv.y),
+                 "f"(bv.z), "f"(bv.w) : "memory");
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "f"(cv.x), "f"(cv.y),
+                 "f"(cv.z), "f"(cv.w) : "memory");
+  }
+}
+
+// The two bf16 halves of a 32-bit word as fp32 (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
 __device__ __forceinline__ void sts_f32x4(uint32_t a, float x, float y, float z, float w) {
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x), "f"(y), "f"(z),
                "f"(w) : "memory");
@@ -136,6 +166,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
   constexpr int kS = N / 4;
   constexpr int kRow = S::kRow;
   constexpr int kEs = int(sizeof(IO));
+  static_assert(kPrecise == (sizeof(IO) == 4), "fp32 I/O takes the precise math, bf16 the fast");
 
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
@@ -219,13 +250,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       const uint32_t pr = sb + uint32_t(S::kPrepBase + r * S::kPrepBytes);
       const int64_t tt = t_begin + int64_t(k) * kTileT;
 
-      // B (and C) to fp32 for this warp's steps: [t][j]{B[kS], C[kS]}
-      for (int idx = lane; idx < kPrepSteps * N; idx += 32) {
-        const int t = kPrepSteps * w + idx / N, n = idx % N;
-        const int jj = n / kS, ss = n % kS;
-        const uint32_t dst = pr + uint32_t(((t * 4 + jj) * (2 * kS) + ss) * 4);
-        sts_f32(dst, lds_io<IO>(st + S::kBOff + (t * N + n) * kEs));
-        if constexpr (!kPrepass) sts_f32(dst + kS * 4, lds_io<IO>(st + S::kCOff + (t * N + n) * kEs));
+      // B and C re-laid out for this warp's steps as [t][j]{B[kS], C[kS]} (no conversion):
+      // lane (t, j) copies B[t][j*kS ..] and C[t][j*kS ..] into one record
+      {
+        constexpr int kHalf = S::kBCRec / 2;            // bytes of B (or C) per record
+        for (int idx = lane; idx < kPrepSteps * 4; idx += 32) {
+          const int t = kPrepSteps * w + idx / 4, jj = idx % 4;
+          const uint32_t src = uint32_t(t * N * kEs + jj * kHalf);
+          const uint32_t dst = pr + uint32_t((t * 4 + jj) * S::kBCRec);
+          copy_record<kHalf>(dst, st + S::kBOff + src, st + S::kCOff + src, kPrepass);
+        }
       }
 
       // scalars of this warp's steps for channel cl; x' tile row r holds t = tt - 4 + r
@@ -233,8 +267,9 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       float xa = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 1, col));
       float xb = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 2, col));
       float xc = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 3, col));
-#pragma unroll 1
-      for (int q = t0 / 4; q < (t0 + kPrepSteps) / 4; ++q) {
+#pragma unroll
+      for (int qq = 0; qq < kPrepSteps / 4; ++qq) {
+        const int q = t0 / 4 + qq;
         float dv[4], duv[4], skv[4], szv[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -332,7 +367,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
                     mbar_wait(&prep_ready[r], uint32_t(k / kPrepBufs) & 1u, p.status));
     if (!ok) break;
     const uint32_t pr = sb + uint32_t(S::kPrepBase + r * S::kPrepBytes);
-    const uint32_t bcf = pr + uint32_t(j * 2 * kS * 4);
+    const uint32_t bcf = pr + uint32_t(j * S::kBCRec);
     const uint32_t rec = pr + S::kScOff;
     const int64_t rem = t_end - (t_begin + int64_t(k) * kTileT) - j;  // my step valid if 4q < rem
 
@@ -348,19 +383,19 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         // Delta*A, two ex2, one f32x2 multiply for Delta*u*B and f32x2 FMAs for h and C.h
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
+          const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * S::kBCRec);
           const f32x2 d2 = pk2(di[i], di[i]), du2 = pk2(dui[i], dui[i]);
           f32x2 Bp[kS / 2], Cp[kS / 2];
-          if constexpr (kS == 4) {
-            const float4 bv = lds_f32x4(row);
-            Bp[0] = pk2(bv.x, bv.y); Bp[1] = pk2(bv.z, bv.w);
-            if constexpr (!kPrepass) {
-              const float4 cv = lds_f32x4(row + 16);
-              Cp[0] = pk2(cv.x, cv.y); Cp[1] = pk2(cv.z, cv.w);
-            }
-          } else {
-            const float4 v = lds_f32x4(row);
-            Bp[0] = pk2(v.x, v.y); Cp[0] = pk2(v.z, v.w);
+          if constexpr (kS == 4) {   // bf16 record {B0..B3, C0..C3}
+            uint32_t w0, w1, w2, w3;
+            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(row));
+            Bp[0] = pk2(bf16_lo(w0), bf16_hi(w0)); Bp[1] = pk2(bf16_lo(w1), bf16_hi(w1));
+            Cp[0] = pk2(bf16_lo(w2), bf16_hi(w2)); Cp[1] = pk2(bf16_lo(w3), bf16_hi(w3));
+          } else {                   // bf16 record {B0, B1, C0, C1}
+            uint32_t w0, w1;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(row));
+            Bp[0] = pk2(bf16_lo(w0), bf16_hi(w0)); Cp[0] = pk2(bf16_lo(w1), bf16_hi(w1));
           }
           f32x2 acc2 = pk2(0.0f, 0.0f);
 #pragma unroll
@@ -379,8 +414,8 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       } else {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * 2 * kS * 4);
-        float Bv[kS], Cv[kS];
+        const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * S::kBCRec);
+        float Bv[kS], Cv[kS];   // fp32 record {B[kS], C[kS]}
         if constexpr (kS == 4) {
           const float4 bv = lds_f32x4(row);
           Bv[0] = bv.x; Bv[1] = bv.y; Bv[2] = bv.z; Bv[3] = bv.w;
