@@ -38,6 +38,33 @@ struct StepArgs {
 constexpr int kStepThreads = 256;
 constexpr int kStepLanes = 4;
 
+// Streaming (evict-first) 16/8-byte accesses for the state, which is touched once.
+__device__ __forceinline__ float4 ldcs4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+__device__ __forceinline__ float2 ldcs2(const float* p) { return __ldcs(reinterpret_cast<const float2*>(p)); }
+
+// kS consecutive I/O elements (8 or 4 bytes for bf16, 16 or 8 for fp32) as fp32.
+template <int kS, typename IO>
+__device__ __forceinline__ void ld_small(const IO* p, float* out) {
+  if constexpr (sizeof(IO) == 2) {
+    if constexpr (kS == 4) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+      out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
+      out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+    } else {
+      const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(p));
+      out[0] = __uint_as_float(v << 16); out[1] = __uint_as_float(v & 0xffff0000u);
+    }
+  } else {
+    if constexpr (kS == 4) {
+      const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+      out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    } else {
+      const float2 v = __ldg(reinterpret_cast<const float2*>(p));
+      out[0] = v.x; out[1] = v.y;
+    }
+  }
+}
+
 template <int N, typename IO, bool kPrecise>
 __global__ void __launch_bounds__(kStepThreads)
 step_kernel(StepArgs a) {
@@ -51,45 +78,46 @@ step_kernel(StepArgs a) {
   const int64_t b = ch / a.Di;
   const int64_t d = ch - b * a.Di;
 
-  const IO* cs_in = static_cast<const IO*>(a.cs_in);
-  // --- loads
-  float h[S], Ak[S], Bv[S], Cv[S];
+  // --- loads: the state first (the bulk of the bytes), then the rest
+  float h[S], A2[S], Bv[S], Cv[S];
   const float* hp = a.h_in + ch * N + j * S;
   if constexpr (S == 4) {
-    const float4 v = *reinterpret_cast<const float4*>(hp);
+    const float4 v = ldcs4(hp);
     h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+    const float4 al = __ldg(reinterpret_cast<const float4*>(a.A_log + d * N + j * S));
+    A2[0] = al.x; A2[1] = al.y; A2[2] = al.z; A2[3] = al.w;
   } else {
-    const float2 v = *reinterpret_cast<const float2*>(hp);
+    const float2 v = ldcs2(hp);
     h[0] = v.x; h[1] = v.y;
+    const float2 al = __ldg(reinterpret_cast<const float2*>(a.A_log + d * N + j * S));
+    A2[0] = al.x; A2[1] = al.y;
   }
-  const IO* Bm = static_cast<const IO*>(a.B) + b * N + j * S;
-  const IO* Cm = static_cast<const IO*>(a.C) + b * N + j * S;
-#pragma unroll
-  for (int s = 0; s < S; ++s) {
-    Ak[s] = M::neg_exp(__ldg(a.A_log + d * N + j * S + s)) * M::a_scale();
-    Bv[s] = IOT<IO>::ld(Bm + s);
-    Cv[s] = IOT<IO>::ld(Cm + s);
-  }
-  const float s0 = IOT<IO>::to_f(cs_in[ch * 3 + 0]);
-  const float s1 = IOT<IO>::to_f(cs_in[ch * 3 + 1]);
-  const float s2 = IOT<IO>::to_f(cs_in[ch * 3 + 2]);
+  ld_small<S>(static_cast<const IO*>(a.B) + b * N + j * S, Bv);
+  ld_small<S>(static_cast<const IO*>(a.C) + b * N + j * S, Cv);
+  const IO* cs_in = static_cast<const IO*>(a.cs_in) + ch * 3;
+  const float s0 = IOT<IO>::to_f(cs_in[0]);
+  const float s1 = IOT<IO>::to_f(cs_in[1]);
+  const float s2 = IOT<IO>::to_f(cs_in[2]);
   const float xt = IOT<IO>::ld(static_cast<const IO*>(a.xp) + ch);
   const float zt = IOT<IO>::ld(static_cast<const IO*>(a.z) + ch);
   const float dtr = IOT<IO>::ld(static_cast<const IO*>(a.dt) + ch);
+  const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w + d * 4));
+  const float cb = a.conv_b ? __ldg(a.conv_b + d) : 0.0f;
+  const float dtb = __ldg(a.dt_bias + d);
+  const float Dd = __ldg(a.D + d);
 
   // --- conv + SiLU, softplus (same on the four lanes)
-  const float cb = a.conv_b ? __ldg(a.conv_b + d) : 0.0f;
-  const float* w = a.conv_w + d * 4;
-  const float pre = cb + __ldg(w) * s0 + __ldg(w + 1) * s1 + __ldg(w + 2) * s2 + __ldg(w + 3) * xt;
+  const float pre = cb + w.x * s0 + w.y * s1 + w.z * s2 + w.w * xt;
   const float u = M::silu(pre);
-  const float delta = M::softplus(dtr + __ldg(a.dt_bias + d));
+  const float delta = M::softplus(dtr + dtb);
   const float du = delta * u;
 
   // --- one recurrence step on this lane's states
   float part = 0.0f;
 #pragma unroll
   for (int s = 0; s < S; ++s) {
-    h[s] = M::decay(delta, Ak[s]) * h[s] + du * Bv[s];
+    const float Ak = M::neg_exp(A2[s]) * M::a_scale();
+    h[s] = M::decay(delta, Ak) * h[s] + du * Bv[s];
     part += Cv[s] * h[s];
   }
   part += __shfl_xor_sync(0xffffffffu, part, 1);
@@ -98,18 +126,78 @@ step_kernel(StepArgs a) {
   // --- stores
   float* ho = a.h_out + ch * N + j * S;
   if constexpr (S == 4) {
-    *reinterpret_cast<float4*>(ho) = make_float4(h[0], h[1], h[2], h[3]);
+    __stcs(reinterpret_cast<float4*>(ho), make_float4(h[0], h[1], h[2], h[3]));
   } else {
-    *reinterpret_cast<float2*>(ho) = make_float2(h[0], h[1]);
+    __stcs(reinterpret_cast<float2*>(ho), make_float2(h[0], h[1]));
   }
   if (j == 0) {
-    const float out = (part + __ldg(a.D + d) * u) * M::silu(zt);
+    const float out = (part + Dd * u) * M::silu(zt);
     static_cast<IO*>(a.y)[ch] = IOT<IO>::from_f(out);
     IO* cso = static_cast<IO*>(a.cs_out) + ch * 3;
     cso[0] = IOT<IO>::from_f(s1);
     cso[1] = IOT<IO>::from_f(s2);
     cso[2] = IOT<IO>::from_f(xt);
   }
+}
+
+// One thread per channel (b, d) with all N states: 4 (N = 16) or 2 (N = 8) 16-byte state
+// loads in flight per thread, and the per-channel scalar work done once.
+template <int N, typename IO, bool kPrecise>
+__global__ void __launch_bounds__(kStepThreads)
+step_kernel_1t(StepArgs a) {
+  using M = Math<kPrecise>;
+  const int64_t ch = int64_t(blockIdx.x) * kStepThreads + threadIdx.x;  // flat (b, d)
+  if (ch >= a.batch * a.Di) return;
+  const int64_t b = ch / a.Di;
+  const int64_t d = ch - b * a.Di;
+
+  float h[N], A2[N], Bv[N], Cv[N];
+  const float* hp = a.h_in + ch * N;
+#pragma unroll
+  for (int k = 0; k < N; k += 4) {
+    const float4 v = ldcs4(hp + k);
+    h[k] = v.x; h[k + 1] = v.y; h[k + 2] = v.z; h[k + 3] = v.w;
+  }
+#pragma unroll
+  for (int k = 0; k < N; k += 4) {
+    const float4 al = __ldg(reinterpret_cast<const float4*>(a.A_log + d * N + k));
+    A2[k] = al.x; A2[k + 1] = al.y; A2[k + 2] = al.z; A2[k + 3] = al.w;
+  }
+  load_row<N>(static_cast<const IO*>(a.B) + b * N, Bv);
+  load_row<N>(static_cast<const IO*>(a.C) + b * N, Cv);
+  const IO* cs_in = static_cast<const IO*>(a.cs_in) + ch * 3;
+  const float s0 = IOT<IO>::to_f(cs_in[0]);
+  const float s1 = IOT<IO>::to_f(cs_in[1]);
+  const float s2 = IOT<IO>::to_f(cs_in[2]);
+  const float xt = IOT<IO>::ld(static_cast<const IO*>(a.xp) + ch);
+  const float zt = IOT<IO>::ld(static_cast<const IO*>(a.z) + ch);
+  const float dtr = IOT<IO>::ld(static_cast<const IO*>(a.dt) + ch);
+  const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w + d * 4));
+  const float cb = a.conv_b ? __ldg(a.conv_b + d) : 0.0f;
+  const float dtb = __ldg(a.dt_bias + d);
+  const float Dd = __ldg(a.D + d);
+
+  const float pre = cb + w.x * s0 + w.y * s1 + w.z * s2 + w.w * xt;
+  const float u = M::silu(pre);
+  const float delta = M::softplus(dtr + dtb);
+  const float du = delta * u;
+  float acc = 0.0f;
+#pragma unroll
+  for (int n = 0; n < N; ++n) {
+    const float Ak = M::neg_exp(A2[n]) * M::a_scale();
+    h[n] = M::decay(delta, Ak) * h[n] + du * Bv[n];
+    acc += Cv[n] * h[n];
+  }
+  float* ho = a.h_out + ch * N;
+#pragma unroll
+  for (int k = 0; k < N; k += 4)
+    __stcs(reinterpret_cast<float4*>(ho + k), make_float4(h[k], h[k + 1], h[k + 2], h[k + 3]));
+  const float out = (acc + Dd * u) * M::silu(zt);
+  static_cast<IO*>(a.y)[ch] = IOT<IO>::from_f(out);
+  IO* cso = static_cast<IO*>(a.cs_out) + ch * 3;
+  cso[0] = IOT<IO>::from_f(s1);
+  cso[1] = IOT<IO>::from_f(s2);
+  cso[2] = IOT<IO>::from_f(xt);
 }
 
 }  // namespace mm

@@ -49,14 +49,20 @@ def test_noalloc_matches_fwd_on_two_calls(w):
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch():
-    """1 x 65536 x 4096 (d_state 16) needs 2 MiB + 256 bytes of scratch: refused before any
-    CUDA call, with the reason in mamba_last_error."""
+    """Sizes whose forward needs more than the fixed 2 MiB of scratch are refused before any
+    CUDA call, with the reason in mamba_last_error.  (The dims are searched for, since the
+    scratch a forward needs depends on how the library splits long sequences.)"""
     Bld.build()
     lib = M.load_library()
     lib.mamba_mixer_fwd_noalloc.restype = ctypes.c_int
     lib.mamba_mixer_fwd_noalloc.argtypes = [ctypes.POINTER(M.mamba_dims)] + [ctypes.c_void_p] * 14
-    dims = M.make_dims(1, 65536, 4096, 16)
-    assert M.mamba_mixer_fwd_workspace_bytes(dims) > (2 << 20)
+    dims = None
+    for Di in range(256, 65536, 256):
+        cand = M.make_dims(1, 1 << 20, Di, 16)
+        if M.mamba_mixer_fwd_workspace_bytes(cand) > (2 << 20):
+            dims = cand
+            break
+    assert dims is not None, "no size exceeds the scratch: the refusal path would be dead"
     fake = [ctypes.c_void_p(0x10000000 + i * (1 << 36)) for i in range(13)]
     rc = lib.mamba_mixer_fwd_noalloc(ctypes.byref(dims), *fake, None)
     assert rc == 4, M.mamba_last_error()
