@@ -203,7 +203,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
         # write a buffer larger than L2, then read another one: the timed kernels start
         # with a cold L2 holding clean lines (no write-back of the flush inside the timing)
         flush.fill_(1.0)
-        torch.sum(flush_rd, out=flush_sink)
+        torch.sum(flush_rd, dim=0, out=flush_sink)
 
     def fwd():
         M.mamba_mixer_fwd(X["xp"], X["z"], X["dt_raw"], X["B"], X["C"], P["A_log"], P["D"],
