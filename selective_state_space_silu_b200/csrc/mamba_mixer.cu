@@ -86,6 +86,10 @@ int check_dims(const mamba_dims* d, Sizes* s) {
       !mul_ok(d->batch * d->d_inner, d->d_conv - 1, &s->cstate) || s->act > (INT64_MAX >> 3))
     return fail(MAMBA_ERR_INVALID_ARGUMENT, "sizes overflow");
   if (d->batch > 65535) return fail(MAMBA_ERR_UNSUPPORTED, "batch > 65535");
+  if (d->d_inner > (int64_t(1) << 28))
+    return fail(MAMBA_ERR_UNSUPPORTED, "d_inner > 2^28");
+  if (d->seqlen > (int64_t(1) << 31) - 512)
+    return fail(MAMBA_ERR_UNSUPPORTED, "seqlen >= 2^31 - 512");
   s->esize = d->io_dtype == MAMBA_F32 ? 4 : 2;
   return MAMBA_OK;
 }
@@ -206,9 +210,8 @@ cudaError_t launch_fwd(const FwdMaps& m, const mm::FwdParams& a, int64_t batch, 
 
 template <int N, typename IO, bool P>
 cudaError_t launch_step(const mm::StepArgs& a, cudaStream_t st) {
-  const int64_t threads = a.batch * a.Di * mm::kStepLanes;
-  const int64_t blocks = (threads + mm::kStepThreads - 1) / mm::kStepThreads;
-  mm::step_kernel<N, IO, P><<<unsigned(blocks), mm::kStepThreads, 0, st>>>(a);
+  const int64_t bx = (a.Di * mm::kStepLanes + mm::kStepThreads - 1) / mm::kStepThreads;
+  mm::step_kernel<N, IO, P><<<dim3(unsigned(bx), unsigned(a.batch)), mm::kStepThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

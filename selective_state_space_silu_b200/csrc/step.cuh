@@ -37,6 +37,7 @@ struct StepArgs {
 
 constexpr int kStepThreads = 256;
 constexpr int kStepLanes = 4;
+static_assert(kStepLanes == 4, "the index math below assumes 4 lanes per channel");
 
 // Streaming (evict-first) 16/8-byte accesses for the state, which is touched once.
 __device__ __forceinline__ float4 ldcs4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
@@ -70,13 +71,14 @@ __global__ void __launch_bounds__(kStepThreads)
 step_kernel(StepArgs a) {
   using M = Math<kPrecise>;
   constexpr int S = N / kStepLanes;  // states per lane
-  const int64_t gt = int64_t(blockIdx.x) * kStepThreads + threadIdx.x;
-  const int64_t ch = gt / kStepLanes;      // flat (b, d)
-  const int j = int(gt % kStepLanes);
-  // batch*Di*4 is a multiple of 32 (Di % 8 == 0): a warp is all in range or all out.
-  if (ch >= a.batch * a.Di) return;
-  const int64_t b = ch / a.Di;
-  const int64_t d = ch - b * a.Di;
+  // grid: (ceil(4*Di / kStepThreads), batch); no integer division on the device
+  const int t = blockIdx.x * kStepThreads + threadIdx.x;
+  const int64_t b = blockIdx.y;
+  const int64_t d = t >> 2;                // kStepLanes == 4
+  const int j = t & 3;
+  // 4*Di is a multiple of 32 (Di % 8 == 0): a warp is all in range or all out.
+  if (d >= a.Di) return;
+  const int64_t ch = b * a.Di + d;         // flat (b, d)
 
   // --- loads: the state first (the bulk of the bytes), then the rest
   float h[S], A2[S], Bv[S], Cv[S];
@@ -138,66 +140,6 @@ step_kernel(StepArgs a) {
     cso[1] = IOT<IO>::from_f(s2);
     cso[2] = IOT<IO>::from_f(xt);
   }
-}
-
-// One thread per channel (b, d) with all N states: 4 (N = 16) or 2 (N = 8) 16-byte state
-// loads in flight per thread, and the per-channel scalar work done once.
-template <int N, typename IO, bool kPrecise>
-__global__ void __launch_bounds__(kStepThreads)
-step_kernel_1t(StepArgs a) {
-  using M = Math<kPrecise>;
-  const int64_t ch = int64_t(blockIdx.x) * kStepThreads + threadIdx.x;  // flat (b, d)
-  if (ch >= a.batch * a.Di) return;
-  const int64_t b = ch / a.Di;
-  const int64_t d = ch - b * a.Di;
-
-  float h[N], A2[N], Bv[N], Cv[N];
-  const float* hp = a.h_in + ch * N;
-#pragma unroll
-  for (int k = 0; k < N; k += 4) {
-    const float4 v = ldcs4(hp + k);
-    h[k] = v.x; h[k + 1] = v.y; h[k + 2] = v.z; h[k + 3] = v.w;
-  }
-#pragma unroll
-  for (int k = 0; k < N; k += 4) {
-    const float4 al = __ldg(reinterpret_cast<const float4*>(a.A_log + d * N + k));
-    A2[k] = al.x; A2[k + 1] = al.y; A2[k + 2] = al.z; A2[k + 3] = al.w;
-  }
-  load_row<N>(static_cast<const IO*>(a.B) + b * N, Bv);
-  load_row<N>(static_cast<const IO*>(a.C) + b * N, Cv);
-  const IO* cs_in = static_cast<const IO*>(a.cs_in) + ch * 3;
-  const float s0 = IOT<IO>::to_f(cs_in[0]);
-  const float s1 = IOT<IO>::to_f(cs_in[1]);
-  const float s2 = IOT<IO>::to_f(cs_in[2]);
-  const float xt = IOT<IO>::ld(static_cast<const IO*>(a.xp) + ch);
-  const float zt = IOT<IO>::ld(static_cast<const IO*>(a.z) + ch);
-  const float dtr = IOT<IO>::ld(static_cast<const IO*>(a.dt) + ch);
-  const float4 w = __ldg(reinterpret_cast<const float4*>(a.conv_w + d * 4));
-  const float cb = a.conv_b ? __ldg(a.conv_b + d) : 0.0f;
-  const float dtb = __ldg(a.dt_bias + d);
-  const float Dd = __ldg(a.D + d);
-
-  const float pre = cb + w.x * s0 + w.y * s1 + w.z * s2 + w.w * xt;
-  const float u = M::silu(pre);
-  const float delta = M::softplus(dtr + dtb);
-  const float du = delta * u;
-  float acc = 0.0f;
-#pragma unroll
-  for (int n = 0; n < N; ++n) {
-    const float Ak = M::neg_exp(A2[n]) * M::a_scale();
-    h[n] = M::decay(delta, Ak) * h[n] + du * Bv[n];
-    acc += Cv[n] * h[n];
-  }
-  float* ho = a.h_out + ch * N;
-#pragma unroll
-  for (int k = 0; k < N; k += 4)
-    __stcs(reinterpret_cast<float4*>(ho + k), make_float4(h[k], h[k + 1], h[k + 2], h[k + 3]));
-  const float out = (acc + Dd * u) * M::silu(zt);
-  static_cast<IO*>(a.y)[ch] = IOT<IO>::from_f(out);
-  IO* cso = static_cast<IO*>(a.cs_out) + ch * 3;
-  cso[0] = IOT<IO>::from_f(s1);
-  cso[1] = IOT<IO>::from_f(s2);
-  cso[2] = IOT<IO>::from_f(xt);
 }
 
 }  // namespace mm
