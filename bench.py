@@ -64,6 +64,53 @@ def workload_bytes(w: I.Workload) -> dict:
     return {"fwd": fwd_bytes(w), "step": step_bytes(w.with_(seqlen=1))}
 
 
+# ----------------------------------------------------------------------------- rooflines
+SMS = 148
+MUFU_PER_CLK_SM = 16      # special-function (ex2/lg2/rcp) lane-ops per clock per SM
+FMA_PER_CLK_SM = 128      # fp32 FMA-pipe lane-ops per clock per SM
+POLY_EXP_FMA_OPS = 9      # FMA-pipe ops for one exp done by polynomial instead of MUFU
+
+
+def alu_elements_per_clk_sm(N: int) -> float:
+    """Upper bound on scan elements (t, d, n) per clock per SM from the arithmetic alone.
+
+    Per element the method needs T = 1 + 4/N transcendentals (exp(Delta*A) per state, and
+    per (t, d) the exps of the two SiLUs and the exp + log of softplus) and F = 4 + 20/N
+    fp32 ops (Delta*A, Delta*u*B, the h FMA, the C.h FMA; per (t, d) about 20 for the conv,
+    gate and the arithmetic around the transcendentals).  Transcendentals go to MUFU (16 per
+    clock per SM) or, as a degree-5 polynomial, to the FMA pipe (9 ops each).  With MUFU
+    saturated and the rest of the transcendentals on the FMA pipe:
+        F*x + 9*(T*x - 16) = 128   ->   x = (128 + 9*16) / (F + 9*T).
+    """
+    T = 1.0 + 4.0 / N
+    F = 4.0 + 20.0 / N
+    x = (FMA_PER_CLK_SM + POLY_EXP_FMA_OPS * MUFU_PER_CLK_SM) / (F + POLY_EXP_FMA_OPS * T)
+    if T * x < MUFU_PER_CLK_SM:          # MUFU alone suffices; the FMA pipe binds
+        x = FMA_PER_CLK_SM / F
+    return x
+
+
+def alu_floor_s(elements: int, N: int, sm_hz: float) -> float:
+    return elements / (alu_elements_per_clk_sm(N) * SMS * sm_hz)
+
+
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The largest x over all ranks (the job's time is its slowest rank's time)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_rank_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank moves bytes_per_rank_step per step (weak scaling);
+    the job takes as long as its slowest rank."""
+    return world * bytes_per_rank_step * steps / (max_ms * 1e-3) / 1e9
+
+
 # ----------------------------------------------------------------------------- misc
 def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -82,10 +129,11 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per forward launch from the committed ncu summary, if it was taken on
-    the current kernel sources; else None."""
-    p = os.path.join(ROOT, "profiles", f"fwd_{workload}_traffic.txt")
+def recorded_traffic(kind: str, workload: str):
+    """DRAM bytes (read + write) per call of the dominant entry point, from the committed
+    ncu summary profiles/<kind>_<workload>_traffic.txt, if those counters were taken on the
+    current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", f"{kind}_{workload}_traffic.txt")
     if not os.path.exists(p):
         return None
     kv = {}
@@ -96,7 +144,7 @@ def recorded_traffic(workload: str):
     if kv.get("kernel_source_sha") != kernel_source_hash():
         return None
     try:
-        return int(float(kv["dram_bytes_per_fwd_call"]))
+        return int(float(kv["dram_bytes_per_call"]))
     except (KeyError, ValueError):
         return None
 
@@ -245,11 +293,8 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
     step_ms = [e[0].elapsed_time(e[2]) for e in evs]
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    total_ms = sum(step_ms)
+    total_ms = max_over_ranks(sum(step_ms), dist if world > 1 else None, dev)
     if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
 
     # end to end through the public API: pinned host inputs -> device -> mixer -> host
@@ -293,11 +338,8 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
             if i >= 2:
                 ev1[i - 2].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = sum(a.elapsed_time(b) for a, b in zip(ev0, ev1))
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(ev0, ev1)),
+                                dist if world > 1 else None, dev)
         e2e = {"ms_per_step": e2e_ms / e2e_steps, "h2d": h2d, "d2h": d2h}
 
     bytes_ = workload_bytes(w)
@@ -305,7 +347,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
     if rank != 0:
         return None
     peaks = measured_peaks()
-    value = world * step_total * args.steps / (total_ms * 1e-3) / 1e9
+    value = job_gbs(step_total, args.steps, world, total_ms)
     # dominant kernel: the forward call (the decode step when timing decode alone)
     if w.decode:
         dom_ms = statistics.mean(dec_ms)
@@ -317,8 +359,30 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
         dom = "mamba_mixer_fwd"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     clocks = clk.summary()
-    e2e_val = world * step_total / (e2e["ms_per_step"] * 1e-3) / 1e9
-    traffic = recorded_traffic(w.name) if not w.decode else None
+    sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
+    # the binding roofline of the dominant kernel: HBM bytes or ALU arithmetic
+    t_hbm = dom_bytes / (peaks["hbm_gbs"] * 1e9)
+    dom_elems = w.batch * (1 if w.decode else w.seqlen) * w.d_inner * w.d_state
+    t_alu = alu_floor_s(dom_elems, w.d_state, sm_hz)
+    if t_alu > t_hbm:
+        roof = {"kernel": dom, "bound": "alu", "achieved": round(achieved, 2),
+                "peak": round(dom_bytes / t_alu / 1e9, 2), "unit": "GB/s",
+                "frac": round(t_alu / (dom_ms * 1e-3), 4),
+                "peak_source": (f"arithmetic floor: {alu_elements_per_clk_sm(w.d_state):.2f} scan "
+                                f"elements/clk/SM (MUFU 16 + FMA 128 per clk per SM) x {SMS} SMs x "
+                                f"{sm_hz/1e6:.0f} MHz, as GB/s of the kernel's algorithmic bytes"),
+                "hbm_frac": round(achieved / peaks["hbm_gbs"], 4),
+                "hbm_peak": peaks["hbm_gbs"], "hbm_peak_source": peaks["source"]}
+    else:
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 2),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
+                                else "fallback 6650 GB/s")}
+    roof["traffic"] = recorded_traffic("step" if w.decode else "fwd", w.name)
+    roof["algorithmic_bytes_per_launch"] = dom_bytes
+    roof["avg_launch_ms"] = round(dom_ms, 5)
+    e2e_val = job_gbs(step_total, 1, world, e2e["ms_per_step"])
     return {
         "metric": METRIC,
         "value": round(value, 2),
@@ -346,18 +410,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
                                         / (total_ms * 1e-3), 1),
         "fwd_ms_mean": round(statistics.mean(fwd_ms), 5) if not w.decode else None,
         "decode_ms_mean": round(statistics.mean(dec_ms), 5),
-        "roofline": {
-            "kernel": dom,
-            "bound": "hbm",
-            "achieved": round(achieved, 2),
-            "peak": peaks["hbm_gbs"],
-            "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured" else "fallback",
-            "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic,
-            "algorithmic_bytes_per_launch": dom_bytes,
-            "avg_launch_ms": round(dom_ms, 5),
-        },
+        "roofline": roof,
         "e2e": {"value": round(e2e_val, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                 "ms_per_step": round(e2e["ms_per_step"], 4)},
@@ -429,6 +482,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="m130", choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=None,
+                    help="override the workload's sequence length (smaller profiling captures)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -437,6 +492,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = I.WORKLOADS[args.workload]
+    if args.seqlen is not None and not w.decode:
+        w = w.with_(seqlen=args.seqlen, name=f"{w.name}_L{args.seqlen}")
 
     if args.impl == "reference":
         res = run_reference(args, w, rank)
