@@ -277,14 +277,16 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
           const float xt = lds_io<IO>(st + S::kXOff + swz<kRow>(t + 4, col));
           const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
           xa = xb; xb = xc; xc = xt;
-          const float u = M::silu(pre);
+          const float u = kPrecise ? M::silu(pre) : silu_fma(pre);
           const bool valid = tt + t < t_end;
-          const float dl = M::softplus(lds_io<IO>(st + S::kDtOff + swz<kRow>(t, col)) + dtb);
+          const float dtv = lds_io<IO>(st + S::kDtOff + swz<kRow>(t, col)) + dtb;
+          const float dl = kPrecise ? M::softplus(dtv) : softplus_fma(dtv);
           dv[i] = valid ? dl : 0.0f;
           duv[i] = valid ? dl * u : 0.0f;
           if constexpr (!kPrepass) {
             skv[i] = Dd * u;
-            szv[i] = M::silu(lds_io<IO>(st + S::kZOff + swz<kRow>(t, col)));
+            const float zv = lds_io<IO>(st + S::kZOff + swz<kRow>(t, col));
+            szv[i] = kPrecise ? M::silu(zv) : silu_fma(zv);
           }
         }
         const uint32_t rec = pr + S::kScOff;
