@@ -1,6 +1,6 @@
 /*
  * Body of the CPU oracle, written once and compiled for two arithmetic types.
- * mixer_oracle.c includes this file with REAL = double (the judge of parity) and
+ * mixer_oracle.c includes this file with REAL = double (the reference for parity) and
  * REAL = float (used only to show that a plain fp32 recurrence lies inside the fp32
  * tolerance band).  ORACLE_FN(name) appends the precision suffix; REXP, RLOG1P, RFABS
  * and RFMAX are the libm functions of that type.

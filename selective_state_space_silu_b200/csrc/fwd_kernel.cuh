@@ -58,6 +58,9 @@ struct FwdParams {
   int64_t L, Di;
   int64_t chunk_len;    // multiple of kTileT
   int nchunks;
+  // Failure injection for tests (-1 = off): block (0, 0, 0) arms tile `inject_skip_tile`'s
+  // barrier but issues none of its copies, so the waits on it run out.
+  int inject_skip_tile;
 };
 
 constexpr int kCh = 32;          // channels per CTA
@@ -219,11 +222,13 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     int issued = 0;
     auto issue = [&](int k) {
       const int s = k % kStages;
-      if (lane == 0) {
+      const bool skip = k == p.inject_skip_tile && blockIdx.x == 0 && blockIdx.y == 0 &&
+                        blockIdx.z == 0;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], kTxBytes);
+      if (lane == 0 && !skip) {
         const uint32_t st = sb + uint32_t(s * S::kRawStage);
         const int tt = int(t_begin) + k * kTileT;
         constexpr uint32_t kSwzAlign = 1024, kPlainAlign = 128;
-        mbar_arrive_expect_tx(&full[s], kTxBytes);
         tma_load_3d(st + S::kXOff, &tm_x, &full[s], d0, tt - kHalo, b, kSwzAlign, kEs, p.status);
         tma_load_3d(st + S::kDtOff, &tm_dt, &full[s], d0, tt, b, kSwzAlign, kEs, p.status);
         tma_load_3d(st + S::kBOff, &tm_B, &full[s], 0, tt, b, kPlainAlign, kEs, p.status);

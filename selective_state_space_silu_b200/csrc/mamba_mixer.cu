@@ -8,6 +8,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -314,6 +315,10 @@ int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const
   a.status = static_cast<int*>(workspace);
   a.L = dims->seqlen; a.Di = Di;
   a.nchunks = plan.nchunks; a.chunk_len = plan.chunk_len;
+  // Test-only failure injection (bounded-wait path): MAMBA_MIXER_INJECT_SKIP_TILE=k makes one
+  // CTA skip the copies of its tile k; unset (the default) injects nothing.
+  a.inject_skip_tile = -1;
+  if (const char* inj = getenv("MAMBA_MIXER_INJECT_SKIP_TILE")) a.inject_skip_tile = atoi(inj);
   if (plan.nchunks > 1) {
     const size_t agg = (need - kWsHeader) / sizeof(float) / 2;
     a.ws_P = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + kWsHeader);
