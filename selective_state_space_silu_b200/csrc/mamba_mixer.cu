@@ -212,7 +212,8 @@ cudaError_t launch_fwd(const FwdMaps& m, const mm::FwdParams& a, int64_t batch, 
 template <int N, typename IO, bool P>
 cudaError_t launch_step(const mm::StepArgs& a, cudaStream_t st) {
   const int64_t bx = (a.Di * mm::kStepLanes + mm::kStepThreads - 1) / mm::kStepThreads;
-  mm::step_kernel<N, IO, P><<<dim3(unsigned(bx), unsigned(a.batch)), mm::kStepThreads, 0, st>>>(a);
+  mm::step_kernel<N, IO, P, mm::kStepLanes><<<dim3(unsigned(bx), unsigned(a.batch)),
+                                             mm::kStepThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 

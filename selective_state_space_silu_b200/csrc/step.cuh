@@ -36,18 +36,28 @@ struct StepArgs {
 };
 
 constexpr int kStepThreads = 256;
-constexpr int kStepLanes = 4;
-static_assert(kStepLanes == 4, "the index math below assumes 4 lanes per channel");
+#ifndef MM_STEP_LANES
+#define MM_STEP_LANES 4
+#endif
+constexpr int kStepLanes = MM_STEP_LANES;   // lanes per channel
 
 // Streaming (evict-first) 16/8-byte accesses for the state, which is touched once.
 __device__ __forceinline__ float4 ldcs4(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
 __device__ __forceinline__ float2 ldcs2(const float* p) { return __ldcs(reinterpret_cast<const float2*>(p)); }
 
-// kS consecutive I/O elements (8 or 4 bytes for bf16, 16 or 8 for fp32) as fp32.
+// kS consecutive I/O elements (kS = 8, 4 or 2) as fp32 through vector loads.
 template <int kS, typename IO>
 __device__ __forceinline__ void ld_small(const IO* p, float* out) {
   if constexpr (sizeof(IO) == 2) {
-    if constexpr (kS == 4) {
+    if constexpr (kS == 8) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+      const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        out[2 * k] = __uint_as_float(wv[k] << 16);
+        out[2 * k + 1] = __uint_as_float(wv[k] & 0xffff0000u);
+      }
+    } else if constexpr (kS == 4) {
       const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
       out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
       out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
@@ -56,7 +66,12 @@ __device__ __forceinline__ void ld_small(const IO* p, float* out) {
       out[0] = __uint_as_float(v << 16); out[1] = __uint_as_float(v & 0xffff0000u);
     }
   } else {
-    if constexpr (kS == 4) {
+    if constexpr (kS == 8) {
+      const float4 v0 = __ldg(reinterpret_cast<const float4*>(p));
+      const float4 v1 = __ldg(reinterpret_cast<const float4*>(p + 4));
+      out[0] = v0.x; out[1] = v0.y; out[2] = v0.z; out[3] = v0.w;
+      out[4] = v1.x; out[5] = v1.y; out[6] = v1.z; out[7] = v1.w;
+    } else if constexpr (kS == 4) {
       const float4 v = __ldg(reinterpret_cast<const float4*>(p));
       out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
     } else {
@@ -66,34 +81,44 @@ __device__ __forceinline__ void ld_small(const IO* p, float* out) {
   }
 }
 
-template <int N, typename IO, bool kPrecise>
+// kS consecutive fp32 values (kS multiple of 2) through 16- or 8-byte loads.
+template <int kS, bool kStream>
+__device__ __forceinline__ void ld_f32s(const float* p, float* out) {
+#pragma unroll
+  for (int i = 0; i < kS; i += 4) {
+    if constexpr (kS - 0 >= 4) {
+      const float4 v = kStream ? __ldcs(reinterpret_cast<const float4*>(p + i))
+                               : __ldg(reinterpret_cast<const float4*>(p + i));
+      out[i] = v.x; out[i + 1] = v.y; out[i + 2] = v.z; out[i + 3] = v.w;
+    } else {
+      const float2 v = kStream ? __ldcs(reinterpret_cast<const float2*>(p + i))
+                               : __ldg(reinterpret_cast<const float2*>(p + i));
+      out[i] = v.x; out[i + 1] = v.y;
+    }
+  }
+}
+
+template <int N, typename IO, bool kPrecise, int kLanes>
 __global__ void __launch_bounds__(kStepThreads)
 step_kernel(StepArgs a) {
   using M = Math<kPrecise>;
-  constexpr int S = N / kStepLanes;  // states per lane
-  // grid: (ceil(4*Di / kStepThreads), batch); no integer division on the device
+  constexpr int S = N / kLanes;  // states per lane
+  static_assert(kLanes == 2 || kLanes == 4, "2 or 4 lanes per channel");
+  // grid: (ceil(kLanes*Di / kStepThreads), batch); no integer division on the device
   const int t = blockIdx.x * kStepThreads + threadIdx.x;
   const int64_t b = blockIdx.y;
-  const int64_t d = t >> 2;                // kStepLanes == 4
-  const int j = t & 3;
-  // 4*Di is a multiple of 32 (Di % 8 == 0): a warp is all in range or all out.
+  const int64_t d = t / kLanes;            // power of two: a shift
+  const int j = t % kLanes;
+  // kLanes*Di is a multiple of 16 (Di % 8 == 0) and of 32 for 4 lanes; for 2 lanes the
+  // half-warp tails of a partial warp are still whole channels, and the shuffles below
+  // only pair lanes of the same channel.
   if (d >= a.Di) return;
   const int64_t ch = b * a.Di + d;         // flat (b, d)
 
   // --- loads: the state first (the bulk of the bytes), then the rest
   float h[S], A2[S], Bv[S], Cv[S];
-  const float* hp = a.h_in + ch * N + j * S;
-  if constexpr (S == 4) {
-    const float4 v = ldcs4(hp);
-    h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
-    const float4 al = __ldg(reinterpret_cast<const float4*>(a.A_log + d * N + j * S));
-    A2[0] = al.x; A2[1] = al.y; A2[2] = al.z; A2[3] = al.w;
-  } else {
-    const float2 v = ldcs2(hp);
-    h[0] = v.x; h[1] = v.y;
-    const float2 al = __ldg(reinterpret_cast<const float2*>(a.A_log + d * N + j * S));
-    A2[0] = al.x; A2[1] = al.y;
-  }
+  ld_f32s<S, true>(a.h_in + ch * N + j * S, h);
+  ld_f32s<S, false>(a.A_log + d * N + j * S, A2);
   ld_small<S>(static_cast<const IO*>(a.B) + b * N + j * S, Bv);
   ld_small<S>(static_cast<const IO*>(a.C) + b * N + j * S, Cv);
   const IO* cs_in = static_cast<const IO*>(a.cs_in) + ch * 3;
@@ -108,7 +133,7 @@ step_kernel(StepArgs a) {
   const float dtb = __ldg(a.dt_bias + d);
   const float Dd = __ldg(a.D + d);
 
-  // --- conv + SiLU, softplus (same on the four lanes)
+  // --- conv + SiLU, softplus (same on the lanes of the channel)
   const float pre = cb + w.x * s0 + w.y * s1 + w.z * s2 + w.w * xt;
   const float u = M::silu(pre);
   const float delta = M::softplus(dtr + dtb);
@@ -122,15 +147,19 @@ step_kernel(StepArgs a) {
     h[s] = M::decay(delta, Ak) * h[s] + du * Bv[s];
     part += Cv[s] * h[s];
   }
-  part += __shfl_xor_sync(0xffffffffu, part, 1);
-  part += __shfl_xor_sync(0xffffffffu, part, 2);
+  const unsigned mask = __activemask();
+  part += __shfl_xor_sync(mask, part, 1);
+  if constexpr (kLanes == 4) part += __shfl_xor_sync(mask, part, 2);
 
   // --- stores
   float* ho = a.h_out + ch * N + j * S;
-  if constexpr (S == 4) {
-    __stcs(reinterpret_cast<float4*>(ho), make_float4(h[0], h[1], h[2], h[3]));
-  } else {
-    __stcs(reinterpret_cast<float2*>(ho), make_float2(h[0], h[1]));
+#pragma unroll
+  for (int i = 0; i < S; i += 4) {
+    if constexpr (S >= 4) {
+      __stcs(reinterpret_cast<float4*>(ho + i), make_float4(h[i], h[i + 1], h[i + 2], h[i + 3]));
+    } else {
+      __stcs(reinterpret_cast<float2*>(ho + i), make_float2(h[i], h[i + 1]));
+    }
   }
   if (j == 0) {
     const float out = (part + Dd * u) * M::silu(zt);

@@ -336,3 +336,22 @@ def test_tolerance_rule_counts_nan_as_mismatch():
     assert within(np.array([np.nan]), np.array([np.nan]), "f32")[0]
     assert within(np.array([1.0 + 9e-4]), np.array([1.0]), "f32")[0]
     assert not within(np.array([1.0 + 1.2e-3]), np.array([1.0]), "f32")[0]
+
+
+# ---------------------------------------------------------------- regression fixture
+def test_oracle_matches_its_golden_fixture(oracle):
+    """tests/golden/tiny_oracle_samples.json (written by tests/golden/make_golden.py from
+    the oracle): any later change to the oracle's arithmetic shows up here."""
+    import json
+    import os
+    from selective_state_space_silu_b200 import inputs as I
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                    "tiny_oracle_samples.json")))
+    d = I.make_inputs(I.WORKLOADS["tiny"])
+    y, h, cs = oracle.mixer(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                            d["conv_w"], d["conv_b"], d["dt_bias"])
+    for ix, v in g["y"]:
+        assert y[tuple(ix)] == v
+    for ix, v in g["h_out"]:
+        assert h[tuple(ix)] == v
+    assert list(cs[1, 127]) == g["conv_state_out_b1_d127"]
