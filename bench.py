@@ -7,7 +7,9 @@
 One step = one pass of the whole hot path over one batch: the fused forward
 (conv+SiLU, softplus, selective scan with the chunk carry, gate, state out) over the
 workload's prompt, then one decode step per sequence on the state the forward left
-(in place).  ``--workload decode`` times the decode step alone on its own shapes.
+(in place).  The default workload is the long-sequence one (batch 2, L 65536, d_inner
+2560): the only one whose forward also runs the carry between time chunks, so its step
+covers every stage of the path.  ``--workload decode`` times the decode step alone.
 
 Prints ONE JSON line (rank 0).  ``value`` is achieved algorithmic HBM GB/s over all
 ranks: algorithmic bytes (each input read once, each output written once) divided by
@@ -19,7 +21,6 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import glob
 import json
 import os
 import statistics
@@ -121,11 +122,18 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+KERNEL_SOURCES = {
+    "fwd": ("fwd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh", "mamba_mixer.cu"),
+    "step": ("step.cuh", "device_math.cuh", "mamba_mixer.cu"),
+}
+
+
+def kernel_source_hash(kind: str) -> str:
+    """Hash of the sources that define one entry point's kernels and their launch."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "selective_state_space_silu_b200", "csrc", "*"))):
-        with open(f, "rb") as fh:
-            h.update(os.path.basename(f).encode() + b"\0" + fh.read())
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "selective_state_space_silu_b200", "csrc", name), "rb") as fh:
+            h.update(name.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -141,7 +149,7 @@ def recorded_traffic(kind: str, workload: str):
         if ":" in line:
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("kernel_source_sha") != kernel_source_hash():
+    if kv.get("kernel_source_sha") != kernel_source_hash(kind):
         return None
     try:
         return int(float(kv["dram_bytes_per_call"]))
@@ -477,10 +485,11 @@ def run_reference(args, w: I.Workload, rank: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 100 for long, 2000 otherwise)")
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="m130", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="long", choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="override the workload's sequence length (smaller profiling captures)")
@@ -492,6 +501,8 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     w = I.WORKLOADS[args.workload]
+    if args.steps is None:
+        args.steps = 100 if args.workload == "long" else 2000
     if args.seqlen is not None and not w.decode:
         w = w.with_(seqlen=args.seqlen, name=f"{w.name}_L{args.seqlen}")
 

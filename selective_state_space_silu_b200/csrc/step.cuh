@@ -37,7 +37,7 @@ struct StepArgs {
 
 constexpr int kStepThreads = 256;
 #ifndef MM_STEP_LANES
-#define MM_STEP_LANES 4
+#define MM_STEP_LANES 2
 #endif
 constexpr int kStepLanes = MM_STEP_LANES;   // lanes per channel
 
