@@ -90,9 +90,8 @@ struct FwdSmem {
   static constexpr int kBOff = kDtOff + align1k(kZBytes);
   static constexpr int kCOff = kBOff + align1k(kBBytes);
   static constexpr int kRawStage = kCOff + align1k(kBBytes);
-  // prepared tile: B/C records [t][j]{B[kS], C[kS]} in the I/O type (fp32 or bf16),
-  // then the scalar records [q][c]
-  static constexpr int kBCRec = 2 * (N / 4) * int(sizeof(IO));   // 16 or 32 (N=16), 8/16 (N=8)
+  // prepared tile: fp32 B/C records [t][j]{B[kS], C[kS]}, then the scalar records [q][c]
+  static constexpr int kBCRec = 2 * (N / 4) * 4;                // fp32: 32 (N=16), 16 (N=8)
   static constexpr int kBCfBytes = kTileT * 4 * kBCRec;
   static constexpr int kScOff = align1k(kBCfBytes);
   static constexpr int kPrepBytes = kScOff + kQuads * kCh * kScRec;
@@ -126,33 +125,49 @@ __device__ __forceinline__ float lds_io<__nv_bfloat16>(uint32_t a) {
   return __uint_as_float(lds_u16(a) << 16);
 }
 
-// Copies kHalf bytes of B and kHalf bytes of C into one B/C record.
-template <int kHalf>
-__device__ __forceinline__ void copy_record(uint32_t dst, uint32_t b, uint32_t c, bool b_only) {
-  if constexpr (kHalf == 8) {
-    uint32_t b0, b1, c0 = 0, c1 = 0;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(b));
-    if (!b_only) asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(c0), "=r"(c1) : "r"(c));
-    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(b0), "r"(b1), "r"(c0),
-                 "r"(c1) : "memory");
-  } else if constexpr (kHalf == 4) {
-    uint32_t b0, c0 = 0;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(b0) : "r"(b));
-    if (!b_only) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(c0) : "r"(c));
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(b0), "r"(c0) : "memory");
-  } else {  // 16 bytes each (fp32, 4 states)
-    const float4 bv = lds_f32x4(b);
-    const float4 cv = b_only ? make_float4(0.f, 0.f, 0.f, 0.f) : lds_f32x4(c);
-    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "f"(bv.x), "f"(bv.y),
-                 "f"(bv.z), "f"(bv.w) : "memory");
-    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 16), "f"(cv.x), "f"(cv.y),
-                 "f"(cv.z), "f"(cv.w) : "memory");
-  }
-}
+__device__ __forceinline__ void sts_f32x4(uint32_t a, float x, float y, float z, float w);
 
 // The two bf16 halves of a 32-bit word as fp32 (exact).
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// B[kS] and C[kS] (I/O type) of one (t, j) into one fp32 record {B[kS], C[kS]} (C left 0
+// when b_only).  Widening here, once per CTA, spares the scan lanes of all 32 channels the
+// conversion.
+template <typename IO, int kS>
+__device__ __forceinline__ void widen_record(uint32_t dst, uint32_t b, uint32_t c, bool b_only) {
+  static_assert(kS == 2 || kS == 4, "2 or 4 states per lane");
+  float v[2 * kS];
+  if constexpr (sizeof(IO) == 4) {
+    if constexpr (kS == 4) {
+      const float4 bv = lds_f32x4(b);
+      const float4 cv = b_only ? make_float4(0.f, 0.f, 0.f, 0.f) : lds_f32x4(c);
+      v[0] = bv.x; v[1] = bv.y; v[2] = bv.z; v[3] = bv.w;
+      v[4] = cv.x; v[5] = cv.y; v[6] = cv.z; v[7] = cv.w;
+    } else {
+      v[0] = lds_f32(b); v[1] = lds_f32(b + 4);
+      v[2] = b_only ? 0.0f : lds_f32(c); v[3] = b_only ? 0.0f : lds_f32(c + 4);
+    }
+  } else {
+    uint32_t w[kS];   // kS/2 words of B, then kS/2 words of C
+    if constexpr (kS == 4) {
+      asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(b));
+      w[2] = w[3] = 0;
+      if (!b_only) asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[2]), "=r"(w[3]) : "r"(c));
+    } else {
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[0]) : "r"(b));
+      w[1] = 0;
+      if (!b_only) asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w[1]) : "r"(c));
+    }
+#pragma unroll
+    for (int i = 0; i < kS; ++i) {
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 2 * kS; i += 4) sts_f32x4(dst + 4 * i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+}
 
 __device__ __forceinline__ void sts_f32x4(uint32_t a, float x, float y, float z, float w) {
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(x), "f"(y), "f"(z),
@@ -258,12 +273,11 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       // B and C re-laid out for this warp's steps as [t][j]{B[kS], C[kS]} (no conversion):
       // lane (t, j) copies B[t][j*kS ..] and C[t][j*kS ..] into one record
       {
-        constexpr int kHalf = S::kBCRec / 2;            // bytes of B (or C) per record
         for (int idx = lane; idx < kPrepSteps * 4; idx += 32) {
           const int t = kPrepSteps * w + idx / 4, jj = idx % 4;
-          const uint32_t src = uint32_t(t * N * kEs + jj * kHalf);
+          const uint32_t src = uint32_t(t * N * kEs + jj * kS * kEs);
           const uint32_t dst = pr + uint32_t((t * 4 + jj) * S::kBCRec);
-          copy_record<kHalf>(dst, st + S::kBOff + src, st + S::kCOff + src, kPrepass);
+          widen_record<IO, kS>(dst, st + S::kBOff + src, st + S::kCOff + src, kPrepass);
         }
       }
 
@@ -393,16 +407,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
           const uint32_t row = bcf + uint32_t((4 * q + i) * 4 * S::kBCRec);
           const f32x2 d2 = pk2(di[i], di[i]), du2 = pk2(dui[i], dui[i]);
           f32x2 Bp[kS / 2], Cp[kS / 2];
-          if constexpr (kS == 4) {   // bf16 record {B0..B3, C0..C3}
-            uint32_t w0, w1, w2, w3;
-            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3) : "r"(row));
-            Bp[0] = pk2(bf16_lo(w0), bf16_hi(w0)); Bp[1] = pk2(bf16_lo(w1), bf16_hi(w1));
-            Cp[0] = pk2(bf16_lo(w2), bf16_hi(w2)); Cp[1] = pk2(bf16_lo(w3), bf16_hi(w3));
-          } else {                   // bf16 record {B0, B1, C0, C1}
-            uint32_t w0, w1;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(row));
-            Bp[0] = pk2(bf16_lo(w0), bf16_hi(w0)); Cp[0] = pk2(bf16_lo(w1), bf16_hi(w1));
+          if constexpr (kS == 4) {   // fp32 record {B0..B3, C0..C3}
+            const float4 bv = lds_f32x4(row);
+            Bp[0] = pk2(bv.x, bv.y); Bp[1] = pk2(bv.z, bv.w);
+            if constexpr (!kPrepass) {
+              const float4 cv = lds_f32x4(row + 16);
+              Cp[0] = pk2(cv.x, cv.y); Cp[1] = pk2(cv.z, cv.w);
+            } else {
+              Cp[0] = Cp[1] = pk2(0.0f, 0.0f);
+            }
+          } else {                   // fp32 record {B0, B1, C0, C1}
+            const float4 v = lds_f32x4(row);
+            Bp[0] = pk2(v.x, v.y); Cp[0] = pk2(v.z, v.w);
           }
           f32x2 acc2 = pk2(0.0f, 0.0f);
 #pragma unroll

@@ -107,13 +107,15 @@ int check_ptr(const void* p, const char* name, bool required, size_t align) {
 
 // ---- time-chunk plan ---------------------------------------------------------------
 // A CTA covers one batch row and 32 channels.  When there are too few such tiles to give
-// every SM two resident CTAs (three fit: 66 KiB of shared memory each), the sequence is
+// every SM two resident CTAs (three fit: 68 KiB of shared memory each), the sequence is
 // cut into time chunks (multiples of the tile length, at least 256 steps) that run in
 // parallel with a carried state between them.  Every chunk past the first also costs a
-// chunk-state pass over the chunk before it, yet measured on a 2 x 65536 x 2560 forward
-// the finer split wins up to about eight chunk-CTAs per SM (2, 3, 4, 7 chunks: 5.05,
-// 4.74, 4.39, 4.04 ms), because the scan warps are latency-bound at low occupancy.
-constexpr int kResidentCtas = 148 * 8;
+// chunk-state pass over the chunk before it, yet the finer split keeps winning up to about
+// thirteen chunk-CTAs per SM, because a lone CTA is latency-bound (about 100 clocks per
+// step alone on an SM, 200 with three resident).  Measured on a 2 x 65536 x 2560 forward
+// (160 tiles): 1, 2, 3, 4, 5, 7, 9, 12, 16, 24, 48 chunks take 4.69, 4.95, 4.65, 4.31,
+// 4.11, 3.96, 3.86, 3.77, 3.92, 3.80, 3.86 ms.
+constexpr int kChunkCtas = 148 * 13;
 constexpr size_t kWsHeader = 256;  // status word + padding
 
 struct Plan {
@@ -125,7 +127,7 @@ Plan make_plan(const mamba_dims* d) {
   Plan p{1, d->seqlen > 0 ? d->seqlen : 1};
   const int64_t tiles = d->batch * ((d->d_inner + mm::kCh - 1) / mm::kCh);
   if (tiles <= 0 || d->seqlen < 512 || tiles >= 2 * 148) return p;
-  int64_t c = kResidentCtas / tiles;
+  int64_t c = kChunkCtas / tiles;
   if (c < 2) c = 2;
   const int64_t cmax = d->seqlen / 256;
   if (c > cmax) c = cmax;
