@@ -31,9 +31,15 @@
  *     the same number without overflow;  SiLU(v) = v / (1 + exp(-v));
  *   - the new conv state is the last K-1 entries of xpad (zeros included if L < K-1).
  *
+ * Packed documents (niverel-mamba 0.1.0, section "seq_idx strict reset"): with an int32
+ * seq_idx [batch, L], wherever seq_idx[b, t] != seq_idx[b, t-1] both the conv state and
+ * the SSM state reset to zero before step t, so a packed row equals its documents run
+ * one by one and concatenated.  The initial state (h_in, conv_state_in), if given,
+ * belongs to the row's first document; the states returned are the last document's.
+ *
  * Layouts (row-major): x', z, dt_raw, y [batch, L, d_inner]; B, C [batch, L, d_state];
  * A_log [d_inner, d_state]; D, conv_b, dt_bias [d_inner]; conv_w [d_inner, d_conv];
- * h [batch, d_inner, d_state]; conv_state [batch, d_inner, d_conv-1].
+ * h [batch, d_inner, d_state]; conv_state [batch, d_inner, d_conv-1]; seq_idx [batch, L].
  *
  * Build: gcc -O2 -fPIC -shared -fopenmp -ffp-contract=off (no fast-math), so every
  * operation is the one written.  Channels (b, d) are independent and may run on

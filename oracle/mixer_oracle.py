@@ -50,7 +50,7 @@ def _load():
         for name in ("oracle_mixer_f64", "oracle_mixer_f32"):
             fn = getattr(lib, name)
             fn.restype = ci
-            fn.argtypes = [i64] * 5 + [vp] * 15 + [ci]
+            fn.argtypes = [i64] * 5 + [vp] * 16 + [ci]
         lib.oracle_max_threads.restype = ci
         lib.oracle_max_threads.argtypes = []
         _lib = lib
@@ -73,12 +73,13 @@ def _ptr(a):
 
 def mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
           h_in=None, conv_state_in=None, precision: str = "f64",
-          nthreads: int = 1) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+          nthreads: int = 1, seq_idx=None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Run the oracle.
 
     Arrays are numeric numpy arrays (already widened from bf16 where that applies) in
     the layouts of mixer_oracle.c.  ``conv_b``, ``h_in`` and ``conv_state_in`` may be
-    None (zero bias; zero initial state).  Returns (y [Bt,L,Di], h_out [Bt,Di,N],
+    None (zero bias; zero initial state).  ``seq_idx`` ([Bt, L] integers, optional) marks
+    packed documents: the conv and SSM states reset wherever it changes along t.  Returns (y [Bt,L,Di], h_out [Bt,Di,N],
     conv_state_out [Bt,Di,K-1]) in the requested precision ("f64" or "f32").
     """
     dt = {"f64": np.float64, "f32": np.float32}[precision]
@@ -88,6 +89,7 @@ def mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
     A_log, D, conv_w = _arr(A_log, dt), _arr(D, dt), _arr(conv_w, dt)
     conv_b, dt_bias = _arr(conv_b, dt), _arr(dt_bias, dt)
     h_in, conv_state_in = _arr(h_in, dt), _arr(conv_state_in, dt)
+    seq_idx = _arr(seq_idx, np.int32)
     Bt, L, Di = xp.shape
     N = A_log.shape[1]
     K = conv_w.shape[1]
@@ -97,11 +99,12 @@ def mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
     assert conv_b is None or conv_b.shape == (Di,)
     assert h_in is None or h_in.shape == (Bt, Di, N)
     assert conv_state_in is None or conv_state_in.shape == (Bt, Di, K - 1)
+    assert seq_idx is None or seq_idx.shape == (Bt, L)
     y = np.empty((Bt, L, Di), dtype=dt)
     h_out = np.empty((Bt, Di, N), dtype=dt)
     cs_out = np.empty((Bt, Di, K - 1), dtype=dt)
     rc = fn(Bt, L, Di, N, K, _ptr(xp), _ptr(z), _ptr(dt_raw), _ptr(B), _ptr(C), _ptr(A_log),
-            _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(h_in),
+            _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(seq_idx), _ptr(h_in),
             _ptr(conv_state_in), _ptr(y), _ptr(h_out), _ptr(cs_out), int(nthreads))
     if rc != 0:
         raise RuntimeError(f"oracle failed with code {rc}")
@@ -139,6 +142,9 @@ def mixer_channels(inp: dict, batch_idx, chan_idx, precision: str = "f64",
         h_in = h_in[bi][:, di]
     if cs_in is not None:
         cs_in = w(cs_in[bi][:, di])
+    seq = inp.get("seq_idx")
+    if seq is not None:
+        seq = seq[bi]
     return mixer(sub["xp"], sub["z"], sub["dt_raw"], sub["B"], sub["C"], sub["A_log"],
                  sub["D"], sub["conv_w"], sub["conv_b"], sub["dt_bias"], h_in, cs_in,
-                 precision=precision, nthreads=nthreads)
+                 precision=precision, nthreads=nthreads, seq_idx=seq)

@@ -20,7 +20,8 @@ int ORACLE_FN(oracle_mixer)(int64_t batch, int64_t seqlen, int64_t d_inner, int6
                             int64_t d_conv, const REAL* xp, const REAL* z, const REAL* dt_raw,
                             const REAL* Bm, const REAL* Cm, const REAL* A_log, const REAL* Dv,
                             const REAL* conv_w, const REAL* conv_b, const REAL* dt_bias,
-                            const REAL* h_in, const REAL* conv_state_in, REAL* y, REAL* h_out,
+                            const int32_t* seq_idx, const REAL* h_in, const REAL* conv_state_in,
+                            REAL* y, REAL* h_out,
                             REAL* conv_state_out, int nthreads) {
   if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state < 1 || d_conv < 1) return 1;
   const int64_t L = seqlen, Di = d_inner, N = d_state, K = d_conv;
@@ -51,6 +52,14 @@ int ORACLE_FN(oracle_mixer)(int64_t batch, int64_t seqlen, int64_t d_inner, int6
     }
 
     for (int64_t t = 0; t < L; ++t) {
+      /* document reset (niverel-mamba, section "seq_idx strict reset"): where seq_idx
+         changes between t-1 and t, the conv state (the K-1 inputs before t) and the SSM
+         state are zero before step t */
+      if (seq_idx && t > 0 && seq_idx[b * L + t] != seq_idx[b * L + t - 1]) {
+        for (int64_t k = 0; k < K - 1; ++k) xpad[t + k] = (REAL)0;
+        for (int64_t n = 0; n < N; ++n) h[n] = (REAL)0;
+      }
+
       /* step 2: causal depthwise conv, then SiLU */
       REAL acc = conv_b ? conv_b[d] : (REAL)0;
       for (int64_t k = 0; k < K; ++k) acc = acc + conv_w[d * K + k] * xpad[t + k];

@@ -163,3 +163,72 @@ def as_f32(a: np.ndarray) -> np.ndarray:
     if a.dtype == np.uint16:
         return bf16_bits_to_f32(a)
     return np.asarray(a, dtype=np.float32)
+
+
+# ---------------------------------------------------------------- packed documents
+# seq_idx patterns for rows that pack several documents (niverel-mamba 0.1.0, section
+# "seq_idx strict reset": the states reset wherever seq_idx changes).  The nine shapes
+# follow the structural cases that section lists; they are index patterns only.
+SEQ_IDX_CASES = ("start_of_row", "length_one_docs", "consecutive_boundaries", "boundary_on_edge",
+                 "doc_inside_chunk", "misaligned_rows", "terminal_padding", "nonzero_first_id",
+                 "many_short_docs")
+
+
+def _runs_to_ids(lengths, first_id: int = 0) -> np.ndarray:
+    return np.repeat(np.arange(first_id, first_id + len(lengths)), lengths).astype(np.int32)
+
+
+def _row(L: int, cuts, first_id: int = 0) -> np.ndarray:
+    """Ids for one row with documents starting at the given positions (besides 0)."""
+    cuts = sorted(c for c in set(cuts) if 0 < c < L)
+    bounds = [0] + cuts + [L]
+    return _runs_to_ids(np.diff(bounds), first_id)
+
+
+def seq_idx_case(name: str, batch: int, L: int, edge: int = 8, seed: int = 0) -> np.ndarray:
+    """One of SEQ_IDX_CASES as an int32 [batch, L] array.  ``edge`` is a block length of
+    the implementation (a tile or chunk length) for the boundary-on-edge case."""
+    r = np.random.default_rng(seed)
+    rows = []
+    for b in range(batch):
+        if name == "start_of_row":            # every row opens a new id; no other boundary
+            row = np.full(L, 100 + 7 * b, dtype=np.int32)
+        elif name == "length_one_docs":
+            row = _row(L, [1, 2, 3, L // 2, L // 2 + 1, L - 1], first_id=b)
+        elif name == "consecutive_boundaries":
+            m = L // 3 + b
+            row = _row(L, [m, m + 1, m + 2, m + 3])
+        elif name == "boundary_on_edge":
+            row = _row(L, [k * edge for k in range(1, L // edge + 1)][: 4 + b])
+        elif name == "doc_inside_chunk":
+            a = max(1, L // 2 - 3 + b)
+            row = _row(L, [a, a + 5])
+        elif name == "misaligned_rows":
+            row = _row(L, sorted(r.choice(np.arange(1, L), size=min(L - 1, 3 + b), replace=False)))
+        elif name == "terminal_padding":
+            pad = max(1, L // 5)
+            row = _row(L, [L // 3 + b, L - pad])
+            row[L - pad:] = -1
+        elif name == "nonzero_first_id":
+            row = _row(L, [L // 4 + b], first_id=42)
+        elif name == "many_short_docs":
+            lens = []
+            while sum(lens) < L:
+                lens.append(int(r.integers(1, 6)))
+            row = _runs_to_ids(lens)[:L]
+        else:
+            raise ValueError(name)
+        rows.append(row.astype(np.int32))
+    return np.stack(rows)
+
+
+def packed_seq_idx(batch: int, L: int, mean_len: int, seed: int) -> np.ndarray:
+    """Rows packing documents of geometric length (mean ``mean_len``), for timing."""
+    r = np.random.default_rng(seed)
+    out = np.empty((batch, L), dtype=np.int32)
+    for b in range(batch):
+        lens = []
+        while sum(lens) < L:
+            lens.append(int(r.geometric(1.0 / mean_len)))
+        out[b] = _runs_to_ids(lens)[:L]
+    return out
