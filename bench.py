@@ -48,7 +48,8 @@ def fwd_bytes(w: I.Workload) -> int:
             + 2 * Bt * L * N * s           # B, C
             + Di * (4 * N + 28)            # A_log, D, conv_w, conv_b, dt_bias
             + Bt * Di * N * 4              # h out
-            + Bt * Di * 3 * s)             # conv state out
+            + Bt * Di * 3 * s              # conv state out
+            + (4 * Bt * L if w.packed_mean else 0))   # seq_idx
 
 
 def step_bytes(w: I.Workload) -> int:
@@ -235,6 +236,8 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
 
     P = {k: td(inp[k]) for k in ("A_log", "D", "conv_w", "conv_b", "dt_bias")}
     X = {k: td(inp[k]) for k in ("xp", "z", "dt_raw", "B", "C")}
+    if w.packed_mean:
+        X["seq_idx"] = td(inp["seq_idx"])
     T = {k: td(tok[k]) for k in ("xp", "z", "dt_raw", "B", "C")}
     Bt, L, Di, N = w.batch, w.seqlen, w.d_inner, w.d_state
     iot = X["xp"].dtype
@@ -262,6 +265,12 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
         torch.sum(flush_rd, dim=0, out=flush_sink)
 
     def fwd():
+        if w.packed_mean:
+            M.mamba_mixer_fwd_packed(X["xp"], X["z"], X["dt_raw"], X["B"], X["C"], P["A_log"],
+                                     P["D"], P["conv_w"], P["conv_b"], P["dt_bias"],
+                                     seq_idx=X["seq_idx"], y=y, h_out=h, conv_state_out=cs,
+                                     workspace=ws, stream=stream)
+            return
         M.mamba_mixer_fwd(X["xp"], X["z"], X["dt_raw"], X["B"], X["C"], P["A_log"], P["D"],
                           P["conv_w"], P["conv_b"], P["dt_bias"], y=y, h_out=h,
                           conv_state_out=cs, workspace=ws, stream=stream)
@@ -364,7 +373,7 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
     else:
         dom_ms = statistics.mean(fwd_ms)
         dom_bytes = bytes_["fwd"]
-        dom = "mamba_mixer_fwd"
+        dom = "mamba_mixer_fwd_packed" if w.packed_mean else "mamba_mixer_fwd"
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     clocks = clk.summary()
     sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
@@ -408,7 +417,10 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
             "workload": w.name,
             "batch": w.batch, "seqlen": w.seqlen, "d_inner": w.d_inner, "d_state": w.d_state,
             "d_conv": w.d_conv, "io": w.io_dtype, "state": "f32",
-            "step": "decode step only" if w.decode else "fused forward over the prompt + one decode step (state in place)",
+            "step": ("decode step only" if w.decode else
+                     "fused forward over the prompt + one decode step (state in place)"),
+            "documents": (f"packed, mean length {w.packed_mean} (seq_idx resets)"
+                          if w.packed_mean else None),
             "global_batch": w.batch * world,
             "parallelism": f"replicas x{world} (independent sequences per GPU, no collective)",
             "l2": "flushed between timed steps (256 MiB write + 256 MiB read, outside the timed events)",

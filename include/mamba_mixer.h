@@ -133,6 +133,37 @@ MAMBA_API int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void
                     void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * The fused forward over packed documents and/or from a cached state (niverel-mamba 0.1.0,
+ * section "seq_idx strict reset"; the state pair is the one of section "Autoregressive
+ * decoding").  Same arguments, workspace and result as mamba_mixer_fwd, plus three
+ * optional inputs (each may be NULL):
+ *   seq_idx        int32 [batch, seqlen], 4-byte aligned: document ids.  Wherever
+ *                  seq_idx[b, t] != seq_idx[b, t-1], the conv state and the SSM state reset
+ *                  to zero before token t, so a packed row equals its documents run one by
+ *                  one and concatenated; boundaries need not align with anything.  The ids'
+ *                  values do not matter, only where they change; position 0 never resets.
+ *   h_in           fp32 [batch, d_inner, d_state], 16-byte aligned: the SSM state before
+ *                  token 0 (zero when NULL), e.g. a previous call's h_out, so a long prompt
+ *                  can be fed in pieces.
+ *   conv_state_in  io dtype [batch, d_inner, 3], 2-byte aligned: the 3 inputs before
+ *                  token 0, oldest first (zeros when NULL), e.g. a previous conv_state_out.
+ * The initial state belongs to each row's first document.  h_out and conv_state_out are
+ * the last document's (slots of conv_state_out older than its first token are zero).  With
+ * all three NULL this is mamba_mixer_fwd.  Outputs must not overlap any input (h_in and
+ * conv_state_in included: no in-place update here, since time chunks read the initial
+ * state while the last chunk writes the final one).  A reset is applied as a zero decay of
+ * the state: for finite states this is the reset; a non-finite state stays non-finite.
+ */
+MAMBA_API int mamba_mixer_fwd_packed(const mamba_dims* dims, const void* xp, const void* z,
+                                     const void* dt_raw, const void* B, const void* C,
+                                     const float* A_log, const float* D, const float* conv_w,
+                                     const float* conv_b, const float* dt_bias,
+                                     const int32_t* seq_idx, const float* h_in,
+                                     const void* conv_state_in, void* y, float* h_out,
+                                     void* conv_state_out, void* workspace,
+                                     size_t workspace_bytes, void* cuda_stream);
+
+/*
  * One decode step: one token for each of `batch` sequences (dims->seqlen must be 1) on a
  * cached state.  Inputs: xp, z, dt_raw [batch, 1, d_inner]; B, C [batch, 1, d_state];
  * the parameters as for mamba_mixer_fwd; h_in [batch, d_inner, d_state] fp32 and

@@ -30,6 +30,14 @@
 //   The main pass folds h = P*h + H over the earlier chunks to get its initial state.
 //   Steps past the chunk end get Delta = Delta*u = 0, which leaves the state unchanged.
 //
+// Packed documents and initial state (kExt kernels; niverel-mamba 0.1.0, section "seq_idx
+// strict reset")
+//   Where seq_idx[b, t] != seq_idx[b, t-1] both states restart from zero at step t: the prep
+//   warps drop the conv taps that lie before t, and hand the scan a decay step of +inf
+//   (exp(+inf * A) = 0, A clamped strictly negative) while Delta*u is unchanged, so the scan
+//   and the chunk pairs need no extra work.  An initial state (h_in, conv_state_in, either
+//   optional, any mode) seeds chunk 0's recurrence and conv window and the carry fold.
+//
 // Every mbarrier wait is bounded (sm100_primitives.cuh): a warp that gives up leaves its
 // loop, the CTA meets at a final barrier, waits (bounded) for the copies it started,
 // records MAMBA_ERR_TIMEOUT in the status word and returns without writing states.
@@ -37,6 +45,8 @@
 
 #include <cuda.h>
 #include <float.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "sm100_primitives.cuh"
@@ -62,6 +72,19 @@ struct FwdParams {
   // barrier but issues none of its copies, so the waits on it run out.
   int inject_skip_tile;
 };
+
+// Extra inputs of the kExt kernels (each may be null).  Only those kernels take them, so the
+// plain kernels' parameters stay as they are.
+struct FwdExt {
+  const int32_t* seq_idx;  // [batch, L] document ids
+  const float* h_in;       // [batch, d_inner, N] initial state
+  const void* cs_in;       // [batch, d_inner, 3] initial conv window
+};
+struct FwdParamsExt : FwdParams {
+  FwdExt ext;
+};
+template <bool kExt>
+using FwdArgs = typename std::conditional<kExt, FwdParamsExt, FwdParams>::type;
 
 constexpr int kCh = 32;          // channels per CTA
 constexpr int kTileT = 32;       // time steps per tile
@@ -174,11 +197,11 @@ __device__ __forceinline__ void sts_f32x4(uint32_t a, float x, float y, float z,
                "f"(w) : "memory");
 }
 
-template <int N, typename IO, bool kPrecise, bool kPrepass>
+template <int N, typename IO, bool kPrecise, bool kPrepass, bool kExt>
 __global__ void __launch_bounds__(kFwdThreads)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
            const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_B,
-           const __grid_constant__ CUtensorMap tm_C, const FwdParams p) {
+           const __grid_constant__ CUtensorMap tm_C, const FwdArgs<kExt> p) {
   using M = Math<kPrecise>;
   using S = FwdSmem<IO, N>;
   constexpr int kS = N / 4;
@@ -286,15 +309,88 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
       float xa = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 1, col));
       float xb = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 2, col));
       float xc = lds_io<IO>(st + S::kXOff + swz<kRow>(t0 + 3, col));
+      [[maybe_unused]] uint32_t resets = 0;   // bit i + 3: reset at step tt + t0 + i (i >= -3)
+      if constexpr (kExt) {
+        if (p.ext.cs_in && c == 0 && k == 0 && w == 0 && active) {
+          // t < 0 of the row: the cached window instead of the zero padding
+          const IO* cw = static_cast<const IO*>(p.ext.cs_in) + (int64_t(b) * p.Di + d) * 3;
+          xa = IOT<IO>::to_f(cw[0]);
+          xb = IOT<IO>::to_f(cw[1]);
+          xc = IOT<IO>::to_f(cw[2]);
+        }
+      }
+      // document ids of steps tt + t0 - 3 .. tt + t0 + kPrepSteps - 1: a reset at step T is
+      // an id change between T - 1 and T; the row's first step never resets
+      if constexpr (kExt) if (p.ext.seq_idx) {
+        // lane l reads the id of step T0 - 4 + l (l < kPrepSteps + 4) and compares it with
+        // lane l - 1's: one load, one shuffle and one vote per warp and tile
+        const int64_t T = tt + t0 - 4 + lane;
+        const bool in = T >= 0 && T < p.L && lane < kPrepSteps + 4;
+        const int32_t cur = in ? __ldg(p.ext.seq_idx + int64_t(b) * p.L + T) : 0;
+        const int32_t prv = __shfl_up_sync(0xffffffffu, cur, 1);
+        const bool reset = in && lane >= 1 && T >= 1 && cur != prv;
+        resets = __ballot_sync(0xffffffffu, reset) >> 1;   // bit i + 3 <- lane i + 4
+      }
+      // One tile of per-(t, d) work; kMasked applies the document resets (the plain path
+      // is the kMasked = false instance, and a tile without resets takes it too).
+      auto prep_steps = [&](auto masked_tag) {
+        constexpr bool kMasked = decltype(masked_tag)::value;
 #pragma unroll
       for (int qq = 0; qq < kPrepSteps / 4; ++qq) {
         const int q = t0 / 4 + qq;
-        float dv[4], duv[4], skv[4], szv[4];
+        float dv[4], duv[4];
+        [[maybe_unused]] float skv[4], szv[4];
+        if constexpr (!kPrecise && !kMasked && kExt) {
+          // two steps at a time in f32x2 lanes: same operations and results as the scalar
+          // loop below, fewer issue slots.  Measured faster for the extended kernels (m130
+          // rows of documents 229 -> 218 us) but slower for the plain ones (210 -> 216 us,
+          // a different register allocation), which therefore keep the scalar loop.
+#pragma unroll
+          for (int ip = 0; ip < 2; ++ip) {
+            const int ta = 4 * q + 2 * ip;
+            const float xta = lds_io<IO>(st + S::kXOff + swz<kRow>(ta + 4, col));
+            const float xtb = lds_io<IO>(st + S::kXOff + swz<kRow>(ta + 5, col));
+            f32x2 pre = fma2(pk2(w0, w0), pk2(xa, xb), pk2(cb, cb));
+            pre = fma2(pk2(w1, w1), pk2(xb, xc), pre);
+            pre = fma2(pk2(w2, w2), pk2(xc, xta), pre);
+            pre = fma2(pk2(w3, w3), pk2(xta, xtb), pre);
+            xa = xc; xb = xta; xc = xtb;
+            const f32x2 u2 = silu2_fma(pre);
+            const f32x2 dtv = add2_(pk2(lds_io<IO>(st + S::kDtOff + swz<kRow>(ta, col)),
+                                        lds_io<IO>(st + S::kDtOff + swz<kRow>(ta + 1, col))),
+                                    pk2(dtb, dtb));
+            const f32x2 dl2 = softplus2_fma(dtv);
+            float dla, dlb, dua, dub;
+            upk2(dl2, dla, dlb);
+            upk2(mul2(dl2, u2), dua, dub);
+            const bool va = tt + ta < t_end, vb = tt + ta + 1 < t_end;
+            dv[2 * ip] = va ? dla : 0.0f;
+            dv[2 * ip + 1] = vb ? dlb : 0.0f;
+            duv[2 * ip] = va ? dua : 0.0f;
+            duv[2 * ip + 1] = vb ? dub : 0.0f;
+            if constexpr (!kPrepass) {
+              upk2(mul2(pk2(Dd, Dd), u2), skv[2 * ip], skv[2 * ip + 1]);
+              const f32x2 z2 = pk2(lds_io<IO>(st + S::kZOff + swz<kRow>(ta, col)),
+                                   lds_io<IO>(st + S::kZOff + swz<kRow>(ta + 1, col)));
+              upk2(silu2_fma(z2), szv[2 * ip], szv[2 * ip + 1]);
+            }
+          }
+        } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = 4 * q + i;
           const float xt = lds_io<IO>(st + S::kXOff + swz<kRow>(t + 4, col));
-          const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          float pre;
+          if constexpr (kMasked) {
+            // taps before the document's first step are zero
+            const int r = 4 * qq + i + 3;   // bit of step t
+            const bool m1 = !((resets >> r) & 1u);
+            const bool m2 = m1 && !((resets >> (r - 1)) & 1u);
+            const bool m3 = m2 && !((resets >> (r - 2)) & 1u);
+            pre = cb + w0 * (m3 ? xa : 0.0f) + w1 * (m2 ? xb : 0.0f) + w2 * (m1 ? xc : 0.0f) + w3 * xt;
+          } else {
+            pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          }
           xa = xb; xb = xc; xc = xt;
           const float u = kPrecise ? M::silu(pre) : silu_fma(pre);
           const bool valid = tt + t < t_end;
@@ -302,11 +398,15 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
           const float dl = kPrecise ? M::softplus(dtv) : softplus_fma(dtv);
           dv[i] = valid ? dl : 0.0f;
           duv[i] = valid ? dl * u : 0.0f;
+          if constexpr (kMasked)
+            if (valid && ((resets >> (4 * qq + i + 3)) & 1u))
+              dv[i] = __int_as_float(0x7f800000);   // +inf: this step's decay is 0
           if constexpr (!kPrepass) {
             skv[i] = Dd * u;
             const float zv = lds_io<IO>(st + S::kZOff + swz<kRow>(t, col));
             szv[i] = kPrecise ? M::silu(zv) : silu_fma(zv);
           }
+        }
         }
         const uint32_t rec = pr + S::kScOff;
         sts_f32x4(rec + sc_unit(q, cl, 0), dv[0], dv[1], dv[2], dv[3]);
@@ -316,18 +416,47 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
           sts_f32x4(rec + sc_unit(q, cl, 3), szv[0], szv[1], szv[2], szv[3]);
         }
       }
+      };
+      if (kExt && resets != 0)   // warp-uniform
+        prep_steps(std::true_type{});
+      else
+        prep_steps(std::false_type{});
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&prep_ready[r]);
         mbar_arrive(&raw_free[s]);
       }
-      // new conv state: last 3 entries of xpad, x'[L-3+i] (zeros for negative t)
+      // new conv state: last 3 entries of xpad, x'[L-3+i] (the initial window or zeros for
+      // negative positions); with documents, slots older than the last document's first
+      // step are zero (slot i needs no reset at steps L-2+i .. L-1)
       if (!kPrepass && w == kPrepWarps - 1 && k == ntiles - 1 && c == p.nchunks - 1 && p.cs_out && active) {
         IO* cs = static_cast<IO*>(p.cs_out) + (int64_t(b) * p.Di + d) * 3;
+        if constexpr (kExt) {
+          bool keep0 = true, keep1 = true;
+          if (p.ext.seq_idx) {
+            const int32_t* sq = p.ext.seq_idx + int64_t(b) * p.L;
+            const bool r1 = p.L - 1 >= 1 && __ldg(sq + p.L - 1) != __ldg(sq + p.L - 2);
+            const bool r2 = p.L - 2 >= 1 && __ldg(sq + p.L - 2) != __ldg(sq + p.L - 3);
+            keep1 = !r1;
+            keep0 = !r1 && !r2;
+          }
 #pragma unroll
-        for (int i = 0; i < 3; ++i) {
-          const int rr = int(p.L - 3 + i - (tt - kHalo));
-          cs[i] = IOT<IO>::from_f(lds_io<IO>(st + S::kXOff + swz<kRow>(rr, col)));
+          for (int i = 0; i < 3; ++i) {
+            const int64_t pos = p.L - 3 + i;
+            float v;
+            if (pos < 0 && p.ext.cs_in)
+              v = IOT<IO>::to_f(static_cast<const IO*>(p.ext.cs_in)[(int64_t(b) * p.Di + d) * 3 + (p.L + i)]);
+            else
+              v = lds_io<IO>(st + S::kXOff + swz<kRow>(int(pos - (tt - kHalo)), col));
+            if ((i == 0 && !keep0) || (i == 1 && !keep1)) v = 0.0f;
+            cs[i] = IOT<IO>::from_f(v);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 3; ++i) {
+            const int rr = int(p.L - 3 + i - (tt - kHalo));
+            cs[i] = IOT<IO>::from_f(lds_io<IO>(st + S::kXOff + swz<kRow>(rr, col)));
+          }
         }
       }
       // refill this raw stage with tile k + kStages once both prep warps are done with it
@@ -361,10 +490,18 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     // A = -exp(A_log) (held times log2 e on the fast path); clamped finite so that a
     // masked step (Delta = 0) multiplies to exactly 0 and decays by exactly 1.
     A2[s] = fmaxf(M::neg_exp(__ldg(p.A_log + d * N + j * kS + s)) * M::a_scale(), -FLT_MAX);
+    // with resets, also strictly negative, so that a reset step (+inf) decays to exactly 0
+    if constexpr (kExt) A2[s] = fminf(A2[s], -FLT_MIN);
     h[s] = 0.0f;
     P[s] = 1.0f;
   }
   if constexpr (!kPrepass) {
+    // chunk c starts from the initial state carried through chunks 0..c-1
+    if constexpr (kExt) if (p.ext.h_in) {
+      const float* hi = p.ext.h_in + (int64_t(b) * p.Di + d) * N + j * kS;
+#pragma unroll
+      for (int s = 0; s < kS; ++s) h[s] = __ldg(hi + s);
+    }
     for (int cc = 0; cc < c; ++cc) {
       const int64_t o = ((int64_t(b) * (p.nchunks - 1) + cc) * p.Di + d) * N + j * kS;
 #pragma unroll

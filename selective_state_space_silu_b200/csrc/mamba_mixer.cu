@@ -187,11 +187,11 @@ struct FwdMaps {
   CUtensorMap x, z, dt, B, C;
 };
 
-template <int N, typename IO, bool P, bool kPre>
-cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdParams& a, dim3 grid,
+template <int N, typename IO, bool P, bool kPre, bool kExt>
+cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdArgs<kExt>& a, dim3 grid,
                               cudaStream_t st) {
   using S = mm::FwdSmem<IO, N>;
-  auto kern = mm::fwd_kernel<N, IO, P, kPre>;
+  auto kern = mm::fwd_kernel<N, IO, P, kPre, kExt>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        S::kDynamic);
   if (e != cudaSuccess) return e;
@@ -199,16 +199,28 @@ cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdParams& a, dim3 gri
   return cudaGetLastError();
 }
 
-template <int N, typename IO, bool P>
-cudaError_t launch_fwd(const FwdMaps& m, const mm::FwdParams& a, int64_t batch, cudaStream_t st) {
+template <int N, typename IO, bool P, bool kExt>
+cudaError_t launch_fwd(const FwdMaps& m, const mm::FwdArgs<kExt>& a, int64_t batch,
+                       cudaStream_t st) {
   const unsigned gx = unsigned((a.Di + mm::kCh - 1) / mm::kCh);
   if (a.nchunks > 1) {
-    cudaError_t e = launch_fwd_kernel<N, IO, P, true>(
+    cudaError_t e = launch_fwd_kernel<N, IO, P, true, kExt>(
         m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), st);
     if (e != cudaSuccess) return e;
   }
-  return launch_fwd_kernel<N, IO, P, false>(m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks)),
-                                            st);
+  return launch_fwd_kernel<N, IO, P, false, kExt>(
+      m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks)), st);
+}
+
+template <bool kExt>
+cudaError_t launch_fwd_any(const FwdMaps& m, const mm::FwdArgs<kExt>& a, const mamba_dims* d,
+                           cudaStream_t st) {
+  const bool f32 = d->io_dtype == MAMBA_F32;
+  if (d->d_state == 16)
+    return f32 ? launch_fwd<16, float, true, kExt>(m, a, d->batch, st)
+               : launch_fwd<16, __nv_bfloat16, false, kExt>(m, a, d->batch, st);
+  return f32 ? launch_fwd<8, float, true, kExt>(m, a, d->batch, st)
+             : launch_fwd<8, __nv_bfloat16, false, kExt>(m, a, d->batch, st);
 }
 
 template <int N, typename IO, bool P>
@@ -238,11 +250,18 @@ size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims) {
   return workspace_bytes_for(dims, make_plan(dims));
 }
 
-int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
-                    const void* B, const void* C, const float* A_log, const float* D,
-                    const float* conv_w, const float* conv_b, const float* dt_bias, void* y,
-                    float* h_out, void* conv_state_out, void* workspace,
-                    size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+// The forward behind mamba_mixer_fwd and mamba_mixer_fwd_packed: seq_idx, h_in and
+// conv_state_in are null for the former.
+int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+               const void* B, const void* C, const float* A_log, const float* D,
+               const float* conv_w, const float* conv_b, const float* dt_bias,
+               const int32_t* seq_idx, const float* h_in, const void* conv_state_in, void* y,
+               float* h_out, void* conv_state_out, void* workspace, size_t workspace_bytes,
+               void* cuda_stream) {
   Sizes s;
   int rc = check_dims(dims, &s);
   if (rc) return rc;
@@ -256,7 +275,10 @@ int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const
       (rc = check_ptr(conv_b, "conv_b", false, 4)) ||
       (rc = check_ptr(dt_bias, "dt_bias", dims->d_inner > 0, 4)) ||
       (rc = check_ptr(h_out, "h_out", false, 16)) ||
-      (rc = check_ptr(conv_state_out, "conv_state_out", false, 2)))
+      (rc = check_ptr(conv_state_out, "conv_state_out", false, 2)) ||
+      (rc = check_ptr(seq_idx, "seq_idx", false, 4)) ||
+      (rc = check_ptr(h_in, "h_in", false, 16)) ||
+      (rc = check_ptr(conv_state_in, "conv_state_in", false, 2)))
     return rc;
   const int64_t Di = dims->d_inner, N = dims->d_state;
   const Span ins[] = {{xp, size_t(s.act) * s.esize, "xp"},   {z, size_t(s.act) * s.esize, "z"},
@@ -264,7 +286,10 @@ int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const
                       {B, size_t(s.bc) * s.esize, "B"},     {C, size_t(s.bc) * s.esize, "C"},
                       {A_log, size_t(Di * N) * 4, "A_log"}, {D, size_t(Di) * 4, "D"},
                       {conv_w, size_t(Di) * 16, "conv_w"},  {conv_b, size_t(Di) * 4, "conv_b"},
-                      {dt_bias, size_t(Di) * 4, "dt_bias"}};
+                      {dt_bias, size_t(Di) * 4, "dt_bias"},
+                      {seq_idx, size_t(dims->batch) * size_t(dims->seqlen) * 4, "seq_idx"},
+                      {h_in, size_t(s.state) * 4, "h_in"},
+                      {conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"}};
   const Span outs[] = {{y, size_t(s.act) * s.esize, "y"},
                        {h_out, size_t(s.state) * 4, "h_out"},
                        {conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"}};
@@ -291,11 +316,15 @@ int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const bool f32 = dims->io_dtype == MAMBA_F32;
   if (dims->seqlen == 0) {
-    // empty sequence: the states are the zero initial state and zero padding
+    // empty sequence: the states out are the initial ones (zero when absent)
     cudaError_t e = cudaSuccess;
-    if (h_out) e = cudaMemsetAsync(h_out, 0, size_t(s.state) * 4, st);
+    if (h_out)
+      e = h_in ? cudaMemcpyAsync(h_out, h_in, size_t(s.state) * 4, cudaMemcpyDeviceToDevice, st)
+               : cudaMemsetAsync(h_out, 0, size_t(s.state) * 4, st);
     if (e == cudaSuccess && conv_state_out)
-      e = cudaMemsetAsync(conv_state_out, 0, size_t(s.cstate) * s.esize, st);
+      e = conv_state_in ? cudaMemcpyAsync(conv_state_out, conv_state_in, size_t(s.cstate) * s.esize,
+                                          cudaMemcpyDeviceToDevice, st)
+                        : cudaMemsetAsync(conv_state_out, 0, size_t(s.cstate) * s.esize, st);
     if (e != cudaSuccess)
       return fail(MAMBA_ERR_CUDA, "state reset failed: %s", cudaGetErrorString(e));
     return ok();
@@ -328,15 +357,45 @@ int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const
     a.ws_H = a.ws_P + agg;
   }
   cudaError_t e;
-  if (N == 16)
-    e = f32 ? launch_fwd<16, float, true>(m, a, dims->batch, st)
-            : launch_fwd<16, __nv_bfloat16, false>(m, a, dims->batch, st);
-  else
-    e = f32 ? launch_fwd<8, float, true>(m, a, dims->batch, st)
-            : launch_fwd<8, __nv_bfloat16, false>(m, a, dims->batch, st);
+  if (seq_idx || h_in || conv_state_in) {
+    mm::FwdArgs<true> ax;
+    static_cast<mm::FwdParams&>(ax) = a;
+    ax.ext = mm::FwdExt{seq_idx, h_in, conv_state_in};
+    e = launch_fwd_any<true>(m, ax, dims, st);
+  } else {
+    mm::FwdArgs<false> ap;
+    static_cast<mm::FwdParams&>(ap) = a;
+    e = launch_fwd_any<false>(m, ap, dims, st);
+  }
   if (e != cudaSuccess)
     return fail(MAMBA_ERR_CUDA, "forward launch failed: %s", cudaGetErrorString(e));
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int mamba_mixer_fwd(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+                    const void* B, const void* C, const float* A_log, const float* D,
+                    const float* conv_w, const float* conv_b, const float* dt_bias, void* y,
+                    float* h_out, void* conv_state_out, void* workspace,
+                    size_t workspace_bytes, void* cuda_stream) {
+  return fwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
+                    nullptr, nullptr, y, h_out, conv_state_out, workspace, workspace_bytes,
+                    cuda_stream);
+}
+
+int mamba_mixer_fwd_packed(const mamba_dims* dims, const void* xp, const void* z,
+                           const void* dt_raw, const void* B, const void* C, const float* A_log,
+                           const float* D, const float* conv_w, const float* conv_b,
+                           const float* dt_bias, const int32_t* seq_idx, const float* h_in,
+                           const void* conv_state_in, void* y, float* h_out,
+                           void* conv_state_out, void* workspace, size_t workspace_bytes,
+                           void* cuda_stream) {
+  return fwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, seq_idx, h_in,
+                    conv_state_in, y, h_out, conv_state_out, workspace, workspace_bytes,
+                    cuda_stream);
 }
 
 int mamba_mixer_fwd_launches(const mamba_dims* dims) {

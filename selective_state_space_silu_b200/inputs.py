@@ -51,6 +51,7 @@ class Workload:
     io_dtype: str          # "f32" or "bf16"
     seed: int
     decode: bool = False   # True: one token on top of a cached state
+    packed_mean: int = 0   # > 0: rows pack documents of this mean length (seq_idx)
 
     @property
     def io_bytes(self) -> int:
@@ -66,6 +67,8 @@ WORKLOADS: Dict[str, Workload] = {
     "m130": Workload("m130", 8, 2048, 1536, 16, 4, BF16, 1002),
     "long": Workload("long", 2, 65536, 2560, 16, 4, BF16, 1003),
     "decode": Workload("decode", 256, 1, 5120, 16, 4, BF16, 1004, decode=True),
+    # the 130M-class layer over rows that pack documents of mean length 256
+    "m130_packed": Workload("m130_packed", 8, 2048, 1536, 16, 4, BF16, 1005, packed_mean=256),
 }
 
 
@@ -139,6 +142,8 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray
     if w.decode:
         out["h"] = _normal(rng, (Bt, Di, N))
         out["conv_state"] = _act(_normal(rng, (Bt, Di, K - 1)), w.io_dtype)
+    if w.packed_mean > 0:
+        out["seq_idx"] = packed_seq_idx(Bt, L, w.packed_mean, (w.seed if seed is None else seed) + 1)
     return out
 
 

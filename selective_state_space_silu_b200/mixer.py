@@ -24,7 +24,8 @@ STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPOR
           3: "MAMBA_ERR_ALIGNMENT", 4: "MAMBA_ERR_WORKSPACE", 5: "MAMBA_ERR_CUDA",
           6: "MAMBA_ERR_TIMEOUT"}
 EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba_mixer_fwd",
-           "mamba_mixer_step", "mamba_mixer_check", "mamba_last_error", "mamba_version")
+           "mamba_mixer_fwd_packed", "mamba_mixer_step", "mamba_mixer_check", "mamba_last_error",
+           "mamba_version")
 
 
 class MambaError(RuntimeError):
@@ -63,6 +64,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba_mixer_check.argtypes = [vp, vp]
     lib.mamba_mixer_fwd.restype = i
     lib.mamba_mixer_fwd.argtypes = [P] + [vp] * 13 + [vp, sz, vp]
+    lib.mamba_mixer_fwd_packed.restype = i
+    lib.mamba_mixer_fwd_packed.argtypes = [P] + [vp] * 16 + [vp, sz, vp]
     lib.mamba_mixer_step.restype = i
     lib.mamba_mixer_step.argtypes = [P] + [vp] * 15 + [vp]
     lib.mamba_last_error.restype = ctypes.c_char_p
@@ -171,6 +174,48 @@ def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
         _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
         _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
         _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
+        _ptr(conv_state_out, "conv_state_out", iot, dev),
+        _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
+    _check(rc)
+    return y, h_out, conv_state_out
+
+
+def mamba_mixer_fwd_packed(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
+                           seq_idx=None, h_in=None, conv_state_in=None, y=None, h_out=None,
+                           conv_state_out=None, workspace=None, stream=None
+                           ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Fused forward over packed documents and/or from a cached state.
+
+    As mamba_mixer_fwd, plus optional seq_idx [batch, L] int32 (the states reset wherever
+    the id changes along t), h_in [batch, d_inner, d_state] fp32 and conv_state_in
+    [batch, d_inner, 3] (the state before token 0).  Returns (y, h_out, conv_state_out).
+    """
+    lib = load_library()
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    dims = make_dims(Bt, L, Di, N, K, io)
+    if y is None:
+        y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
+    if h_out is None:
+        h_out = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+    if conv_state_out is None:
+        conv_state_out = torch.empty((Bt, Di, K - 1), dtype=iot, device=dev)
+    if workspace is None:
+        workspace = new_workspace(dims, dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    f32 = torch.float32
+    rc = lib.mamba_mixer_fwd_packed(
+        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(seq_idx, "seq_idx", torch.int32, dev), _ptr(h_in, "h_in", f32, dev),
+        _ptr(conv_state_in, "conv_state_in", iot, dev),
         _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
         _ptr(conv_state_out, "conv_state_out", iot, dev),
         _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))

@@ -160,3 +160,40 @@ def test_empty_batch_is_a_no_op(lib):
 
 def test_check_rejects_null_workspace(lib):
     assert lib.mamba_mixer_check(None, None) == 1
+
+
+def _fwd_packed(lib, dims, ptrs=None, ws=None, ws_bytes=0):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(
+        ["xp", "z", "dt", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias", "seq", "h_in",
+         "cs_in", "y", "h", "cs"])}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba_mixer_fwd_packed(ctypes.byref(dims), p["xp"], p["z"], p["dt"], p["B"],
+                                      p["C"], p["A_log"], p["D"], p["conv_w"], p["conv_b"],
+                                      p["dt_bias"], p["seq"], p["h_in"], p["cs_in"], p["y"],
+                                      p["h"], p["cs"], ws, ws_bytes, None)
+
+
+def test_packed_forward_validation(lib):
+    d = M.make_dims(2, 64, 128, 16)
+    ws = _fake(0x10000000 + 20 * (1 << 36))
+    # alignment of the three optional inputs
+    assert _fwd_packed(lib, d, {"seq": _fake(0x10000000 + 10 * (1 << 36) + 2)}, ws, 256) == 3
+    assert "seq_idx" in M.mamba_last_error()
+    assert _fwd_packed(lib, d, {"h_in": _fake(0x10000000 + 11 * (1 << 36) + 8)}, ws, 256) == 3
+    assert _fwd_packed(lib, d, {"cs_in": _fake(0x10000000 + 12 * (1 << 36) + 1)}, ws, 256) == 3
+    # no in-place update: the final state may not overlap the initial one
+    h_in = 0x10000000 + 11 * (1 << 36)
+    assert _fwd_packed(lib, d, {"h": _fake(h_in)}, ws, 256) == 1
+    assert "overlaps" in M.mamba_last_error()
+    cs_in = 0x10000000 + 12 * (1 << 36)
+    assert _fwd_packed(lib, d, {"cs": _fake(cs_in)}, ws, 256) == 1
+    # an output overlapping seq_idx
+    assert _fwd_packed(lib, d, {"y": _fake(0x10000000 + 10 * (1 << 36))}, ws, 256) == 1
+    # the workspace rule is the forward's
+    assert _fwd_packed(lib, d, ws=None) == 4
+    # all optional inputs absent and nothing to do: OK without touching the GPU
+    e = M.make_dims(0, 64, 128, 16)
+    assert _fwd_packed(lib, e, {k: None for k in ("xp", "z", "dt", "B", "C", "y", "h", "cs",
+                                                  "seq", "h_in", "cs_in")}, ws, 256) == 0
