@@ -1,0 +1,62 @@
+"""Pins for the backward oracle (oracle_mixer_bwd_f64): every gradient against central
+finite differences of the forward oracle (pinned by test_oracle_pins.py) -- an
+independent route, so a dropped chain-rule term, a wrong sign or a wrong index in the
+backward fails here -- plus the special cases that fix whole gradients to zero."""
+
+import numpy as np
+import pytest
+
+from tests.test_oracle_pins import rand_case, run
+
+GRAD_OF = {"dxp": "xp", "dz": "z", "ddt_raw": "dt_raw", "dB": "B", "dC": "C",
+           "dA_log": "A_log", "dD": "D", "dconv_w": "conv_w", "dconv_b": "conv_b",
+           "ddt_bias": "dt_bias"}
+
+
+def loss(oracle, c, dy):
+    y, _, _ = run(oracle, c)
+    return float((y * dy).sum())
+
+
+def bwd(oracle, c, dy):
+    return oracle.mixer_bwd(c["xp"], c["z"], c["dt_raw"], c["B"], c["C"], c["A_log"], c["D"],
+                            c["conv_w"], c["conv_b"], c["dt_bias"], dy)
+
+
+@pytest.mark.parametrize("seed,N,conv_b", [(11, 3, True), (12, 4, False), (13, 2, True)])
+def test_every_gradient_matches_finite_differences(oracle, seed, N, conv_b):
+    c = rand_case(seed, Bt=2, L=7, Di=3, N=N, conv_b=conv_b, A_range=(-1.0, 1.5))
+    dy = np.random.default_rng(seed + 100).standard_normal(c["xp"].shape)
+    g = bwd(oracle, c, dy)
+    eps = 1e-6
+    for gname, name in GRAD_OF.items():
+        if c[name] is None:
+            assert g[gname] is None
+            continue
+        fd = np.zeros_like(c[name])
+        for ix in np.ndindex(c[name].shape):
+            cp = {k: (None if v is None else np.array(v, dtype=np.float64)) for k, v in c.items()}
+            cp[name][ix] += eps
+            lp = loss(oracle, cp, dy)
+            cp[name][ix] -= 2 * eps
+            lm = loss(oracle, cp, dy)
+            fd[ix] = (lp - lm) / (2 * eps)
+        err = np.abs(fd - g[gname]) / (1.0 + np.abs(fd))
+        assert err.max() < 2e-6, (gname, err.max())
+
+
+def test_zero_upstream_gradient_gives_zeros(oracle):
+    c = rand_case(20, Bt=1, L=5, Di=2, N=3)
+    g = bwd(oracle, c, np.zeros(c["xp"].shape))
+    for k, v in g.items():
+        assert v is None or not np.any(v), k
+
+
+def test_zero_B_leaves_no_state_gradients(oracle):
+    """B = 0: the state stays 0, so C and A_log get no gradient (B itself does)."""
+    c = rand_case(21, Bt=2, L=6, Di=2, N=3)
+    c["B"] = np.zeros_like(c["B"])
+    dy = np.random.default_rng(5).standard_normal(c["xp"].shape)
+    g = bwd(oracle, c, dy)
+    assert not np.any(g["dC"]) and not np.any(g["dA_log"])
+    assert np.any(g["dB"])
