@@ -164,6 +164,36 @@ MAMBA_API int mamba_mixer_fwd_packed(const mamba_dims* dims, const void* xp, con
                                      size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * Device workspace, in bytes, that mamba_mixer_bwd needs for `dims`: a 256-byte header,
+ * then the recurrence's state at the start of every 32-step tile (fp32 [batch,
+ * ceil(seqlen/32), d_inner, d_state]).  0 for unsupported dims.
+ */
+MAMBA_API size_t mamba_mixer_bwd_workspace_bytes(const mamba_dims* dims);
+
+/*
+ * Backward of mamba_mixer_fwd (forward from a zero state, no documents), by forward
+ * recompute (calm-mamba 0.1.4, section "GPU acceleration (Triton kernels)"): the gradients
+ * of sum(dy * y) with respect to every input, in fp32 (the openfluke stress-test page keeps
+ * boundary gradients in Float32).
+ * Inputs: the forward's inputs (same layouts, io dtype activations) and dy [batch, seqlen,
+ * d_inner] in the io dtype.  Outputs (fp32, device, all overwritten):
+ *   dxp, dz, ddt_raw [batch, seqlen, d_inner]; dB, dC [batch, seqlen, d_state] (summed over
+ *   the channels that share B and C); dA_log [d_inner, d_state]; dD, ddt_bias [d_inner];
+ *   dconv_w [d_inner, d_conv]; dconv_b [d_inner] (may be NULL: not computed).
+ * The sums over channels, batch rows and time use atomic additions, so the last bits of
+ * those outputs may differ between runs.  Outputs must not overlap any input, each other
+ * or the workspace (16-byte aligned, mamba_mixer_bwd_workspace_bytes(dims) bytes).
+ */
+MAMBA_API int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z,
+                              const void* dt_raw, const void* B, const void* C,
+                              const float* A_log, const float* D, const float* conv_w,
+                              const float* conv_b, const float* dt_bias, const void* dy,
+                              float* dxp, float* dz, float* ddt_raw, float* dB, float* dC,
+                              float* dA_log, float* dD, float* dconv_w, float* dconv_b,
+                              float* ddt_bias, void* workspace, size_t workspace_bytes,
+                              void* cuda_stream);
+
+/*
  * One decode step: one token for each of `batch` sequences (dims->seqlen must be 1) on a
  * cached state.  Inputs: xp, z, dt_raw [batch, 1, d_inner]; B, C [batch, 1, d_state];
  * the parameters as for mamba_mixer_fwd; h_in [batch, d_inner, d_state] fp32 and

@@ -12,10 +12,12 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 
 #include "mamba_mixer.h"
 #include "fwd_kernel.cuh"
 #include "step.cuh"
+#include "bwd_kernel.cuh"
 
 namespace {
 
@@ -224,6 +226,23 @@ cudaError_t launch_fwd_any(const FwdMaps& m, const mm::FwdArgs<kExt>& a, const m
 }
 
 template <int N, typename IO, bool P>
+cudaError_t launch_bwd(const mm::BwdParams& a, int64_t batch, cudaStream_t st) {
+  constexpr int smem = mm::BwdSmem<N>::kTotal;
+  auto kern = mm::bwd_kernel<N, IO, P>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const unsigned gx = unsigned((a.Di + mm::kBwdCh - 1) / mm::kBwdCh);
+  kern<<<dim3(gx, unsigned(batch)), mm::kBwdThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+size_t bwd_workspace_for(const mamba_dims* d) {
+  const int64_t tiles = (d->seqlen + mm::kBwdT - 1) / mm::kBwdT;
+  return kWsHeader + size_t(d->batch) * size_t(tiles) * size_t(d->d_inner) * size_t(d->d_state) *
+                         sizeof(float);
+}
+
+template <int N, typename IO, bool P>
 cudaError_t launch_step(const mm::StepArgs& a, cudaStream_t st) {
   const int64_t bx = (a.Di * mm::kStepLanes + mm::kStepThreads - 1) / mm::kStepThreads;
   mm::step_kernel<N, IO, P, mm::kStepLanes><<<dim3(unsigned(bx), unsigned(a.batch)),
@@ -420,6 +439,99 @@ int mamba_mixer_check(void* workspace, void* cuda_stream) {
                   "alignment self-check (outputs incomplete)");
     return fail(MAMBA_ERR_TIMEOUT, "a forward kernel gave up on a bounded wait (status %d)", status);
   }
+  return ok();
+}
+
+size_t mamba_mixer_bwd_workspace_bytes(const mamba_dims* dims) {
+  Sizes s;
+  if (check_dims(dims, &s) != MAMBA_OK) return 0;
+  return bwd_workspace_for(dims);
+}
+
+int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+                    const void* B, const void* C, const float* A_log, const float* D,
+                    const float* conv_w, const float* conv_b, const float* dt_bias,
+                    const void* dy, float* dxp, float* dz, float* ddt_raw, float* dB, float* dC,
+                    float* dA_log, float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
+                    void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  Sizes s;
+  int rc = check_dims(dims, &s);
+  if (rc) return rc;
+  const bool act = s.act > 0, bc = s.bc > 0, par = dims->d_inner > 0;
+  if ((rc = check_ptr(xp, "xp", act, 16)) || (rc = check_ptr(z, "z", act, 16)) ||
+      (rc = check_ptr(dt_raw, "dt_raw", act, 16)) || (rc = check_ptr(B, "B", bc, 16)) ||
+      (rc = check_ptr(C, "C", bc, 16)) || (rc = check_ptr(dy, "dy", act, 16)) ||
+      (rc = check_ptr(A_log, "A_log", par, 16)) || (rc = check_ptr(D, "D", par, 4)) ||
+      (rc = check_ptr(conv_w, "conv_w", par, 16)) || (rc = check_ptr(conv_b, "conv_b", false, 4)) ||
+      (rc = check_ptr(dt_bias, "dt_bias", par, 4)) ||
+      (rc = check_ptr(dxp, "dxp", act, 16)) || (rc = check_ptr(dz, "dz", act, 16)) ||
+      (rc = check_ptr(ddt_raw, "ddt_raw", act, 16)) || (rc = check_ptr(dB, "dB", bc, 16)) ||
+      (rc = check_ptr(dC, "dC", bc, 16)) || (rc = check_ptr(dA_log, "dA_log", par, 16)) ||
+      (rc = check_ptr(dD, "dD", par, 4)) || (rc = check_ptr(dconv_w, "dconv_w", par, 16)) ||
+      (rc = check_ptr(dconv_b, "dconv_b", false, 4)) ||
+      (rc = check_ptr(ddt_bias, "ddt_bias", par, 4)))
+    return rc;
+  const int64_t Di = dims->d_inner, N = dims->d_state;
+  const Span ins[] = {{xp, size_t(s.act) * s.esize, "xp"},   {z, size_t(s.act) * s.esize, "z"},
+                      {dt_raw, size_t(s.act) * s.esize, "dt_raw"},
+                      {B, size_t(s.bc) * s.esize, "B"},     {C, size_t(s.bc) * s.esize, "C"},
+                      {dy, size_t(s.act) * s.esize, "dy"},
+                      {A_log, size_t(Di * N) * 4, "A_log"}, {D, size_t(Di) * 4, "D"},
+                      {conv_w, size_t(Di) * 16, "conv_w"},  {conv_b, size_t(Di) * 4, "conv_b"},
+                      {dt_bias, size_t(Di) * 4, "dt_bias"}};
+  const Span outs[] = {{dxp, size_t(s.act) * 4, "dxp"},      {dz, size_t(s.act) * 4, "dz"},
+                       {ddt_raw, size_t(s.act) * 4, "ddt_raw"}, {dB, size_t(s.bc) * 4, "dB"},
+                       {dC, size_t(s.bc) * 4, "dC"},          {dA_log, size_t(Di * N) * 4, "dA_log"},
+                       {dD, size_t(Di) * 4, "dD"},            {dconv_w, size_t(Di) * 16, "dconv_w"},
+                       {dconv_b, size_t(Di) * 4, "dconv_b"},  {ddt_bias, size_t(Di) * 4, "ddt_bias"}};
+  const size_t need = bwd_workspace_for(dims);
+  const Span wsp{workspace, need, "workspace"};
+  for (const Span& o : outs) {
+    for (const Span& i : ins)
+      if (overlaps(o, i)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, i.name);
+    for (const Span& o2 : outs)
+      if (&o2 != &o && overlaps(o, o2))
+        return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, o2.name);
+    if (overlaps(o, wsp)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps workspace", o.name);
+  }
+  for (const Span& i : ins)
+    if (overlaps(i, wsp)) return fail(MAMBA_ERR_INVALID_ARGUMENT, "workspace overlaps %s", i.name);
+  if (!workspace || workspace_bytes < need)
+    return fail(MAMBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed",
+                workspace ? workspace_bytes : size_t(0), need);
+  if (reinterpret_cast<uintptr_t>(workspace) % 16 != 0)
+    return fail(MAMBA_ERR_WORKSPACE, "workspace is not 16-byte aligned");
+  if (dims->batch == 0 || Di == 0) return ok();
+
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  // the sums over channels, batch and time accumulate into zeroed outputs
+  cudaError_t e = cudaSuccess;
+  const std::pair<void*, size_t> zero[] = {
+      {dB, size_t(s.bc) * 4}, {dC, size_t(s.bc) * 4}, {dA_log, size_t(Di * N) * 4},
+      {dD, size_t(Di) * 4}, {dconv_w, size_t(Di) * 16}, {dconv_b, size_t(Di) * 4},
+      {ddt_bias, size_t(Di) * 4}};
+  for (const auto& zr : zero)
+    if (e == cudaSuccess && zr.first && zr.second) e = cudaMemsetAsync(zr.first, 0, zr.second, st);
+  if (e != cudaSuccess) return fail(MAMBA_ERR_CUDA, "gradient reset failed: %s", cudaGetErrorString(e));
+  if (dims->seqlen == 0) return ok();
+
+  mm::BwdParams a{};
+  a.xp = xp; a.z = z; a.dt = dt_raw; a.B = B; a.C = C; a.dy = dy;
+  a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
+  a.dxp = dxp; a.dz = dz; a.ddt = ddt_raw; a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
+  a.dconv_w = dconv_w; a.dconv_b = dconv_b; a.ddt_bias = ddt_bias;
+  a.ws_h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + kWsHeader);
+  a.L = dims->seqlen; a.Di = Di;
+  a.ntiles = int((dims->seqlen + mm::kBwdT - 1) / mm::kBwdT);
+  const bool f32 = dims->io_dtype == MAMBA_F32;
+  if (N == 16)
+    e = f32 ? launch_bwd<16, float, true>(a, dims->batch, st)
+            : launch_bwd<16, __nv_bfloat16, false>(a, dims->batch, st);
+  else
+    e = f32 ? launch_bwd<8, float, true>(a, dims->batch, st)
+            : launch_bwd<8, __nv_bfloat16, false>(a, dims->batch, st);
+  if (e != cudaSuccess)
+    return fail(MAMBA_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(e));
   return ok();
 }
 

@@ -24,8 +24,8 @@ STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPOR
           3: "MAMBA_ERR_ALIGNMENT", 4: "MAMBA_ERR_WORKSPACE", 5: "MAMBA_ERR_CUDA",
           6: "MAMBA_ERR_TIMEOUT"}
 EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba_mixer_fwd",
-           "mamba_mixer_fwd_packed", "mamba_mixer_step", "mamba_mixer_check", "mamba_last_error",
-           "mamba_version")
+           "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
+           "mamba_mixer_step", "mamba_mixer_check", "mamba_last_error", "mamba_version")
 
 
 class MambaError(RuntimeError):
@@ -66,6 +66,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba_mixer_fwd.argtypes = [P] + [vp] * 13 + [vp, sz, vp]
     lib.mamba_mixer_fwd_packed.restype = i
     lib.mamba_mixer_fwd_packed.argtypes = [P] + [vp] * 16 + [vp, sz, vp]
+    lib.mamba_mixer_bwd_workspace_bytes.restype = sz
+    lib.mamba_mixer_bwd_workspace_bytes.argtypes = [P]
+    lib.mamba_mixer_bwd.restype = i
+    lib.mamba_mixer_bwd.argtypes = [P] + [vp] * 21 + [vp, sz, vp]
     lib.mamba_mixer_step.restype = i
     lib.mamba_mixer_step.argtypes = [P] + [vp] * 15 + [vp]
     lib.mamba_last_error.restype = ctypes.c_char_p
@@ -221,6 +225,42 @@ def mamba_mixer_fwd_packed(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bia
         _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
     _check(rc)
     return y, h_out, conv_state_out
+
+
+BWD_OUTPUTS = ("dxp", "dz", "ddt_raw", "dB", "dC", "dA_log", "dD", "dconv_w", "dconv_b",
+               "ddt_bias")
+
+
+def mamba_mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, *,
+                    workspace=None, stream=None) -> dict:
+    """Gradients of sum(dy * y) for mamba_mixer_fwd, all fp32; returns a dict keyed by
+    BWD_OUTPUTS (dconv_b is None when conv_b is None)."""
+    lib = load_library()
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    dims = make_dims(Bt, L, Di, N, K, io)
+    f32 = torch.float32
+    e = lambda *shape: torch.empty(shape, dtype=f32, device=dev)
+    g = {"dxp": e(Bt, L, Di), "dz": e(Bt, L, Di), "ddt_raw": e(Bt, L, Di), "dB": e(Bt, L, N),
+         "dC": e(Bt, L, N), "dA_log": e(Di, N), "dD": e(Di), "dconv_w": e(Di, K),
+         "dconv_b": None if conv_b is None else e(Di), "ddt_bias": e(Di)}
+    need = int(lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(dims)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.mamba_mixer_bwd(
+        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(dy, "dy", iot, dev), *[_ptr(g[k], k, f32, dev) for k in BWD_OUTPUTS],
+        _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
+    _check(rc)
+    return g
 
 
 def mamba_mixer_step(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, h_in,

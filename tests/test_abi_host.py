@@ -197,3 +197,29 @@ def test_packed_forward_validation(lib):
     e = M.make_dims(0, 64, 128, 16)
     assert _fwd_packed(lib, e, {k: None for k in ("xp", "z", "dt", "B", "C", "y", "h", "cs",
                                                   "seq", "h_in", "cs_in")}, ws, 256) == 0
+
+
+def _bwd(lib, dims, ptrs=None, ws=None, ws_bytes=0):
+    base = 0x10000000
+    names = ["xp", "z", "dt", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias", "dy",
+             "dxp", "dz", "ddt", "dB", "dC", "dA_log", "dD", "dconv_w", "dconv_b", "ddt_bias"]
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(names)}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba_mixer_bwd(ctypes.byref(dims), *[p[k] for k in names], ws, ws_bytes, None)
+
+
+def test_backward_validation(lib):
+    d = M.make_dims(2, 64, 128, 16)
+    need = lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(d))
+    assert need == 256 + 2 * 2 * 128 * 16 * 4            # header + two 32-step tile states
+    ws = _fake(0x10000000 + 30 * (1 << 36))
+    assert _bwd(lib, d, ws=None) == 4                       # workspace required
+    assert _bwd(lib, d, ws=ws, ws_bytes=need - 16) == 4
+    assert _bwd(lib, d, {"dy": _fake(0x10000000 + 10 * (1 << 36) + 4)}, ws, need) == 3
+    assert "dy" in M.mamba_last_error()
+    # a gradient output on top of an input or of another output
+    assert _bwd(lib, d, {"dxp": _fake(0x10000000 + 0 * (1 << 36))}, ws, need) == 1
+    assert _bwd(lib, d, {"dz": _fake(0x10000000 + 11 * (1 << 36))}, ws, need) == 1
+    assert _bwd(lib, M.make_dims(2, 64, 128, 12), ws=ws, ws_bytes=need) == 2   # d_state 12
+    assert lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(M.make_dims(2, 64, 128, 12))) == 0

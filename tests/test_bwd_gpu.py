@@ -1,0 +1,69 @@
+"""GPU parity of the backward (mamba_mixer_bwd through the C ABI) with the fp64 backward
+oracle (pinned against finite differences in test_oracle_bwd.py): every gradient, element
+by element, in the gradient tolerance of tests/tolerances.py, on several tiles with
+ragged channel and time tails, in fp32 and bf16, d_state 16 and 8, with and without a conv
+bias; the 130M-class shape on sampled channels."""
+
+import numpy as np
+import pytest
+import torch
+
+from selective_state_space_silu_b200 import inputs as I
+from selective_state_space_silu_b200 import mixer as M
+from tests.gpu_util import host, to_device
+from tests.tolerances import assert_close_grad
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(Bt, L, Di, N, io, seed, conv_b=True):
+    w = I.Workload("bwd", Bt, L, Di, N, 4, io, seed)
+    inp = I.make_inputs(w)
+    if not conv_b:
+        inp["conv_b"] = None
+    r = np.random.default_rng(seed + 1)
+    dy = r.standard_normal((Bt, L, Di)).astype(np.float32)
+    inp["dy"] = I.f32_to_bf16_bits(dy) if io == I.BF16 else dy
+    return w, inp
+
+
+def _run(inp):
+    d = to_device(inp)
+    g = M.mamba_mixer_bwd(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                          d["conv_w"], d.get("conv_b"), d["dt_bias"], d["dy"])
+    torch.cuda.synchronize()
+    return {k: (None if v is None else host(v)) for k, v in g.items()}
+
+
+def _oracle(oracle, inp):
+    w = I.as_f64
+    return oracle.mixer_bwd(w(inp["xp"]), w(inp["z"]), w(inp["dt_raw"]), w(inp["B"]),
+                            w(inp["C"]), inp["A_log"], inp["D"], inp["conv_w"], inp.get("conv_b"),
+                            inp["dt_bias"], w(inp["dy"]), nthreads=0)
+
+
+def _compare(g, go, io, what):
+    for k in M.BWD_OUTPUTS:
+        if go[k] is None:
+            assert g[k] is None
+            continue
+        assert_close_grad(g[k], go[k], io, f"{what} {k}")
+
+
+@pytest.mark.parametrize("Bt,L,Di,N,io,conv_b", [
+    (2, 16, 128, 16, I.F32, True),      # tiny config shape
+    (2, 77, 72, 16, I.F32, False),      # ragged time and channel tails
+    (3, 300, 64, 16, I.BF16, True),
+    (2, 129, 104, 8, I.BF16, True),
+    (2, 64, 40, 8, I.F32, True),
+])
+def test_backward_matches_oracle(oracle, Bt, L, Di, N, io, conv_b):
+    w, inp = _case(Bt, L, Di, N, io, 3000 + L + Di, conv_b)
+    _compare(_run(inp), _oracle(oracle, inp), io, f"{Bt}x{L}x{Di} N{N} {io}")
+
+
+def test_backward_130m_two_rows(oracle):
+    """Two batch rows of the 130M-class layer (2 x 2048 x 1536, bf16): every gradient in
+    full, including dB/dC (sums over all 1536 channels) and the parameter gradients."""
+    w, inp = _case(2, 2048, 1536, 16, I.BF16, 3100)
+    _compare(_run(inp), _oracle(oracle, inp), I.BF16, "m130 rows")

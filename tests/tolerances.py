@@ -59,3 +59,33 @@ def assert_close(a, b, io_dtype, what=""):
             f"(max_abs {r['max_abs']:.3e}, max_rel {r['max_rel']:.3e}); first at {idx}: "
             f"got {np.asarray(a)[idx]!r}, oracle {np.asarray(b)[idx]!r}")
     return r
+
+
+def within_grad(a, b, io_dtype):
+    """Tolerance for gradients (device fp32 vs fp64 oracle): the class's bound plus a floor
+    of rtol times the RMS of the oracle tensor.  Most gradients are sums of many terms of
+    both signs (over time, channels or batch rows), whose rounding error scales with the
+    size of the terms rather than with the possibly cancelled result; the tensor's RMS
+    stands in for that size.  Same classes: fp32 I/O (precise math) and bf16 I/O (MUFU)."""
+    atol, rtol = TOL[io_dtype]
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(b[np.isfinite(b)] ** 2))) if b.size else 0.0
+    fin = np.isfinite(a) & np.isfinite(b)
+    ok = np.zeros(a.shape, dtype=bool)
+    ok[fin] = np.abs(a[fin] - b[fin]) <= (atol + rtol * rms +
+                                          rtol * np.maximum(np.abs(a[fin]), np.abs(b[fin])))
+    return ok
+
+
+def assert_close_grad(a, b, io_dtype, what=""):
+    ok = within_grad(a, b, io_dtype)
+    if not ok.all():
+        a = np.asarray(a, dtype=np.float64)
+        b = np.asarray(b, dtype=np.float64)
+        idx = np.unravel_index(int(np.argmin(ok.reshape(-1))), a.shape)
+        d = np.abs(a - b)
+        raise AssertionError(
+            f"{what}: {100 * (1 - ok.mean()):.4f}% outside the {io_dtype} gradient tolerance "
+            f"(max_abs {np.nanmax(d):.3e}, oracle rms {np.sqrt(np.mean(b ** 2)):.3e}); first at "
+            f"{idx}: got {a[idx]!r}, oracle {b[idx]!r}")
