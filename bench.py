@@ -442,6 +442,84 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
     }
 
 
+# ----------------------------------------------------------------------------- backward
+def bwd_bytes(w: I.Workload) -> int:
+    """Algorithmic bytes of one backward: the forward's inputs and dy read once, the fp32
+    gradients written once (the tile-state workspace is not counted)."""
+    s = w.io_bytes
+    Bt, L, Di, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    return (4 * Bt * L * Di * s + 2 * Bt * L * N * s + Di * (4 * N + 28)   # x' z dt dy, B C, params
+            + 3 * Bt * L * Di * 4 + 2 * Bt * L * N * 4 + Di * (4 * N + 28))  # gradients
+
+
+def run_bwd(args, w: I.Workload, local_rank: int):
+    """--pass bwd: times mamba_mixer_bwd alone (device events, L2 flushed between calls)."""
+    import torch
+    from selective_state_space_silu_b200 import mixer as M
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M.load_library()
+    inp = I.make_inputs(w)
+    r = np.random.default_rng(w.seed + 31)
+    dy = r.standard_normal((w.batch, w.seqlen, w.d_inner)).astype(np.float32)
+    inp["dy"] = I.f32_to_bf16_bits(dy) if w.io_dtype == I.BF16 else dy
+
+    def td(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    d = {k: td(v) for k, v in inp.items()}
+    dims = M.make_dims(w.batch, w.seqlen, w.d_inner, w.d_state, 4, M._io_code(d["xp"]))
+    ws = torch.empty(max(M.load_library().mamba_mixer_bwd_workspace_bytes(__import__("ctypes").byref(dims)), 16),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def call():
+        M.mamba_mixer_bwd(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                          d["conv_w"], d["conv_b"], d["dt_bias"], d["dy"], workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for e0, e1 in evs:
+            flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
+            e0.record(stream); call(); e1.record(stream)
+        torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    nbytes = bwd_bytes(w)
+    clocks = clk.summary()
+    sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
+    elems = w.batch * w.seqlen * w.d_inner * w.d_state
+    t_floor = 3 * elems / (MUFU_PER_CLK_SM * SMS * sm_hz)   # three exps per element
+    peaks = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {
+        "metric": "mixer backward: achieved algorithmic GB/s", "pass": "backward",
+        "value": round(achieved, 2), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "dtype": "bf16" if w.io_dtype == I.BF16 else "f32", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                   "d_inner": w.d_inner, "d_state": w.d_state,
+                   "l2": "flushed between calls", "algorithmic_bytes": nbytes},
+        "roofline": {"kernel": "mamba_mixer_bwd", "bound": "alu",
+                     "achieved": round(achieved, 2), "peak": round(nbytes / t_floor / 1e9, 2),
+                     "unit": "GB/s", "frac": round(t_floor / (ms * 1e-3), 4),
+                     "peak_source": "3 exps per (t, d, n) on MUFU (16/clk/SM) x 148 SMs",
+                     "hbm_frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None},
+        "gpu_launches": args.steps, "clocks": clocks,
+    }
+
+
 # ----------------------------------------------------------------------------- oracle
 def oracle_sample(w: I.Workload, target_s: float):
     """Times the CPU oracle, as it stands, on a bounded sample of the workload: all batch
@@ -506,6 +584,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long", choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="bwd: time the backward (mamba_mixer_bwd) alone on the workload")
     ap.add_argument("--seqlen", type=int, default=None,
                     help="override the workload's sequence length (smaller profiling captures)")
     args = ap.parse_args()
@@ -525,6 +605,12 @@ def main():
         res = run_reference(args, w, rank)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+
+    if args.pass_ == "bwd":
+        if w.decode or w.packed_mean:
+            ap.error("--pass bwd needs a plain forward workload")
+        print(json.dumps(run_bwd(args, w, local_rank)), flush=True)
         return
 
     if world > 1:

@@ -165,8 +165,8 @@ MAMBA_API int mamba_mixer_fwd_packed(const mamba_dims* dims, const void* xp, con
 
 /*
  * Device workspace, in bytes, that mamba_mixer_bwd needs for `dims`: a 256-byte header,
- * then the recurrence's state at the start of every 32-step tile (fp32 [batch,
- * ceil(seqlen/32), d_inner, d_state]).  0 for unsupported dims.
+ * then the recurrence's state at the start of every 16-step tile (fp32 [batch,
+ * ceil(seqlen/16), d_inner, d_state]).  0 for unsupported dims.
  */
 MAMBA_API size_t mamba_mixer_bwd_workspace_bytes(const mamba_dims* dims);
 

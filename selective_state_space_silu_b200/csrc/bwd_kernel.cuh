@@ -9,13 +9,15 @@
 // CTA = one batch row x 32 channels, 128 threads = 4 warps of 8 channels x 4 lanes; lane
 // (chl = lane & 7, j = lane >> 3) owns states [j*kS, (j+1)*kS) of channel chl, as in the
 // forward's scan warps.  Two sweeps over time:
-//   forward  -- the recurrence from zero, storing the state at the start of every 32-step
+//   forward  -- the recurrence from zero, storing the state at the start of every 16-step
 //               tile (workspace, fp32 [batch, tiles, d_inner, d_state]);
-//   reverse  -- tiles last to first: reload the tile's start state, recompute its 32
+//   reverse  -- tiles last to first: reload the tile's start state, recompute its 16
 //               states h_t and per-(t, d) scalars into shared memory, then walk the tile
 //               backwards with the adjoint state lam (lam += dyc*C; gradients; lam *= a).
-// The conv's input gradient needs dpre of the 3 following steps, which the reverse walk has
-// just produced: a 3-value window per channel carries it across tiles.  dB and dC are
+// Each tile's inputs are staged in shared memory one tile ahead (16-byte cp.async by all
+// threads, two slots).  The conv's input gradient needs dpre of the 3 following steps,
+// which the reverse walk has just produced: a 3-value window per channel carries it across
+// tiles.  dB and dC are
 // summed over the 8 channels of a warp by butterflies, over the 4 warps in shared memory,
 // and over CTAs (channel tiles) with global atomics; the per-d gradients are summed over
 // batch rows with global atomics.  The gradient outputs must be zero on entry.
@@ -57,39 +59,75 @@ struct BwdParams {
 
 constexpr int kBwdThreads = 128;
 constexpr int kBwdCh = 32;
-constexpr int kBwdT = 32;
+constexpr int kBwdT = 16;       // steps per tile
+constexpr int kBwdHalo = 4;     // x' rows staged before a tile (3 needed)
 
-template <int N>
+template <int N, typename IO>
 struct BwdSmem {
   static constexpr int kS = N / 4;
+  static constexpr int kEs = int(sizeof(IO));
+  static constexpr int kRow = kBwdCh * kEs;                  // one step of 32 channels
+  static constexpr int kBCRow = N * kEs;                     // one step of B (or C)
+  // one staging slot: x' (with halo), dt_raw, z, dy, B, C of one tile
+  static constexpr int kXOff = 0;
+  static constexpr int kDtOff = kXOff + (kBwdT + kBwdHalo) * kRow;
+  static constexpr int kZOff = kDtOff + kBwdT * kRow;
+  static constexpr int kDyOff = kZOff + kBwdT * kRow;
+  static constexpr int kBOff = kDyOff + kBwdT * kRow;
+  static constexpr int kCOff = kBOff + kBwdT * kBCRow;
+  static constexpr int kSlot = kCOff + kBwdT * kBCRow;
   static constexpr int kHs = kBwdT * kBwdThreads * kS * 4;   // h_t per (step, lane)
   static constexpr int kSc = kBwdT * kBwdCh * 16;            // {pre, u, Delta, v} per (step, ch)
-  static constexpr int kX = kBwdT * kBwdCh * 4;              // x'_t per (step, ch)
   static constexpr int kAcc = 2 * kBwdT * N * 4;              // dB, dC partial sums per tile
-  static constexpr int kTotal = kHs + kSc + kX + kAcc;
+  static constexpr int kHsOff = 2 * kSlot;
+  static constexpr int kScOff = kHsOff + kHs;
+  static constexpr int kAccOff = kScOff + kSc;
+  static constexpr int kTotal = kAccOff + kAcc;
+  static_assert(kSlot % 16 == 0 && kRow % 16 == 0 && kBCRow % 16 == 0, "16-byte staging units");
 };
 
-// kS consecutive I/O elements as fp32 (kS = 4 or 2).
+// kS consecutive I/O elements as fp32 from shared memory (kS = 4 or 2).
 template <int kS, typename IO>
-__device__ __forceinline__ void ld_io_row(const IO* p, float* out) {
+__device__ __forceinline__ void lds_io_row(uint32_t a, float* out) {
   if constexpr (sizeof(IO) == 4) {
     if constexpr (kS == 4) {
-      const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+      const float4 v = lds_f32x4(a);
       out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
     } else {
-      const float2 v = __ldg(reinterpret_cast<const float2*>(p));
-      out[0] = v.x; out[1] = v.y;
+      out[0] = lds_f32(a); out[1] = lds_f32(a + 4);
     }
   } else {
     if constexpr (kS == 4) {
-      const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-      out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
-      out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+      uint32_t w0, w1;
+      asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w0), "=r"(w1) : "r"(a));
+      out[0] = __uint_as_float(w0 << 16); out[1] = __uint_as_float(w0 & 0xffff0000u);
+      out[2] = __uint_as_float(w1 << 16); out[3] = __uint_as_float(w1 & 0xffff0000u);
     } else {
-      const uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(p));
-      out[0] = __uint_as_float(v << 16); out[1] = __uint_as_float(v & 0xffff0000u);
+      uint32_t w0;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(a));
+      out[0] = __uint_as_float(w0 << 16); out[1] = __uint_as_float(w0 & 0xffff0000u);
     }
   }
+}
+
+template <typename IO>
+__device__ __forceinline__ float lds_one(uint32_t a) {
+  if constexpr (sizeof(IO) == 4) return lds_f32(a);
+  else return __uint_as_float(lds_u16(a) << 16);
+}
+
+// 16 bytes global -> shared (L2 only), or 16 zero bytes when !valid (src-size 0: the source
+// is not read; a valid address is passed all the same).
+__device__ __forceinline__ void cp_async16_zfill(uint32_t sdst, const void* gsrc, bool valid) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sdst), "l"(gsrc),
+               "r"(valid ? 16 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int kPending>
+__device__ __forceinline__ void cp_async_wait_() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kPending) : "memory");
 }
 
 template <bool kPrecise>
@@ -109,13 +147,14 @@ template <int N, typename IO, bool kPrecise>
 __global__ void __launch_bounds__(kBwdThreads)
 bwd_kernel(const BwdParams p) {
   using M = Math<kPrecise>;
-  using Sm = BwdSmem<N>;
+  using Sm = BwdSmem<N, IO>;
   constexpr int kS = N / 4;
+  constexpr int kEs = Sm::kEs;
   extern __shared__ __align__(16) unsigned char smem[];
-  float* hs = reinterpret_cast<float*>(smem);
-  float4* sc = reinterpret_cast<float4*>(smem + Sm::kHs);
-  float* xs = reinterpret_cast<float*>(smem + Sm::kHs + Sm::kSc);
-  float* acc = reinterpret_cast<float*>(smem + Sm::kHs + Sm::kSc + Sm::kX);  // [2][T][N]
+  const uint32_t sb = smem_addr(smem);
+  float* hs = reinterpret_cast<float*>(smem + Sm::kHsOff);
+  float4* sc = reinterpret_cast<float4*>(smem + Sm::kScOff);
+  float* acc = reinterpret_cast<float*>(smem + Sm::kAccOff);   // [2][T][N]
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -126,16 +165,56 @@ bwd_kernel(const BwdParams p) {
   const int64_t d0 = int64_t(blockIdx.x) * kBwdCh;
   const int64_t b = blockIdx.y;
   // d_inner % 8 == 0: a warp's 8 channels are all in range or all out; an out-of-range warp
-  // takes part in the barriers and shuffles on channel 0's data and stores nothing
+  // takes part in the barriers and shuffles on zero-filled data and stores nothing
   const bool active = d0 + cl < p.Di;
   const int64_t d = active ? d0 + cl : 0;
   const int64_t L = p.L, Di = p.Di;
-  const IO* xp = static_cast<const IO*>(p.xp);
-  const IO* zz = static_cast<const IO*>(p.z);
-  const IO* dt = static_cast<const IO*>(p.dt);
-  const IO* dyp = static_cast<const IO*>(p.dy);
-  const IO* Bp = static_cast<const IO*>(p.B) + b * L * N + j * kS;
-  const IO* Cp = static_cast<const IO*>(p.C) + b * L * N + j * kS;
+
+  // Stage tile k into slot `slot`: x' rows t0-4 .. t0+T-1, dt_raw and B rows t0 .. t0+T-1,
+  // and with `all` also z, dy and C; 16-byte units copied by all threads; rows outside
+  // [0, L) and channels past d_inner read as zeros.
+  auto stage = [&](int k, int slot, bool all) {
+    const int64_t t0 = int64_t(k) * kBwdT;
+    const uint32_t base = sb + uint32_t(slot * Sm::kSlot);
+    constexpr int kU = Sm::kRow / 16;                 // units per staged row of 32 channels
+    constexpr int kUbc = Sm::kBCRow / 16;             // units per row of B or C
+    constexpr int nx = (kBwdT + kBwdHalo) * kU;
+    constexpr int nr = kBwdT * kU;
+    constexpr int nbc = kBwdT * kUbc;
+    const int nrows = all ? 3 : 1;                    // dt (, z, dy)
+    const int nbcs = all ? 2 : 1;                     // B (, C)
+    const int total = nx + nr * nrows + nbc * nbcs;
+    for (int e = tid; e < total; e += kBwdThreads) {
+      const unsigned char* src;
+      uint32_t dst;
+      bool ok;
+      if (e < nx + nr * nrows) {
+        int arr = 0, r = e;                            // arr: 0 x', 1 dt, 2 z, 3 dy
+        if (r >= nx) { r -= nx; arr = 1 + r / nr; r %= nr; }
+        const int row = r / kU, u = r % kU;
+        const int64_t t = t0 + row - (arr == 0 ? kBwdHalo : 0);
+        const int64_t ch = d0 + int64_t(u) * (16 / kEs);
+        ok = t >= 0 && t < L && ch < Di;
+        const void* g = arr == 0 ? p.xp : arr == 1 ? p.dt : arr == 2 ? p.z : p.dy;
+        src = static_cast<const unsigned char*>(g) + (ok ? ((b * L + t) * Di + ch) * kEs : 0);
+        const int off = arr == 0 ? Sm::kXOff : arr == 1 ? Sm::kDtOff : arr == 2 ? Sm::kZOff
+                                                                               : Sm::kDyOff;
+        dst = base + uint32_t(off + r * 16);
+      } else {
+        int r = e - nx - nr * nrows;
+        const int arr = r / nbc;                       // 0 B, 1 C
+        r %= nbc;
+        const int row = r / kUbc, u = r % kUbc;
+        const int64_t t = t0 + row;
+        ok = t < L;
+        const void* g = arr == 0 ? p.B : p.C;
+        src = static_cast<const unsigned char*>(g) + (ok ? (b * L + t) * N * kEs + u * 16 : 0);
+        dst = base + uint32_t((arr == 0 ? Sm::kBOff : Sm::kCOff) + r * 16);
+      }
+      cp_async16_zfill(dst, src, ok);
+    }
+    cp_async_commit_();
+  };
 
   float A[kS], A2[kS];
 #pragma unroll
@@ -149,35 +228,43 @@ bwd_kernel(const BwdParams p) {
   const float cb = p.conv_b ? __ldg(p.conv_b + d) : 0.0f;
   const float dtb = __ldg(p.dt_bias + d);
   const float Dd = __ldg(p.D + d);
-  auto X = [&](int64_t t) -> float {   // x'[b, t, d], zero before the sequence
-    return t >= 0 ? IOT<IO>::to_f(xp[(b * L + t) * Di + d]) : 0.0f;
-  };
   float* ck = p.ws_h + ((b * p.ntiles) * Di + d) * N + j * kS;   // + k * Di * N per tile
+  const uint32_t colx = uint32_t(cl * kEs);
+  const uint32_t colbc = uint32_t(j * kS * kEs);
 
   // ---- forward sweep: tile start states
   {
     float h[kS];
 #pragma unroll
     for (int s = 0; s < kS; ++s) h[s] = 0.0f;
-    float xa = 0.0f, xb = 0.0f, xc = 0.0f;
+    stage(0, 0, false);
     for (int k = 0; k < p.ntiles; ++k) {
+      if (k + 1 < p.ntiles) stage(k + 1, (k + 1) & 1, false);
+      else cp_async_commit_();
       if (active) {
 #pragma unroll
         for (int s = 0; s < kS; ++s) ck[int64_t(k) * Di * N + s] = h[s];
       }
+      cp_async_wait_<1>();
+      __syncthreads();
+      const uint32_t sl = sb + uint32_t((k & 1) * Sm::kSlot);
       const int64_t t0 = int64_t(k) * kBwdT;
-      const int64_t t1 = t0 + kBwdT < L ? t0 + kBwdT : L;
-      for (int64_t t = t0; t < t1; ++t) {
-        const float xt = X(t);
+      const int cnt = int(t0 + kBwdT < L ? kBwdT : L - t0);
+      float xa = lds_one<IO>(sl + Sm::kXOff + 1 * Sm::kRow + colx);
+      float xb = lds_one<IO>(sl + Sm::kXOff + 2 * Sm::kRow + colx);
+      float xc = lds_one<IO>(sl + Sm::kXOff + 3 * Sm::kRow + colx);
+      for (int i = 0; i < cnt; ++i) {
+        const float xt = lds_one<IO>(sl + Sm::kXOff + (i + kBwdHalo) * Sm::kRow + colx);
         const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
         xa = xb; xb = xc; xc = xt;
         const float u = M::silu(pre);
-        const float del = M::softplus(IOT<IO>::to_f(dt[(b * L + t) * Di + d]) + dtb);
+        const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
         float Bv[kS];
-        ld_io_row<kS>(Bp + t * N, Bv);
+        lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
 #pragma unroll
         for (int s = 0; s < kS; ++s) h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
       }
+      __syncthreads();   // the slot is refilled by the next iteration's stage
     }
   }
 
@@ -188,51 +275,65 @@ bwd_kernel(const BwdParams p) {
   float dp1 = 0.0f, dp2 = 0.0f, dp3 = 0.0f;          // dpre of steps t+1, t+2, t+3
   float aD = 0.0f, aDtb = 0.0f, aCb = 0.0f, aW0 = 0.0f, aW1 = 0.0f, aW2 = 0.0f, aW3 = 0.0f;
   for (int i = tid; i < 2 * kBwdT * N; i += kBwdThreads) acc[i] = 0.0f;
-  __syncthreads();
+  __syncthreads();   // also orders this thread's checkpoint stores before its reloads
 
-  for (int k = p.ntiles - 1; k >= 0; --k) {
-    const int64_t t0 = int64_t(k) * kBwdT;
-    const int cnt = int(t0 + kBwdT < L ? kBwdT : L - t0);
-    // recompute the tile: h_t, {pre, u, Delta, v}, x'_t
+  float hn[kS];   // start state of the tile processed next (loaded one tile ahead)
+#pragma unroll
+  for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(p.ntiles - 1) * Di * N + s];
+  stage(p.ntiles - 1, 0, true);
+  for (int k = p.ntiles - 1, it = 0; k >= 0; --k, ++it) {
+    if (k >= 1) stage(k - 1, (it + 1) & 1, true);
+    else cp_async_commit_();
     float h0[kS], h[kS];
 #pragma unroll
-    for (int s = 0; s < kS; ++s) h0[s] = h[s] = ck[int64_t(k) * Di * N + s];
-    float xa = X(t0 - 3), xb = X(t0 - 2), xc = X(t0 - 1);
-    const float xm3 = xa, xm2 = xb, xm1 = xc;        // x' before the tile, for dconv_w
-    for (int i = 0; i < cnt; ++i) {
-      const int64_t t = t0 + i;
-      const float xt = X(t);
-      const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
-      xa = xb; xb = xc; xc = xt;
-      const float u = M::silu(pre);
-      const float v = IOT<IO>::to_f(dt[(b * L + t) * Di + d]) + dtb;
-      const float del = M::softplus(v);
-      float Bv[kS];
-      ld_io_row<kS>(Bp + t * N, Bv);
+    for (int s = 0; s < kS; ++s) h0[s] = h[s] = hn[s];
+    if (k >= 1) {
 #pragma unroll
-      for (int s = 0; s < kS; ++s) {
-        h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
-        hs[(i * kBwdThreads + tid) * kS + s] = h[s];
-      }
-      if (j == 0) {
-        sc[i * kBwdCh + cl] = make_float4(pre, u, del, v);
-        xs[i * kBwdCh + cl] = xt;
+      for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(k - 1) * Di * N + s];
+    }
+    cp_async_wait_<1>();
+    __syncthreads();
+    const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
+    const int64_t t0 = int64_t(k) * kBwdT;
+    const int cnt = int(t0 + kBwdT < L ? kBwdT : L - t0);
+    auto xrow = [&](int i) {   // x' of step t0 + i, i >= -4 (the halo rows)
+      return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
+    };
+
+    // recompute the tile: h_t and {pre, u, Delta, v}
+    {
+      float xa = xrow(-3), xb = xrow(-2), xc = xrow(-1);
+      for (int i = 0; i < cnt; ++i) {
+        const float xt = xrow(i);
+        const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+        xa = xb; xb = xc; xc = xt;
+        const float u = M::silu(pre);
+        const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
+        const float del = M::softplus(v);
+        float Bv[kS];
+        lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
+#pragma unroll
+        for (int s = 0; s < kS; ++s) {
+          h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
+          hs[(i * kBwdThreads + tid) * kS + s] = h[s];
+        }
+        if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, u, del, v);
       }
     }
     __syncwarp();
 
+#pragma unroll 2
     for (int i = cnt - 1; i >= 0; --i) {
       const int64_t t = t0 + i;
       const float4 q = sc[i * kBwdCh + cl];
       const float pre = q.x, u = q.y, del = q.z, v = q.w;
-      const int64_t o = (b * L + t) * Di + d;
-      const float zt = IOT<IO>::to_f(zz[o]);
-      const float dyt = IOT<IO>::to_f(dyp[o]);
+      const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
+      const float dyt = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx);
       const float sz = sigmoid_<kPrecise>(zt);
       const float dyc = dyt * zt * sz;
       float Bv[kS], Cv[kS], hp[kS], ht[kS];
-      ld_io_row<kS>(Bp + t * N, Bv);
-      ld_io_row<kS>(Cp + t * N, Cv);
+      lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
+      lds_io_row<kS, IO>(sl + Sm::kCOff + i * Sm::kBCRow + colbc, Cv);
       float ycp = 0.0f, duP = 0.0f, ddP = 0.0f, cB[kS], cC[kS];
 #pragma unroll
       for (int s = 0; s < kS; ++s) {
@@ -256,39 +357,49 @@ bwd_kernel(const BwdParams p) {
         duP += __shfl_xor_sync(0xffffffffu, duP, m);
         ddP += __shfl_xor_sync(0xffffffffu, ddP, m);
       }
-      // dB, dC summed over the warp's 8 channels (lane bits 0..2)
+      // dB, dC summed over the warp's 8 channels (lane bits 0..2) by a reduce-scatter:
+      // the 2*kS values {cB, cC} are halved at each round, so lane chl ends with value chl
+      // (kS = 4) or, after a last all-reduce round, value chl >> 1 (kS = 2)
+      {
+        float vv[2 * kS];
 #pragma unroll
-      for (int m = 1; m <= 4; m <<= 1) {
+        for (int s = 0; s < kS; ++s) { vv[s] = cB[s]; vv[kS + s] = cC[s]; }
+        int m = 4;
 #pragma unroll
-        for (int s = 0; s < kS; ++s) {
-          cB[s] += __shfl_xor_sync(0xffffffffu, cB[s], m);
-          cC[s] += __shfl_xor_sync(0xffffffffu, cC[s], m);
+        for (int half = kS; half >= 1; half >>= 1, m >>= 1) {
+          const bool hi = (chl & m) != 0;
+#pragma unroll
+          for (int e = 0; e < half; ++e) {
+            const float keep = hi ? vv[half + e] : vv[e];
+            const float send = hi ? vv[e] : vv[half + e];
+            vv[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+          }
         }
-      }
-      if (chl == 0 && active) {
-#pragma unroll
-        for (int s = 0; s < kS; ++s) {
-          atomicAdd(&acc[i * N + j * kS + s], cB[s]);
-          atomicAdd(&acc[(kBwdT + i) * N + j * kS + s], cC[s]);
+        int idx = chl;                                   // kS = 4: 3 rounds, one value each
+        if constexpr (kS == 2) {
+          vv[0] += __shfl_xor_sync(0xffffffffu, vv[0], 1);
+          idx = chl >> 1;
+        }
+        if (active && (kS == 4 || (chl & 1) == 0)) {
+          const int which = idx / kS, s = idx % kS;     // 0: dB, 1: dC
+          atomicAdd(&acc[(which * kBwdT + i) * N + j * kS + s], vv[0]);
         }
       }
       const float yc = ycp + Dd * u;
       const float du = duP + dyc * Dd;
       const float dv = ddP * sigmoid_<kPrecise>(v);
       const float dpre = du * silu_grad<kPrecise>(pre);
-      // x' of steps t-3..t for the weight gradient
-      const float x0 = xs[i * kBwdCh + cl];
-      const float x1 = i >= 1 ? xs[(i - 1) * kBwdCh + cl] : xm1;
-      const float x2 = i >= 2 ? xs[(i - 2) * kBwdCh + cl] : (i == 1 ? xm1 : xm2);
-      const float x3 = i >= 3 ? xs[(i - 3) * kBwdCh + cl] : (i == 2 ? xm1 : (i == 1 ? xm2 : xm3));
-      aW3 += dpre * x0; aW2 += dpre * x1; aW1 += dpre * x2; aW0 += dpre * x3;
+      // x' of steps t .. t-3 (the halo rows hold the steps before the tile, zeros before 0)
+      aW3 += dpre * xrow(i); aW2 += dpre * xrow(i - 1);
+      aW1 += dpre * xrow(i - 2); aW0 += dpre * xrow(i - 3);
       aCb += dpre;
       aDtb += dv;
       aD += dyc * u;
       const float dx = w3 * dpre + w2 * dp1 + w1 * dp2 + w0 * dp3;
       dp3 = dp2; dp2 = dp1; dp1 = dpre;
       if (j == 0 && active) {
-        p.dz[o] = dyt * yc * silu_grad<kPrecise>(zt);
+        const int64_t o = (b * L + t) * Di + d;
+        p.dz[o] = dyt * yc * (sz * (1.0f + zt * (1.0f - sz)));
         p.ddt[o] = dv;
         p.dxp[o] = dx;
       }
@@ -305,6 +416,7 @@ bwd_kernel(const BwdParams p) {
     }
     __syncthreads();
   }
+  cp_async_wait_<0>();
 
   if (!active) return;
 #pragma unroll

@@ -227,7 +227,7 @@ cudaError_t launch_fwd_any(const FwdMaps& m, const mm::FwdArgs<kExt>& a, const m
 
 template <int N, typename IO, bool P>
 cudaError_t launch_bwd(const mm::BwdParams& a, int64_t batch, cudaStream_t st) {
-  constexpr int smem = mm::BwdSmem<N>::kTotal;
+  constexpr int smem = mm::BwdSmem<N, IO>::kTotal;
   auto kern = mm::bwd_kernel<N, IO, P>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -212,7 +212,7 @@ def _bwd(lib, dims, ptrs=None, ws=None, ws_bytes=0):
 def test_backward_validation(lib):
     d = M.make_dims(2, 64, 128, 16)
     need = lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(d))
-    assert need == 256 + 2 * 2 * 128 * 16 * 4            # header + two 32-step tile states
+    assert need == 256 + 2 * 4 * 128 * 16 * 4            # header + four 16-step tile states
     ws = _fake(0x10000000 + 30 * (1 << 36))
     assert _bwd(lib, d, ws=None) == 4                       # workspace required
     assert _bwd(lib, d, ws=ws, ws_bytes=need - 16) == 4
