@@ -520,6 +520,38 @@ def run_bwd(args, w: I.Workload, local_rank: int):
     }
 
 
+def oracle_sample_bwd(w: I.Workload, target_s: float):
+    """The fp64 backward oracle on a bounded sample of the workload: all batch rows, a
+    subset of channels, the full sequence (dB/dC then sum over the sample's channels only,
+    which costs the same per channel).  Returns (GB/s of backward bytes, cores, description)."""
+    from oracle import mixer_oracle as O
+    O.build()
+    inp = I.make_inputs(w)
+    Bt, L, Di = w.batch, w.seqlen, w.d_inner
+    dy = np.random.default_rng(w.seed + 31).standard_normal((Bt, L, Di)).astype(np.float32)
+    inp["dy"] = I.f32_to_bf16_bits(dy) if w.io_dtype == I.BF16 else dy
+    f = I.as_f64
+
+    def run(chans):
+        O.mixer_bwd(f(inp["xp"][:, :, chans]), f(inp["z"][:, :, chans]),
+                    f(inp["dt_raw"][:, :, chans]), f(inp["B"]), f(inp["C"]), inp["A_log"][chans],
+                    inp["D"][chans], inp["conv_w"][chans], inp["conv_b"][chans],
+                    inp["dt_bias"][chans], f(inp["dy"][:, :, chans]), nthreads=0)
+
+    probe = np.arange(min(Di, 4))
+    t0 = time.perf_counter()
+    run(probe)
+    dt = max(time.perf_counter() - t0, 1e-4)
+    nch = int(min(Di, max(4, len(probe) * target_s / dt)))
+    chans = np.linspace(0, Di - 1, nch).astype(np.int64)
+    t0 = time.perf_counter()
+    run(chans)
+    el = time.perf_counter() - t0
+    gbs = Bt * L * nch * (bwd_bytes(w) / (Bt * L * Di)) / el / 1e9
+    return gbs, O.max_threads(), (f"{w.name} backward: all {Bt} batch rows x {nch} of {Di} channels "
+                                  f"x L={L} (fp64 oracle, {el:.2f} s)")
+
+
 # ----------------------------------------------------------------------------- oracle
 def oracle_sample(w: I.Workload, target_s: float):
     """Times the CPU oracle, as it stands, on a bounded sample of the workload: all batch
@@ -610,7 +642,12 @@ def main():
     if args.pass_ == "bwd":
         if w.decode or w.packed_mean:
             ap.error("--pass bwd needs a plain forward workload")
-        print(json.dumps(run_bwd(args, w, local_rank)), flush=True)
+        res = run_bwd(args, w, local_rank)
+        if not args.no_cpu_baseline:
+            gbs, cores, desc = oracle_sample_bwd(w, 10.0)
+            res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                   "kind": "oracle", "sample": desc}
+        print(json.dumps(res), flush=True)
         return
 
     if world > 1:

@@ -12,7 +12,8 @@
 //   forward  -- the recurrence from zero, storing the state at the start of every 16-step
 //               tile (workspace, fp32 [batch, tiles, d_inner, d_state]);
 //   reverse  -- tiles last to first: reload the tile's start state, recompute its 16
-//               states h_t and per-(t, d) scalars into shared memory, then walk the tile
+//               states h_t and per-(t, d) scalars (pre-activations and their sigmoids)
+//               into shared memory, then walk the tile
 //               backwards with the adjoint state lam (lam += dyc*C; gradients; lam *= a).
 // Each tile's inputs are staged in shared memory one tile ahead (16-byte cp.async by all
 // threads, two slots).  The conv's input gradient needs dpre of the 3 following steps,
@@ -77,7 +78,7 @@ struct BwdSmem {
   static constexpr int kCOff = kBOff + kBwdT * kBCRow;
   static constexpr int kSlot = kCOff + kBwdT * kBCRow;
   static constexpr int kHs = kBwdT * kBwdThreads * kS * 4;   // h_t per (step, lane)
-  static constexpr int kSc = kBwdT * kBwdCh * 16;            // {pre, u, Delta, v} per (step, ch)
+  static constexpr int kSc = kBwdT * kBwdCh * 16;            // {pre, s(pre), Delta, s(v)} per (step, ch)
   static constexpr int kAcc = 2 * kBwdT * N * 4;              // dB, dC partial sums per tile
   static constexpr int kHsOff = 2 * kSlot;
   static constexpr int kScOff = kHsOff + kHs;
@@ -134,13 +135,6 @@ template <bool kPrecise>
 __device__ __forceinline__ float sigmoid_(float v) {
   if constexpr (kPrecise) return 1.0f / (1.0f + expf(-v));
   else return rcp_approx(1.0f + ex2_approx(-v * kLog2e));
-}
-
-// SiLU'(v) = s (1 + v (1 - s)), s = sigmoid(v)
-template <bool kPrecise>
-__device__ __forceinline__ float silu_grad(float v) {
-  const float s = sigmoid_<kPrecise>(v);
-  return s * (1.0f + v * (1.0f - s));
 }
 
 template <int N, typename IO, bool kPrecise>
@@ -253,6 +247,7 @@ bwd_kernel(const BwdParams p) {
       float xa = lds_one<IO>(sl + Sm::kXOff + 1 * Sm::kRow + colx);
       float xb = lds_one<IO>(sl + Sm::kXOff + 2 * Sm::kRow + colx);
       float xc = lds_one<IO>(sl + Sm::kXOff + 3 * Sm::kRow + colx);
+#pragma unroll 2
       for (int i = 0; i < cnt; ++i) {
         const float xt = lds_one<IO>(sl + Sm::kXOff + (i + kBwdHalo) * Sm::kRow + colx);
         const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
@@ -303,11 +298,13 @@ bwd_kernel(const BwdParams p) {
     // recompute the tile: h_t and {pre, u, Delta, v}
     {
       float xa = xrow(-3), xb = xrow(-2), xc = xrow(-1);
+#pragma unroll 2
       for (int i = 0; i < cnt; ++i) {
         const float xt = xrow(i);
         const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
         xa = xb; xb = xc; xc = xt;
-        const float u = M::silu(pre);
+        const float sp = sigmoid_<kPrecise>(pre);
+        const float u = pre * sp;
         const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
         const float del = M::softplus(v);
         float Bv[kS];
@@ -317,7 +314,7 @@ bwd_kernel(const BwdParams p) {
           h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
           hs[(i * kBwdThreads + tid) * kS + s] = h[s];
         }
-        if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, u, del, v);
+        if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, sp, del, sigmoid_<kPrecise>(v));
       }
     }
     __syncwarp();
@@ -326,7 +323,8 @@ bwd_kernel(const BwdParams p) {
     for (int i = cnt - 1; i >= 0; --i) {
       const int64_t t = t0 + i;
       const float4 q = sc[i * kBwdCh + cl];
-      const float pre = q.x, u = q.y, del = q.z, v = q.w;
+      const float pre = q.x, sp = q.y, del = q.z, sv = q.w;   // sp, sv: sigmoid(pre), sigmoid(v)
+      const float u = pre * sp;
       const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
       const float dyt = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx);
       const float sz = sigmoid_<kPrecise>(zt);
@@ -387,8 +385,8 @@ bwd_kernel(const BwdParams p) {
       }
       const float yc = ycp + Dd * u;
       const float du = duP + dyc * Dd;
-      const float dv = ddP * sigmoid_<kPrecise>(v);
-      const float dpre = du * silu_grad<kPrecise>(pre);
+      const float dv = ddP * sv;                              // softplus' = sigmoid
+      const float dpre = du * (sp * (1.0f + pre * (1.0f - sp)));   // SiLU'(pre)
       // x' of steps t .. t-3 (the halo rows hold the steps before the tile, zeros before 0)
       aW3 += dpre * xrow(i); aW2 += dpre * xrow(i - 1);
       aW1 += dpre * xrow(i - 2); aW0 += dpre * xrow(i - 3);
