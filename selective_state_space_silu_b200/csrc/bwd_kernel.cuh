@@ -22,6 +22,14 @@
 // summed over the 8 channels of a warp by butterflies, over the 4 warps in shared memory,
 // and over CTAs (channel tiles) with global atomics; the per-d gradients are summed over
 // batch rows with global atomics.  The gradient outputs must be zero on entry.
+//
+// Time chunks (long rows with few channel tiles): chunk c starts its forward sweep from the
+// state carried through chunks 0..c-1 (the forward's chunk-state pass gives each chunk's
+// decay product P and end state H from zero: h = P*h + H) and its reverse walk from the
+// adjoint carried back from chunks c+1..C-1, composed the same way from each chunk's P and
+// its adjoint carried out from zero (Lambda, written by this kernel's kAdj instance).  The
+// input gradient of a chunk's last 3 steps also takes dpre of the next chunk's first 3: both
+// chunks add their parts atomically into those (zeroed) rows.
 #pragma once
 
 #include <float.h>
@@ -55,7 +63,13 @@ struct BwdParams {
   float* ddt_bias;
   float* ws_h;           // [batch, tiles, d_inner, N] tile start states
   int64_t L, Di;
-  int ntiles;
+  int ntiles;            // 16-step tiles over the whole sequence
+  // time chunks (as the forward's plan; chunk_len a multiple of the tile length)
+  int64_t chunk_len;
+  int nchunks;
+  const float* ws_P;     // [batch, nchunks-1, d_inner, N] decay product of each chunk
+  const float* ws_H;     // [batch, nchunks-1, d_inner, N] end state of each chunk from zero
+  float* ws_L;           // [batch, nchunks, d_inner, N] adjoint carried out of each chunk from zero
 };
 
 constexpr int kBwdThreads = 128;
@@ -111,6 +125,25 @@ __device__ __forceinline__ void lds_io_row(uint32_t a, float* out) {
   }
 }
 
+// A lane's kS fp32 states at shared address a (16- or 8-byte aligned): one vector access.
+template <int kS>
+__device__ __forceinline__ void sts_states(uint32_t a, const float* v) {
+  if constexpr (kS == 4)
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(a), "f"(v[0]), "f"(v[1]),
+                 "f"(v[2]), "f"(v[3]) : "memory");
+  else
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(v[0]), "f"(v[1]) : "memory");
+}
+template <int kS>
+__device__ __forceinline__ void lds_states(uint32_t a, float* v) {
+  if constexpr (kS == 4) {
+    const float4 x = lds_f32x4(a);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+  } else {
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v[0]), "=f"(v[1]) : "r"(a));
+  }
+}
+
 template <typename IO>
 __device__ __forceinline__ float lds_one(uint32_t a) {
   if constexpr (sizeof(IO) == 4) return lds_f32(a);
@@ -137,7 +170,7 @@ __device__ __forceinline__ float sigmoid_(float v) {
   else return rcp_approx(1.0f + ex2_approx(-v * kLog2e));
 }
 
-template <int N, typename IO, bool kPrecise>
+template <int N, typename IO, bool kPrecise, bool kAdj>
 __global__ void __launch_bounds__(kBwdThreads)
 bwd_kernel(const BwdParams p) {
   using M = Math<kPrecise>;
@@ -146,7 +179,7 @@ bwd_kernel(const BwdParams p) {
   constexpr int kEs = Sm::kEs;
   extern __shared__ __align__(16) unsigned char smem[];
   const uint32_t sb = smem_addr(smem);
-  float* hs = reinterpret_cast<float*>(smem + Sm::kHsOff);
+  const uint32_t hsa = sb + uint32_t(Sm::kHsOff) + uint32_t(threadIdx.x * (N / 4) * 4);  // this lane's h_t slots
   float4* sc = reinterpret_cast<float4*>(smem + Sm::kScOff);
   float* acc = reinterpret_cast<float*>(smem + Sm::kAccOff);   // [2][T][N]
 
@@ -163,6 +196,12 @@ bwd_kernel(const BwdParams p) {
   const bool active = d0 + cl < p.Di;
   const int64_t d = active ? d0 + cl : 0;
   const int64_t L = p.L, Di = p.Di;
+  // this CTA's time chunk (the kAdj instance runs chunks 1..C-1)
+  const int c = kAdj ? int(blockIdx.z) + 1 : int(blockIdx.z);
+  const int64_t t_begin = int64_t(c) * p.chunk_len;
+  const int64_t t_end = t_begin + p.chunk_len < L ? t_begin + p.chunk_len : L;
+  const int kb = int(t_begin / kBwdT);                        // first and one-past-last tile
+  const int ke = int((t_end + kBwdT - 1) / kBwdT);
 
   // Stage tile k into slot `slot`: x' rows t0-4 .. t0+T-1, dt_raw and B rows t0 .. t0+T-1,
   // and with `all` also z, dy and C; 16-byte units copied by all threads; rows outside
@@ -226,208 +265,274 @@ bwd_kernel(const BwdParams p) {
   const uint32_t colx = uint32_t(cl * kEs);
   const uint32_t colbc = uint32_t(j * kS * kEs);
 
-  // ---- forward sweep: tile start states
-  {
-    float h[kS];
+  if constexpr (kAdj) {
+    // ---- adjoint carried out of chunk c from zero: lam += dyc*C; lam *= a, last step first
+    float lam[kS];
 #pragma unroll
-    for (int s = 0; s < kS; ++s) h[s] = 0.0f;
-    stage(0, 0, false);
-    for (int k = 0; k < p.ntiles; ++k) {
-      if (k + 1 < p.ntiles) stage(k + 1, (k + 1) & 1, false);
+    for (int s = 0; s < kS; ++s) lam[s] = 0.0f;
+    stage(ke - 1, 0, true);
+    for (int k = ke - 1, it = 0; k >= kb; --k, ++it) {
+      if (k - 1 >= kb) stage(k - 1, (it + 1) & 1, true);
       else cp_async_commit_();
-      if (active) {
+      cp_async_wait_<1>();
+      __syncthreads();
+      const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
+      const int64_t t0 = int64_t(k) * kBwdT;
+      const int cnt = int(t0 + kBwdT < t_end ? kBwdT : t_end - t0);
+#pragma unroll 2
+      for (int i = cnt - 1; i >= 0; --i) {
+        const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
+        const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
+        const float dyc = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx) * zt * sigmoid_<kPrecise>(zt);
+        float Cv[kS];
+        lds_io_row<kS, IO>(sl + Sm::kCOff + i * Sm::kBCRow + colbc, Cv);
 #pragma unroll
-        for (int s = 0; s < kS; ++s) ck[int64_t(k) * Di * N + s] = h[s];
+        for (int s = 0; s < kS; ++s) lam[s] = (lam[s] + dyc * Cv[s]) * M::decay(del, A2[s]);
+      }
+      __syncthreads();
+    }
+    cp_async_wait_<0>();
+    if (active) {
+      float* o = p.ws_L + ((b * p.nchunks + c) * Di + d) * N + j * kS;
+#pragma unroll
+      for (int s = 0; s < kS; ++s) o[s] = lam[s];
+    }
+  } else {
+    // ---- forward sweep: tile start states, from the state carried into this chunk
+    {
+      float h[kS];
+  #pragma unroll
+      for (int s = 0; s < kS; ++s) h[s] = 0.0f;
+      for (int cc = 0; cc < c; ++cc) {
+        const int64_t o = ((b * (p.nchunks - 1) + cc) * Di + d) * N + j * kS;
+  #pragma unroll
+        for (int s = 0; s < kS; ++s) h[s] = p.ws_P[o + s] * h[s] + p.ws_H[o + s];
+      }
+      stage(kb, 0, false);
+      for (int k = kb, it = 0; k < ke; ++k, ++it) {
+        if (k + 1 < ke) stage(k + 1, (it + 1) & 1, false);
+        else cp_async_commit_();
+        if (active) {
+  #pragma unroll
+          for (int s = 0; s < kS; ++s) ck[int64_t(k) * Di * N + s] = h[s];
+        }
+        cp_async_wait_<1>();
+        __syncthreads();
+        const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
+        const int64_t t0 = int64_t(k) * kBwdT;
+        const int cnt = int(t0 + kBwdT < t_end ? kBwdT : t_end - t0);
+        float xa = lds_one<IO>(sl + Sm::kXOff + 1 * Sm::kRow + colx);
+        float xb = lds_one<IO>(sl + Sm::kXOff + 2 * Sm::kRow + colx);
+        float xc = lds_one<IO>(sl + Sm::kXOff + 3 * Sm::kRow + colx);
+  #pragma unroll 2
+        for (int i = 0; i < cnt; ++i) {
+          const float xt = lds_one<IO>(sl + Sm::kXOff + (i + kBwdHalo) * Sm::kRow + colx);
+          const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          xa = xb; xb = xc; xc = xt;
+          const float u = M::silu(pre);
+          const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
+          float Bv[kS];
+          lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
+  #pragma unroll
+          for (int s = 0; s < kS; ++s) h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
+        }
+        __syncthreads();   // the slot is refilled by the next iteration's stage
+      }
+    }
+
+    // ---- reverse sweep
+    float lam[kS], dA[kS];
+  #pragma unroll
+    for (int s = 0; s < kS; ++s) { lam[s] = 0.0f; dA[s] = 0.0f; }
+    // the adjoint carried back into this chunk: lam = P_c' * lam + Lambda_c', c' = C-1 .. c+1
+    for (int cc = p.nchunks - 1; cc > c; --cc) {
+      const int64_t oL = ((b * p.nchunks + cc) * Di + d) * N + j * kS;
+      const int64_t oP = ((b * (p.nchunks - 1) + cc) * Di + d) * N + j * kS;
+  #pragma unroll
+      for (int s = 0; s < kS; ++s)
+        lam[s] = (cc < p.nchunks - 1 ? p.ws_P[oP + s] * lam[s] : 0.0f) + p.ws_L[oL + s];
+    }
+    float dp1 = 0.0f, dp2 = 0.0f, dp3 = 0.0f;          // dpre of steps t+1, t+2, t+3
+    float aD = 0.0f, aDtb = 0.0f, aCb = 0.0f, aW0 = 0.0f, aW1 = 0.0f, aW2 = 0.0f, aW3 = 0.0f;
+    for (int i = tid; i < 2 * kBwdT * N; i += kBwdThreads) acc[i] = 0.0f;
+    __syncthreads();   // also orders this thread's checkpoint stores before its reloads
+
+    float hn[kS];   // start state of the tile processed next (loaded one tile ahead)
+  #pragma unroll
+    for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(ke - 1) * Di * N + s];
+    stage(ke - 1, 0, true);
+    for (int k = ke - 1, it = 0; k >= kb; --k, ++it) {
+      if (k - 1 >= kb) stage(k - 1, (it + 1) & 1, true);
+      else cp_async_commit_();
+      float h0[kS], h[kS];
+  #pragma unroll
+      for (int s = 0; s < kS; ++s) h0[s] = h[s] = hn[s];
+      if (k - 1 >= kb) {
+  #pragma unroll
+        for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(k - 1) * Di * N + s];
       }
       cp_async_wait_<1>();
       __syncthreads();
-      const uint32_t sl = sb + uint32_t((k & 1) * Sm::kSlot);
+      const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
       const int64_t t0 = int64_t(k) * kBwdT;
-      const int cnt = int(t0 + kBwdT < L ? kBwdT : L - t0);
-      float xa = lds_one<IO>(sl + Sm::kXOff + 1 * Sm::kRow + colx);
-      float xb = lds_one<IO>(sl + Sm::kXOff + 2 * Sm::kRow + colx);
-      float xc = lds_one<IO>(sl + Sm::kXOff + 3 * Sm::kRow + colx);
-#pragma unroll 2
-      for (int i = 0; i < cnt; ++i) {
-        const float xt = lds_one<IO>(sl + Sm::kXOff + (i + kBwdHalo) * Sm::kRow + colx);
-        const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
-        xa = xb; xb = xc; xc = xt;
-        const float u = M::silu(pre);
-        const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
-        float Bv[kS];
-        lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-#pragma unroll
-        for (int s = 0; s < kS; ++s) h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
-      }
-      __syncthreads();   // the slot is refilled by the next iteration's stage
-    }
-  }
+      const int cnt = int(t0 + kBwdT < t_end ? kBwdT : t_end - t0);
+      auto xrow = [&](int i) {   // x' of step t0 + i, i >= -4 (the halo rows)
+        return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
+      };
 
-  // ---- reverse sweep
-  float lam[kS], dA[kS];
-#pragma unroll
-  for (int s = 0; s < kS; ++s) { lam[s] = 0.0f; dA[s] = 0.0f; }
-  float dp1 = 0.0f, dp2 = 0.0f, dp3 = 0.0f;          // dpre of steps t+1, t+2, t+3
-  float aD = 0.0f, aDtb = 0.0f, aCb = 0.0f, aW0 = 0.0f, aW1 = 0.0f, aW2 = 0.0f, aW3 = 0.0f;
-  for (int i = tid; i < 2 * kBwdT * N; i += kBwdThreads) acc[i] = 0.0f;
-  __syncthreads();   // also orders this thread's checkpoint stores before its reloads
-
-  float hn[kS];   // start state of the tile processed next (loaded one tile ahead)
-#pragma unroll
-  for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(p.ntiles - 1) * Di * N + s];
-  stage(p.ntiles - 1, 0, true);
-  for (int k = p.ntiles - 1, it = 0; k >= 0; --k, ++it) {
-    if (k >= 1) stage(k - 1, (it + 1) & 1, true);
-    else cp_async_commit_();
-    float h0[kS], h[kS];
-#pragma unroll
-    for (int s = 0; s < kS; ++s) h0[s] = h[s] = hn[s];
-    if (k >= 1) {
-#pragma unroll
-      for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(k - 1) * Di * N + s];
-    }
-    cp_async_wait_<1>();
-    __syncthreads();
-    const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
-    const int64_t t0 = int64_t(k) * kBwdT;
-    const int cnt = int(t0 + kBwdT < L ? kBwdT : L - t0);
-    auto xrow = [&](int i) {   // x' of step t0 + i, i >= -4 (the halo rows)
-      return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
-    };
-
-    // recompute the tile: h_t and {pre, u, Delta, v}
-    {
-      float xa = xrow(-3), xb = xrow(-2), xc = xrow(-1);
-#pragma unroll 2
-      for (int i = 0; i < cnt; ++i) {
-        const float xt = xrow(i);
-        const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
-        xa = xb; xb = xc; xc = xt;
-        const float sp = sigmoid_<kPrecise>(pre);
-        const float u = pre * sp;
-        const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
-        const float del = M::softplus(v);
-        float Bv[kS];
-        lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-#pragma unroll
-        for (int s = 0; s < kS; ++s) {
-          h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
-          hs[(i * kBwdThreads + tid) * kS + s] = h[s];
-        }
-        if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, sp, del, sigmoid_<kPrecise>(v));
-      }
-    }
-    __syncwarp();
-
-#pragma unroll 2
-    for (int i = cnt - 1; i >= 0; --i) {
-      const int64_t t = t0 + i;
-      const float4 q = sc[i * kBwdCh + cl];
-      const float pre = q.x, sp = q.y, del = q.z, sv = q.w;   // sp, sv: sigmoid(pre), sigmoid(v)
-      const float u = pre * sp;
-      const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
-      const float dyt = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx);
-      const float sz = sigmoid_<kPrecise>(zt);
-      const float dyc = dyt * zt * sz;
-      float Bv[kS], Cv[kS], hp[kS], ht[kS];
-      lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-      lds_io_row<kS, IO>(sl + Sm::kCOff + i * Sm::kBCRow + colbc, Cv);
-      float ycp = 0.0f, duP = 0.0f, ddP = 0.0f, cB[kS], cC[kS];
-#pragma unroll
-      for (int s = 0; s < kS; ++s) {
-        ht[s] = hs[(i * kBwdThreads + tid) * kS + s];
-        hp[s] = i > 0 ? hs[((i - 1) * kBwdThreads + tid) * kS + s] : h0[s];
-        ycp += Cv[s] * ht[s];
-        const float a = M::decay(del, A2[s]);
-        lam[s] += dyc * Cv[s];
-        cB[s] = lam[s] * del * u;
-        cC[s] = dyc * ht[s];
-        duP += lam[s] * del * Bv[s];
-        const float ah = lam[s] * hp[s] * a;
-        ddP += lam[s] * Bv[s] * u + ah * A[s];
-        dA[s] += ah * del;
-        lam[s] *= a;
-      }
-      // channel sums over the 4 lanes of a channel (lane bits 3 and 4)
-#pragma unroll
-      for (int m = 8; m <= 16; m <<= 1) {
-        ycp += __shfl_xor_sync(0xffffffffu, ycp, m);
-        duP += __shfl_xor_sync(0xffffffffu, duP, m);
-        ddP += __shfl_xor_sync(0xffffffffu, ddP, m);
-      }
-      // dB, dC summed over the warp's 8 channels (lane bits 0..2) by a reduce-scatter:
-      // the 2*kS values {cB, cC} are halved at each round, so lane chl ends with value chl
-      // (kS = 4) or, after a last all-reduce round, value chl >> 1 (kS = 2)
+      // recompute the tile: h_t and {pre, u, Delta, v}
       {
-        float vv[2 * kS];
-#pragma unroll
-        for (int s = 0; s < kS; ++s) { vv[s] = cB[s]; vv[kS + s] = cC[s]; }
-        int m = 4;
-#pragma unroll
-        for (int half = kS; half >= 1; half >>= 1, m >>= 1) {
-          const bool hi = (chl & m) != 0;
-#pragma unroll
-          for (int e = 0; e < half; ++e) {
-            const float keep = hi ? vv[half + e] : vv[e];
-            const float send = hi ? vv[e] : vv[half + e];
-            vv[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        float xa = xrow(-3), xb = xrow(-2), xc = xrow(-1);
+  #pragma unroll 2
+        for (int i = 0; i < cnt; ++i) {
+          const float xt = xrow(i);
+          const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          xa = xb; xb = xc; xc = xt;
+          const float sp = sigmoid_<kPrecise>(pre);
+          const float u = pre * sp;
+          const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
+          const float del = M::softplus(v);
+          float Bv[kS];
+          lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
+  #pragma unroll
+          for (int s = 0; s < kS; ++s) h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
+          sts_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), h);
+          if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, sp, del, sigmoid_<kPrecise>(v));
+        }
+      }
+      __syncwarp();
+
+  #pragma unroll 2
+      for (int i = cnt - 1; i >= 0; --i) {
+        const int64_t t = t0 + i;
+        const float4 q = sc[i * kBwdCh + cl];
+        const float pre = q.x, sp = q.y, del = q.z, sv = q.w;   // sp, sv: sigmoid(pre), sigmoid(v)
+        const float u = pre * sp;
+        const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
+        const float dyt = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx);
+        const float sz = sigmoid_<kPrecise>(zt);
+        const float dyc = dyt * zt * sz;
+        float Bv[kS], Cv[kS], hp[kS], ht[kS];
+        lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
+        lds_io_row<kS, IO>(sl + Sm::kCOff + i * Sm::kBCRow + colbc, Cv);
+        float ycp = 0.0f, duP = 0.0f, ddP = 0.0f, cB[kS], cC[kS];
+        lds_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), ht);
+        if (i > 0) {
+          lds_states<kS>(hsa + uint32_t((i - 1) * kBwdThreads * kS * 4), hp);
+        } else {
+  #pragma unroll
+          for (int s = 0; s < kS; ++s) hp[s] = h0[s];
+        }
+  #pragma unroll
+        for (int s = 0; s < kS; ++s) {
+          ycp += Cv[s] * ht[s];
+          const float a = M::decay(del, A2[s]);
+          lam[s] += dyc * Cv[s];
+          cB[s] = lam[s] * del * u;
+          cC[s] = dyc * ht[s];
+          duP += lam[s] * del * Bv[s];
+          const float ah = lam[s] * hp[s] * a;
+          ddP += lam[s] * Bv[s] * u + ah * A[s];
+          dA[s] += ah * del;
+          lam[s] *= a;
+        }
+        // channel sums over the 4 lanes of a channel (lane bits 3 and 4)
+  #pragma unroll
+        for (int m = 8; m <= 16; m <<= 1) {
+          ycp += __shfl_xor_sync(0xffffffffu, ycp, m);
+          duP += __shfl_xor_sync(0xffffffffu, duP, m);
+          ddP += __shfl_xor_sync(0xffffffffu, ddP, m);
+        }
+        // dB, dC summed over the warp's 8 channels (lane bits 0..2) by a reduce-scatter:
+        // the 2*kS values {cB, cC} are halved at each round, so lane chl ends with value chl
+        // (kS = 4) or, after a last all-reduce round, value chl >> 1 (kS = 2)
+        {
+          float vv[2 * kS];
+  #pragma unroll
+          for (int s = 0; s < kS; ++s) { vv[s] = cB[s]; vv[kS + s] = cC[s]; }
+          int m = 4;
+  #pragma unroll
+          for (int half = kS; half >= 1; half >>= 1, m >>= 1) {
+            const bool hi = (chl & m) != 0;
+  #pragma unroll
+            for (int e = 0; e < half; ++e) {
+              const float keep = hi ? vv[half + e] : vv[e];
+              const float send = hi ? vv[e] : vv[half + e];
+              vv[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+            }
+          }
+          int idx = chl;                                   // kS = 4: 3 rounds, one value each
+          if constexpr (kS == 2) {
+            vv[0] += __shfl_xor_sync(0xffffffffu, vv[0], 1);
+            idx = chl >> 1;
+          }
+          if (active && (kS == 4 || (chl & 1) == 0)) {
+            const int which = idx / kS, s = idx % kS;     // 0: dB, 1: dC
+            atomicAdd(&acc[(which * kBwdT + i) * N + j * kS + s], vv[0]);
           }
         }
-        int idx = chl;                                   // kS = 4: 3 rounds, one value each
-        if constexpr (kS == 2) {
-          vv[0] += __shfl_xor_sync(0xffffffffu, vv[0], 1);
-          idx = chl >> 1;
+        const float yc = ycp + Dd * u;
+        const float du = duP + dyc * Dd;
+        const float dv = ddP * sv;                              // softplus' = sigmoid
+        const float dpre = du * (sp * (1.0f + pre * (1.0f - sp)));   // SiLU'(pre)
+        // x' of steps t .. t-3 (the halo rows hold the steps before the tile, zeros before 0)
+        aW3 += dpre * xrow(i); aW2 += dpre * xrow(i - 1);
+        aW1 += dpre * xrow(i - 2); aW0 += dpre * xrow(i - 3);
+        aCb += dpre;
+        aDtb += dv;
+        aD += dyc * u;
+        const float dx = w3 * dpre + w2 * dp1 + w1 * dp2 + w0 * dp3;
+        dp3 = dp2; dp2 = dp1; dp1 = dpre;
+        if (j == 0 && active) {
+          const int64_t o = (b * L + t) * Di + d;
+          p.dz[o] = dyt * yc * (sz * (1.0f + zt * (1.0f - sz)));
+          p.ddt[o] = dv;
+          if (c < p.nchunks - 1 && t >= t_end - 3) atomicAdd(p.dxp + o, dx);  // + next chunk's part
+          else p.dxp[o] = dx;
         }
-        if (active && (kS == 4 || (chl & 1) == 0)) {
-          const int which = idx / kS, s = idx % kS;     // 0: dB, 1: dC
-          atomicAdd(&acc[(which * kBwdT + i) * N + j * kS + s], vv[0]);
+      }
+      __syncthreads();
+      // this tile's dB, dC of the CTA's 32 channels into the global sums
+      for (int e = tid; e < 2 * kBwdT * N; e += kBwdThreads) {
+        const int which = e / (kBwdT * N), r = e % (kBwdT * N), i = r / N, n = r % N;
+        if (i < cnt) {
+          float* dst = which ? p.dC : p.dB;
+          atomicAdd(dst + (b * L + t0 + i) * N + n, acc[e]);
         }
+        acc[e] = 0.0f;
       }
-      const float yc = ycp + Dd * u;
-      const float du = duP + dyc * Dd;
-      const float dv = ddP * sv;                              // softplus' = sigmoid
-      const float dpre = du * (sp * (1.0f + pre * (1.0f - sp)));   // SiLU'(pre)
-      // x' of steps t .. t-3 (the halo rows hold the steps before the tile, zeros before 0)
-      aW3 += dpre * xrow(i); aW2 += dpre * xrow(i - 1);
-      aW1 += dpre * xrow(i - 2); aW0 += dpre * xrow(i - 3);
-      aCb += dpre;
-      aDtb += dv;
-      aD += dyc * u;
-      const float dx = w3 * dpre + w2 * dp1 + w1 * dp2 + w0 * dp3;
-      dp3 = dp2; dp2 = dp1; dp1 = dpre;
-      if (j == 0 && active) {
-        const int64_t o = (b * L + t) * Di + d;
-        p.dz[o] = dyt * yc * (sz * (1.0f + zt * (1.0f - sz)));
-        p.ddt[o] = dv;
-        p.dxp[o] = dx;
-      }
+      __syncthreads();
     }
-    __syncthreads();
-    // this tile's dB, dC of the CTA's 32 channels into the global sums
-    for (int e = tid; e < 2 * kBwdT * N; e += kBwdThreads) {
-      const int which = e / (kBwdT * N), r = e % (kBwdT * N), i = r / N, n = r % N;
-      if (i < cnt) {
-        float* dst = which ? p.dC : p.dB;
-        atomicAdd(dst + (b * L + t0 + i) * N + n, acc[e]);
-      }
-      acc[e] = 0.0f;
-    }
-    __syncthreads();
-  }
-  cp_async_wait_<0>();
+    cp_async_wait_<0>();
 
-  if (!active) return;
-#pragma unroll
-  for (int s = 0; s < kS; ++s) atomicAdd(p.dA_log + d * N + j * kS + s, dA[s] * A[s]);
-  if (j == 0) {
-    atomicAdd(p.dD + d, aD);
-    atomicAdd(p.ddt_bias + d, aDtb);
-    if (p.dconv_b) atomicAdd(p.dconv_b + d, aCb);
-    atomicAdd(p.dconv_w + d * 4 + 0, aW0);
-    atomicAdd(p.dconv_w + d * 4 + 1, aW1);
-    atomicAdd(p.dconv_w + d * 4 + 2, aW2);
-    atomicAdd(p.dconv_w + d * 4 + 3, aW3);
+    if (!active) return;
+    // this chunk's part of the input gradient of the previous chunk's last 3 steps
+    if (c > 0 && j == 0) {
+      float* o = p.dxp + (b * L + t_begin) * Di + d;
+      atomicAdd(o - Di, w2 * dp1 + w1 * dp2 + w0 * dp3);
+      atomicAdd(o - 2 * Di, w1 * dp1 + w0 * dp2);
+      atomicAdd(o - 3 * Di, w0 * dp1);
+    }
+  #pragma unroll
+    for (int s = 0; s < kS; ++s) atomicAdd(p.dA_log + d * N + j * kS + s, dA[s] * A[s]);
+    if (j == 0) {
+      atomicAdd(p.dD + d, aD);
+      atomicAdd(p.ddt_bias + d, aDtb);
+      if (p.dconv_b) atomicAdd(p.dconv_b + d, aCb);
+      atomicAdd(p.dconv_w + d * 4 + 0, aW0);
+      atomicAdd(p.dconv_w + d * 4 + 1, aW1);
+      atomicAdd(p.dconv_w + d * 4 + 2, aW2);
+      atomicAdd(p.dconv_w + d * 4 + 3, aW3);
+    }
   }
+}
+
+// Zeroes the 3 rows of dxp before every chunk start (c >= 1), which two chunks then add to.
+__global__ void bwd_zero_bounds(float* dxp, int64_t L, int64_t Di, int64_t chunk_len) {
+  const int64_t b = blockIdx.y;
+  const int64_t t0 = int64_t(blockIdx.x + 1) * chunk_len - 3;
+  float* row = dxp + (b * L + t0) * Di;
+  for (int64_t e = threadIdx.x; e < 3 * Di; e += blockDim.x) row[e] = 0.0f;
 }
 
 }  // namespace mm

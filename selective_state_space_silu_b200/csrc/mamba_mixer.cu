@@ -225,22 +225,54 @@ cudaError_t launch_fwd_any(const FwdMaps& m, const mm::FwdArgs<kExt>& a, const m
              : launch_fwd<8, __nv_bfloat16, false, kExt>(m, a, d->batch, st);
 }
 
+// The backward's kernels: with time chunks, the forward's chunk-state pass (P, H), the
+// adjoint pass (Lambda), the zeroing of the rows two chunks add to, then the main pass.
 template <int N, typename IO, bool P>
-cudaError_t launch_bwd(const mm::BwdParams& a, int64_t batch, cudaStream_t st) {
+cudaError_t launch_bwd(const FwdMaps* m, const mm::FwdParams& fp, const mm::BwdParams& a,
+                       int64_t batch, cudaStream_t st) {
   constexpr int smem = mm::BwdSmem<N, IO>::kTotal;
-  auto kern = mm::bwd_kernel<N, IO, P>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
   const unsigned gx = unsigned((a.Di + mm::kBwdCh - 1) / mm::kBwdCh);
-  kern<<<dim3(gx, unsigned(batch)), mm::kBwdThreads, smem, st>>>(a);
+  cudaError_t e;
+  if (a.nchunks > 1) {
+    mm::FwdArgs<false> pre;
+    static_cast<mm::FwdParams&>(pre) = fp;
+    e = launch_fwd_kernel<N, IO, P, true, false>(
+        *m, pre, dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), st);
+    if (e != cudaSuccess) return e;
+    auto adj = mm::bwd_kernel<N, IO, P, true>;
+    e = cudaFuncSetAttribute(adj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    adj<<<dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), mm::kBwdThreads, smem, st>>>(a);
+    mm::bwd_zero_bounds<<<dim3(unsigned(a.nchunks - 1), unsigned(batch)), 256, 0, st>>>(
+        a.dxp, a.L, a.Di, a.chunk_len);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  auto kern = mm::bwd_kernel<N, IO, P, false>;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(gx, unsigned(batch), unsigned(a.nchunks)), mm::kBwdThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-size_t bwd_workspace_for(const mamba_dims* d) {
-  const int64_t tiles = (d->seqlen + mm::kBwdT - 1) / mm::kBwdT;
-  return kWsHeader + size_t(d->batch) * size_t(tiles) * size_t(d->d_inner) * size_t(d->d_state) *
-                         sizeof(float);
+// Backward workspace: header, tile start states, and with time chunks each chunk's
+// (P, H) from the chunk-state pass and its adjoint Lambda.
+struct BwdLayout {
+  size_t states, P, H, Lam, total;   // byte offsets (total = size)
+};
+BwdLayout bwd_layout(const mamba_dims* d, const Plan& plan) {
+  const size_t per = size_t(d->batch) * size_t(d->d_inner) * size_t(d->d_state) * sizeof(float);
+  const size_t tiles = size_t((d->seqlen + mm::kBwdT - 1) / mm::kBwdT);
+  BwdLayout l;
+  l.states = kWsHeader;
+  l.P = l.states + tiles * per;
+  const size_t agg = plan.nchunks > 1 ? size_t(plan.nchunks - 1) * per : 0;
+  l.H = l.P + agg;
+  l.Lam = l.H + agg;
+  l.total = l.Lam + (plan.nchunks > 1 ? size_t(plan.nchunks) * per : 0);
+  return l;
 }
+
+size_t bwd_workspace_for(const mamba_dims* d) { return bwd_layout(d, make_plan(d)).total; }
 
 template <int N, typename IO, bool P>
 cudaError_t launch_step(const mm::StepArgs& a, cudaStream_t st) {
@@ -515,21 +547,50 @@ int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const
   if (e != cudaSuccess) return fail(MAMBA_ERR_CUDA, "gradient reset failed: %s", cudaGetErrorString(e));
   if (dims->seqlen == 0) return ok();
 
+  const Plan plan = make_plan(dims);
+  const BwdLayout lay = bwd_layout(dims, plan);
+  unsigned char* wsb = static_cast<unsigned char*>(workspace);
   mm::BwdParams a{};
   a.xp = xp; a.z = z; a.dt = dt_raw; a.B = B; a.C = C; a.dy = dy;
   a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
   a.dxp = dxp; a.dz = dz; a.ddt = ddt_raw; a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
   a.dconv_w = dconv_w; a.dconv_b = dconv_b; a.ddt_bias = ddt_bias;
-  a.ws_h = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + kWsHeader);
+  a.ws_h = reinterpret_cast<float*>(wsb + lay.states);
   a.L = dims->seqlen; a.Di = Di;
   a.ntiles = int((dims->seqlen + mm::kBwdT - 1) / mm::kBwdT);
+  a.chunk_len = plan.chunk_len;
+  a.nchunks = plan.nchunks;
+  a.ws_P = reinterpret_cast<const float*>(wsb + lay.P);
+  a.ws_H = reinterpret_cast<const float*>(wsb + lay.H);
+  a.ws_L = reinterpret_cast<float*>(wsb + lay.Lam);
   const bool f32 = dims->io_dtype == MAMBA_F32;
+  FwdMaps m;
+  mm::FwdParams fp{};
+  if (plan.nchunks > 1) {
+    // the forward's chunk-state pass over the same inputs gives each chunk's (P, H)
+    const uint64_t Bt = uint64_t(dims->batch), L = uint64_t(dims->seqlen);
+    const CUtensorMapSwizzle swz = f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const uint32_t nrow = uint32_t(mm::kTileT);
+    if (!make_map(&m.x, xp, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow + mm::kHalo, swz) ||
+        !make_map(&m.z, z, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) ||
+        !make_map(&m.dt, dt_raw, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) ||
+        !make_map(&m.B, B, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&m.C, C, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return fail(MAMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
+    fp.A_log = A_log; fp.D = D; fp.conv_w = conv_w; fp.conv_b = conv_b; fp.dt_bias = dt_bias;
+    fp.ws_P = const_cast<float*>(a.ws_P);
+    fp.ws_H = const_cast<float*>(a.ws_H);
+    fp.status = static_cast<int*>(workspace);
+    fp.L = dims->seqlen; fp.Di = Di;
+    fp.chunk_len = plan.chunk_len; fp.nchunks = plan.nchunks;
+    fp.inject_skip_tile = -1;
+  }
   if (N == 16)
-    e = f32 ? launch_bwd<16, float, true>(a, dims->batch, st)
-            : launch_bwd<16, __nv_bfloat16, false>(a, dims->batch, st);
+    e = f32 ? launch_bwd<16, float, true>(&m, fp, a, dims->batch, st)
+            : launch_bwd<16, __nv_bfloat16, false>(&m, fp, a, dims->batch, st);
   else
-    e = f32 ? launch_bwd<8, float, true>(a, dims->batch, st)
-            : launch_bwd<8, __nv_bfloat16, false>(a, dims->batch, st);
+    e = f32 ? launch_bwd<8, float, true>(&m, fp, a, dims->batch, st)
+            : launch_bwd<8, __nv_bfloat16, false>(&m, fp, a, dims->batch, st);
   if (e != cudaSuccess)
     return fail(MAMBA_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(e));
   return ok();

@@ -67,3 +67,18 @@ def test_backward_130m_two_rows(oracle):
     full, including dB/dC (sums over all 1536 channels) and the parameter gradients."""
     w, inp = _case(2, 2048, 1536, 16, I.BF16, 3100)
     _compare(_run(inp), _oracle(oracle, inp), I.BF16, "m130 rows")
+
+
+@pytest.mark.parametrize("Bt,L,Di,N,io", [
+    (1, 4096, 64, 16, I.BF16),     # 16 chunks of 256 steps
+    (2, 1500, 64, 8, I.F32),       # 5 chunks of 320 steps, the last one ragged
+    (1, 2600, 40, 16, I.F32),      # ragged channel tile and sequence
+])
+def test_backward_with_time_chunks(oracle, Bt, L, Di, N, io):
+    """Rows with few channel tiles are cut into time chunks: the state and the adjoint are
+    carried across chunk edges, and the input gradient of each chunk's last 3 steps takes
+    the next chunk's part."""
+    dims = M.make_dims(Bt, L, Di, N, 4, M.MAMBA_BF16 if io == I.BF16 else M.MAMBA_F32)
+    assert M.mamba_mixer_fwd_launches(dims) == 2      # the plan splits the sequence
+    w, inp = _case(Bt, L, Di, N, io, 3200 + L)
+    _compare(_run(inp), _oracle(oracle, inp), io, f"chunked {Bt}x{L}x{Di} N{N} {io}")
