@@ -87,11 +87,16 @@ int oracle_max_threads(void) { return 1; }
  * fp32 on the openfluke stress-test page ("Activations and boundary gradients are
  * Float32"); this oracle computes them in fp64.
  *
- * Given dy = dLoss/dy [batch, L, d_inner] for a forward from zero state (no cached
- * state, no document ids), it returns dLoss with respect to every input:
+ * Given dy = dLoss/dy [batch, L, d_inner], it returns dLoss with respect to every input:
  *   dxp, dz, ddt_raw [batch, L, d_inner]; dB, dC [batch, L, d_state];
- *   dA_log [d_inner, d_state]; dD, dconv_b, ddt_bias [d_inner]; dconv_w [d_inner, d_conv].
- * All outputs are overwritten.  dconv_b may be NULL when the forward had no conv bias.
+ *   dA_log [d_inner, d_state]; dD, dconv_b, ddt_bias [d_inner]; dconv_w [d_inner, d_conv];
+ *   and, when the forward started from a cached state (h_in, conv_state_in), dh_in
+ *   [batch, d_inner, d_state] and dconv_state_in [batch, d_inner, d_conv-1].
+ * All outputs are overwritten.  dconv_b may be NULL when the forward had no conv bias;
+ * seq_idx, h_in, conv_state_in (forward inputs) and dh_in, dconv_state_in may be NULL.
+ * With seq_idx the forward resets both states at every id change (see oracle_mixer): a
+ * conv tap lying before the step's document start is zero, so it passes no gradient; the
+ * state entering a reset step is zero, so the adjoint stops there.
  *
  * Per channel (b, d), with xpad = [0 (K-1) ; x'], pre_t = conv_b + sum_k w_k xpad[t+k],
  * u_t = SiLU(pre_t), v_t = dt_raw_t + dt_bias, Delta_t = softplus(v_t),
@@ -109,7 +114,9 @@ int oracle_max_threads(void) { return 1; }
  *   dv_t = dDelta_t sigmoid(v_t):  ddt_raw_t = dv_t,  ddt_bias += dv_t
  *   dpre_t = du_t SiLU'(pre_t):  dconv_b += dpre_t,  dconv_w_k += dpre_t xpad[t+k],
  *                                dxp_{t'} += dpre_t w_k  for xpad[t+k] = x'[t'] (t' = t+k-K+1 >= 0)
- *   dA_log_n = dA_n A_n   (dA/dA_log = -exp(A_log) = A).
+ *   dA_log_n = dA_n A_n   (dA/dA_log = -exp(A_log) = A);
+ *   dh_in = lam after step 0 (the adjoint carried into the initial state);
+ *   dconv_state_in_k = the gradient of xpad[k], k < K-1, collected like dxp.
  */
 static double sigm(double v) { return 1.0 / (1.0 + exp(-v)); }
 static double silu_d(double v) { const double s = sigm(v); return s * (1.0 + v * (1.0 - s)); }
@@ -118,9 +125,11 @@ int oracle_mixer_bwd_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t
                          int64_t d_conv, const double* xp, const double* z, const double* dt_raw,
                          const double* Bm, const double* Cm, const double* A_log, const double* Dv,
                          const double* conv_w, const double* conv_b, const double* dt_bias,
-                         const double* dy, double* dxp, double* dz, double* ddt_raw, double* dB,
-                         double* dC, double* dA_log, double* dD, double* dconv_w,
-                         double* dconv_b, double* ddt_bias, int nthreads) {
+                         const int32_t* seq_idx, const double* h_in,
+                         const double* conv_state_in, const double* dy, double* dxp, double* dz,
+                         double* ddt_raw, double* dB, double* dC, double* dA_log, double* dD,
+                         double* dconv_w, double* dconv_b, double* ddt_bias, double* dh_in,
+                         double* dconv_state_in, int nthreads) {
   if (batch < 0 || seqlen < 0 || d_inner < 0 || d_state < 1 || d_conv < 1) return 1;
   const int64_t L = seqlen, Di = d_inner, N = d_state, K = d_conv;
   int nth = nthreads > 0 ? nthreads : oracle_max_threads();
@@ -149,23 +158,36 @@ int oracle_mixer_bwd_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t
     double* h = (double*)malloc(sizeof(double) * (size_t)((L + 1) * N));   /* h[-1..L-1] */
     double* A = (double*)malloc(sizeof(double) * (size_t)N);
     double* lam = (double*)malloc(sizeof(double) * (size_t)N);
-    if (!xpad || !pre || !u || !vv || !del || !du || !ddel || !h || !A || !lam) {
+    double* dxpad = (double*)malloc(sizeof(double) * (size_t)(K - 1 + L));
+    char* rs = (char*)malloc((size_t)(L > 0 ? L : 1));      /* reset at step t */
+    if (!xpad || !pre || !u || !vv || !del || !du || !ddel || !h || !A || !lam || !dxpad || !rs) {
       bad = 1;
     } else {
       for (int64_t d = 0; d < Di; ++d) {
-        /* forward, keeping every intermediate */
-        for (int64_t k = 0; k < K - 1; ++k) xpad[k] = 0.0;
+        /* forward, keeping every intermediate; tap k of step t is live unless a reset lies
+           in (its position, t] */
+        for (int64_t k = 0; k < K - 1; ++k)
+          xpad[k] = conv_state_in ? conv_state_in[(b * Di + d) * (K - 1) + k] : 0.0;
         for (int64_t t = 0; t < L; ++t) xpad[K - 1 + t] = xp[(b * L + t) * Di + d];
-        for (int64_t n = 0; n < N; ++n) { A[n] = -exp(A_log[d * N + n]); h[n] = 0.0; }
+        for (int64_t t = 0; t < L; ++t)
+          rs[t] = (char)(seq_idx && t > 0 && seq_idx[b * L + t] != seq_idx[b * L + t - 1]);
+        for (int64_t n = 0; n < N; ++n) {
+          A[n] = -exp(A_log[d * N + n]);
+          h[n] = h_in ? h_in[(b * Di + d) * N + n] : 0.0;
+        }
         for (int64_t t = 0; t < L; ++t) {
           double acc = conv_b ? conv_b[d] : 0.0;
-          for (int64_t k = 0; k < K; ++k) acc += conv_w[d * K + k] * xpad[t + k];
+          for (int64_t k = 0; k < K; ++k) {
+            int live = 1;
+            for (int64_t s2 = t + k - (K - 1) + 1; s2 <= t; ++s2) if (s2 >= 0 && rs[s2]) live = 0;
+            if (live) acc += conv_w[d * K + k] * xpad[t + k];
+          }
           pre[t] = acc;
           u[t] = acc * sigm(acc);
           vv[t] = dt_raw[(b * L + t) * Di + d] + dt_bias[d];
           del[t] = fmax(vv[t], 0.0) + log1p(exp(-fabs(vv[t])));
           for (int64_t n = 0; n < N; ++n)
-            h[(t + 1) * N + n] = exp(del[t] * A[n]) * h[t * N + n] +
+            h[(t + 1) * N + n] = exp(del[t] * A[n]) * (rs[t] ? 0.0 : h[t * N + n]) +
                                  del[t] * Bm[(b * L + t) * N + n] * u[t];
         }
         /* gate and output readout */
@@ -190,16 +212,19 @@ int oracle_mixer_bwd_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t
           for (int64_t n = 0; n < N; ++n) {
             const double Bn = Bm[(b * L + t) * N + n], Cn = Cm[(b * L + t) * N + n];
             const double a = exp(del[t] * A[n]);
+            const double hprev = rs[t] ? 0.0 : h[t * N + n];   /* the state entering step t */
             lam[n] += dyc * Cn;
             dB[(b * L + t) * N + n] += lam[n] * del[t] * u[t];
             du[t] += lam[n] * del[t] * Bn;
-            ddel[t] += lam[n] * Bn * u[t] + lam[n] * h[t * N + n] * a * A[n];
-            pA[d * N + n] += lam[n] * h[t * N + n] * a * del[t];
-            lam[n] *= a;
+            ddel[t] += lam[n] * Bn * u[t] + lam[n] * hprev * a * A[n];
+            pA[d * N + n] += lam[n] * hprev * a * del[t];
+            lam[n] = rs[t] ? 0.0 : lam[n] * a;
           }
         }
+        if (dh_in)
+          for (int64_t n = 0; n < N; ++n) dh_in[(b * Di + d) * N + n] = lam[n];
         /* softplus and conv + SiLU */
-        for (int64_t t = 0; t < L; ++t) dxp[(b * L + t) * Di + d] = 0.0;
+        for (int64_t k = 0; k < K - 1 + L; ++k) dxpad[k] = 0.0;
         for (int64_t t = 0; t < L; ++t) {
           const int64_t o = (b * L + t) * Di + d;
           const double dv = ddel[t] * sigm(vv[t]);
@@ -208,15 +233,21 @@ int oracle_mixer_bwd_f64(int64_t batch, int64_t seqlen, int64_t d_inner, int64_t
           const double dpre = du[t] * silu_d(pre[t]);
           pCb[d] += dpre;
           for (int64_t k = 0; k < K; ++k) {
+            int live = 1;
+            for (int64_t s2 = t + k - (K - 1) + 1; s2 <= t; ++s2) if (s2 >= 0 && rs[s2]) live = 0;
+            if (!live) continue;
             pW[d * K + k] += dpre * xpad[t + k];
-            const int64_t tp = t + k - (K - 1);      /* xpad[t+k] = x'[tp] */
-            if (tp >= 0) dxp[(b * L + tp) * Di + d] += dpre * conv_w[d * K + k];
+            dxpad[t + k] += dpre * conv_w[d * K + k];
           }
         }
+        for (int64_t t = 0; t < L; ++t) dxp[(b * L + t) * Di + d] = dxpad[K - 1 + t];
+        if (dconv_state_in)
+          for (int64_t k = 0; k < K - 1; ++k)
+            dconv_state_in[(b * Di + d) * (K - 1) + k] = dxpad[k];
       }
     }
     free(xpad); free(pre); free(u); free(vv); free(del); free(du); free(ddel); free(h);
-    free(A); free(lam);
+    free(A); free(lam); free(dxpad); free(rs);
   }
   /* sum the rows' parameter gradients; chain dA -> dA_log */
   for (int64_t i = 0; i < Di * N; ++i) dA_log[i] = 0.0;

@@ -153,20 +153,24 @@ def mixer_channels(inp: dict, batch_idx, chan_idx, precision: str = "f64",
 BWD_NAMES = ("dxp", "dz", "ddt_raw", "dB", "dC", "dA_log", "dD", "dconv_w", "dconv_b", "ddt_bias")
 
 
-def mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, nthreads: int = 1):
-    """Gradients of sum(dy * y) with respect to every forward input (fp64 oracle; forward
-    from zero state).  Returns a dict keyed by BWD_NAMES (dconv_b is None without conv_b)."""
+def mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, nthreads: int = 1,
+              seq_idx=None, h_in=None, conv_state_in=None):
+    """Gradients of sum(dy * y) with respect to every forward input (fp64 oracle).  Returns
+    a dict keyed by BWD_NAMES (dconv_b None without conv_b), plus "dh_in" and
+    "dconv_state_in" (None unless the forward started from that cached state)."""
     lib = _load()
     fn = lib.oracle_mixer_bwd_f64
     if getattr(fn, "_typed", None) is None:
         i64, vp, ci = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
         fn.restype = ci
-        fn.argtypes = [i64] * 5 + [vp] * 21 + [ci]
+        fn.argtypes = [i64] * 5 + [vp] * 26 + [ci]
         fn._typed = True
     f = np.float64
     xp, z, dt_raw, B, C = (_arr(a, f) for a in (xp, z, dt_raw, B, C))
     A_log, D, conv_w, dt_bias, dy = (_arr(a, f) for a in (A_log, D, conv_w, dt_bias, dy))
     conv_b = _arr(conv_b, f)
+    seq_idx = _arr(seq_idx, np.int32)
+    h_in, conv_state_in = _arr(h_in, f), _arr(conv_state_in, f)
     Bt, L, Di = xp.shape
     N = A_log.shape[1]
     K = conv_w.shape[1]
@@ -176,10 +180,13 @@ def mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, nthrea
         "dB": np.empty((Bt, L, N)), "dC": np.empty((Bt, L, N)), "dA_log": np.empty((Di, N)),
         "dD": np.empty(Di), "dconv_w": np.empty((Di, K)),
         "dconv_b": None if conv_b is None else np.empty(Di), "ddt_bias": np.empty(Di),
+        "dh_in": None if h_in is None else np.empty((Bt, Di, N)),
+        "dconv_state_in": None if conv_state_in is None else np.empty((Bt, Di, K - 1)),
     }
     rc = fn(Bt, L, Di, N, K, _ptr(xp), _ptr(z), _ptr(dt_raw), _ptr(B), _ptr(C), _ptr(A_log),
-            _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(dy),
-            *[_ptr(out[k]) for k in BWD_NAMES], int(nthreads))
+            _ptr(D), _ptr(conv_w), _ptr(conv_b), _ptr(dt_bias), _ptr(seq_idx), _ptr(h_in),
+            _ptr(conv_state_in), _ptr(dy), *[_ptr(out[k]) for k in BWD_NAMES],
+            _ptr(out["dh_in"]), _ptr(out["dconv_state_in"]), int(nthreads))
     if rc != 0:
         raise RuntimeError(f"backward oracle failed with code {rc}")
     return out

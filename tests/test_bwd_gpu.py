@@ -82,3 +82,32 @@ def test_backward_with_time_chunks(oracle, Bt, L, Di, N, io):
     assert M.mamba_mixer_fwd_launches(dims) == 2      # the plan splits the sequence
     w, inp = _case(Bt, L, Di, N, io, 3200 + L)
     _compare(_run(inp), _oracle(oracle, inp), io, f"chunked {Bt}x{L}x{Di} N{N} {io}")
+
+
+def test_backward_long_sampled_channels(oracle):
+    """The long-sequence shape in full (2 x 65536 x 2560, bf16; 12 time chunks): every
+    gradient of a channel depends only on that channel and B/C, so the per-channel
+    gradients (dxp, dz, ddt_raw and the parameter gradients) of sampled channels are checked
+    against the oracle run on those channels alone; dB/dC (sums over all channels) are
+    covered by the other tests."""
+    from tests.gpu_util import pick_channels
+    w, inp = _case(2, 65536, 2560, 16, I.BF16, 3300)
+    di = pick_channels(2560, 10, 5)
+    d = to_device(inp)
+    gd = M.mamba_mixer_bwd(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                           d["conv_w"], d["conv_b"], d["dt_bias"], d["dy"])
+    torch.cuda.synchronize()
+    idx = torch.as_tensor(di, device="cuda")
+    g = {k: host(v[:, :, idx] if v.dim() == 3 and k in ("dxp", "dz", "ddt_raw") else v)
+         for k, v in gd.items() if k not in ("dB", "dC")}
+    del gd, d
+    sub = dict(inp)
+    for k in ("xp", "z", "dt_raw", "dy"):
+        sub[k] = inp[k][:, :, di]
+    for k in ("A_log", "D", "conv_w", "conv_b", "dt_bias"):
+        sub[k] = inp[k][di]
+    go = _oracle(oracle, sub)
+    for k in ("dxp", "dz", "ddt_raw"):
+        assert_close_grad(g[k], go[k], I.BF16, f"long {k}")
+    for k in ("dA_log", "dD", "dconv_w", "dconv_b", "ddt_bias"):
+        assert_close_grad(g[k][di], go[k], I.BF16, f"long {k}")
