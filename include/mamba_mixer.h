@@ -194,6 +194,28 @@ MAMBA_API int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void
                               void* cuda_stream);
 
 /*
+ * Backward of mamba_mixer_fwd_packed: as mamba_mixer_bwd, with the forward's optional
+ * seq_idx, h_in and conv_state_in (each may be NULL; see mamba_mixer_fwd_packed), and two
+ * optional gradient outputs (fp32, may be NULL = not computed): dh_in [batch, d_inner,
+ * d_state] and dconv_state_in [batch, d_inner, 3], the gradients of the initial state and
+ * conv window (defined, as zero-input gradients, even when h_in / conv_state_in are NULL).
+ * Where seq_idx changes, the conv taps before the document start pass no gradient and the
+ * adjoint state stops (niverel-mamba 0.1.0, section "seq_idx strict reset").  Same
+ * workspace as mamba_mixer_bwd.  Outputs must not overlap inputs, each other or the
+ * workspace.
+ */
+MAMBA_API int mamba_mixer_bwd_packed(const mamba_dims* dims, const void* xp, const void* z,
+                                     const void* dt_raw, const void* B, const void* C,
+                                     const float* A_log, const float* D, const float* conv_w,
+                                     const float* conv_b, const float* dt_bias,
+                                     const int32_t* seq_idx, const float* h_in,
+                                     const void* conv_state_in, const void* dy, float* dxp,
+                                     float* dz, float* ddt_raw, float* dB, float* dC,
+                                     float* dA_log, float* dD, float* dconv_w, float* dconv_b,
+                                     float* ddt_bias, float* dh_in, float* dconv_state_in,
+                                     void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * One decode step: one token for each of `batch` sequences (dims->seqlen must be 1) on a
  * cached state.  Inputs: xp, z, dt_raw [batch, 1, d_inner]; B, C [batch, 1, d_state];
  * the parameters as for mamba_mixer_fwd; h_in [batch, d_inner, d_state] fp32 and

@@ -30,9 +30,17 @@
 // its adjoint carried out from zero (Lambda, written by this kernel's kAdj instance).  The
 // input gradient of a chunk's last 3 steps also takes dpre of the next chunk's first 3: both
 // chunks add their parts atomically into those (zeroed) rows.
+//
+// Documents and a cached start (kExt instances, mamba_mixer_bwd_packed): where seq_idx
+// changes at step t, the conv taps before t carry no gradient and the state entering t is
+// zero, so the adjoint is cut there (lam = 0 after step t); the adjoint left after step 0 is
+// the gradient of h_in, and the conv input gradient of the 3 positions before 0 is that of
+// conv_state_in.
 #pragma once
 
 #include <float.h>
+
+#include <type_traits>
 
 #include "device_math.cuh"
 #include "sm100_primitives.cuh"
@@ -71,6 +79,18 @@ struct BwdParams {
   const float* ws_H;     // [batch, nchunks-1, d_inner, N] end state of each chunk from zero
   float* ws_L;           // [batch, nchunks, d_inner, N] adjoint carried out of each chunk from zero
 };
+
+// Extra arguments of the kExt instances (documents and a cached start; each may be null).
+// Only those instances take them, so the plain kernels' argument block stays as it is.
+struct BwdParamsExt : BwdParams {
+  const int32_t* seq_idx;  // [batch, L] document ids
+  const float* h_in;       // [batch, d_inner, N] state before token 0
+  const void* cs_in;       // [batch, d_inner, 3] conv window before token 0
+  float* dh_in;            // [batch, d_inner, N] gradient of h_in
+  float* dcs_in;           // [batch, d_inner, 3] gradient of conv_state_in (fp32)
+};
+template <bool kExt>
+using BwdArgs = typename std::conditional<kExt, BwdParamsExt, BwdParams>::type;
 
 constexpr int kBwdThreads = 128;
 constexpr int kBwdCh = 32;
@@ -170,9 +190,9 @@ __device__ __forceinline__ float sigmoid_(float v) {
   else return rcp_approx(1.0f + ex2_approx(-v * kLog2e));
 }
 
-template <int N, typename IO, bool kPrecise, bool kAdj>
+template <int N, typename IO, bool kPrecise, bool kAdj, bool kExt>
 __global__ void __launch_bounds__(kBwdThreads)
-bwd_kernel(const BwdParams p) {
+bwd_kernel(const BwdArgs<kExt> p) {
   using M = Math<kPrecise>;
   using Sm = BwdSmem<N, IO>;
   constexpr int kS = N / 4;
@@ -249,6 +269,33 @@ bwd_kernel(const BwdParams p) {
     cp_async_commit_();
   };
 
+  // Document ids of steps t0-4 .. t0+15 of tile k, one per lane (lanes 0..19), and the reset
+  // bits they give: bit i + 4 set when step t0 + i starts a document (i >= -3).
+  [[maybe_unused]] auto ids_for = [&](int k) -> int32_t {
+    if constexpr (kExt) {
+      const int64_t T = int64_t(k) * kBwdT - 4 + lane;
+      if (p.seq_idx && lane < kBwdT + 4 && T >= 0 && T < L) return __ldg(p.seq_idx + b * L + T);
+    }
+    return 0;
+  };
+  [[maybe_unused]] auto reset_bits = [&](int k, int32_t id) -> uint32_t {
+    if constexpr (kExt) {
+      if (!p.seq_idx) return 0u;
+      const int64_t T = int64_t(k) * kBwdT - 4 + lane;
+      const int32_t prv = __shfl_up_sync(0xffffffffu, id, 1);
+      return __ballot_sync(0xffffffffu, lane >= 1 && lane < kBwdT + 4 && T >= 1 && T < L &&
+                                            id != prv);
+    }
+    return 0u;
+  };
+  // x' of step t < 0 from the cached conv window (zero without one)
+  [[maybe_unused]] auto x_before = [&](int64_t t) -> float {
+    if constexpr (kExt) {
+      if (p.cs_in) return IOT<IO>::to_f(static_cast<const IO*>(p.cs_in)[(b * Di + d) * 3 + (3 + t)]);
+    }
+    return 0.0f;
+  };
+
   float A[kS], A2[kS];
 #pragma unroll
   for (int s = 0; s < kS; ++s) {
@@ -256,24 +303,44 @@ bwd_kernel(const BwdParams p) {
     A[s] = fmaxf(-expf(al), -FLT_MAX);              // A = -exp(A_log), for the gradients
     A2[s] = fmaxf(M::neg_exp(al) * M::a_scale(), -FLT_MAX);   // as the forward holds it
   }
+  // one step of the forward recurrence; with a reset at this step the entering state is zero
+  auto step_state = [&](float* h, float del, float du, const float* Bv, bool reset) {
+#pragma unroll
+    for (int s = 0; s < kS; ++s) {
+      const float a = M::decay(del, A2[s]);
+      h[s] = (reset ? 0.0f : a * h[s]) + du * Bv[s];
+    }
+  };
   const float w0 = __ldg(p.conv_w + d * 4 + 0), w1 = __ldg(p.conv_w + d * 4 + 1);
   const float w2 = __ldg(p.conv_w + d * 4 + 2), w3 = __ldg(p.conv_w + d * 4 + 3);
   const float cb = p.conv_b ? __ldg(p.conv_b + d) : 0.0f;
   const float dtb = __ldg(p.dt_bias + d);
   const float Dd = __ldg(p.D + d);
+  // the conv pre-activation of step t0 + i from x' of steps t-3..t (taps before a document
+  // start dropped): bits are the tile's reset bits
+  auto conv_pre = [&](float xa, float xb, float xc, float xt, uint32_t bits, int i) {
+    const bool m1 = !((bits >> (i + 4)) & 1u);
+    const bool m2 = m1 && !((bits >> (i + 3)) & 1u);
+    const bool m3 = m2 && !((bits >> (i + 2)) & 1u);
+    return cb + w0 * (m3 ? xa : 0.0f) + w1 * (m2 ? xb : 0.0f) + w2 * (m1 ? xc : 0.0f) + w3 * xt;
+  };
   float* ck = p.ws_h + ((b * p.ntiles) * Di + d) * N + j * kS;   // + k * Di * N per tile
   const uint32_t colx = uint32_t(cl * kEs);
   const uint32_t colbc = uint32_t(j * kS * kEs);
 
   if constexpr (kAdj) {
-    // ---- adjoint carried out of chunk c from zero: lam += dyc*C; lam *= a, last step first
+    // ---- adjoint carried out of chunk c from zero, last step first:
+    //      lam += dyc*C; lam = reset ? 0 : a*lam
     float lam[kS];
 #pragma unroll
     for (int s = 0; s < kS; ++s) lam[s] = 0.0f;
     stage(ke - 1, 0, true);
+    int32_t id = ids_for(ke - 1);
     for (int k = ke - 1, it = 0; k >= kb; --k, ++it) {
       if (k - 1 >= kb) stage(k - 1, (it + 1) & 1, true);
       else cp_async_commit_();
+      const uint32_t bits = reset_bits(k, id);
+      if (k - 1 >= kb) id = ids_for(k - 1);
       cp_async_wait_<1>();
       __syncthreads();
       const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
@@ -284,10 +351,12 @@ bwd_kernel(const BwdParams p) {
         const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
         const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
         const float dyc = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx) * zt * sigmoid_<kPrecise>(zt);
+        const bool reset = (bits >> (i + 4)) & 1u;
         float Cv[kS];
         lds_io_row<kS, IO>(sl + Sm::kCOff + i * Sm::kBCRow + colbc, Cv);
 #pragma unroll
-        for (int s = 0; s < kS; ++s) lam[s] = (lam[s] + dyc * Cv[s]) * M::decay(del, A2[s]);
+        for (int s = 0; s < kS; ++s)
+          lam[s] = reset ? 0.0f : (lam[s] + dyc * Cv[s]) * M::decay(del, A2[s]);
       }
       __syncthreads();
     }
@@ -301,19 +370,28 @@ bwd_kernel(const BwdParams p) {
     // ---- forward sweep: tile start states, from the state carried into this chunk
     {
       float h[kS];
-  #pragma unroll
+#pragma unroll
       for (int s = 0; s < kS; ++s) h[s] = 0.0f;
+      if constexpr (kExt) {
+        if (p.h_in) {
+#pragma unroll
+          for (int s = 0; s < kS; ++s) h[s] = __ldg(p.h_in + (b * Di + d) * N + j * kS + s);
+        }
+      }
       for (int cc = 0; cc < c; ++cc) {
         const int64_t o = ((b * (p.nchunks - 1) + cc) * Di + d) * N + j * kS;
-  #pragma unroll
+#pragma unroll
         for (int s = 0; s < kS; ++s) h[s] = p.ws_P[o + s] * h[s] + p.ws_H[o + s];
       }
       stage(kb, 0, false);
+      int32_t id = ids_for(kb);
       for (int k = kb, it = 0; k < ke; ++k, ++it) {
         if (k + 1 < ke) stage(k + 1, (it + 1) & 1, false);
         else cp_async_commit_();
+        const uint32_t bits = reset_bits(k, id);
+        if (k + 1 < ke) id = ids_for(k + 1);
         if (active) {
-  #pragma unroll
+#pragma unroll
           for (int s = 0; s < kS; ++s) ck[int64_t(k) * Di * N + s] = h[s];
         }
         cp_async_wait_<1>();
@@ -324,17 +402,17 @@ bwd_kernel(const BwdParams p) {
         float xa = lds_one<IO>(sl + Sm::kXOff + 1 * Sm::kRow + colx);
         float xb = lds_one<IO>(sl + Sm::kXOff + 2 * Sm::kRow + colx);
         float xc = lds_one<IO>(sl + Sm::kXOff + 3 * Sm::kRow + colx);
-  #pragma unroll 2
+        if (kExt && t0 == 0) { xa = x_before(-3); xb = x_before(-2); xc = x_before(-1); }
+#pragma unroll 2
         for (int i = 0; i < cnt; ++i) {
           const float xt = lds_one<IO>(sl + Sm::kXOff + (i + kBwdHalo) * Sm::kRow + colx);
-          const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          const float pre = conv_pre(xa, xb, xc, xt, bits, i);
           xa = xb; xb = xc; xc = xt;
           const float u = M::silu(pre);
           const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
           float Bv[kS];
           lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-  #pragma unroll
-          for (int s = 0; s < kS; ++s) h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
+          step_state(h, del, del * u, Bv, (bits >> (i + 4)) & 1u);
         }
         __syncthreads();   // the slot is refilled by the next iteration's stage
       }
@@ -342,33 +420,37 @@ bwd_kernel(const BwdParams p) {
 
     // ---- reverse sweep
     float lam[kS], dA[kS];
-  #pragma unroll
+#pragma unroll
     for (int s = 0; s < kS; ++s) { lam[s] = 0.0f; dA[s] = 0.0f; }
     // the adjoint carried back into this chunk: lam = P_c' * lam + Lambda_c', c' = C-1 .. c+1
     for (int cc = p.nchunks - 1; cc > c; --cc) {
       const int64_t oL = ((b * p.nchunks + cc) * Di + d) * N + j * kS;
       const int64_t oP = ((b * (p.nchunks - 1) + cc) * Di + d) * N + j * kS;
-  #pragma unroll
+#pragma unroll
       for (int s = 0; s < kS; ++s)
         lam[s] = (cc < p.nchunks - 1 ? p.ws_P[oP + s] * lam[s] : 0.0f) + p.ws_L[oL + s];
     }
-    float dp1 = 0.0f, dp2 = 0.0f, dp3 = 0.0f;          // dpre of steps t+1, t+2, t+3
+    // conv input gradient still to add to the positions 1, 2, 3 before the current step
+    float q1 = 0.0f, q2 = 0.0f, q3 = 0.0f;
     float aD = 0.0f, aDtb = 0.0f, aCb = 0.0f, aW0 = 0.0f, aW1 = 0.0f, aW2 = 0.0f, aW3 = 0.0f;
     for (int i = tid; i < 2 * kBwdT * N; i += kBwdThreads) acc[i] = 0.0f;
     __syncthreads();   // also orders this thread's checkpoint stores before its reloads
 
     float hn[kS];   // start state of the tile processed next (loaded one tile ahead)
-  #pragma unroll
+#pragma unroll
     for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(ke - 1) * Di * N + s];
     stage(ke - 1, 0, true);
+    int32_t id = ids_for(ke - 1);
     for (int k = ke - 1, it = 0; k >= kb; --k, ++it) {
       if (k - 1 >= kb) stage(k - 1, (it + 1) & 1, true);
       else cp_async_commit_();
+      const uint32_t bits = reset_bits(k, id);
+      if (k - 1 >= kb) id = ids_for(k - 1);
       float h0[kS], h[kS];
-  #pragma unroll
+#pragma unroll
       for (int s = 0; s < kS; ++s) h0[s] = h[s] = hn[s];
       if (k - 1 >= kb) {
-  #pragma unroll
+#pragma unroll
         for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(k - 1) * Di * N + s];
       }
       cp_async_wait_<1>();
@@ -377,16 +459,17 @@ bwd_kernel(const BwdParams p) {
       const int64_t t0 = int64_t(k) * kBwdT;
       const int cnt = int(t0 + kBwdT < t_end ? kBwdT : t_end - t0);
       auto xrow = [&](int i) {   // x' of step t0 + i, i >= -4 (the halo rows)
+        if (kExt && t0 + i < 0) return x_before(t0 + i);
         return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
       };
 
-      // recompute the tile: h_t and {pre, u, Delta, v}
+      // recompute the tile: h_t and {pre, sigmoid(pre), Delta, sigmoid(v)}
       {
         float xa = xrow(-3), xb = xrow(-2), xc = xrow(-1);
-  #pragma unroll 2
+#pragma unroll 2
         for (int i = 0; i < cnt; ++i) {
           const float xt = xrow(i);
-          const float pre = cb + w0 * xa + w1 * xb + w2 * xc + w3 * xt;
+          const float pre = conv_pre(xa, xb, xc, xt, bits, i);
           xa = xb; xb = xc; xc = xt;
           const float sp = sigmoid_<kPrecise>(pre);
           const float u = pre * sp;
@@ -394,17 +477,19 @@ bwd_kernel(const BwdParams p) {
           const float del = M::softplus(v);
           float Bv[kS];
           lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-  #pragma unroll
-          for (int s = 0; s < kS; ++s) h[s] = M::decay(del, A2[s]) * h[s] + del * u * Bv[s];
+          step_state(h, del, del * u, Bv, (bits >> (i + 4)) & 1u);
           sts_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), h);
           if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, sp, del, sigmoid_<kPrecise>(v));
         }
       }
       __syncwarp();
 
-  #pragma unroll 2
+#pragma unroll 2
       for (int i = cnt - 1; i >= 0; --i) {
         const int64_t t = t0 + i;
+        const bool m1 = !((bits >> (i + 4)) & 1u);           // no reset at t
+        const bool m2 = m1 && !((bits >> (i + 3)) & 1u);
+        const bool m3 = m2 && !((bits >> (i + 2)) & 1u);
         const float4 q = sc[i * kBwdCh + cl];
         const float pre = q.x, sp = q.y, del = q.z, sv = q.w;   // sp, sv: sigmoid(pre), sigmoid(v)
         const float u = pre * sp;
@@ -420,11 +505,12 @@ bwd_kernel(const BwdParams p) {
         if (i > 0) {
           lds_states<kS>(hsa + uint32_t((i - 1) * kBwdThreads * kS * 4), hp);
         } else {
-  #pragma unroll
+#pragma unroll
           for (int s = 0; s < kS; ++s) hp[s] = h0[s];
         }
-  #pragma unroll
+#pragma unroll
         for (int s = 0; s < kS; ++s) {
+          if (!m1) hp[s] = 0.0f;                               // the state entering a reset
           ycp += Cv[s] * ht[s];
           const float a = M::decay(del, A2[s]);
           lam[s] += dyc * Cv[s];
@@ -434,10 +520,10 @@ bwd_kernel(const BwdParams p) {
           const float ah = lam[s] * hp[s] * a;
           ddP += lam[s] * Bv[s] * u + ah * A[s];
           dA[s] += ah * del;
-          lam[s] *= a;
+          lam[s] = m1 ? lam[s] * a : 0.0f;
         }
         // channel sums over the 4 lanes of a channel (lane bits 3 and 4)
-  #pragma unroll
+#pragma unroll
         for (int m = 8; m <= 16; m <<= 1) {
           ycp += __shfl_xor_sync(0xffffffffu, ycp, m);
           duP += __shfl_xor_sync(0xffffffffu, duP, m);
@@ -448,13 +534,13 @@ bwd_kernel(const BwdParams p) {
         // (kS = 4) or, after a last all-reduce round, value chl >> 1 (kS = 2)
         {
           float vv[2 * kS];
-  #pragma unroll
+#pragma unroll
           for (int s = 0; s < kS; ++s) { vv[s] = cB[s]; vv[kS + s] = cC[s]; }
           int m = 4;
-  #pragma unroll
+#pragma unroll
           for (int half = kS; half >= 1; half >>= 1, m >>= 1) {
             const bool hi = (chl & m) != 0;
-  #pragma unroll
+#pragma unroll
             for (int e = 0; e < half; ++e) {
               const float keep = hi ? vv[half + e] : vv[e];
               const float send = hi ? vv[e] : vv[half + e];
@@ -475,14 +561,19 @@ bwd_kernel(const BwdParams p) {
         const float du = duP + dyc * Dd;
         const float dv = ddP * sv;                              // softplus' = sigmoid
         const float dpre = du * (sp * (1.0f + pre * (1.0f - sp)));   // SiLU'(pre)
-        // x' of steps t .. t-3 (the halo rows hold the steps before the tile, zeros before 0)
-        aW3 += dpre * xrow(i); aW2 += dpre * xrow(i - 1);
-        aW1 += dpre * xrow(i - 2); aW0 += dpre * xrow(i - 3);
+        // the taps of step t: x' of steps t .. t-3, live unless before the document start
+        aW3 += dpre * xrow(i);
+        if (m1) aW2 += dpre * xrow(i - 1);
+        if (m2) aW1 += dpre * xrow(i - 2);
+        if (m3) aW0 += dpre * xrow(i - 3);
         aCb += dpre;
         aDtb += dv;
         aD += dyc * u;
-        const float dx = w3 * dpre + w2 * dp1 + w1 * dp2 + w0 * dp3;
-        dp3 = dp2; dp2 = dp1; dp1 = dpre;
+        // the conv input gradient of step t is complete; pass the taps' parts back
+        const float dx = w3 * dpre + q1;
+        q1 = q2 + (m1 ? w2 * dpre : 0.0f);
+        q2 = q3 + (m2 ? w1 * dpre : 0.0f);
+        q3 = m3 ? w0 * dpre : 0.0f;
         if (j == 0 && active) {
           const int64_t o = (b * L + t) * Di + d;
           p.dz[o] = dyt * yc * (sz * (1.0f + zt * (1.0f - sz)));
@@ -506,14 +597,27 @@ bwd_kernel(const BwdParams p) {
     cp_async_wait_<0>();
 
     if (!active) return;
-    // this chunk's part of the input gradient of the previous chunk's last 3 steps
-    if (c > 0 && j == 0) {
-      float* o = p.dxp + (b * L + t_begin) * Di + d;
-      atomicAdd(o - Di, w2 * dp1 + w1 * dp2 + w0 * dp3);
-      atomicAdd(o - 2 * Di, w1 * dp1 + w0 * dp2);
-      atomicAdd(o - 3 * Di, w0 * dp1);
+    if (c > 0) {
+      // this chunk's part of the input gradient of the previous chunk's last 3 steps
+      if (j == 0) {
+        float* o = p.dxp + (b * L + t_begin) * Di + d;
+        atomicAdd(o - Di, q1);
+        atomicAdd(o - 2 * Di, q2);
+        atomicAdd(o - 3 * Di, q3);
+      }
+    } else if constexpr (kExt) {
+      // the adjoint after step 0 is the gradient of the initial state; the conv input
+      // gradient of the 3 positions before 0, that of the initial conv window
+      if (p.dh_in) {
+#pragma unroll
+        for (int s = 0; s < kS; ++s) p.dh_in[(b * Di + d) * N + j * kS + s] = lam[s];
+      }
+      if (p.dcs_in && j == 0) {
+        float* o = p.dcs_in + (b * Di + d) * 3;
+        o[2] = q1; o[1] = q2; o[0] = q3;
+      }
     }
-  #pragma unroll
+#pragma unroll
     for (int s = 0; s < kS; ++s) atomicAdd(p.dA_log + d * N + j * kS + s, dA[s] * A[s]);
     if (j == 0) {
       atomicAdd(p.dD + d, aD);

@@ -227,19 +227,17 @@ cudaError_t launch_fwd_any(const FwdMaps& m, const mm::FwdArgs<kExt>& a, const m
 
 // The backward's kernels: with time chunks, the forward's chunk-state pass (P, H), the
 // adjoint pass (Lambda), the zeroing of the rows two chunks add to, then the main pass.
-template <int N, typename IO, bool P>
-cudaError_t launch_bwd(const FwdMaps* m, const mm::FwdParams& fp, const mm::BwdParams& a,
-                       int64_t batch, cudaStream_t st) {
+template <int N, typename IO, bool P, bool kExt>
+cudaError_t launch_bwd(const FwdMaps* m, const mm::FwdArgs<kExt>& pre,
+                       const mm::BwdArgs<kExt>& a, int64_t batch, cudaStream_t st) {
   constexpr int smem = mm::BwdSmem<N, IO>::kTotal;
   const unsigned gx = unsigned((a.Di + mm::kBwdCh - 1) / mm::kBwdCh);
   cudaError_t e;
   if (a.nchunks > 1) {
-    mm::FwdArgs<false> pre;
-    static_cast<mm::FwdParams&>(pre) = fp;
-    e = launch_fwd_kernel<N, IO, P, true, false>(
+    e = launch_fwd_kernel<N, IO, P, true, kExt>(
         *m, pre, dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), st);
     if (e != cudaSuccess) return e;
-    auto adj = mm::bwd_kernel<N, IO, P, true>;
+    auto adj = mm::bwd_kernel<N, IO, P, true, kExt>;
     e = cudaFuncSetAttribute(adj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     adj<<<dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), mm::kBwdThreads, smem, st>>>(a);
@@ -247,11 +245,22 @@ cudaError_t launch_bwd(const FwdMaps* m, const mm::FwdParams& fp, const mm::BwdP
         a.dxp, a.L, a.Di, a.chunk_len);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  auto kern = mm::bwd_kernel<N, IO, P, false>;
+  auto kern = mm::bwd_kernel<N, IO, P, false, kExt>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   kern<<<dim3(gx, unsigned(batch), unsigned(a.nchunks)), mm::kBwdThreads, smem, st>>>(a);
   return cudaGetLastError();
+}
+
+template <bool kExt>
+cudaError_t launch_bwd_any(const FwdMaps* m, const mm::FwdArgs<kExt>& pre,
+                           const mm::BwdArgs<kExt>& a, const mamba_dims* d, cudaStream_t st) {
+  const bool f32 = d->io_dtype == MAMBA_F32;
+  if (d->d_state == 16)
+    return f32 ? launch_bwd<16, float, true, kExt>(m, pre, a, d->batch, st)
+               : launch_bwd<16, __nv_bfloat16, false, kExt>(m, pre, a, d->batch, st);
+  return f32 ? launch_bwd<8, float, true, kExt>(m, pre, a, d->batch, st)
+             : launch_bwd<8, __nv_bfloat16, false, kExt>(m, pre, a, d->batch, st);
 }
 
 // Backward workspace: header, tile start states, and with time chunks each chunk's
@@ -480,12 +489,20 @@ size_t mamba_mixer_bwd_workspace_bytes(const mamba_dims* dims) {
   return bwd_workspace_for(dims);
 }
 
-int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
-                    const void* B, const void* C, const float* A_log, const float* D,
-                    const float* conv_w, const float* conv_b, const float* dt_bias,
-                    const void* dy, float* dxp, float* dz, float* ddt_raw, float* dB, float* dC,
-                    float* dA_log, float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
-                    void* workspace, size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+// The backward behind mamba_mixer_bwd and mamba_mixer_bwd_packed (the latter's documents,
+// cached start and state gradients are null for the former).
+int bwd_common(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+               const void* B, const void* C, const float* A_log, const float* D,
+               const float* conv_w, const float* conv_b, const float* dt_bias,
+               const int32_t* seq_idx, const float* h_in, const void* conv_state_in,
+               const void* dy, float* dxp, float* dz, float* ddt_raw, float* dB, float* dC,
+               float* dA_log, float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
+               float* dh_in, float* dconv_state_in, void* workspace, size_t workspace_bytes,
+               void* cuda_stream) {
   Sizes s;
   int rc = check_dims(dims, &s);
   if (rc) return rc;
@@ -501,7 +518,11 @@ int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const
       (rc = check_ptr(dC, "dC", bc, 16)) || (rc = check_ptr(dA_log, "dA_log", par, 16)) ||
       (rc = check_ptr(dD, "dD", par, 4)) || (rc = check_ptr(dconv_w, "dconv_w", par, 16)) ||
       (rc = check_ptr(dconv_b, "dconv_b", false, 4)) ||
-      (rc = check_ptr(ddt_bias, "ddt_bias", par, 4)))
+      (rc = check_ptr(ddt_bias, "ddt_bias", par, 4)) ||
+      (rc = check_ptr(seq_idx, "seq_idx", false, 4)) || (rc = check_ptr(h_in, "h_in", false, 16)) ||
+      (rc = check_ptr(conv_state_in, "conv_state_in", false, 2)) ||
+      (rc = check_ptr(dh_in, "dh_in", false, 16)) ||
+      (rc = check_ptr(dconv_state_in, "dconv_state_in", false, 4)))
     return rc;
   const int64_t Di = dims->d_inner, N = dims->d_state;
   const Span ins[] = {{xp, size_t(s.act) * s.esize, "xp"},   {z, size_t(s.act) * s.esize, "z"},
@@ -510,12 +531,17 @@ int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const
                       {dy, size_t(s.act) * s.esize, "dy"},
                       {A_log, size_t(Di * N) * 4, "A_log"}, {D, size_t(Di) * 4, "D"},
                       {conv_w, size_t(Di) * 16, "conv_w"},  {conv_b, size_t(Di) * 4, "conv_b"},
-                      {dt_bias, size_t(Di) * 4, "dt_bias"}};
+                      {dt_bias, size_t(Di) * 4, "dt_bias"},
+                      {seq_idx, size_t(dims->batch) * size_t(dims->seqlen) * 4, "seq_idx"},
+                      {h_in, size_t(s.state) * 4, "h_in"},
+                      {conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"}};
   const Span outs[] = {{dxp, size_t(s.act) * 4, "dxp"},      {dz, size_t(s.act) * 4, "dz"},
                        {ddt_raw, size_t(s.act) * 4, "ddt_raw"}, {dB, size_t(s.bc) * 4, "dB"},
                        {dC, size_t(s.bc) * 4, "dC"},          {dA_log, size_t(Di * N) * 4, "dA_log"},
                        {dD, size_t(Di) * 4, "dD"},            {dconv_w, size_t(Di) * 16, "dconv_w"},
-                       {dconv_b, size_t(Di) * 4, "dconv_b"},  {ddt_bias, size_t(Di) * 4, "ddt_bias"}};
+                       {dconv_b, size_t(Di) * 4, "dconv_b"},  {ddt_bias, size_t(Di) * 4, "ddt_bias"},
+                       {dh_in, size_t(s.state) * 4, "dh_in"},
+                       {dconv_state_in, size_t(s.cstate) * 4, "dconv_state_in"}};
   const size_t need = bwd_workspace_for(dims);
   const Span wsp{workspace, need, "workspace"};
   for (const Span& o : outs) {
@@ -545,7 +571,15 @@ int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const
   for (const auto& zr : zero)
     if (e == cudaSuccess && zr.first && zr.second) e = cudaMemsetAsync(zr.first, 0, zr.second, st);
   if (e != cudaSuccess) return fail(MAMBA_ERR_CUDA, "gradient reset failed: %s", cudaGetErrorString(e));
-  if (dims->seqlen == 0) return ok();
+  if (dims->seqlen == 0) {
+    // nothing flows back but into the initial state: the gradients of h_in and of the conv
+    // window are zero (y is empty)
+    if (dh_in && e == cudaSuccess) e = cudaMemsetAsync(dh_in, 0, size_t(s.state) * 4, st);
+    if (dconv_state_in && e == cudaSuccess)
+      e = cudaMemsetAsync(dconv_state_in, 0, size_t(s.cstate) * 4, st);
+    if (e != cudaSuccess) return fail(MAMBA_ERR_CUDA, "gradient reset failed: %s", cudaGetErrorString(e));
+    return ok();
+  }
 
   const Plan plan = make_plan(dims);
   const BwdLayout lay = bwd_layout(dims, plan);
@@ -585,15 +619,50 @@ int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const
     fp.chunk_len = plan.chunk_len; fp.nchunks = plan.nchunks;
     fp.inject_skip_tile = -1;
   }
-  if (N == 16)
-    e = f32 ? launch_bwd<16, float, true>(&m, fp, a, dims->batch, st)
-            : launch_bwd<16, __nv_bfloat16, false>(&m, fp, a, dims->batch, st);
-  else
-    e = f32 ? launch_bwd<8, float, true>(&m, fp, a, dims->batch, st)
-            : launch_bwd<8, __nv_bfloat16, false>(&m, fp, a, dims->batch, st);
+  if (seq_idx || h_in || conv_state_in || dh_in || dconv_state_in) {
+    mm::BwdParamsExt ax;
+    static_cast<mm::BwdParams&>(ax) = a;
+    ax.seq_idx = seq_idx; ax.h_in = h_in; ax.cs_in = conv_state_in;
+    ax.dh_in = dh_in; ax.dcs_in = dconv_state_in;
+    mm::FwdParamsExt px;
+    static_cast<mm::FwdParams&>(px) = fp;
+    px.ext = mm::FwdExt{seq_idx, nullptr, conv_state_in};   // chunk pairs start from zero
+    e = launch_bwd_any<true>(&m, px, ax, dims, st);
+  } else {
+    e = launch_bwd_any<false>(&m, fp, a, dims, st);
+  }
   if (e != cudaSuccess)
     return fail(MAMBA_ERR_CUDA, "backward launch failed: %s", cudaGetErrorString(e));
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
+                    const void* B, const void* C, const float* A_log, const float* D,
+                    const float* conv_w, const float* conv_b, const float* dt_bias,
+                    const void* dy, float* dxp, float* dz, float* ddt_raw, float* dB, float* dC,
+                    float* dA_log, float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
+                    void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  return bwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
+                    nullptr, nullptr, dy, dxp, dz, ddt_raw, dB, dC, dA_log, dD, dconv_w, dconv_b,
+                    ddt_bias, nullptr, nullptr, workspace, workspace_bytes, cuda_stream);
+}
+
+int mamba_mixer_bwd_packed(const mamba_dims* dims, const void* xp, const void* z,
+                           const void* dt_raw, const void* B, const void* C, const float* A_log,
+                           const float* D, const float* conv_w, const float* conv_b,
+                           const float* dt_bias, const int32_t* seq_idx, const float* h_in,
+                           const void* conv_state_in, const void* dy, float* dxp, float* dz,
+                           float* ddt_raw, float* dB, float* dC, float* dA_log, float* dD,
+                           float* dconv_w, float* dconv_b, float* ddt_bias, float* dh_in,
+                           float* dconv_state_in, void* workspace, size_t workspace_bytes,
+                           void* cuda_stream) {
+  return bwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, seq_idx, h_in,
+                    conv_state_in, dy, dxp, dz, ddt_raw, dB, dC, dA_log, dD, dconv_w, dconv_b,
+                    ddt_bias, dh_in, dconv_state_in, workspace, workspace_bytes, cuda_stream);
 }
 
 int mamba_mixer_step(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,

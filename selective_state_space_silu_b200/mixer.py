@@ -25,6 +25,7 @@ STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPOR
           6: "MAMBA_ERR_TIMEOUT"}
 EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba_mixer_fwd",
            "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
+           "mamba_mixer_bwd_packed",
            "mamba_mixer_step", "mamba_mixer_check", "mamba_last_error", "mamba_version")
 
 
@@ -70,6 +71,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba_mixer_bwd_workspace_bytes.argtypes = [P]
     lib.mamba_mixer_bwd.restype = i
     lib.mamba_mixer_bwd.argtypes = [P] + [vp] * 21 + [vp, sz, vp]
+    lib.mamba_mixer_bwd_packed.restype = i
+    lib.mamba_mixer_bwd_packed.argtypes = [P] + [vp] * 26 + [vp, sz, vp]
     lib.mamba_mixer_step.restype = i
     lib.mamba_mixer_step.argtypes = [P] + [vp] * 15 + [vp]
     lib.mamba_last_error.restype = ctypes.c_char_p
@@ -258,6 +261,45 @@ def mamba_mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, 
         _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
         _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
         _ptr(dy, "dy", iot, dev), *[_ptr(g[k], k, f32, dev) for k in BWD_OUTPUTS],
+        _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
+    _check(rc)
+    return g
+
+
+def mamba_mixer_bwd_packed(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, *,
+                           seq_idx=None, h_in=None, conv_state_in=None, want_state_grads=True,
+                           workspace=None, stream=None) -> dict:
+    """Gradients of sum(dy * y) for mamba_mixer_fwd_packed (documents and/or a cached
+    start), all fp32: the keys of BWD_OUTPUTS plus "dh_in" and "dconv_state_in" (None when
+    want_state_grads is False)."""
+    lib = load_library()
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    dims = make_dims(Bt, L, Di, N, K, io)
+    f32 = torch.float32
+    e = lambda *shape: torch.empty(shape, dtype=f32, device=dev)
+    g = {"dxp": e(Bt, L, Di), "dz": e(Bt, L, Di), "ddt_raw": e(Bt, L, Di), "dB": e(Bt, L, N),
+         "dC": e(Bt, L, N), "dA_log": e(Di, N), "dD": e(Di), "dconv_w": e(Di, K),
+         "dconv_b": None if conv_b is None else e(Di), "ddt_bias": e(Di),
+         "dh_in": e(Bt, Di, N) if want_state_grads else None,
+         "dconv_state_in": e(Bt, Di, K - 1) if want_state_grads else None}
+    need = int(lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(dims)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib.mamba_mixer_bwd_packed(
+        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(seq_idx, "seq_idx", torch.int32, dev), _ptr(h_in, "h_in", f32, dev),
+        _ptr(conv_state_in, "conv_state_in", iot, dev), _ptr(dy, "dy", iot, dev),
+        *[_ptr(g[k], k, f32, dev) for k in BWD_OUTPUTS],
+        _ptr(g["dh_in"], "dh_in", f32, dev), _ptr(g["dconv_state_in"], "dconv_state_in", f32, dev),
         _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
     _check(rc)
     return g

@@ -223,3 +223,23 @@ def test_backward_validation(lib):
     assert _bwd(lib, d, {"dz": _fake(0x10000000 + 11 * (1 << 36))}, ws, need) == 1
     assert _bwd(lib, M.make_dims(2, 64, 128, 12), ws=ws, ws_bytes=need) == 2   # d_state 12
     assert lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(M.make_dims(2, 64, 128, 12))) == 0
+
+
+def test_packed_backward_validation(lib):
+    d = M.make_dims(2, 64, 128, 16)
+    need = lib.mamba_mixer_bwd_workspace_bytes(ctypes.byref(d))
+    ws = _fake(0x10000000 + 40 * (1 << 36))
+    base = 0x10000000
+    names = ["xp", "z", "dt", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias", "seq", "h_in",
+             "cs_in", "dy", "dxp", "dz", "ddt", "dB", "dC", "dA_log", "dD", "dconv_w", "dconv_b",
+             "ddt_bias", "dh_in", "dcs_in"]
+
+    def call(over):
+        p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(names)}
+        p.update(over)
+        return lib.mamba_mixer_bwd_packed(ctypes.byref(d), *[p[k] for k in names], ws, need, None)
+
+    assert call({"seq": _fake(base + 10 * (1 << 36) + 2)}) == 3
+    assert call({"dh_in": _fake(base + 11 * (1 << 36))}) == 1          # on top of h_in
+    assert "overlaps" in M.mamba_last_error()
+    assert call({"dcs_in": _fake(base + 24 * (1 << 36) + 2)}) == 3      # fp32 gradient, 4-aligned

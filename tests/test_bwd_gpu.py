@@ -111,3 +111,66 @@ def test_backward_long_sampled_channels(oracle):
         assert_close_grad(g[k], go[k], I.BF16, f"long {k}")
     for k in ("dA_log", "dD", "dconv_w", "dconv_b", "ddt_bias"):
         assert_close_grad(g[k][di], go[k], I.BF16, f"long {k}")
+
+
+def _case_packed(Bt, L, Di, N, io, seed, case, state, edge):
+    w = I.Workload("bwdp", Bt, L, Di, N, 4, io, seed, decode=state)
+    inp = I.make_inputs(w)
+    dy = np.random.default_rng(seed + 1).standard_normal((Bt, L, Di)).astype(np.float32)
+    inp["dy"] = I.f32_to_bf16_bits(dy) if io == I.BF16 else dy
+    inp["seq_idx"] = None if case is None else I.seq_idx_case(case, Bt, L, edge=edge, seed=9)
+    return w, inp
+
+
+def _run_packed(inp, state):
+    d = to_device({k: v for k, v in inp.items() if k != "seq_idx"})
+    seq = None if inp["seq_idx"] is None else torch.from_numpy(inp["seq_idx"]).cuda()
+    g = M.mamba_mixer_bwd_packed(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                                 d["conv_w"], d.get("conv_b"), d["dt_bias"], d["dy"], seq_idx=seq,
+                                 h_in=d["h"] if state else None,
+                                 conv_state_in=d["conv_state"] if state else None)
+    torch.cuda.synchronize()
+    return {k: (None if v is None else host(v)) for k, v in g.items()}
+
+
+def _oracle_packed(oracle, inp, state):
+    w = I.as_f64
+    return oracle.mixer_bwd(w(inp["xp"]), w(inp["z"]), w(inp["dt_raw"]), w(inp["B"]), w(inp["C"]),
+                            inp["A_log"], inp["D"], inp["conv_w"], inp.get("conv_b"),
+                            inp["dt_bias"], w(inp["dy"]), nthreads=0, seq_idx=inp["seq_idx"],
+                            h_in=inp["h"] if state else None,
+                            conv_state_in=w(inp["conv_state"]) if state else None)
+
+
+def _compare_packed(g, go, io, what):
+    _compare(g, go, io, what)
+    for k in ("dh_in", "dconv_state_in"):
+        if go[k] is None:
+            # no cached start in the forward: the device still returns the zero-input gradient
+            continue
+        assert_close_grad(g[k], go[k], io, f"{what} {k}")
+
+
+@pytest.mark.parametrize("state", [False, True])
+@pytest.mark.parametrize("io", [I.F32, I.BF16])
+@pytest.mark.parametrize("case", ["length_one_docs", "consecutive_boundaries", "boundary_on_edge",
+                                  "terminal_padding", "many_short_docs"])
+def test_packed_backward_matches_oracle(oracle, case, io, state):
+    w, inp = _case_packed(3, 300, 64, 16, io, 3400 + len(case), case, state, edge=16)
+    _compare_packed(_run_packed(inp, state), _oracle_packed(oracle, inp, state), io,
+                    f"packed {case} {io} state={state}")
+
+
+@pytest.mark.parametrize("case", ["boundary_on_edge", "many_short_docs", "misaligned_rows"])
+def test_packed_backward_with_time_chunks(oracle, case):
+    """16 chunks of 256 steps with boundaries on the chunk edges (and everywhere)."""
+    w, inp = _case_packed(2, 4096, 64, 16, I.BF16, 3500 + len(case), case, True, edge=256)
+    assert M.mamba_mixer_fwd_launches(M.make_dims(2, 4096, 64, 16, 4, M.MAMBA_BF16)) == 2
+    _compare_packed(_run_packed(inp, True), _oracle_packed(oracle, inp, True), I.BF16,
+                    f"packed chunked {case}")
+
+
+def test_packed_backward_cached_start_only(oracle):
+    """No documents, a cached start: the state gradients against the oracle's."""
+    w, inp = _case_packed(2, 777, 72, 8, I.F32, 3600, None, True, edge=16)
+    _compare_packed(_run_packed(inp, True), _oracle_packed(oracle, inp, True), I.F32, "cached")
