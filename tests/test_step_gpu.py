@@ -109,3 +109,22 @@ def test_steps_from_zero_state_equal_forward(oracle):
     yo, ho, _ = oracle_full(oracle, inp)
     assert_close(host(torch.cat(ys, 1)), yo, "bf16", "steps from zero")
     assert_close(host(h), ho, "bf16", "steps from zero h")
+
+
+
+def test_decode_unaligned_conv_state(oracle):
+    """A conv state 2 bytes off a 16-byte boundary (the API allows 2-byte alignment)."""
+    w = I.Workload("dec_u", 5, 1, 200, 16, 4, "bf16", 321, decode=True)
+    inp = I.make_inputs(w)
+    d = to_device(inp)
+    n = d["conv_state"].numel()
+    buf = torch.empty(n + 8, dtype=d["conv_state"].dtype, device="cuda")
+    cs_in = buf[1:1 + n].view(d["conv_state"].shape)
+    cs_in.copy_(d["conv_state"])
+    assert cs_in.data_ptr() % 16 != 0
+    y, h, cs = gpu_step(d, d["h"], cs_in)
+    torch.cuda.synchronize()
+    yo, ho, cso = oracle_full(oracle, inp, with_state=True)
+    assert_close(host(y), yo, w.io_dtype, "unaligned y")
+    assert_close(host(h), ho, w.io_dtype, "unaligned h_out")
+    np.testing.assert_array_equal(host(cs), cso)
