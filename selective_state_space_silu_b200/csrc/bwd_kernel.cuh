@@ -327,6 +327,22 @@ bwd_kernel(const BwdArgs<kExt> p) {
   float* ck = p.ws_h + ((b * p.ntiles) * Di + d) * N + j * kS;   // + k * Di * N per tile
   const uint32_t colx = uint32_t(cl * kEs);
   const uint32_t colbc = uint32_t(j * kS * kEs);
+  // The per-(t, d) scalars of a tile -- {pre, sigmoid(pre), Delta, sigmoid(v)} into sc --
+  // computed once per (t, d): the 4 lanes of a channel take steps j, j+4, j+8, j+12.
+  // xr(i) is x' of step t0 + i (i >= -3).
+  auto tile_scalars = [&](uint32_t sl, int cnt, uint32_t bits, auto xr) {
+#pragma unroll
+    for (int m = 0; m < kBwdT / 4; ++m) {
+      const int i = j + 4 * m;
+      if (i < cnt) {
+        const float pre = conv_pre(xr(i - 3), xr(i - 2), xr(i - 1), xr(i), bits, i);
+        const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
+        sc[i * kBwdCh + cl] = make_float4(pre, sigmoid_<kPrecise>(pre), M::softplus(v),
+                                          sigmoid_<kPrecise>(v));
+      }
+    }
+    __syncwarp();
+  };
 
   if constexpr (kAdj) {
     // ---- adjoint carried out of chunk c from zero, last step first:
@@ -399,22 +415,19 @@ bwd_kernel(const BwdArgs<kExt> p) {
         const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
         const int64_t t0 = int64_t(k) * kBwdT;
         const int cnt = int(t0 + kBwdT < t_end ? kBwdT : t_end - t0);
-        float xa = lds_one<IO>(sl + Sm::kXOff + 1 * Sm::kRow + colx);
-        float xb = lds_one<IO>(sl + Sm::kXOff + 2 * Sm::kRow + colx);
-        float xc = lds_one<IO>(sl + Sm::kXOff + 3 * Sm::kRow + colx);
-        if (kExt && t0 == 0) { xa = x_before(-3); xb = x_before(-2); xc = x_before(-1); }
+        tile_scalars(sl, cnt, bits, [&](int i) {
+          if (kExt && t0 + i < 0) return x_before(t0 + i);
+          return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
+        });
 #pragma unroll 2
         for (int i = 0; i < cnt; ++i) {
-          const float xt = lds_one<IO>(sl + Sm::kXOff + (i + kBwdHalo) * Sm::kRow + colx);
-          const float pre = conv_pre(xa, xb, xc, xt, bits, i);
-          xa = xb; xb = xc; xc = xt;
-          const float u = M::silu(pre);
-          const float del = M::softplus(lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb);
+          const float4 q = sc[i * kBwdCh + cl];
+          const float del = q.z;
           float Bv[kS];
           lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-          step_state(h, del, del * u, Bv, (bits >> (i + 4)) & 1u);
+          step_state(h, del, del * (q.x * q.y), Bv, (bits >> (i + 4)) & 1u);
         }
-        __syncthreads();   // the slot is refilled by the next iteration's stage
+        __syncthreads();   // the slot (and sc) are refilled by the next iteration
       }
     }
 
@@ -463,24 +476,15 @@ bwd_kernel(const BwdArgs<kExt> p) {
         return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
       };
 
-      // recompute the tile: h_t and {pre, sigmoid(pre), Delta, sigmoid(v)}
-      {
-        float xa = xrow(-3), xb = xrow(-2), xc = xrow(-1);
+      // recompute the tile: {pre, sigmoid(pre), Delta, sigmoid(v)}, then the states h_t
+      tile_scalars(sl, cnt, bits, xrow);
 #pragma unroll 2
-        for (int i = 0; i < cnt; ++i) {
-          const float xt = xrow(i);
-          const float pre = conv_pre(xa, xb, xc, xt, bits, i);
-          xa = xb; xb = xc; xc = xt;
-          const float sp = sigmoid_<kPrecise>(pre);
-          const float u = pre * sp;
-          const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
-          const float del = M::softplus(v);
-          float Bv[kS];
-          lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-          step_state(h, del, del * u, Bv, (bits >> (i + 4)) & 1u);
-          sts_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), h);
-          if (j == 0) sc[i * kBwdCh + cl] = make_float4(pre, sp, del, sigmoid_<kPrecise>(v));
-        }
+      for (int i = 0; i < cnt; ++i) {
+        const float4 q = sc[i * kBwdCh + cl];
+        float Bv[kS];
+        lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
+        step_state(h, q.z, q.z * (q.x * q.y), Bv, (bits >> (i + 4)) & 1u);
+        sts_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), h);
       }
       __syncwarp();
 
