@@ -11,7 +11,7 @@ import pytest
 import torch
 
 from selective_state_space_silu_b200 import inputs as I
-from tests.gpu_util import (dev_tensor, gpu_fwd, host, host_bits, oracle_full,
+from tests.gpu_util import (gpu_fwd, host, host_bits, oracle_full,
                             pick_channels, to_device)
 from tests.tolerances import assert_close
 

@@ -13,7 +13,7 @@ import torch
 
 from selective_state_space_silu_b200 import inputs as I
 from selective_state_space_silu_b200 import mixer as M
-from tests.gpu_util import dev_tensor, host, to_device
+from tests.gpu_util import host, to_device
 from tests.tolerances import assert_close
 
 pytestmark = pytest.mark.gpu
