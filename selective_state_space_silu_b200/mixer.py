@@ -383,3 +383,31 @@ def mamba_mixer_fwd_noalloc(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bi
         _ptr(conv_state_out, "conv_state_out", iot, dev), _stream_handle(stream, dev))
     _check(rc)
     return y, h_out, conv_state_out
+
+
+class MambaMixerFunction(torch.autograd.Function):
+    """The fused forward as a differentiable op: forward = mamba_mixer_fwd (from a zero
+    state), backward = mamba_mixer_bwd; gradients come back in each input's dtype."""
+
+    @staticmethod
+    def forward(ctx, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias):
+        xp, z, dt_raw, B, C = (t.contiguous() for t in (xp, z, dt_raw, B, C))
+        y, _, _ = mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
+                                  want_states=False)
+        ctx.save_for_backward(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias)
+        return y
+
+    @staticmethod
+    def backward(ctx, dy):
+        xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias = ctx.saved_tensors
+        g = mamba_mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
+                            dy.to(xp.dtype).contiguous())
+        as_ = lambda k, ref: None if g[k] is None else g[k].to(ref.dtype)
+        return (as_("dxp", xp), as_("dz", z), as_("ddt_raw", dt_raw), as_("dB", B), as_("dC", C),
+                as_("dA_log", A_log), as_("dD", D), as_("dconv_w", conv_w),
+                None if conv_b is None else as_("dconv_b", conv_b), as_("ddt_bias", dt_bias))
+
+
+def mamba_mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias):
+    """y = the fused mixer forward, differentiable with respect to every input."""
+    return MambaMixerFunction.apply(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias)

@@ -174,3 +174,22 @@ def test_packed_backward_cached_start_only(oracle):
     """No documents, a cached start: the state gradients against the oracle's."""
     w, inp = _case_packed(2, 777, 72, 8, I.F32, 3600, None, True, edge=16)
     _compare_packed(_run_packed(inp, True), _oracle_packed(oracle, inp, True), I.F32, "cached")
+
+
+@pytest.mark.parametrize("io", [I.F32, I.BF16])
+def test_autograd_function_matches_oracle(oracle, io):
+    """mixer.mamba_mixer as a torch autograd op: y.backward(dy) fills every input's .grad
+    (in the input's dtype) with the oracle's gradients."""
+    w, inp = _case(2, 200, 64, 16, io, 3700)
+    d = to_device(inp)
+    names = ("xp", "z", "dt_raw", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias")
+    leaves = {k: d[k].clone().requires_grad_(True) for k in names}
+    y = M.mamba_mixer(*(leaves[k] for k in names))
+    y.backward(d["dy"])
+    torch.cuda.synchronize()
+    go = _oracle(oracle, inp)
+    for k in names:
+        assert leaves[k].grad is not None and leaves[k].grad.dtype == leaves[k].dtype, k
+        # bf16 gradients of activations carry bf16 rounding on top of the fp32 result
+        assert_close_grad(host(leaves[k].grad), go["d" + k], io,
+                          f"autograd {io} {k}")
