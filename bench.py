@@ -128,7 +128,7 @@ def measured_peaks() -> dict:
 # record names the plan it was taken with.)
 KERNEL_SOURCES = {
     "fwd": ("fwd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
-    "step": ("step.cuh", "device_math.cuh"),
+    "step": ("step.cuh", "device_math.cuh", "sm100_primitives.cuh"),
 }
 
 
