@@ -556,6 +556,120 @@ def oracle_sample_bwd(w: I.Workload, target_s: float):
                                   f"x L={L} (fp64 oracle, {el:.2f} s)")
 
 
+# ----------------------------------------------------------------------------- Mamba2 scan
+SSD_Q = 64  # chunk length of the Mamba2 scan kernel
+
+
+def ssd_bytes(w) -> int:
+    """Algorithmic bytes of one Mamba2 scan call: x (and z), dt_raw, B, C read once, y
+    written once (bf16), the per-head parameters, h_in read and h_out written (fp32)."""
+    Bt, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.d_state, w.ngroups
+    act = Bt * L * H * P * 2
+    return (act * (3 if w.gate else 2) + Bt * L * H * 2 + 2 * Bt * L * G * N * 2 + 3 * H * 4
+            + Bt * H * P * N * 4 * (2 if w.state else 1))
+
+
+def ssd_flops(w) -> int:
+    """Algorithmic tensor FLOPs of the chunked evaluation with 64-step chunks, causal half
+    only: per (row, head, chunk of q steps) q(q+1)/2 (N + P) multiply-adds for C B^T and
+    its product with x, plus q N P each for the inter-chunk term and the state update."""
+    Bt, L, H, P, N = w.batch, w.seqlen, w.nheads, w.headdim, w.d_state
+    total = 0
+    full, tail = divmod(L, SSD_Q)
+    for q, cnt in ((SSD_Q, full), (tail, 1 if tail else 0)):
+        total += cnt * 2 * (q * (q + 1) // 2 * (N + P) + 2 * q * N * P)
+    return Bt * H * total
+
+
+def run_ssd(args, w, local_rank: int):
+    """--pass ssd: times mamba2_ssd_fwd alone (device events, L2 flushed between calls)."""
+    import torch
+    from selective_state_space_silu_b200 import mixer as M
+    from selective_state_space_silu_b200 import ssd as S
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M.load_library()
+    inp = I.make_ssd_inputs(w)
+
+    def td(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    d = {k: td(v) for k, v in inp.items()}
+    y = torch.empty_like(d["x"])
+    h_out = torch.empty(w.batch, w.nheads, w.headdim, w.d_state, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def call():
+        S.mamba2_ssd_fwd(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"], d["dt_bias"],
+                         z=d["z"], h_in=d["h_in"], y=y, h_out=h_out, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for e0, e1 in evs:
+            flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
+            e0.record(stream); call(); e1.record(stream)
+        torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    nbytes, flops = ssd_bytes(w), ssd_flops(w)
+    peaks = measured_peaks()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    tflops = flops / (ms * 1e-3) / 1e12
+    bf16_peak = peaks.get("bf16_tflops", 1590.0)
+    t_floor = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (bf16_peak * 1e12))
+    return {
+        "metric": "Mamba2 scan (SSD) forward: achieved algorithmic GB/s", "pass": "ssd",
+        "value": round(achieved, 2), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                   "nheads": w.nheads, "headdim": w.headdim, "d_state": w.d_state,
+                   "ngroups": w.ngroups, "gate": w.gate, "initial_state": w.state,
+                   "chunk": SSD_Q, "l2": "flushed between calls", "algorithmic_bytes": nbytes,
+                   "algorithmic_flops": flops},
+        "roofline": {"kernel": "ssd_fwd_kernel", "bound": "hbm", "achieved": round(achieved, 2),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)",
+                     "tensor_tflops": round(tflops, 2), "tensor_frac": round(tflops / bf16_peak, 4),
+                     "tensor_peak_source": "measured cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops)",
+                     "floor_frac": round(t_floor / (ms * 1e-3), 4), "traffic": None},
+        "gpu_launches": args.steps, "clocks": clk.summary(),
+    }
+
+
+def oracle_sample_ssd(w, target_s: float):
+    """The fp64 Mamba2 oracle on a bounded sample: whole sequences of some (row, head)
+    pairs.  Returns (GB/s of the workload's bytes per (row, head), cores, description)."""
+    from oracle import ssd_oracle as so
+    inp = I.make_ssd_inputs(w)
+    pairs = [(b, h) for b in range(w.batch) for h in range(w.nheads)]
+    t0 = time.perf_counter()
+    so.ssd_channels(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"], inp["D"],
+                    inp["dt_bias"], pairs[:1], z=inp["z"], h_in=inp["h_in"])
+    dt = max(time.perf_counter() - t0, 1e-4)
+    n = int(min(len(pairs), max(1, target_s / dt)))
+    sel = pairs[:: max(1, len(pairs) // n)][:n]
+    t0 = time.perf_counter()
+    so.ssd_channels(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"], inp["D"],
+                    inp["dt_bias"], sel, z=inp["z"], h_in=inp["h_in"])
+    el = time.perf_counter() - t0
+    gbs = len(sel) * (ssd_bytes(w) / len(pairs)) / el / 1e9
+    return gbs, 1, (f"{w.name}: {len(sel)} of {len(pairs)} (batch row, head) pairs x L={w.seqlen} "
+                    f"(fp64 numpy oracle, one thread, {el:.2f} s)")
+
+
 # ----------------------------------------------------------------------------- oracle
 def oracle_sample(w: I.Workload, target_s: float):
     """Times the CPU oracle, as it stands, on a bounded sample of the workload: all batch
@@ -620,8 +734,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long", choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
-                    help="bwd: time the backward (mamba_mixer_bwd) alone on the workload")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "ssd"], default="fwd",
+                    help="bwd: time the backward (mamba_mixer_bwd) alone on the workload; "
+                         "ssd: time the Mamba2 scan (mamba2_ssd_fwd) on --ssd-workload")
+    ap.add_argument("--ssd-workload", default="ssd_v3", choices=sorted(I.SSD_WORKLOADS))
     ap.add_argument("--seqlen", type=int, default=None,
                     help="override the workload's sequence length (smaller profiling captures)")
     args = ap.parse_args()
@@ -641,6 +757,21 @@ def main():
         res = run_reference(args, w, rank)
         if res is not None:
             print(json.dumps(res), flush=True)
+        return
+
+    if args.pass_ == "ssd":
+        sw = I.SSD_WORKLOADS[args.ssd_workload]
+        if args.seqlen is not None:
+            import dataclasses
+            sw = dataclasses.replace(sw, seqlen=args.seqlen, name=f"{sw.name}_L{args.seqlen}")
+        if args.steps == 2000:
+            args.steps = 200
+        res = run_ssd(args, sw, local_rank)
+        if not args.no_cpu_baseline:
+            gbs, cores, desc = oracle_sample_ssd(sw, 10.0)
+            res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
+                                   "kind": "oracle", "sample": desc}
+        print(json.dumps(res), flush=True)
         return
 
     if args.pass_ == "bwd":

@@ -1,0 +1,83 @@
+/*
+ * mamba2_ssd.h -- C ABI of the B200 (sm_100a) Mamba2 selective scan (the SSD layer).
+ *
+ * The recurrence is that of the Mamba2 layer whose weight contract niverel-mamba 0.1.0
+ * describes (section "The weight contract": dt_bias, A_log and D hold one value per
+ * head; headdim 64, ngroups 1 and chunk_size 256 in the reference configuration
+ * d_model 768, d_state 128, expand 2), i.e. the Mamba recurrence of calm-mamba 0.1.4
+ * ("Mamba operator") with one scalar A, Delta and D per head and one B/C pair per group
+ * of heads.  For batch row b, head h in group g = h / (nheads / ngroups), channel p < 64,
+ * state n < d_state:
+ *
+ *   Delta_t    = softplus(dt_raw[b,t,h] + dt_bias[h]),   A = -exp(A_log[h])
+ *   h[p, n]   <- exp(Delta_t * A) * h[p, n] + Delta_t * x[b,t,h,p] * B[b,t,g,n]
+ *   y[b,t,h,p] = sum_n C[b,t,g,n] * h[p, n] + D[h] * x[b,t,h,p]
+ *   out        = y * SiLU(z[b,t,h,p])        (only when z is given)
+ *
+ * x is the activation after the layer's causal conv and SiLU; the conv, the projections
+ * and the gated RMSNorm of the full layer stay outside this entry point (with the norm,
+ * pass z = NULL and apply the gate inside the norm).  The state starts from h_in (zero
+ * when NULL).  The computation is chunked (64 steps per chunk) on the tensor cores; the
+ * result equals the sequential recurrence up to rounding (niverel-mamba 0.1.0, section
+ * "Measured tolerances": chunked and sequential evaluation agree).
+ *
+ * Conventions are those of mamba_mixer.h (caller-owned device memory, stream-ordered,
+ * host-side checks before anything is enqueued, mamba_last_error for the message):
+ *
+ *   Layouts   x, z, y       [batch, seqlen, nheads, headdim]    bf16
+ *             dt_raw        [batch, seqlen, nheads]             bf16
+ *             B, C          [batch, seqlen, ngroups, d_state]   bf16
+ *             A_log, D, dt_bias  [nheads]                       fp32
+ *             h_in, h_out   [batch, nheads, headdim, d_state]   fp32
+ *   Support   io_dtype MAMBA_BF16, headdim 64, d_state 64 or 128, ngroups >= 1 dividing
+ *             nheads, batch <= 65535; batch, seqlen or nheads may be 0.
+ *   Numerics  the products run with bf16 operands (the inputs exactly; the masked C B^T,
+ *             the state for the inter-chunk term and Delta-weighted x are rounded once
+ *             to bf16) and fp32 accumulation; the carried state is fp32.
+ *   Errors    MAMBA_ERR_INVALID_ARGUMENT  NULL required pointer, negative size, ngroups
+ *                                         not dividing nheads, an output overlapping an
+ *                                         input (h_out == h_in exactly is allowed)
+ *             MAMBA_ERR_UNSUPPORTED       dtype, headdim, d_state or batch outside the above
+ *             MAMBA_ERR_ALIGNMENT         x, z, y, B, C, h_in or h_out not 16-byte
+ *                                         aligned; dt_raw not 2-byte; A_log, D, dt_bias
+ *                                         not 4-byte aligned
+ *             MAMBA_ERR_CUDA              a launch failed
+ */
+#ifndef MAMBA2_SSD_H_
+#define MAMBA2_SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "mamba_mixer.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct {
+  int64_t batch;
+  int64_t seqlen;
+  int64_t nheads;
+  int64_t headdim;
+  int64_t d_state;
+  int64_t ngroups;
+  int32_t io_dtype; /* mamba_dtype */
+  int32_t reserved; /* set to 0 */
+} mamba2_dims;
+
+/*
+ * Forward of the Mamba2 scan over [0, seqlen).  Writes y (every element) and, when h_out
+ * is not NULL, the state after the last step (h_in when seqlen == 0).  z and h_in may be
+ * NULL.  No workspace: the carried state stays on chip.
+ */
+MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void* dt_raw,
+                             const float* A_log, const void* B, const void* C, const float* D,
+                             const float* dt_bias, const void* z, const float* h_in, void* y,
+                             float* h_out, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA2_SSD_H_ */

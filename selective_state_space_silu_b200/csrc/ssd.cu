@@ -1,0 +1,136 @@
+// mamba2_ssd_fwd: host side of the Mamba2 scan (argument checks and the launch).
+
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "mamba2_ssd.h"
+#include "ssd_kernel.cuh"
+
+namespace mm_internal {
+void set_last_error(const char* msg);  // mamba_mixer.cu: the message mamba_last_error returns
+}
+
+namespace {
+
+int ssd_fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  mm_internal::set_last_error(buf);
+  return code;
+}
+
+int ssd_ok() {
+  mm_internal::set_last_error("");
+  return MAMBA_OK;
+}
+
+int need(const void* p, const char* name, bool required, size_t align) {
+  if (!p) return required ? ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "%s is NULL", name) : MAMBA_OK;
+  if (reinterpret_cast<uintptr_t>(p) % align)
+    return ssd_fail(MAMBA_ERR_ALIGNMENT, "%s is not %zu-byte aligned", name, align);
+  return MAMBA_OK;
+}
+
+struct Range {
+  const void* p;
+  size_t bytes;
+  const char* name;
+};
+
+bool overlap(const Range& a, const Range& b) {
+  if (!a.p || !b.p || !a.bytes || !b.bytes) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.p), b0 = reinterpret_cast<uintptr_t>(b.p);
+  return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
+}
+
+template <int N, bool kGate>
+cudaError_t launch(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
+  auto kern = ssd::ssd_fwd_kernel<N, kGate>;
+  constexpr int smem = ssd::SsdSmem<N>::kBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(unsigned(a.H), unsigned(batch)), ssd::kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void* dt_raw,
+                                        const float* A_log, const void* B, const void* C,
+                                        const float* D, const float* dt_bias, const void* z,
+                                        const float* h_in, void* y, float* h_out,
+                                        void* cuda_stream) {
+  if (!dims) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "dims is NULL");
+  if (dims->reserved != 0) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "dims.reserved must be 0");
+  const int64_t Bt = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
+                N = dims->d_state, G = dims->ngroups;
+  if (Bt < 0 || L < 0 || H < 0 || P < 0 || N < 0 || G < 0)
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "negative size in dims");
+  if (dims->io_dtype != MAMBA_BF16)
+    return ssd_fail(MAMBA_ERR_UNSUPPORTED, "io_dtype %d: only MAMBA_BF16 is supported", dims->io_dtype);
+  if (P != ssd::kP) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "headdim %lld: only 64 is supported", (long long)P);
+  if (N != 64 && N != 128)
+    return ssd_fail(MAMBA_ERR_UNSUPPORTED, "d_state %lld: only 64 and 128 are supported", (long long)N);
+  if (G < 1 || (H > 0 && H % G))
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "ngroups %lld must be >= 1 and divide nheads %lld",
+                    (long long)G, (long long)H);
+  if (Bt > 65535) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "batch %lld > 65535", (long long)Bt);
+  if (H > 0x7fffffff) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "nheads too large");
+  // element counts, checked for overflow of 64-bit byte sizes
+  const double act_d = double(Bt) * double(L) * double(H) * double(P);
+  const double bc_d = double(Bt) * double(L) * double(G) * double(N);
+  if (act_d * 2 > 9e18 || bc_d * 2 > 9e18) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "sizes overflow");
+  const size_t act = size_t(Bt * L * H * P), bc = size_t(Bt * L * G * N), dtn = size_t(Bt * L * H);
+  const size_t state = size_t(Bt * H * P * N);
+  const bool any = act > 0;
+  int rc;
+  if ((rc = need(x, "x", any, 16)) || (rc = need(dt_raw, "dt_raw", any, 2)) ||
+      (rc = need(A_log, "A_log", H > 0, 4)) || (rc = need(B, "B", any, 16)) ||
+      (rc = need(C, "C", any, 16)) || (rc = need(D, "D", H > 0, 4)) ||
+      (rc = need(dt_bias, "dt_bias", H > 0, 4)) || (rc = need(z, "z", false, 16)) ||
+      (rc = need(h_in, "h_in", false, 16)) || (rc = need(y, "y", any, 16)) ||
+      (rc = need(h_out, "h_out", false, 16)))
+    return rc;
+  const Range ins[] = {{x, act * 2, "x"},         {dt_raw, dtn * 2, "dt_raw"}, {A_log, size_t(H) * 4, "A_log"},
+                       {B, bc * 2, "B"},          {C, bc * 2, "C"},            {D, size_t(H) * 4, "D"},
+                       {dt_bias, size_t(H) * 4, "dt_bias"}, {z, act * 2, "z"}};
+  const Range y_r{y, act * 2, "y"}, hin_r{h_in, state * 4, "h_in"}, hout_r{h_out, state * 4, "h_out"};
+  for (const Range& i : ins) {
+    if (overlap(y_r, i) || overlap(hout_r, i))
+      return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "an output overlaps %s", i.name);
+  }
+  if (overlap(y_r, hout_r) || overlap(y_r, hin_r))
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "y overlaps a state buffer");
+  if (overlap(hout_r, hin_r) && h_out != h_in)
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "h_out partially overlaps h_in");
+  if (Bt == 0 || H == 0) return ssd_ok();
+
+  ssd::SsdArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.dt = static_cast<const __nv_bfloat16*>(dt_raw);
+  a.A_log = A_log;
+  a.B = static_cast<const __nv_bfloat16*>(B);
+  a.C = static_cast<const __nv_bfloat16*>(C);
+  a.D = D;
+  a.dt_bias = dt_bias;
+  a.z = static_cast<const __nv_bfloat16*>(z);
+  a.h_in = h_in;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.h_out = h_out;
+  a.L = L;
+  a.H = int(H);
+  a.G = int(G);
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e;
+  if (N == 128)
+    e = z ? launch<128, true>(a, Bt, st) : launch<128, false>(a, Bt, st);
+  else
+    e = z ? launch<64, true>(a, Bt, st) : launch<64, false>(a, Bt, st);
+  if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "ssd launch failed: %s", cudaGetErrorString(e));
+  return ssd_ok();
+}

@@ -237,3 +237,57 @@ def packed_seq_idx(batch: int, L: int, mean_len: int, seed: int) -> np.ndarray:
             lens.append(int(r.geometric(1.0 / mean_len)))
         out[b] = _runs_to_ids(lens)[:L]
     return out
+
+
+# ---------------------------------------------------------------- Mamba2 (SSD) scan
+# niverel-mamba 0.1.0, section "The weight contract": the reference layer has d_model 768,
+# expand 2 (1536 inner channels = 24 heads of headdim 64), d_state 128, ngroups 1, and
+# dt_bias, A_log and D of one value per head.
+@dataclasses.dataclass(frozen=True)
+class SsdWorkload:
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    d_state: int
+    ngroups: int
+    seed: int
+    gate: bool = False      # draw z (the y * SiLU(z) gate of the rmsnorm=False layer)
+    state: bool = False     # draw an initial state h_in
+
+
+SSD_WORKLOADS: Dict[str, SsdWorkload] = {
+    "ssd_tiny": SsdWorkload("ssd_tiny", 2, 100, 4, 64, 64, 1, 2000, gate=True),
+    # the reference layer (24 heads x 64, d_state 128) over 8 rows of 2048 tokens
+    "ssd_v3": SsdWorkload("ssd_v3", 8, 2048, 24, 64, 128, 1, 2001),
+    # the same layer over 2 rows of 8192 tokens (the length the pages certify resets at)
+    "ssd_v3_long": SsdWorkload("ssd_v3_long", 2, 8192, 24, 64, 128, 1, 2002),
+}
+
+
+def make_ssd_inputs(w: SsdWorkload, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Draw every input of Mamba2 scan workload ``w`` (activations as bf16 bit patterns).
+
+    Layouts: x, z [batch, L, nheads, headdim]; dt_raw [batch, L, nheads]; B, C [batch, L,
+    ngroups, d_state]; A_log, D, dt_bias [nheads]; h_in [batch, nheads, headdim, d_state].
+    Draw order x, dt_raw, B, C, then z, dt_bias, A, h_in (PCG64(seed), float32):
+    x, B, C, z ~ N(0, 1) (x stands in for the post-conv activation); dt_raw ~ N(0, 0.5);
+    dt0 log-uniform on [1e-3, 1e-1] per head and dt_bias = log(expm1(dt0)); A ~ U(1, 16)
+    per head and A_log = ln(A); D = 1; h_in ~ N(0, 1) fp32.
+    """
+    rng = np.random.Generator(np.random.PCG64(w.seed if seed is None else seed))
+    Bt, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.d_state, w.ngroups
+    out: Dict[str, np.ndarray] = {}
+    out["x"] = f32_to_bf16_bits(_normal(rng, (Bt, L, H, P)))
+    out["dt_raw"] = f32_to_bf16_bits(_normal(rng, (Bt, L, H), std=0.5))
+    out["B"] = f32_to_bf16_bits(_normal(rng, (Bt, L, G, N)))
+    out["C"] = f32_to_bf16_bits(_normal(rng, (Bt, L, G, N)))
+    out["z"] = f32_to_bf16_bits(_normal(rng, (Bt, L, H, P))) if w.gate else None
+    lo, hi = np.log(1e-3), np.log(1e-1)
+    dt0 = np.exp(rng.uniform(lo, hi, size=H))
+    out["dt_bias"] = np.log(np.expm1(dt0)).astype(np.float32)
+    out["A_log"] = np.log(rng.uniform(1.0, 16.0, size=H)).astype(np.float32)
+    out["D"] = np.ones(H, dtype=np.float32)
+    out["h_in"] = _normal(rng, (Bt, H, P, N)) if w.state else None
+    return out

@@ -1,0 +1,72 @@
+"""Python binding of the Mamba2 scan entry point (include/mamba2_ssd.h) in libmamba_mixer.so.
+
+Argument marshalling only: every step of the computation runs in the library's CUDA
+kernel.  The library is the one mixer.load_library() loads; its absence is an error.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import mixer as _m
+
+EXPORTS = ("mamba2_ssd_fwd",)
+
+
+class mamba2_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("nheads", ctypes.c_int64), ("headdim", ctypes.c_int64),
+                ("d_state", ctypes.c_int64), ("ngroups", ctypes.c_int64),
+                ("io_dtype", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_bound = None
+
+
+def _lib() -> ctypes.CDLL:
+    global _bound
+    lib = _m.load_library()
+    if _bound is not lib:
+        vp = ctypes.c_void_p
+        lib.mamba2_ssd_fwd.restype = ctypes.c_int
+        lib.mamba2_ssd_fwd.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 12
+        _bound = lib
+    return lib
+
+
+def make_dims(batch, seqlen, nheads, headdim, d_state, ngroups, io_dtype=_m.MAMBA_BF16) -> mamba2_dims:
+    return mamba2_dims(int(batch), int(seqlen), int(nheads), int(headdim), int(d_state),
+                       int(ngroups), int(io_dtype), 0)
+
+
+def mamba2_ssd_fwd(x, dt_raw, A_log, B, C, D, dt_bias, *, z=None, h_in=None, y=None,
+                   h_out=None, want_state: bool = True, stream=None
+                   ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Mamba2 scan forward.  Shapes: x (and z) [batch, L, nheads, 64] bf16; dt_raw
+    [batch, L, nheads] bf16; B, C [batch, L, ngroups, d_state] bf16; A_log, D, dt_bias
+    [nheads] fp32; h_in [batch, nheads, 64, d_state] fp32 or None.  Returns (y, h_out)
+    (h_out None when want_state is False)."""
+    lib = _lib()
+    dev = x.device
+    Bt, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = _m._io_code(x)
+    iot = x.dtype
+    f32 = torch.float32
+    if y is None:
+        y = torch.empty_like(x)
+    if h_out is None and want_state:
+        h_out = torch.empty(Bt, H, P, N, dtype=f32, device=dev)
+    dims = make_dims(Bt, L, H, P, N, G, io)
+    p = _m._ptr
+    rc = lib.mamba2_ssd_fwd(
+        ctypes.byref(dims), p(x, "x", iot, dev), p(dt_raw, "dt_raw", iot, dev),
+        p(A_log, "A_log", f32, dev), p(B, "B", iot, dev), p(C, "C", iot, dev),
+        p(D, "D", f32, dev), p(dt_bias, "dt_bias", f32, dev), p(z, "z", iot, dev),
+        p(h_in, "h_in", f32, dev), p(y, "y", iot, dev), p(h_out, "h_out", f32, dev),
+        _m._stream_handle(stream, dev))
+    _m._check(rc)
+    return y, h_out

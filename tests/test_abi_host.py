@@ -15,6 +15,7 @@ import pytest
 
 from selective_state_space_silu_b200 import build as B
 from selective_state_space_silu_b200 import mixer as M
+from selective_state_space_silu_b200 import ssd as SSD
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -29,16 +30,17 @@ def declared_symbols():
     names = set()
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         src = open(h).read()
-        names |= set(re.findall(r"MAMBA_API\s+[\w\s\*]+?\b(mamba_\w+)\s*\(", src))
+        names |= set(re.findall(r"MAMBA_API\s+[\w\s\*]+?\b(mamba2?_\w+)\s*\(", src))
     return names
 
 
 def test_exports_every_declared_symbol(lib):
     names = declared_symbols()
     assert set(M.EXPORTS) <= names
+    assert set(SSD.EXPORTS) <= names
     out = subprocess.run(["nm", "-D", "--defined-only", M.LIB_PATH], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\sT\s(mamba_\w+)", out))
+    exported = set(re.findall(r"\sT\s(mamba2?_\w+)", out))
     assert names <= exported, names - exported
     for n in names:
         assert hasattr(lib, n)

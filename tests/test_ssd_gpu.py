@@ -1,0 +1,110 @@
+"""Parity of the Mamba2 scan (mamba2_ssd_fwd, CUDA, through the C ABI) with the fp64 oracle.
+
+Shapes span several 64-step chunks with ragged tails, both supported d_state values, one
+and several groups, the gate, an initial state (also updated in place), the empty and
+single-step sequences, and the reference layer (24 heads x 64, d_state 128) at full size
+on sampled (batch row, head) pairs.  Tolerance: tests/tolerances.py assert_close_tc.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import ssd_oracle as so
+from selective_state_space_silu_b200 import inputs as I
+from selective_state_space_silu_b200 import ssd as S
+from tests.gpu_util import dev_tensor, host
+from tests.tolerances import assert_close_tc
+
+pytestmark = pytest.mark.gpu
+
+
+def draw(Bt, L, H, N, G, gate, state, seed):
+    w = I.SsdWorkload("case", Bt, L, H, 64, N, G, seed, gate=gate, state=state)
+    return I.make_ssd_inputs(w)
+
+
+def run_gpu(inp, h_in_inplace=False):
+    d = {k: (None if v is None else dev_tensor(v)) for k, v in inp.items()}
+    h_out = d["h_in"] if h_in_inplace else None
+    y, h = S.mamba2_ssd_fwd(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"],
+                            d["dt_bias"], z=d["z"], h_in=d["h_in"], h_out=h_out)
+    torch.cuda.synchronize()
+    return host(y), host(h)
+
+
+def run_oracle(inp):
+    return so.ssd(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"], inp["D"],
+                  inp["dt_bias"], z=inp["z"], h_in=inp["h_in"])
+
+
+CASES = [
+    # Bt, L, H, N, G, gate, state
+    (2, 100, 4, 64, 1, True, False),
+    (1, 257, 3, 128, 1, False, True),
+    (2, 64, 4, 128, 2, True, True),
+    (1, 63, 2, 128, 1, False, False),
+    (3, 130, 6, 64, 3, True, False),
+    (1, 1, 2, 64, 1, True, True),
+    (2, 200, 8, 128, 4, False, False),
+    (1, 640, 2, 128, 1, True, True),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(map(str, c)))
+def test_ssd_matches_oracle(case):
+    Bt, L, H, N, G, gate, state = case
+    inp = draw(Bt, L, H, N, G, gate, state, seed=3000 + sum(case[:5]))
+    y, h = run_gpu(inp)
+    yo, ho = run_oracle(inp)
+    assert_close_tc(y, yo, "y")
+    assert_close_tc(h, ho, "h_out")
+
+
+def test_state_in_place():
+    inp = draw(2, 150, 4, 128, 1, False, True, seed=3100)
+    yo, ho = run_oracle(inp)
+    y, h = run_gpu(inp, h_in_inplace=True)
+    assert_close_tc(y, yo, "y")
+    assert_close_tc(h, ho, "h_out in place")
+
+
+def test_empty_sequence_passes_state_through():
+    inp = draw(2, 0, 4, 64, 1, True, True, seed=3200)
+    y, h = run_gpu(inp)
+    assert y.size == 0
+    assert np.array_equal(h, inp["h_in"].astype(np.float64))
+    inp["h_in"] = None
+    _, h = run_gpu(inp)
+    assert np.array_equal(h, np.zeros_like(h))
+
+
+def test_prefix_then_continue():
+    # a sequence split at a non-chunk boundary: the second call starts from the first's state
+    inp = draw(1, 300, 4, 128, 1, True, False, seed=3300)
+    yo, ho = run_oracle(inp)
+    cut = 137
+    first = {k: (v[:, :cut] if k in ("x", "dt_raw", "B", "C", "z") else v) for k, v in inp.items()}
+    y1, h1 = run_gpu(first)
+    second = {k: (np.ascontiguousarray(v[:, cut:]) if k in ("x", "dt_raw", "B", "C", "z") else v)
+              for k, v in inp.items()}
+    second["h_in"] = h1.astype(np.float32)
+    y2, h2 = run_gpu(second)
+    assert_close_tc(np.concatenate([y1, y2], axis=1), yo, "y (two calls)")
+    assert_close_tc(h2, ho, "h_out (two calls)")
+
+
+@pytest.mark.parametrize("name", ["ssd_v3", "ssd_v3_long"])
+def test_reference_layer_full_size_sampled(name):
+    w = I.SSD_WORKLOADS[name]
+    inp = I.make_ssd_inputs(w)
+    y, h = run_gpu(inp)
+    assert np.isfinite(y).all() and np.isfinite(h).all()
+    rng = np.random.default_rng(7)
+    sel = [(int(rng.integers(w.batch)), int(rng.integers(w.nheads))) for _ in range(4)]
+    sel += [(0, 0), (w.batch - 1, w.nheads - 1)]
+    outs, hs = so.ssd_channels(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"],
+                               inp["D"], inp["dt_bias"], sel, z=inp["z"], h_in=inp["h_in"])
+    for (b, hh), o, hf in zip(sel, outs, hs):
+        assert_close_tc(y[b, :, hh], o, f"y[{b}, :, {hh}]")
+        assert_close_tc(h[b, hh], hf, f"h_out[{b}, {hh}]")

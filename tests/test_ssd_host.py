@@ -1,0 +1,86 @@
+"""Host-side checks of mamba2_ssd_fwd: argument validation before anything is enqueued.
+
+Nothing here launches a kernel: every call fails validation (before the first CUDA call)
+or has nothing to do (batch 0 or nheads 0).
+"""
+
+import ctypes
+
+import pytest
+
+from selective_state_space_silu_b200 import build as Bld
+from selective_state_space_silu_b200 import mixer as M
+from selective_state_space_silu_b200 import ssd as S
+
+NAMES = ["x", "dt", "A_log", "B", "C", "D", "dt_bias", "z", "h_in", "y", "h_out"]
+
+
+@pytest.fixture(scope="module")
+def lib():
+    Bld.build()
+    return S._lib()
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def _call(lib, dims, ptrs=None):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(NAMES)}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba2_ssd_fwd(ctypes.byref(dims) if dims is not None else None,
+                              *[p[k] for k in NAMES], None)
+
+
+def dims(**kw):
+    a = dict(batch=2, seqlen=100, nheads=4, headdim=64, d_state=128, ngroups=1,
+             io_dtype=M.MAMBA_BF16)
+    a.update(kw)
+    return S.make_dims(**a)
+
+
+def test_unsupported_and_invalid_dims(lib):
+    for kw, code in [(dict(io_dtype=M.MAMBA_F32), 2), (dict(headdim=32), 2),
+                     (dict(d_state=16), 2), (dict(d_state=256), 2), (dict(batch=70000), 2),
+                     (dict(ngroups=3), 1), (dict(ngroups=0), 1), (dict(seqlen=-1), 1),
+                     (dict(nheads=-4), 1)]:
+        rc = _call(lib, dims(**kw))
+        assert rc == code, (kw, rc, M.mamba_last_error())
+        assert M.mamba_last_error()
+
+
+def test_null_dims_and_reserved(lib):
+    assert _call(lib, None) == 1
+    d = dims()
+    d.reserved = 5
+    assert _call(lib, d) == 1
+    assert "reserved" in M.mamba_last_error()
+
+
+def test_null_required_pointers(lib):
+    for k in ("x", "dt", "A_log", "B", "C", "D", "dt_bias", "y"):
+        assert _call(lib, dims(), {k: None}) == 1, k
+        assert k.replace("dt", "dt_raw") in M.mamba_last_error() or k in M.mamba_last_error()
+
+
+def test_misaligned_pointers(lib):
+    assert _call(lib, dims(), {"x": _fake(0x10000008)}) == 3
+    assert _call(lib, dims(), {"B": _fake(0x3010000004)}) == 3
+    assert _call(lib, dims(), {"dt": _fake(0x1010000001)}) == 3
+    assert _call(lib, dims(), {"D": _fake(0x5010000002)}) == 3
+    assert _call(lib, dims(), {"h_out": _fake(0xa010000008)}) == 3
+
+
+def test_overlaps_rejected(lib):
+    assert _call(lib, dims(), {"y": _fake(0x10000000)}) == 1            # y on top of x
+    assert _call(lib, dims(), {"h_out": _fake(0x9010000000)}) == 1      # h_out inside y
+    # h_out == h_in exactly is in-place and allowed at validation; partial overlap is not
+    assert _call(lib, dims(), {"h_out": _fake(0x8010000010)}) == 1
+    assert "partially" in M.mamba_last_error()
+
+
+def test_nothing_to_do(lib):
+    assert _call(lib, dims(batch=0)) == 0
+    assert _call(lib, dims(nheads=0), {k: None for k in ("A_log", "D", "dt_bias")}) == 0

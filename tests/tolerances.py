@@ -89,3 +89,18 @@ def assert_close_grad(a, b, io_dtype, what=""):
             f"{what}: {100 * (1 - ok.mean()):.4f}% outside the {io_dtype} gradient tolerance "
             f"(max_abs {np.nanmax(d):.3e}, oracle rms {np.sqrt(np.mean(b ** 2)):.3e}); first at "
             f"{idx}: got {a[idx]!r}, oracle {b[idx]!r}")
+
+
+def assert_close_tc(a, b, what=""):
+    """Tolerance for the Mamba2 scan's tensor-core path (bf16 operands, fp32 sums) against
+    the fp64 oracle: abs(a-b) <= 1e-3 + 2e-2*max(|a|,|b|) + 2e-2*RMS(oracle tensor).
+
+    Derivation: besides the bf16 output rounding (the 2e-2 relative term), each output
+    is a sum of many products whose operands include values rounded once to bf16 (relative
+    error at most 2^-9, about 1.1e-3 RMS for round-to-nearest): the masked C B^T entries,
+    the carried state used for the inter-chunk term, and the Delta-weighted x of the state
+    update.  The error of such a sum is about 2^-9/sqrt(3) times the root of the summed
+    squares of its terms, which for terms of both signs is of the order of the output's
+    RMS: about 1.1e-3 RMS per rounded operand set, under 6e-3 RMS at five standard
+    deviations for the two sets that meet in one output.  2e-2 RMS leaves a factor of 3 over that."""
+    assert_close_grad(a, b, "bf16", what)
