@@ -764,8 +764,6 @@ def main():
         if args.seqlen is not None:
             import dataclasses
             sw = dataclasses.replace(sw, seqlen=args.seqlen, name=f"{sw.name}_L{args.seqlen}")
-        if args.steps == 2000:
-            args.steps = 200
         res = run_ssd(args, sw, local_rank)
         if not args.no_cpu_baseline:
             gbs, cores, desc = oracle_sample_ssd(sw, 10.0)

@@ -19,13 +19,15 @@
  * pass z = NULL and apply the gate inside the norm).  The state starts from h_in (zero
  * when NULL).  The computation is chunked (64 steps per chunk) on the tensor cores; the
  * result equals the sequential recurrence up to rounding (niverel-mamba 0.1.0, section
- * "Measured tolerances": chunked and sequential evaluation agree).
+ * "Measured tolerances": chunked and sequential evaluation agree).  Long sequences of few
+ * (batch row, head) pairs are also cut into time segments (see the workspace below).
  *
  * Conventions are those of mamba_mixer.h (caller-owned device memory, stream-ordered,
  * host-side checks before anything is enqueued, mamba_last_error for the message):
  *
  *   Layouts   x, z, y       [batch, seqlen, nheads, headdim]    bf16
  *             dt_raw        [batch, seqlen, nheads]             bf16
+ *             seq_idx       [batch, seqlen]                     int32
  *             B, C          [batch, seqlen, ngroups, d_state]   bf16
  *             A_log, D, dt_bias  [nheads]                       fp32
  *             h_in, h_out   [batch, nheads, headdim, d_state]   fp32
@@ -39,8 +41,10 @@
  *                                         input (h_out == h_in exactly is allowed)
  *             MAMBA_ERR_UNSUPPORTED       dtype, headdim, d_state or batch outside the above
  *             MAMBA_ERR_ALIGNMENT         x, z, y, B, C, h_in or h_out not 16-byte
- *                                         aligned; dt_raw not 2-byte; A_log, D, dt_bias
- *                                         not 4-byte aligned
+ *                                         aligned; dt_raw not 2-byte; A_log, D, dt_bias,
+ *                                         seq_idx not 4-byte aligned
+ *             MAMBA_ERR_WORKSPACE         workspace missing, too small, or not 256-byte
+ *                                         aligned
  *             MAMBA_ERR_CUDA              a launch failed
  */
 #ifndef MAMBA2_SSD_H_
@@ -67,14 +71,30 @@ typedef struct {
 } mamba2_dims;
 
 /*
+ * Device workspace, in bytes, that mamba2_ssd_fwd needs for `dims` (0 for invalid dims, and
+ * 0 when the sequence is not split).  With few (batch row, head) pairs the sequence of each
+ * pair is cut into time segments that run in parallel: a state pass leaves each segment's
+ * end state (fp32, headdim x d_state) and summed decay exponent here, with a copy of h_in,
+ * and the main pass starts every segment from the earlier ones folded together.
+ */
+MAMBA_API size_t mamba2_ssd_fwd_workspace_bytes(const mamba2_dims* dims);
+
+/*
  * Forward of the Mamba2 scan over [0, seqlen).  Writes y (every element) and, when h_out
- * is not NULL, the state after the last step (h_in when seqlen == 0).  z and h_in may be
- * NULL.  No workspace: the carried state stays on chip.
+ * is not NULL, the state after the last step (h_in when seqlen == 0).  z, seq_idx and
+ * h_in may be NULL.  seq_idx [batch, seqlen] int32 packs documents into rows: the state is
+ * zeroed before every step t > 0 whose id differs from step t - 1's (niverel-mamba 0.1.0,
+ * section "seq_idx strict reset"), so h_in belongs to the row's first document and h_out
+ * to its last.  workspace: device memory of at least mamba2_ssd_fwd_workspace_bytes(dims) bytes,
+ * 256-byte aligned, overlapping no other argument (may be NULL when that size is 0);
+ * fully rewritten by every call, nothing needs clearing.  MAMBA_ERR_WORKSPACE when it is
+ * missing or too small.
  */
 MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void* dt_raw,
                              const float* A_log, const void* B, const void* C, const float* D,
-                             const float* dt_bias, const void* z, const float* h_in, void* y,
-                             float* h_out, void* cuda_stream);
+                             const float* dt_bias, const void* z, const int32_t* seq_idx,
+                             const float* h_in, void* y, float* h_out, void* workspace,
+                             size_t workspace_bytes, void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -48,23 +48,68 @@ bool overlap(const Range& a, const Range& b) {
   return a0 < b0 + b.bytes && b0 < a0 + a.bytes;
 }
 
-template <int N, bool kGate>
-cudaError_t launch(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
-  auto kern = ssd::ssd_fwd_kernel<N, kGate>;
-  constexpr int smem = ssd::SsdSmem<N>::kBytes;
+// Time segments: with few (batch row, head) pairs, each pair's chunks are cut into
+// segments that run as separate CTAs (a state pass over segments 0 .. nseg - 2 first).
+// Target: about two waves of the main pass at two CTAs per SM on the 148 SMs.
+struct SegPlan {
+  int nseg, cps;
+};
+
+constexpr int64_t kSms = 148;
+
+SegPlan seg_plan(int64_t Bt, int64_t L, int64_t H) {
+  const int64_t nchunks = (L + ssd::kQ - 1) / ssd::kQ;
+  const int64_t pairs = Bt * H;
+  const int64_t target = 4 * kSms;
+  int64_t nseg = 1;
+  if (pairs > 0 && nchunks > 1 && pairs < target) nseg = (target + pairs / 2) / pairs;
+  if (nseg > 16) nseg = 16;
+  if (nseg > nchunks) nseg = nchunks;
+  if (nseg < 1) nseg = 1;
+  const int64_t cps = nchunks > 0 ? (nchunks + nseg - 1) / nseg : 1;
+  nseg = nchunks > 0 ? (nchunks + cps - 1) / cps : 1;
+  return {int(nseg), int(cps)};
+}
+
+// nseg state slots per (row, head) -- nseg - 1 segment end states and the copy of h_in --
+// then nseg - 1 floats per (row, head)
+size_t ws_h_bytes(int64_t Bt, int64_t H, int64_t N, const SegPlan& sp) {
+  return size_t(Bt * H) * size_t(sp.nseg) * size_t(ssd::kP * N) * 4;
+}
+
+size_t ws_bytes_for(int64_t Bt, int64_t H, int64_t N, const SegPlan& sp) {
+  if (sp.nseg <= 1) return 0;
+  const size_t nA = size_t(Bt * H) * size_t(sp.nseg - 1);
+  return ws_h_bytes(Bt, H, N, sp) + ((nA * 4 + 255) / 256) * 256;
+}
+
+template <int N, bool kGate, bool kPre, bool kSeq>
+cudaError_t launch_one(const ssd::SsdArgs& a, int64_t batch, int nz, cudaStream_t st) {
+  auto kern = ssd::ssd_fwd_kernel<N, kGate, kPre, kSeq>;
+  constexpr int smem = ssd::SsdSmem<N, kPre>::kBytes;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(unsigned(a.H), unsigned(batch)), ssd::kThreads, smem, st>>>(a);
+  kern<<<dim3(unsigned(a.H), unsigned(batch), unsigned(nz)), ssd::kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
-}  // namespace
+template <int N, bool kGate, bool kSeq>
+cudaError_t launch(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
+  if (a.nseg > 1) {
+    cudaError_t e = launch_one<N, false, true, kSeq>(a, batch, a.nseg - 1, st);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_one<N, kGate, false, kSeq>(a, batch, a.nseg, st);
+}
 
-extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void* dt_raw,
-                                        const float* A_log, const void* B, const void* C,
-                                        const float* D, const float* dt_bias, const void* z,
-                                        const float* h_in, void* y, float* h_out,
-                                        void* cuda_stream) {
+template <int N>
+cudaError_t launch_n(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
+  if (a.z)
+    return a.seq_idx ? launch<N, true, true>(a, batch, st) : launch<N, true, false>(a, batch, st);
+  return a.seq_idx ? launch<N, false, true>(a, batch, st) : launch<N, false, false>(a, batch, st);
+}
+
+int check_dims(const mamba2_dims* dims) {
   if (!dims) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "dims is NULL");
   if (dims->reserved != 0) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "dims.reserved must be 0");
   const int64_t Bt = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
@@ -81,24 +126,46 @@ extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, 
                     (long long)G, (long long)H);
   if (Bt > 65535) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "batch %lld > 65535", (long long)Bt);
   if (H > 0x7fffffff) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "nheads too large");
-  // element counts, checked for overflow of 64-bit byte sizes
   const double act_d = double(Bt) * double(L) * double(H) * double(P);
   const double bc_d = double(Bt) * double(L) * double(G) * double(N);
   if (act_d * 2 > 9e18 || bc_d * 2 > 9e18) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "sizes overflow");
+  return MAMBA_OK;
+}
+
+}  // namespace
+
+extern "C" MAMBA_API size_t mamba2_ssd_fwd_workspace_bytes(const mamba2_dims* dims) {
+  if (check_dims(dims) != MAMBA_OK) return 0;
+  const SegPlan sp = seg_plan(dims->batch, dims->seqlen, dims->nheads);
+  return ws_bytes_for(dims->batch, dims->nheads, dims->d_state, sp);
+}
+
+extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void* dt_raw,
+                                        const float* A_log, const void* B, const void* C,
+                                        const float* D, const float* dt_bias, const void* z,
+                                        const int32_t* seq_idx, const float* h_in, void* y,
+                                        float* h_out,
+                                        void* workspace, size_t workspace_bytes,
+                                        void* cuda_stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const int64_t Bt = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
+                N = dims->d_state, G = dims->ngroups;
   const size_t act = size_t(Bt * L * H * P), bc = size_t(Bt * L * G * N), dtn = size_t(Bt * L * H);
   const size_t state = size_t(Bt * H * P * N);
   const bool any = act > 0;
-  int rc;
   if ((rc = need(x, "x", any, 16)) || (rc = need(dt_raw, "dt_raw", any, 2)) ||
       (rc = need(A_log, "A_log", H > 0, 4)) || (rc = need(B, "B", any, 16)) ||
       (rc = need(C, "C", any, 16)) || (rc = need(D, "D", H > 0, 4)) ||
       (rc = need(dt_bias, "dt_bias", H > 0, 4)) || (rc = need(z, "z", false, 16)) ||
+      (rc = need(seq_idx, "seq_idx", false, 4)) ||
       (rc = need(h_in, "h_in", false, 16)) || (rc = need(y, "y", any, 16)) ||
       (rc = need(h_out, "h_out", false, 16)))
     return rc;
   const Range ins[] = {{x, act * 2, "x"},         {dt_raw, dtn * 2, "dt_raw"}, {A_log, size_t(H) * 4, "A_log"},
                        {B, bc * 2, "B"},          {C, bc * 2, "C"},            {D, size_t(H) * 4, "D"},
-                       {dt_bias, size_t(H) * 4, "dt_bias"}, {z, act * 2, "z"}};
+                       {dt_bias, size_t(H) * 4, "dt_bias"}, {z, act * 2, "z"},
+                       {seq_idx, size_t(Bt * L) * 4, "seq_idx"}};
   const Range y_r{y, act * 2, "y"}, hin_r{h_in, state * 4, "h_in"}, hout_r{h_out, state * 4, "h_out"};
   for (const Range& i : ins) {
     if (overlap(y_r, i) || overlap(hout_r, i))
@@ -108,6 +175,19 @@ extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, 
     return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "y overlaps a state buffer");
   if (overlap(hout_r, hin_r) && h_out != h_in)
     return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "h_out partially overlaps h_in");
+  const SegPlan sp = seg_plan(Bt, L, H);
+  const size_t need = ws_bytes_for(Bt, H, N, sp);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need)
+      return ssd_fail(MAMBA_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", workspace_bytes, need);
+    if (reinterpret_cast<uintptr_t>(workspace) % 256)
+      return ssd_fail(MAMBA_ERR_ALIGNMENT, "workspace is not 256-byte aligned");
+    const Range ws_r{workspace, need, "workspace"};
+    for (const Range& i : ins)
+      if (overlap(ws_r, i)) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "workspace overlaps %s", i.name);
+    if (overlap(ws_r, y_r) || overlap(ws_r, hin_r) || overlap(ws_r, hout_r))
+      return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "workspace overlaps an output or the state");
+  }
   if (Bt == 0 || H == 0) return ssd_ok();
 
   ssd::SsdArgs a{};
@@ -120,17 +200,21 @@ extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, 
   a.dt_bias = dt_bias;
   a.z = static_cast<const __nv_bfloat16*>(z);
   a.h_in = h_in;
+  a.seq_idx = seq_idx;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.h_out = h_out;
   a.L = L;
   a.H = int(H);
   a.G = int(G);
+  a.nseg = sp.nseg;
+  a.cps = sp.cps;
+  if (sp.nseg > 1) {
+    a.ws_H = static_cast<float*>(workspace);
+    a.ws_A = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + ws_h_bytes(Bt, H, N, sp));
+  }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e;
-  if (N == 128)
-    e = z ? launch<128, true>(a, Bt, st) : launch<128, false>(a, Bt, st);
-  else
-    e = z ? launch<64, true>(a, Bt, st) : launch<64, false>(a, Bt, st);
+  e = N == 128 ? launch_n<128>(a, Bt, st) : launch_n<64>(a, Bt, st);
   if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "ssd launch failed: %s", cudaGetErrorString(e));
   return ssd_ok();
 }

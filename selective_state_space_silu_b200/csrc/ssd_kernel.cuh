@@ -65,26 +65,38 @@ struct SsdArgs {
   const float* dt_bias;     // [H]
   const __nv_bfloat16* z;   // [Bt, L, H, P] or null
   const float* h_in;        // [Bt, H, P, N] or null
+  const int32_t* seq_idx;   // [Bt, L] or null: the state resets where the id changes
   __nv_bfloat16* y;         // [Bt, L, H, P]
   float* h_out;             // [Bt, H, P, N] or null
+  // time segments: CTA z covers chunks [z cps, (z + 1) cps); segments 0 .. nseg - 2 leave
+  // their local end state (from zero) and summed Delta A log2 e in the workspace; slot
+  // nseg - 1 of ws_H holds a copy of h_in made by the state pass, so that the main pass
+  // never reads h_in while its last segment writes h_out (which may be the same buffer)
+  float* ws_H;              // [Bt, H, nseg, P, N]
+  float* ws_A;              // [Bt, H, nseg - 1]
   int64_t L;
   int H, G;
+  int nseg, cps;
 };
 
-// Shared memory: two stages of (C, B, x) chunk tiles, then the masked C B^T (hi and lo
-// planes), w o x, cs and Delta.
-template <int N>
+// Shared memory: two stages of (C, B, x) chunk tiles (B and x only for the state pass),
+// then the masked C B^T (hi and lo planes; main pass only), w o x, cs, Delta and the
+// in-chunk reset positions.
+template <int N, bool kPre>
 struct SsdSmem {
   static constexpr int kBC = kQ * N * 2;
   static constexpr int kX = kQ * kP * 2;
-  static constexpr int kStage = 2 * kBC + kX;  // C at 0, B at kBC, x at 2 kBC
-  static constexpr int kG = kQ * kQ * 2;       // one bf16 plane of the 64 x 64 matrix
+  static constexpr int kOffB = kPre ? 0 : kBC;  // within a stage; C at 0 (main pass)
+  static constexpr int kOffX = kOffB + kBC;
+  static constexpr int kStage = kOffX + kX;
+  static constexpr int kG = kPre ? 0 : kQ * kQ * 2;  // one bf16 plane of the 64 x 64 matrix
   static constexpr int kOffGhi = 2 * kStage;
   static constexpr int kOffGlo = kOffGhi + kG;
   static constexpr int kOffXw = kOffGlo + kG;
   static constexpr int kOffCs = kOffXw + kQ * kP * 2;
   static constexpr int kOffDl = kOffCs + kQ * 4;
-  static constexpr int kBytes = kOffDl + kQ * 4;
+  static constexpr int kOffRs = kOffDl + kQ * 4;  // int: last reset position <= t, or -1
+  static constexpr int kBytes = kOffRs + kQ * 4;
 };
 
 // The causal 16 x 16 blocks (t block, s block) of the chunk's 64 x 64 matrix, by warp.
@@ -171,10 +183,24 @@ __device__ __forceinline__ void sts_u128(uint32_t a, uint4 v) {
                ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
-// Grid (H, Bt); kThreads threads; SsdSmem<N>::kBytes of dynamic shared memory.
-template <int N, bool kGate>
-__global__ void __launch_bounds__(kThreads, 2) ssd_fwd_kernel(const SsdArgs a) {
-  using S = SsdSmem<N>;
+// Grid (H, Bt, nseg) -- (H, Bt, nseg - 1) for the state pass; kThreads threads;
+// SsdSmem<N, kPre>::kBytes of dynamic shared memory.
+//
+// kPre (state pass): run segment z from a zero state over B and x only and leave its end
+// state and its summed Delta A in the workspace.  Main pass: start segment z from h_in
+// (zero when absent) folded with the end states of segments 0 .. z - 1,
+//   H <- 2^(sum of segment s's Delta A log2 e) H + H_s,
+// produce y for the segment's chunks, and (last segment) write h_out.
+//
+// kSeq (documents, niverel-mamba 0.1.0, section "seq_idx strict reset"): the state is
+// zeroed before every step t > 0 whose seq_idx differs from step t - 1's.  With rs_t the
+// last reset position <= t inside the chunk (-1 for none): M[t, s] keeps only s >= rs_t,
+// the inter-chunk term of step t only when rs_t < 0, the state update only steps
+// s >= rs_last, and the carried state decays by 0 instead of 2^cs_last when the chunk holds
+// a reset; a segment holding a reset folds with factor 0.
+template <int N, bool kGate, bool kPre, bool kSeq>
+__global__ void __launch_bounds__(kThreads, kPre ? 4 : 2) ssd_fwd_kernel(const SsdArgs a) {
+  using S = SsdSmem<N, kPre>;
   constexpr int R = N / 8;   // 16-byte pieces per row of B and C
   constexpr int NT = N / 8;  // 8-column tiles of the state
   static_assert(N % 16 == 0 && R >= 8, "d_state must be a multiple of 16, at least 64");
@@ -183,37 +209,66 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_fwd_kernel(const SsdArgs a) {
   const uint32_t sGhi = sbase + S::kOffGhi, sGlo = sbase + S::kOffGlo, sXw = sbase + S::kOffXw;
   float* cs2 = reinterpret_cast<float*>(smem + S::kOffCs);  // in-chunk cumsum of Delta A log2 e
   float* dls = reinterpret_cast<float*>(smem + S::kOffDl);  // Delta
+  int* rsp = reinterpret_cast<int*>(smem + S::kOffRs);      // last reset position <= t, or -1
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, tig = lane & 3;  // mma fragment row / column pair
   const int mi = lane >> 3, ri = lane & 7;  // ldmatrix: matrix and row this lane addresses
   const int h = blockIdx.x;
   const int64_t b = blockIdx.y;
+  const int seg = blockIdx.z;
   const int grp = h / (a.H / a.G);
   const int64_t L = a.L;
   const int64_t nchunks = (L + kQ - 1) / kQ;
+  const int64_t c_begin = int64_t(seg) * a.cps;
+  const int64_t c_end = c_begin + a.cps < nchunks ? c_begin + a.cps : nchunks;
   const float A2 = -expf(a.A_log[h]) * mm::kLog2e;  // A log2(e)
   const float bias = a.dt_bias[h];
-  const float Dh = a.D[h];
-  const bool has_h_in = a.h_in != nullptr;
+  const bool has_h_in = !kPre && a.h_in != nullptr;
+  const int64_t bh = b * a.H + h;
 
   // H: rows p0 = 16 warp + g and p0 + 8, columns n = 8 j + 2 tig (+1)
   const int p0 = 16 * warp + g;
   float hacc[NT][4];
-  {
-    const float* hi = has_h_in ? a.h_in + (b * a.H + h) * int64_t(kP * N) : nullptr;
 #pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      float2 v0 = make_float2(0.f, 0.f), v1 = v0;
-      if (has_h_in) {
-        v0 = *reinterpret_cast<const float2*>(hi + p0 * N + 8 * j + 2 * tig);
-        v1 = *reinterpret_cast<const float2*>(hi + (p0 + 8) * N + 8 * j + 2 * tig);
+  for (int j = 0; j < NT; ++j) hacc[j][0] = hacc[j][1] = hacc[j][2] = hacc[j][3] = 0.f;
+  if constexpr (kPre) {
+    if (seg == 0 && a.h_in) {  // the copy of h_in the main pass starts from
+      const float* hi = a.h_in + bh * int64_t(kP * N);
+      float* hc = a.ws_H + (bh * a.nseg + a.nseg - 1) * int64_t(kP * N);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        *reinterpret_cast<float2*>(hc + p0 * N + 8 * j + 2 * tig) =
+            *reinterpret_cast<const float2*>(hi + p0 * N + 8 * j + 2 * tig);
+        *reinterpret_cast<float2*>(hc + (p0 + 8) * N + 8 * j + 2 * tig) =
+            *reinterpret_cast<const float2*>(hi + (p0 + 8) * N + 8 * j + 2 * tig);
       }
-      hacc[j][0] = v0.x; hacc[j][1] = v0.y; hacc[j][2] = v1.x; hacc[j][3] = v1.y;
+    }
+  } else {
+    if (has_h_in) {
+      const float* hi = a.nseg > 1 ? a.ws_H + (bh * a.nseg + a.nseg - 1) * int64_t(kP * N)
+                                   : a.h_in + bh * int64_t(kP * N);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const float2 v0 = *reinterpret_cast<const float2*>(hi + p0 * N + 8 * j + 2 * tig);
+        const float2 v1 = *reinterpret_cast<const float2*>(hi + (p0 + 8) * N + 8 * j + 2 * tig);
+        hacc[j][0] = v0.x; hacc[j][1] = v0.y; hacc[j][2] = v1.x; hacc[j][3] = v1.y;
+      }
+    }
+    for (int sp = 0; sp < seg; ++sp) {  // fold the end states of the earlier segments
+      const float f = mm::ex2_approx(a.ws_A[bh * (a.nseg - 1) + sp]);
+      const float* hs = a.ws_H + (bh * a.nseg + sp) * int64_t(kP * N);
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        const float2 v0 = *reinterpret_cast<const float2*>(hs + p0 * N + 8 * j + 2 * tig);
+        const float2 v1 = *reinterpret_cast<const float2*>(hs + (p0 + 8) * N + 8 * j + 2 * tig);
+        hacc[j][0] = fmaf(f, hacc[j][0], v0.x); hacc[j][1] = fmaf(f, hacc[j][1], v0.y);
+        hacc[j][2] = fmaf(f, hacc[j][2], v1.x); hacc[j][3] = fmaf(f, hacc[j][3], v1.y);
+      }
     }
   }
 
-  // chunk c's C, B and x tiles into stage st; rows past L are zero-filled
+  // chunk c's (C,) B and x tiles into stage st; rows past L are zero-filled
   auto load_chunk = [&](int64_t c, int st) {
     const int64_t t0 = c * kQ;
     const uint32_t s0 = sbase + st * S::kStage;
@@ -222,45 +277,73 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_fwd_kernel(const SsdArgs a) {
       const int64_t t = t0 + r;
       const bool ok = t < L;
       const int64_t row = ((b * L + (ok ? t : 0)) * a.G + grp) * N + 8 * k;
-      cp_async16(s0 + swz(r, k, R), a.C + row, ok);
-      cp_async16(s0 + S::kBC + swz(r, k, R), a.B + row, ok);
+      if constexpr (!kPre) cp_async16(s0 + swz(r, k, R), a.C + row, ok);
+      cp_async16(s0 + S::kOffB + swz(r, k, R), a.B + row, ok);
     }
     for (int i = tid; i < kQ * 8; i += kThreads) {
       const int r = i >> 3, k = i & 7;
       const int64_t t = t0 + r;
       const bool ok = t < L;
       const int64_t row = ((b * L + (ok ? t : 0)) * a.H + h) * kP + 8 * k;
-      cp_async16(s0 + 2 * S::kBC + swz(r, k, 8), a.x + row, ok);
+      cp_async16(s0 + S::kOffX + swz(r, k, 8), a.x + row, ok);
     }
     cp_async_commit();
   };
-  // warp 0 holds dt_raw of steps 2 lane and 2 lane + 1 of the next chunk
+  // warp 0 holds dt_raw (and seq_idx) of steps 2 lane and 2 lane + 1 of the next chunk,
+  // and lane 0 the seq_idx of the step before the chunk
   float dtn0 = 0.f, dtn1 = 0.f;
+  int32_t idn0 = 0, idn1 = 0, idp = 0;
   auto load_dt = [&](int64_t c) {
     const int64_t t = c * kQ + 2 * lane;
     dtn0 = t < L ? __bfloat162float(a.dt[(b * L + t) * a.H + h]) : 0.f;
     dtn1 = t + 1 < L ? __bfloat162float(a.dt[(b * L + t + 1) * a.H + h]) : 0.f;
+    if constexpr (kSeq) {
+      const int32_t* ids = a.seq_idx + b * L;
+      idn0 = t < L ? ids[t] : 0;
+      idn1 = t + 1 < L ? ids[t + 1] : 0;
+      if (lane == 0) idp = c > 0 ? ids[c * kQ - 1] : idn0;
+    }
   };
 
-  if (nchunks > 0) {
-    load_chunk(0, 0);
-    if (warp == 0) load_dt(0);
+  float seg_a = 0.f;  // state pass: summed Delta A log2 e of the segment
+  if (c_begin < c_end) {
+    load_chunk(c_begin, 0);
+    if (warp == 0) load_dt(c_begin);
   }
-  for (int64_t c = 0; c < nchunks; ++c) {
-    const int st = int(c & 1);
+  for (int64_t c = c_begin; c < c_end; ++c) {
+    const int st = int((c - c_begin) & 1);
     const int64_t t0 = c * kQ;
-    const uint32_t sC = sbase + st * S::kStage, sB = sC + S::kBC, sX = sC + 2 * S::kBC;
+    const uint32_t sC = sbase + st * S::kStage, sB = sC + S::kOffB, sX = sC + S::kOffX;
     const bool has_state = c > 0 || has_h_in;
     cp_async_wait_all();
     __syncthreads();  // this chunk's tiles are in; every warp is done with the previous chunk
-    if (c + 1 < nchunks) load_chunk(c + 1, st ^ 1);
+    if (c + 1 < c_end) load_chunk(c + 1, st ^ 1);
 
     // Delta and the inclusive cumulative sum of Delta A (log2 units) over the chunk
     if (warp == 0) {
       const int64_t t = t0 + 2 * lane;
       const float d0 = t < L ? mm::Math<false>::softplus(dtn0 + bias) : 0.f;
       const float d1 = t + 1 < L ? mm::Math<false>::softplus(dtn1 + bias) : 0.f;
-      if (c + 1 < nchunks) load_dt(c + 1);
+      if constexpr (kSeq) {
+        // reset flags of steps 2 lane, 2 lane + 1 (none past L, none at t = 0), then the
+        // last reset position <= t by a max-scan over the lanes
+        const int32_t i0 = idn0, i1 = idn1;
+        const int32_t prev = __shfl_up_sync(0xffffffffu, i1, 1);
+        const bool r0 = t < L && (lane == 0 ? (t > 0 && i0 != idp) : i0 != prev);
+        const bool r1 = t + 1 < L && i1 != i0;
+        int m = r1 ? 2 * lane + 1 : (r0 ? 2 * lane : -1);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, m, o);
+          if (lane >= o) m = max(m, v);
+        }
+        int mex = __shfl_up_sync(0xffffffffu, m, 1);
+        if (lane == 0) mex = -1;
+        const int rs0 = r0 ? 2 * lane : mex;
+        rsp[2 * lane] = rs0;
+        rsp[2 * lane + 1] = r1 ? 2 * lane + 1 : rs0;
+      }
+      if (c + 1 < c_end) load_dt(c + 1);
       const float e0 = d0 * A2, e1 = d1 * A2;
       float s = e0 + e1;
 #pragma unroll
@@ -275,14 +358,71 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_fwd_kernel(const SsdArgs a) {
       dls[2 * lane] = d0;
       dls[2 * lane + 1] = d1;
     }
+
+    // before Delta is known: this warp's causal blocks of C B^T and the inter-chunk term
+    // C H^T for headdim columns [16 warp, 16 warp + 16), H's B operand (hi + lo) taken from
+    // this warp's own state rows
+    const int nblk = warp < 2 ? 3 : 2;
+    float gacc[3][2][4];
+    float yacc[4][2][4];
+    if constexpr (!kPre) {
+#pragma unroll
+      for (int i = 0; i < 3; ++i) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) gacc[i][j][0] = gacc[i][j][1] = gacc[i][j][2] = gacc[i][j][3] = 0.f;
+        if (i < nblk) {
+          int tb, sb;
+          gblock(warp, i, tb, sb);
+#pragma unroll
+          for (int kk = 0; kk < N / 16; ++kk) {
+            uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+            ldsm_x4(sC + swz(16 * tb + (mi & 1) * 8 + ri, 2 * kk + (mi >> 1), R), a0, a1, a2, a3);
+            ldsm_x4(sB + swz(16 * sb + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1), R), b0, b1, b2, b3);
+            mma16816(gacc[i][0], a0, a1, a2, a3, b0, b1);
+            mma16816(gacc[i][1], a0, a1, a2, a3, b2, b3);
+          }
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+        for (int np = 0; np < 2; ++np) yacc[mt][np][0] = yacc[mt][np][1] = yacc[mt][np][2] = yacc[mt][np][3] = 0.f;
+      if (has_state) {
+#pragma unroll
+        for (int kk = 0; kk < N / 16; ++kk) {
+          uint32_t bhi[2][2], blo[2][2];
+#pragma unroll
+          for (int np = 0; np < 2; ++np) {
+            split_bf16(hacc[2 * kk][2 * np], hacc[2 * kk][2 * np + 1], bhi[np][0], blo[np][0]);
+            split_bf16(hacc[2 * kk + 1][2 * np], hacc[2 * kk + 1][2 * np + 1], bhi[np][1], blo[np][1]);
+          }
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(sC + swz(16 * mt + (mi & 1) * 8 + ri, 2 * kk + (mi >> 1), R), a0, a1, a2, a3);
+            mma16816(yacc[mt][0], a0, a1, a2, a3, bhi[0][0], bhi[0][1]);
+            mma16816(yacc[mt][1], a0, a1, a2, a3, bhi[1][0], bhi[1][1]);
+          }
+#pragma unroll
+          for (int mt = 0; mt < 4; ++mt) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(sC + swz(16 * mt + (mi & 1) * 8 + ri, 2 * kk + (mi >> 1), R), a0, a1, a2, a3);
+            mma16816(yacc[mt][0], a0, a1, a2, a3, blo[0][0], blo[0][1]);
+            mma16816(yacc[mt][1], a0, a1, a2, a3, blo[1][0], blo[1][1]);
+          }
+        }
+      }
+    }
     __syncthreads();  // cs2 and dls visible
 
-    // w o x for the state update: w_s = 2^(cs2_last - cs2_s) Delta_s
     const float csl = cs2[kQ - 1];
+    const int rsl = kSeq ? rsp[kQ - 1] : -1;  // last reset in the chunk
+    if constexpr (kPre) seg_a = rsl >= 0 ? -INFINITY : seg_a + csl;
+    // w o x for the state update: w_s = 2^(cs2_last - cs2_s) Delta_s (0 before a reset)
     for (int i = tid; i < kQ * 8; i += kThreads) {
       const int r = i >> 3, k = i & 7;
       const uint32_t off = swz(r, k, 8);
-      const float w = mm::ex2_approx(csl - cs2[r]) * dls[r];
+      const float w = r >= rsl ? mm::ex2_approx(csl - cs2[r]) * dls[r] : 0.f;
       const uint4 v = lds_u128(sX + off);
       uint4 o;
       o.x = pack_bf16(w * bf16_lo(v.x), w * bf16_hi(v.x));
@@ -292,130 +432,99 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_fwd_kernel(const SsdArgs a) {
       sts_u128(sXw + off, o);
     }
 
-    // this warp's causal blocks of M o C B^T, as hi / lo planes [t][s]
-    const int nblk = warp < 2 ? 3 : 2;
+    if constexpr (!kPre) {
+      // mask the blocks: M[t, s] = 2^(cs2_t - cs2_s) Delta_s for s <= t; hi / lo planes [t][s]
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
-      if (i < nblk) {
-        int tb, sb;
-        gblock(warp, i, tb, sb);
-        float gacc[2][4];
+      for (int i = 0; i < 3; ++i) {
+        if (i < nblk) {
+          int tb, sb;
+          gblock(warp, i, tb, sb);
+          const int t0r = 16 * tb + g, t1r = t0r + 8;
+          const float ct0 = cs2[t0r], ct1 = cs2[t1r];
+          const int lo0 = kSeq ? rsp[t0r] : 0, lo1 = kSeq ? rsp[t1r] : 0;  // same document: s >= lo
 #pragma unroll
-        for (int j = 0; j < 2; ++j) gacc[j][0] = gacc[j][1] = gacc[j][2] = gacc[j][3] = 0.f;
-#pragma unroll
-        for (int kk = 0; kk < N / 16; ++kk) {
-          uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-          ldsm_x4(sC + swz(16 * tb + (mi & 1) * 8 + ri, 2 * kk + (mi >> 1), R), a0, a1, a2, a3);
-          ldsm_x4(sB + swz(16 * sb + (mi >> 1) * 8 + ri, 2 * kk + (mi & 1), R), b0, b1, b2, b3);
-          mma16816(gacc[0], a0, a1, a2, a3, b0, b1);
-          mma16816(gacc[1], a0, a1, a2, a3, b2, b3);
-        }
-        const int t0r = 16 * tb + g, t1r = t0r + 8;
-        const float ct0 = cs2[t0r], ct1 = cs2[t1r];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int s0 = 16 * sb + 8 * j + 2 * tig, s1 = s0 + 1;
-          const float cs0 = cs2[s0], cs1 = cs2[s1], w0 = dls[s0], w1 = dls[s1];
-          const float v00 = s0 <= t0r ? gacc[j][0] * mm::ex2_approx(ct0 - cs0) * w0 : 0.f;
-          const float v01 = s1 <= t0r ? gacc[j][1] * mm::ex2_approx(ct0 - cs1) * w1 : 0.f;
-          const float v10 = s0 <= t1r ? gacc[j][2] * mm::ex2_approx(ct1 - cs0) * w0 : 0.f;
-          const float v11 = s1 <= t1r ? gacc[j][3] * mm::ex2_approx(ct1 - cs1) * w1 : 0.f;
-          uint32_t hi, lo;
-          split_bf16(v00, v01, hi, lo);
-          sts_u32(sGhi + swz(t0r, 2 * sb + j, 8) + 4 * tig, hi);
-          sts_u32(sGlo + swz(t0r, 2 * sb + j, 8) + 4 * tig, lo);
-          split_bf16(v10, v11, hi, lo);
-          sts_u32(sGhi + swz(t1r, 2 * sb + j, 8) + 4 * tig, hi);
-          sts_u32(sGlo + swz(t1r, 2 * sb + j, 8) + 4 * tig, lo);
-        }
-      }
-    }
-
-    // Y[:, 16 warp + (0..15)] = diag(2^cs2) C H^T, with H's B operand (hi + lo) taken from
-    // this warp's own state rows
-    float yacc[4][2][4];
-#pragma unroll
-    for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-      for (int np = 0; np < 2; ++np) yacc[mt][np][0] = yacc[mt][np][1] = yacc[mt][np][2] = yacc[mt][np][3] = 0.f;
-    if (has_state) {
-#pragma unroll
-      for (int kk = 0; kk < N / 16; ++kk) {
-        uint32_t bh[2][2], bl[2][2];
-#pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          split_bf16(hacc[2 * kk][2 * np], hacc[2 * kk][2 * np + 1], bh[np][0], bl[np][0]);
-          split_bf16(hacc[2 * kk + 1][2 * np], hacc[2 * kk + 1][2 * np + 1], bh[np][1], bl[np][1]);
-        }
-#pragma unroll
-        for (int mt = 0; mt < 4; ++mt) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(sC + swz(16 * mt + (mi & 1) * 8 + ri, 2 * kk + (mi >> 1), R), a0, a1, a2, a3);
-#pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            mma16816(yacc[mt][np], a0, a1, a2, a3, bh[np][0], bh[np][1]);
-            mma16816(yacc[mt][np], a0, a1, a2, a3, bl[np][0], bl[np][1]);
+          for (int j = 0; j < 2; ++j) {
+            const int s0 = 16 * sb + 8 * j + 2 * tig, s1 = s0 + 1;
+            const float cs0 = cs2[s0], cs1 = cs2[s1], w0 = dls[s0], w1 = dls[s1];
+            const float v00 = s0 <= t0r && s0 >= lo0 ? gacc[i][j][0] * mm::ex2_approx(ct0 - cs0) * w0 : 0.f;
+            const float v01 = s1 <= t0r && s1 >= lo0 ? gacc[i][j][1] * mm::ex2_approx(ct0 - cs1) * w1 : 0.f;
+            const float v10 = s0 <= t1r && s0 >= lo1 ? gacc[i][j][2] * mm::ex2_approx(ct1 - cs0) * w0 : 0.f;
+            const float v11 = s1 <= t1r && s1 >= lo1 ? gacc[i][j][3] * mm::ex2_approx(ct1 - cs1) * w1 : 0.f;
+            uint32_t hi, lo;
+            split_bf16(v00, v01, hi, lo);
+            sts_u32(sGhi + swz(t0r, 2 * sb + j, 8) + 4 * tig, hi);
+            sts_u32(sGlo + swz(t0r, 2 * sb + j, 8) + 4 * tig, lo);
+            split_bf16(v10, v11, hi, lo);
+            sts_u32(sGhi + swz(t1r, 2 * sb + j, 8) + 4 * tig, hi);
+            sts_u32(sGlo + swz(t1r, 2 * sb + j, 8) + 4 * tig, lo);
           }
         }
       }
+      if (has_state) {  // the inter-chunk term decays by 2^cs2_t at step t (0 after a reset)
 #pragma unroll
-      for (int mt = 0; mt < 4; ++mt) {
-        const float e0 = mm::ex2_approx(cs2[16 * mt + g]), e1 = mm::ex2_approx(cs2[16 * mt + g + 8]);
+        for (int mt = 0; mt < 4; ++mt) {
+          const int ta = 16 * mt + g, tb2 = ta + 8;
+          const float e0 = (!kSeq || rsp[ta] < 0) ? mm::ex2_approx(cs2[ta]) : 0.f;
+          const float e1 = (!kSeq || rsp[tb2] < 0) ? mm::ex2_approx(cs2[tb2]) : 0.f;
 #pragma unroll
-        for (int np = 0; np < 2; ++np) {
-          yacc[mt][np][0] *= e0; yacc[mt][np][1] *= e0; yacc[mt][np][2] *= e1; yacc[mt][np][3] *= e1;
+          for (int np = 0; np < 2; ++np) {
+            yacc[mt][np][0] *= e0; yacc[mt][np][1] *= e0; yacc[mt][np][2] *= e1; yacc[mt][np][3] *= e1;
+          }
         }
       }
     }
     __syncthreads();  // M o C B^T and w o x visible
 
-    // Y += (M o C B^T) x for s blocks kb <= t block mt
+    if constexpr (!kPre) {
+      // Y += (M o C B^T) x for s blocks kb <= t block mt
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
+      for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        if (kb <= mt) {
-          uint32_t h0, h1, h2, h3, l0, l1, l2, l3, b0, b1, b2, b3;
-          const uint32_t ga = swz(16 * mt + (mi & 1) * 8 + ri, 2 * kb + (mi >> 1), 8);
-          ldsm_x4(sGhi + ga, h0, h1, h2, h3);
-          ldsm_x4(sGlo + ga, l0, l1, l2, l3);
-          ldsm_x4_t(sX + swz(16 * kb + (mi & 1) * 8 + ri, 2 * warp + (mi >> 1), 8), b0, b1, b2, b3);
-          mma16816(yacc[mt][0], h0, h1, h2, h3, b0, b1);
-          mma16816(yacc[mt][1], h0, h1, h2, h3, b2, b3);
-          mma16816(yacc[mt][0], l0, l1, l2, l3, b0, b1);
-          mma16816(yacc[mt][1], l0, l1, l2, l3, b2, b3);
+        for (int kb = 0; kb < 4; ++kb) {
+          if (kb <= mt) {
+            uint32_t h0, h1, h2, h3, l0, l1, l2, l3, b0, b1, b2, b3;
+            const uint32_t ga = swz(16 * mt + (mi & 1) * 8 + ri, 2 * kb + (mi >> 1), 8);
+            ldsm_x4(sGhi + ga, h0, h1, h2, h3);
+            ldsm_x4(sGlo + ga, l0, l1, l2, l3);
+            ldsm_x4_t(sX + swz(16 * kb + (mi & 1) * 8 + ri, 2 * warp + (mi >> 1), 8), b0, b1, b2, b3);
+            mma16816(yacc[mt][0], h0, h1, h2, h3, b0, b1);
+            mma16816(yacc[mt][1], h0, h1, h2, h3, b2, b3);
+            mma16816(yacc[mt][0], l0, l1, l2, l3, b0, b1);
+            mma16816(yacc[mt][1], l0, l1, l2, l3, b2, b3);
+          }
         }
       }
-    }
 
-    // out = (Y + D x) [* SiLU(z)], bf16 pairs at (t = 16 mt + g (+8), p = 16 warp + 8 np + 2 tig)
+      // out = (Y + D x) [* SiLU(z)], bf16 pairs at (t = 16 mt + g (+8), p = 16 warp + 8 np + 2 tig)
+      const float Dh = a.D[h];
 #pragma unroll
-    for (int mt = 0; mt < 4; ++mt) {
+      for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int tr = 16 * mt + g + 8 * hf;
-        const int64_t t = t0 + tr;
-        if (t < L) {
-          const int64_t row = ((b * L + t) * a.H + h) * kP;
+        for (int hf = 0; hf < 2; ++hf) {
+          const int tr = 16 * mt + g + 8 * hf;
+          const int64_t t = t0 + tr;
+          if (t < L) {
+            const int64_t row = ((b * L + t) * a.H + h) * kP;
 #pragma unroll
-          for (int np = 0; np < 2; ++np) {
-            const int p = 16 * warp + 8 * np + 2 * tig;
-            const uint32_t xv = lds_u32(sX + swz(tr, 2 * warp + np, 8) + 4 * tig);
-            float o0 = yacc[mt][np][2 * hf] + Dh * bf16_lo(xv);
-            float o1 = yacc[mt][np][2 * hf + 1] + Dh * bf16_hi(xv);
-            if constexpr (kGate) {
-              const uint32_t zv = *reinterpret_cast<const uint32_t*>(a.z + row + p);
-              o0 *= mm::Math<false>::silu(bf16_lo(zv));
-              o1 *= mm::Math<false>::silu(bf16_hi(zv));
+            for (int np = 0; np < 2; ++np) {
+              const int p = 16 * warp + 8 * np + 2 * tig;
+              const uint32_t xv = lds_u32(sX + swz(tr, 2 * warp + np, 8) + 4 * tig);
+              float o0 = yacc[mt][np][2 * hf] + Dh * bf16_lo(xv);
+              float o1 = yacc[mt][np][2 * hf + 1] + Dh * bf16_hi(xv);
+              if constexpr (kGate) {
+                const uint32_t zv = *reinterpret_cast<const uint32_t*>(a.z + row + p);
+                o0 *= mm::Math<false>::silu(bf16_lo(zv));
+                o1 *= mm::Math<false>::silu(bf16_hi(zv));
+              }
+              *reinterpret_cast<uint32_t*>(a.y + row + p) = pack_bf16(o0, o1);
             }
-            *reinterpret_cast<uint32_t*>(a.y + row + p) = pack_bf16(o0, o1);
           }
         }
       }
     }
 
     // H <- 2^cs2_last H + (w o x)^T B   (rows p of this warp, all n)
-    const float dec = mm::ex2_approx(csl);
+    const float dec = rsl < 0 ? mm::ex2_approx(csl) : 0.f;
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       hacc[j][0] *= dec; hacc[j][1] *= dec; hacc[j][2] *= dec; hacc[j][3] *= dec;
@@ -434,12 +543,19 @@ __global__ void __launch_bounds__(kThreads, 2) ssd_fwd_kernel(const SsdArgs a) {
     }
   }
 
-  if (a.h_out) {
-    float* ho = a.h_out + (b * a.H + h) * int64_t(kP * N);
+  float* out = nullptr;
+  if constexpr (kPre) {
+    out = a.ws_H + (bh * a.nseg + seg) * int64_t(kP * N);
+    if (tid == 0) a.ws_A[bh * (a.nseg - 1) + seg] = seg_a;
+  } else {
+    if (seg == a.nseg - 1) out = a.h_out;
+    if (out) out += bh * int64_t(kP * N);
+  }
+  if (out) {
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
-      *reinterpret_cast<float2*>(ho + p0 * N + 8 * j + 2 * tig) = make_float2(hacc[j][0], hacc[j][1]);
-      *reinterpret_cast<float2*>(ho + (p0 + 8) * N + 8 * j + 2 * tig) = make_float2(hacc[j][2], hacc[j][3]);
+      *reinterpret_cast<float2*>(out + p0 * N + 8 * j + 2 * tig) = make_float2(hacc[j][0], hacc[j][1]);
+      *reinterpret_cast<float2*>(out + (p0 + 8) * N + 8 * j + 2 * tig) = make_float2(hacc[j][2], hacc[j][3]);
     }
   }
 }

@@ -13,7 +13,7 @@ import torch
 
 from . import mixer as _m
 
-EXPORTS = ("mamba2_ssd_fwd",)
+EXPORTS = ("mamba2_ssd_fwd_workspace_bytes", "mamba2_ssd_fwd")
 
 
 class mamba2_dims(ctypes.Structure):
@@ -31,8 +31,10 @@ def _lib() -> ctypes.CDLL:
     lib = _m.load_library()
     if _bound is not lib:
         vp = ctypes.c_void_p
+        lib.mamba2_ssd_fwd_workspace_bytes.restype = ctypes.c_size_t
+        lib.mamba2_ssd_fwd_workspace_bytes.argtypes = [ctypes.POINTER(mamba2_dims)]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
-        lib.mamba2_ssd_fwd.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 12
+        lib.mamba2_ssd_fwd.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 13 + [ctypes.c_size_t, vp]
         _bound = lib
     return lib
 
@@ -42,13 +44,19 @@ def make_dims(batch, seqlen, nheads, headdim, d_state, ngroups, io_dtype=_m.MAMB
                        int(ngroups), int(io_dtype), 0)
 
 
-def mamba2_ssd_fwd(x, dt_raw, A_log, B, C, D, dt_bias, *, z=None, h_in=None, y=None,
-                   h_out=None, want_state: bool = True, stream=None
+def workspace_bytes(dims: mamba2_dims) -> int:
+    return int(_lib().mamba2_ssd_fwd_workspace_bytes(ctypes.byref(dims)))
+
+
+def mamba2_ssd_fwd(x, dt_raw, A_log, B, C, D, dt_bias, *, z=None, seq_idx=None, h_in=None, y=None,
+                   h_out=None, want_state: bool = True, workspace=None, stream=None
                    ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Mamba2 scan forward.  Shapes: x (and z) [batch, L, nheads, 64] bf16; dt_raw
     [batch, L, nheads] bf16; B, C [batch, L, ngroups, d_state] bf16; A_log, D, dt_bias
-    [nheads] fp32; h_in [batch, nheads, 64, d_state] fp32 or None.  Returns (y, h_out)
-    (h_out None when want_state is False)."""
+    [nheads] fp32; seq_idx [batch, L] int32 or None (documents packed in rows: the state
+    resets where the id changes); h_in [batch, nheads, 64, d_state] fp32 or None.  workspace: a uint8
+    device tensor of at least workspace_bytes(dims) bytes (allocated when None).  Returns
+    (y, h_out) (h_out None when want_state is False)."""
     lib = _lib()
     dev = x.device
     Bt, L, H, P = x.shape
@@ -61,12 +69,16 @@ def mamba2_ssd_fwd(x, dt_raw, A_log, B, C, D, dt_bias, *, z=None, h_in=None, y=N
     if h_out is None and want_state:
         h_out = torch.empty(Bt, H, P, N, dtype=f32, device=dev)
     dims = make_dims(Bt, L, H, P, N, G, io)
+    need = workspace_bytes(dims)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     p = _m._ptr
     rc = lib.mamba2_ssd_fwd(
         ctypes.byref(dims), p(x, "x", iot, dev), p(dt_raw, "dt_raw", iot, dev),
         p(A_log, "A_log", f32, dev), p(B, "B", iot, dev), p(C, "C", iot, dev),
         p(D, "D", f32, dev), p(dt_bias, "dt_bias", f32, dev), p(z, "z", iot, dev),
-        p(h_in, "h_in", f32, dev), p(y, "y", iot, dev), p(h_out, "h_out", f32, dev),
-        _m._stream_handle(stream, dev))
+        p(seq_idx, "seq_idx", torch.int32, dev), p(h_in, "h_in", f32, dev), p(y, "y", iot, dev), p(h_out, "h_out", f32, dev),
+        p(workspace, "workspace", None, dev), ws_bytes, _m._stream_handle(stream, dev))
     _m._check(rc)
     return y, h_out

@@ -2,8 +2,10 @@
 
 Shapes span several 64-step chunks with ragged tails, both supported d_state values, one
 and several groups, the gate, an initial state (also updated in place), the empty and
-single-step sequences, and the reference layer (24 heads x 64, d_state 128) at full size
-on sampled (batch row, head) pairs.  Tolerance: tests/tolerances.py assert_close_tc.
+single-step sequences, rows packing documents (the nine structural seq_idx cases of
+niverel-mamba 0.1.0, section "seq_idx strict reset", with and without an initial state and
+time segments), and the reference layer (24 heads x 64, d_state 128) at full size on
+sampled (batch row, head) pairs.  Tolerance: tests/tolerances.py assert_close_tc.
 """
 
 import numpy as np
@@ -24,18 +26,19 @@ def draw(Bt, L, H, N, G, gate, state, seed):
     return I.make_ssd_inputs(w)
 
 
-def run_gpu(inp, h_in_inplace=False):
+def run_gpu(inp, h_in_inplace=False, seq_idx=None):
     d = {k: (None if v is None else dev_tensor(v)) for k, v in inp.items()}
     h_out = d["h_in"] if h_in_inplace else None
+    ids = None if seq_idx is None else torch.from_numpy(np.ascontiguousarray(seq_idx, dtype=np.int32)).cuda()
     y, h = S.mamba2_ssd_fwd(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"],
-                            d["dt_bias"], z=d["z"], h_in=d["h_in"], h_out=h_out)
+                            d["dt_bias"], z=d["z"], seq_idx=ids, h_in=d["h_in"], h_out=h_out)
     torch.cuda.synchronize()
     return host(y), host(h)
 
 
-def run_oracle(inp):
+def run_oracle(inp, seq_idx=None):
     return so.ssd(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"], inp["D"],
-                  inp["dt_bias"], z=inp["z"], h_in=inp["h_in"])
+                  inp["dt_bias"], z=inp["z"], h_in=inp["h_in"], seq_idx=seq_idx)
 
 
 CASES = [
@@ -105,6 +108,33 @@ def test_reference_layer_full_size_sampled(name):
     sel += [(0, 0), (w.batch - 1, w.nheads - 1)]
     outs, hs = so.ssd_channels(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"],
                                inp["D"], inp["dt_bias"], sel, z=inp["z"], h_in=inp["h_in"])
+    for (b, hh), o, hf in zip(sel, outs, hs):
+        assert_close_tc(y[b, :, hh], o, f"y[{b}, :, {hh}]")
+        assert_close_tc(h[b, hh], hf, f"h_out[{b}, {hh}]")
+
+
+@pytest.mark.parametrize("name", I.SEQ_IDX_CASES)
+@pytest.mark.parametrize("state", [False, True])
+def test_packed_documents(name, state):
+    Bt, L, H = 2, 200, 4
+    inp = draw(Bt, L, H, 128, 1, True, state, seed=3400 + I.SEQ_IDX_CASES.index(name))
+    ids = I.seq_idx_case(name, Bt, L, edge=64, seed=9)
+    yo, ho = run_oracle(inp, ids)
+    y, h = run_gpu(inp, seq_idx=ids)
+    assert_close_tc(y, yo, f"y ({name})")
+    assert_close_tc(h, ho, f"h_out ({name})")
+
+
+def test_packed_long_row_sampled():
+    # 2 rows of 8192 steps packing documents of mean length 256, time segments on
+    w = I.SsdWorkload("packed_long", 2, 8192, 24, 64, 128, 1, 3500, state=True)
+    inp = I.make_ssd_inputs(w)
+    ids = I.packed_seq_idx(2, 8192, 256, 3501)
+    y, h = run_gpu(inp, seq_idx=ids)
+    sel = [(0, 0), (1, 23), (0, 11), (1, 5)]
+    outs, hs = so.ssd_channels(inp["x"], inp["dt_raw"], inp["A_log"], inp["B"], inp["C"],
+                               inp["D"], inp["dt_bias"], sel, z=inp["z"], h_in=inp["h_in"],
+                               seq_idx=ids)
     for (b, hh), o, hf in zip(sel, outs, hs):
         assert_close_tc(y[b, :, hh], o, f"y[{b}, :, {hh}]")
         assert_close_tc(h[b, hh], hf, f"h_out[{b}, {hh}]")

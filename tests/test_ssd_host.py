@@ -12,7 +12,7 @@ from selective_state_space_silu_b200 import build as Bld
 from selective_state_space_silu_b200 import mixer as M
 from selective_state_space_silu_b200 import ssd as S
 
-NAMES = ["x", "dt", "A_log", "B", "C", "D", "dt_bias", "z", "h_in", "y", "h_out"]
+NAMES = ["x", "dt", "A_log", "B", "C", "D", "dt_bias", "z", "seq", "h_in", "y", "h_out"]
 
 
 @pytest.fixture(scope="module")
@@ -30,8 +30,10 @@ def _call(lib, dims, ptrs=None):
     p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(NAMES)}
     if ptrs:
         p.update(ptrs)
+    ws = p.get("ws", _fake(0xf000000000))
+    ws_bytes = p.get("ws_bytes", 1 << 40)
     return lib.mamba2_ssd_fwd(ctypes.byref(dims) if dims is not None else None,
-                              *[p[k] for k in NAMES], None)
+                              *[p[k] for k in NAMES], ws, ws_bytes, None)
 
 
 def dims(**kw):
@@ -70,17 +72,41 @@ def test_misaligned_pointers(lib):
     assert _call(lib, dims(), {"B": _fake(0x3010000004)}) == 3
     assert _call(lib, dims(), {"dt": _fake(0x1010000001)}) == 3
     assert _call(lib, dims(), {"D": _fake(0x5010000002)}) == 3
-    assert _call(lib, dims(), {"h_out": _fake(0xa010000008)}) == 3
+    assert _call(lib, dims(), {"h_out": _fake(0xb010000008)}) == 3
+    assert _call(lib, dims(), {"seq": _fake(0x8010000002)}) == 3
 
 
 def test_overlaps_rejected(lib):
     assert _call(lib, dims(), {"y": _fake(0x10000000)}) == 1            # y on top of x
-    assert _call(lib, dims(), {"h_out": _fake(0x9010000000)}) == 1      # h_out inside y
+    assert _call(lib, dims(), {"h_out": _fake(0xa010000000)}) == 1      # h_out inside y
+    assert _call(lib, dims(), {"y": _fake(0x8010000000)}) == 1          # y on top of seq_idx
     # h_out == h_in exactly is in-place and allowed at validation; partial overlap is not
-    assert _call(lib, dims(), {"h_out": _fake(0x8010000010)}) == 1
+    assert _call(lib, dims(), {"h_out": _fake(0x9010000010)}) == 1
     assert "partially" in M.mamba_last_error()
 
 
 def test_nothing_to_do(lib):
     assert _call(lib, dims(batch=0)) == 0
     assert _call(lib, dims(nheads=0), {k: None for k in ("A_log", "D", "dt_bias")}) == 0
+
+
+def test_workspace_rules(lib):
+    # few (row, head) pairs and a long sequence: split into time segments, workspace needed
+    d = dims(batch=1, seqlen=8192, nheads=2)
+    need = lib.mamba2_ssd_fwd_workspace_bytes(ctypes.byref(d))
+    assert need > 0
+    assert _call(lib, d, {"ws": None, "ws_bytes": 0}) == 4
+    assert _call(lib, d, {"ws_bytes": need - 1}) == 4
+    assert _call(lib, d, {"ws": _fake(0xf000000080), "ws_bytes": need}) == 3
+    assert _call(lib, d, {"ws": _fake(0x10000000), "ws_bytes": need}) == 1   # overlaps x
+    # many pairs: one segment, no workspace
+    d = dims(batch=64, seqlen=256, nheads=24)
+    assert lib.mamba2_ssd_fwd_workspace_bytes(ctypes.byref(d)) == 0
+    assert lib.mamba2_ssd_fwd_workspace_bytes(ctypes.byref(dims(headdim=32))) == 0
+    # size: per (row, head), segments - 1 end states and one copy of h_in (headdim x
+    # d_state fp32 each), then segments - 1 floats, padded to 256 bytes
+    d = dims(batch=2, seqlen=8192, nheads=24, d_state=128)
+    need = lib.mamba2_ssd_fwd_workspace_bytes(ctypes.byref(d))
+    nseg = need // (48 * 64 * 128 * 4)
+    assert nseg >= 2
+    assert need == 48 * nseg * 64 * 128 * 4 + (48 * (nseg - 1) * 4 + 255) // 256 * 256
