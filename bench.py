@@ -759,6 +759,8 @@ def main():
             print(json.dumps(res), flush=True)
         return
 
+    if args.pass_ != "fwd" and world > 1:
+        ap.error("--pass bwd and --pass ssd time one GPU: run them without torchrun")
     if args.pass_ == "ssd":
         sw = I.SSD_WORKLOADS[args.ssd_workload]
         if args.seqlen is not None:

@@ -50,25 +50,36 @@ bool overlap(const Range& a, const Range& b) {
 
 // Time segments: with few (batch row, head) pairs, each pair's chunks are cut into
 // segments that run as separate CTAs (a state pass over segments 0 .. nseg - 2 first).
-// Target: about two waves of the main pass at two CTAs per SM on the 148 SMs.
+// With fewer pairs than resident main-pass CTAs (2 per SM on the 148 SMs), the count
+// minimises (waves of main-pass CTAs) x (chunks per segment), the fewest segments on a tie
+// (each extra one adds state-pass and fold work).
+// Measured (B200, 24 heads x 64, d_state 128): 8 x 2048 steps -> 3 segments, 165 us (2: 204,
+// 6: 200); 2 x 8192 -> 6 segments, 189 us (12: 200, 16: 218).
 struct SegPlan {
   int nseg, cps;
 };
 
 constexpr int64_t kSms = 148;
+constexpr int64_t kMainSlots = 2 * kSms;  // main-pass CTAs resident at once
 
 SegPlan seg_plan(int64_t Bt, int64_t L, int64_t H) {
   const int64_t nchunks = (L + ssd::kQ - 1) / ssd::kQ;
   const int64_t pairs = Bt * H;
-  const int64_t target = 4 * kSms;
-  int64_t nseg = 1;
-  if (pairs > 0 && nchunks > 1 && pairs < target) nseg = (target + pairs / 2) / pairs;
-  if (nseg > 16) nseg = 16;
-  if (nseg > nchunks) nseg = nchunks;
-  if (nseg < 1) nseg = 1;
-  const int64_t cps = nchunks > 0 ? (nchunks + nseg - 1) / nseg : 1;
-  nseg = nchunks > 0 ? (nchunks + cps - 1) / cps : 1;
-  return {int(nseg), int(cps)};
+  // pairs that fill the resident slots by themselves gain nothing from a split
+  if (nchunks <= 1 || pairs <= 0 || pairs >= kMainSlots) return {1, int(nchunks > 0 ? nchunks : 1)};
+  int64_t best_cost = -1, best_n = 1, best_cps = nchunks;
+  for (int64_t n = 1; n <= 16 && n <= nchunks; ++n) {
+    const int64_t cps = (nchunks + n - 1) / n;
+    const int64_t n_eff = (nchunks + cps - 1) / cps;
+    const int64_t waves = (pairs * n_eff + kMainSlots - 1) / kMainSlots;
+    const int64_t cost = waves * cps;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_n = n_eff;
+      best_cps = cps;
+    }
+  }
+  return {int(best_n), int(best_cps)};
 }
 
 // nseg state slots per (row, head) -- nseg - 1 segment end states and the copy of h_in --
