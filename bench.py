@@ -129,6 +129,7 @@ def measured_peaks() -> dict:
 KERNEL_SOURCES = {
     "fwd": ("fwd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
     "step": ("step.cuh", "device_math.cuh", "sm100_primitives.cuh"),
+    "ssd": ("ssd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
 }
 
 
@@ -644,7 +645,8 @@ def run_ssd(args, w, local_rank: int):
                      "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)",
                      "tensor_tflops": round(tflops, 2), "tensor_frac": round(tflops / bf16_peak, 4),
                      "tensor_peak_source": "measured cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops)",
-                     "floor_frac": round(t_floor / (ms * 1e-3), 4), "traffic": None},
+                     "floor_frac": round(t_floor / (ms * 1e-3), 4),
+                     "traffic": recorded_traffic("ssd", w.name)},
         "gpu_launches": args.steps, "clocks": clk.summary(),
     }
 

@@ -138,3 +138,23 @@ def test_packed_long_row_sampled():
     for (b, hh), o, hf in zip(sel, outs, hs):
         assert_close_tc(y[b, :, hh], o, f"y[{b}, :, {hh}]")
         assert_close_tc(h[b, hh], hf, f"h_out[{b}, {hh}]")
+
+
+PACKED_VARIANTS = [
+    # name, Bt, L, H, N, G, gate, state, in_place
+    ("many_short_docs", 3, 300, 4, 64, 2, True, True, False),
+    ("misaligned_rows", 1, 700, 2, 64, 1, False, True, True),
+    ("consecutive_boundaries", 2, 130, 6, 128, 3, True, False, False),
+    ("terminal_padding", 2, 513, 2, 128, 2, True, True, True),
+]
+
+
+@pytest.mark.parametrize("case", PACKED_VARIANTS, ids=lambda c: c[0] + "-" + "x".join(map(str, c[1:])))
+def test_packed_variants(case):
+    name, Bt, L, H, N, G, gate, state, in_place = case
+    inp = draw(Bt, L, H, N, G, gate, state, seed=3600 + L)
+    ids = I.seq_idx_case(name, Bt, L, edge=64, seed=11)
+    yo, ho = run_oracle(inp, ids)
+    y, h = run_gpu(inp, h_in_inplace=in_place, seq_idx=ids)
+    assert_close_tc(y, yo, f"y ({name})")
+    assert_close_tc(h, ho, f"h_out ({name})")
