@@ -110,3 +110,23 @@ def test_workspace_rules(lib):
     nseg = need // (48 * 64 * 128 * 4)
     assert nseg >= 2
     assert need == 48 * nseg * 64 * 128 * 4 + (48 * (nseg - 1) * 4 + 255) // 256 * 256
+
+
+def _nseg(lib, **kw):
+    d = dims(**kw)
+    need = lib.mamba2_ssd_fwd_workspace_bytes(ctypes.byref(d))
+    if need == 0:
+        return 1
+    pairs = d.batch * d.nheads
+    return need // (pairs * 64 * d.d_state * 4)
+
+
+def test_segment_plan(lib):
+    # fewer (row, head) pairs than resident main-pass CTAs (2 per SM x 148): minimise
+    # waves x chunks per segment, fewest segments on a tie; otherwise no split
+    assert _nseg(lib, batch=8, seqlen=2048, nheads=24) == 3
+    assert _nseg(lib, batch=2, seqlen=8192, nheads=24) == 6
+    assert _nseg(lib, batch=1, seqlen=640, nheads=2) == 10        # 10 chunks, one each
+    assert _nseg(lib, batch=1, seqlen=65536, nheads=2) == 16      # at most 16
+    assert _nseg(lib, batch=64, seqlen=4096, nheads=24) == 1      # pairs fill the GPU
+    assert _nseg(lib, batch=1, seqlen=64, nheads=4) == 1          # one chunk
