@@ -583,7 +583,8 @@ def ssd_flops(w) -> int:
 
 
 def run_ssd(args, w, local_rank: int):
-    """--pass ssd: times mamba2_ssd_fwd alone (device events, L2 flushed between calls)."""
+    """--pass ssd: times mamba2_ssd_fwd alone (device events, L2 flushed between calls);
+    for a one-token workload with a cached state, mamba2_ssd_step (the state in place)."""
     import torch
     from selective_state_space_silu_b200 import mixer as M
     from selective_state_space_silu_b200 import ssd as S
@@ -607,9 +608,17 @@ def run_ssd(args, w, local_rank: int):
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
 
+    step = w.seqlen == 1 and w.state
+
     def call():
-        S.mamba2_ssd_fwd(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"], d["dt_bias"],
-                         z=d["z"], h_in=d["h_in"], y=y, h_out=h_out, stream=stream)
+        if step:
+            S.mamba2_ssd_step(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"],
+                              d["dt_bias"], d["h_in"], z=d["z"], y=y, h_out=d["h_in"],
+                              stream=stream)
+        else:
+            S.mamba2_ssd_fwd(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"],
+                             d["dt_bias"], z=d["z"], h_in=d["h_in"], y=y, h_out=h_out,
+                             stream=stream)
 
     for _ in range(args.warmup):
         flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
@@ -623,14 +632,15 @@ def run_ssd(args, w, local_rank: int):
             e0.record(stream); call(); e1.record(stream)
         torch.cuda.synchronize()
     ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    nbytes, flops = ssd_bytes(w), ssd_flops(w)
+    nbytes, flops = ssd_bytes(w), (0 if step else ssd_flops(w))  # the step runs no products
     peaks = measured_peaks()
     achieved = nbytes / (ms * 1e-3) / 1e9
     tflops = flops / (ms * 1e-3) / 1e12
     bf16_peak = peaks.get("bf16_tflops", 1590.0)
     t_floor = max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (bf16_peak * 1e12))
     return {
-        "metric": "Mamba2 scan (SSD) forward: achieved algorithmic GB/s", "pass": "ssd",
+        "metric": ("Mamba2 decode step" if step else "Mamba2 scan (SSD) forward")
+                  + ": achieved algorithmic GB/s", "pass": "ssd",
         "value": round(achieved, 2), "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
         "dtype": "bf16", "data": "synthetic",
@@ -639,11 +649,13 @@ def run_ssd(args, w, local_rank: int):
                    "ngroups": w.ngroups, "gate": w.gate, "initial_state": w.state,
                    "chunk": SSD_Q, "l2": "flushed between calls", "algorithmic_bytes": nbytes,
                    "algorithmic_flops": flops},
-        "roofline": {"kernel": "ssd_fwd_kernel", "bound": "hbm", "achieved": round(achieved, 2),
+        "roofline": {"kernel": "ssd_step_kernel" if step else "ssd_fwd_kernel", "bound": "hbm",
+                     "achieved": round(achieved, 2),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)",
-                     "tensor_tflops": round(tflops, 2), "tensor_frac": round(tflops / bf16_peak, 4),
+                     "tensor_tflops": None if step else round(tflops, 2),
+                     "tensor_frac": None if step else round(tflops / bf16_peak, 4),
                      "tensor_peak_source": "measured cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops)",
                      "floor_frac": round(t_floor / (ms * 1e-3), 4),
                      "traffic": recorded_traffic("ssd", w.name)},

@@ -96,6 +96,19 @@ MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void*
                              const float* h_in, void* y, float* h_out, void* workspace,
                              size_t workspace_bytes, void* cuda_stream);
 
+/*
+ * One decode step of the Mamba2 scan on a cached state (niverel-mamba 0.1.0, section
+ * "Autoregressive decoding": step(x_t, state) returns the output and a new state, and
+ * concatenated steps equal the forward).  dims->seqlen must be 1; the layouts are those of
+ * mamba2_ssd_fwd with seqlen 1.  h_in is required; the new state goes to h_out, which may be
+ * h_in itself (in-place update; any other overlap is MAMBA_ERR_INVALID_ARGUMENT).  z may be
+ * NULL.  No workspace.
+ */
+MAMBA_API int mamba2_ssd_step(const mamba2_dims* dims, const void* x, const void* dt_raw,
+                              const float* A_log, const void* B, const void* C, const float* D,
+                              const float* dt_bias, const void* z, const float* h_in, void* y,
+                              float* h_out, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -7,6 +7,7 @@
 
 #include "mamba2_ssd.h"
 #include "ssd_kernel.cuh"
+#include "ssd_step.cuh"
 
 namespace mm_internal {
 void set_last_error(const char* msg);  // mamba_mixer.cu: the message mamba_last_error returns
@@ -227,5 +228,72 @@ extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, 
   cudaError_t e;
   e = N == 128 ? launch_n<128>(a, Bt, st) : launch_n<64>(a, Bt, st);
   if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "ssd launch failed: %s", cudaGetErrorString(e));
+  return ssd_ok();
+}
+
+extern "C" MAMBA_API int mamba2_ssd_step(const mamba2_dims* dims, const void* x, const void* dt_raw,
+                                         const float* A_log, const void* B, const void* C,
+                                         const float* D, const float* dt_bias, const void* z,
+                                         const float* h_in, void* y, float* h_out,
+                                         void* cuda_stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const int64_t Bt = dims->batch, H = dims->nheads, P = dims->headdim, N = dims->d_state,
+                G = dims->ngroups;
+  if (dims->seqlen != 1)
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "seqlen %lld: the step takes one token",
+                    (long long)dims->seqlen);
+  const size_t rows = size_t(Bt * H * P), state = rows * size_t(N);
+  const bool any = rows > 0;
+  if ((rc = need(x, "x", any, 16)) || (rc = need(dt_raw, "dt_raw", any, 2)) ||
+      (rc = need(A_log, "A_log", H > 0, 4)) || (rc = need(B, "B", any, 16)) ||
+      (rc = need(C, "C", any, 16)) || (rc = need(D, "D", H > 0, 4)) ||
+      (rc = need(dt_bias, "dt_bias", H > 0, 4)) || (rc = need(z, "z", false, 16)) ||
+      (rc = need(h_in, "h_in", any, 16)) || (rc = need(y, "y", any, 16)) ||
+      (rc = need(h_out, "h_out", any, 16)))
+    return rc;
+  const size_t bc = size_t(Bt * G * N);
+  const Range ins[] = {{x, rows * 2, "x"},       {dt_raw, size_t(Bt * H) * 2, "dt_raw"},
+                       {A_log, size_t(H) * 4, "A_log"}, {B, bc * 2, "B"}, {C, bc * 2, "C"},
+                       {D, size_t(H) * 4, "D"},  {dt_bias, size_t(H) * 4, "dt_bias"},
+                       {z, rows * 2, "z"}};
+  const Range y_r{y, rows * 2, "y"}, hin_r{h_in, state * 4, "h_in"}, hout_r{h_out, state * 4, "h_out"};
+  for (const Range& i : ins)
+    if (overlap(y_r, i) || overlap(hout_r, i))
+      return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "an output overlaps %s", i.name);
+  if (overlap(y_r, hout_r) || overlap(y_r, hin_r))
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "y overlaps a state buffer");
+  if (overlap(hout_r, hin_r) && h_out != h_in)
+    return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "h_out partially overlaps h_in");
+  if (!any) return ssd_ok();
+
+  ssd::StepArgs a{};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.dt = static_cast<const __nv_bfloat16*>(dt_raw);
+  a.A_log = A_log;
+  a.B = static_cast<const __nv_bfloat16*>(B);
+  a.C = static_cast<const __nv_bfloat16*>(C);
+  a.D = D;
+  a.dt_bias = dt_bias;
+  a.z = static_cast<const __nv_bfloat16*>(z);
+  a.h_in = h_in;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.h_out = h_out;
+  a.rows = int64_t(rows);
+  a.H = int(H);
+  a.G = int(G);
+  a.P = int(P);
+  const int64_t threads = int64_t(rows) * (N / 4);
+  const int64_t grid = (threads + ssd::kStepThreads - 1) / ssd::kStepThreads;
+  if (grid > 0x7fffffff) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "too many rows for one launch");
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (N == 128)
+    z ? ssd::ssd_step_kernel<128, true><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a)
+      : ssd::ssd_step_kernel<128, false><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a);
+  else
+    z ? ssd::ssd_step_kernel<64, true><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a)
+      : ssd::ssd_step_kernel<64, false><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "step launch failed: %s", cudaGetErrorString(e));
   return ssd_ok();
 }

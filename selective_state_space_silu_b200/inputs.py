@@ -263,6 +263,8 @@ SSD_WORKLOADS: Dict[str, SsdWorkload] = {
     "ssd_v3": SsdWorkload("ssd_v3", 8, 2048, 24, 64, 128, 1, 2001),
     # the same layer over 2 rows of 8192 tokens (the length the pages certify resets at)
     "ssd_v3_long": SsdWorkload("ssd_v3_long", 2, 8192, 24, 64, 128, 1, 2002),
+    # one decode step of the same layer for 256 sequences on cached states (gated)
+    "ssd_v3_decode": SsdWorkload("ssd_v3_decode", 256, 1, 24, 64, 128, 1, 2003, gate=True, state=True),
 }
 
 

@@ -13,7 +13,7 @@ import torch
 
 from . import mixer as _m
 
-EXPORTS = ("mamba2_ssd_fwd_workspace_bytes", "mamba2_ssd_fwd")
+EXPORTS = ("mamba2_ssd_fwd_workspace_bytes", "mamba2_ssd_fwd", "mamba2_ssd_step")
 
 
 class mamba2_dims(ctypes.Structure):
@@ -35,6 +35,8 @@ def _lib() -> ctypes.CDLL:
         lib.mamba2_ssd_fwd_workspace_bytes.argtypes = [ctypes.POINTER(mamba2_dims)]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
         lib.mamba2_ssd_fwd.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 13 + [ctypes.c_size_t, vp]
+        lib.mamba2_ssd_step.restype = ctypes.c_int
+        lib.mamba2_ssd_step.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 12
         _bound = lib
     return lib
 
@@ -80,5 +82,33 @@ def mamba2_ssd_fwd(x, dt_raw, A_log, B, C, D, dt_bias, *, z=None, seq_idx=None, 
         p(D, "D", f32, dev), p(dt_bias, "dt_bias", f32, dev), p(z, "z", iot, dev),
         p(seq_idx, "seq_idx", torch.int32, dev), p(h_in, "h_in", f32, dev), p(y, "y", iot, dev), p(h_out, "h_out", f32, dev),
         p(workspace, "workspace", None, dev), ws_bytes, _m._stream_handle(stream, dev))
+    _m._check(rc)
+    return y, h_out
+
+
+def mamba2_ssd_step(x, dt_raw, A_log, B, C, D, dt_bias, h_in, *, z=None, y=None, h_out=None,
+                    stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """One decode step: the layouts of mamba2_ssd_fwd with L = 1 (x, z [batch, 1, nheads, 64];
+    dt_raw [batch, 1, nheads]; B, C [batch, 1, ngroups, d_state]); h_in [batch, nheads, 64,
+    d_state] fp32.  Returns (y, h_out); pass h_out=h_in to update the state in place."""
+    lib = _lib()
+    dev = x.device
+    Bt, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = _m._io_code(x)
+    iot = x.dtype
+    f32 = torch.float32
+    if y is None:
+        y = torch.empty_like(x)
+    if h_out is None:
+        h_out = torch.empty(Bt, H, P, N, dtype=f32, device=dev)
+    dims = make_dims(Bt, L, H, P, N, G, io)
+    p = _m._ptr
+    rc = lib.mamba2_ssd_step(
+        ctypes.byref(dims), p(x, "x", iot, dev), p(dt_raw, "dt_raw", iot, dev),
+        p(A_log, "A_log", f32, dev), p(B, "B", iot, dev), p(C, "C", iot, dev),
+        p(D, "D", f32, dev), p(dt_bias, "dt_bias", f32, dev), p(z, "z", iot, dev),
+        p(h_in, "h_in", f32, dev), p(y, "y", iot, dev), p(h_out, "h_out", f32, dev),
+        _m._stream_handle(stream, dev))
     _m._check(rc)
     return y, h_out

@@ -158,3 +158,43 @@ def test_packed_variants(case):
     y, h = run_gpu(inp, h_in_inplace=in_place, seq_idx=ids)
     assert_close_tc(y, yo, f"y ({name})")
     assert_close_tc(h, ho, f"h_out ({name})")
+
+
+# ---------------------------------------------------------------- decode step
+def run_step(inp, in_place=False):
+    d = {k: (None if v is None else dev_tensor(v)) for k, v in inp.items()}
+    h_out = d["h_in"] if in_place else None
+    y, h = S.mamba2_ssd_step(d["x"], d["dt_raw"], d["A_log"], d["B"], d["C"], d["D"],
+                             d["dt_bias"], d["h_in"], z=d["z"], h_out=h_out)
+    torch.cuda.synchronize()
+    return host(y), host(h)
+
+
+@pytest.mark.parametrize("case", [(3, 4, 128, 1, True, False), (5, 6, 64, 3, False, True),
+                                  (1, 1, 64, 1, True, True), (2, 8, 128, 4, False, False)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_step_matches_oracle(case):
+    Bt, H, N, G, gate, in_place = case
+    inp = draw(Bt, 1, H, N, G, gate, True, seed=3700 + Bt * H)
+    yo, ho = run_oracle(inp)
+    y, h = run_step(inp, in_place)
+    assert_close_tc(y, yo, "step y")
+    assert_close_tc(h, ho, "step h")
+
+
+def test_prefill_then_steps_equal_forward():
+    # niverel-mamba 0.1.0, "Autoregressive decoding": concatenated steps equal the forward
+    Bt, L, H, N, k = 2, 100, 4, 128, 7
+    inp = draw(Bt, L, H, N, 2, True, True, seed=3800)
+    yo, ho = run_oracle(inp)
+    acts = ("x", "dt_raw", "B", "C", "z")
+    pre = {kk: (np.ascontiguousarray(v[:, :L - k]) if kk in acts else v) for kk, v in inp.items()}
+    y1, h = run_gpu(pre)
+    ys = [y1]
+    for t in range(L - k, L):
+        one = {kk: (np.ascontiguousarray(v[:, t:t + 1]) if kk in acts else v) for kk, v in inp.items()}
+        one["h_in"] = h.astype(np.float32)
+        yt, h = run_step(one, in_place=True)
+        ys.append(yt)
+    assert_close_tc(np.concatenate(ys, axis=1), yo, "prefill + steps y")
+    assert_close_tc(h, ho, "prefill + steps h")

@@ -130,3 +130,28 @@ def test_segment_plan(lib):
     assert _nseg(lib, batch=1, seqlen=65536, nheads=2) == 16      # at most 16
     assert _nseg(lib, batch=64, seqlen=4096, nheads=24) == 1      # pairs fill the GPU
     assert _nseg(lib, batch=1, seqlen=64, nheads=4) == 1          # one chunk
+
+
+STEP = ["x", "dt", "A_log", "B", "C", "D", "dt_bias", "z", "h_in", "y", "h_out"]
+
+
+def _step(lib, d, ptrs=None):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(STEP)}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba2_ssd_step(ctypes.byref(d), *[p[k] for k in STEP], None)
+
+
+def test_step_validation(lib):
+    assert _step(lib, dims(seqlen=2)) == 1
+    assert "one token" in M.mamba_last_error()
+    for k in ("x", "dt", "B", "C", "h_in", "y", "h_out"):
+        assert _step(lib, dims(seqlen=1), {k: None}) == 1, k
+    assert _step(lib, dims(seqlen=1, d_state=16)) == 2
+    assert _step(lib, dims(seqlen=1), {"h_in": _fake(0x8010000008)}) == 3
+    # a partial overlap of the states is rejected (exact aliasing, in place, is allowed:
+    # it passes validation, so it is exercised only by the GPU tests, never with fake pointers)
+    assert _step(lib, dims(seqlen=1), {"h_out": _fake(0x8010000100)}) == 1
+    assert _step(lib, dims(seqlen=1), {"y": _fake(0x10000000)}) == 1      # y on x
+    assert _step(lib, dims(seqlen=1, batch=0)) == 0
