@@ -10,9 +10,9 @@
 //   y[b,h,p] = C[b,g,:] . h[p, :] + D[h] x[b,h,p]     (times SiLU(z[b,h,p]) when z is given)
 //
 // The state (headdim x d_state fp32 per head) is nearly all of the bytes, so the kernel is
-// an HBM stream: each thread owns 4 consecutive states of one row (b, h, p) and moves
-// them with one 16-byte streaming load and store; the row's readout C . h is reduced with
-// xor shuffles over its d_state / 4 lanes.  In-place update (h_out == h_in) is safe: every
+// an HBM stream: each thread owns kStepStates consecutive states of one row (b, h, p) and
+// moves them with 16-byte streaming loads and stores; the row's readout C . h is reduced
+// with xor shuffles over its d_state / kStepStates lanes.  In-place update (h_out == h_in) is safe: every
 // element is read and then written by the same thread.
 #pragma once
 
@@ -40,46 +40,90 @@ struct StepArgs {
 };
 
 constexpr int kStepThreads = 256;
+#ifndef MM_SSD_STEP_STATES
+#define MM_SSD_STEP_STATES 8
+#endif
+// consecutive states per thread: 8 (two 16-byte loads of the state in flight per thread)
+// measured 69.8 us on 256 sequences x 24 heads x 64 x d_state 128 (0.89 of the measured
+// copy bandwidth), against 108.9 us with 4 and 90.6 us with 16
+constexpr int kStepStates = MM_SSD_STEP_STATES;
 
-// Grid: ceil(rows * N / 4 / kStepThreads) CTAs of kStepThreads threads.
-template <int N, bool kGate>
+// kS bf16 values as fp32 (kS = 4, 8 or 16), from 8- or 16-byte loads.
+template <int kS>
+__device__ __forceinline__ void ld_bf16s(const __nv_bfloat16* p, float* out) {
+  if constexpr (kS == 4) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+    out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
+    out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+  } else {
+#pragma unroll
+    for (int i = 0; i < kS / 8; ++i) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p) + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        out[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+        out[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+      }
+    }
+  }
+}
+
+// Grid: ceil(rows * N / kS / kStepThreads) CTAs of kStepThreads threads.
+template <int N, int kS, bool kGate>
 __global__ void __launch_bounds__(kStepThreads) ssd_step_kernel(const StepArgs a) {
-  constexpr int LPR = N / 4;  // lanes per row (32 or 16): a row never straddles warps
-  static_assert(LPR == 32 || LPR == 16, "d_state 128 or 64");
+  constexpr int LPR = N / kS;  // lanes per row: a row never straddles warps
+  static_assert(kS % 4 == 0 && LPR >= 4 && LPR <= 32 && 32 % LPR == 0, "states per thread");
+  static_assert(64 % (32 / LPR) == 0, "a warp's rows must share one (b, h) at headdim 64");
   const int64_t gt = int64_t(blockIdx.x) * kStepThreads + threadIdx.x;
-  const int64_t row = gt / LPR;  // (b, h, p) flattened
-  const int q = int(gt % LPR);   // this thread's states 4q .. 4q + 3
-  if (row >= a.rows) return;     // whole rows drop out together (LPR divides 32)
+  const int64_t grow = gt / LPR;  // (b, h, p) flattened
+  const int q = int(gt % LPR);    // this thread's states kS q .. kS q + kS - 1
+  // lanes past the last row work on the last row and store nothing, so that every shuffle
+  // below sees the whole warp
+  const bool valid = grow < a.rows;
+  const int64_t row = valid ? grow : a.rows - 1;
   const int64_t bh = row / a.P;
   const int h = int(bh % a.H);
   const int64_t b = bh / a.H;
   const int g = h / (a.H / a.G);
+  const int lane = threadIdx.x & 31;
 
-  const float4 hv = __ldcs(reinterpret_cast<const float4*>(a.h_in + row * N) + q);
-  const uint2 bb = __ldg(reinterpret_cast<const uint2*>(a.B + (b * a.G + g) * N) + q);
-  const uint2 cc = __ldg(reinterpret_cast<const uint2*>(a.C + (b * a.G + g) * N) + q);
+  float hv[kS], bv[kS], cv[kS];
+  const float4* hin = reinterpret_cast<const float4*>(a.h_in + row * N + kS * q);
+#pragma unroll
+  for (int i = 0; i < kS / 4; ++i) {
+    const float4 v = __ldcs(hin + i);
+    hv[4 * i] = v.x; hv[4 * i + 1] = v.y; hv[4 * i + 2] = v.z; hv[4 * i + 3] = v.w;
+  }
+  ld_bf16s<kS>(a.B + (b * a.G + g) * N + kS * q, bv);
+  ld_bf16s<kS>(a.C + (b * a.G + g) * N + kS * q, cv);
   const float xv = __bfloat162float(a.x[row]);
-  const float dtr = __bfloat162float(a.dt[bh]);
-  const float A2 = -mm::ex2_approx(__ldg(a.A_log + h) * mm::kLog2e) * mm::kLog2e;  // A log2 e
-  const float delta = mm::Math<false>::softplus(dtr + __ldg(a.dt_bias + h));
-  const float dec = mm::ex2_approx(delta * A2);
+  // Delta and the decay depend on (b, h) only, and a warp's 32 / LPR consecutive rows share
+  // one (b, h) (headdim 64 is a multiple of them): lane 0 computes them for the warp
+  float delta = 0.f, dec = 0.f;
+  if (lane == 0) {
+    const float dtr = __bfloat162float(a.dt[bh]);
+    const float A2 = -mm::ex2_approx(__ldg(a.A_log + h) * mm::kLog2e) * mm::kLog2e;  // A log2 e
+    delta = mm::Math<false>::softplus(dtr + __ldg(a.dt_bias + h));
+    dec = mm::ex2_approx(delta * A2);
+  }
+  delta = __shfl_sync(0xffffffffu, delta, 0);
+  dec = __shfl_sync(0xffffffffu, dec, 0);
   const float dx = delta * xv;
 
-  const float b0 = __uint_as_float(bb.x << 16), b1 = __uint_as_float(bb.x & 0xffff0000u);
-  const float b2 = __uint_as_float(bb.y << 16), b3 = __uint_as_float(bb.y & 0xffff0000u);
-  const float c0 = __uint_as_float(cc.x << 16), c1 = __uint_as_float(cc.x & 0xffff0000u);
-  const float c2 = __uint_as_float(cc.y << 16), c3 = __uint_as_float(cc.y & 0xffff0000u);
-  float4 ho;
-  ho.x = fmaf(dec, hv.x, dx * b0);
-  ho.y = fmaf(dec, hv.y, dx * b1);
-  ho.z = fmaf(dec, hv.z, dx * b2);
-  ho.w = fmaf(dec, hv.w, dx * b3);
-  float part = c0 * ho.x + c1 * ho.y + c2 * ho.z + c3 * ho.w;
-  // only this row's lanes: with 16 lanes per row the other half-warp may have exited
-  const unsigned mask = LPR == 32 ? 0xffffffffu : (0xffffu << (threadIdx.x & 16));
+  float part = 0.f;
 #pragma unroll
-  for (int o = 1; o < LPR; o <<= 1) part += __shfl_xor_sync(mask, part, o);
-  __stcs(reinterpret_cast<float4*>(a.h_out + row * N) + q, ho);
+  for (int i = 0; i < kS; ++i) {
+    hv[i] = fmaf(dec, hv[i], dx * bv[i]);
+    part = fmaf(cv[i], hv[i], part);
+  }
+#pragma unroll
+  for (int o = 1; o < LPR; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if (!valid) return;
+  float4* hout = reinterpret_cast<float4*>(a.h_out + row * N + kS * q);
+#pragma unroll
+  for (int i = 0; i < kS / 4; ++i)
+    __stcs(hout + i, make_float4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]));
   if (q == 0) {
     float out = part + __ldg(a.D + h) * xv;
     if constexpr (kGate) out *= mm::Math<false>::silu(__bfloat162float(a.z[row]));
