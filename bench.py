@@ -130,6 +130,7 @@ KERNEL_SOURCES = {
     "fwd": ("fwd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
     "step": ("step.cuh", "device_math.cuh", "sm100_primitives.cuh"),
     "ssd": ("ssd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
+    "ssd_step": ("ssd_step.cuh", "device_math.cuh"),
 }
 
 
@@ -658,7 +659,7 @@ def run_ssd(args, w, local_rank: int):
                      "tensor_frac": None if step else round(tflops / bf16_peak, 4),
                      "tensor_peak_source": "measured cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops)",
                      "floor_frac": round(t_floor / (ms * 1e-3), 4),
-                     "traffic": recorded_traffic("ssd", w.name)},
+                     "traffic": recorded_traffic("ssd_step" if step else "ssd", w.name)},
         "gpu_launches": args.steps, "clocks": clk.summary(),
     }
 

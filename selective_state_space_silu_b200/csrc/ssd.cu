@@ -266,6 +266,8 @@ extern "C" MAMBA_API int mamba2_ssd_step(const mamba2_dims* dims, const void* x,
   if (overlap(hout_r, hin_r) && h_out != h_in)
     return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "h_out partially overlaps h_in");
   if (!any) return ssd_ok();
+  if (H > (int64_t(0x7fffffff) / 4))
+    return ssd_fail(MAMBA_ERR_UNSUPPORTED, "nheads %lld too large for the step's grid", (long long)H);
 
   ssd::StepArgs a{};
   a.x = static_cast<const __nv_bfloat16*>(x);
@@ -279,20 +281,20 @@ extern "C" MAMBA_API int mamba2_ssd_step(const mamba2_dims* dims, const void* x,
   a.h_in = h_in;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.h_out = h_out;
-  a.rows = int64_t(rows);
   a.H = int(H);
   a.G = int(G);
-  a.P = int(P);
-  const int64_t threads = int64_t(rows) * (N / 4);
-  const int64_t grid = (threads + ssd::kStepThreads - 1) / ssd::kStepThreads;
-  if (grid > 0x7fffffff) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "too many rows for one launch");
+  (void)P;  // headdim is 64 (checked above)
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
-  if (N == 128)
-    z ? ssd::ssd_step_kernel<128, true><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a)
-      : ssd::ssd_step_kernel<128, false><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a);
-  else
-    z ? ssd::ssd_step_kernel<64, true><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a)
-      : ssd::ssd_step_kernel<64, false><<<unsigned(grid), ssd::kStepThreads, 0, st>>>(a);
+  constexpr int kS = ssd::kStepStates;
+  if (N == 128) {
+    const dim3 grid(unsigned(H * ssd::StepShape<128, kS>::kCtaPerHead), unsigned(Bt));
+    z ? ssd::ssd_step_kernel<128, kS, true><<<grid, ssd::kStepThreads, 0, st>>>(a)
+      : ssd::ssd_step_kernel<128, kS, false><<<grid, ssd::kStepThreads, 0, st>>>(a);
+  } else {
+    const dim3 grid(unsigned(H * ssd::StepShape<64, kS>::kCtaPerHead), unsigned(Bt));
+    z ? ssd::ssd_step_kernel<64, kS, true><<<grid, ssd::kStepThreads, 0, st>>>(a)
+      : ssd::ssd_step_kernel<64, kS, false><<<grid, ssd::kStepThreads, 0, st>>>(a);
+  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "step launch failed: %s", cudaGetErrorString(e));
   return ssd_ok();

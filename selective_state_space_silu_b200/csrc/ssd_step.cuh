@@ -35,8 +35,7 @@ struct StepArgs {
   const float* h_in;        // [Bt, H, P, N]
   __nv_bfloat16* y;         // [Bt, H, P]
   float* h_out;             // [Bt, H, P, N]
-  int64_t rows;             // Bt * H * P
-  int H, G, P;
+  int H, G;
 };
 
 constexpr int kStepThreads = 256;
@@ -69,24 +68,42 @@ __device__ __forceinline__ void ld_bf16s(const __nv_bfloat16* p, float* out) {
   }
 }
 
-// Grid: ceil(rows * N / kS / kStepThreads) CTAs of kStepThreads threads.
+// Rows (b, h, p) per CTA and CTAs per (b, h): headdim is 64.
+template <int N, int kS>
+struct StepShape {
+  static constexpr int kLpr = N / kS;                    // lanes per row
+  static constexpr int kRowsPerCta = kStepThreads / kLpr;
+  static constexpr int kCtaPerHead = 64 / kRowsPerCta;
+};
+
+// Grid: (H * kCtaPerHead, Bt) CTAs of kStepThreads threads; every index is a shift.
 template <int N, int kS, bool kGate>
 __global__ void __launch_bounds__(kStepThreads) ssd_step_kernel(const StepArgs a) {
-  constexpr int LPR = N / kS;  // lanes per row: a row never straddles warps
+  using Sh = StepShape<N, kS>;
+  constexpr int LPR = Sh::kLpr;  // lanes per row: a row never straddles warps
   static_assert(kS % 4 == 0 && LPR >= 4 && LPR <= 32 && 32 % LPR == 0, "states per thread");
-  static_assert(64 % (32 / LPR) == 0, "a warp's rows must share one (b, h) at headdim 64");
-  const int64_t gt = int64_t(blockIdx.x) * kStepThreads + threadIdx.x;
-  const int64_t grow = gt / LPR;  // (b, h, p) flattened
-  const int q = int(gt % LPR);    // this thread's states kS q .. kS q + kS - 1
-  // lanes past the last row work on the last row and store nothing, so that every shuffle
-  // below sees the whole warp
-  const bool valid = grow < a.rows;
-  const int64_t row = valid ? grow : a.rows - 1;
-  const int64_t bh = row / a.P;
-  const int h = int(bh % a.H);
-  const int64_t b = bh / a.H;
-  const int g = h / (a.H / a.G);
+  static_assert(64 % Sh::kRowsPerCta == 0, "a CTA's rows must belong to one (b, h)");
+  const int h = blockIdx.x / Sh::kCtaPerHead;
+  const int64_t b = blockIdx.y;
+  const int p = (blockIdx.x % Sh::kCtaPerHead) * Sh::kRowsPerCta + threadIdx.x / LPR;
+  const int q = threadIdx.x % LPR;  // this thread's states kS q .. kS q + kS - 1
+  const int64_t bh = b * a.H + h;
+  const int64_t row = bh * 64 + p;
   const int lane = threadIdx.x & 31;
+  // Delta, the decay and the group depend on (b, h) only, shared by the whole CTA: lane 0
+  // of each warp computes them and broadcasts them
+  float delta = 0.f, dec = 0.f;
+  int g = 0;
+  if (lane == 0) {
+    const float dtr = __bfloat162float(a.dt[bh]);
+    const float A2 = -mm::ex2_approx(__ldg(a.A_log + h) * mm::kLog2e) * mm::kLog2e;  // A log2 e
+    delta = mm::Math<false>::softplus(dtr + __ldg(a.dt_bias + h));
+    dec = mm::ex2_approx(delta * A2);
+    g = h / (a.H / a.G);
+  }
+  delta = __shfl_sync(0xffffffffu, delta, 0);
+  dec = __shfl_sync(0xffffffffu, dec, 0);
+  g = __shfl_sync(0xffffffffu, g, 0);
 
   float hv[kS], bv[kS], cv[kS];
   const float4* hin = reinterpret_cast<const float4*>(a.h_in + row * N + kS * q);
@@ -98,17 +115,6 @@ __global__ void __launch_bounds__(kStepThreads) ssd_step_kernel(const StepArgs a
   ld_bf16s<kS>(a.B + (b * a.G + g) * N + kS * q, bv);
   ld_bf16s<kS>(a.C + (b * a.G + g) * N + kS * q, cv);
   const float xv = __bfloat162float(a.x[row]);
-  // Delta and the decay depend on (b, h) only, and a warp's 32 / LPR consecutive rows share
-  // one (b, h) (headdim 64 is a multiple of them): lane 0 computes them for the warp
-  float delta = 0.f, dec = 0.f;
-  if (lane == 0) {
-    const float dtr = __bfloat162float(a.dt[bh]);
-    const float A2 = -mm::ex2_approx(__ldg(a.A_log + h) * mm::kLog2e) * mm::kLog2e;  // A log2 e
-    delta = mm::Math<false>::softplus(dtr + __ldg(a.dt_bias + h));
-    dec = mm::ex2_approx(delta * A2);
-  }
-  delta = __shfl_sync(0xffffffffu, delta, 0);
-  dec = __shfl_sync(0xffffffffu, dec, 0);
   const float dx = delta * xv;
 
   float part = 0.f;
@@ -119,7 +125,6 @@ __global__ void __launch_bounds__(kStepThreads) ssd_step_kernel(const StepArgs a
   }
 #pragma unroll
   for (int o = 1; o < LPR; o <<= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  if (!valid) return;
   float4* hout = reinterpret_cast<float4*>(a.h_out + row * N + kS * q);
 #pragma unroll
   for (int i = 0; i < kS / 4; ++i)
