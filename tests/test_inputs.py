@@ -39,3 +39,23 @@ def test_distributions():
     dt0 = np.logaddexp(0.0, a["dt_bias"].astype(np.float64))   # softplus(dt_bias) = dt0
     assert dt0.min() >= 1e-3 * (1 - 1e-5) and dt0.max() <= 1e-1 * (1 + 1e-5)
     assert np.all(np.abs(a["conv_w"]) <= 0.5) and np.all(a["D"] == 1.0)
+
+
+def test_ssd_inputs_shapes_determinism_distributions():
+    w = I.SsdWorkload("t", 3, 50, 6, 64, 128, 2, 77, gate=True, state=True)
+    a = I.make_ssd_inputs(w)
+    b = I.make_ssd_inputs(w)
+    for k in a:
+        np.testing.assert_array_equal(a[k], b[k])
+    assert a["x"].shape == (3, 50, 6, 64) and a["z"].shape == (3, 50, 6, 64)
+    assert a["dt_raw"].shape == (3, 50, 6) and a["B"].shape == (3, 50, 2, 128)
+    assert a["A_log"].shape == (6,) and a["h_in"].shape == (3, 6, 64, 128)
+    assert a["x"].dtype == np.uint16 and a["h_in"].dtype == np.float32
+    A = np.exp(a["A_log"].astype(np.float64))
+    assert (A >= 1.0 - 1e-6).all() and (A <= 16.0 + 1e-5).all()
+    dt0 = np.logaddexp(0.0, a["dt_bias"].astype(np.float64))
+    assert dt0.min() >= 1e-3 * (1 - 1e-5) and dt0.max() <= 1e-1 * (1 + 1e-5)
+    big = I.make_ssd_inputs(I.SsdWorkload("u", 4, 512, 8, 64, 64, 1, 78))
+    x = I.bf16_bits_to_f32(big["x"])
+    assert abs(x.std() - 1.0) < 0.01 and big["z"] is None and big["h_in"] is None
+    assert abs(I.bf16_bits_to_f32(big["dt_raw"]).std() - 0.5) < 0.02
