@@ -23,6 +23,10 @@ only: no chunking, no reordering.  The chunked (quadratic-within-a-chunk) evalua
 what the CUDA path does; tests/test_oracle_ssd.py checks this oracle against that form
 written out independently, an O(L^2) unrolled sum, closed forms and numpy.cumsum.
 
+The same module holds the layer's two neighbours of the scan: conv_silu (the causal
+depthwise conv + SiLU over the concatenated x, B, C channels) and gated_rmsnorm (the norm
+of y * SiLU(z)).
+
 Parity status: pinned (tests/test_oracle_ssd.py).
 """
 
@@ -114,3 +118,63 @@ def ssd_channels(x, dt_raw, A_log, B, C, D, dt_bias, sel, z=None, h_in=None, seq
         outs.append(o[0, :, 0])
         hs.append(hf[0, 0])
     return outs, hs
+
+
+def conv_silu(xbc, conv_w, conv_b=None, seq_idx=None, conv_state_in=None):
+    """The Mamba2 layer's causal depthwise conv + SiLU over the concatenated x, B, C channels
+    (niverel-mamba 0.1.0, section "The weight contract": conv1d.weight [channels, 1, 4] and
+    conv1d.bias over d_inner + 2 ngroups d_state channels), fp64, one step at a time.
+
+    xbc [Bt, L, Cc] (floats or bf16 bit patterns); conv_w [Cc, K]; conv_b [Cc] or None;
+    conv_state_in [Bt, Cc, K - 1] (the K - 1 inputs before step 0, oldest first) or None
+    (zeros).  out[b, t, c] = SiLU(conv_b[c] + sum_k conv_w[c, k] * xpad[b, t + k, c]) with
+    xpad = [conv state ; xbc] (cross-correlation, left padding; conv_w[c, K - 1] multiplies
+    the current input).  With seq_idx, a tap reads zero when an id change lies between its
+    input's step and t (the conv state resets where the id changes; the state before step 0
+    belongs to the row's first document).  Returns (out [Bt, L,
+    Cc], conv_state_out [Bt, Cc, K - 1] = the last K - 1 entries of xpad, zeroed where they
+    precede the last document's first step).
+    """
+    x = as_f64(xbc)
+    Bt, L, Cc = x.shape
+    w = np.asarray(conv_w, dtype=np.float64)
+    K = w.shape[1]
+    bias = np.zeros(Cc) if conv_b is None else np.asarray(conv_b, dtype=np.float64)
+    st = np.zeros((Bt, Cc, K - 1)) if conv_state_in is None else as_f64(conv_state_in)
+    xpad = np.concatenate([np.transpose(st, (0, 2, 1)), x], axis=1)   # [Bt, K-1+L, Cc]
+    ids = None if seq_idx is None else np.asarray(seq_idx)
+    out = np.empty((Bt, L, Cc))
+    for b in range(Bt):
+        for t in range(L):
+            acc = bias.copy()
+            for k in range(K):
+                src = t + k - (K - 1)          # time of the tap's input (negative: the state)
+                # the tap is dropped when a reset (an id change) lies in (src, t]
+                if ids is not None and np.any(ids[b, max(src, 0):t + 1] != ids[b, t]):
+                    continue
+                acc = acc + w[:, k] * xpad[b, t + k]
+            out[b, t] = _silu(acc)
+    cs = np.transpose(xpad[:, L:L + K - 1], (0, 2, 1)).copy()         # [Bt, Cc, K-1]
+    if ids is not None and L > 0:
+        for b in range(Bt):
+            for j in range(K - 1):
+                src = L - (K - 1) + j          # time of the slot's input (negative: the state)
+                if np.any(ids[b, max(src, 0):L] != ids[b, L - 1]):
+                    cs[b, :, j] = 0.0
+    return out, cs
+
+
+def gated_rmsnorm(y, z, weight, eps=1e-5, group_size=None):
+    """The Mamba2 layer's gated RMSNorm with the gate before the norm (niverel-mamba 0.1.0,
+    section "The weight contract": norm.weight over d_inner, eps 1e-5): g = y * SiLU(z);
+    out = g / sqrt(mean(g^2) + eps) * weight, the mean over each group of group_size
+    consecutive channels (d_inner when None).  y, z [..., d_inner]; fp64."""
+    yy = as_f64(y)
+    zz = as_f64(z)
+    w = np.asarray(weight, dtype=np.float64)
+    D = yy.shape[-1]
+    gs = D if group_size is None else int(group_size)
+    g = yy * _silu(zz)
+    gg = g.reshape(g.shape[:-1] + (D // gs, gs))
+    r = 1.0 / np.sqrt(np.mean(gg * gg, axis=-1, keepdims=True) + eps)
+    return (gg * r).reshape(g.shape) * w

@@ -14,6 +14,11 @@
 
 A dropped term, a wrong sign of A, a swapped B/C, a transposed state, a wrong group
 mapping or a missed reset each fail at least one of these.
+
+The layer's conv + SiLU over x, B, C is pinned against numpy.convolve with
+scipy.special.expit, the conv-state orientation for L = 0..5, and a packed row against its
+documents run alone; the gated RMSNorm against unit mean square per row or group, scale
+invariance, the separate-group identity and the gate's direction.
 """
 
 import numpy as np
@@ -281,3 +286,99 @@ def test_channel_subset():
     for (b, h), o, hf in zip(sel, outs, hs):
         close(o, y[b, :, h])
         close(hf, hT[b, h])
+
+
+# ---------------------------------------------------------------- conv + SiLU over x, B, C
+def _np_conv_silu(x_bc, w_c, b_c, state_c=None):
+    """One channel through numpy.convolve over the left-padded sequence, then SiLU."""
+    K = w_c.shape[0]
+    pad = np.zeros(K - 1) if state_c is None else np.asarray(state_c, dtype=np.float64)
+    xpad = np.concatenate([pad, x_bc])
+    pre = np.convolve(xpad, w_c[::-1], mode="valid") + b_c
+    return silu(pre), xpad[-(K - 1):]
+
+
+def test_conv_matches_numpy_convolve():
+    r = np.random.default_rng(200)
+    Bt, L, Cc, K = 2, 11, 5, 4
+    x = r.standard_normal((Bt, L, Cc))
+    w = r.standard_normal((Cc, K))
+    bias = r.standard_normal(Cc)
+    st = r.standard_normal((Bt, Cc, K - 1))
+    out, cs = so.conv_silu(x, w, bias, conv_state_in=st)
+    for b in range(Bt):
+        for c in range(Cc):
+            o, last = _np_conv_silu(x[b, :, c], w[c], bias[c], st[b, c])
+            close(out[b, :, c], o)
+            close(cs[b, c], last)
+    out0, cs0 = so.conv_silu(x, w)
+    o, last = _np_conv_silu(x[1, :, 3], w[3], 0.0)
+    close(out0[1, :, 3], o)
+    close(cs0[1, 3], last)
+
+
+@pytest.mark.parametrize("L", [0, 1, 2, 3, 5])
+def test_conv_state_out_orientation(L):
+    r = np.random.default_rng(210 + L)
+    x = r.standard_normal((1, L, 2))
+    st = r.standard_normal((1, 2, 3))
+    _, cs = so.conv_silu(x, r.standard_normal((2, 4)), conv_state_in=st)
+    expect = np.concatenate([st[0].T, x[0]], axis=0)[-3:].T          # last 3 of [state; x]
+    close(cs[0], expect)
+
+
+def test_conv_packed_row_equals_documents():
+    r = np.random.default_rng(220)
+    L, Cc = 14, 3
+    x = r.standard_normal((1, L, Cc))
+    w = r.standard_normal((Cc, 4))
+    bias = r.standard_normal(Cc)
+    st = r.standard_normal((1, Cc, 3))
+    ids = np.array([[4, 4, 4, 4, 4, 7, 7, 1, 1, 1, 1, 1, 1, 1]])
+    out, cs = so.conv_silu(x, w, bias, seq_idx=ids, conv_state_in=st)
+    o0, _ = so.conv_silu(x[:, 0:5], w, bias, conv_state_in=st)        # first document: the state
+    o1, _ = so.conv_silu(x[:, 5:7], w, bias)
+    o2, c2 = so.conv_silu(x[:, 7:], w, bias)
+    close(out, np.concatenate([o0, o1, o2], axis=1))
+    close(cs, c2)
+    # a repeated id after another document still resets (changes count, not values)
+    ids2 = np.array([[4, 4, 4, 4, 4, 7, 7, 4, 4, 4, 4, 4, 4, 4]])
+    out2, _ = so.conv_silu(x, w, bias, seq_idx=ids2, conv_state_in=st)
+    close(out2, out)
+    # a short last document: the state slots before it are zero
+    ids3 = np.array([[4] * 13 + [9]])
+    _, cs3 = so.conv_silu(x, w, bias, seq_idx=ids3, conv_state_in=st)
+    close(cs3[0, :, :2], np.zeros((Cc, 2)))
+    close(cs3[0, :, 2], x[0, -1])
+
+
+# ---------------------------------------------------------------- gated RMSNorm
+def test_gated_rmsnorm_unit_mean_square_and_weight():
+    r = np.random.default_rng(230)
+    y, z = r.standard_normal((3, 5, 24)), r.standard_normal((3, 5, 24))
+    out = so.gated_rmsnorm(y, z, np.ones(24), eps=0.0)
+    close(np.mean(out ** 2, axis=-1), np.ones((3, 5)))                  # unit RMS per row
+    g = y * expit(z) * z
+    close(out * np.sqrt(np.mean(g ** 2, axis=-1, keepdims=True)), g)     # direction of the gated input
+    w = r.standard_normal(24)
+    close(so.gated_rmsnorm(y, z, w, eps=0.0), out * w)
+
+
+def test_gated_rmsnorm_scale_invariance_and_eps():
+    r = np.random.default_rng(240)
+    y, z = r.standard_normal((4, 16)), r.standard_normal((4, 16))
+    w = r.standard_normal(16)
+    close(so.gated_rmsnorm(7.5 * y, z, w, eps=0.0), so.gated_rmsnorm(y, z, w, eps=0.0))
+    # eps matters only against the mean square: a tiny input is pulled toward zero
+    tiny = so.gated_rmsnorm(1e-4 * y, z, w, eps=1e-5)
+    assert np.max(np.abs(tiny)) < 0.1 * np.max(np.abs(so.gated_rmsnorm(y, z, w, eps=1e-5)))
+
+
+def test_gated_rmsnorm_groups_are_separate_norms():
+    r = np.random.default_rng(250)
+    y, z = r.standard_normal((2, 3, 32)), r.standard_normal((2, 3, 32))
+    w = r.standard_normal(32)
+    out = so.gated_rmsnorm(y, z, w, group_size=8)
+    for gi in range(4):
+        sl = slice(8 * gi, 8 * gi + 8)
+        close(out[..., sl], so.gated_rmsnorm(y[..., sl], z[..., sl], w[sl]))
