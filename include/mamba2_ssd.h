@@ -109,6 +109,49 @@ MAMBA_API int mamba2_ssd_step(const mamba2_dims* dims, const void* x, const void
                               const float* dt_bias, const void* z, const float* h_in, void* y,
                               float* h_out, void* cuda_stream);
 
+/*
+ * The layer's causal depthwise conv + SiLU before the scan, over the concatenated channels
+ * x | B | C (niverel-mamba 0.1.0, section "The weight contract": conv1d over d_inner +
+ * 2 ngroups d_state channels, 4 taps):
+ *
+ *   out[b,t,c] = SiLU(conv_b[c] + sum_{k<4} conv_w[c,k] * xpad[b,t+k,c]),
+ *   xpad = [conv_state_in (3 inputs, oldest first; zeros when NULL) ; xbc]
+ *
+ * with conv_w[c, 3] on the current input.  With seq_idx [batch, seqlen] (may be NULL) a tap
+ * reads zero when an id change lies between its input's step and t (the state before step 0
+ * belongs to the row's first document).  The output is split as the scan takes it:
+ *
+ *   xbc                          [batch, seqlen, Cc]            bf16, Cc = nheads*64 + 2*ngroups*d_state
+ *   conv_w                       [Cc, 4]                        fp32 (16-byte aligned)
+ *   conv_b                       [Cc]                           fp32 or NULL
+ *   x                            [batch, seqlen, nheads*64]     bf16 (channels 0 .. nheads*64-1)
+ *   B, C                         [batch, seqlen, ngroups*d_state] bf16 (the next two blocks)
+ *   conv_state_in / _out         [batch, Cc, 3]                 bf16 or NULL
+ *
+ * conv_state_out receives the last 3 entries of xpad (zero where an id change lies between
+ * the entry's step and the last step); it may not overlap conv_state_in.  Outputs may not
+ * overlap inputs or each other.  SiLU and the sums are fp32; outputs round to nearest even.
+ */
+MAMBA_API int mamba2_conv_silu(const mamba2_dims* dims, const void* xbc, const float* conv_w,
+                               const float* conv_b, const int32_t* seq_idx,
+                               const void* conv_state_in, void* x, void* B, void* C,
+                               void* conv_state_out, void* cuda_stream);
+
+/*
+ * The layer's gated RMSNorm after the scan, gate first (niverel-mamba 0.1.0, section "The
+ * weight contract": norm.weight over d_inner, eps 1e-5):
+ *
+ *   g = y * SiLU(z);  out = g / sqrt(mean(g^2) + eps) * weight
+ *
+ * the mean over each group of nheads*64/ngroups consecutive channels of a (b, t).  y, z, out
+ * [batch, seqlen, nheads*64] bf16 (16-byte aligned); weight [nheads*64] fp32 (16-byte
+ * aligned); eps >= 0.  out may not overlap an input.  fp32 arithmetic.  dims->d_state is
+ * not used (it must still be 64 or 128).
+ */
+MAMBA_API int mamba2_gated_rmsnorm(const mamba2_dims* dims, const void* y, const void* z,
+                                   const float* weight, float eps, void* out,
+                                   void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

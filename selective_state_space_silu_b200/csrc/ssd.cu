@@ -8,6 +8,7 @@
 #include "mamba2_ssd.h"
 #include "ssd_kernel.cuh"
 #include "ssd_step.cuh"
+#include "ssd_layer.cuh"
 
 namespace mm_internal {
 void set_last_error(const char* msg);  // mamba_mixer.cu: the message mamba_last_error returns
@@ -297,5 +298,107 @@ extern "C" MAMBA_API int mamba2_ssd_step(const mamba2_dims* dims, const void* x,
   }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "step launch failed: %s", cudaGetErrorString(e));
+  return ssd_ok();
+}
+
+extern "C" MAMBA_API int mamba2_conv_silu(const mamba2_dims* dims, const void* xbc,
+                                          const float* conv_w, const float* conv_b,
+                                          const int32_t* seq_idx, const void* conv_state_in,
+                                          void* x, void* B, void* C, void* conv_state_out,
+                                          void* cuda_stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const int64_t Bt = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
+                N = dims->d_state, G = dims->ngroups;
+  const int64_t DI = H * P, GN = G * N, Cc = DI + 2 * GN;
+  if (Cc > (int64_t(1) << 24)) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "too many channels");
+  const size_t act = size_t(Bt * L * Cc), cst = size_t(Bt * Cc * 3);
+  const bool any = Bt > 0 && Cc > 0;
+  const bool rows = any && L > 0;
+  if ((rc = need(xbc, "xbc", rows, 16)) || (rc = need(conv_w, "conv_w", any, 16)) ||
+      (rc = need(conv_b, "conv_b", false, 4)) || (rc = need(seq_idx, "seq_idx", false, 4)) ||
+      (rc = need(conv_state_in, "conv_state_in", false, 2)) ||
+      (rc = need(x, "x", rows, 16)) || (rc = need(B, "B", rows && GN > 0, 16)) ||
+      (rc = need(C, "C", rows && GN > 0, 16)) ||
+      (rc = need(conv_state_out, "conv_state_out", false, 2)))
+    return rc;
+  const Range ins[] = {{xbc, act * 2, "xbc"}, {conv_w, size_t(Cc) * 16, "conv_w"},
+                       {conv_b, size_t(Cc) * 4, "conv_b"}, {seq_idx, size_t(Bt * L) * 4, "seq_idx"},
+                       {conv_state_in, cst * 2, "conv_state_in"}};
+  const Range outs[] = {{x, size_t(Bt * L * DI) * 2, "x"}, {B, size_t(Bt * L * GN) * 2, "B"},
+                        {C, size_t(Bt * L * GN) * 2, "C"}, {conv_state_out, cst * 2, "conv_state_out"}};
+  for (const Range& o : outs) {
+    for (const Range& i : ins)
+      if (overlap(o, i)) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, i.name);
+    for (const Range& o2 : outs)
+      if (&o != &o2 && overlap(o, o2))
+        return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "%s overlaps %s", o.name, o2.name);
+  }
+  if (!any) return ssd_ok();
+  ssd::ConvArgs a{};
+  a.xbc = static_cast<const __nv_bfloat16*>(xbc);
+  a.w = conv_w;
+  a.bias = conv_b;
+  a.seq_idx = seq_idx;
+  a.cs_in = static_cast<const __nv_bfloat16*>(conv_state_in);
+  a.x = static_cast<__nv_bfloat16*>(x);
+  a.B = static_cast<__nv_bfloat16*>(B);
+  a.C = static_cast<__nv_bfloat16*>(C);
+  a.cs_out = static_cast<__nv_bfloat16*>(conv_state_out);
+  a.L = L;
+  a.Cc = int(Cc);
+  a.DI = int(DI);
+  a.GN = int(GN);
+  if (L == 0 && !conv_state_out) return ssd_ok();
+  const int64_t tiles = L > 0 ? (L + ssd::kConvSteps - 1) / ssd::kConvSteps : 1;  // L = 0: the state
+  if (tiles > 65535) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "seqlen too long for one launch");
+  const dim3 grid(unsigned((Cc / 8 + ssd::kConvThreads - 1) / ssd::kConvThreads), unsigned(tiles),
+                  unsigned(Bt));
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (seq_idx)
+    ssd::conv_silu_kernel<true><<<grid, ssd::kConvThreads, 0, st>>>(a);
+  else
+    ssd::conv_silu_kernel<false><<<grid, ssd::kConvThreads, 0, st>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "conv launch failed: %s", cudaGetErrorString(e));
+  return ssd_ok();
+}
+
+extern "C" MAMBA_API int mamba2_gated_rmsnorm(const mamba2_dims* dims, const void* y, const void* z,
+                                              const float* weight, float eps, void* out,
+                                              void* cuda_stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  const int64_t Bt = dims->batch, L = dims->seqlen, H = dims->nheads, P = dims->headdim,
+                G = dims->ngroups;
+  const int64_t D = H * P, rows = Bt * L;
+  if (!(eps >= 0.f)) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "eps must be >= 0");
+  if (D > (int64_t(1) << 24)) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "too many channels");
+  const size_t act = size_t(rows * D);
+  const bool any = act > 0;
+  if ((rc = need(y, "y", any, 16)) || (rc = need(z, "z", any, 16)) ||
+      (rc = need(weight, "weight", any, 16)) || (rc = need(out, "out", any, 16)))
+    return rc;
+  const Range out_r{out, act * 2, "out"};
+  const Range ins[] = {{y, act * 2, "y"}, {z, act * 2, "z"}, {weight, size_t(D) * 4, "weight"}};
+  for (const Range& i : ins)
+    if (overlap(out_r, i)) return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "out overlaps %s", i.name);
+  if (!any) return ssd_ok();
+  ssd::NormArgs a{};
+  a.y = static_cast<const __nv_bfloat16*>(y);
+  a.z = static_cast<const __nv_bfloat16*>(z);
+  a.w = weight;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.rows = rows;
+  a.D = int(D);
+  a.gs = int(D / G);
+  a.eps = eps;
+  const int64_t items = rows * G;
+  const int64_t grid = (items + ssd::kNormWarps - 1) / ssd::kNormWarps;
+  if (grid > 0x7fffffff) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "too many rows for one launch");
+  ssd::gated_rmsnorm_kernel<<<unsigned(grid), ssd::kNormWarps * 32, 0,
+                              static_cast<cudaStream_t>(cuda_stream)>>>(a);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "norm launch failed: %s", cudaGetErrorString(e));
   return ssd_ok();
 }

@@ -13,7 +13,8 @@ import torch
 
 from . import mixer as _m
 
-EXPORTS = ("mamba2_ssd_fwd_workspace_bytes", "mamba2_ssd_fwd", "mamba2_ssd_step")
+EXPORTS = ("mamba2_ssd_fwd_workspace_bytes", "mamba2_ssd_fwd", "mamba2_ssd_step",
+           "mamba2_conv_silu", "mamba2_gated_rmsnorm")
 
 
 class mamba2_dims(ctypes.Structure):
@@ -37,6 +38,11 @@ def _lib() -> ctypes.CDLL:
         lib.mamba2_ssd_fwd.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 13 + [ctypes.c_size_t, vp]
         lib.mamba2_ssd_step.restype = ctypes.c_int
         lib.mamba2_ssd_step.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 12
+        lib.mamba2_conv_silu.restype = ctypes.c_int
+        lib.mamba2_conv_silu.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 10
+        lib.mamba2_gated_rmsnorm.restype = ctypes.c_int
+        lib.mamba2_gated_rmsnorm.argtypes = [ctypes.POINTER(mamba2_dims), vp, vp, vp,
+                                             ctypes.c_float, vp, vp]
         _bound = lib
     return lib
 
@@ -112,3 +118,55 @@ def mamba2_ssd_step(x, dt_raw, A_log, B, C, D, dt_bias, h_in, *, z=None, y=None,
         _m._stream_handle(stream, dev))
     _m._check(rc)
     return y, h_out
+
+
+def mamba2_conv_silu(xbc, conv_w, conv_b=None, *, nheads, ngroups, d_state, seq_idx=None,
+                     conv_state_in=None, want_state: bool = True, stream=None):
+    """Causal conv + SiLU over the concatenated x | B | C channels of the Mamba2 layer.
+    xbc [batch, L, nheads*64 + 2*ngroups*d_state] bf16; conv_w [channels, 4] fp32; conv_b
+    [channels] fp32 or None; seq_idx [batch, L] int32 or None; conv_state_in [batch,
+    channels, 3] bf16 or None.  Returns (x [batch, L, nheads, 64], B, C [batch, L, ngroups,
+    d_state], conv_state_out [batch, channels, 3] or None), ready for mamba2_ssd_fwd."""
+    lib = _lib()
+    dev = xbc.device
+    Bt, L, Cc = xbc.shape
+    iot = xbc.dtype
+    H, G, N = int(nheads), int(ngroups), int(d_state)
+    x = torch.empty(Bt, L, H, 64, dtype=iot, device=dev)
+    B = torch.empty(Bt, L, G, N, dtype=iot, device=dev)
+    C = torch.empty(Bt, L, G, N, dtype=iot, device=dev)
+    cs_out = torch.empty(Bt, Cc, 3, dtype=iot, device=dev) if want_state else None
+    dims = make_dims(Bt, L, H, 64, N, G, _m._io_code(xbc))
+    if Cc != H * 64 + 2 * G * N:
+        raise ValueError(f"xbc has {Cc} channels, expected {H * 64 + 2 * G * N}")
+    p = _m._ptr
+    f32 = torch.float32
+    rc = lib.mamba2_conv_silu(
+        ctypes.byref(dims), p(xbc, "xbc", iot, dev), p(conv_w, "conv_w", f32, dev),
+        p(conv_b, "conv_b", f32, dev), p(seq_idx, "seq_idx", torch.int32, dev),
+        p(conv_state_in, "conv_state_in", iot, dev), p(x, "x", iot, dev), p(B, "B", iot, dev),
+        p(C, "C", iot, dev), p(cs_out, "conv_state_out", iot, dev), _m._stream_handle(stream, dev))
+    _m._check(rc)
+    return x, B, C, cs_out
+
+
+def mamba2_gated_rmsnorm(y, z, weight, eps: float = 1e-5, *, ngroups: int = 1, out=None,
+                         stream=None):
+    """out = y * SiLU(z) normalised to unit RMS over each of ngroups channel groups, times
+    weight.  y, z [batch, L, nheads, 64] (or [batch, L, nheads*64]) bf16; weight
+    [nheads*64] fp32."""
+    lib = _lib()
+    dev = y.device
+    Bt, L = y.shape[0], y.shape[1]
+    D = y.numel() // max(Bt * L, 1) if Bt * L else (y.shape[2] * (y.shape[3] if y.dim() == 4 else 1))
+    iot = y.dtype
+    if out is None:
+        out = torch.empty_like(y)
+    dims = make_dims(Bt, L, D // 64, 64, 64, ngroups, _m._io_code(y))
+    p = _m._ptr
+    rc = lib.mamba2_gated_rmsnorm(
+        ctypes.byref(dims), p(y, "y", iot, dev), p(z, "z", iot, dev),
+        p(weight, "weight", torch.float32, dev), ctypes.c_float(eps), p(out, "out", iot, dev),
+        _m._stream_handle(stream, dev))
+    _m._check(rc)
+    return out

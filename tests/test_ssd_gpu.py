@@ -198,3 +198,85 @@ def test_prefill_then_steps_equal_forward():
         ys.append(yt)
     assert_close_tc(np.concatenate(ys, axis=1), yo, "prefill + steps y")
     assert_close_tc(h, ho, "prefill + steps h")
+
+
+# ---------------------------------------------------------------- the layer around the scan
+from tests.tolerances import assert_close  # noqa: E402
+
+
+def draw_layer(Bt, L, H, N, G, seed, state=True):
+    r = np.random.default_rng(seed)
+    Cc = H * 64 + 2 * G * N
+    return dict(
+        xbc=I.f32_to_bf16_bits(r.standard_normal((Bt, L, Cc)).astype(np.float32)),
+        conv_w=r.uniform(-0.5, 0.5, size=(Cc, 4)).astype(np.float32),
+        conv_b=r.uniform(-0.5, 0.5, size=Cc).astype(np.float32),
+        cs_in=I.f32_to_bf16_bits(r.standard_normal((Bt, Cc, 3)).astype(np.float32)) if state else None,
+    )
+
+
+@pytest.mark.parametrize("case", [(2, 150, 4, 64, 1, None, True), (1, 2, 2, 128, 2, "length_one_docs", True),
+                                  (2, 200, 6, 128, 3, "many_short_docs", False),
+                                  (1, 130, 2, 64, 1, "boundary_on_edge", True), (2, 0, 2, 64, 1, None, True)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_conv_silu_matches_oracle(case):
+    Bt, L, H, N, G, name, state = case
+    inp = draw_layer(Bt, L, H, N, G, seed=3900 + L + H, state=state)
+    ids = None if name is None else I.seq_idx_case(name, Bt, L, edge=64, seed=5)
+    ref, cs_ref = so.conv_silu(inp["xbc"], inp["conv_w"], inp["conv_b"], seq_idx=ids,
+                               conv_state_in=inp["cs_in"])
+    d = {k: (None if v is None else dev_tensor(v)) for k, v in inp.items()}
+    tid = None if ids is None else torch.from_numpy(ids.astype(np.int32)).cuda()
+    x, B, C, cs = S.mamba2_conv_silu(d["xbc"], d["conv_w"], d["conv_b"], nheads=H, ngroups=G,
+                                     d_state=N, seq_idx=tid, conv_state_in=d["cs_in"])
+    torch.cuda.synchronize()
+    got = np.concatenate([host(x).reshape(Bt, L, H * 64), host(B).reshape(Bt, L, G * N),
+                          host(C).reshape(Bt, L, G * N)], axis=2)
+    assert_close(got, ref, "bf16", "conv + SiLU")
+    np.testing.assert_array_equal(host(cs), cs_ref)   # a copy of inputs (or zeros): bitwise
+
+
+@pytest.mark.parametrize("case", [(2, 50, 24, 1), (3, 17, 8, 2), (1, 5, 6, 3)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_gated_rmsnorm_matches_oracle(case):
+    Bt, L, H, G = case
+    r = np.random.default_rng(4000 + H)
+    y = I.f32_to_bf16_bits(r.standard_normal((Bt, L, H * 64)).astype(np.float32))
+    z = I.f32_to_bf16_bits(r.standard_normal((Bt, L, H * 64)).astype(np.float32))
+    w = r.standard_normal(H * 64).astype(np.float32)
+    ref = so.gated_rmsnorm(y, z, w, 1e-5, group_size=H * 64 // G)
+    out = S.mamba2_gated_rmsnorm(dev_tensor(y), dev_tensor(z), dev_tensor(w), 1e-5, ngroups=G)
+    torch.cuda.synchronize()
+    assert_close(host(out), ref, "bf16", "gated RMSNorm")
+
+
+def test_layer_conv_scan_norm_matches_oracle():
+    # everything between the projections: conv + SiLU over x|B|C, the scan with a gate-free
+    # output, then the gated RMSNorm (the rmsnorm=True layer of the weight contract)
+    Bt, L, H, N, G = 2, 300, 4, 128, 1
+    lay = draw_layer(Bt, L, H, N, G, seed=4100)
+    w = I.SsdWorkload("layer", Bt, L, H, 64, N, G, 4101, gate=True)
+    scan = I.make_ssd_inputs(w)
+    ids = I.packed_seq_idx(Bt, L, 80, 4102)
+    nw = np.random.default_rng(4103).standard_normal(H * 64).astype(np.float32)
+    # oracle chain (the oracle's conv output rounded to bf16, as the scan takes it)
+    conv_ref, _ = so.conv_silu(lay["xbc"], lay["conv_w"], lay["conv_b"], seq_idx=ids,
+                               conv_state_in=lay["cs_in"])
+    cb = I.f32_to_bf16_bits(conv_ref.astype(np.float32))
+    xr = cb[..., :H * 64].reshape(Bt, L, H, 64)
+    Br = np.ascontiguousarray(cb[..., H * 64:H * 64 + G * N]).reshape(Bt, L, G, N)
+    Cr = np.ascontiguousarray(cb[..., H * 64 + G * N:]).reshape(Bt, L, G, N)
+    yr, _ = so.ssd(xr, scan["dt_raw"], scan["A_log"], Br, Cr, scan["D"], scan["dt_bias"],
+                   seq_idx=ids)
+    yb = I.f32_to_bf16_bits(yr.astype(np.float32))
+    ref = so.gated_rmsnorm(yb.reshape(Bt, L, -1), scan["z"].reshape(Bt, L, -1), nw, 1e-5)
+    # the library
+    d = {k: (None if v is None else dev_tensor(v)) for k, v in lay.items()}
+    tid = torch.from_numpy(ids.astype(np.int32)).cuda()
+    x, B, C, _ = S.mamba2_conv_silu(d["xbc"], d["conv_w"], d["conv_b"], nheads=H, ngroups=G,
+                                    d_state=N, seq_idx=tid, conv_state_in=d["cs_in"])
+    sd = {k: (None if v is None else dev_tensor(v)) for k, v in scan.items()}
+    y, _ = S.mamba2_ssd_fwd(x, sd["dt_raw"], sd["A_log"], B, C, sd["D"], sd["dt_bias"], seq_idx=tid)
+    out = S.mamba2_gated_rmsnorm(y, sd["z"], dev_tensor(nw), 1e-5)
+    torch.cuda.synchronize()
+    assert_close_tc(host(out).reshape(Bt, L, H * 64), ref, "layer output")

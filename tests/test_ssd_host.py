@@ -155,3 +155,44 @@ def test_step_validation(lib):
     assert _step(lib, dims(seqlen=1), {"h_out": _fake(0x8010000100)}) == 1
     assert _step(lib, dims(seqlen=1), {"y": _fake(0x10000000)}) == 1      # y on x
     assert _step(lib, dims(seqlen=1, batch=0)) == 0
+
+
+CONV = ["xbc", "w", "bias", "seq", "cs_in", "x", "B", "C", "cs_out"]
+
+
+def _conv(lib, d, ptrs=None):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(CONV)}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba2_conv_silu(ctypes.byref(d), *[p[k] for k in CONV], None)
+
+
+def test_conv_validation(lib):
+    assert _conv(lib, dims(), {"xbc": None}) == 1
+    assert _conv(lib, dims(), {"x": None}) == 1
+    assert _conv(lib, dims(), {"w": _fake(0x1010000008)}) == 3          # conv_w needs 16 bytes
+    assert _conv(lib, dims(), {"B": _fake(0x6010000002)}) == 3
+    assert _conv(lib, dims(), {"x": _fake(0x10000000)}) == 1            # x on top of xbc
+    assert _conv(lib, dims(), {"C": _fake(0x6010000000)}) == 1          # C on top of B
+    assert _conv(lib, dims(headdim=32)) == 2
+    assert _conv(lib, dims(batch=0)) == 0
+
+
+def _norm(lib, d, eps=1e-5, ptrs=None):
+    base = 0x10000000
+    p = {k: _fake(base + i * (1 << 36)) for i, k in enumerate(["y", "z", "w", "out"])}
+    if ptrs:
+        p.update(ptrs)
+    return lib.mamba2_gated_rmsnorm(ctypes.byref(d), p["y"], p["z"], p["w"], ctypes.c_float(eps),
+                                    p["out"], None)
+
+
+def test_norm_validation(lib):
+    assert _norm(lib, dims(), eps=-1.0) == 1
+    assert _norm(lib, dims(), eps=float("nan")) == 1
+    assert _norm(lib, dims(), ptrs={"z": None}) == 1
+    assert _norm(lib, dims(), ptrs={"w": _fake(0x2010000004)}) == 3
+    assert _norm(lib, dims(), ptrs={"out": _fake(0x10000000)}) == 1    # out on top of y
+    assert _norm(lib, dims(ngroups=3)) == 1                             # 4 heads, 3 groups
+    assert _norm(lib, dims(seqlen=0)) == 0
