@@ -664,6 +664,76 @@ def run_ssd(args, w, local_rank: int):
     }
 
 
+def run_layer(args, w, local_rank: int):
+    """--pass layer: the Mamba2 layer's conv + SiLU over x|B|C and its gated RMSNorm, each
+    timed alone (device events, L2 flushed between calls) on workload w's shapes."""
+    import torch
+    from selective_state_space_silu_b200 import mixer as M
+    from selective_state_space_silu_b200 import ssd as S
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M.load_library()
+    Bt, L, H, N, G = w.batch, w.seqlen, w.nheads, w.d_state, w.ngroups
+    D, Cc = H * 64, H * 64 + 2 * G * N
+    r = np.random.default_rng(w.seed + 7)
+
+    def td(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    xbc = td(I.f32_to_bf16_bits(r.standard_normal((Bt, L, Cc), dtype=np.float32)))
+    cw = td(r.uniform(-0.5, 0.5, size=(Cc, 4)).astype(np.float32))
+    cb = td(r.uniform(-0.5, 0.5, size=Cc).astype(np.float32))
+    y = td(I.f32_to_bf16_bits(r.standard_normal((Bt, L, D), dtype=np.float32)))
+    z = td(I.f32_to_bf16_bits(r.standard_normal((Bt, L, D), dtype=np.float32)))
+    nw = td(r.standard_normal(D).astype(np.float32))
+    out = torch.empty_like(y)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    calls = {
+        "conv": (lambda: S.mamba2_conv_silu(xbc, cw, cb, nheads=H, ngroups=G, d_state=N,
+                                            want_state=False, stream=stream),
+                 2 * Bt * L * Cc * 2 + Cc * 20),
+        "norm": (lambda: S.mamba2_gated_rmsnorm(y, z, nw, 1e-5, out=out, stream=stream),
+                 3 * Bt * L * D * 2 + D * 4),
+    }
+    peaks = measured_peaks()
+    res = {}
+    with ClockSampler(local_rank) as clk:
+        for name, (fn, nbytes) in calls.items():
+            for _ in range(args.warmup):
+                flush.fill_(1.0); fn()
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for e0, e1 in evs:
+                flush.fill_(1.0)
+                e0.record(stream); fn(); e1.record(stream)
+            torch.cuda.synchronize()
+            ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            res[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 2),
+                         "frac": round(gbs / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes}
+    tot_b = sum(v[1] for v in calls.values())
+    tot_ms = sum(v["ms"] for v in res.values())
+    top = max(res, key=lambda k: res[k]["ms"])
+    return {
+        "metric": "Mamba2 layer conv + SiLU and gated RMSNorm: achieved algorithmic GB/s",
+        "pass": "layer", "value": round(tot_b / (tot_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(tot_ms, 5),
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": Bt, "seqlen": L, "nheads": H, "d_state": N,
+                   "ngroups": G, "channels_conv": Cc, "l2": "flushed between calls"},
+        "kernels": res,
+        "roofline": {"kernel": "conv_silu_kernel" if top == "conv" else "gated_rmsnorm_kernel",
+                     "bound": "hbm", "achieved": res[top]["GB/s"], "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": res[top]["frac"],
+                     "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)", "traffic": None},
+        "gpu_launches": 2 * args.steps, "clocks": clk.summary(),
+    }
+
+
 def oracle_sample_ssd(w, target_s: float):
     """The fp64 Mamba2 oracle on a bounded sample: whole sequences of some (row, head)
     pairs.  Returns (GB/s of the workload's bytes per (row, head), cores, description)."""
@@ -749,7 +819,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long", choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "ssd"], default="fwd",
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "ssd", "layer"], default="fwd",
                     help="bwd: time the backward (mamba_mixer_bwd) alone on the workload; "
                          "ssd: time the Mamba2 scan (mamba2_ssd_fwd) on --ssd-workload")
     ap.add_argument("--ssd-workload", default="ssd_v3", choices=sorted(I.SSD_WORKLOADS))
@@ -775,7 +845,10 @@ def main():
         return
 
     if args.pass_ != "fwd" and world > 1:
-        ap.error("--pass bwd and --pass ssd time one GPU: run them without torchrun")
+        ap.error("--pass bwd, ssd and layer time one GPU: run them without torchrun")
+    if args.pass_ == "layer":
+        print(json.dumps(run_layer(args, I.SSD_WORKLOADS[args.ssd_workload], local_rank)), flush=True)
+        return
     if args.pass_ == "ssd":
         sw = I.SSD_WORKLOADS[args.ssd_workload]
         if args.seqlen is not None:
