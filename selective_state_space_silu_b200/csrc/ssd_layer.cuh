@@ -28,7 +28,7 @@ struct ConvArgs {
 };
 
 constexpr int kConvThreads = 128;
-constexpr int kConvSteps = 64;  // time steps per thread
+constexpr int kConvSteps = 16;  // time steps per thread
 
 __device__ __forceinline__ void bf16x8_to_f32(uint4 v, float* o) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
