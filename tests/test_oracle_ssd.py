@@ -382,3 +382,24 @@ def test_gated_rmsnorm_groups_are_separate_norms():
     for gi in range(4):
         sl = slice(8 * gi, 8 * gi + 8)
         close(out[..., sl], so.gated_rmsnorm(y[..., sl], z[..., sl], w[sl]))
+
+
+# ---------------------------------------------------------------- regression fixture
+def test_oracle_matches_its_golden_fixture():
+    """tests/golden/ssd_tiny_oracle_samples.json (written by tests/golden/make_golden_ssd.py
+    from the oracle): a later change to the oracle's arithmetic shows up here (to 1e-12:
+    numpy's exp and log may differ in the last bit between machines)."""
+    import importlib.util
+    import json
+    import os
+    here = os.path.join(os.path.dirname(__file__), "golden")
+    spec = importlib.util.spec_from_file_location("make_golden_ssd", os.path.join(here, "make_golden_ssd.py"))
+    mk = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mk)
+    g = json.load(open(os.path.join(here, "ssd_tiny_oracle_samples.json")))
+    now = mk.compute()
+    for key in ("y", "h_out", "conv", "norm"):
+        for (ix, v), (ix2, v2) in zip(g[key], now[key]):
+            assert ix == ix2
+            assert abs(v - v2) <= 1e-12 * max(1.0, abs(v)), (key, ix, v, v2)
+    np.testing.assert_allclose(now["conv_state_out_b0_c7"], g["conv_state_out_b0_c7"], rtol=1e-12, atol=0)
