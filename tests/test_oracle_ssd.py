@@ -403,3 +403,69 @@ def test_oracle_matches_its_golden_fixture():
             assert ix == ix2
             assert abs(v - v2) <= 1e-12 * max(1.0, abs(v)), (key, ix, v, v2)
     np.testing.assert_allclose(now["conv_state_out_b0_c7"], g["conv_state_out_b0_c7"], rtol=1e-12, atol=0)
+
+
+# ---------------------------------------------------------------- random shapes
+def chunked_with_resets(c, Q, ids):
+    """The chunked form with documents: within a chunk the mask also needs s and t in one
+    document, the inter-chunk term of step t needs no reset in (chunk start, t], and the
+    state update takes the chunk's last document only (zero carried decay after a reset)."""
+    x, dtr, Bm, Cm = c["x"], c["dt_raw"], c["B"], c["C"]
+    Bt, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    y = np.zeros((Bt, L, H, P))
+    hT = np.zeros((Bt, H, P, N))
+    for b in range(Bt):
+        reset = np.zeros(L, dtype=bool)
+        reset[1:] = ids[b, 1:] != ids[b, :-1]
+        for h in range(H):
+            g = h // (H // G)
+            A = -np.exp(c["A_log"][h])
+            Hs = np.zeros((P, N)) if c.get("h_in") is None else c["h_in"][b, h].copy()
+            for c0 in range(0, L, Q):
+                idx = np.arange(c0, min(L, c0 + Q))
+                q = len(idx)
+                last_reset = np.full(q, -1)
+                lr = -1
+                for i, t in enumerate(idx):
+                    if reset[t]:
+                        lr = i
+                    last_reset[i] = lr
+                dl = softplus(dtr[b, idx, h] + c["dt_bias"][h])
+                cs = np.cumsum(dl * A)
+                Mm = np.zeros((q, q))
+                for i in range(q):
+                    for j in range(max(last_reset[i], 0), i + 1):
+                        Mm[i, j] = np.exp(cs[i] - cs[j]) * dl[j]
+                inter = np.where(last_reset < 0, np.exp(cs), 0.0)
+                Y = (Mm * (Cm[b, idx, g] @ Bm[b, idx, g].T)) @ x[b, idx, h] \
+                    + inter[:, None] * (Cm[b, idx, g] @ Hs.T) + c["D"][h] * x[b, idx, h]
+                if c.get("z") is not None:
+                    Y = Y * silu(c["z"][b, idx, h])
+                y[b, idx, h] = Y
+                lo = max(last_reset[-1], 0)
+                wl = np.where(np.arange(q) >= lo, np.exp(cs[-1] - cs) * dl, 0.0)
+                dec = np.exp(cs[-1]) if last_reset[-1] < 0 else 0.0
+                Hs = dec * Hs + (x[b, idx, h] * wl[:, None]).T @ Bm[b, idx, g]
+            hT[b, h] = Hs
+    return y, hT
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(seed=st.integers(0, 10 ** 6), L=st.integers(1, 19), Q=st.integers(1, 8),
+       G=st.sampled_from([1, 2]), hpg=st.integers(1, 2), P=st.integers(1, 3),
+       N=st.integers(1, 4), gate=st.booleans(), state=st.booleans(), docs=st.integers(0, 4))
+def test_random_shapes_chunked_and_unrolled(seed, L, Q, G, hpg, P, N, gate, state, docs):
+    c = case(seed, Bt=2, L=L, H=G * hpg, P=P, N=N, G=G, z=gate, h_in=state)
+    r = np.random.default_rng(seed + 1)
+    ids = np.cumsum(r.random((2, L)) < docs / 10.0, axis=1)         # random document starts
+    y, hT = run(c, seq_idx=ids)
+    yc, hc = chunked_with_resets(c, Q, ids)
+    close(y, yc, 1e-10)
+    close(hT, hc, 1e-10)
+    yu, hu = unrolled(c, seq_idx=ids)
+    close(y, yu, 1e-10)
+    close(hT, hu, 1e-10)
