@@ -17,8 +17,11 @@
 //
 // (the decay between two steps of a chunk is a difference of that cumulative sum, as the
 // pages describe for the reference kernels).  One CTA of 4 warps owns one (batch row,
-// head) and walks the chunks in order; the state H (headdim 64 x d_state) stays in the
-// fp32 accumulators of the state GEMM for the whole sequence -- it never goes to HBM.
+// head, time segment) and walks the segment's chunks in order; the state H (headdim 64 x
+// d_state) stays in the fp32 accumulators of the state GEMM for the whole segment -- it
+// never goes to HBM.  Sequences of few (row, head) pairs are cut into segments, each
+// started from the earlier ones' end states (see the kernel below); document resets
+// (seq_idx) mask the chunk's products.
 //
 // Work split per chunk (warp w):
 //   * M o C B^T: the 10 causal 16 x 16 blocks of the 64 x 64 matrix, 3/3/2/2 per warp,
