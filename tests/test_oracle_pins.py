@@ -16,7 +16,7 @@ import numpy as np
 import pytest
 from scipy.special import expit
 
-from tests.tolerances import assert_close, within
+from tests.tolerances import assert_close, same_nonfinite_pattern, within
 
 
 # ---------------------------------------------------------------- independent pieces
@@ -331,9 +331,16 @@ def test_nonfinite_inputs_propagate(oracle):
     assert np.all(np.isnan(h[0, 1]))
 
 
-def test_tolerance_rule_counts_nan_as_mismatch():
+def test_tolerance_rule_counts_nonfinite_as_mismatch():
     assert not within(np.array([np.nan]), np.array([1.0]), "f32")[0]
-    assert within(np.array([np.nan]), np.array([np.nan]), "f32")[0]
+    assert not within(np.array([np.nan]), np.array([np.nan]), "f32")[0]
+    assert not within(np.array([np.inf]), np.array([np.inf]), "f32")[0]
+    fin = same_nonfinite_pattern(np.array([np.nan, np.inf, 1.0]), np.array([np.nan, np.inf, 2.0]))
+    assert fin.tolist() == [False, False, True]
+    with pytest.raises(AssertionError):
+        same_nonfinite_pattern(np.array([np.nan, 1.0]), np.array([1.0, 1.0]))
+    with pytest.raises(AssertionError):
+        same_nonfinite_pattern(np.array([np.inf]), np.array([-np.inf]))
     assert within(np.array([1.0 + 9e-4]), np.array([1.0]), "f32")[0]
     assert not within(np.array([1.0 + 1.2e-3]), np.array([1.0]), "f32")[0]
 
