@@ -250,18 +250,30 @@ MAMBA_API int mamba_mixer_check(void* workspace, void* cuda_stream);
  * Limits and conventions:
  *   - dims whose mamba_mixer_fwd_workspace_bytes exceeds 2 MiB are rejected with
  *     MAMBA_ERR_WORKSPACE (message via mamba_last_error); use mamba_mixer_fwd for them;
- *   - the first call on each device looks up the array's device address with that device
- *     current (cudaGetSymbolAddress); make that first call before any stream capture;
- *   - all calls on a device share the one array and it keeps the last call's contents:
+ *   - the first call in each CUDA context looks up the array's device address in that
+ *     context (cudaGetSymbolAddress, which also makes the device's primary context current
+ *     on a thread that has none) and caches it under the context's unique id; a second
+ *     context on the same device, or one re-created after a reset, does its own lookup.
+ *     Make the first call in a context before any stream capture;
+ *   - all calls in a context share the one array and it keeps the last call's contents:
  *     calls that overlap on the GPU (e.g. on two streams at once) race; serialize them;
- *   - a bounded-wait timeout in this variant is recorded only in the array and is not
- *     reported (there is no workspace to pass to mamba_mixer_check).
+ *   - a bounded-wait timeout is recorded in the array's status word, like the workspace's
+ *     for mamba_mixer_fwd: mamba_mixer_noalloc_check reports and clears it.
  */
 MAMBA_API int mamba_mixer_fwd_noalloc(const mamba_dims* dims, const void* xp, const void* z,
                                       const void* dt_raw, const void* B, const void* C,
                                       const float* A_log, const float* D, const float* conv_w,
                                       const float* conv_b, const float* dt_bias, void* y,
                                       float* h_out, void* conv_state_out, void* cuda_stream);
+
+/*
+ * The status check of mamba_mixer_fwd_noalloc, which has no workspace to hand to
+ * mamba_mixer_check: waits for `cuda_stream`, then reads and clears the status word of the
+ * library's scratch array in the current context.  Returns MAMBA_ERR_TIMEOUT if a no-alloc
+ * forward since the last check gave up on a bounded wait (its outputs are then
+ * incomplete), MAMBA_OK otherwise.  Allocates nothing.  No counterpart on the pages.
+ */
+MAMBA_API int mamba_mixer_noalloc_check(void* cuda_stream);
 
 /* Message for the last non-OK return on this thread ("" if none). Never NULL. */
 MAMBA_API const char* mamba_last_error(void);

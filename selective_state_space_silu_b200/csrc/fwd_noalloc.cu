@@ -8,7 +8,9 @@
 // point takes the same inputs and outputs as mamba_mixer_fwd and uses instead a
 // library-owned scratch array of kNoAllocScratchBytes per device (held by every GPU that
 // loads the library, until the process exits).  It allocates nothing.
+// mamba_mixer_noalloc_check reads and clears that array's status word.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -23,35 +25,75 @@ void set_last_error(const char* msg);  // mamba_mixer.cu: the message mamba_last
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;  // 2 MiB per device
-constexpr int kMaxDevices = 64;
 
 // Scratch for the forward's workspace: a 256-byte header (status word) followed by the
 // carry aggregates of the time chunks.  Zero at module load; the forward writes every
 // aggregate before reading it, so nothing has to be cleared between calls.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on each device, looked up once per device with that
-// device current.  In host code the symbol itself is only a host-side stand-in.
-void* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
+// The array's device address belongs to a CUDA context, not to a device: a second context
+// on the same device (cuCtxCreate) or a context re-created after a reset has its own copy
+// of the module and so its own address.  The lookup is therefore cached per context, keyed
+// by the context's unique id (cuCtxGetId: unique for the life of the process, never reused).
+// In host code the symbol itself is only a host-side stand-in, never a device address.
+struct CtxEntry {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+constexpr int kCacheEntries = 64;
+CtxEntry g_cache[kCacheEntries] = {};
+int g_cache_next = 0;
+std::mutex g_cache_mu;
+
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+CtxGetIdFn ctx_get_id_fn() {
+  static CtxGetIdFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<CtxGetIdFn>(nullptr);
+    return reinterpret_cast<CtxGetIdFn>(p);
+  }();
+  return fn;
+}
 
 int noalloc_fail(int code, const char* msg) {
   mm_internal::set_last_error(msg);
   return code;
 }
 
-int scratch_for_current_device(void** out) {
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MAMBA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p) return MAMBA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+// Looks up (or finds cached) the scratch array's address in the current context.  The
+// lookup itself (cudaGetSymbolAddress) makes the device's primary context current when the
+// thread has none yet.  On failure writes the reason to `why`.
+int scratch_for_current_context(void** out, const char* who, char* why, size_t why_len) {
+  const CtxGetIdFn get_id = ctx_get_id_fn();
+  unsigned long long id = 0;
+  bool have_id = get_id && get_id(nullptr, &id) == CUDA_SUCCESS;
+  if (have_id) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    for (const CtxEntry& e : g_cache)
+      if (e.ptr && e.ctx_id == id) {
+        *out = e.ptr;
+        return MAMBA_OK;
+      }
   }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p) {
+    snprintf(why, why_len, "%s: cudaGetSymbolAddress of the scratch array failed: %s", who,
+             e != cudaSuccess ? cudaGetErrorString(e) : "null address");
+    return MAMBA_ERR_CUDA;
+  }
+  // the lookup may just have made a primary context current: take its id now
+  if (!have_id) have_id = get_id && get_id(nullptr, &id) == CUDA_SUCCESS;
+  if (have_id) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    g_cache[g_cache_next] = CtxEntry{id, p};
+    g_cache_next = (g_cache_next + 1) % kCacheEntries;
+  }
+  *out = p;
   return MAMBA_OK;
 }
 
@@ -74,9 +116,17 @@ extern "C" MAMBA_API int mamba_mixer_fwd_noalloc(
     return noalloc_fail(MAMBA_ERR_WORKSPACE, msg);
   }
   void* scratch = nullptr;
-  if (scratch_for_current_device(&scratch) != MAMBA_OK)
-    return noalloc_fail(MAMBA_ERR_CUDA,
-                        "mamba_mixer_fwd_noalloc: cudaGetSymbolAddress of the scratch failed");
+  char why[256];
+  if (scratch_for_current_context(&scratch, "mamba_mixer_fwd_noalloc", why, sizeof(why)) != MAMBA_OK)
+    return noalloc_fail(MAMBA_ERR_CUDA, why);
   return mamba_mixer_fwd(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, y, h_out,
                          conv_state_out, scratch, kNoAllocScratchBytes, cuda_stream);
+}
+
+extern "C" MAMBA_API int mamba_mixer_noalloc_check(void* cuda_stream) {
+  void* scratch = nullptr;
+  char why[256];
+  if (scratch_for_current_context(&scratch, "mamba_mixer_noalloc_check", why, sizeof(why)) != MAMBA_OK)
+    return noalloc_fail(MAMBA_ERR_CUDA, why);
+  return mamba_mixer_check(scratch, cuda_stream);
 }

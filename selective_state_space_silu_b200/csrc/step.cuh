@@ -14,9 +14,13 @@
 // (256 x 5120; 8 CTAs per SM spills and takes 48.7 us).  No barrier is needed: every
 // lane reads back only what it copied itself.
 //
-// In-place update (h_out == h_in, conv_state_out == conv_state_in) is safe: every
-// element is read and then written by the same lane, the write after the lane's
-// cp.async has completed.
+// In-place update (h_out == h_in, conv_state_out == conv_state_in) is safe.  The state:
+// every element is read and then written by the same lane, the write after the lane's
+// cp.async has completed.  The conv state: both lanes of a channel read cs_in but only
+// lane j == 0 writes cs_out; the ordering point is the __shfl_xor_sync of the readout,
+// whose operands depend on both lanes' cs_in loads, so neither lane passes it before its
+// loads have returned, and lane 0's stores come after it.  An edit that moves those stores
+// above the shuffle (or the shuffle above the loads' use) breaks in-place decode.
 #pragma once
 
 #include "device_math.cuh"
