@@ -372,6 +372,20 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
     step_total = bytes_["fwd"] + bytes_["step"]
     if rank != 0:
         return None
+    # outputs of one clean call (outside the timing) for the parity sample
+    if w.decode:
+        h.copy_(td(inp["h"]))
+        cs.copy_(td(inp["conv_state"]))
+        hs = torch.empty_like(h)
+        css = torch.empty_like(cs)
+        M.mamba_mixer_step(T["xp"], T["z"], T["dt_raw"], T["B"], T["C"], P["A_log"], P["D"],
+                           P["conv_w"], P["conv_b"], P["dt_bias"], h, cs, y=yt, h_out=hs,
+                           conv_state_out=css, stream=stream)
+        outs = (yt, hs, css)
+    else:
+        fwd()
+        outs = (y, h, cs)
+    torch.cuda.synchronize()
     peaks = measured_peaks()
     value = job_gbs(step_total, args.steps, world, total_ms)
     # dominant kernel: the forward call (the decode step when timing decode alone)
@@ -383,31 +397,9 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
         dom_ms = statistics.mean(fwd_ms)
         dom_bytes = bytes_["fwd"]
         dom = "mamba_mixer_fwd_packed" if w.packed_mean else "mamba_mixer_fwd"
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     clocks = clk.summary()
     sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
-    # the binding roofline of the dominant kernel: HBM bytes or ALU arithmetic
-    t_hbm = dom_bytes / (peaks["hbm_gbs"] * 1e9)
-    dom_elems = w.batch * (1 if w.decode else w.seqlen) * w.d_inner * w.d_state
-    t_alu = alu_floor_s(dom_elems, w.d_state, sm_hz)
-    if t_alu > t_hbm:
-        roof = {"kernel": dom, "bound": "alu", "achieved": round(achieved, 2),
-                "peak": round(dom_bytes / t_alu / 1e9, 2), "unit": "GB/s",
-                "frac": round(t_alu / (dom_ms * 1e-3), 4),
-                "peak_source": (f"arithmetic floor: {alu_elements_per_clk_sm(w.d_state):.2f} scan "
-                                f"elements/clk/SM (MUFU 16 + FMA 128 per clk per SM) x {SMS} SMs x "
-                                f"{sm_hz/1e6:.0f} MHz, as GB/s of the kernel's algorithmic bytes"),
-                "hbm_frac": round(achieved / peaks["hbm_gbs"], 4),
-                "hbm_peak": peaks["hbm_gbs"], "hbm_peak_source": peaks["source"]}
-    else:
-        roof = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 2),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
-                                else "fallback 6650 GB/s")}
-    roof["traffic"] = recorded_traffic("step" if w.decode else "fwd", w.name)
-    roof["algorithmic_bytes_per_launch"] = dom_bytes
-    roof["avg_launch_ms"] = round(dom_ms, 5)
+    roof = roofline_of("step" if w.decode else "fwd", w, dom_bytes, dom_ms, peaks, sm_hz, dom)
     e2e_val = job_gbs(step_total, 1, world, e2e["ms_per_step"])
     return {
         "metric": METRIC,
@@ -445,7 +437,145 @@ def run_ours(args, w: I.Workload, rank: int, world: int, local_rank: int):
                 "ms_per_step": round(e2e["ms_per_step"], 4)},
         "gpu_launches": launches_per_step * args.steps if not w.decode else args.steps,
         "clocks": clocks,
+        "_outs": (inp, outs),
     }
+
+
+# ----------------------------------------------------------------------------- parity
+def parity_report(got: np.ndarray, ref: np.ndarray, io: str, rounded_io: bool) -> dict:
+    """Agreement of device results with the fp64 oracle, in the openfluke stress test's
+    terms (section "What the results mean"): the share within the sealed tolerance class,
+    the share of exact bits, max abs / rel error; non-finite values count as errors.
+    ``rounded_io``: the device result is stored in the I/O type, so "exact" compares it with
+    the oracle value rounded to that type (round to nearest even, via fp32)."""
+    from tests.tolerances import report
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    r = report(got, ref, io)
+    if rounded_io and io == I.BF16:
+        rb = I.bf16_bits_to_f32(I.f32_to_bf16_bits(ref.astype(np.float32))).astype(np.float64)
+    else:
+        rb = ref.astype(np.float32).astype(np.float64)
+    exact = float((got == rb).mean()) * 100.0 if got.size else 100.0
+    return {"n": r["n"], "within_pct": round(r["within_pct"], 4), "exact_pct": round(exact, 3),
+            "max_abs": float(f"{r['max_abs']:.3e}"), "max_rel": float(f"{r['max_rel']:.3e}"),
+            "nonfinite": int((~np.isfinite(got)).sum())}
+
+
+def parity_of(w: I.Workload, inp: dict, y, h, cs, chans, oracle_out=None) -> dict:
+    """Compares the device outputs (torch tensors of the whole workload) on the sampled
+    channels (all batch rows) with the oracle run on those channels."""
+    from oracle import mixer_oracle as O
+    if oracle_out is None:
+        oracle_out = O.mixer_channels(inp, np.arange(w.batch), chans, widen=I.as_f64, nthreads=0)
+    yo, ho, cso = oracle_out
+    yg = y.float().cpu().numpy()[:, :, chans]
+    hg = h.cpu().numpy()[:, chans]
+    cg = cs.float().cpu().numpy()[:, chans]
+    return {"sample": f"all {w.batch} batch rows x {len(chans)} of {w.d_inner} channels x L={w.seqlen}",
+            "tolerance": w.io_dtype,
+            "y": parity_report(yg, yo, w.io_dtype, True),
+            "h": parity_report(hg, ho, w.io_dtype, False),
+            "conv_state_bitwise": bool(np.array_equal(cg, cso.astype(np.float32)))}
+
+
+def roofline_of(kind: str, w: I.Workload, dom_bytes: int, dom_ms: float, peaks: dict,
+                sm_hz: float, kernel: str) -> dict:
+    """The binding roofline of one entry point's call: HBM bytes or the ALU floor."""
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    t_hbm = dom_bytes / (peaks["hbm_gbs"] * 1e9)
+    elems = w.batch * (1 if w.decode else w.seqlen) * w.d_inner * w.d_state
+    t_alu = alu_floor_s(elems, w.d_state, sm_hz)
+    src = ("measured (MEASURED_PEAKS.json hbm_gbs)" if peaks["source"] == "measured"
+           else f"fallback {FALLBACK_HBM_GBS:.0f} GB/s")
+    if t_alu > t_hbm:
+        roof = {"kernel": kernel, "bound": "alu", "achieved": round(achieved, 2),
+                "peak": round(dom_bytes / t_alu / 1e9, 2), "unit": "GB/s",
+                "frac": round(t_alu / (dom_ms * 1e-3), 4),
+                "peak_source": (f"arithmetic floor: {alu_elements_per_clk_sm(w.d_state):.2f} scan "
+                                f"elements/clk/SM (MUFU 16 + FMA 128 per clk per SM) x {SMS} SMs x "
+                                f"{sm_hz/1e6:.0f} MHz, as GB/s of the kernel's algorithmic bytes"),
+                "hbm_frac": round(achieved / peaks["hbm_gbs"], 4),
+                "hbm_peak": peaks["hbm_gbs"], "hbm_peak_source": src}
+    else:
+        roof = {"kernel": kernel, "bound": "hbm", "achieved": round(achieved, 2),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "peak_source": src}
+    roof["traffic"] = recorded_traffic(kind, w.name)
+    roof["algorithmic_bytes_per_launch"] = dom_bytes
+    roof["avg_launch_ms"] = round(dom_ms, 5)
+    return roof
+
+
+def measure_extra(w: I.Workload, dev, calls: int, peaks: dict, n_chans: int) -> dict:
+    """One more configuration on this GPU, outside the headline step: ``calls`` forward
+    calls (or decode steps) timed one by one with CUDA events on the launching stream, L2
+    flushed before each; then one call's outputs against the oracle on sampled channels."""
+    import torch
+    from selective_state_space_silu_b200 import mixer as M
+
+    inp = I.make_inputs(w)
+
+    def td(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    d = {k: td(v) for k, v in inp.items()}
+    Bt, L, Di, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    stream = torch.cuda.current_stream(dev)
+    iot = d["xp"].dtype
+    y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
+    h = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+    cs = torch.empty((Bt, Di, 3), dtype=iot, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    if w.decode:
+        kernel = "mamba_mixer_step"
+        nbytes = step_bytes(w)
+
+        def call():
+            M.mamba_mixer_step(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                               d["conv_w"], d["conv_b"], d["dt_bias"], d["h"], d["conv_state"],
+                               y=y, h_out=h, conv_state_out=cs, stream=stream)
+    else:
+        kernel = "mamba_mixer_fwd"
+        nbytes = fwd_bytes(w)
+        ws = M.new_workspace(M.make_dims(Bt, L, Di, N, 4, M._io_code(d["xp"])), dev)
+
+        def call():
+            M.mamba_mixer_fwd(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
+                              d["conv_w"], d["conv_b"], d["dt_bias"], y=y, h_out=h,
+                              conv_state_out=cs, workspace=ws, stream=stream)
+    for _ in range(5):
+        flush.fill_(1.0)
+        call()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(calls)]
+    with ClockSampler(dev.index or 0) as clk:
+        for a, b in evs:
+            flush.fill_(1.0)
+            a.record(stream)
+            call()
+            b.record(stream)
+        torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    clocks = clk.summary()
+    sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
+    call()
+    torch.cuda.synchronize()
+    from tests.gpu_util import pick_channels
+    chans = pick_channels(Di, n_chans, w.seed)
+    return {"config": {"batch": Bt, "seqlen": L, "d_inner": Di, "d_state": N, "io": w.io_dtype,
+                       "entry_point": kernel},
+            "calls": calls, "ms": round(ms, 5), "gbs": round(nbytes / (ms * 1e-3) / 1e9, 2),
+            "hbm_frac": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "roofline": roofline_of("step" if w.decode else "fwd", w, nbytes, ms, peaks, sm_hz,
+                                    kernel),
+            "parity": parity_of(w, inp, y, h, cs, chans),
+            "clocks": clocks}
 
 
 # ----------------------------------------------------------------------------- backward
@@ -774,13 +904,13 @@ def oracle_sample(w: I.Workload, target_s: float):
     nch = int(min(Di, max(8, len(probe) * target_s / dt)))
     chans = np.linspace(0, Di - 1, nch).astype(np.int64)
     t0 = time.perf_counter()
-    O.mixer_channels(inp, np.arange(Bt), chans, widen=I.as_f64, nthreads=0)
+    out = O.mixer_channels(inp, np.arange(Bt), chans, widen=I.as_f64, nthreads=0)
     el = time.perf_counter() - t0
     tc = Bt * L * nch
     gbs = tc / el * bytes_per_tc / 1e9
     desc = (f"{w.name}: all {Bt} batch rows x {nch} of {Di} channels x L={L} "
             f"({tc} token-channels, fp64 oracle, {el:.2f} s)")
-    return gbs, cores, desc, el
+    return gbs, cores, desc, el, (chans, out)
 
 
 def run_reference(args, w: I.Workload, rank: int):
@@ -792,7 +922,7 @@ def run_reference(args, w: I.Workload, rank: int):
     for _ in range(max(1, args.warmup and 1)):
         oracle_sample(w, 1.0)
     for _ in range(args.steps):
-        gbs, cores, desc, _ = oracle_sample(w, max(2.0, 20.0 / max(args.steps, 1)))
+        gbs, cores, desc, _, _ = oracle_sample(w, max(2.0, 20.0 / max(args.steps, 1)))
         vals.append(gbs)
     v = statistics.mean(vals)
     return {
@@ -819,6 +949,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long", choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the m130 forward and decode step measured beside the default line")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "ssd", "layer"], default="fwd",
                     help="bwd: time the backward (mamba_mixer_bwd) alone on the workload; "
                          "ssd: time the Mamba2 scan (mamba2_ssd_fwd) on --ssd-workload")
@@ -883,10 +1015,25 @@ def main():
     try:
         res = run_ours(args, w, rank, world, local_rank)
         if res is not None:
+            inp, outs = res.pop("_outs")
             if not args.no_cpu_baseline:
-                gbs, cores, desc, _ = oracle_sample(w, 10.0)
+                gbs, cores, desc, _, (chans, oout) = oracle_sample(w, 10.0)
                 res["cpu_baseline"] = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores,
                                        "kind": "oracle", "sample": desc}
+                if not w.decode:
+                    res["parity"] = parity_of(w, inp, *outs, chans, oout)
+            if not w.decode and args.no_cpu_baseline:
+                from tests.gpu_util import pick_channels
+                res["parity"] = parity_of(w, inp, *outs, pick_channels(w.d_inner, 24, w.seed))
+            if w.decode:
+                from tests.gpu_util import pick_channels
+                res["parity"] = parity_of(w, inp, *outs, pick_channels(w.d_inner, 256, w.seed))
+            if world == 1 and args.workload == "long" and not args.no_extra:
+                import torch
+                dev = torch.device("cuda", local_rank)
+                peaks = measured_peaks()
+                res["m130"] = measure_extra(I.WORKLOADS["m130"], dev, 200, peaks, 96)
+                res["decode"] = measure_extra(I.WORKLOADS["decode"], dev, 500, peaks, 512)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

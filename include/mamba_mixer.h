@@ -232,6 +232,18 @@ MAMBA_API int mamba_mixer_step(const mamba_dims* dims, const void* xp, const voi
                      void* y, float* h_out, void* conv_state_out, void* cuda_stream);
 
 /*
+ * How mamba_mixer_fwd / mamba_mixer_fwd_packed split a forward with these dims (a query; it
+ * launches nothing).  nchunks: time chunks per row; chunk_len: steps per chunk (the last may
+ * be shorter); time_groups: time groups per CTA (1, or 4 for the two-level scan of rows with
+ * few channels); chained: 1 when each chunk starts from the end state its predecessor left in
+ * the workspace, 0 when chunks past the first are preceded by a chunk-state pass.  Any output
+ * pointer may be NULL.  Returns MAMBA_OK, or the dims' validation error.  The pages have no
+ * counterpart: it documents this library's schedule for tests and tuning.
+ */
+MAMBA_API int mamba_mixer_fwd_plan(const mamba_dims* dims, int* nchunks, int64_t* chunk_len,
+                                   int* time_groups, int* chained);
+
+/*
  * Waits for `cuda_stream`, then reads and clears the status word of `workspace`.
  * Returns MAMBA_ERR_TIMEOUT if a forward that used this workspace since the last check
  * gave up on a bounded wait (its outputs are then incomplete), MAMBA_OK otherwise.

@@ -16,6 +16,7 @@
 
 #include "mamba_mixer.h"
 #include "fwd_kernel.cuh"
+#include "fwd2_kernel.cuh"
 #include "step.cuh"
 #include "bwd_kernel.cuh"
 
@@ -36,6 +37,15 @@ int fail(int code, const char* fmt, ...) {
 int ok() {
   g_last_error.clear();
   return MAMBA_OK;
+}
+
+// Test-only failure injection for the bounded-wait path: MAMBA_MIXER_INJECT_SKIP_TILE=k makes
+// one CTA of the next forwards skip the copies of its tile k; unset (the default) injects
+// nothing.  Read at every call (a getenv is negligible next to a forward launch), so that a
+// test can set and clear it within one process.
+int inject_skip_tile() {
+  const char* inj = getenv("MAMBA_MIXER_INJECT_SKIP_TILE");
+  return inj ? atoi(inj) : -1;
 }
 
 struct Span {
@@ -142,12 +152,107 @@ Plan make_plan(const mamba_dims* d) {
   return p;
 }
 
+// ---- forward plan --------------------------------------------------------------------
+// Two 32-channel tiles per SM or more (the 130M-class layer: 384 tiles), and fp32 I/O: the
+// warp-specialised kernel of fwd_kernel.cuh, with the parallel chunks of make_plan when
+// there are few tiles.  bf16 I/O with fewer tiles (a long row over few channels: the long
+// workload has 160): the fwd2 kernel, with four time groups per CTA (the two-level scan)
+// for the parallelism one SM needs, and the sequence cut into chained chunks for the
+// balance between SMs.  The CTA of chunk c starts from the end state that the CTA of chunk
+// c-1 of the same tile left in the workspace, so nothing is recomputed; the units are
+// claimed in order, so a unit's predecessor is always running or done.  Measured on the
+// long workload (2 x 65536 x 2560): 3.45-3.48 ms with 8, 16 or 32 chunks per row, against
+// 3.65 ms for the parallel chunks with their chunk-state pass.
+#ifndef MM_FWD_G4_UNITS
+#define MM_FWD_G4_UNITS 16
+#endif
+constexpr int64_t kG4MinChunkLen = 1024;
+constexpr int64_t kG4MaxChunks = MM_FWD_G4_UNITS;
+constexpr size_t kUnitCounterOff = 64;                // in the header, after the status word
+
+struct FwdPlan {
+  Plan p;
+  bool chained;
+  bool v2;     // the fwd2 kernel
+  int G;       // its time groups
+};
+
+FwdPlan make_fwd_plan(const mamba_dims* d) {
+  FwdPlan f{make_plan(d), false, false, 1};
+  const int64_t tiles = d->batch * ((d->d_inner + mm::kCh - 1) / mm::kCh);
+  if (d->io_dtype != MAMBA_BF16 || tiles >= 2 * 148) return f;
+  const int64_t L = d->seqlen > 0 ? d->seqlen : 1;
+  f.v2 = true;
+  f.G = 4;
+  int64_t c = 1;
+  if (L >= 2 * kG4MinChunkLen) c = L / kG4MinChunkLen < kG4MaxChunks ? L / kG4MinChunkLen : kG4MaxChunks;
+  f.p.nchunks = 1;
+  f.p.chunk_len = L;
+  if (c > 1) {
+    int64_t len = (L + c - 1) / c;
+    len = (len + mm::kTileT - 1) / mm::kTileT * mm::kTileT;
+    f.p.nchunks = int((L + len - 1) / len);
+    f.p.chunk_len = len;
+  }
+  f.chained = f.p.nchunks > 1;
+  return f;
+}
+
+// Chained workspace: header (status word, unit counter), one flag per (tile, scan warp),
+// then each tile's carried state [kCh][N] fp32.
+struct ChainLayout {
+  size_t flags, carry, total;
+};
+ChainLayout chain_layout(const mamba_dims* d) {
+  const size_t tiles = size_t(d->batch) * size_t((d->d_inner + mm::kCh - 1) / mm::kCh);
+  ChainLayout l;
+  l.flags = kWsHeader;
+  l.carry = l.flags + (tiles * mm::kScanWarps * sizeof(int) + 255) / 256 * 256;
+  l.total = l.carry + tiles * size_t(mm::kCh) * size_t(d->d_state) * sizeof(float);
+  return l;
+}
+
 size_t workspace_bytes_for(const mamba_dims* d, const Plan& p) {
   size_t agg = 0;
   if (p.nchunks > 1)
     agg = size_t(2) * size_t(d->batch) * size_t(p.nchunks - 1) * size_t(d->d_inner) *
           size_t(d->d_state) * sizeof(float);
   return kWsHeader + agg;
+}
+
+size_t fwd_workspace_for(const mamba_dims* d, const FwdPlan& f) {
+  if (f.chained) return chain_layout(d).total;
+  if (f.v2) return kWsHeader;
+  return workspace_bytes_for(d, f.p);
+}
+
+struct FwdMaps {
+  CUtensorMap x, z, dt, B, C;
+};
+
+template <int N, bool kExt, int G, bool kChained>
+cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 grid,
+                               cudaStream_t st) {
+  using S = mm::f2::Smem<N, G>;
+  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained>;
+  static bool attr_set = false;   // the attribute is set once per instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::kDynamic);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, mm::f2::threads<G>(), S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, a);
+  return cudaGetLastError();
+}
+
+template <int N, bool kExt>
+cudaError_t launch_fwd2(const FwdMaps& m, const mm::f2::Params& a, const FwdPlan& f,
+                        cudaStream_t st) {
+  const unsigned gx = unsigned(a.ntd);
+  if (f.chained)
+    return launch_fwd2_kernel<N, kExt, 4, true>(m, a, dim3(gx * unsigned(a.batch) * unsigned(a.nchunks)), st);
+  return launch_fwd2_kernel<N, kExt, 4, false>(m, a, dim3(gx, unsigned(a.batch), 1), st);
 }
 
 // ---- TMA descriptors ---------------------------------------------------------------
@@ -185,9 +290,6 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t d0, uint64_t
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-struct FwdMaps {
-  CUtensorMap x, z, dt, B, C;
-};
 
 template <int N, typename IO, bool P, bool kPre, bool kExt>
 cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdArgs<kExt>& a, dim3 grid,
@@ -307,7 +409,7 @@ const char* mamba_version(void) { return "mamba_mixer 0.1.0 (abi 1, sm_100a)"; }
 size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims) {
   Sizes s;
   if (check_dims(dims, &s) != MAMBA_OK) return 0;
-  return workspace_bytes_for(dims, make_plan(dims));
+  return fwd_workspace_for(dims, make_fwd_plan(dims));
 }
 
 }  // extern "C"
@@ -353,8 +455,9 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   const Span outs[] = {{y, size_t(s.act) * s.esize, "y"},
                        {h_out, size_t(s.state) * 4, "h_out"},
                        {conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"}};
-  const Plan plan = make_plan(dims);
-  const size_t need = workspace_bytes_for(dims, plan);
+  const FwdPlan fplan = make_fwd_plan(dims);
+  const Plan& plan = fplan.p;
+  const size_t need = fwd_workspace_for(dims, fplan);
   const Span wsp{workspace, need, "workspace"};
   for (const Span& o : outs) {
     for (const Span& i : ins)
@@ -401,6 +504,43 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
       !make_map(&m.C, C, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE))
     return fail(MAMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
 
+  unsigned char* wsb = static_cast<unsigned char*>(workspace);
+  if (fplan.v2) {
+    mm::f2::Params a2{};
+    a2.A_log = A_log; a2.D = D; a2.conv_w = conv_w; a2.conv_b = conv_b; a2.dt_bias = dt_bias;
+    a2.y = static_cast<__nv_bfloat16*>(y);
+    a2.h_out = h_out;
+    a2.cs_out = static_cast<__nv_bfloat16*>(conv_state_out);
+    a2.status = static_cast<int*>(workspace);
+    a2.seq_idx = seq_idx;
+    a2.h_in = h_in;
+    a2.cs_in = static_cast<const __nv_bfloat16*>(conv_state_in);
+    a2.L = dims->seqlen; a2.Di = Di;
+    a2.chunk_len = plan.chunk_len; a2.nchunks = plan.nchunks;
+    a2.ntd = int((Di + mm::kCh - 1) / mm::kCh);
+    a2.batch = int(dims->batch);
+    a2.inject_skip_tile = inject_skip_tile();
+    cudaError_t e = cudaSuccess;
+    if (fplan.chained) {
+      const ChainLayout lay = chain_layout(dims);
+      a2.unit_counter = reinterpret_cast<int*>(wsb + kUnitCounterOff);
+      a2.carry_flag = reinterpret_cast<int*>(wsb + lay.flags);
+      a2.carry = reinterpret_cast<float*>(wsb + lay.carry);
+      // unit counter and carry flags start at zero (the status word at offset 0 is kept)
+      e = cudaMemsetAsync(wsb + kUnitCounterOff, 0, lay.carry - kUnitCounterOff, st);
+      if (e != cudaSuccess)
+        return fail(MAMBA_ERR_CUDA, "workspace reset failed: %s", cudaGetErrorString(e));
+    }
+    const bool ext = seq_idx || h_in || conv_state_in;
+    if (N == 16)
+      e = ext ? launch_fwd2<16, true>(m, a2, fplan, st) : launch_fwd2<16, false>(m, a2, fplan, st);
+    else
+      e = ext ? launch_fwd2<8, true>(m, a2, fplan, st) : launch_fwd2<8, false>(m, a2, fplan, st);
+    if (e != cudaSuccess)
+      return fail(MAMBA_ERR_CUDA, "forward launch failed: %s", cudaGetErrorString(e));
+    return ok();
+  }
+
   mm::FwdParams a{};
   a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
   a.y = y; a.h_out = h_out; a.cs_out = conv_state_out;
@@ -409,14 +549,13 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   a.nchunks = plan.nchunks; a.chunk_len = plan.chunk_len;
   // Test-only failure injection (bounded-wait path): MAMBA_MIXER_INJECT_SKIP_TILE=k makes one
   // CTA skip the copies of its tile k; unset (the default) injects nothing.
-  a.inject_skip_tile = -1;
-  if (const char* inj = getenv("MAMBA_MIXER_INJECT_SKIP_TILE")) a.inject_skip_tile = atoi(inj);
+  a.inject_skip_tile = inject_skip_tile();
+  cudaError_t e;
   if (plan.nchunks > 1) {
     const size_t agg = (need - kWsHeader) / sizeof(float) / 2;
-    a.ws_P = reinterpret_cast<float*>(static_cast<unsigned char*>(workspace) + kWsHeader);
+    a.ws_P = reinterpret_cast<float*>(wsb + kWsHeader);
     a.ws_H = a.ws_P + agg;
   }
-  cudaError_t e;
   if (seq_idx || h_in || conv_state_in) {
     mm::FwdArgs<true> ax;
     static_cast<mm::FwdParams&>(ax) = a;
@@ -462,7 +601,21 @@ int mamba_mixer_fwd_launches(const mamba_dims* dims) {
   Sizes s;
   if (check_dims(dims, &s) != MAMBA_OK) return -1;
   if (dims->batch == 0 || dims->d_inner == 0 || dims->seqlen == 0) return 0;
-  return make_plan(dims).nchunks > 1 ? 2 : 1;
+  const FwdPlan f = make_fwd_plan(dims);
+  return (f.p.nchunks > 1 && !f.chained) ? 2 : 1;
+}
+
+int mamba_mixer_fwd_plan(const mamba_dims* dims, int* nchunks, int64_t* chunk_len,
+                         int* time_groups, int* chained) {
+  Sizes s;
+  int rc = check_dims(dims, &s);
+  if (rc) return rc;
+  const FwdPlan f = make_fwd_plan(dims);
+  if (nchunks) *nchunks = f.p.nchunks;
+  if (chunk_len) *chunk_len = f.p.chunk_len;
+  if (time_groups) *time_groups = f.G;
+  if (chained) *chained = f.chained ? 1 : 0;
+  return ok();
 }
 
 int mamba_mixer_check(void* workspace, void* cuda_stream) {

@@ -61,6 +61,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   }
 }
 
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *flag >= value (a flag another CTA of the same grid sets with a release store).
+// Bounded like mbar_wait: after kWaitLimitNs records MAMBA_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool wait_flag_geq(const int* flag, int value, int* status) {
+  if (ld_acquire_gpu(flag) >= value) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) >= value) return true;
+    if (global_ns() - t0 > kWaitLimitNs) {
+      if (status) atomicExch(status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
 // 3-D tiled TMA load (no multicast): coordinates innermost first.  Self-checked: the
 // tensor map must be 64-byte aligned, the destination `dst_align`-byte aligned (1024 for
 // swizzled tiles, 128 otherwise) and the innermost coordinate times the element size a

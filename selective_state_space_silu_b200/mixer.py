@@ -26,7 +26,8 @@ STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPOR
 EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba_mixer_fwd",
            "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
            "mamba_mixer_bwd_packed",
-           "mamba_mixer_step", "mamba_mixer_check", "mamba_mixer_fwd_noalloc",
+           "mamba_mixer_step", "mamba_mixer_check", "mamba_mixer_fwd_plan",
+           "mamba_mixer_fwd_noalloc",
            "mamba_mixer_noalloc_check", "mamba_last_error", "mamba_version")
 
 
@@ -131,6 +132,10 @@ def _check(rc: int):
 
 def mamba_mixer_fwd_workspace_bytes(dims: mamba_dims) -> int:
     return int(load_library().mamba_mixer_fwd_workspace_bytes(ctypes.byref(dims)))
+
+
+def mamba_mixer_bwd_workspace_bytes(dims: mamba_dims) -> int:
+    return int(load_library().mamba_mixer_bwd_workspace_bytes(ctypes.byref(dims)))
 
 
 def new_workspace(dims: mamba_dims, device) -> torch.Tensor:
@@ -340,6 +345,21 @@ def mamba_mixer_step(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, h_i
         _ptr(conv_state_out, "conv_state_out", iot, dev), _stream_handle(stream, dev))
     _check(rc)
     return y, h_out, conv_state_out
+
+
+def mamba_mixer_fwd_plan(dims: mamba_dims) -> dict:
+    """How the forward splits ``dims``: nchunks, chunk_len, time_groups, chained."""
+    lib = load_library()
+    lib.mamba_mixer_fwd_plan.restype = ctypes.c_int
+    lib.mamba_mixer_fwd_plan.argtypes = [ctypes.POINTER(mamba_dims), ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_int)]
+    n, g, ch = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    ln = ctypes.c_int64()
+    _check(lib.mamba_mixer_fwd_plan(ctypes.byref(dims), ctypes.byref(n), ctypes.byref(ln),
+                                    ctypes.byref(g), ctypes.byref(ch)))
+    return {"nchunks": n.value, "chunk_len": ln.value, "time_groups": g.value,
+            "chained": bool(ch.value)}
 
 
 def mamba_mixer_fwd_launches(dims: mamba_dims) -> int:

@@ -142,7 +142,7 @@ def test_workspace_rules(lib):
     assert lib.mamba_mixer_fwd_launches(ctypes.byref(short)) == 1
     assert _fwd(lib, short) == 4                                          # workspace required
     long = M.make_dims(2, 65536, 2560, 16)
-    assert lib.mamba_mixer_fwd_launches(ctypes.byref(long)) == 2
+    assert M.mamba_mixer_fwd_plan(long)["nchunks"] > 1
     need = lib.mamba_mixer_fwd_workspace_bytes(ctypes.byref(long))
     assert need > 0 and need % 16 == 0
     assert _fwd(lib, long) == 4

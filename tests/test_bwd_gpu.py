@@ -79,7 +79,10 @@ def test_backward_with_time_chunks(oracle, Bt, L, Di, N, io):
     carried across chunk edges, and the input gradient of each chunk's last 3 steps takes
     the next chunk's part."""
     dims = M.make_dims(Bt, L, Di, N, 4, M.MAMBA_BF16 if io == I.BF16 else M.MAMBA_F32)
-    assert M.mamba_mixer_fwd_launches(dims) == 2      # the plan splits the sequence
+    # the backward's plan splits the sequence: its workspace holds per-chunk aggregates
+    # beyond the header and the per-tile start states
+    per = Bt * Di * N * 4
+    assert M.mamba_mixer_bwd_workspace_bytes(dims) > 256 + (L + 15) // 16 * per
     w, inp = _case(Bt, L, Di, N, io, 3200 + L)
     _compare(_run(inp), _oracle(oracle, inp), io, f"chunked {Bt}x{L}x{Di} N{N} {io}")
 
@@ -165,7 +168,8 @@ def test_packed_backward_matches_oracle(oracle, case, io, state):
 def test_packed_backward_with_time_chunks(oracle, case):
     """16 chunks of 256 steps with boundaries on the chunk edges (and everywhere)."""
     w, inp = _case_packed(2, 4096, 64, 16, I.BF16, 3500 + len(case), case, True, edge=256)
-    assert M.mamba_mixer_fwd_launches(M.make_dims(2, 4096, 64, 16, 4, M.MAMBA_BF16)) == 2
+    dims = M.make_dims(2, 4096, 64, 16, 4, M.MAMBA_BF16)    # the backward's plan chunks it
+    assert M.mamba_mixer_bwd_workspace_bytes(dims) > 256 + 4096 // 16 * 2 * 64 * 16 * 4
     _compare_packed(_run_packed(inp, True), _oracle_packed(oracle, inp, True), I.BF16,
                     f"packed chunked {case}")
 

@@ -65,8 +65,10 @@ def test_nine_cases_short_rows(oracle, case, io, N, state):
 def test_chunked_rows_at_8192(oracle, case, state):
     w, inp = _inputs(2, 8192, 64, 16, I.BF16, 2100 + len(case), state)
     dims = M.make_dims(2, 8192, 64, 16, 4, M.MAMBA_BF16)
-    assert M.mamba_mixer_fwd_launches(dims) == 2           # the chunk-state pass runs
-    seq = I.seq_idx_case(case, 2, 8192, edge=256, seed=11)  # 256 = this plan's chunk length
+    plan = M.mamba_mixer_fwd_plan(dims)
+    assert plan["nchunks"] > 1                              # the rows are cut into chunks
+    # documents placed against the plan's chunk edges
+    seq = I.seq_idx_case(case, 2, 8192, edge=plan["chunk_len"], seed=11)
     _compare(oracle, w, inp, seq, state, f"L8192 {case} state={state}")
 
 

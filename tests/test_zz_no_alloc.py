@@ -99,10 +99,13 @@ def test_noalloc_refuses_sizes_beyond_its_scratch():
     lib.mamba_mixer_fwd_noalloc.restype = ctypes.c_int
     lib.mamba_mixer_fwd_noalloc.argtypes = [ctypes.POINTER(M.mamba_dims)] + [ctypes.c_void_p] * 14
     dims = None
-    for Di in range(256, 65536, 256):
-        cand = M.make_dims(1, 1 << 20, Di, 16)
-        if M.mamba_mixer_fwd_workspace_bytes(cand) > (2 << 20):
-            dims = cand
+    for io in (M.MAMBA_BF16, M.MAMBA_F32):
+        for Di in range(256, 65536, 256):
+            cand = M.make_dims(1, 1 << 20, Di, 16, 4, io)
+            if M.mamba_mixer_fwd_workspace_bytes(cand) > (2 << 20):
+                dims = cand
+                break
+        if dims is not None:
             break
     assert dims is not None, "no size exceeds the scratch: the refusal path would be dead"
     fake = [ctypes.c_void_p(0x10000000 + i * (1 << 36)) for i in range(13)]
