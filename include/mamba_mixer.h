@@ -244,6 +244,14 @@ MAMBA_API int mamba_mixer_fwd_plan(const mamba_dims* dims, int* nchunks, int64_t
                                    int* time_groups, int* chained);
 
 /*
+ * The status check of mamba_mixer_step, which takes no workspace: waits for `cuda_stream`,
+ * then reads and clears the step's status word (library-owned, one per CUDA context).
+ * Returns MAMBA_ERR_TIMEOUT if a decode step since the last check gave up on a bounded wait
+ * (its outputs are then incomplete), MAMBA_OK otherwise.  Allocates nothing.
+ */
+MAMBA_API int mamba_mixer_step_check(void* cuda_stream);
+
+/*
  * Waits for `cuda_stream`, then reads and clears the status word of `workspace`.
  * Returns MAMBA_ERR_TIMEOUT if a forward that used this workspace since the last check
  * gave up on a bounded wait (its outputs are then incomplete), MAMBA_OK otherwise.

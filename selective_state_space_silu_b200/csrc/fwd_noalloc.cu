@@ -14,8 +14,8 @@
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
+#include "context_symbol.h"
 #include "mamba_mixer.h"
 
 namespace mm_internal {
@@ -26,75 +26,21 @@ namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;  // 2 MiB per device
 
-// Scratch for the forward's workspace: a 256-byte header (status word) followed by the
-// carry aggregates of the time chunks.  Zero at module load; the forward writes every
-// aggregate before reading it, so nothing has to be cleared between calls.
+// Scratch for the forward's workspace: a 256-byte header (status word, chunk-unit counter)
+// followed by the carried states of the time chunks and their flags.  The forward resets
+// the counter and flags itself (cudaMemsetAsync on the stream, no allocation) and writes
+// every carried state before reading it, so nothing else has to be cleared between calls.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
-
-// The array's device address belongs to a CUDA context, not to a device: a second context
-// on the same device (cuCtxCreate) or a context re-created after a reset has its own copy
-// of the module and so its own address.  The lookup is therefore cached per context, keyed
-// by the context's unique id (cuCtxGetId: unique for the life of the process, never reused).
-// In host code the symbol itself is only a host-side stand-in, never a device address.
-struct CtxEntry {
-  unsigned long long ctx_id;
-  void* ptr;
-};
-constexpr int kCacheEntries = 64;
-CtxEntry g_cache[kCacheEntries] = {};
-int g_cache_next = 0;
-std::mutex g_cache_mu;
-
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-
-CtxGetIdFn ctx_get_id_fn() {
-  static CtxGetIdFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<CtxGetIdFn>(nullptr);
-    return reinterpret_cast<CtxGetIdFn>(p);
-  }();
-  return fn;
-}
 
 int noalloc_fail(int code, const char* msg) {
   mm_internal::set_last_error(msg);
   return code;
 }
 
-// Looks up (or finds cached) the scratch array's address in the current context.  The
-// lookup itself (cudaGetSymbolAddress) makes the device's primary context current when the
-// thread has none yet.  On failure writes the reason to `why`.
+// The scratch array's device address in the current context (looked up once per context).
 int scratch_for_current_context(void** out, const char* who, char* why, size_t why_len) {
-  const CtxGetIdFn get_id = ctx_get_id_fn();
-  unsigned long long id = 0;
-  bool have_id = get_id && get_id(nullptr, &id) == CUDA_SUCCESS;
-  if (have_id) {
-    std::lock_guard<std::mutex> lock(g_cache_mu);
-    for (const CtxEntry& e : g_cache)
-      if (e.ptr && e.ctx_id == id) {
-        *out = e.ptr;
-        return MAMBA_OK;
-      }
-  }
-  void* p = nullptr;
-  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-  if (e != cudaSuccess || !p) {
-    snprintf(why, why_len, "%s: cudaGetSymbolAddress of the scratch array failed: %s", who,
-             e != cudaSuccess ? cudaGetErrorString(e) : "null address");
-    return MAMBA_ERR_CUDA;
-  }
-  // the lookup may just have made a primary context current: take its id now
-  if (!have_id) have_id = get_id && get_id(nullptr, &id) == CUDA_SUCCESS;
-  if (have_id) {
-    std::lock_guard<std::mutex> lock(g_cache_mu);
-    g_cache[g_cache_next] = CtxEntry{id, p};
-    g_cache_next = (g_cache_next + 1) % kCacheEntries;
-  }
-  *out = p;
-  return MAMBA_OK;
+  return mm_host::symbol_in_context(reinterpret_cast<const void*>(&g_noalloc_scratch), out, who,
+                                    why, why_len) == 0 ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
 }  // namespace

@@ -26,7 +26,8 @@ STATUS = {0: "MAMBA_OK", 1: "MAMBA_ERR_INVALID_ARGUMENT", 2: "MAMBA_ERR_UNSUPPOR
 EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba_mixer_fwd",
            "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
            "mamba_mixer_bwd_packed",
-           "mamba_mixer_step", "mamba_mixer_check", "mamba_mixer_fwd_plan",
+           "mamba_mixer_step", "mamba_mixer_step_check", "mamba_mixer_check",
+           "mamba_mixer_fwd_plan",
            "mamba_mixer_fwd_noalloc",
            "mamba_mixer_noalloc_check", "mamba_last_error", "mamba_version")
 
@@ -404,6 +405,16 @@ def mamba_mixer_fwd_noalloc(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bi
         _ptr(conv_state_out, "conv_state_out", iot, dev), _stream_handle(stream, dev))
     _check(rc)
     return y, h_out, conv_state_out
+
+
+def mamba_mixer_step_check(stream=None, device=None) -> None:
+    """Wait for the stream; raise MambaError(MAMBA_ERR_TIMEOUT) if a decode step in the
+    current context gave up on a bounded wait since the last check (clears the status)."""
+    lib = load_library()
+    lib.mamba_mixer_step_check.restype = ctypes.c_int
+    lib.mamba_mixer_step_check.argtypes = [ctypes.c_void_p]
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    _check(lib.mamba_mixer_step_check(_stream_handle(stream, dev)))
 
 
 def mamba_mixer_noalloc_check(stream=None, device=None) -> None:

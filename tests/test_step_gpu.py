@@ -7,6 +7,7 @@ import pytest
 import torch
 
 from selective_state_space_silu_b200 import inputs as I
+from selective_state_space_silu_b200 import mixer as M
 from tests.gpu_util import gpu_fwd, gpu_step, host, host_bits, oracle_full, to_device
 from tests.tolerances import assert_close
 
@@ -128,3 +129,14 @@ def test_decode_unaligned_conv_state(oracle):
     assert_close(host(y), yo, w.io_dtype, "unaligned y")
     assert_close(host(h), ho, w.io_dtype, "unaligned h_out")
     np.testing.assert_array_equal(host(cs), cso)
+
+
+def test_step_status_word_is_clear_after_clean_steps(oracle):
+    """The step reports bounded-wait timeouts through its own status word (it takes no
+    workspace); after ordinary steps mamba_mixer_step_check finds it clear."""
+    w = I.WORKLOADS["decode"].with_(batch=5, d_inner=200, seed=4242)
+    inp = I.make_inputs(w)
+    d = to_device(inp)
+    for _ in range(2):
+        gpu_step(d, d["h"], d["conv_state"])
+    M.mamba_mixer_step_check()
