@@ -578,6 +578,97 @@ def measure_extra(w: I.Workload, dev, calls: int, peaks: dict, n_chans: int) -> 
             "clocks": clocks}
 
 
+# ----------------------------------------------------------------------------- dt proj
+def dtproj_rank(w: I.Workload) -> int:
+    """dt_rank of the workload's model: ceil(d_model / 16) with d_model = d_inner / 2 (the
+    calm-mamba layer: expand 2, dt_rank 'auto'), rounded up to a multiple of 8."""
+    r = -(-(w.d_inner // 2) // 16)
+    return -(-r // 8) * 8
+
+
+def run_dtproj(args, w: I.Workload, local_rank: int):
+    """--pass dtproj: the forward with the dt projection fused (mamba_mixer_fwd_dtproj)
+    against the unfused pair (dt_proj as a cuBLAS bf16 GEMM through torch, then
+    mamba_mixer_fwd), both timed with CUDA events, L2 flushed before each call."""
+    import torch
+    from selective_state_space_silu_b200 import mixer as M
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    M.load_library()
+    R = dtproj_rank(w)
+    inp = I.make_dtproj_inputs(w, R)
+
+    def td(a):
+        if a is None:
+            return None
+        if a.dtype == np.uint16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    d = {k: td(v) for k, v in inp.items()}
+    Bt, L, Di, N = w.batch, w.seqlen, w.d_inner, w.d_state
+    stream = torch.cuda.current_stream(dev)
+    y = torch.empty((Bt, L, Di), dtype=torch.bfloat16, device=dev)
+    h = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+    cs = torch.empty((Bt, Di, 3), dtype=torch.bfloat16, device=dev)
+    dt_raw = torch.empty((Bt, L, Di), dtype=torch.bfloat16, device=dev)
+    ws = M.new_workspace(M.make_dims(Bt, L, Di, N, 4, M.MAMBA_BF16), dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def fused():
+        M.mamba_mixer_fwd_dtproj(d["xp"], d["z"], d["dt_low"], d["W_dt"], d["B"], d["C"],
+                                 d["A_log"], d["D"], d["conv_w"], d["conv_b"], d["dt_bias"],
+                                 y=y, h_out=h, conv_state_out=cs, workspace=ws, stream=stream)
+
+    def unfused():
+        torch.matmul(d["dt_low"], d["W_dt"].t(), out=dt_raw)
+        M.mamba_mixer_fwd(d["xp"], d["z"], dt_raw, d["B"], d["C"], d["A_log"], d["D"],
+                          d["conv_w"], d["conv_b"], d["dt_bias"], y=y, h_out=h,
+                          conv_state_out=cs, workspace=ws, stream=stream)
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            flush.fill_(1.0)
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
+        for a, b in evs:
+            flush.fill_(1.0)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    n = min(args.steps, 50 if w.seqlen > 8192 else 200)
+    with ClockSampler(local_rank) as clk:
+        ms_f = timed(fused, n)
+        ms_u = timed(unfused, n)
+    fused()
+    torch.cuda.synchronize()
+    from tests.gpu_util import pick_channels
+    from oracle import mixer_oracle as O
+    chans = pick_channels(Di, 24 if w.seqlen > 8192 else 64, w.seed)
+    oout = O.mixer_dtproj_channels(inp, np.arange(Bt), chans, nthreads=0, widen=I.as_f64)
+    par = parity_of(w, inp, y, h, cs, chans, oout)
+    fb = fwd_bytes(w) - 2 * Bt * L * Di + 2 * Bt * L * R + 2 * Di * R
+    peaks = measured_peaks()
+    clocks = clk.summary()
+    sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
+    roof = roofline_of("fwd", w, fb, ms_f, peaks, sm_hz, "mamba_mixer_fwd_dtproj")
+    roof["traffic"] = None
+    return {"metric": "fused conv+selective-scan+gate with dt_proj on the tensor cores: "
+                      "algorithmic HBM GB/s", "pass": "dtproj", "unit": "GB/s",
+            "value": round(fb / (ms_f * 1e-3) / 1e9, 2), "higher_is_better": True,
+            "config": {"workload": w.name, "batch": Bt, "seqlen": L, "d_inner": Di,
+                       "d_state": N, "dt_rank": R},
+            "fused_ms": round(ms_f, 5), "unfused_ms": round(ms_u, 5),
+            "unfused_is": "torch.matmul (cuBLAS bf16) for dt_raw, then mamba_mixer_fwd",
+            "algorithmic_bytes_fused": fb, "roofline": roof, "parity": par, "clocks": clocks,
+            "gpu_launches": n}
+
+
 # ----------------------------------------------------------------------------- backward
 def bwd_bytes(w: I.Workload) -> int:
     """Algorithmic bytes of one backward: the forward's inputs and dy read once, the fp32
@@ -951,7 +1042,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the m130 forward and decode step measured beside the default line")
-    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "ssd", "layer"], default="fwd",
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd", "ssd", "layer", "dtproj"], default="fwd",
                     help="bwd: time the backward (mamba_mixer_bwd) alone on the workload; "
                          "ssd: time the Mamba2 scan (mamba2_ssd_fwd) on --ssd-workload")
     ap.add_argument("--ssd-workload", default="ssd_v3", choices=sorted(I.SSD_WORKLOADS))
@@ -994,6 +1085,11 @@ def main():
         print(json.dumps(res), flush=True)
         return
 
+    if args.pass_ == "dtproj":
+        if w.decode or w.io_dtype != I.BF16:
+            ap.error("--pass dtproj needs a bf16 forward workload")
+        print(json.dumps(run_dtproj(args, w, local_rank)), flush=True)
+        return
     if args.pass_ == "bwd":
         if w.decode or w.packed_mean:
             ap.error("--pass bwd needs a plain forward workload")

@@ -232,6 +232,26 @@ MAMBA_API int mamba_mixer_step(const mamba_dims* dims, const void* xp, const voi
                      void* y, float* h_out, void* conv_state_out, void* cuda_stream);
 
 /*
+ * The fused forward with the dt projection folded in (calm-mamba 0.1.4, section "Mamba
+ * operator", step 4: dt = dt_proj(dt_low)): instead of dt_raw [batch, L, d_inner] it takes
+ * dt_low [batch, L, dt_rank] (the low-rank slice of x_proj's output) and W_dt [d_inner,
+ * dt_rank], both bf16 row-major and 16-byte aligned, and forms dt_raw = dt_low W_dt^T per
+ * 32-step tile on the tensor cores (tcgen05, fp32 accumulation in tensor memory), kept in
+ * fp32 (no bf16 rounding of dt_raw); dt_bias is added as in mamba_mixer_fwd.  Everything else
+ * -- arguments, layouts, outputs, workspace (mamba_mixer_fwd_workspace_bytes of the same
+ * dims), errors -- is mamba_mixer_fwd's.  bf16 I/O only (MAMBA_ERR_UNSUPPORTED otherwise);
+ * dt_rank a multiple of 8 from 8 to 128 (MAMBA_ERR_UNSUPPORTED otherwise).  HBM traffic per
+ * token and channel drops from 8 to 6 bytes (dt_raw is neither written by a GEMM nor read).
+ */
+MAMBA_API int mamba_mixer_fwd_dtproj(const mamba_dims* dims, int64_t dt_rank, const void* xp,
+                                     const void* z, const void* dt_low, const void* W_dt,
+                                     const void* B, const void* C, const float* A_log,
+                                     const float* D, const float* conv_w, const float* conv_b,
+                                     const float* dt_bias, void* y, float* h_out,
+                                     void* conv_state_out, void* workspace,
+                                     size_t workspace_bytes, void* cuda_stream);
+
+/*
  * How mamba_mixer_fwd / mamba_mixer_fwd_packed split a forward with these dims (a query; it
  * launches nothing).  nchunks: time chunks per row; chunk_len: steps per chunk (the last may
  * be shorter); time_groups: time groups per CTA (1, or 4 for the two-level scan of rows with

@@ -150,6 +150,27 @@ def mixer_channels(inp: dict, batch_idx, chan_idx, precision: str = "f64",
                  precision=precision, nthreads=nthreads, seq_idx=seq)
 
 
+def mixer_dtproj(xp, z, dt_low, W_dt, B, C, A_log, D, conv_w, conv_b, dt_bias, nthreads: int = 1):
+    """The forward with the dt projection fused (calm-mamba 0.1.4, "Mamba operator", step 4:
+    dt = dt_proj(dt_low)): dt_raw = dt_low W_dt^T, a library matmul in fp64 with no rounding
+    between the two steps, then the mixer oracle above.  dt_low [Bt, L, R], W_dt [Di, R]."""
+    dt_raw = np.matmul(np.asarray(dt_low, dtype=np.float64), np.asarray(W_dt, dtype=np.float64).T)
+    return mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, nthreads=nthreads)
+
+
+def mixer_dtproj_channels(inp: dict, batch_idx, chan_idx, nthreads: int = 1, widen=None):
+    """mixer_dtproj over a subset of channels (as mixer_channels): the projection is formed
+    for the selected batch rows and channels only, dt_raw[b, :, d] = dt_low[b] W_dt[d]^T."""
+    w = widen or (lambda a: np.asarray(a, dtype=np.float64))
+    bi = np.asarray(batch_idx)
+    di = np.asarray(chan_idx)
+    dt_raw = np.matmul(w(inp["dt_low"][bi]), w(inp["W_dt"][di]).T)
+    cb = inp.get("conv_b")
+    return mixer(w(inp["xp"][bi][:, :, di]), w(inp["z"][bi][:, :, di]), dt_raw, w(inp["B"][bi]),
+                 w(inp["C"][bi]), inp["A_log"][di], inp["D"][di], inp["conv_w"][di],
+                 None if cb is None else cb[di], inp["dt_bias"][di], nthreads=nthreads)
+
+
 BWD_NAMES = ("dxp", "dz", "ddt_raw", "dB", "dC", "dA_log", "dD", "dconv_w", "dconv_b", "ddt_bias")
 
 

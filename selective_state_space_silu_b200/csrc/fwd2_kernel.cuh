@@ -81,17 +81,25 @@ struct Params {
   int64_t chunk_len;        // multiple of kTileT
   int nchunks, ntd, batch;
   int inject_skip_tile;     // test hook: -1 = off
+  int dt_rank;              // kDtProj: columns of dt_low and W_dt (<= 64 * kDtBlocks)
 };
 
-template <int N, int G>
+constexpr int kDtBlocks = 2;  // kDtProj: dt_rank up to 128, in K blocks of 64
+
+template <int N, int G, bool kDtProj = false>
 struct Smem {
   static constexpr int kS = N / 4;
   static constexpr int kRow = kCh * 2;                         // 64-byte rows (bf16)
   static constexpr int align1k(int v) { return (v + 1023) / 1024 * 1024; }
   static constexpr int kXOff = 0;
   static constexpr int kZOff = align1k((kTileT + kHalo) * kRow);
+  // dt_raw tile (bf16, 64-byte swizzle) -- or, with the dt projection fused, the tile's
+  // dt_low rows (bf16, 128-byte swizzle, K blocks of 64) and the product in fp32 [t][33]
   static constexpr int kDtOff = kZOff + align1k(kTileT * kRow);
-  static constexpr int kBOff = kDtOff + align1k(kTileT * kRow);
+  static constexpr int kDtBytes = kDtProj ? kDtBlocks * kTileT * 128 : align1k(kTileT * kRow);
+  static constexpr int kDt32Off = kDtOff + kDtBytes;
+  static constexpr int kDt32Stride = 33;                       // floats per step row
+  static constexpr int kBOff = kDt32Off + (kDtProj ? align1k(kTileT * kDt32Stride * 4) : 0);
   static constexpr int kCOff = kBOff + align1k(kTileT * N * 2);
   static constexpr int kBCRec = 2 * kS * 4;                    // fp32 {B[kS], C[kS]}
   static constexpr int kBCfOff = kCOff + align1k(kTileT * N * 2);
@@ -101,9 +109,12 @@ struct Smem {
   static constexpr int kXchWarp = (kTileT / G / 4) * 8 * kXchRec;   // quads x channels
   static constexpr int kSlotOff = kXchOff + kGroupWarps * G * kXchWarp;
   static constexpr int kSlotBytes = G > 1 ? G * kGroupWarps * 32 * kS * 4 : 0;
-  static constexpr int kBarOff = kSlotOff + kSlotBytes;
-  static constexpr int kBars = 3 * kStages + G * kGroupWarps;
-  static constexpr int kTotal = kBarOff + 8 * kBars;
+  // kDtProj: W_dt of the CTA's channels as the M = 128 operand (rows 32..127 zero), per K block
+  static constexpr int kWOff = align1k(kSlotOff + kSlotBytes);
+  static constexpr int kWBytes = kDtProj ? kDtBlocks * 128 * 128 : 0;
+  static constexpr int kBarOff = kWOff + kWBytes;
+  static constexpr int kBars = 3 * kStages + G * kGroupWarps + 2;   // + W landed, MMA done
+  static constexpr int kTotal = kBarOff + 8 * kBars + 16;      // + the TMEM address
   static constexpr int kDynamic = kTotal + 1024;               // slack to align to 1 KiB
 };
 
@@ -147,12 +158,13 @@ __device__ __forceinline__ uint64_t tile_resets(const int32_t* seq, int64_t tt, 
          (uint64_t(__ballot_sync(0xffffffffu, r_hi)) << 32);
 }
 
-template <int N, bool kExt, int G, bool kChained>
-__global__ void __launch_bounds__(threads<G>(), G == 1 ? 3 : 1)
+template <int N, bool kExt, int G, bool kChained, bool kDtProj = false>
+__global__ void __launch_bounds__(threads<G>(), G == 1 ? (kDtProj ? 2 : 3) : 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
             const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_B,
-            const __grid_constant__ CUtensorMap tm_C, const Params p) {
-  using S = Smem<N, G>;
+            const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_w,
+            const Params p) {
+  using S = Smem<N, G, kDtProj>;
   constexpr int kS = N / 4;
   constexpr int kP = kS / 2;              // f32x2 pairs per lane
   constexpr int R = kTileT / G;           // steps per group per tile
@@ -170,6 +182,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
   uint64_t* bc_ready = full + kStages;                               // B/C widened
   uint64_t* empty = bc_ready + kStages;                              // all scan warps done
   uint64_t* end_ready = empty + kStages;                             // [G][kGroupWarps]
+  uint64_t* w_bar = end_ready + G * kGroupWarps;                     // kDtProj: W_dt landed
+  uint64_t* mma_bar = w_bar + 1;                                     // kDtProj: product done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_bar + 1);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int tile = 0, d0 = int(blockIdx.x) * kCh, b = int(blockIdx.y), c = int(blockIdx.z);
@@ -194,13 +209,41 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
       mbar_init(&empty[s], kScanWarps);
     }
     for (int i = 0; i < G * kGroupWarps; ++i) mbar_init(&end_ready[i], 1);
+    mbar_init(w_bar, 1);
+    mbar_init(mma_bar, 1);
   }
   __syncthreads();
 
   if (warp == kScanWarps) {
     // ================================================================ producer warp
-    constexpr uint32_t kTx = uint32_t((kTileT + kHalo) * S::kRow + 2 * kTileT * S::kRow +
-                                      2 * kTileT * N * 2);
+    const int kb_n = kDtProj ? (p.dt_rank + 63) / 64 : 0;   // K blocks of dt_low / W_dt
+    const uint32_t kTx = uint32_t((kTileT + kHalo) * S::kRow + kTileT * S::kRow +
+                                  (kDtProj ? kb_n * kTileT * 128 : kTileT * S::kRow) +
+                                  2 * kTileT * N * 2);
+    uint32_t tbase = 0;
+    if constexpr (kDtProj) {
+      // the product's accumulator: 32 TMEM columns (lanes = the CTA's 32 channels)
+      tmem_alloc(tmem_slot, 32);
+      tmem_relinquish();
+      // W_dt rows 32..127 of the M = 128 operand are zero (rows 0..31 come by TMA)
+      const uint32_t wb = sb + uint32_t(S::kWOff);
+      for (int kb = 0; kb < kb_n; ++kb)
+        for (int i = lane; i < 96 * 8; i += 32)
+          sts_v4(wb + uint32_t(kb * 16384 + 4096 + i * 16), 0.f, 0.f, 0.f, 0.f);
+      fence_async_shared();
+      __syncwarp();
+      tc_fence_before();
+      __syncwarp();
+      tc_fence_after();
+      tbase = *tmem_slot;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(w_bar, uint32_t(kb_n * 32 * 128));
+        for (int kb = 0; kb < kb_n; ++kb)
+          tma_load_2d(wb + uint32_t(kb * 16384), &tm_w, w_bar, kb * 64, d0, 1024, 2, p.status);
+      }
+      __syncwarp();
+    }
+    int mma_issued = 0, mma_waited = 0;
     int issued = 0;
     auto issue = [&](int k) {
       const int s = k % kStages;
@@ -212,7 +255,13 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
           const int tt = int(t_begin) + k * kTileT;
           tma_load_3d(st + S::kXOff, &tm_x, &full[s], d0, tt - kHalo, b, 1024, 2, p.status);
           tma_load_3d(st + S::kZOff, &tm_z, &full[s], d0, tt, b, 1024, 2, p.status);
-          tma_load_3d(st + S::kDtOff, &tm_dt, &full[s], d0, tt, b, 1024, 2, p.status);
+          if constexpr (kDtProj) {
+            for (int kb = 0; kb < kb_n; ++kb)
+              tma_load_3d(st + S::kDtOff + kb * kTileT * 128, &tm_dt, &full[s], kb * 64, tt, b,
+                          1024, 2, p.status);
+          } else {
+            tma_load_3d(st + S::kDtOff, &tm_dt, &full[s], d0, tt, b, 1024, 2, p.status);
+          }
           tma_load_3d(st + S::kBOff, &tm_B, &full[s], 0, tt, b, 128, 2, p.status);
           tma_load_3d(st + S::kCOff, &tm_C, &full[s], 0, tt, b, 128, 2, p.status);
         }
@@ -246,6 +295,37 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
           sts_v4(dst, bf(b0 & 0xffffu), bf(b0 >> 16), bf(c0 & 0xffffu), bf(c0 >> 16));
         }
       }
+      if constexpr (kDtProj) {
+        // dt_raw of the tile = W_dt (channels x rank) * dt_low (steps x rank)^T on the tensor
+        // cores: D[channel][step] in TMEM, read back by this warp (TMEM lanes 0..31 are the
+        // channels) into the fp32 tile [step][33] the prep reads
+        if (k == 0) good = __all_sync(0xffffffffu, mbar_wait(w_bar, 0, p.status));
+        if (!good) break;
+        if (lane == 0) {
+          tc_fence_after();
+          constexpr uint32_t idesc = umma_idesc_bf16_f32<128, kTileT>();
+          int n = 0;
+          for (int kb = 0; kb < kb_n; ++kb)
+            for (int kk = 0; kk < 4 && kb * 64 + kk * 16 < p.dt_rank; ++kk, ++n)
+              umma_bf16(tbase, umma_desc_sw128(sb + uint32_t(S::kWOff + kb * 16384 + kk * 32)),
+                        umma_desc_sw128(st + uint32_t(S::kDtOff + kb * kTileT * 128 + kk * 32)),
+                        idesc, n > 0 ? 1u : 0u);
+          umma_commit(mma_bar);
+        }
+        __syncwarp();
+        ++mma_issued;
+        good = __all_sync(0xffffffffu, mbar_wait(mma_bar, uint32_t(k) & 1u, p.status));
+        if (!good) break;
+        ++mma_waited;
+        tc_fence_after();
+        float v[kTileT];
+        tmem_ld32(tbase, v);
+        tmem_wait_ld();
+        const uint32_t dt32 = st + uint32_t(S::kDt32Off) + uint32_t(lane) * 4u;
+#pragma unroll
+        for (int t = 0; t < kTileT; ++t) sts_f32(dt32 + uint32_t(t * S::kDt32Stride * 4), v[t]);
+        tc_fence_before();
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bc_ready[s]);
       // refill the stage of the previous tile once every scan warp is done with it
@@ -262,6 +342,14 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
       // every copy this CTA started must land before it exits
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         mbar_wait(&full[k % kStages], uint32_t(k / kStages) & 1u, nullptr);
+      if (kDtProj && mma_issued == 0) mbar_wait(w_bar, 0, nullptr);
+    }
+    if constexpr (kDtProj) {
+      // no product may still be writing the accumulator when it is freed
+      if (mma_issued > mma_waited) mbar_wait(mma_bar, uint32_t(mma_issued - 1) & 1u, nullptr);
+      __syncwarp();
+      tc_fence_after();
+      tmem_dealloc(tbase, 32);
     }
     return;
   }
@@ -335,7 +423,8 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const int t = (g * QG + e) * 4 + j;
 #pragma unroll
     for (int m = 0; m < 4; ++m) xoff[e][m] = uint32_t(S::kXOff) + swz64(t + 1 + m, col);
-    dtoff[e] = uint32_t(S::kDtOff) + swz64(t, col);
+    dtoff[e] = kDtProj ? uint32_t(S::kDt32Off + (t * S::kDt32Stride + cl) * 4)
+                       : uint32_t(S::kDtOff) + swz64(t, col);
     zoff[e] = uint32_t(S::kZOff) + swz64(t, col);
   }
 
@@ -402,7 +491,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
       }
       const float pre = fmaf(cw.w, x0, fmaf(cw.z, x1, fmaf(cw.y, x2, fmaf(cw.x, x3, cb))));
       const float u = silu_tanh(pre);
-      const float dl = softplus_lg2(bf(lds_u16(rb + dtoff[e])) + dtb);
+      const float dtv = kDtProj ? lds_f32(st + dtoff[e] + uint32_t((qq >> 1) * 8 * S::kDt32Stride * 4))
+                                : bf(lds_u16(rb + dtoff[e]));
+      const float dl = softplus_lg2(dtv + dtb);
       const bool valid = t < valid_n;
       float dlt = valid ? dl : 0.0f;
       const float du = valid ? dl * u : 0.0f;

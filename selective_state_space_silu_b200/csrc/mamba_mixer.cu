@@ -178,11 +178,22 @@ struct FwdPlan {
   int G;       // its time groups
 };
 
-FwdPlan make_fwd_plan(const mamba_dims* d) {
+// dtproj: the forward with the dt projection fused (always the fwd2 kernel, one time group
+// when there are two tiles per SM or more); its chunking matches the plain forward's, so the
+// two take the same workspace.
+FwdPlan make_fwd_plan(const mamba_dims* d, bool dtproj = false) {
   FwdPlan f{make_plan(d), false, false, 1};
   const int64_t tiles = d->batch * ((d->d_inner + mm::kCh - 1) / mm::kCh);
-  if (d->io_dtype != MAMBA_BF16 || tiles >= 2 * 148) return f;
+  if (d->io_dtype != MAMBA_BF16) return f;
   const int64_t L = d->seqlen > 0 ? d->seqlen : 1;
+  if (tiles >= 2 * 148) {
+    if (dtproj) {
+      f.v2 = true;
+      f.p.nchunks = 1;
+      f.p.chunk_len = L;
+    }
+    return f;
+  }
   f.v2 = true;
   f.G = 4;
   int64_t c = 1;
@@ -227,35 +238,6 @@ size_t fwd_workspace_for(const mamba_dims* d, const FwdPlan& f) {
   return workspace_bytes_for(d, f.p);
 }
 
-struct FwdMaps {
-  CUtensorMap x, z, dt, B, C;
-};
-
-template <int N, bool kExt, int G, bool kChained>
-cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 grid,
-                               cudaStream_t st) {
-  using S = mm::f2::Smem<N, G>;
-  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained>;
-  static bool attr_set = false;   // the attribute is set once per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         S::kDynamic);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  kern<<<grid, mm::f2::threads<G>(), S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, a);
-  return cudaGetLastError();
-}
-
-template <int N, bool kExt>
-cudaError_t launch_fwd2(const FwdMaps& m, const mm::f2::Params& a, const FwdPlan& f,
-                        cudaStream_t st) {
-  const unsigned gx = unsigned(a.ntd);
-  if (f.chained)
-    return launch_fwd2_kernel<N, kExt, 4, true>(m, a, dim3(gx * unsigned(a.batch) * unsigned(a.nchunks)), st);
-  return launch_fwd2_kernel<N, kExt, 4, false>(m, a, dim3(gx, unsigned(a.batch), 1), st);
-}
-
 // ---- TMA descriptors ---------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -290,6 +272,73 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t d0, uint64_t
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+// 2-D map over a row-major [d1][d0] bf16 tensor, box (b0, b1), 128-byte swizzle.
+bool make_map2d_sw128(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t b0,
+                      uint32_t b1) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {d0, d1};
+  const cuuint64_t strides[1] = {d0 * 2};
+  const cuuint32_t box[2] = {b0, b1};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over a row-major [d2][d1][d0] bf16 tensor, box (b0, b1, 1), 128-byte swizzle.
+bool make_map3d_sw128(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint32_t b0, uint32_t b1) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+  const cuuint32_t box[3] = {b0, b1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct FwdMaps {
+  CUtensorMap x, z, dt, B, C;
+  CUtensorMap w;    // the fused dt projection's W_dt (unused otherwise)
+};
+
+template <int N, bool kExt, int G, bool kChained, bool kDtProj>
+cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 grid,
+                               cudaStream_t st) {
+  using S = mm::f2::Smem<N, G, kDtProj>;
+  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained, kDtProj>;
+  static bool attr_set = false;   // the attribute is set once per instantiation
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         S::kDynamic);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<grid, mm::f2::threads<G>(), S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, m.w, a);
+  return cudaGetLastError();
+}
+
+template <int N, bool kExt, bool kDtProj = false>
+cudaError_t launch_fwd2(const FwdMaps& m, const mm::f2::Params& a, const FwdPlan& f,
+                        cudaStream_t st) {
+  const unsigned gx = unsigned(a.ntd);
+  const dim3 units(gx * unsigned(a.batch) * unsigned(a.nchunks)), tiles(gx, unsigned(a.batch), 1);
+  if constexpr (kDtProj) {
+    if (f.G == 1)
+      return f.chained ? launch_fwd2_kernel<N, false, 1, true, true>(m, a, units, st)
+                       : launch_fwd2_kernel<N, false, 1, false, true>(m, a, tiles, st);
+    return f.chained ? launch_fwd2_kernel<N, false, 4, true, true>(m, a, units, st)
+                     : launch_fwd2_kernel<N, false, 4, false, true>(m, a, tiles, st);
+  } else {
+    return f.chained ? launch_fwd2_kernel<N, kExt, 4, true, false>(m, a, units, st)
+                     : launch_fwd2_kernel<N, kExt, 4, false, false>(m, a, tiles, st);
+  }
+}
+
 
 
 template <int N, typename IO, bool P, bool kPre, bool kExt>
@@ -431,18 +480,32 @@ namespace {
 
 // The forward behind mamba_mixer_fwd and mamba_mixer_fwd_packed: seq_idx, h_in and
 // conv_state_in are null for the former.
+// dt_rank > 0: the dt projection is fused (dt_raw is NULL; dt_low [batch, L, dt_rank] and
+// W_dt [d_inner, dt_rank], bf16, give dt_raw = dt_low W_dt^T inside the kernel).
 int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void* dt_raw,
                const void* B, const void* C, const float* A_log, const float* D,
                const float* conv_w, const float* conv_b, const float* dt_bias,
                const int32_t* seq_idx, const float* h_in, const void* conv_state_in, void* y,
                float* h_out, void* conv_state_out, void* workspace, size_t workspace_bytes,
-               void* cuda_stream) {
+               void* cuda_stream, const void* dt_low = nullptr, const void* W_dt = nullptr,
+               int64_t dt_rank = 0) {
   Sizes s;
   int rc = check_dims(dims, &s);
   if (rc) return rc;
   const bool act = s.act > 0, bc = s.bc > 0;
+  const bool dtproj = dt_rank > 0;
+  if (dtproj) {
+    if (dims->io_dtype != MAMBA_BF16)
+      return fail(MAMBA_ERR_UNSUPPORTED, "the fused dt projection takes bf16 I/O only");
+    if (dt_rank % 8 != 0 || dt_rank > 64 * mm::f2::kDtBlocks)
+      return fail(MAMBA_ERR_UNSUPPORTED, "dt_rank %lld unsupported (a multiple of 8 up to %d)",
+                  (long long)dt_rank, 64 * mm::f2::kDtBlocks);
+    if ((rc = check_ptr(dt_low, "dt_low", act, 16)) ||
+        (rc = check_ptr(W_dt, "W_dt", dims->d_inner > 0, 16)))
+      return rc;
+  }
   if ((rc = check_ptr(xp, "xp", act, 16)) || (rc = check_ptr(z, "z", act, 16)) ||
-      (rc = check_ptr(dt_raw, "dt_raw", act, 16)) || (rc = check_ptr(B, "B", bc, 16)) ||
+      (rc = check_ptr(dt_raw, "dt_raw", act && !dtproj, 16)) || (rc = check_ptr(B, "B", bc, 16)) ||
       (rc = check_ptr(C, "C", bc, 16)) || (rc = check_ptr(y, "y", act, 16)) ||
       (rc = check_ptr(A_log, "A_log", dims->d_inner > 0, 16)) ||
       (rc = check_ptr(D, "D", dims->d_inner > 0, 4)) ||
@@ -464,11 +527,13 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
                       {dt_bias, size_t(Di) * 4, "dt_bias"},
                       {seq_idx, size_t(dims->batch) * size_t(dims->seqlen) * 4, "seq_idx"},
                       {h_in, size_t(s.state) * 4, "h_in"},
-                      {conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"}};
+                      {conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"},
+                      {dt_low, dtproj ? size_t(dims->batch) * size_t(dims->seqlen) * size_t(dt_rank) * 2 : 0, "dt_low"},
+                      {W_dt, dtproj ? size_t(Di) * size_t(dt_rank) * 2 : 0, "W_dt"}};
   const Span outs[] = {{y, size_t(s.act) * s.esize, "y"},
                        {h_out, size_t(s.state) * 4, "h_out"},
                        {conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"}};
-  const FwdPlan fplan = make_fwd_plan(dims);
+  const FwdPlan fplan = make_fwd_plan(dims, dtproj);
   const Plan& plan = fplan.p;
   const size_t need = fwd_workspace_for(dims, fplan);
   const Span wsp{workspace, need, "workspace"};
@@ -510,9 +575,13 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   const uint64_t Bt = uint64_t(dims->batch), L = uint64_t(dims->seqlen);
   const CUtensorMapSwizzle swz = f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const uint32_t nrow = uint32_t(mm::kTileT);
+  const bool dt_ok = dtproj
+      ? make_map3d_sw128(&m.dt, dt_low, uint64_t(dt_rank), L, Bt, 64, nrow) &&
+        make_map2d_sw128(&m.w, W_dt, uint64_t(dt_rank), uint64_t(Di), 64, mm::kCh)
+      : make_map(&m.dt, dt_raw, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz);
+  if (!dtproj) m.w = m.dt;   // not read
   if (!make_map(&m.x, xp, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow + mm::kHalo, swz) ||
-      !make_map(&m.z, z, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) ||
-      !make_map(&m.dt, dt_raw, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) ||
+      !make_map(&m.z, z, !f32, uint64_t(Di), L, Bt, mm::kCh, nrow, swz) || !dt_ok ||
       !make_map(&m.B, B, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE) ||
       !make_map(&m.C, C, !f32, uint64_t(N), L, Bt, uint32_t(N), nrow, CU_TENSOR_MAP_SWIZZLE_NONE))
     return fail(MAMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
@@ -533,6 +602,7 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
     a2.ntd = int((Di + mm::kCh - 1) / mm::kCh);
     a2.batch = int(dims->batch);
     a2.inject_skip_tile = inject_skip_tile();
+    a2.dt_rank = int(dt_rank);
     cudaError_t e = cudaSuccess;
     if (fplan.chained) {
       const ChainLayout lay = chain_layout(dims);
@@ -545,7 +615,10 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
         return fail(MAMBA_ERR_CUDA, "workspace reset failed: %s", cudaGetErrorString(e));
     }
     const bool ext = seq_idx || h_in || conv_state_in;
-    if (N == 16)
+    if (dtproj)
+      e = N == 16 ? launch_fwd2<16, false, true>(m, a2, fplan, st)
+                  : launch_fwd2<8, false, true>(m, a2, fplan, st);
+    else if (N == 16)
       e = ext ? launch_fwd2<16, true>(m, a2, fplan, st) : launch_fwd2<16, false>(m, a2, fplan, st);
     else
       e = ext ? launch_fwd2<8, true>(m, a2, fplan, st) : launch_fwd2<8, false>(m, a2, fplan, st);
@@ -608,6 +681,18 @@ int mamba_mixer_fwd_packed(const mamba_dims* dims, const void* xp, const void* z
   return fwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, seq_idx, h_in,
                     conv_state_in, y, h_out, conv_state_out, workspace, workspace_bytes,
                     cuda_stream);
+}
+
+int mamba_mixer_fwd_dtproj(const mamba_dims* dims, int64_t dt_rank, const void* xp,
+                           const void* z, const void* dt_low, const void* W_dt, const void* B,
+                           const void* C, const float* A_log, const float* D,
+                           const float* conv_w, const float* conv_b, const float* dt_bias,
+                           void* y, float* h_out, void* conv_state_out, void* workspace,
+                           size_t workspace_bytes, void* cuda_stream) {
+  if (dt_rank <= 0) return fail(MAMBA_ERR_INVALID_ARGUMENT, "dt_rank must be positive");
+  return fwd_common(dims, xp, z, nullptr, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
+                    nullptr, nullptr, y, h_out, conv_state_out, workspace, workspace_bytes,
+                    cuda_stream, dt_low, W_dt, dt_rank);
 }
 
 int mamba_mixer_fwd_launches(const mamba_dims* dims) {

@@ -148,6 +148,101 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
   return d;
 }
 
+// ---- 5th-generation tensor cores (tcgen05) and tensor memory ----------------------------
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte-swizzle layout that a
+// TMA copy with CU_TENSOR_MAP_SWIZZLE_128B writes: rows of 128 bytes (64 bf16 of K), 8-row
+// atoms of 1024 bytes (the atom must start 1024-byte aligned), the 16-byte chunk index XORed
+// with the row index within the atom.  Fields: start address >> 4 (bits 0-13), leading byte
+// offset >> 4 (16-29; unused for swizzled K-major, set to 1), stride byte offset >> 4 (32-45:
+// 1024 bytes between 8-row atoms), version 1 (46-47), layout 2 = 128-byte swizzle (61-63).
+// The K = 16 slice kk of a row starts 32*kk bytes further on.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(1) << 16) | (uint64_t(1024 >> 4) << 32) |
+         (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A and B, fp32 D, both K-major:
+// D format (bits 4-5) = 1 (f32), A format (7-9) = 1 (bf16), B format (10-12) = 1 (bf16),
+// A and B major (15, 16) = 0 (K), N >> 3 (17-22), M >> 4 (24-28).
+template <int M, int N>
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32() {
+  static_assert(M == 64 || M == 128, "M = 64 or 128 (cta_group::1)");
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N a multiple of 16 up to 256");
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread; accumulate = 0 overwrites D.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// The mbarrier receives one arrival when every tcgen05.mma this thread issued has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_addr(bar)) : "memory");
+}
+// Tensor-memory allocation: warp-wide; the column base is written to *dst_smem.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_addr(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// 32 consecutive 32-bit columns of this thread's TMEM lane (the warp's 32-lane quarter):
+// thread i of the warp gets lane (32*(warp%4) + i), columns col..col+31 of taddr.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void fence_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// 2-D tiled TMA load (no multicast); same self-checks as tma_load_3d.
+__device__ __forceinline__ bool tma_load_2d(uint32_t sdst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, uint32_t dst_align, int elem_bytes,
+                                            int* status) {
+  const uint64_t gmap = reinterpret_cast<uint64_t>(map);
+  if ((sdst & (dst_align - 1)) != 0 || (gmap & 63u) != 0 || ((c0 * elem_bytes) & 15) != 0) {
+    atomicExch(status, kStatusBadCopy);
+    return false;
+  }
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      ::"r"(sdst), "l"(gmap), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
+      : "memory");
+  return true;
+}
+
 // Named barrier that tolerates divergent arrival (non-.aligned form).
 __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

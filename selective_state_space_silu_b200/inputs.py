@@ -147,6 +147,19 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> Dict[str, np.ndarray
     return out
 
 
+def make_dtproj_inputs(w: Workload, dt_rank: int, seed: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Inputs of the forward with the dt projection fused: those of ``make_inputs`` (same
+    seed, same draws) plus dt_low [batch, L, dt_rank] ~ N(0, 1) and W_dt [d_inner, dt_rank]
+    ~ N(0, 0.5^2 / dt_rank), so that dt_low W_dt^T has the N(0, 0.5^2) spread of dt_raw;
+    both rounded to bf16 (bit patterns, uint16).  dt_raw is dropped."""
+    out = make_inputs(w, seed)
+    out.pop("dt_raw")
+    rng = np.random.Generator(np.random.PCG64((w.seed if seed is None else seed) + 7777))
+    out["dt_low"] = f32_to_bf16_bits(_normal(rng, (w.batch, w.seqlen, dt_rank)))
+    out["W_dt"] = f32_to_bf16_bits(_normal(rng, (w.d_inner, dt_rank), std=0.5 / np.sqrt(dt_rank)))
+    return out
+
+
 def random_params(w: Workload, seed: int) -> Dict[str, np.ndarray]:
     """Random A_log and D (instead of the structured ln(1..N) and 1) for extra cases."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -27,7 +27,7 @@ EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba
            "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
            "mamba_mixer_bwd_packed",
            "mamba_mixer_step", "mamba_mixer_step_check", "mamba_mixer_check",
-           "mamba_mixer_fwd_plan",
+           "mamba_mixer_fwd_plan", "mamba_mixer_fwd_dtproj",
            "mamba_mixer_fwd_noalloc",
            "mamba_mixer_noalloc_check", "mamba_last_error", "mamba_version")
 
@@ -344,6 +344,49 @@ def mamba_mixer_step(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, h_i
         _ptr(h_in, "h_in", f32, dev), _ptr(conv_state_in, "conv_state_in", iot, dev),
         _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
         _ptr(conv_state_out, "conv_state_out", iot, dev), _stream_handle(stream, dev))
+    _check(rc)
+    return y, h_out, conv_state_out
+
+
+def mamba_mixer_fwd_dtproj(xp, z, dt_low, W_dt, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
+                           y=None, h_out=None, conv_state_out=None, workspace=None,
+                           stream=None, want_states: bool = True):
+    """The fused forward with the dt projection folded in: dt_raw = dt_low W_dt^T is formed
+    per tile on the tensor cores.  dt_low [batch, L, dt_rank] and W_dt [d_inner, dt_rank] are
+    bf16; every other argument and the results are those of ``mamba_mixer_fwd`` (bf16 I/O)."""
+    lib = load_library()
+    lib.mamba_mixer_fwd_dtproj.restype = ctypes.c_int
+    lib.mamba_mixer_fwd_dtproj.argtypes = ([ctypes.POINTER(mamba_dims), ctypes.c_int64] +
+                                           [ctypes.c_void_p] * 15 + [ctypes.c_size_t, ctypes.c_void_p])
+    dev = xp.device
+    io = _io_code(xp)
+    iot = xp.dtype
+    Bt, L, Di = xp.shape
+    N = A_log.shape[1]
+    K = conv_w.shape[1]
+    R = dt_low.shape[2]
+    if tuple(W_dt.shape) != (Di, R) or tuple(dt_low.shape[:2]) != (Bt, L):
+        raise MambaError(1, "dt_low must be [batch, L, dt_rank] and W_dt [d_inner, dt_rank]")
+    dims = make_dims(Bt, L, Di, N, K, io)
+    if y is None:
+        y = torch.empty((Bt, L, Di), dtype=iot, device=dev)
+    if want_states and h_out is None:
+        h_out = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
+    if want_states and conv_state_out is None:
+        conv_state_out = torch.empty((Bt, Di, K - 1), dtype=iot, device=dev)
+    if workspace is None:
+        workspace = new_workspace(dims, dev)
+    f32 = torch.float32
+    rc = lib.mamba_mixer_fwd_dtproj(
+        ctypes.byref(dims), R, _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+        _ptr(dt_low, "dt_low", torch.bfloat16, dev), _ptr(W_dt, "W_dt", torch.bfloat16, dev),
+        _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
+        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
+        _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
+        _ptr(conv_state_out, "conv_state_out", iot, dev),
+        workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+        _stream_handle(stream, dev))
     _check(rc)
     return y, h_out, conv_state_out
 
