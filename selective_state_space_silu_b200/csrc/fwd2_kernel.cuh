@@ -55,11 +55,18 @@ namespace f2 {
 constexpr int kCh = 32;        // channels per CTA
 constexpr int kTileT = 32;     // steps per tile
 constexpr int kHalo = 4;       // x' rows before each tile (3 needed)
-constexpr int kStages = 4;     // TMA ring depth
+constexpr int kMaxDtBlocks = 2;  // fused dt projection: dt_rank up to 128, K blocks of 64
+
+// TMA ring depth: 3 for one time group with the dt projection fused (its operands would
+// otherwise keep three CTAs from sharing an SM), else 4
+__host__ __device__ constexpr int ring_depth(int G, int KB) { return KB > 0 && G == 1 ? 3 : 4; }
 constexpr int kGroupWarps = 4; // scan warps per time group (8 channels x 4 lanes each)
 
-template <int G>
-__host__ __device__ constexpr int threads() { return 32 * (kGroupWarps * G + 1); }
+// scan warps, the producer warp, and (the dt projection fused with G > 1) the product warp
+template <int G, int KB = 0>
+__host__ __device__ constexpr int threads() {
+  return 32 * (kGroupWarps * G + 1 + (KB > 0 && G > 1 ? 1 : 0));
+}
 
 struct Params {
   const float* A_log;
@@ -81,37 +88,39 @@ struct Params {
   int64_t chunk_len;        // multiple of kTileT
   int nchunks, ntd, batch;
   int inject_skip_tile;     // test hook: -1 = off
-  int dt_rank;              // kDtProj: columns of dt_low and W_dt (<= 64 * kDtBlocks)
+  int dt_rank;              // KB > 0: columns of dt_low and W_dt (<= 64 * KB)
 };
 
-constexpr int kDtBlocks = 2;  // kDtProj: dt_rank up to 128, in K blocks of 64
-
-template <int N, int G, bool kDtProj = false>
+// KB = K blocks of the fused dt projection (0: dt_raw is an input)
+template <int N, int G, int KB = 0>
 struct Smem {
+  static constexpr bool kDtProj = KB > 0;
+  static constexpr int kStages = ring_depth(G, KB);
   static constexpr int kS = N / 4;
   static constexpr int kRow = kCh * 2;                         // 64-byte rows (bf16)
   static constexpr int align1k(int v) { return (v + 1023) / 1024 * 1024; }
   static constexpr int kXOff = 0;
   static constexpr int kZOff = align1k((kTileT + kHalo) * kRow);
   // dt_raw tile (bf16, 64-byte swizzle) -- or, with the dt projection fused, the tile's
-  // dt_low rows (bf16, 128-byte swizzle, K blocks of 64) and the product in fp32 [t][33]
+  // dt_low rows (bf16, 128-byte swizzle, K blocks of 64), which the product in fp32 then
+  // overwrites once the tensor cores have read them: [t][32], channel c of step t at word
+  // t*32 + (c ^ 8*(t & 3)), so that both the producer's row writes and the scan lanes'
+  // reads (steps 4q..4q+3 x 8 channels) hit 32 distinct banks
   static constexpr int kDtOff = kZOff + align1k(kTileT * kRow);
-  static constexpr int kDtBytes = kDtProj ? kDtBlocks * kTileT * 128 : align1k(kTileT * kRow);
-  static constexpr int kDt32Off = kDtOff + kDtBytes;
-  static constexpr int kDt32Stride = 33;                       // floats per step row
-  static constexpr int kBOff = kDt32Off + (kDtProj ? align1k(kTileT * kDt32Stride * 4) : 0);
+  static constexpr int kDtBytes = kDtProj ? KB * kTileT * 128 : align1k(kTileT * kRow);
+  static constexpr int kBOff = kDtOff + kDtBytes;
   static constexpr int kCOff = kBOff + align1k(kTileT * N * 2);
   static constexpr int kBCRec = 2 * kS * 4;                    // fp32 {B[kS], C[kS]}
   static constexpr int kBCfOff = kCOff + align1k(kTileT * N * 2);
   static constexpr int kStage = kBCfOff + align1k(kTileT * 4 * kBCRec);
   static constexpr int kXchOff = kStages * kStage;             // Delta / Delta*u swap
   static constexpr int kXchRec = 48;                           // {Delta[4]}, {Delta*u[4]}, pad
-  static constexpr int kXchWarp = (kTileT / G / 4) * 8 * kXchRec;   // quads x channels
+  static constexpr int kXchWarp = 2 * 8 * kXchRec;             // quad parity x channels
   static constexpr int kSlotOff = kXchOff + kGroupWarps * G * kXchWarp;
   static constexpr int kSlotBytes = G > 1 ? G * kGroupWarps * 32 * kS * 4 : 0;
-  // kDtProj: W_dt of the CTA's channels as the M = 128 operand (rows 32..127 zero), per K block
+  // KB > 0: W_dt of the CTA's channels as the M = 128 operand (rows 32..127 zero), per K block
   static constexpr int kWOff = align1k(kSlotOff + kSlotBytes);
-  static constexpr int kWBytes = kDtProj ? kDtBlocks * 128 * 128 : 0;
+  static constexpr int kWBytes = KB * 128 * 128;
   static constexpr int kBarOff = kWOff + kWBytes;
   static constexpr int kBars = 3 * kStages + G * kGroupWarps + 2;   // + W landed, MMA done
   static constexpr int kTotal = kBarOff + 8 * kBars + 16;      // + the TMEM address
@@ -158,19 +167,28 @@ __device__ __forceinline__ uint64_t tile_resets(const int32_t* seq, int64_t tt, 
          (uint64_t(__ballot_sync(0xffffffffu, r_hi)) << 32);
 }
 
-template <int N, bool kExt, int G, bool kChained, bool kDtProj = false>
-__global__ void __launch_bounds__(threads<G>(), G == 1 ? (kDtProj ? 2 : 3) : 1)
+template <int N, bool kExt, int G, bool kChained, int KB = 0>
+__global__ void __launch_bounds__(threads<G, KB>(), G == 1 ? 3 : 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
             const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_B,
             const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_w,
             const Params p) {
-  using S = Smem<N, G, kDtProj>;
+  using S = Smem<N, G, KB>;
+  constexpr bool kDtProj = KB > 0;
+  constexpr int kStages = S::kStages;
   constexpr int kS = N / 4;
   constexpr int kP = kS / 2;              // f32x2 pairs per lane
   constexpr int R = kTileT / G;           // steps per group per tile
   constexpr int QG = R / 4;               // quads per group per tile
   constexpr int kScanWarps = kGroupWarps * G;
-  constexpr int kThreads = threads<G>();
+  constexpr int kThreads = threads<G, KB>();
+  // the products run on a warp of their own beside many scan warps (whose tiles come fast),
+  // else on the producer warp
+  constexpr bool kMmaWarp = kDtProj && G > 1;
+  constexpr bool kProdMma = kDtProj && !kMmaWarp;
+  constexpr int kDLane = kMmaWarp ? 32 : 0;
+  static_assert(!kMmaWarp || (kGroupWarps * G + 1) % 4 == 1, "product warp reads TMEM lanes 32..63");
+  static_assert(!kProdMma || (kGroupWarps * G) % 4 == 0, "producer reads TMEM lanes 0..31");
   static_assert(G == 1 || G == 2 || G == 4, "1, 2 or 4 time groups");
   static_assert(N == 8 || N == 16, "d_state 8 or 16");
 
@@ -205,7 +223,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&bc_ready[s], 1);
+      mbar_init(&bc_ready[s], kMmaWarp ? 2 : 1);   // B/C widened (and the product read back)
       mbar_init(&empty[s], kScanWarps);
     }
     for (int i = 0; i < G * kGroupWarps; ++i) mbar_init(&end_ready[i], 1);
@@ -214,36 +232,108 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
   }
   __syncthreads();
 
+  // ---- the fused dt projection (KB > 0): dt_raw of tile k = W_dt (channels x rank) *
+  // dt_low (steps x rank)^T on the tensor cores, D[channel][step] in 32 TMEM columns of lanes
+  // kDLane..kDLane+31 (the lanes the issuing warp may read: warp index mod 4 = kDLane / 32).
+  // The product is read back over the tile's consumed dt_low rows in the swizzled fp32 layout
+  // the prep reads, and the next tile's product is issued right after, so that it runs while
+  // the warp waits for the next tile.
+  [[maybe_unused]] uint32_t tbase = 0;
+  [[maybe_unused]] int mma_issued = 0, mma_waited = 0;
+  [[maybe_unused]] auto dt_setup = [&]() {
+    tmem_alloc(tmem_slot, 32);
+    tmem_relinquish();
+    // the M = 128 operand: W_dt's 32 rows at kDLane by TMA, the other 96 rows zero
+    const uint32_t wb = sb + uint32_t(S::kWOff);
+    for (int kb = 0; kb < KB; ++kb)
+      for (int i = lane; i < 96 * 8; i += 32) {
+        const int chunk = i < kDLane * 8 ? i : i + 32 * 8;   // 16-byte chunks, 8 per row
+        sts_v4(wb + uint32_t(kb * 16384 + chunk * 16), 0.f, 0.f, 0.f, 0.f);
+      }
+    fence_async_shared();
+    __syncwarp();
+    tc_fence_before();
+    __syncwarp();
+    tc_fence_after();
+    tbase = *tmem_slot;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(w_bar, uint32_t(KB * 32 * 128));
+      for (int kb = 0; kb < KB; ++kb)
+        tma_load_2d(wb + uint32_t(kb * 16384 + kDLane * 128), &tm_w, w_bar, kb * 64, d0, 1024, 2,
+                    p.status);
+    }
+    __syncwarp();
+  };
+  [[maybe_unused]] auto dt_issue = [&](int k) -> bool {
+    const int s = k % kStages;
+    if (!__all_sync(0xffffffffu, mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status)))
+      return false;
+    if (k == 0 && !__all_sync(0xffffffffu, mbar_wait(w_bar, 0, p.status))) return false;
+    if (lane == 0) {
+      tc_fence_after();
+      const uint32_t st = sb + uint32_t(s * S::kStage);
+      constexpr uint32_t idesc = umma_idesc_bf16_f32<128, kTileT>();
+      int n = 0;
+      for (int kb = 0; kb < KB; ++kb)
+        for (int kk = 0; kk < 4 && kb * 64 + kk * 16 < p.dt_rank; ++kk, ++n)
+          umma_bf16(tbase, umma_desc_sw128(sb + uint32_t(S::kWOff + kb * 16384 + kk * 32)),
+                    umma_desc_sw128(st + uint32_t(S::kDtOff + kb * kTileT * 128 + kk * 32)), idesc,
+                    n > 0 ? 1u : 0u);
+      umma_commit(mma_bar);
+    }
+    __syncwarp();
+    ++mma_issued;
+    return true;
+  };
+  [[maybe_unused]] auto dt_readback = [&](int k) -> bool {
+    if (!__all_sync(0xffffffffu, mbar_wait(mma_bar, uint32_t(k) & 1u, p.status))) return false;
+    ++mma_waited;
+    tc_fence_after();
+    float v[kTileT];
+    tmem_ld32(tbase + (uint32_t(kDLane) << 16), v);
+    tmem_wait_ld();
+    const uint32_t dt32 = sb + uint32_t((k % kStages) * S::kStage + S::kDtOff);
+#pragma unroll
+    for (int t = 0; t < kTileT; ++t)
+      sts_f32(dt32 + uint32_t((t * 32 + (lane ^ ((t & 3) << 3))) * 4), v[t]);
+    // these generic writes precede the refill's TMA writes to the same bytes
+    fence_async_shared();
+    tc_fence_before();
+    __syncwarp();
+    return true;
+  };
+  [[maybe_unused]] auto dt_teardown = [&]() {
+    // W_dt's copy must have landed and no product may still be writing the accumulator
+    if (mma_issued == 0) mbar_wait(w_bar, 0, nullptr);
+    if (mma_issued > mma_waited) mbar_wait(mma_bar, uint32_t(mma_issued - 1) & 1u, nullptr);
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tbase, 32);
+  };
+
+  if constexpr (kMmaWarp) {
+    if (warp == kScanWarps + 1) {
+      // ============================================================== product warp
+      dt_setup();
+      bool good = dt_issue(0);
+      for (int k = 0; good && k < ntiles; ++k) {
+        good = dt_readback(k);
+        if (!good) break;
+        if (lane == 0) mbar_arrive(&bc_ready[k % kStages]);
+        if (k + 1 < ntiles) good = dt_issue(k + 1);
+      }
+      named_bar_sync(0, kThreads);
+      dt_teardown();
+      return;
+    }
+  }
+
   if (warp == kScanWarps) {
     // ================================================================ producer warp
-    const int kb_n = kDtProj ? (p.dt_rank + 63) / 64 : 0;   // K blocks of dt_low / W_dt
     const uint32_t kTx = uint32_t((kTileT + kHalo) * S::kRow + kTileT * S::kRow +
-                                  (kDtProj ? kb_n * kTileT * 128 : kTileT * S::kRow) +
+                                  (kDtProj ? KB * kTileT * 128 : kTileT * S::kRow) +
                                   2 * kTileT * N * 2);
-    uint32_t tbase = 0;
-    if constexpr (kDtProj) {
-      // the product's accumulator: 32 TMEM columns (lanes = the CTA's 32 channels)
-      tmem_alloc(tmem_slot, 32);
-      tmem_relinquish();
-      // W_dt rows 32..127 of the M = 128 operand are zero (rows 0..31 come by TMA)
-      const uint32_t wb = sb + uint32_t(S::kWOff);
-      for (int kb = 0; kb < kb_n; ++kb)
-        for (int i = lane; i < 96 * 8; i += 32)
-          sts_v4(wb + uint32_t(kb * 16384 + 4096 + i * 16), 0.f, 0.f, 0.f, 0.f);
-      fence_async_shared();
-      __syncwarp();
-      tc_fence_before();
-      __syncwarp();
-      tc_fence_after();
-      tbase = *tmem_slot;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(w_bar, uint32_t(kb_n * 32 * 128));
-        for (int kb = 0; kb < kb_n; ++kb)
-          tma_load_2d(wb + uint32_t(kb * 16384), &tm_w, w_bar, kb * 64, d0, 1024, 2, p.status);
-      }
-      __syncwarp();
-    }
-    int mma_issued = 0, mma_waited = 0;
+    if constexpr (kProdMma) dt_setup();
     int issued = 0;
     auto issue = [&](int k) {
       const int s = k % kStages;
@@ -256,7 +346,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
           tma_load_3d(st + S::kXOff, &tm_x, &full[s], d0, tt - kHalo, b, 1024, 2, p.status);
           tma_load_3d(st + S::kZOff, &tm_z, &full[s], d0, tt, b, 1024, 2, p.status);
           if constexpr (kDtProj) {
-            for (int kb = 0; kb < kb_n; ++kb)
+            for (int kb = 0; kb < KB; ++kb)
               tma_load_3d(st + S::kDtOff + kb * kTileT * 128, &tm_dt, &full[s], kb * 64, tt, b,
                           1024, 2, p.status);
           } else {
@@ -271,7 +361,8 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     };
     for (int k = 0; k < ntiles && k < kStages; ++k) issue(k);
     bool good = true;
-    for (int k = 0; k < ntiles; ++k) {
+    if constexpr (kProdMma) good = dt_issue(0);
+    for (int k = 0; good && k < ntiles; ++k) {
       const int s = k % kStages;
       good = __all_sync(0xffffffffu, mbar_wait(&full[s], uint32_t(k / kStages) & 1u, p.status));
       if (!good) break;
@@ -295,39 +386,18 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
           sts_v4(dst, bf(b0 & 0xffffu), bf(b0 >> 16), bf(c0 & 0xffffu), bf(c0 >> 16));
         }
       }
-      if constexpr (kDtProj) {
-        // dt_raw of the tile = W_dt (channels x rank) * dt_low (steps x rank)^T on the tensor
-        // cores: D[channel][step] in TMEM, read back by this warp (TMEM lanes 0..31 are the
-        // channels) into the fp32 tile [step][33] the prep reads
-        if (k == 0) good = __all_sync(0xffffffffu, mbar_wait(w_bar, 0, p.status));
+      if constexpr (kProdMma) {
+        good = dt_readback(k);
         if (!good) break;
-        if (lane == 0) {
-          tc_fence_after();
-          constexpr uint32_t idesc = umma_idesc_bf16_f32<128, kTileT>();
-          int n = 0;
-          for (int kb = 0; kb < kb_n; ++kb)
-            for (int kk = 0; kk < 4 && kb * 64 + kk * 16 < p.dt_rank; ++kk, ++n)
-              umma_bf16(tbase, umma_desc_sw128(sb + uint32_t(S::kWOff + kb * 16384 + kk * 32)),
-                        umma_desc_sw128(st + uint32_t(S::kDtOff + kb * kTileT * 128 + kk * 32)),
-                        idesc, n > 0 ? 1u : 0u);
-          umma_commit(mma_bar);
-        }
-        __syncwarp();
-        ++mma_issued;
-        good = __all_sync(0xffffffffu, mbar_wait(mma_bar, uint32_t(k) & 1u, p.status));
-        if (!good) break;
-        ++mma_waited;
-        tc_fence_after();
-        float v[kTileT];
-        tmem_ld32(tbase, v);
-        tmem_wait_ld();
-        const uint32_t dt32 = st + uint32_t(S::kDt32Off) + uint32_t(lane) * 4u;
-#pragma unroll
-        for (int t = 0; t < kTileT; ++t) sts_f32(dt32 + uint32_t(t * S::kDt32Stride * 4), v[t]);
-        tc_fence_before();
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&bc_ready[s]);
+      if constexpr (kProdMma) {
+        if (k + 1 < ntiles) {
+          good = dt_issue(k + 1);
+          if (!good) break;
+        }
+      }
       // refill the stage of the previous tile once every scan warp is done with it
       if (k >= 1 && k - 1 + kStages < ntiles) {
         const int sp = (k - 1) % kStages;
@@ -342,18 +412,10 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
       // every copy this CTA started must land before it exits
       for (int k = issued - kStages < 0 ? 0 : issued - kStages; k < issued; ++k)
         mbar_wait(&full[k % kStages], uint32_t(k / kStages) & 1u, nullptr);
-      if (kDtProj && mma_issued == 0) mbar_wait(w_bar, 0, nullptr);
     }
-    if constexpr (kDtProj) {
-      // no product may still be writing the accumulator when it is freed
-      if (mma_issued > mma_waited) mbar_wait(mma_bar, uint32_t(mma_issued - 1) & 1u, nullptr);
-      __syncwarp();
-      tc_fence_after();
-      tmem_dealloc(tbase, 32);
-    }
+    if constexpr (kProdMma) dt_teardown();
     return;
   }
-
   // ================================================================== scan warps
   const int g = warp / kGroupWarps;       // time group
   const int w4 = warp % kGroupWarps;      // channel slice of the group
@@ -423,7 +485,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
     const int t = (g * QG + e) * 4 + j;
 #pragma unroll
     for (int m = 0; m < 4; ++m) xoff[e][m] = uint32_t(S::kXOff) + swz64(t + 1 + m, col);
-    dtoff[e] = kDtProj ? uint32_t(S::kDt32Off + (t * S::kDt32Stride + cl) * 4)
+    dtoff[e] = kDtProj ? uint32_t(S::kDtOff + (t * 32 + (cl ^ (j << 3))) * 4)
                        : uint32_t(S::kDtOff) + swz64(t, col);
     zoff[e] = uint32_t(S::kZOff) + swz64(t, col);
   }
@@ -491,7 +553,7 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
       }
       const float pre = fmaf(cw.w, x0, fmaf(cw.z, x1, fmaf(cw.y, x2, fmaf(cw.x, x3, cb))));
       const float u = silu_tanh(pre);
-      const float dtv = kDtProj ? lds_f32(st + dtoff[e] + uint32_t((qq >> 1) * 8 * S::kDt32Stride * 4))
+      const float dtv = kDtProj ? lds_f32(st + dtoff[e] + uint32_t((qq >> 1) * 8 * 32 * 4))
                                 : bf(lds_u16(rb + dtoff[e]));
       const float dl = softplus_lg2(dtv + dtb);
       const bool valid = t < valid_n;
@@ -501,9 +563,11 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
         if (valid && ((rs >> (t + 4)) & 1u)) dlt = __int_as_float(0x7f800000);   // decay 0
       const float sk = Dd * u;
       const float sz = silu_tanh(bf(lds_u16(rb + zoff[e])));
-      // swap area of quad qq: channel chl's {Delta[4], Delta*u[4]} (48-byte records: both the
-      // lanes' 4-byte stores and the 16-byte loads are free of bank conflicts)
-      const uint32_t xa = xch + uint32_t((qq * 8 + chl) * S::kXchRec);
+      // swap area of quad parity qq & 1: channel chl's {Delta[4], Delta*u[4]} (48-byte records:
+      // both the lanes' 4-byte stores and the 16-byte loads are free of bank conflicts).  Two
+      // areas suffice: quad qq + 2 overwrites quad qq's only after the __syncwarp of quad
+      // qq + 1, which every lane reaches after its loads of quad qq.
+      const uint32_t xa = xch + uint32_t(((qq & 1) * 8 + chl) * S::kXchRec);
       sts_f32(xa + 4 * j, dlt);
       sts_f32(xa + 16 + 4 * j, du);
       __syncwarp();

@@ -306,11 +306,11 @@ struct FwdMaps {
   CUtensorMap w;    // the fused dt projection's W_dt (unused otherwise)
 };
 
-template <int N, bool kExt, int G, bool kChained, bool kDtProj>
+template <int N, bool kExt, int G, bool kChained, int KB>
 cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 grid,
                                cudaStream_t st) {
-  using S = mm::f2::Smem<N, G, kDtProj>;
-  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained, kDtProj>;
+  using S = mm::f2::Smem<N, G, KB>;
+  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained, KB>;
   static bool attr_set = false;   // the attribute is set once per instantiation
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -318,24 +318,24 @@ cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 g
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  kern<<<grid, mm::f2::threads<G>(), S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, m.w, a);
+  kern<<<grid, mm::f2::threads<G, KB>(), S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, m.w, a);
   return cudaGetLastError();
 }
 
-template <int N, bool kExt, bool kDtProj = false>
+// KB = K blocks of 64 of the fused dt projection (0: dt_raw is an input).  One time group
+// runs unchained only (the plan picks it for many channel tiles, one chunk per row).
+template <int N, bool kExt, int KB = 0>
 cudaError_t launch_fwd2(const FwdMaps& m, const mm::f2::Params& a, const FwdPlan& f,
                         cudaStream_t st) {
   const unsigned gx = unsigned(a.ntd);
   const dim3 units(gx * unsigned(a.batch) * unsigned(a.nchunks)), tiles(gx, unsigned(a.batch), 1);
-  if constexpr (kDtProj) {
-    if (f.G == 1)
-      return f.chained ? launch_fwd2_kernel<N, false, 1, true, true>(m, a, units, st)
-                       : launch_fwd2_kernel<N, false, 1, false, true>(m, a, tiles, st);
-    return f.chained ? launch_fwd2_kernel<N, false, 4, true, true>(m, a, units, st)
-                     : launch_fwd2_kernel<N, false, 4, false, true>(m, a, tiles, st);
+  if constexpr (KB > 0) {
+    if (f.G == 1) return launch_fwd2_kernel<N, false, 1, false, KB>(m, a, tiles, st);
+    return f.chained ? launch_fwd2_kernel<N, false, 4, true, KB>(m, a, units, st)
+                     : launch_fwd2_kernel<N, false, 4, false, KB>(m, a, tiles, st);
   } else {
-    return f.chained ? launch_fwd2_kernel<N, kExt, 4, true, false>(m, a, units, st)
-                     : launch_fwd2_kernel<N, kExt, 4, false, false>(m, a, tiles, st);
+    return f.chained ? launch_fwd2_kernel<N, kExt, 4, true, 0>(m, a, units, st)
+                     : launch_fwd2_kernel<N, kExt, 4, false, 0>(m, a, tiles, st);
   }
 }
 
@@ -497,9 +497,9 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   if (dtproj) {
     if (dims->io_dtype != MAMBA_BF16)
       return fail(MAMBA_ERR_UNSUPPORTED, "the fused dt projection takes bf16 I/O only");
-    if (dt_rank % 8 != 0 || dt_rank > 64 * mm::f2::kDtBlocks)
+    if (dt_rank % 8 != 0 || dt_rank > 64 * mm::f2::kMaxDtBlocks)
       return fail(MAMBA_ERR_UNSUPPORTED, "dt_rank %lld unsupported (a multiple of 8 up to %d)",
-                  (long long)dt_rank, 64 * mm::f2::kDtBlocks);
+                  (long long)dt_rank, 64 * mm::f2::kMaxDtBlocks);
     if ((rc = check_ptr(dt_low, "dt_low", act, 16)) ||
         (rc = check_ptr(W_dt, "W_dt", dims->d_inner > 0, 16)))
       return rc;
@@ -615,9 +615,12 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
         return fail(MAMBA_ERR_CUDA, "workspace reset failed: %s", cudaGetErrorString(e));
     }
     const bool ext = seq_idx || h_in || conv_state_in;
-    if (dtproj)
-      e = N == 16 ? launch_fwd2<16, false, true>(m, a2, fplan, st)
-                  : launch_fwd2<8, false, true>(m, a2, fplan, st);
+    if (dtproj && dt_rank <= 64)
+      e = N == 16 ? launch_fwd2<16, false, 1>(m, a2, fplan, st)
+                  : launch_fwd2<8, false, 1>(m, a2, fplan, st);
+    else if (dtproj)
+      e = N == 16 ? launch_fwd2<16, false, 2>(m, a2, fplan, st)
+                  : launch_fwd2<8, false, 2>(m, a2, fplan, st);
     else if (N == 16)
       e = ext ? launch_fwd2<16, true>(m, a2, fplan, st) : launch_fwd2<16, false>(m, a2, fplan, st);
     else
