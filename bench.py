@@ -127,7 +127,7 @@ def measured_peaks() -> dict:
 # while they are unchanged.  (Host code and the time-chunk plan live in mamba_mixer.cu; each
 # record names the plan it was taken with.)
 KERNEL_SOURCES = {
-    "fwd": ("fwd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
+    "fwd": ("fwd_kernel.cuh", "fwd2_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
     "step": ("step.cuh", "device_math.cuh", "sm100_primitives.cuh"),
     "ssd": ("ssd_kernel.cuh", "device_math.cuh", "sm100_primitives.cuh"),
     "ssd_step": ("ssd_step.cuh", "device_math.cuh"),

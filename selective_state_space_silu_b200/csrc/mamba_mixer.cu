@@ -164,11 +164,8 @@ Plan make_plan(const mamba_dims* d) {
 // claimed in order, so a unit's predecessor is always running or done.  Measured on the
 // long workload (2 x 65536 x 2560): 3.45-3.48 ms with 8, 16 or 32 chunks per row, against
 // 3.65 ms for the parallel chunks with their chunk-state pass.
-#ifndef MM_FWD_G4_UNITS
-#define MM_FWD_G4_UNITS 16
-#endif
 constexpr int64_t kG4MinChunkLen = 1024;
-constexpr int64_t kG4MaxChunks = MM_FWD_G4_UNITS;
+constexpr int64_t kG4MaxChunks = 16;
 constexpr size_t kUnitCounterOff = 64;                // in the header, after the status word
 
 struct FwdPlan {

@@ -32,6 +32,7 @@ def _dims(w):
     (3, 77, 40, 8, 24, 4),         # d_state 8, dt_rank not a multiple of 16, ragged tile
     (10, 200, 1024, 16, 16, 1),    # 320 channel tiles: one time group
     (10, 65, 968, 16, 128, 1),     # one time group, ragged channel tile, dt_rank 128
+    (10, 100, 1024, 8, 64, 1),     # one time group, d_state 8, one full K block
 ])
 def test_dtproj_matches_oracle(oracle, Bt, L, Di, N, R, groups):
     w = I.Workload("dtproj", Bt, L, Di, N, 4, I.BF16, 5000 + L + R)
