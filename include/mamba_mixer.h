@@ -99,19 +99,24 @@ typedef struct {
 
 /*
  * Device workspace, in bytes, that mamba_mixer_fwd needs for `dims`: a 256-byte header
- * whose first 4 bytes are the status word, then -- when the sequence is split into time
- * chunks that run in parallel -- each chunk's carry aggregate (decay product and local end
- * state, fp32 [batch, chunks-1, d_inner, d_state] each).  The status word must be zero
- * before the first forward that uses the workspace (clear the header once after
- * allocating it); the library only sets it on a timeout and mamba_mixer_check clears it.
- * Returns 0 for dims the library does not support (mamba_mixer_fwd then reports why).
+ * whose first 4 bytes are the status word, then, when the sequence is split into time
+ * chunks, what the chunks hand on:
+ *   - bf16 I/O (chained chunks, one launch): one flag per (32-channel tile, scan warp) and
+ *     each tile's carried state, fp32 [tiles, 32, d_state]; the forward resets the flags
+ *     and its unit counter (header bytes 64..67) itself on the stream;
+ *   - fp32 I/O (a chunk-state pass, then the main pass): each chunk's carry aggregate
+ *     (decay product and local end state, fp32 [batch, chunks-1, d_inner, d_state] each).
+ * The status word must be zero before the first forward that uses the workspace (clear the
+ * header once after allocating it); the library only sets it on a timeout and
+ * mamba_mixer_check clears it.  Returns 0 for dims the library does not support
+ * (mamba_mixer_fwd then reports why).
  */
 MAMBA_API size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims);
 
 /*
- * Number of kernels one mamba_mixer_fwd call with `dims` launches (1, or 2 when the
- * sequence is split into time chunks: the chunk-state pass, then the main pass); 0 when
- * there is nothing to compute; -1 for unsupported dims.
+ * Number of kernels one mamba_mixer_fwd call with `dims` launches (1, or 2 for fp32 I/O
+ * with time chunks: the chunk-state pass, then the main pass); 0 when there is nothing to
+ * compute; -1 for unsupported dims.
  */
 MAMBA_API int mamba_mixer_fwd_launches(const mamba_dims* dims);
 
@@ -277,6 +282,16 @@ MAMBA_API int mamba_mixer_step_check(void* cuda_stream);
  * gave up on a bounded wait (its outputs are then incomplete), MAMBA_OK otherwise.
  */
 MAMBA_API int mamba_mixer_check(void* workspace, void* cuda_stream);
+
+/*
+ * Test hook for the bounded-wait path; not for production use.  tile >= 0 makes the CTA
+ * of channel tile 0, batch row 0 and time chunk 0 of every following forward arm the
+ * barrier of its time tile `tile` without issuing that tile's copies, so that its waits run
+ * out (after about one second), it stops cleanly and the call's status word reads
+ * MAMBA_ERR_TIMEOUT; no GPU fault is involved.  tile = -1 (the default) turns it off.
+ * Process-wide; takes effect for launches enqueued after the call.
+ */
+MAMBA_API void mamba_mixer_set_fault_injection(int tile);
 
 /*
  * The fused forward for callers that cannot allocate device memory.  The pages describe no

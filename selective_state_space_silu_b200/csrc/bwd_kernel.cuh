@@ -112,11 +112,17 @@ struct BwdSmem {
   static constexpr int kCOff = kBOff + kBwdT * kBCRow;
   static constexpr int kSlot = kCOff + kBwdT * kBCRow;
   static constexpr int kHs = kBwdT * kBwdThreads * kS * 4;   // h_t per (step, lane)
-  static constexpr int kSc = kBwdT * kBwdCh * 16;            // {pre, s(pre), Delta, s(v)} per (step, ch)
+  static constexpr int kSc = kBwdT * kBwdCh * 16;            // {Delta, u, dyc, 0} per (step, ch)
+  static constexpr int kSc2 = kBwdT * kBwdCh * 16;           // {SiLU'(pre), s(v), gate', 0}
+  static constexpr int kE = kBwdT * kBwdCh * 16;             // {C.h, lam.B, sum ah A, dpre}
+  static constexpr int kDn = 4 * kBwdCh * 4;                 // dpre of the later tile's steps 0..2
   static constexpr int kAcc = 2 * kBwdT * N * 4;              // dB, dC partial sums per tile
   static constexpr int kHsOff = 2 * kSlot;
   static constexpr int kScOff = kHsOff + kHs;
-  static constexpr int kAccOff = kScOff + kSc;
+  static constexpr int kSc2Off = kScOff + kSc;
+  static constexpr int kEOff = kSc2Off + kSc2;
+  static constexpr int kDnOff = kEOff + kE;
+  static constexpr int kAccOff = kDnOff + kDn;
   static constexpr int kTotal = kAccOff + kAcc;
   static_assert(kSlot % 16 == 0 && kRow % 16 == 0 && kBCRow % 16 == 0, "16-byte staging units");
 };
@@ -201,6 +207,9 @@ bwd_kernel(const BwdArgs<kExt> p) {
   const uint32_t sb = smem_addr(smem);
   const uint32_t hsa = sb + uint32_t(Sm::kHsOff) + uint32_t(threadIdx.x * (N / 4) * 4);  // this lane's h_t slots
   float4* sc = reinterpret_cast<float4*>(smem + Sm::kScOff);
+  float4* sc2 = reinterpret_cast<float4*>(smem + Sm::kSc2Off);
+  float4* E = reinterpret_cast<float4*>(smem + Sm::kEOff);
+  float* dnext = reinterpret_cast<float*>(smem + Sm::kDnOff);   // [3][kBwdCh]
   float* acc = reinterpret_cast<float*>(smem + Sm::kAccOff);   // [2][T][N]
 
   const int tid = threadIdx.x;
@@ -327,18 +336,31 @@ bwd_kernel(const BwdArgs<kExt> p) {
   float* ck = p.ws_h + ((b * p.ntiles) * Di + d) * N + j * kS;   // + k * Di * N per tile
   const uint32_t colx = uint32_t(cl * kEs);
   const uint32_t colbc = uint32_t(j * kS * kEs);
-  // The per-(t, d) scalars of a tile -- {pre, sigmoid(pre), Delta, sigmoid(v)} into sc --
-  // computed once per (t, d): the 4 lanes of a channel take steps j, j+4, j+8, j+12.
-  // xr(i) is x' of step t0 + i (i >= -3).
-  auto tile_scalars = [&](uint32_t sl, int cnt, uint32_t bits, auto xr) {
+  // The per-(t, d) scalars of a tile, computed once per (t, d): the 4 lanes of a channel take
+  // steps j, j+4, j+8, j+12.  sc gets {Delta, u, dyc, 0}; with kFull (the reverse sweep,
+  // whose tiles also hold z and dy) dyc = dy*z*s(z) is the gated output's gradient and sc2
+  // gets {SiLU'(pre), s(v), dy*SiLU'(z), 0}, s the logistic function.  xr(i) is x' of step
+  // t0 + i (i >= -3).
+  auto tile_scalars = [&](auto full_tag, uint32_t sl, int cnt, uint32_t bits, auto xr) {
+    constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
     for (int m = 0; m < kBwdT / 4; ++m) {
       const int i = j + 4 * m;
       if (i < cnt) {
         const float pre = conv_pre(xr(i - 3), xr(i - 2), xr(i - 1), xr(i), bits, i);
         const float v = lds_one<IO>(sl + Sm::kDtOff + i * Sm::kRow + colx) + dtb;
-        sc[i * kBwdCh + cl] = make_float4(pre, sigmoid_<kPrecise>(pre), M::softplus(v),
-                                          sigmoid_<kPrecise>(v));
+        const float sp = sigmoid_<kPrecise>(pre);
+        const float u = pre * sp;
+        float dyc = 0.0f;
+        if constexpr (kFull) {
+          const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
+          const float dyt = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx);
+          const float sz = sigmoid_<kPrecise>(zt);
+          dyc = dyt * zt * sz;
+          sc2[i * kBwdCh + cl] = make_float4(sp * (1.0f + pre * (1.0f - sp)), sigmoid_<kPrecise>(v),
+                                             dyt * (sz * (1.0f + zt * (1.0f - sz))), 0.0f);
+        }
+        sc[i * kBwdCh + cl] = make_float4(M::softplus(v), u, dyc, 0.0f);
       }
     }
     __syncwarp();
@@ -415,17 +437,16 @@ bwd_kernel(const BwdArgs<kExt> p) {
         const uint32_t sl = sb + uint32_t((it & 1) * Sm::kSlot);
         const int64_t t0 = int64_t(k) * kBwdT;
         const int cnt = int(t0 + kBwdT < t_end ? kBwdT : t_end - t0);
-        tile_scalars(sl, cnt, bits, [&](int i) {
+        tile_scalars(std::false_type{}, sl, cnt, bits, [&](int i) {
           if (kExt && t0 + i < 0) return x_before(t0 + i);
           return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
         });
 #pragma unroll 2
         for (int i = 0; i < cnt; ++i) {
           const float4 q = sc[i * kBwdCh + cl];
-          const float del = q.z;
           float Bv[kS];
           lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-          step_state(h, del, del * (q.x * q.y), Bv, (bits >> (i + 4)) & 1u);
+          step_state(h, q.x, q.x * q.y, Bv, (bits >> (i + 4)) & 1u);
         }
         __syncthreads();   // the slot (and sc) are refilled by the next iteration
       }
@@ -443,10 +464,13 @@ bwd_kernel(const BwdArgs<kExt> p) {
       for (int s = 0; s < kS; ++s)
         lam[s] = (cc < p.nchunks - 1 ? p.ws_P[oP + s] * lam[s] : 0.0f) + p.ws_L[oL + s];
     }
-    // conv input gradient still to add to the positions 1, 2, 3 before the current step
-    float q1 = 0.0f, q2 = 0.0f, q3 = 0.0f;
+    // per-d gradient sums of this lane's steps (reduced over the channel's 4 lanes at the end)
     float aD = 0.0f, aDtb = 0.0f, aCb = 0.0f, aW0 = 0.0f, aW1 = 0.0f, aW2 = 0.0f, aW3 = 0.0f;
     for (int i = tid; i < 2 * kBwdT * N; i += kBwdThreads) acc[i] = 0.0f;
+    // no tile after the chunk's last: the dpre of the steps after it count as zero here (the
+    // next chunk adds its own part of those input gradients)
+    if (j < 3) dnext[j * kBwdCh + cl] = 0.0f;
+    uint32_t bits_later = 0u;   // reset bits of the tile after the current one
     __syncthreads();   // also orders this thread's checkpoint stores before its reloads
 
     float hn[kS];   // start state of the tile processed next (loaded one tile ahead)
@@ -454,6 +478,11 @@ bwd_kernel(const BwdArgs<kExt> p) {
     for (int s = 0; s < kS; ++s) hn[s] = ck[int64_t(ke - 1) * Di * N + s];
     stage(ke - 1, 0, true);
     int32_t id = ids_for(ke - 1);
+    // no reset at s, s-1, .., s-r+1 (step s of a tile with reset bits `bt`): the conv tap r
+    // of step s (x' of step s - r) reaches its pre-activation
+    auto tap_live = [](uint32_t bt, int s, int r) -> bool {
+      return ((bt >> (s + 5 - r)) & ((1u << r) - 1u)) == 0u;
+    };
     for (int k = ke - 1, it = 0; k >= kb; --k, ++it) {
       if (k - 1 >= kb) stage(k - 1, (it + 1) & 1, true);
       else cp_async_commit_();
@@ -476,62 +505,66 @@ bwd_kernel(const BwdArgs<kExt> p) {
         return lds_one<IO>(sl + Sm::kXOff + uint32_t((i + kBwdHalo) * Sm::kRow) + colx);
       };
 
-      // recompute the tile: {pre, sigmoid(pre), Delta, sigmoid(v)}, then the states h_t
-      tile_scalars(sl, cnt, bits, xrow);
+      // recompute the tile: the per-(t, d) scalars, then the states h_t
+      tile_scalars(std::true_type{}, sl, cnt, bits, xrow);
 #pragma unroll 2
       for (int i = 0; i < cnt; ++i) {
         const float4 q = sc[i * kBwdCh + cl];
         float Bv[kS];
         lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
-        step_state(h, q.z, q.z * (q.x * q.y), Bv, (bits >> (i + 4)) & 1u);
+        step_state(h, q.x, q.x * q.y, Bv, (bits >> (i + 4)) & 1u);
         sts_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), h);
       }
       __syncwarp();
 
+      // walk the tile backwards with the adjoint state; per step, this lane's partial sums
+      // of C.h, lam.B and sum_n lam h_{t-1} a A go to the step's record (one per lane after a
+      // reduce-scatter over the channel's 4 lanes), dB and dC to the tile's sums
+      float ht[kS];
+      lds_states<kS>(hsa + uint32_t((cnt - 1) * kBwdThreads * kS * 4), ht);
 #pragma unroll 2
       for (int i = cnt - 1; i >= 0; --i) {
-        const int64_t t = t0 + i;
         const bool m1 = !((bits >> (i + 4)) & 1u);           // no reset at t
-        const bool m2 = m1 && !((bits >> (i + 3)) & 1u);
-        const bool m3 = m2 && !((bits >> (i + 2)) & 1u);
         const float4 q = sc[i * kBwdCh + cl];
-        const float pre = q.x, sp = q.y, del = q.z, sv = q.w;   // sp, sv: sigmoid(pre), sigmoid(v)
-        const float u = pre * sp;
-        const float zt = lds_one<IO>(sl + Sm::kZOff + i * Sm::kRow + colx);
-        const float dyt = lds_one<IO>(sl + Sm::kDyOff + i * Sm::kRow + colx);
-        const float sz = sigmoid_<kPrecise>(zt);
-        const float dyc = dyt * zt * sz;
-        float Bv[kS], Cv[kS], hp[kS], ht[kS];
+        const float del = q.x, u = q.y, dyc = q.z;
+        const float delu = del * u;
+        float Bv[kS], Cv[kS], hp[kS];
         lds_io_row<kS, IO>(sl + Sm::kBOff + i * Sm::kBCRow + colbc, Bv);
         lds_io_row<kS, IO>(sl + Sm::kCOff + i * Sm::kBCRow + colbc, Cv);
-        float ycp = 0.0f, duP = 0.0f, ddP = 0.0f, cB[kS], cC[kS];
-        lds_states<kS>(hsa + uint32_t(i * kBwdThreads * kS * 4), ht);
         if (i > 0) {
           lds_states<kS>(hsa + uint32_t((i - 1) * kBwdThreads * kS * 4), hp);
         } else {
 #pragma unroll
           for (int s = 0; s < kS; ++s) hp[s] = h0[s];
         }
+        float ycp = 0.0f, lamB = 0.0f, ahA = 0.0f, cB[kS], cC[kS];
 #pragma unroll
         for (int s = 0; s < kS; ++s) {
-          if (!m1) hp[s] = 0.0f;                               // the state entering a reset
+          const float hin = m1 ? hp[s] : 0.0f;                 // the state entering step t
           ycp += Cv[s] * ht[s];
           const float a = M::decay(del, A2[s]);
           lam[s] += dyc * Cv[s];
-          cB[s] = lam[s] * del * u;
+          cB[s] = lam[s] * delu;
           cC[s] = dyc * ht[s];
-          duP += lam[s] * del * Bv[s];
-          const float ah = lam[s] * hp[s] * a;
-          ddP += lam[s] * Bv[s] * u + ah * A[s];
+          lamB += lam[s] * Bv[s];
+          const float ah = lam[s] * hin * a;
+          ahA += ah * A[s];
           dA[s] += ah * del;
           lam[s] = m1 ? lam[s] * a : 0.0f;
+          ht[s] = hp[s];                                       // h_t of step t - 1
         }
-        // channel sums over the 4 lanes of a channel (lane bits 3 and 4)
-#pragma unroll
-        for (int m = 8; m <= 16; m <<= 1) {
-          ycp += __shfl_xor_sync(0xffffffffu, ycp, m);
-          duP += __shfl_xor_sync(0xffffffffu, duP, m);
-          ddP += __shfl_xor_sync(0xffffffffu, ddP, m);
+        // reduce-scatter of {C.h, lam.B, sum ah A} over the channel's 4 lanes (lane bits 4,
+        // 3): lane j ends with the channel's sum of value j (lane 3 with nothing)
+        {
+          const bool hi = (j & 2) != 0;
+          float k0 = hi ? ahA : ycp, k1 = hi ? 0.0f : lamB;
+          const float s0 = hi ? ycp : ahA, s1 = hi ? lamB : 0.0f;
+          k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+          k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+          const bool odd = (j & 1) != 0;
+          float kp = odd ? k1 : k0;
+          kp += __shfl_xor_sync(0xffffffffu, odd ? k0 : k1, 8);
+          if (j < 3) reinterpret_cast<float*>(E + i * kBwdCh + cl)[j] = kp;
         }
         // dB, dC summed over the warp's 8 channels (lane bits 0..2) by a reduce-scatter:
         // the 2*kS values {cB, cC} are halved at each round, so lane chl ends with value chl
@@ -561,31 +594,69 @@ bwd_kernel(const BwdArgs<kExt> p) {
             atomicAdd(&acc[(which * kBwdT + i) * N + j * kS + s], vv[0]);
           }
         }
-        const float yc = ycp + Dd * u;
-        const float du = duP + dyc * Dd;
-        const float dv = ddP * sv;                              // softplus' = sigmoid
-        const float dpre = du * (sp * (1.0f + pre * (1.0f - sp)));   // SiLU'(pre)
-        // the taps of step t: x' of steps t .. t-3, live unless before the document start
-        aW3 += dpre * xrow(i);
-        if (m1) aW2 += dpre * xrow(i - 1);
-        if (m2) aW1 += dpre * xrow(i - 2);
-        if (m3) aW0 += dpre * xrow(i - 3);
-        aCb += dpre;
-        aDtb += dv;
-        aD += dyc * u;
-        // the conv input gradient of step t is complete; pass the taps' parts back
-        const float dx = w3 * dpre + q1;
-        q1 = q2 + (m1 ? w2 * dpre : 0.0f);
-        q2 = q3 + (m2 ? w1 * dpre : 0.0f);
-        q3 = m3 ? w0 * dpre : 0.0f;
-        if (j == 0 && active) {
-          const int64_t o = (b * L + t) * Di + d;
-          p.dz[o] = dyt * yc * (sz * (1.0f + zt * (1.0f - sz)));
-          p.ddt[o] = dv;
-          if (c < p.nchunks - 1 && t >= t_end - 3) atomicAdd(p.dxp + o, dx);  // + next chunk's part
-          else p.dxp[o] = dx;
+      }
+      __syncwarp();
+
+      // per (t, d), once (lane j takes steps j, j+4, j+8, j+12): the gate, Delta and conv
+      // pre-activation gradients
+      float dp[kBwdT / 4];
+#pragma unroll
+      for (int m = 0; m < kBwdT / 4; ++m) {
+        const int i = j + 4 * m;
+        dp[m] = 0.0f;
+        if (i < cnt) {
+          const float4 e = E[i * kBwdCh + cl];             // {C.h, lam.B, sum ah A, -}
+          const float4 q = sc[i * kBwdCh + cl];            // {Delta, u, dyc, -}
+          const float4 g = sc2[i * kBwdCh + cl];           // {SiLU'(pre), s(v), gate', -}
+          const float yc = e.x + Dd * q.y;
+          const float du = q.x * e.y + q.z * Dd;
+          const float dv = (q.y * e.y + e.z) * g.y;        // softplus' = s
+          dp[m] = du * g.x;
+          reinterpret_cast<float*>(E + i * kBwdCh + cl)[3] = dp[m];
+          aD += q.z * q.y;
+          aDtb += dv;
+          aCb += dp[m];
+          if (active) {
+            const int64_t o = (b * L + t0 + i) * Di + d;
+            p.dz[o] = yc * g.z;
+            p.ddt[o] = dv;
+          }
         }
       }
+      __syncwarp();
+      // the conv: x' of step t feeds the pre-activations of steps t .. t+3 (taps 0..3 back);
+      // its input gradient takes their dpre, the later tile's first 3 from dnext
+#pragma unroll
+      for (int m = 0; m < kBwdT / 4; ++m) {
+        const int i = j + 4 * m;
+        if (i < cnt) {
+          const float d0v = dp[m];
+          aW3 += d0v * xrow(i);
+          if (tap_live(bits, i, 1)) aW2 += d0v * xrow(i - 1);
+          if (tap_live(bits, i, 2)) aW1 += d0v * xrow(i - 2);
+          if (tap_live(bits, i, 3)) aW0 += d0v * xrow(i - 3);
+          float dx = w3 * d0v;
+#pragma unroll
+          for (int r = 1; r <= 3; ++r) {
+            const int sidx = i + r;
+            const float wr = r == 1 ? w2 : r == 2 ? w1 : w0;
+            if (sidx < cnt) {
+              if (tap_live(bits, sidx, r)) dx += wr * reinterpret_cast<const float*>(E + sidx * kBwdCh + cl)[3];
+            } else if (sidx >= kBwdT) {
+              if (tap_live(bits_later, sidx - kBwdT, r)) dx += wr * dnext[(sidx - kBwdT) * kBwdCh + cl];
+            }
+          }
+          if (active) {
+            const int64_t t = t0 + i;
+            const int64_t o = (b * L + t) * Di + d;
+            if (c < p.nchunks - 1 && t >= t_end - 3) atomicAdd(p.dxp + o, dx);  // + next chunk's part
+            else p.dxp[o] = dx;
+          }
+        }
+      }
+      __syncwarp();
+      if (j < 3) dnext[j * kBwdCh + cl] = dp[0];           // steps 0..2 of this tile, for the next
+      bits_later = bits;
       __syncthreads();
       // this tile's dB, dC of the CTA's 32 channels into the global sums
       for (int e = tid; e < 2 * kBwdT * N; e += kBwdThreads) {
@@ -600,25 +671,53 @@ bwd_kernel(const BwdArgs<kExt> p) {
     }
     cp_async_wait_<0>();
 
+    // sums over the channel's 4 lanes (lane bits 3 and 4)
+#pragma unroll
+    for (int m = 8; m <= 16; m <<= 1) {
+      aD += __shfl_xor_sync(0xffffffffu, aD, m);
+      aDtb += __shfl_xor_sync(0xffffffffu, aDtb, m);
+      aCb += __shfl_xor_sync(0xffffffffu, aCb, m);
+      aW0 += __shfl_xor_sync(0xffffffffu, aW0, m);
+      aW1 += __shfl_xor_sync(0xffffffffu, aW1, m);
+      aW2 += __shfl_xor_sync(0xffffffffu, aW2, m);
+      aW3 += __shfl_xor_sync(0xffffffffu, aW3, m);
+    }
     if (!active) return;
-    if (c > 0) {
-      // this chunk's part of the input gradient of the previous chunk's last 3 steps
-      if (j == 0) {
-        float* o = p.dxp + (b * L + t_begin) * Di + d;
-        atomicAdd(o - Di, q1);
-        atomicAdd(o - 2 * Di, q2);
-        atomicAdd(o - 3 * Di, q3);
+    // the input gradient of the 3 positions before the chunk from its first 3 steps' dpre
+    // (dnext now holds them; bits_later the reset bits of the chunk's first tile)
+    if (j == 0) {
+      float qv[3];
+#pragma unroll
+      for (int qq = 1; qq <= 3; ++qq) {
+        float v = 0.0f;
+#pragma unroll
+        for (int r = qq; r <= 3; ++r) {
+          const int sidx = r - qq;                           // step of the chunk's first tile
+          const float wr = r == 1 ? w2 : r == 2 ? w1 : w0;
+          if (sidx < int(t_end - t_begin) && tap_live(bits_later, sidx, r))
+            v += wr * dnext[sidx * kBwdCh + cl];
+        }
+        qv[qq - 1] = v;
       }
-    } else if constexpr (kExt) {
-      // the adjoint after step 0 is the gradient of the initial state; the conv input
-      // gradient of the 3 positions before 0, that of the initial conv window
-      if (p.dh_in) {
+      if (c > 0) {
+        // this chunk's part of the input gradient of the previous chunk's last 3 steps
+        float* o = p.dxp + (b * L + t_begin) * Di + d;
+        atomicAdd(o - Di, qv[0]);
+        atomicAdd(o - 2 * Di, qv[1]);
+        atomicAdd(o - 3 * Di, qv[2]);
+      } else if constexpr (kExt) {
+        // the conv input gradient of the 3 positions before 0 is that of the initial window
+        if (p.dcs_in) {
+          float* o = p.dcs_in + (b * Di + d) * 3;
+          o[2] = qv[0]; o[1] = qv[1]; o[0] = qv[2];
+        }
+      }
+    }
+    if constexpr (kExt) {
+      // the adjoint after step 0 is the gradient of the initial state
+      if (c == 0 && p.dh_in) {
 #pragma unroll
         for (int s = 0; s < kS; ++s) p.dh_in[(b * Di + d) * N + j * kS + s] = lam[s];
-      }
-      if (p.dcs_in && j == 0) {
-        float* o = p.dcs_in + (b * Di + d) * 3;
-        o[2] = q1; o[1] = q2; o[0] = q3;
       }
     }
 #pragma unroll

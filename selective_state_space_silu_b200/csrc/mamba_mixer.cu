@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -40,13 +41,20 @@ int ok() {
   return MAMBA_OK;
 }
 
-// Test-only failure injection for the bounded-wait path: MAMBA_MIXER_INJECT_SKIP_TILE=k makes
-// one CTA of the next forwards skip the copies of its tile k; unset (the default) injects
-// nothing.  Read at every call (a getenv is negligible next to a forward launch), so that a
-// test can set and clear it within one process.
-int inject_skip_tile() {
-  const char* inj = getenv("MAMBA_MIXER_INJECT_SKIP_TILE");
-  return inj ? atoi(inj) : -1;
+// Test-only failure injection for the bounded-wait path (mamba_mixer_set_fault_injection):
+// k >= 0 makes one CTA of the next forwards skip the copies of its tile k; -1 (the default)
+// injects nothing.
+std::atomic<int> g_inject_skip_tile{-1};
+int inject_skip_tile() { return g_inject_skip_tile.load(std::memory_order_relaxed); }
+
+// cudaFuncSetAttribute for a kernel's dynamic shared memory, once per kernel instantiation
+// (each call site is its own template instance, so its static flag covers one kernel).
+template <typename K>
+cudaError_t set_smem_once(K kern, int bytes, bool& done) {
+  if (done) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done = true;
+  return e;
 }
 
 struct Span {
@@ -308,13 +316,9 @@ cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 g
                                cudaStream_t st) {
   using S = mm::f2::Smem<N, G, KB>;
   auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained, KB>;
-  static bool attr_set = false;   // the attribute is set once per instantiation
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         S::kDynamic);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static bool attr_set = false;
+  const cudaError_t e = set_smem_once(kern, S::kDynamic, attr_set);
+  if (e != cudaSuccess) return e;
   kern<<<grid, mm::f2::threads<G, KB>(), S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, m.w, a);
   return cudaGetLastError();
 }
@@ -343,8 +347,8 @@ cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdArgs<kExt>& a, dim3
                               cudaStream_t st) {
   using S = mm::FwdSmem<IO, N>;
   auto kern = mm::fwd_kernel<N, IO, P, kPre, kExt>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       S::kDynamic);
+  static bool attr_set = false;
+  const cudaError_t e = set_smem_once(kern, S::kDynamic, attr_set);
   if (e != cudaSuccess) return e;
   kern<<<grid, mm::kFwdThreads, S::kDynamic, st>>>(m.x, m.z, m.dt, m.B, m.C, a);
   return cudaGetLastError();
@@ -387,7 +391,8 @@ cudaError_t launch_bwd(const FwdMaps* m, const mm::FwdArgs<kExt>& pre,
         *m, pre, dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), st);
     if (e != cudaSuccess) return e;
     auto adj = mm::bwd_kernel<N, IO, P, true, kExt>;
-    e = cudaFuncSetAttribute(adj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    static bool adj_attr_set = false;
+    e = set_smem_once(adj, smem, adj_attr_set);
     if (e != cudaSuccess) return e;
     adj<<<dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), mm::kBwdThreads, smem, st>>>(a);
     mm::bwd_zero_bounds<<<dim3(unsigned(a.nchunks - 1), unsigned(batch)), 256, 0, st>>>(
@@ -395,7 +400,8 @@ cudaError_t launch_bwd(const FwdMaps* m, const mm::FwdArgs<kExt>& pre,
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   auto kern = mm::bwd_kernel<N, IO, P, false, kExt>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static bool attr_set = false;
+  e = set_smem_once(kern, smem, attr_set);
   if (e != cudaSuccess) return e;
   kern<<<dim3(gx, unsigned(batch), unsigned(a.nchunks)), mm::kBwdThreads, smem, st>>>(a);
   return cudaGetLastError();
@@ -633,8 +639,8 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   a.status = static_cast<int*>(workspace);
   a.L = dims->seqlen; a.Di = Di;
   a.nchunks = plan.nchunks; a.chunk_len = plan.chunk_len;
-  // Test-only failure injection (bounded-wait path): MAMBA_MIXER_INJECT_SKIP_TILE=k makes one
-  // CTA skip the copies of its tile k; unset (the default) injects nothing.
+  // Test-only failure injection (bounded-wait path, mamba_mixer_set_fault_injection): k >= 0
+  // makes one CTA skip the copies of its tile k; -1 (the default) injects nothing.
   a.inject_skip_tile = inject_skip_tile();
   cudaError_t e;
   if (plan.nchunks > 1) {
@@ -723,6 +729,10 @@ int mamba_mixer_step_check(void* cuda_stream) {
                                  "mamba_mixer_step_check", why, sizeof(why)) != 0)
     return fail(MAMBA_ERR_CUDA, "%s", why);
   return mamba_mixer_check(sp, cuda_stream);
+}
+
+void mamba_mixer_set_fault_injection(int tile) {
+  g_inject_skip_tile.store(tile < 0 ? -1 : tile, std::memory_order_relaxed);
 }
 
 int mamba_mixer_check(void* workspace, void* cuda_stream) {

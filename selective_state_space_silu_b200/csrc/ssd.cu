@@ -100,8 +100,12 @@ template <int N, bool kGate, bool kPre, bool kSeq>
 cudaError_t launch_one(const ssd::SsdArgs& a, int64_t batch, int nz, cudaStream_t st) {
   auto kern = ssd::ssd_fwd_kernel<N, kGate, kPre, kSeq>;
   constexpr int smem = ssd::SsdSmem<N, kPre>::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;   // the attribute is set once per instantiation
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   kern<<<dim3(unsigned(a.H), unsigned(batch), unsigned(nz)), ssd::kThreads, smem, st>>>(a);
   return cudaGetLastError();
 }

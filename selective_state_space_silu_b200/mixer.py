@@ -27,6 +27,7 @@ EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba
            "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
            "mamba_mixer_bwd_packed",
            "mamba_mixer_step", "mamba_mixer_step_check", "mamba_mixer_check",
+           "mamba_mixer_set_fault_injection",
            "mamba_mixer_fwd_plan", "mamba_mixer_fwd_dtproj",
            "mamba_mixer_fwd_noalloc",
            "mamba_mixer_noalloc_check", "mamba_last_error", "mamba_version")
@@ -66,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba_mixer_fwd_launches.argtypes = [P]
     lib.mamba_mixer_check.restype = i
     lib.mamba_mixer_check.argtypes = [vp, vp]
+    lib.mamba_mixer_set_fault_injection.restype = None
+    lib.mamba_mixer_set_fault_injection.argtypes = [i]
     lib.mamba_mixer_fwd.restype = i
     lib.mamba_mixer_fwd.argtypes = [P] + [vp] * 13 + [vp, sz, vp]
     lib.mamba_mixer_fwd_packed.restype = i
@@ -153,6 +156,13 @@ def mamba_mixer_check(workspace: torch.Tensor, stream=None) -> None:
     rc = load_library().mamba_mixer_check(workspace.data_ptr(),
                                           _stream_handle(stream, workspace.device))
     _check(rc)
+
+
+def mamba_mixer_set_fault_injection(tile: int) -> None:
+    """Test hook: tile >= 0 makes one CTA of every following forward skip the copies of
+    its time tile ``tile`` so that its bounded waits run out (MAMBA_ERR_TIMEOUT, no GPU
+    fault); -1 turns it off."""
+    load_library().mamba_mixer_set_fault_injection(int(tile))
 
 
 def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,

@@ -20,7 +20,7 @@ from tests.tolerances import assert_close
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_reports_timeout_and_context_survives(monkeypatch, oracle):
+def test_bounded_wait_reports_timeout_and_context_survives(oracle):
     w = I.Workload("fail", 1, 300, 64, 16, 4, "bf16", 77)      # one kernel, 10 tiles
     inp = I.make_inputs(w)
     d = to_device(inp)
@@ -28,14 +28,16 @@ def test_bounded_wait_reports_timeout_and_context_survives(monkeypatch, oracle):
     assert M.mamba_mixer_fwd_launches(dims) == 1
     ws = M.new_workspace(dims, "cuda")
 
-    monkeypatch.setenv("MAMBA_MIXER_INJECT_SKIP_TILE", "1")
-    gpu_fwd(d, workspace=ws)
+    M.mamba_mixer_set_fault_injection(1)   # read by the host when it builds the launch
+    try:
+        gpu_fwd(d, workspace=ws)
+    finally:
+        M.mamba_mixer_set_fault_injection(-1)
     with pytest.raises(M.MambaError) as err:
         M.mamba_mixer_check(ws)
     assert err.value.code == 6 and "bounded wait" in str(err.value)
     M.mamba_mixer_check(ws)            # the check cleared the status word
 
-    monkeypatch.delenv("MAMBA_MIXER_INJECT_SKIP_TILE")
     y, h, cs = gpu_fwd(d, workspace=ws)
     M.mamba_mixer_check(ws)            # clean run: no error
     torch.cuda.synchronize()

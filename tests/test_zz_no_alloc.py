@@ -66,7 +66,7 @@ def test_noalloc_matches_fwd_on_two_calls(w, oracle):
 
 
 @pytest.mark.gpu
-def test_noalloc_check_reports_a_bounded_wait_timeout(monkeypatch, oracle):
+def test_noalloc_check_reports_a_bounded_wait_timeout(oracle):
     """A wait that runs out (the library's test-only injection: one CTA arms a tile's barrier
     but issues none of its copies) is reported by mamba_mixer_noalloc_check, which clears
     it; the next call on the same scratch is correct again.  No GPU fault is involved."""
@@ -76,13 +76,15 @@ def test_noalloc_check_reports_a_bounded_wait_timeout(monkeypatch, oracle):
     inp = I.make_inputs(w)
     d = to_device(inp)
     M.mamba_mixer_noalloc_check()                      # start from a clear status word
-    monkeypatch.setenv("MAMBA_MIXER_INJECT_SKIP_TILE", "1")
-    _noalloc(d)
+    M.mamba_mixer_set_fault_injection(1)              # read by the host at launch
+    try:
+        _noalloc(d)
+    finally:
+        M.mamba_mixer_set_fault_injection(-1)
     with pytest.raises(M.MambaError) as err:
         M.mamba_mixer_noalloc_check()
     assert err.value.code == 6 and "bounded wait" in str(err.value)
     M.mamba_mixer_noalloc_check()                      # the check cleared it
-    monkeypatch.delenv("MAMBA_MIXER_INJECT_SKIP_TILE")
     y, h, _ = _noalloc(d)
     M.mamba_mixer_noalloc_check()
     yo, ho, _ = oracle_full(oracle, inp)
