@@ -707,22 +707,42 @@ def run_bwd(args, w: I.Workload, local_rank: int):
     flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
 
-    def call():
-        M.mamba_mixer_bwd(d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"],
-                          d["conv_w"], d["conv_b"], d["dt_bias"], d["dy"], workspace=ws, stream=stream)
+    fargs = (d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"], d["conv_w"],
+             d["conv_b"], d["dt_bias"])
+    ck = M.new_ckpt(dims, dev)
+    y = torch.empty_like(d["xp"])
+    fws = M.new_workspace(dims, dev)
 
-    for _ in range(args.warmup):
-        flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
-        call()
-    torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    with ClockSampler(local_rank) as clk:
+    def call():
+        M.mamba_mixer_bwd(*fargs, d["dy"], workspace=ws, stream=stream)
+
+    def call_ck():
+        M.mamba_mixer_bwd(*fargs, d["dy"], workspace=ws, stream=stream, h_ckpt=ck)
+
+    def fwd_plain():
+        M.mamba_mixer_fwd(*fargs, y=y, workspace=fws, stream=stream, want_states=False)
+
+    def fwd_ck():
+        M.mamba_mixer_fwd(*fargs, y=y, workspace=fws, stream=stream, want_states=False, h_ckpt=ck)
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n)]
         for e0, e1 in evs:
             flush.fill_(1.0); torch.sum(flush_rd, dim=0, out=sink)
-            e0.record(stream); call(); e1.record(stream)
+            e0.record(stream); fn(); e1.record(stream)
         torch.cuda.synchronize()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+        return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    with ClockSampler(local_rank) as clk:
+        ms = timed(call, args.steps)
+        ms_fwd = timed(fwd_plain, args.steps)
+        ms_fwd_ck = timed(fwd_ck, args.steps)      # also leaves ck for the next one
+        ms_ck = timed(call_ck, args.steps)
     nbytes = bwd_bytes(w)
     clocks = clk.summary()
     sm_hz = (clocks.get("sm_max_mhz") or 1965.0) * 1e6
@@ -743,6 +763,14 @@ def run_bwd(args, w: I.Workload, local_rank: int):
                      "unit": "GB/s", "frac": round(t_floor / (ms * 1e-3), 4),
                      "peak_source": "3 exps per (t, d, n) on MUFU (16/clk/SM) x 148 SMs",
                      "hbm_frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None},
+        "checkpointed": {
+            "what": "mamba_mixer_fwd_ckpt writes the state before every 16-step tile; "
+                    "mamba_mixer_bwd_ckpt reads them instead of recomputing them",
+            "bwd_ms": round(ms_ck, 5), "fwd_ckpt_ms": round(ms_fwd_ck, 5),
+            "fwd_plain_ms": round(ms_fwd, 5),
+            "train_step_ms": round(ms_fwd_ck + ms_ck, 5),
+            "train_step_recompute_ms": round(ms_fwd + ms, 5),
+            "ckpt_bytes": ck.numel() * 4},
         "gpu_launches": args.steps, "clocks": clocks,
     }
 

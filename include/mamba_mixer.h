@@ -221,6 +221,40 @@ MAMBA_API int mamba_mixer_bwd_packed(const mamba_dims* dims, const void* xp, con
                                      void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * Training pair that trades memory for the backward's forward sweep.  The backward needs
+ * the state at the start of every 16-step tile; mamba_mixer_bwd recomputes them (one extra
+ * pass over x', dt_raw and B), while mamba_mixer_fwd_ckpt writes them during the forward
+ * and mamba_mixer_bwd_ckpt reads them back.
+ *
+ * mamba_mixer_ckpt_bytes: bytes of that buffer, fp32 [batch, ceil(seqlen/16), d_inner,
+ * d_state] (entry k = the state before step 16k; entry 0 is zero); 0 for unsupported dims.
+ *
+ * mamba_mixer_fwd_ckpt: mamba_mixer_fwd (same inputs, outputs, workspace and errors) that
+ * also writes every entry of h_ckpt (device, 16-byte aligned, mamba_mixer_ckpt_bytes(dims)
+ * bytes, overlapping no input, output or the workspace; required unless there is nothing
+ * to compute).  Not for dims the forward's dt-projection or packed entry points need.
+ *
+ * mamba_mixer_bwd_ckpt: mamba_mixer_bwd (same arguments, outputs, workspace and errors)
+ * with h_ckpt as written by mamba_mixer_fwd_ckpt on the same inputs, read only.  Its results
+ * equal mamba_mixer_bwd's up to the rounding of the recomputed states.
+ */
+MAMBA_API size_t mamba_mixer_ckpt_bytes(const mamba_dims* dims);
+MAMBA_API int mamba_mixer_fwd_ckpt(const mamba_dims* dims, const void* xp, const void* z,
+                                   const void* dt_raw, const void* B, const void* C,
+                                   const float* A_log, const float* D, const float* conv_w,
+                                   const float* conv_b, const float* dt_bias, void* y,
+                                   float* h_out, void* conv_state_out, float* h_ckpt,
+                                   void* workspace, size_t workspace_bytes, void* cuda_stream);
+MAMBA_API int mamba_mixer_bwd_ckpt(const mamba_dims* dims, const void* xp, const void* z,
+                                   const void* dt_raw, const void* B, const void* C,
+                                   const float* A_log, const float* D, const float* conv_w,
+                                   const float* conv_b, const float* dt_bias,
+                                   const float* h_ckpt, const void* dy, float* dxp, float* dz,
+                                   float* ddt_raw, float* dB, float* dC, float* dA_log,
+                                   float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
+                                   void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * One decode step: one token for each of `batch` sequences (dims->seqlen must be 1) on a
  * cached state.  Inputs: xp, z, dt_raw [batch, 1, d_inner]; B, C [batch, 1, d_state];
  * the parameters as for mamba_mixer_fwd; h_in [batch, d_inner, d_state] fp32 and

@@ -70,6 +70,7 @@ struct BwdParams {
   float* dconv_b;        // may be null
   float* ddt_bias;
   float* ws_h;           // [batch, tiles, d_inner, N] tile start states
+  int states_given;      // 1: ws_h already holds them (the forward's checkpoints), no forward sweep
   int64_t L, Di;
   int ntiles;            // 16-step tiles over the whole sequence
   // time chunks (as the forward's plan; chunk_len a multiple of the tile length)
@@ -197,7 +198,7 @@ __device__ __forceinline__ float sigmoid_(float v) {
 }
 
 template <int N, typename IO, bool kPrecise, bool kAdj, bool kExt>
-__global__ void __launch_bounds__(kBwdThreads)
+__global__ void __launch_bounds__(kBwdThreads, 3)   // 3 CTAs per SM: 70 KB of shared memory each
 bwd_kernel(const BwdArgs<kExt> p) {
   using M = Math<kPrecise>;
   using Sm = BwdSmem<N, IO>;
@@ -405,8 +406,9 @@ bwd_kernel(const BwdArgs<kExt> p) {
       for (int s = 0; s < kS; ++s) o[s] = lam[s];
     }
   } else {
-    // ---- forward sweep: tile start states, from the state carried into this chunk
-    {
+    // ---- forward sweep: tile start states, from the state carried into this chunk (not
+    // needed when the forward left them: mamba_mixer_fwd_ckpt)
+    if (!p.states_given) {
       float h[kS];
 #pragma unroll
       for (int s = 0; s < kS; ++s) h[s] = 0.0f;
@@ -522,7 +524,7 @@ bwd_kernel(const BwdArgs<kExt> p) {
       // reduce-scatter over the channel's 4 lanes), dB and dC to the tile's sums
       float ht[kS];
       lds_states<kS>(hsa + uint32_t((cnt - 1) * kBwdThreads * kS * 4), ht);
-#pragma unroll 2
+#pragma unroll 4
       for (int i = cnt - 1; i >= 0; --i) {
         const bool m1 = !((bits >> (i + 4)) & 1u);           // no reset at t
         const float4 q = sc[i * kBwdCh + cl];

@@ -84,6 +84,8 @@ struct Params {
   int* unit_counter;        // kChained
   int* carry_flag;          // kChained: [tiles][kGroupWarps]
   float* carry;             // kChained: [tiles][kCh][N]
+  float* ckpt;              // kCkpt: the state at the start of every 16-step tile,
+                            // fp32 [batch, ceil(L/16), d_inner, N]
   int64_t L, Di;
   int64_t chunk_len;        // multiple of kTileT
   int nchunks, ntd, batch;
@@ -167,7 +169,7 @@ __device__ __forceinline__ uint64_t tile_resets(const int32_t* seq, int64_t tt, 
          (uint64_t(__ballot_sync(0xffffffffu, r_hi)) << 32);
 }
 
-template <int N, bool kExt, int G, bool kChained, int KB = 0>
+template <int N, bool kExt, int G, bool kChained, int KB = 0, bool kCkpt = false>
 __global__ void __launch_bounds__(threads<G, KB>(), G == 1 ? 3 : 1)
 fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
             const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_B,
@@ -474,6 +476,19 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
 #pragma unroll
   for (int pp = 0; pp < kP; ++pp) hin[pp] = hp[pp];
 
+  // the state entering the 16-step tile that starts at step t < L, when checkpoints are asked
+  [[maybe_unused]] auto put_ckpt = [&](int64_t t, const f32x2* hv) {
+    if (kCkpt && active && t < p.L) {
+      float v[kS];
+#pragma unroll
+      for (int pp = 0; pp < kP; ++pp) upk2(hv[pp], v[2 * pp], v[2 * pp + 1]);
+      float* o = p.ckpt + ((int64_t(b) * ((p.L + 15) / 16) + t / 16) * p.Di + d) * N + j * kS;
+      if constexpr (kS == 4) __stcg(reinterpret_cast<float4*>(o), make_float4(v[0], v[1], v[2], v[3]));
+      else __stcg(reinterpret_cast<float2*>(o), make_float2(v[0], v[1]));
+    }
+  };
+  if (kCkpt && G > 1 && c == 0 && g == 0) put_ckpt(0, hp);
+
   const uint32_t xch = sb + uint32_t(S::kXchOff + warp * S::kXchWarp);
   __nv_bfloat16* yrow = p.y + (int64_t(b) * p.L + t_begin + j) * p.Di + d;
   const int col = cl * 2;
@@ -640,6 +655,9 @@ fwd2_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CU
       f32x2 endp[kP];
 #pragma unroll
       for (int pp = 0; pp < kP; ++pp) endp[pp] = fma2(Pp[pp], hin[pp], hp[pp]);
+      // checkpoints (when asked): the blocks that end on a 16-step boundary leave the state
+      // entering the next 16-step tile
+      if (kCkpt && (R * (g + 1)) % 16 == 0) put_ckpt(tt + R * (g + 1), endp);
       if (g < G - 1 || k < ntiles - 1) {
         const uint32_t da = sb + uint32_t(S::kSlotOff + ((g * kGroupWarps + w4) * 32 + lane) * kS * 4);
         float e[kS];

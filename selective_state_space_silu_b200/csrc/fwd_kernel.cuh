@@ -64,6 +64,8 @@ struct FwdParams {
   void* cs_out;         // may be null
   float* ws_P;          // [batch, nchunks-1, d_inner, N]
   float* ws_H;          // [batch, nchunks-1, d_inner, N]
+  float* ckpt;          // kCkpt: the state at the start of every 16-step tile,
+                        // fp32 [batch, ceil(L/16), d_inner, N] (main pass only)
   int* status;          // device status word
   int64_t L, Di;
   int64_t chunk_len;    // multiple of kTileT
@@ -197,7 +199,7 @@ __device__ __forceinline__ void sts_f32x4(uint32_t a, float x, float y, float z,
                "f"(w) : "memory");
 }
 
-template <int N, typename IO, bool kPrecise, bool kPrepass, bool kExt>
+template <int N, typename IO, bool kPrecise, bool kPrepass, bool kExt, bool kCkpt = false>
 __global__ void __launch_bounds__(kFwdThreads)
 fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
            const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_B,
@@ -483,6 +485,27 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
     Pp[pp] = pk2(1.0f, 1.0f);
   }
 
+  // checkpoints (main pass, when asked): the state entering the 16-step tile that starts at
+  // step t < L; chunk 0 writes the row's first, every chunk those that its own steps end
+  [[maybe_unused]] auto put_ckpt = [&](int64_t t) {
+    if constexpr (kCkpt && !kPrepass) {
+      if (active && t < p.L) {
+        float v[kS];
+        if constexpr (!kPrecise) {
+#pragma unroll
+          for (int pp = 0; pp < kS / 2; ++pp) upk2(hp[pp], v[2 * pp], v[2 * pp + 1]);
+        } else {
+#pragma unroll
+          for (int s = 0; s < kS; ++s) v[s] = h[s];
+        }
+        float* o = p.ckpt + ((int64_t(b) * ((p.L + 15) / 16) + t / 16) * p.Di + d) * N + j * kS;
+        if constexpr (kS == 4) __stcg(reinterpret_cast<float4*>(o), make_float4(v[0], v[1], v[2], v[3]));
+        else __stcg(reinterpret_cast<float2*>(o), make_float2(v[0], v[1]));
+      }
+    }
+  };
+  if (c == 0) put_ckpt(0);
+
   IO* yrow = static_cast<IO*>(p.y) + (int64_t(b) * p.L + t_begin + j) * p.Di + d;
   bool ok = true;
   for (int k = 0; k < ntiles; ++k) {
@@ -578,6 +601,7 @@ fwd_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUt
         const float skip = lds_f32(rec + sc_unit(q, cl, 2) + 4 * j);
         const float sz = lds_f32(rec + sc_unit(q, cl, 3) + 4 * j);
         if (4 * q < rem && active) yrow[int64_t(4 * q) * p.Di] = IOT<IO>::from_f((kp + skip) * sz);
+        if ((q & 3) == 3) put_ckpt(t_begin + int64_t(k) * kTileT + 4 * q + 4);
       }
     }
     yrow += int64_t(kTileT) * p.Di;

@@ -311,11 +311,11 @@ struct FwdMaps {
   CUtensorMap w;    // the fused dt projection's W_dt (unused otherwise)
 };
 
-template <int N, bool kExt, int G, bool kChained, int KB>
+template <int N, bool kExt, int G, bool kChained, int KB, bool kCkpt = false>
 cudaError_t launch_fwd2_kernel(const FwdMaps& m, const mm::f2::Params& a, dim3 grid,
                                cudaStream_t st) {
   using S = mm::f2::Smem<N, G, KB>;
-  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained, KB>;
+  auto kern = mm::f2::fwd2_kernel<N, kExt, G, kChained, KB, kCkpt>;
   static bool attr_set = false;
   const cudaError_t e = set_smem_once(kern, S::kDynamic, attr_set);
   if (e != cudaSuccess) return e;
@@ -334,6 +334,9 @@ cudaError_t launch_fwd2(const FwdMaps& m, const mm::f2::Params& a, const FwdPlan
     if (f.G == 1) return launch_fwd2_kernel<N, false, 1, false, KB>(m, a, tiles, st);
     return f.chained ? launch_fwd2_kernel<N, false, 4, true, KB>(m, a, units, st)
                      : launch_fwd2_kernel<N, false, 4, false, KB>(m, a, tiles, st);
+  } else if (!kExt && a.ckpt) {
+    return f.chained ? launch_fwd2_kernel<N, false, 4, true, 0, true>(m, a, units, st)
+                     : launch_fwd2_kernel<N, false, 4, false, 0, true>(m, a, tiles, st);
   } else {
     return f.chained ? launch_fwd2_kernel<N, kExt, 4, true, 0>(m, a, units, st)
                      : launch_fwd2_kernel<N, kExt, 4, false, 0>(m, a, tiles, st);
@@ -342,11 +345,11 @@ cudaError_t launch_fwd2(const FwdMaps& m, const mm::f2::Params& a, const FwdPlan
 
 
 
-template <int N, typename IO, bool P, bool kPre, bool kExt>
+template <int N, typename IO, bool P, bool kPre, bool kExt, bool kCkpt = false>
 cudaError_t launch_fwd_kernel(const FwdMaps& m, const mm::FwdArgs<kExt>& a, dim3 grid,
                               cudaStream_t st) {
   using S = mm::FwdSmem<IO, N>;
-  auto kern = mm::fwd_kernel<N, IO, P, kPre, kExt>;
+  auto kern = mm::fwd_kernel<N, IO, P, kPre, kExt, kCkpt>;
   static bool attr_set = false;
   const cudaError_t e = set_smem_once(kern, S::kDynamic, attr_set);
   if (e != cudaSuccess) return e;
@@ -363,6 +366,9 @@ cudaError_t launch_fwd(const FwdMaps& m, const mm::FwdArgs<kExt>& a, int64_t bat
         m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks - 1)), st);
     if (e != cudaSuccess) return e;
   }
+  if (!kExt && a.ckpt)
+    return launch_fwd_kernel<N, IO, P, false, false, true>(
+        m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks)), st);
   return launch_fwd_kernel<N, IO, P, false, kExt>(
       m, a, dim3(gx, unsigned(batch), unsigned(a.nchunks)), st);
 }
@@ -481,6 +487,12 @@ size_t mamba_mixer_fwd_workspace_bytes(const mamba_dims* dims) {
 
 namespace {
 
+// Bytes of the state checkpoints: fp32 [batch, ceil(L/16), d_inner, d_state].
+size_t ckpt_bytes_for(const mamba_dims* d) {
+  return size_t(d->batch) * size_t((d->seqlen + 15) / 16) * size_t(d->d_inner) *
+         size_t(d->d_state) * sizeof(float);
+}
+
 // The forward behind mamba_mixer_fwd and mamba_mixer_fwd_packed: seq_idx, h_in and
 // conv_state_in are null for the former.
 // dt_rank > 0: the dt projection is fused (dt_raw is NULL; dt_low [batch, L, dt_rank] and
@@ -491,12 +503,13 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
                const int32_t* seq_idx, const float* h_in, const void* conv_state_in, void* y,
                float* h_out, void* conv_state_out, void* workspace, size_t workspace_bytes,
                void* cuda_stream, const void* dt_low = nullptr, const void* W_dt = nullptr,
-               int64_t dt_rank = 0) {
+               int64_t dt_rank = 0, float* ckpt = nullptr) {
   Sizes s;
   int rc = check_dims(dims, &s);
   if (rc) return rc;
   const bool act = s.act > 0, bc = s.bc > 0;
   const bool dtproj = dt_rank > 0;
+  if ((rc = check_ptr(ckpt, "h_ckpt", false, 16))) return rc;
   if (dtproj) {
     if (dims->io_dtype != MAMBA_BF16)
       return fail(MAMBA_ERR_UNSUPPORTED, "the fused dt projection takes bf16 I/O only");
@@ -535,7 +548,8 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
                       {W_dt, dtproj ? size_t(Di) * size_t(dt_rank) * 2 : 0, "W_dt"}};
   const Span outs[] = {{y, size_t(s.act) * s.esize, "y"},
                        {h_out, size_t(s.state) * 4, "h_out"},
-                       {conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"}};
+                       {conv_state_out, size_t(s.cstate) * s.esize, "conv_state_out"},
+                       {ckpt, ckpt ? ckpt_bytes_for(dims) : 0, "h_ckpt"}};
   const FwdPlan fplan = make_fwd_plan(dims, dtproj);
   const Plan& plan = fplan.p;
   const size_t need = fwd_workspace_for(dims, fplan);
@@ -598,6 +612,7 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
     a2.cs_out = static_cast<__nv_bfloat16*>(conv_state_out);
     a2.status = static_cast<int*>(workspace);
     a2.seq_idx = seq_idx;
+    a2.ckpt = ckpt;
     a2.h_in = h_in;
     a2.cs_in = static_cast<const __nv_bfloat16*>(conv_state_in);
     a2.L = dims->seqlen; a2.Di = Di;
@@ -636,6 +651,7 @@ int fwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   mm::FwdParams a{};
   a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
   a.y = y; a.h_out = h_out; a.cs_out = conv_state_out;
+  a.ckpt = ckpt;
   a.status = static_cast<int*>(workspace);
   a.L = dims->seqlen; a.Di = Di;
   a.nchunks = plan.nchunks; a.chunk_len = plan.chunk_len;
@@ -699,6 +715,25 @@ int mamba_mixer_fwd_dtproj(const mamba_dims* dims, int64_t dt_rank, const void* 
   return fwd_common(dims, xp, z, nullptr, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
                     nullptr, nullptr, y, h_out, conv_state_out, workspace, workspace_bytes,
                     cuda_stream, dt_low, W_dt, dt_rank);
+}
+
+size_t mamba_mixer_ckpt_bytes(const mamba_dims* dims) {
+  Sizes s;
+  if (!dims || check_dims(dims, &s) != MAMBA_OK) return 0;
+  return ckpt_bytes_for(dims);
+}
+
+int mamba_mixer_fwd_ckpt(const mamba_dims* dims, const void* xp, const void* z,
+                         const void* dt_raw, const void* B, const void* C, const float* A_log,
+                         const float* D, const float* conv_w, const float* conv_b,
+                         const float* dt_bias, void* y, float* h_out, void* conv_state_out,
+                         float* h_ckpt, void* workspace, size_t workspace_bytes,
+                         void* cuda_stream) {
+  if (!h_ckpt && dims && dims->batch > 0 && dims->seqlen > 0 && dims->d_inner > 0)
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "h_ckpt is NULL");
+  return fwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
+                    nullptr, nullptr, y, h_out, conv_state_out, workspace, workspace_bytes,
+                    cuda_stream, nullptr, nullptr, 0, h_ckpt);
 }
 
 int mamba_mixer_fwd_launches(const mamba_dims* dims) {
@@ -772,11 +807,12 @@ int bwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
                const void* dy, float* dxp, float* dz, float* ddt_raw, float* dB, float* dC,
                float* dA_log, float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
                float* dh_in, float* dconv_state_in, void* workspace, size_t workspace_bytes,
-               void* cuda_stream) {
+               void* cuda_stream, const float* ckpt = nullptr) {
   Sizes s;
   int rc = check_dims(dims, &s);
   if (rc) return rc;
   const bool act = s.act > 0, bc = s.bc > 0, par = dims->d_inner > 0;
+  if ((rc = check_ptr(ckpt, "h_ckpt", false, 16))) return rc;
   if ((rc = check_ptr(xp, "xp", act, 16)) || (rc = check_ptr(z, "z", act, 16)) ||
       (rc = check_ptr(dt_raw, "dt_raw", act, 16)) || (rc = check_ptr(B, "B", bc, 16)) ||
       (rc = check_ptr(C, "C", bc, 16)) || (rc = check_ptr(dy, "dy", act, 16)) ||
@@ -804,7 +840,8 @@ int bwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
                       {dt_bias, size_t(Di) * 4, "dt_bias"},
                       {seq_idx, size_t(dims->batch) * size_t(dims->seqlen) * 4, "seq_idx"},
                       {h_in, size_t(s.state) * 4, "h_in"},
-                      {conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"}};
+                      {conv_state_in, size_t(s.cstate) * s.esize, "conv_state_in"},
+                      {ckpt, ckpt ? ckpt_bytes_for(dims) : 0, "h_ckpt"}};
   const Span outs[] = {{dxp, size_t(s.act) * 4, "dxp"},      {dz, size_t(s.act) * 4, "dz"},
                        {ddt_raw, size_t(s.act) * 4, "ddt_raw"}, {dB, size_t(s.bc) * 4, "dB"},
                        {dC, size_t(s.bc) * 4, "dC"},          {dA_log, size_t(Di * N) * 4, "dA_log"},
@@ -859,7 +896,8 @@ int bwd_common(const mamba_dims* dims, const void* xp, const void* z, const void
   a.A_log = A_log; a.D = D; a.conv_w = conv_w; a.conv_b = conv_b; a.dt_bias = dt_bias;
   a.dxp = dxp; a.dz = dz; a.ddt = ddt_raw; a.dB = dB; a.dC = dC; a.dA_log = dA_log; a.dD = dD;
   a.dconv_w = dconv_w; a.dconv_b = dconv_b; a.ddt_bias = ddt_bias;
-  a.ws_h = reinterpret_cast<float*>(wsb + lay.states);
+  a.ws_h = ckpt ? const_cast<float*>(ckpt) : reinterpret_cast<float*>(wsb + lay.states);
+  a.states_given = ckpt ? 1 : 0;
   a.L = dims->seqlen; a.Di = Di;
   a.ntiles = int((dims->seqlen + mm::kBwdT - 1) / mm::kBwdT);
   a.chunk_len = plan.chunk_len;
@@ -919,6 +957,20 @@ int mamba_mixer_bwd(const mamba_dims* dims, const void* xp, const void* z, const
   return bwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
                     nullptr, nullptr, dy, dxp, dz, ddt_raw, dB, dC, dA_log, dD, dconv_w, dconv_b,
                     ddt_bias, nullptr, nullptr, workspace, workspace_bytes, cuda_stream);
+}
+
+int mamba_mixer_bwd_ckpt(const mamba_dims* dims, const void* xp, const void* z,
+                         const void* dt_raw, const void* B, const void* C, const float* A_log,
+                         const float* D, const float* conv_w, const float* conv_b,
+                         const float* dt_bias, const float* h_ckpt, const void* dy, float* dxp,
+                         float* dz, float* ddt_raw, float* dB, float* dC, float* dA_log,
+                         float* dD, float* dconv_w, float* dconv_b, float* ddt_bias,
+                         void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (!h_ckpt && dims && dims->batch > 0 && dims->seqlen > 0 && dims->d_inner > 0)
+    return fail(MAMBA_ERR_INVALID_ARGUMENT, "h_ckpt is NULL");
+  return bwd_common(dims, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, nullptr,
+                    nullptr, nullptr, dy, dxp, dz, ddt_raw, dB, dC, dA_log, dD, dconv_w, dconv_b,
+                    ddt_bias, nullptr, nullptr, workspace, workspace_bytes, cuda_stream, h_ckpt);
 }
 
 int mamba_mixer_bwd_packed(const mamba_dims* dims, const void* xp, const void* z,

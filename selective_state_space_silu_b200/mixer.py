@@ -27,7 +27,8 @@ EXPORTS = ("mamba_mixer_fwd_workspace_bytes", "mamba_mixer_fwd_launches", "mamba
            "mamba_mixer_fwd_packed", "mamba_mixer_bwd_workspace_bytes", "mamba_mixer_bwd",
            "mamba_mixer_bwd_packed",
            "mamba_mixer_step", "mamba_mixer_step_check", "mamba_mixer_check",
-           "mamba_mixer_set_fault_injection",
+           "mamba_mixer_set_fault_injection", "mamba_mixer_ckpt_bytes", "mamba_mixer_fwd_ckpt",
+           "mamba_mixer_bwd_ckpt",
            "mamba_mixer_fwd_plan", "mamba_mixer_fwd_dtproj",
            "mamba_mixer_fwd_noalloc",
            "mamba_mixer_noalloc_check", "mamba_last_error", "mamba_version")
@@ -69,6 +70,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.mamba_mixer_check.argtypes = [vp, vp]
     lib.mamba_mixer_set_fault_injection.restype = None
     lib.mamba_mixer_set_fault_injection.argtypes = [i]
+    lib.mamba_mixer_ckpt_bytes.restype = sz
+    lib.mamba_mixer_ckpt_bytes.argtypes = [P]
+    lib.mamba_mixer_fwd_ckpt.restype = i
+    lib.mamba_mixer_fwd_ckpt.argtypes = [P] + [vp] * 14 + [vp, sz, vp]
+    lib.mamba_mixer_bwd_ckpt.restype = i
+    lib.mamba_mixer_bwd_ckpt.argtypes = [P] + [vp] * 12 + [vp] * 10 + [vp, sz, vp]
     lib.mamba_mixer_fwd.restype = i
     lib.mamba_mixer_fwd.argtypes = [P] + [vp] * 13 + [vp, sz, vp]
     lib.mamba_mixer_fwd_packed.restype = i
@@ -167,13 +174,15 @@ def mamba_mixer_set_fault_injection(tile: int) -> None:
 
 def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
                     y=None, h_out=None, conv_state_out=None, workspace=None,
-                    stream=None, want_states: bool = True
+                    stream=None, want_states: bool = True, h_ckpt=None
                     ) -> Tuple[torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
     """Fused forward (conv + SiLU, softplus, selective scan, gate) from a zero state.
 
     Shapes: xp, z, dt_raw [batch, L, d_inner]; B, C [batch, L, d_state]; A_log
     [d_inner, d_state]; D, dt_bias, conv_b [d_inner]; conv_w [d_inner, 4].  Returns
-    (y, h_out, conv_state_out).
+    (y, h_out, conv_state_out).  With ``h_ckpt`` (fp32 [batch, ceil(L/16), d_inner,
+    d_state], see ``new_ckpt``) it also writes the state before every 16-step tile
+    (mamba_mixer_fwd_ckpt), which ``mamba_mixer_bwd(..., h_ckpt=)`` then reads.
     """
     lib = load_library()
     dev = xp.device
@@ -193,16 +202,27 @@ def mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
         workspace = new_workspace(dims, dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     f32 = torch.float32
-    rc = lib.mamba_mixer_fwd(
-        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
-        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
-        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
-        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
-        _ptr(y, "y", iot, dev), _ptr(h_out, "h_out", f32, dev),
-        _ptr(conv_state_out, "conv_state_out", iot, dev),
-        _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
+    args = [ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+            _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+            _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev),
+            _ptr(conv_w, "conv_w", f32, dev), _ptr(conv_b, "conv_b", f32, dev),
+            _ptr(dt_bias, "dt_bias", f32, dev), _ptr(y, "y", iot, dev),
+            _ptr(h_out, "h_out", f32, dev), _ptr(conv_state_out, "conv_state_out", iot, dev)]
+    tail = [_ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev)]
+    if h_ckpt is None:
+        rc = lib.mamba_mixer_fwd(*args, *tail)
+    else:
+        rc = lib.mamba_mixer_fwd_ckpt(*args, _ptr(h_ckpt, "h_ckpt", f32, dev), *tail)
     _check(rc)
     return y, h_out, conv_state_out
+
+
+def new_ckpt(dims: mamba_dims, device) -> torch.Tensor:
+    """The state checkpoints of mamba_mixer_fwd_ckpt for ``dims``: fp32 [batch,
+    ceil(L/16), d_inner, d_state]."""
+    t16 = (dims.seqlen + 15) // 16
+    return torch.empty((dims.batch, t16, dims.d_inner, dims.d_state), dtype=torch.float32,
+                       device=device)
 
 
 def mamba_mixer_fwd_packed(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
@@ -252,9 +272,11 @@ BWD_OUTPUTS = ("dxp", "dz", "ddt_raw", "dB", "dC", "dA_log", "dD", "dconv_w", "d
 
 
 def mamba_mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, *,
-                    workspace=None, stream=None) -> dict:
+                    workspace=None, stream=None, h_ckpt=None) -> dict:
     """Gradients of sum(dy * y) for mamba_mixer_fwd, all fp32; returns a dict keyed by
-    BWD_OUTPUTS (dconv_b is None when conv_b is None)."""
+    BWD_OUTPUTS (dconv_b is None when conv_b is None).  With ``h_ckpt`` (written by
+    mamba_mixer_fwd(..., h_ckpt=) on the same inputs) the backward reads the tile states
+    instead of recomputing them (mamba_mixer_bwd_ckpt)."""
     lib = load_library()
     dev = xp.device
     io = _io_code(xp)
@@ -272,13 +294,17 @@ def mamba_mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, dy, 
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    rc = lib.mamba_mixer_bwd(
-        ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
-        _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
-        _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev), _ptr(conv_w, "conv_w", f32, dev),
-        _ptr(conv_b, "conv_b", f32, dev), _ptr(dt_bias, "dt_bias", f32, dev),
-        _ptr(dy, "dy", iot, dev), *[_ptr(g[k], k, f32, dev) for k in BWD_OUTPUTS],
-        _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev))
+    ins = [ctypes.byref(dims), _ptr(xp, "xp", iot, dev), _ptr(z, "z", iot, dev),
+           _ptr(dt_raw, "dt_raw", iot, dev), _ptr(B, "B", iot, dev), _ptr(C, "C", iot, dev),
+           _ptr(A_log, "A_log", f32, dev), _ptr(D, "D", f32, dev),
+           _ptr(conv_w, "conv_w", f32, dev), _ptr(conv_b, "conv_b", f32, dev),
+           _ptr(dt_bias, "dt_bias", f32, dev)]
+    rest = [_ptr(dy, "dy", iot, dev), *[_ptr(g[k], k, f32, dev) for k in BWD_OUTPUTS],
+            _ptr(workspace, "workspace", None, dev), ws_bytes, _stream_handle(stream, dev)]
+    if h_ckpt is None:
+        rc = lib.mamba_mixer_bwd(*ins, *rest)
+    else:
+        rc = lib.mamba_mixer_bwd_ckpt(*ins, _ptr(h_ckpt, "h_ckpt", f32, dev), *rest)
     _check(rc)
     return g
 
@@ -483,27 +509,38 @@ def mamba_mixer_noalloc_check(stream=None, device=None) -> None:
 
 class MambaMixerFunction(torch.autograd.Function):
     """The fused forward as a differentiable op: forward = mamba_mixer_fwd (from a zero
-    state), backward = mamba_mixer_bwd; gradients come back in each input's dtype."""
+    state), backward = mamba_mixer_bwd; gradients come back in each input's dtype.  With
+    checkpoint_states the forward also keeps the state before every 16-step tile (fp32,
+    4 * d_state bytes per token and channel / 16) and the backward reads them instead of
+    recomputing them."""
 
     @staticmethod
-    def forward(ctx, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias):
+    def forward(ctx, xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, checkpoint_states):
         xp, z, dt_raw, B, C = (t.contiguous() for t in (xp, z, dt_raw, B, C))
+        ck = None
+        if checkpoint_states:
+            Bt, L, Di = xp.shape
+            ck = new_ckpt(make_dims(Bt, L, Di, A_log.shape[1], conv_w.shape[1], _io_code(xp)),
+                          xp.device)
         y, _, _ = mamba_mixer_fwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
-                                  want_states=False)
-        ctx.save_for_backward(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias)
+                                  want_states=False, h_ckpt=ck)
+        ctx.save_for_backward(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, ck)
         return y
 
     @staticmethod
     def backward(ctx, dy):
-        xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias = ctx.saved_tensors
+        xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, ck = ctx.saved_tensors
         g = mamba_mixer_bwd(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
-                            dy.to(xp.dtype).contiguous())
+                            dy.to(xp.dtype).contiguous(), h_ckpt=ck)
         as_ = lambda k, ref: None if g[k] is None else g[k].to(ref.dtype)
         return (as_("dxp", xp), as_("dz", z), as_("ddt_raw", dt_raw), as_("dB", B), as_("dC", C),
                 as_("dA_log", A_log), as_("dD", D), as_("dconv_w", conv_w),
-                None if conv_b is None else as_("dconv_b", conv_b), as_("ddt_bias", dt_bias))
+                None if conv_b is None else as_("dconv_b", conv_b), as_("ddt_bias", dt_bias),
+                None)
 
 
-def mamba_mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias):
+def mamba_mixer(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias, *,
+                checkpoint_states: bool = False):
     """y = the fused mixer forward, differentiable with respect to every input."""
-    return MambaMixerFunction.apply(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias)
+    return MambaMixerFunction.apply(xp, z, dt_raw, B, C, A_log, D, conv_w, conv_b, dt_bias,
+                                    checkpoint_states)

@@ -11,7 +11,8 @@ import torch
 from selective_state_space_silu_b200 import inputs as I
 from selective_state_space_silu_b200 import mixer as M
 from tests.gpu_util import host, to_device
-from tests.tolerances import assert_close_grad
+from tests.gpu_util import oracle_full
+from tests.tolerances import assert_close, assert_close_grad
 
 pytestmark = pytest.mark.gpu
 
@@ -197,3 +198,71 @@ def test_autograd_function_matches_oracle(oracle, io):
         # bf16 gradients of activations carry bf16 rounding on top of the fp32 result
         assert_close_grad(host(leaves[k].grad), go["d" + k], io,
                           f"autograd {io} {k}")
+
+
+# ---- the training pair with state checkpoints (mamba_mixer_fwd_ckpt / mamba_mixer_bwd_ckpt)
+
+@pytest.mark.parametrize("Bt,L,Di,N,io", [
+    (12, 200, 1024, 16, I.BF16),   # 384 channel tiles: the prep/scan forward kernel
+    (2, 4100, 96, 16, I.BF16),     # few tiles: four time groups, chained chunks, ragged tail
+    (3, 300, 64, 8, I.BF16),       # four time groups, one chunk, d_state 8
+    (2, 77, 72, 16, I.F32),        # fp32, ragged time and channel tails
+    (1, 2600, 40, 16, I.F32),      # fp32 with a chunk-state pass (time chunks)
+])
+def test_checkpointed_backward_matches_oracle(oracle, Bt, L, Di, N, io):
+    """The forward that writes the state before every 16-step tile gives the same y as the
+    plain forward (bit for bit), its checkpoints start from zero and match the oracle's
+    state after each 16-step prefix, and the backward that reads them matches the oracle
+    in the gradient tolerance."""
+    w, inp = _case(Bt, L, Di, N, io, 3400 + L + Di)
+    d = to_device(inp)
+    args = (d["xp"], d["z"], d["dt_raw"], d["B"], d["C"], d["A_log"], d["D"], d["conv_w"],
+            d.get("conv_b"), d["dt_bias"])
+    dims = M.make_dims(Bt, L, Di, N, 4, M.MAMBA_BF16 if io == I.BF16 else M.MAMBA_F32)
+    ck = M.new_ckpt(dims, d["xp"].device)
+    assert ck.numel() * 4 == M.load_library().mamba_mixer_ckpt_bytes(__import__("ctypes").byref(dims))
+    ck.fill_(float("nan"))                   # every entry must be written
+    y_ck, h_ck, _ = M.mamba_mixer_fwd(*args, h_ckpt=ck)
+    y, h, _ = M.mamba_mixer_fwd(*args)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host(y_ck), host(y))
+    np.testing.assert_array_equal(host(h_ck), host(h))
+    ckh = host(ck)
+    assert np.isfinite(ckh).all()
+    assert (ckh[:, 0] == 0).all()
+    # the oracle's state after 16k steps, for a few k (prefix runs)
+    rng = np.random.default_rng(L)
+    t16 = (L + 15) // 16
+    for k in sorted(set([1, t16 - 1] + [int(v) for v in rng.integers(1, t16, 2)])):
+        if k < 1 or k >= t16:
+            continue
+        pre = {key: (np.ascontiguousarray(v[:, :16 * k]) if key in ("xp", "z", "dt_raw", "B", "C")
+                     else v) for key, v in inp.items() if key != "dy"}
+        _, ho, _ = oracle_full(oracle, pre)
+        assert_close(ckh[:, k], ho, io, f"checkpoint {k} (state after {16 * k} steps)")
+    g = M.mamba_mixer_bwd(*args, d["dy"], h_ckpt=ck)
+    torch.cuda.synchronize()
+    g = {k: (None if v is None else host(v)) for k, v in g.items()}
+    _compare(g, _oracle(oracle, inp), io, f"checkpointed {Bt}x{L}x{Di} N{N} {io}")
+
+
+def test_checkpointed_autograd_matches_recompute(oracle):
+    """MambaMixerFunction with checkpoint_states gives the recomputing path's gradients in
+    the gradient tolerance of each other and of the oracle."""
+    w, inp = _case(2, 300, 256, 16, I.BF16, 3500)
+    d = to_device(inp)
+    outs = []
+    for ckpt in (False, True):
+        leaves = {k: d[k].clone().requires_grad_(d[k].dtype.is_floating_point)
+                  for k in ("xp", "z", "dt_raw", "B", "C", "A_log", "D", "conv_w", "conv_b", "dt_bias")}
+        y = M.mamba_mixer(*(leaves[k] for k in ("xp", "z", "dt_raw", "B", "C", "A_log", "D",
+                                                "conv_w", "conv_b", "dt_bias")),
+                          checkpoint_states=ckpt)
+        y.backward(d["dy"])
+        outs.append({k: host(v.grad.float()) for k, v in leaves.items()})
+    go = _oracle(oracle, inp)
+    names = {"xp": "dxp", "z": "dz", "dt_raw": "ddt_raw", "B": "dB", "C": "dC", "A_log": "dA_log",
+             "D": "dD", "conv_w": "dconv_w", "conv_b": "dconv_b", "dt_bias": "ddt_bias"}
+    for k, gk in names.items():
+        assert_close_grad(outs[1][k], go[gk], I.BF16, f"checkpointed autograd {k}")
+        assert_close_grad(outs[1][k], outs[0][k], I.BF16, f"checkpointed vs recompute {k}")
