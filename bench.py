@@ -531,6 +531,13 @@ def measure_extra(w: I.Workload, dev, calls: int, peaks: dict, n_chans: int) -> 
     h = torch.empty((Bt, Di, N), dtype=torch.float32, device=dev)
     cs = torch.empty((Bt, Di, 3), dtype=iot, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    flush_rd = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def flush_l2():   # as in the headline loop: a write, then a read, so L2 holds clean lines
+        flush.fill_(1.0)
+        torch.sum(flush_rd, dim=0, out=sink)
+
     if w.decode:
         kernel = "mamba_mixer_step"
         nbytes = step_bytes(w)
@@ -549,14 +556,14 @@ def measure_extra(w: I.Workload, dev, calls: int, peaks: dict, n_chans: int) -> 
                               d["conv_w"], d["conv_b"], d["dt_bias"], y=y, h_out=h,
                               conv_state_out=cs, workspace=ws, stream=stream)
     for _ in range(5):
-        flush.fill_(1.0)
+        flush_l2()
         call()
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(calls)]
     with ClockSampler(dev.index or 0) as clk:
         for a, b in evs:
-            flush.fill_(1.0)
+            flush_l2()
             a.record(stream)
             call()
             b.record(stream)
@@ -1157,7 +1164,7 @@ def main():
                 dev = torch.device("cuda", local_rank)
                 peaks = measured_peaks()
                 res["m130"] = measure_extra(I.WORKLOADS["m130"], dev, 200, peaks, 96)
-                res["decode"] = measure_extra(I.WORKLOADS["decode"], dev, 500, peaks, 512)
+                res["decode"] = measure_extra(I.WORKLOADS["decode"], dev, 3000, peaks, 512)
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:
