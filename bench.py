@@ -1165,6 +1165,17 @@ def main():
                 peaks = measured_peaks()
                 res["m130"] = measure_extra(I.WORKLOADS["m130"], dev, 200, peaks, 96)
                 res["decode"] = measure_extra(I.WORKLOADS["decode"], dev, 3000, peaks, 512)
+                # the rows beside the forward, timed the same way (their parity is in tests/)
+                sub = argparse.Namespace(**{**vars(args), "steps": 20, "warmup": 3})
+                bw = run_bwd(sub, I.WORKLOADS["m130"], local_rank)
+                res["m130_backward"] = {"ms": bw["ms_per_step"], "gbs": bw["value"],
+                                        "roofline": bw["roofline"],
+                                        "checkpointed": bw["checkpointed"],
+                                        "clocks": bw["clocks"]}
+                dp = run_dtproj(sub, I.WORKLOADS["m130"], local_rank)
+                res["m130_dtproj"] = {k: dp[k] for k in ("fused_ms", "unfused_ms", "unfused_is",
+                                                         "value", "unit", "parity", "clocks")}
+                res["m130_dtproj"]["dt_rank"] = dp["config"]["dt_rank"]
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:
