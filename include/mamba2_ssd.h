@@ -97,6 +97,15 @@ MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void*
                              size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * Status of mamba2_ssd_fwd's tensor-core pass (rows without seq_idx), which waits on its own
+ * asynchronous copies and products: waits for `cuda_stream`, then reads and clears the
+ * library's status word for the Mamba2 scan (one per CUDA context).  Returns
+ * MAMBA_ERR_TIMEOUT if a call since the last check gave up on a bounded wait (about one
+ * second; its outputs are then incomplete), MAMBA_OK otherwise.  Allocates nothing.
+ */
+MAMBA_API int mamba2_ssd_check(void* cuda_stream);
+
+/*
  * One decode step of the Mamba2 scan on a cached state (niverel-mamba 0.1.0, section
  * "Autoregressive decoding": step(x_t, state) returns the output and a new state, and
  * concatenated steps equal the forward).  dims->seqlen must be 1; the layouts are those of

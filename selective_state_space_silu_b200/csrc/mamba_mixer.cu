@@ -469,6 +469,21 @@ cudaError_t launch_step(mm::StepArgs& a, cudaStream_t st) {
 namespace mm_internal {
 // Lets the other translation units of the library report through mamba_last_error.
 void set_last_error(const char* msg) { g_last_error = msg; }
+
+// 4-D map over a row-major [d3][d2][d1][d0] bf16 tensor, box (b0, b1, b2, b3), 128-byte
+// swizzle (b0 * 2 must be 128 bytes); for the other translation units' TMA copies.
+bool make_map4d_sw128(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {d0, d1, d2, d3};
+  const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  const cuuint32_t box[4] = {b0, b1, b2, b3};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 }  // namespace mm_internal
 
 extern "C" {

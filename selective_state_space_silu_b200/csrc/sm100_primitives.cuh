@@ -223,6 +223,19 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 16 consecutive 32-bit columns of this thread's TMEM lane (as tmem_ld32).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void fence_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -241,6 +254,43 @@ __device__ __forceinline__ bool tma_load_2d(uint32_t sdst, const CUtensorMap* ma
       ::"r"(sdst), "l"(gmap), "r"(smem_addr(bar)), "r"(c0), "r"(c1)
       : "memory");
   return true;
+}
+
+// 4-D tiled TMA load (no multicast), self-checked like tma_load_3d.
+__device__ __forceinline__ bool tma_load_4d(uint32_t sdst, const CUtensorMap* map, uint64_t* bar,
+                                            int c0, int c1, int c2, int c3, uint32_t dst_align,
+                                            int elem_bytes, int* status) {
+  const uint64_t gmap = reinterpret_cast<uint64_t>(map);
+  if ((sdst & (dst_align - 1)) != 0 || (gmap & 63u) != 0 || ((c0 * elem_bytes) & 15) != 0) {
+    atomicExch(status, kStatusBadCopy);
+    return false;
+  }
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+      ::"r"(sdst), "l"(gmap), "r"(smem_addr(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+  return true;
+}
+
+// Shared-memory matrix descriptor of an MN-major operand in the 128-byte-swizzle layout:
+// rows of 128 bytes hold 64 consecutive M (or N) elements of one K index, 8-row atoms of
+// 1024 bytes (one atom = 8 consecutive K), atoms along K 1024 bytes apart (stride byte
+// offset), 64-wide M/N panels `panel_bytes` apart (leading byte offset).  One K = 16 step of
+// the instruction advances the start address by 16 rows = 2048 bytes.
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t panel_bytes) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((panel_bytes >> 4) & 0x3FFFu) << 16) |
+         (uint64_t(1024 >> 4) << 32) | (uint64_t(1) << 46) | (uint64_t(2) << 61);
+}
+
+// Instruction descriptor of tcgen05.mma kind::f16 (bf16 A and B, fp32 D) with the operands'
+// major-ness: a_mn / b_mn = 1 for MN-major (bits 15, 16).
+template <int M, int N, int AMn, int BMn>
+__host__ __device__ constexpr uint32_t umma_idesc_bf16_f32_mj() {
+  static_assert(M == 64 || M == 128, "M = 64 or 128 (cta_group::1)");
+  static_assert(N % 16 == 0 && N >= 16 && N <= 256, "N a multiple of 16 up to 256");
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(AMn) << 15) | (uint32_t(BMn) << 16) |
+         (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
 // Named barrier that tolerates divergent arrival (non-.aligned form).

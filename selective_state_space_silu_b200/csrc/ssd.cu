@@ -1,18 +1,28 @@
 // mamba2_ssd_fwd: host side of the Mamba2 scan (argument checks and the launch).
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdarg>
 #include <cstdio>
 
+#include "context_symbol.h"
 #include "mamba2_ssd.h"
 #include "ssd_kernel.cuh"
 #include "ssd_step.cuh"
 #include "ssd_layer.cuh"
+#include "ssd_tc_kernel.cuh"
 
 namespace mm_internal {
 void set_last_error(const char* msg);  // mamba_mixer.cu: the message mamba_last_error returns
+bool make_map4d_sw128(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                      uint64_t d3, uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3);
 }
+
+// The Mamba2 scan's status word: its tensor-core main pass waits on its own copies and
+// products (bounded), and a wait that runs out is recorded here (one word per context;
+// mamba2_ssd_check reads and clears it).
+static __device__ __align__(256) int g_ssd_status[64];
 
 namespace {
 
@@ -62,7 +72,13 @@ struct SegPlan {
 };
 
 constexpr int64_t kSms = 148;
-constexpr int64_t kMainSlots = 2 * kSms;  // main-pass CTAs resident at once
+
+constexpr int64_t kMainSlots = 2 * kSms;  // main-pass CTAs resident at once (mma.sync pass)
+
+// Rows without document resets take the tensor-core main pass (one CTA per SM: 9 warps of
+// 168 registers; for d_state 128 also 138 KB of shared memory and 512 TMEM columns); both
+// passes use the same segment plan (at one CTA per SM its segments make about 2 waves more).
+bool use_tc(const int32_t* seq_idx) { return seq_idx == nullptr; }
 
 SegPlan seg_plan(int64_t Bt, int64_t L, int64_t H) {
   const int64_t nchunks = (L + ssd::kQ - 1) / ssd::kQ;
@@ -119,6 +135,29 @@ cudaError_t launch(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
   return launch_one<N, kGate, false, kSeq>(a, batch, a.nseg, st);
 }
 
+// The tensor-core main pass (no document resets), after the mma.sync state pass when the
+// rows are cut into segments.
+template <int N, bool kGate>
+cudaError_t launch_tc(const ssd::SsdArgs& a, int64_t batch, const CUtensorMap* maps, int* status,
+                      cudaStream_t st) {
+  using S = ssd::tc::Smem<N>;
+  if (a.nseg > 1) {
+    cudaError_t e = launch_one<N, false, true, false>(a, batch, a.nseg - 1, st);
+    if (e != cudaSuccess) return e;
+  }
+  auto kern = ssd::tc::ssd_tc_kernel<N, kGate>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               S::kDynamic);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<dim3(unsigned(a.H), unsigned(batch), unsigned(a.nseg)), ssd::tc::kThreads, S::kDynamic,
+         st>>>(maps[0], maps[1], maps[2], a, status);
+  return cudaGetLastError();
+}
+
 template <int N>
 cudaError_t launch_n(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
   if (a.z)
@@ -157,6 +196,15 @@ extern "C" MAMBA_API size_t mamba2_ssd_fwd_workspace_bytes(const mamba2_dims* di
   return ws_bytes_for(dims->batch, dims->nheads, dims->d_state, sp);
 }
 
+extern "C" MAMBA_API int mamba2_ssd_check(void* cuda_stream) {
+  void* word = nullptr;
+  char why[256];
+  if (mm_host::symbol_in_context(reinterpret_cast<const void*>(&g_ssd_status), &word,
+                                 "mamba2_ssd_check", why, sizeof(why)) != 0)
+    return ssd_fail(MAMBA_ERR_CUDA, "%s", why);
+  return mamba_mixer_check(word, cuda_stream);
+}
+
 extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, const void* dt_raw,
                                         const float* A_log, const void* B, const void* C,
                                         const float* D, const float* dt_bias, const void* z,
@@ -192,6 +240,7 @@ extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, 
     return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "y overlaps a state buffer");
   if (overlap(hout_r, hin_r) && h_out != h_in)
     return ssd_fail(MAMBA_ERR_INVALID_ARGUMENT, "h_out partially overlaps h_in");
+  const bool tc = use_tc(seq_idx) && L > 0;   // an empty sequence only passes h_in through
   const SegPlan sp = seg_plan(Bt, L, H);
   const size_t need = ws_bytes_for(Bt, H, N, sp);
   if (need > 0) {
@@ -231,7 +280,28 @@ extern "C" MAMBA_API int mamba2_ssd_fwd(const mamba2_dims* dims, const void* x, 
   }
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e;
-  e = N == 128 ? launch_n<128>(a, Bt, st) : launch_n<64>(a, Bt, st);
+  if (tc) {
+    CUtensorMap maps[3];
+    if (!mm_internal::make_map4d_sw128(&maps[0], C, uint64_t(N), uint64_t(G), uint64_t(L),
+                                       uint64_t(Bt), 64, 1, uint32_t(ssd::kQ), 1) ||
+        !mm_internal::make_map4d_sw128(&maps[1], B, uint64_t(N), uint64_t(G), uint64_t(L),
+                                       uint64_t(Bt), 64, 1, uint32_t(ssd::kQ), 1) ||
+        !mm_internal::make_map4d_sw128(&maps[2], x, uint64_t(P), uint64_t(H), uint64_t(L),
+                                       uint64_t(Bt), 64, 1, uint32_t(ssd::kQ), 1))
+      return ssd_fail(MAMBA_ERR_CUDA, "cuTensorMapEncodeTiled failed or is unavailable");
+    void* word = nullptr;
+    char why[256];
+    if (mm_host::symbol_in_context(reinterpret_cast<const void*>(&g_ssd_status), &word,
+                                   "mamba2_ssd_fwd", why, sizeof(why)) != 0)
+      return ssd_fail(MAMBA_ERR_CUDA, "%s", why);
+    int* status = static_cast<int*>(word);
+    if (N == 128)
+      e = z ? launch_tc<128, true>(a, Bt, maps, status, st) : launch_tc<128, false>(a, Bt, maps, status, st);
+    else
+      e = z ? launch_tc<64, true>(a, Bt, maps, status, st) : launch_tc<64, false>(a, Bt, maps, status, st);
+  } else {
+    e = N == 128 ? launch_n<128>(a, Bt, st) : launch_n<64>(a, Bt, st);
+  }
   if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "ssd launch failed: %s", cudaGetErrorString(e));
   return ssd_ok();
 }

@@ -1,0 +1,546 @@
+// Mamba2 selective scan (the SSD layer) forward, main pass on the 5th-generation tensor cores
+// (tcgen05): the same chunked evaluation as ssd_kernel.cuh (niverel-mamba 0.1.0, sections
+// "The weight contract" and "Measured tolerances"), for rows without document resets.
+//
+// Per chunk of kQ = 64 steps, with cs the in-chunk cumulative sum of Delta A (log2 units)
+// and H [headdim p x d_state n] the state entering the chunk:
+//   G  = C B^T                                   (M 64 t, N 64 s, K n)       K-major A and B
+//   Y1 = C H^T        (H as bf16 hi + lo planes)  (M 64 t, N 64 p, K n)       K-major A and B
+//   Y2 = (M o G) x    (M o G as hi + lo planes)   (M 64 t, N 64 p, K 64 s)    x MN-major
+//   U  = (w o x)^T B                              (M 64 p, N n, K 64 s)       both MN-major
+//   y_t = 2^cs_t Y1[t] + Y2[t] + D x_t (times SiLU(z_t)),   H <- 2^cs_last H + U
+// with M[t, s] = 2^(cs_t - cs_s) Delta_s for s <= t and w_s = 2^(cs_last - cs_s) Delta_s.
+// The accumulators live in TMEM (an M = 64 accumulator puts row m in lane
+// (m mod 16) + 32 floor(m / 16)); the operand tiles in shared memory use the 128-byte
+// swizzle the TMA copies write (64-element rows, 8-row atoms of 1024 bytes).
+//
+// CTA = one (batch row, head, time segment), 9 warps:
+//   warp 8 (copy / MMA warp): lane 0 issues the TMA copies of each chunk's C, B and x tiles
+//     into a 2-deep ring and every tcgen05.mma, committing each group to an mbarrier;
+//   warps 0..7 (math warps, warp w reads TMEM lanes 32 (w mod 4) .. + 31, column half w / 4):
+//     Delta and cs (warp 0), the mask of G into bf16 hi/lo planes and w o x, the outputs from
+//     Y1 and Y2, and the state: H is held in registers (row p = 16 (w mod 4) + lane mod 16,
+//     a quarter of the n columns per lane), updated from U and written back as the hi/lo
+//     planes that the next chunk's C H^T reads.  An M = 64 accumulator's rows sit in lanes
+//     0..15 of each quarter; lanes 16..31 take the second half of their row's columns by a
+//     shuffle, so all lanes work.
+//   Per chunk k the math warps: mask G_k (warp 0 then forms chunk k + 1's cs), write the
+//   outputs of chunk k - 1 while (M o G_k) x and U_k run, update the state -- after which
+//   the copy/MMA warp can start C H^T of chunk k + 1.  Y1 and Y2 are double-buffered in TMEM,
+//   the tiles triple-buffered in shared memory.
+// Numerics match ssd_kernel.cuh: bf16 inputs enter exactly, the masked G and the state enter
+// as hi + lo bf16 pairs, w o x is rounded once to bf16, accumulation is fp32.
+//
+// Every wait is bounded: a warp that gives up records MAMBA_ERR_TIMEOUT in *status and leaves
+// its loop; the copy/MMA warp waits (bounded) for its copies and products in flight before
+// it frees TMEM.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "device_math.cuh"
+#include "sm100_primitives.cuh"
+#include "ssd_kernel.cuh"
+
+namespace ssd {
+namespace tc {
+
+constexpr int kMathWarps = 8;
+constexpr int kThreads = 32 * (kMathWarps + 1);
+constexpr int kCS = kMathWarps / 4;  // math warps per TMEM lane quarter: each takes 1/kCS of the columns
+constexpr int kCW = 64 / kCS;        // columns of a 64-column accumulator per math warp
+constexpr int kLW = kCW / 2;         // ... per lane
+constexpr int kNS = 3;             // TMA ring depth (chunks in flight)
+constexpr int kPanel = kQ * 128;   // 64 rows of 128 bytes: one swizzled operand panel
+
+template <int N>
+struct Smem {
+  static constexpr int NP = N / 64;                // 64-wide panels of d_state
+  static constexpr int kC = 0;                     // C [64 t][N n]
+  static constexpr int kB = NP * kPanel;           // B [64 s][N n]
+  static constexpr int kX = 2 * NP * kPanel;       // x [64 s][64 p]
+  static constexpr int kStage = (2 * NP + 1) * kPanel;
+  static constexpr int kMGh = kNS * kStage;        // masked G, hi and lo planes [64 t][64 s]
+  static constexpr int kMGl = kMGh + kPanel;
+  static constexpr int kXw = kMGl + kPanel;        // w o x [64 s][64 p]
+  static constexpr int kHh = kXw + kPanel;         // H hi and lo planes [64 p][N n]
+  static constexpr int kHl = kHh + NP * kPanel;
+  static constexpr int kCs = kHl + NP * kPanel;    // [3][kQ] cs (log2 units), chunk k in k % 3
+  static constexpr int kDl = kCs + 3 * kQ * 4;     // [3][kQ] Delta
+  static constexpr int kBar = kDl + 3 * kQ * 4;
+  // full[kNS], empty[kNS], g_done, y_done[2], u_done, mg_ready, h_ready
+  static constexpr int kNBar = 2 * kNS + 6;
+  static constexpr int kTotal = kBar + 8 * kNBar + 16;
+  static constexpr int kDynamic = kTotal + 1024;   // slack to align to 1 KiB
+  // TMEM: G (64 columns), Y1 and Y2 (64 columns each, two buffers by chunk parity), U (N)
+  static constexpr uint32_t kTG = 0, kTY1 = 64, kTY2 = 192, kTU = 320;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// All math warps agree on a flag at named barrier `id` (each of `threads` threads votes).
+__device__ __forceinline__ bool bar_and(int id, int threads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "barrier.cta.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r) : "r"(uint32_t(v)), "r"(id), "r"(threads) : "memory");
+  return r != 0;
+}
+
+// kW consecutive 32-bit TMEM columns of this thread's lane.
+template <int kW>
+__device__ __forceinline__ void ld_cols(uint32_t taddr, float (&v)[kW]) {
+  if constexpr (kW == 32) mm::tmem_ld32(taddr, v);
+  else mm::tmem_ld16(taddr, v);
+}
+
+// Byte offset of element (row r, column c) of a 64-column swizzled panel.
+__device__ __forceinline__ uint32_t pofs(int r, int c) {
+  return uint32_t(r * 128 + ((((c >> 3) ^ r) & 7) << 4) + (c & 7) * 2);
+}
+
+template <int N, bool kGate>
+__global__ void __launch_bounds__(kThreads, 1)
+ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ CUtensorMap tm_B,
+              const __grid_constant__ CUtensorMap tm_x, const SsdArgs a, int* status) {
+  using S = Smem<N>;
+  constexpr int NP = S::NP;
+  constexpr int NH = N / kCS;                      // state columns per math warp
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = mm::smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sb = mm::smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* full = bars;                // [kNS] a chunk's tiles landed
+  uint64_t* empty = bars + kNS;         // [kNS] the math warps are done with a stage
+  uint64_t* g_done = bars + 2 * kNS;    // G of the chunk is in TMEM
+  uint64_t* y_done = g_done + 1;        // [2] Y1 and Y2 of chunk k (barrier k & 1) are in TMEM
+  uint64_t* u_done = y_done + 2;        // U of the chunk is in TMEM
+  uint64_t* mg_ready = u_done + 1;      // the masked G planes and w o x are in shared memory
+  uint64_t* h_ready = mg_ready + 1;     // the hi/lo planes of the state entering a chunk
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kNBar);
+  float* cs_all = reinterpret_cast<float*>(smem + S::kCs);
+  float* dl_all = reinterpret_cast<float*>(smem + S::kDl);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int64_t b = blockIdx.y;
+  const int seg = blockIdx.z;
+  const int grp = h / (a.H / a.G);
+  const int64_t L = a.L;
+  const int64_t nchunks = (L + kQ - 1) / kQ;
+  const int64_t c_begin = int64_t(seg) * a.cps;
+  const int64_t c_end = c_begin + a.cps < nchunks ? c_begin + a.cps : nchunks;
+  const int nck = c_end > c_begin ? int(c_end - c_begin) : 0;
+  const int64_t bh = b * a.H + h;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mm::mbar_init(&full[i], 1);
+      mm::mbar_init(&empty[i], kMathWarps);
+    }
+    mm::mbar_init(g_done, 1);
+    mm::mbar_init(&y_done[0], 1);
+    mm::mbar_init(&y_done[1], 1);
+    mm::mbar_init(u_done, 1);
+    mm::mbar_init(mg_ready, kMathWarps);
+    mm::mbar_init(h_ready, kMathWarps);
+  }
+  if (warp == kMathWarps) {
+    mm::tmem_alloc(tmem_slot, S::kTmemCols);
+    mm::tmem_relinquish();
+  }
+  mm::tc_fence_before();
+  __syncthreads();
+  mm::tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == kMathWarps) {
+    // ============================================================== copy / MMA warp
+    bool good = true;
+    int issued = 0;
+    uint64_t* last_bar = nullptr;   // the barrier of the last commit, and its phase
+    uint32_t last_par = 0;
+    auto issue = [&](int k) {
+      const int s = k % kNS;
+      const int t0 = int((c_begin + k) * kQ);
+      const uint32_t st = sb + uint32_t(s * S::kStage);
+      mm::mbar_arrive_expect_tx(&full[s], uint32_t(S::kStage));
+      for (int pn = 0; pn < NP; ++pn) {
+        mm::tma_load_4d(st + S::kC + pn * kPanel, &tm_C, &full[s], pn * 64, grp, t0, int(b), 1024,
+                        2, status);
+        mm::tma_load_4d(st + S::kB + pn * kPanel, &tm_B, &full[s], pn * 64, grp, t0, int(b), 1024,
+                        2, status);
+      }
+      mm::tma_load_4d(st + S::kX, &tm_x, &full[s], 0, h, t0, int(b), 1024, 2, status);
+    };
+    if (lane == 0)
+      for (int k = 0; k < nck && k < kNS; ++k) issue(k);
+    issued = nck < kNS ? nck : kNS;
+    __syncwarp();
+    for (int k = 0; good && k < nck; ++k) {
+      const int s = k % kNS;
+      const uint32_t st = sb + uint32_t(s * S::kStage);
+      const uint32_t ty1 = S::kTY1 + uint32_t(k & 1) * 64u, ty2 = S::kTY2 + uint32_t(k & 1) * 64u;
+      good = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status));
+      if (!good) break;
+      // G of this chunk as soon as its tiles are in (the math warps read the previous G before
+      // they signalled mg_ready, which this warp waited for)
+      if (lane == 0) {
+        mm::tc_fence_after();
+        constexpr uint32_t idG = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 0>();
+        for (int kk = 0; kk < N / 16; ++kk) {
+          const uint32_t o = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+          mm::umma_bf16(tbase + S::kTG, mm::umma_desc_sw128(st + S::kC + o),
+                        mm::umma_desc_sw128(st + S::kB + o), idG, kk > 0 ? 1u : 0u);
+        }
+        mm::umma_commit(g_done);
+        last_bar = g_done;
+        last_par = uint32_t(k) & 1u;
+      }
+      __syncwarp();
+      // C H^T takes the state entering this chunk (hi, then lo), into this chunk's Y1 buffer
+      good = __all_sync(0xffffffffu, mm::mbar_wait(h_ready, uint32_t(k) & 1u, status));
+      if (!good) break;
+      if (lane == 0) {
+        mm::tc_fence_after();
+        constexpr uint32_t idY = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 0>();
+        int n = 0;
+        for (int pl = 0; pl < 2; ++pl)
+          for (int kk = 0; kk < N / 16; ++kk, ++n) {
+            const uint32_t o = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
+            mm::umma_bf16(tbase + ty1, mm::umma_desc_sw128(st + S::kC + o),
+                          mm::umma_desc_sw128(sb + uint32_t(pl ? S::kHl : S::kHh) + o), idY,
+                          n > 0 ? 1u : 0u);
+          }
+      }
+      __syncwarp();
+      good = __all_sync(0xffffffffu, mm::mbar_wait(mg_ready, uint32_t(k) & 1u, status));
+      if (!good) break;
+      if (lane == 0) {
+        mm::tc_fence_after();
+        constexpr uint32_t idY2 = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 1>();
+        int n = 0;
+        for (int pl = 0; pl < 2; ++pl)
+          for (int kk = 0; kk < kQ / 16; ++kk, ++n)
+            mm::umma_bf16(tbase + ty2,
+                          mm::umma_desc_sw128(sb + uint32_t(pl ? S::kMGl : S::kMGh) + kk * 32),
+                          mm::umma_desc_mn_sw128(st + S::kX + kk * 2048, kPanel), idY2,
+                          n > 0 ? 1u : 0u);
+        mm::umma_commit(&y_done[k & 1]);
+        constexpr uint32_t idU = mm::umma_idesc_bf16_f32_mj<64, N, 1, 1>();
+        for (int kk = 0; kk < kQ / 16; ++kk)
+          mm::umma_bf16(tbase + S::kTU, mm::umma_desc_mn_sw128(sb + S::kXw + kk * 2048, kPanel),
+                        mm::umma_desc_mn_sw128(st + S::kB + kk * 2048, kPanel), idU,
+                        kk > 0 ? 1u : 0u);
+        mm::umma_commit(u_done);
+        last_bar = u_done;
+      }
+      __syncwarp();
+      // the stage of chunk k - 1 takes chunk k + kNS - 1 once the math warps are done with it
+      // (they finish a chunk's outputs during the next chunk)
+      if (k >= 1 && k + kNS - 1 < nck) {
+        good = __all_sync(0xffffffffu, mm::mbar_wait(&empty[(k - 1) % kNS],
+                                                     uint32_t((k - 1) / kNS) & 1u, status));
+        if (!good) break;
+        if (lane == 0) issue(k + kNS - 1);
+        __syncwarp();
+        issued = k + kNS;
+      }
+    }
+    mm::named_bar_sync(0, kThreads);
+    if (lane == 0) {
+      // nothing may still write the stages or TMEM when the CTA leaves
+      for (int k = issued - kNS < 0 ? 0 : issued - kNS; !good && k < issued; ++k)
+        mm::mbar_wait(&full[k % kNS], uint32_t(k / kNS) & 1u, nullptr);
+      if (last_bar) mm::mbar_wait(last_bar, last_par, nullptr);
+    }
+    __syncwarp();
+    mm::tc_fence_after();
+    mm::tmem_dealloc(tbase, S::kTmemCols);
+    return;
+  }
+
+  // ================================================================== math warps
+  const int q = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column block
+  // An M = 64 accumulator holds row m in TMEM lane (m mod 16) + 32 (m / 16): a 32x32b load
+  // gives lanes 0..15 of the warp its rows; lanes 16..31 take the second half of the same
+  // rows' columns from them by a shuffle, so every lane works.
+  const int part = lane >> 4;                      // 0: first half of the columns, 1: second
+  const int src = lane & 15;                       // the lane that holds this lane's row
+  const int r = 16 * q + (lane & 15);              // accumulator row of this lane (t, or p)
+  const uint32_t tq = tbase + (uint32_t(32 * q) << 16);
+  const float A2 = -expf(a.A_log[h]) * mm::kLog2e;
+  const float bias = a.dt_bias[h];
+  const float Dh = a.D[h];
+  const bool has_h_in = a.h_in != nullptr;
+  constexpr int NH2 = NH / 2;                      // state columns per lane
+  const int ncol0 = hf * NH + part * NH2;          // this lane's first state column
+
+  // the state entering the segment: row p = r, columns [ncol0, ncol0 + NH2)
+  float H[NH2];
+#pragma unroll
+  for (int i = 0; i < NH2; ++i) H[i] = 0.0f;
+  {
+    const int64_t col0 = int64_t(r) * N + ncol0;
+    if (has_h_in) {
+      const float* hi = a.nseg > 1 ? a.ws_H + (bh * a.nseg + a.nseg - 1) * int64_t(kP * N)
+                                   : a.h_in + bh * int64_t(kP * N);
+#pragma unroll
+      for (int i = 0; i < NH2; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(hi + col0 + i);
+        H[i] = v.x; H[i + 1] = v.y; H[i + 2] = v.z; H[i + 3] = v.w;
+      }
+    }
+    for (int sp = 0; sp < seg; ++sp) {
+      const float f = mm::ex2_approx(a.ws_A[bh * (a.nseg - 1) + sp]);
+      const float* hs = a.ws_H + (bh * a.nseg + sp) * int64_t(kP * N);
+#pragma unroll
+      for (int i = 0; i < NH2; i += 4) {
+        const float4 v = *reinterpret_cast<const float4*>(hs + col0 + i);
+        H[i] = fmaf(f, H[i], v.x); H[i + 1] = fmaf(f, H[i + 1], v.y);
+        H[i + 2] = fmaf(f, H[i + 2], v.z); H[i + 3] = fmaf(f, H[i + 3], v.w);
+      }
+    }
+  }
+  // the state's hi/lo planes (B operand of C H^T): row p = r, this lane's columns
+  auto put_state = [&]() {
+#pragma unroll
+    for (int i = 0; i < NH2; i += 8) {
+      const int n = ncol0 + i;
+      const uint32_t off = uint32_t((n >> 6) * kPanel) + pofs(r, n & 63);
+      uint4 vh, vl;
+      split_bf16(H[i], H[i + 1], vh.x, vl.x);
+      split_bf16(H[i + 2], H[i + 3], vh.y, vl.y);
+      split_bf16(H[i + 4], H[i + 5], vh.z, vl.z);
+      split_bf16(H[i + 6], H[i + 7], vh.w, vl.w);
+      sts_u128(sb + S::kHh + off, vh);
+      sts_u128(sb + S::kHl + off, vl);
+    }
+    mm::fence_async_shared();
+    mm::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mm::mbar_arrive(h_ready);
+  };
+  put_state();
+
+  // the kLW of kCW loaded columns that are this lane's (lanes 16..31 take the upper half from
+  // their row's lane)
+  auto my_half = [&](const float (&v)[kCW], float (&out)[kLW]) {
+#pragma unroll
+    for (int i = 0; i < kLW; ++i) {
+      const float o = __shfl_sync(0xffffffffu, v[kLW + i], src);
+      out[i] = part ? o : v[i];
+    }
+  };
+
+  // warp 0: dt_raw of steps 2 lane, 2 lane + 1 of a chunk, then Delta and the inclusive
+  // cumulative sum of Delta A (log2 units) over it into the chunk's parity buffer
+  float dtn0 = 0.f, dtn1 = 0.f;
+  auto load_dt = [&](int64_t c) {
+    const int64_t t = c * kQ + 2 * lane;
+    dtn0 = t < L ? __bfloat162float(a.dt[(b * L + t) * a.H + h]) : 0.f;
+    dtn1 = t + 1 < L ? __bfloat162float(a.dt[(b * L + t + 1) * a.H + h]) : 0.f;
+  };
+  auto chunk_cs = [&](int k) {   // warp 0; dt of chunk k loaded
+    float* cs = cs_all + (k % 3) * kQ;
+    float* dl = dl_all + (k % 3) * kQ;
+    const int64_t t = (c_begin + k) * kQ + 2 * lane;
+    const float d0 = t < L ? mm::Math<false>::softplus(dtn0 + bias) : 0.f;
+    const float d1 = t + 1 < L ? mm::Math<false>::softplus(dtn1 + bias) : 0.f;
+    if (k + 1 < nck) load_dt(c_begin + k + 1);
+    const float e0 = d0 * A2, e1 = d1 * A2;
+    float sum = e0 + e1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float v = __shfl_up_sync(0xffffffffu, sum, o);
+      if (lane >= o) sum += v;
+    }
+    float ex = __shfl_up_sync(0xffffffffu, sum, 1);
+    if (lane == 0) ex = 0.f;
+    cs[2 * lane] = ex + e0;
+    cs[2 * lane + 1] = ex + e0 + e1;
+    dl[2 * lane] = d0;
+    dl[2 * lane + 1] = d1;
+  };
+  if (warp == 0 && nck > 0) {
+    load_dt(c_begin);
+    chunk_cs(0);
+  }
+
+  // the outputs of chunk k: y_t = 2^cs_t Y1[t] + Y2[t] + D x_t (times SiLU(z_t)), t = r, p in
+  // the half; then the chunk's stage is free
+  auto epilogue = [&](int k) -> bool {
+    if (!__all_sync(0xffffffffu, mm::mbar_wait(&y_done[k & 1], uint32_t(k >> 1) & 1u, status)))
+      return false;
+    mm::tc_fence_after();
+    const uint32_t ty1 = S::kTY1 + uint32_t(k & 1) * 64u, ty2 = S::kTY2 + uint32_t(k & 1) * 64u;
+    const uint32_t st = sb + uint32_t((k % kNS) * S::kStage);
+    const float* cs = cs_all + (k % 3) * kQ;
+    float y1f[kCW], y2f[kCW], y1[kLW], y2[kLW];
+    ld_cols(tq + ty1 + uint32_t(kCW * hf), y1f);
+    ld_cols(tq + ty2 + uint32_t(kCW * hf), y2f);
+    mm::tmem_wait_ld();
+    my_half(y1f, y1);
+    my_half(y2f, y2);
+    const int64_t t = (c_begin + k) * kQ + r;
+    if (t < L) {
+      const float et = mm::ex2_approx(cs[r]);
+      const int p0 = kCW * hf + kLW * part;
+      const int64_t row = ((b * L + t) * a.H + h) * kP + p0;
+#pragma unroll
+      for (int j = 0; j < kLW / 8; ++j) {
+        const uint4 xv = lds_u128(st + S::kX + pofs(r, p0 + 8 * j));
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint4 zv = make_uint4(0, 0, 0, 0);
+        if constexpr (kGate) zv = *reinterpret_cast<const uint4*>(a.z + row + 8 * j);
+        const uint32_t zw[4] = {zv.x, zv.y, zv.z, zv.w};
+        uint32_t ow[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = 8 * j + 2 * e;
+          float o0 = fmaf(et, y1[c], y2[c]) + Dh * bf16_lo(xw[e]);
+          float o1 = fmaf(et, y1[c + 1], y2[c + 1]) + Dh * bf16_hi(xw[e]);
+          if constexpr (kGate) {
+            o0 *= mm::Math<false>::silu(bf16_lo(zw[e]));
+            o1 *= mm::Math<false>::silu(bf16_hi(zw[e]));
+          }
+          ow[e] = pack_bf16(o0, o1);
+        }
+        *reinterpret_cast<uint4*>(a.y + row + 8 * j) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+      }
+    }
+    mm::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mm::mbar_arrive(&empty[k % kNS]);
+    return true;
+  };
+
+  // Every math warp passes the same named barrier once per chunk, where all agree whether to
+  // go on: a wait that gave up in one warp stops them all at the next chunk, never at an
+  // unbounded barrier.  Per chunk k: the mask (then warp 0 forms chunk k + 1's cs), the
+  // outputs of chunk k - 1 (while this chunk's products run), then the state update, after
+  // which the next chunk's C H^T can start.
+  bool ok = true;
+  for (int k = 0; k < nck; ++k) {
+    const int s = k % kNS;
+    const uint32_t st = sb + uint32_t(s * S::kStage);
+    const float* cs = cs_all + (k % 3) * kQ;
+    const float* dl = dl_all + (k % 3) * kQ;
+    ok = bar_and(1, 32 * kMathWarps, ok);      // this chunk's cs and Delta visible
+    if (!ok) break;
+    const float csl = cs[kQ - 1];
+
+    // ---- the mask of G: M[t, s] = G[t, s] 2^(cs_t - cs_s) Delta_s for s <= t, as hi/lo planes
+    ok = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status)) &&
+         __all_sync(0xffffffffu, mm::mbar_wait(g_done, uint32_t(k) & 1u, status));
+    if (!ok) continue;
+    mm::tc_fence_after();
+    {
+      float gf[kCW], g[kLW];
+      ld_cols(tq + S::kTG + uint32_t(kCW * hf), gf);
+      mm::tmem_wait_ld();
+      my_half(gf, g);
+      const int c0 = kCW * hf + kLW * part;        // this lane's kLW columns s
+      float csv[kLW], dlv[kLW];
+#pragma unroll
+      for (int i = 0; i < kLW; i += 4) {
+        const float4 cv = *reinterpret_cast<const float4*>(cs + c0 + i);
+        const float4 dv = *reinterpret_cast<const float4*>(dl + c0 + i);
+        csv[i] = cv.x; csv[i + 1] = cv.y; csv[i + 2] = cv.z; csv[i + 3] = cv.w;
+        dlv[i] = dv.x; dlv[i + 1] = dv.y; dlv[i + 2] = dv.z; dlv[i + 3] = dv.w;
+      }
+      const float ct = cs[r];
+#pragma unroll
+      for (int j = 0; j < kLW / 8; ++j) {
+        uint4 vh, vl;
+        uint32_t* ph = &vh.x;
+        uint32_t* plo = &vl.x;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i0 = 8 * j + 2 * e;
+          const float v0 = c0 + i0 <= r ? g[i0] * mm::ex2_approx(ct - csv[i0]) * dlv[i0] : 0.f;
+          const float v1 = c0 + i0 + 1 <= r ? g[i0 + 1] * mm::ex2_approx(ct - csv[i0 + 1]) * dlv[i0 + 1] : 0.f;
+          split_bf16(v0, v1, ph[e], plo[e]);
+        }
+        const uint32_t off = pofs(r, c0 + 8 * j);
+        sts_u128(sb + S::kMGh + off, vh);
+        sts_u128(sb + S::kMGl + off, vl);
+      }
+    }
+    // w o x, w_s = 2^(cs_last - cs_s) Delta_s: thread i of the math warps takes kXE
+    // consecutive elements of row i / (64 / kXE)
+    {
+      constexpr int kXE = kQ * kP / (32 * kMathWarps);
+      const int row = tid / (kP / kXE), c0 = (tid % (kP / kXE)) * kXE;
+      const float w = mm::ex2_approx(csl - cs[row]) * dl[row];
+#pragma unroll
+      for (int j = 0; j < kXE / 8; ++j) {
+        const uint32_t off = pofs(row, c0 + 8 * j);
+        const uint4 v = lds_u128(st + S::kX + off);
+        uint4 o;
+        o.x = pack_bf16(w * bf16_lo(v.x), w * bf16_hi(v.x));
+        o.y = pack_bf16(w * bf16_lo(v.y), w * bf16_hi(v.y));
+        o.z = pack_bf16(w * bf16_lo(v.z), w * bf16_hi(v.z));
+        o.w = pack_bf16(w * bf16_lo(v.w), w * bf16_hi(v.w));
+        sts_u128(sb + S::kXw + off, o);
+      }
+    }
+    mm::fence_async_shared();
+    mm::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mm::mbar_arrive(mg_ready);
+    if (warp == 0 && k + 1 < nck) chunk_cs(k + 1);   // read by all after the next barrier
+
+    // ---- the outputs of the previous chunk, while this chunk's (M o G) x and U run
+    if (k > 0) {
+      ok = epilogue(k - 1);
+      if (!ok) continue;
+    }
+
+    // ---- the state: H <- 2^cs_last H + U, then its hi/lo planes for the next chunk (u_done
+    // also means this chunk's C H^T and (M o G) x are complete)
+    ok = __all_sync(0xffffffffu, mm::mbar_wait(u_done, uint32_t(k) & 1u, status));
+    if (!ok) continue;
+    mm::tc_fence_after();
+    {
+      const float dec = mm::ex2_approx(csl);
+      // this lane's NH2 columns: lanes 0..15 the first NH2 of the (q, hf) block's NH loaded
+      // columns, lanes 16..31 the last NH2, from their row's lane
+      constexpr int kUW = NH < 32 ? NH : 32;
+#pragma unroll
+      for (int c = 0; c < NH; c += kUW) {
+        float u[kUW];
+        ld_cols(tq + S::kTU + uint32_t(hf * NH + c), u);
+        mm::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < kUW; ++i) {
+          const int n = c + i;                      // column within the block of NH
+          if (n < NH2) {
+            if (!part) H[n] = fmaf(dec, H[n], u[i]);
+          }
+          const float o = __shfl_sync(0xffffffffu, u[i], src);
+          if (n >= NH2 && part) H[n - NH2] = fmaf(dec, H[n - NH2], o);
+        }
+      }
+    }
+    put_state();
+  }
+  if (ok && nck > 0) ok = epilogue(nck - 1);
+
+  if (nck > 0) ok = bar_and(1, 32 * kMathWarps, ok);   // a failure in the last chunk counts
+  mm::named_bar_sync(0, kThreads);   // pairs with the copy / MMA warp's barrier
+  // the last segment leaves the final state
+  if (ok && seg == a.nseg - 1 && a.h_out) {
+    float* ho = a.h_out + bh * int64_t(kP * N) + int64_t(r) * N + ncol0;
+#pragma unroll
+    for (int i = 0; i < NH2; i += 4)
+      *reinterpret_cast<float4*>(ho + i) = make_float4(H[i], H[i + 1], H[i + 2], H[i + 3]);
+  }
+}
+
+}  // namespace tc
+}  // namespace ssd

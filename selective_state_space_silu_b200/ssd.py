@@ -14,7 +14,7 @@ import torch
 from . import mixer as _m
 
 EXPORTS = ("mamba2_ssd_fwd_workspace_bytes", "mamba2_ssd_fwd", "mamba2_ssd_step",
-           "mamba2_conv_silu", "mamba2_gated_rmsnorm")
+           "mamba2_conv_silu", "mamba2_gated_rmsnorm", "mamba2_ssd_check")
 
 
 class mamba2_dims(ctypes.Structure):
@@ -36,6 +36,8 @@ def _lib() -> ctypes.CDLL:
         lib.mamba2_ssd_fwd_workspace_bytes.argtypes = [ctypes.POINTER(mamba2_dims)]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
         lib.mamba2_ssd_fwd.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 13 + [ctypes.c_size_t, vp]
+        lib.mamba2_ssd_check.restype = ctypes.c_int
+        lib.mamba2_ssd_check.argtypes = [vp]
         lib.mamba2_ssd_step.restype = ctypes.c_int
         lib.mamba2_ssd_step.argtypes = [ctypes.POINTER(mamba2_dims)] + [vp] * 12
         lib.mamba2_conv_silu.restype = ctypes.c_int
@@ -90,6 +92,13 @@ def mamba2_ssd_fwd(x, dt_raw, A_log, B, C, D, dt_bias, *, z=None, seq_idx=None, 
         p(workspace, "workspace", None, dev), ws_bytes, _m._stream_handle(stream, dev))
     _m._check(rc)
     return y, h_out
+
+
+def mamba2_ssd_check(stream=None, device=None) -> None:
+    """Wait for the stream; raise MambaError(MAMBA_ERR_TIMEOUT) if a mamba2_ssd_fwd since the
+    last check gave up on a bounded wait (clears the status)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _m._check(_lib().mamba2_ssd_check(_m._stream_handle(stream, dev)))
 
 
 def mamba2_ssd_step(x, dt_raw, A_log, B, C, D, dt_bias, h_in, *, z=None, y=None, h_out=None,

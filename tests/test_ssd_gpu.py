@@ -72,6 +72,20 @@ def test_state_in_place():
     assert_close_tc(h, ho, "h_out in place")
 
 
+def test_status_word_is_clear_after_clean_calls():
+    """The tensor-core pass (rows without document ids) waits on its own copies and products
+    with bounded waits; after clean calls (one segment and several) mamba2_ssd_check finds
+    no timeout, and calls with document ids (the other pass) leave it clear as well."""
+    S.mamba2_ssd_check()                                  # start from a clear word
+    for L in (300, 4096):
+        run_gpu(draw(1, L, 2, 128, 1, True, True, seed=3150 + L))
+    ids = np.zeros((2, 130), dtype=np.int32)
+    ids[:, 70:] = 1                                       # one document change per row
+    run_gpu(draw(2, 130, 4, 64, 1, False, False, seed=3151), seq_idx=ids)
+    torch.cuda.synchronize()
+    S.mamba2_ssd_check()
+
+
 def test_empty_sequence_passes_state_through():
     inp = draw(2, 0, 4, 64, 1, True, True, seed=3200)
     y, h = run_gpu(inp)
