@@ -22,8 +22,8 @@
 //     Y1 and Y2, and the state: H is held in registers (row p = 16 (w mod 4) + lane mod 16,
 //     a quarter of the n columns per lane), updated from U and written back as the hi/lo
 //     planes that the next chunk's C H^T reads.  An M = 64 accumulator's rows sit in lanes
-//     0..15 of each quarter; lanes 16..31 take the second half of their row's columns by a
-//     shuffle, so all lanes work.
+//     0..15 of each quarter; the 16x32bx2 load shape hands lanes 16..31 of the warp the
+//     second half of the same rows' columns, so all lanes work.
 //   Per chunk k the math warps: mask G_k (warp 0 then forms chunk k + 1's cs), write the
 //   outputs of chunk k - 1 while (M o G_k) x and U_k run, update the state -- after which
 //   the copy/MMA warp can start C H^T of chunk k + 1.  Y1 and Y2 are double-buffered in TMEM,
@@ -90,11 +90,12 @@ __device__ __forceinline__ bool bar_and(int id, int threads, bool v) {
   return r != 0;
 }
 
-// kW consecutive 32-bit TMEM columns of this thread's lane.
+// kW consecutive 32-bit columns of an M = 64 accumulator's row 16 (warp % 4) + lane % 16:
+// lanes 0..15 from column col, lanes 16..31 from column col + kW.
 template <int kW>
-__device__ __forceinline__ void ld_cols(uint32_t taddr, float (&v)[kW]) {
-  if constexpr (kW == 32) mm::tmem_ld32(taddr, v);
-  else mm::tmem_ld16(taddr, v);
+__device__ __forceinline__ void ld_half(uint32_t taddr, float (&v)[kW]) {
+  if constexpr (kW == 32) mm::tmem_ld_half32<32>(taddr, v);
+  else mm::tmem_ld_half16<16>(taddr, v);
 }
 
 // Byte offset of element (row r, column c) of a 64-column swizzled panel.
@@ -266,11 +267,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
 
   // ================================================================== math warps
   const int q = warp & 3, hf = warp >> 2;          // TMEM lane quarter, column block
-  // An M = 64 accumulator holds row m in TMEM lane (m mod 16) + 32 (m / 16): a 32x32b load
-  // gives lanes 0..15 of the warp its rows; lanes 16..31 take the second half of the same
-  // rows' columns from them by a shuffle, so every lane works.
+  // An M = 64 accumulator holds row m in TMEM lane (m mod 16) + 32 (m / 16): lanes 0..15
+  // of the warp load the first half of their rows' columns, lanes 16..31 the second half.
   const int part = lane >> 4;                      // 0: first half of the columns, 1: second
-  const int src = lane & 15;                       // the lane that holds this lane's row
   const int r = 16 * q + (lane & 15);              // accumulator row of this lane (t, or p)
   const uint32_t tq = tbase + (uint32_t(32 * q) << 16);
   const float A2 = -expf(a.A_log[h]) * mm::kLog2e;
@@ -327,16 +326,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
   };
   put_state();
 
-  // the kLW of kCW loaded columns that are this lane's (lanes 16..31 take the upper half from
-  // their row's lane)
-  auto my_half = [&](const float (&v)[kCW], float (&out)[kLW]) {
-#pragma unroll
-    for (int i = 0; i < kLW; ++i) {
-      const float o = __shfl_sync(0xffffffffu, v[kLW + i], src);
-      out[i] = part ? o : v[i];
-    }
-  };
-
   // warp 0: dt_raw of steps 2 lane, 2 lane + 1 of a chunk, then Delta and the inclusive
   // cumulative sum of Delta A (log2 units) over it into the chunk's parity buffer
   float dtn0 = 0.f, dtn1 = 0.f;
@@ -380,12 +369,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     const uint32_t ty1 = S::kTY1 + uint32_t(k & 1) * 64u, ty2 = S::kTY2 + uint32_t(k & 1) * 64u;
     const uint32_t st = sb + uint32_t((k % kNS) * S::kStage);
     const float* cs = cs_all + (k % 3) * kQ;
-    float y1f[kCW], y2f[kCW], y1[kLW], y2[kLW];
-    ld_cols(tq + ty1 + uint32_t(kCW * hf), y1f);
-    ld_cols(tq + ty2 + uint32_t(kCW * hf), y2f);
+    float y1[kLW], y2[kLW];
+    ld_half(tq + ty1 + uint32_t(kCW * hf), y1);
+    ld_half(tq + ty2 + uint32_t(kCW * hf), y2);
     mm::tmem_wait_ld();
-    my_half(y1f, y1);
-    my_half(y2f, y2);
     const int64_t t = (c_begin + k) * kQ + r;
     if (t < L) {
       const float et = mm::ex2_approx(cs[r]);
@@ -440,10 +427,9 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     if (!ok) continue;
     mm::tc_fence_after();
     {
-      float gf[kCW], g[kLW];
-      ld_cols(tq + S::kTG + uint32_t(kCW * hf), gf);
+      float g[kLW];
+      ld_half(tq + S::kTG + uint32_t(kCW * hf), g);
       mm::tmem_wait_ld();
-      my_half(gf, g);
       const int c0 = kCW * hf + kLW * part;        // this lane's kLW columns s
       float csv[kLW], dlv[kLW];
 #pragma unroll
@@ -508,24 +494,13 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     mm::tc_fence_after();
     {
       const float dec = mm::ex2_approx(csl);
-      // this lane's NH2 columns: lanes 0..15 the first NH2 of the (q, hf) block's NH loaded
-      // columns, lanes 16..31 the last NH2, from their row's lane
-      constexpr int kUW = NH < 32 ? NH : 32;
+      // this lane's NH2 columns of U: the first NH2 of the (q, hf) block's NH for lanes 0..15,
+      // the last NH2 for lanes 16..31
+      float u[NH2];
+      ld_half(tq + S::kTU + uint32_t(hf * NH), u);
+      mm::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < NH; c += kUW) {
-        float u[kUW];
-        ld_cols(tq + S::kTU + uint32_t(hf * NH + c), u);
-        mm::tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < kUW; ++i) {
-          const int n = c + i;                      // column within the block of NH
-          if (n < NH2) {
-            if (!part) H[n] = fmaf(dec, H[n], u[i]);
-          }
-          const float o = __shfl_sync(0xffffffffu, u[i], src);
-          if (n >= NH2 && part) H[n - NH2] = fmaf(dec, H[n - NH2], o);
-        }
-      }
+      for (int i = 0; i < NH2; ++i) H[i] = fmaf(dec, H[i], u[i]);
     }
     put_state();
   }
