@@ -6,8 +6,8 @@
 // and H [headdim p x d_state n] the state entering the chunk:
 //   G  = C B^T                                   (M 64 t, N 64 s, K n)       K-major A and B
 //   Y1 = C H^T        (H as bf16 hi + lo planes)  (M 64 t, N 64 p, K n)       K-major A and B
-//   Y2 = (M o G) x    (M o G as hi + lo planes)   (M 64 t, N 64 p, K 64 s)    x MN-major
-//   U  = (w o x)^T B                              (M 64 p, N n, K 64 s)       both MN-major
+//   Y2 = (M o G) x    (M o G rounded to bf16)     (M 64 t, N 64 p, K 64 s)    x MN-major
+//   U  = (w o x)^T B  (w o x rounded to bf16)     (M 64 p, N n, K 64 s)       both MN-major
 //   y_t = 2^cs_t Y1[t] + Y2[t] + D x_t (times SiLU(z_t)),   H <- 2^cs_last H + U
 // with M[t, s] = 2^(cs_t - cs_s) Delta_s for s <= t and w_s = 2^(cs_last - cs_s) Delta_s.
 // The accumulators live in TMEM (an M = 64 accumulator puts row m in lane
@@ -16,20 +16,24 @@
 //
 // CTA = one (batch row, head, time segment), 9 warps:
 //   warp 8 (copy / MMA warp): lane 0 issues the TMA copies of each chunk's C, B and x tiles
-//     into a 2-deep ring and every tcgen05.mma, committing each group to an mbarrier;
+//     into a 3-deep ring and every tcgen05.mma, committing each group to an mbarrier;
 //   warps 0..7 (math warps, warp w reads TMEM lanes 32 (w mod 4) .. + 31, column half w / 4):
-//     Delta and cs (warp 0), the mask of G into bf16 hi/lo planes and w o x, the outputs from
+//     Delta and cs (warp 3), the mask of G into a bf16 plane and w o x, the outputs from
 //     Y1 and Y2, and the state: H is held in registers (row p = 16 (w mod 4) + lane mod 16,
 //     a quarter of the n columns per lane), updated from U and written back as the hi/lo
-//     planes that the next chunk's C H^T reads.  An M = 64 accumulator's rows sit in lanes
+//     bf16 planes that the next chunk's C H^T reads.  An M = 64 accumulator's rows sit in lanes
 //     0..15 of each quarter; the 16x32bx2 load shape hands lanes 16..31 of the warp the
 //     second half of the same rows' columns, so all lanes work.
 //   Per chunk k the math warps: mask G_k (warp 0 then forms chunk k + 1's cs), write the
 //   outputs of chunk k - 1 while (M o G_k) x and U_k run, update the state -- after which
-//   the copy/MMA warp can start C H^T of chunk k + 1.  Y1 and Y2 are double-buffered in TMEM,
-//   the tiles triple-buffered in shared memory.
-// Numerics match ssd_kernel.cuh: bf16 inputs enter exactly, the masked G and the state enter
-// as hi + lo bf16 pairs, w o x is rounded once to bf16, accumulation is fp32.
+//   the copy/MMA warp can start C H^T of chunk k + 1.  The tensor pipe is the scarce unit (an
+//   M = 64, N = 64, K = 16 product takes about 47 clocks, N = 128 about 67), so the copy/MMA
+//   warp keeps it fed: G of chunk k + 1 is issued right behind C H^T of chunk k and runs
+//   while the math warps mask G_k.  G, Y1 and Y2 are double-buffered in TMEM, the tiles
+//   triple-buffered in shared memory.
+// Numerics: bf16 inputs enter exactly; the masked G and w o x are each rounded once to bf16
+// (round to nearest), the state used by C H^T enters as a hi + lo bf16 pair; accumulation
+// is fp32 and the carried state itself stays fp32 in registers.
 //
 // Every wait is bounded: a warp that gives up records MAMBA_ERR_TIMEOUT in *status and leaves
 // its loop; the copy/MMA warp waits (bounded) for its copies and products in flight before
@@ -52,7 +56,19 @@ constexpr int kCS = kMathWarps / 4;  // math warps per TMEM lane quarter: each t
 constexpr int kCW = 64 / kCS;        // columns of a 64-column accumulator per math warp
 constexpr int kLW = kCW / 2;         // ... per lane
 constexpr int kNS = 3;             // TMA ring depth (chunks in flight)
+// The copy/MMA warp (warp 8) shares sub-partition 0 with math warps 0 and 4, and its
+// tcgen05.mma issue slows to about half rate when they issue back to back; the math work
+// that is not tied to TMEM lane quarter 0 therefore runs on the other sub-partitions: the
+// cumulative sums on warp kCsWarp, w o x on the six math warps with warp % 4 != 0.
+constexpr int kCsWarp = 3;
 constexpr int kPanel = kQ * 128;   // 64 rows of 128 bytes: one swizzled operand panel
+// bf16 planes of the masked G and of the state that C H^T reads.  The state takes two
+// (hi = bf16(H), lo = bf16(H - hi)): rounded once, its inter-chunk term C H^T carries an
+// error of 2^-9 times |C| |H| summed over d_state, which with a carried-in state of order one
+// and d_state 128 exceeds the output tolerance (measured: 1 element in 82k at 1.5x the bound).
+// The masked G takes one.
+constexpr int kMGPl = 1;
+constexpr int kHPl = 2;
 
 template <int N>
 struct Smem {
@@ -61,20 +77,18 @@ struct Smem {
   static constexpr int kB = NP * kPanel;           // B [64 s][N n]
   static constexpr int kX = 2 * NP * kPanel;       // x [64 s][64 p]
   static constexpr int kStage = (2 * NP + 1) * kPanel;
-  static constexpr int kMGh = kNS * kStage;        // masked G, hi and lo planes [64 t][64 s]
-  static constexpr int kMGl = kMGh + kPanel;
-  static constexpr int kXw = kMGl + kPanel;        // w o x [64 s][64 p]
-  static constexpr int kHh = kXw + kPanel;         // H hi and lo planes [64 p][N n]
-  static constexpr int kHl = kHh + NP * kPanel;
-  static constexpr int kCs = kHl + NP * kPanel;    // [3][kQ] cs (log2 units), chunk k in k % 3
+  static constexpr int kMG = kNS * kStage;         // masked G [64 t][64 s], bf16 planes
+  static constexpr int kXw = kMG + kMGPl * kPanel; // w o x [64 s][64 p]
+  static constexpr int kH = kXw + kPanel;          // H [64 p][N n], bf16 planes
+  static constexpr int kCs = kH + kHPl * NP * kPanel;   // [3][kQ] cs (log2), chunk k in k % 3
   static constexpr int kDl = kCs + 3 * kQ * 4;     // [3][kQ] Delta
   static constexpr int kBar = kDl + 3 * kQ * 4;
-  // full[kNS], empty[kNS], g_done, y_done[2], u_done, mg_ready, h_ready
-  static constexpr int kNBar = 2 * kNS + 6;
+  // full[kNS], empty[kNS], g_done[2], y_done[2], u_done, mg_ready, h_ready
+  static constexpr int kNBar = 2 * kNS + 7;
   static constexpr int kTotal = kBar + 8 * kNBar + 16;
   static constexpr int kDynamic = kTotal + 1024;   // slack to align to 1 KiB
-  // TMEM: G (64 columns), Y1 and Y2 (64 columns each, two buffers by chunk parity), U (N)
-  static constexpr uint32_t kTG = 0, kTY1 = 64, kTY2 = 192, kTU = 320;
+  // TMEM: G, Y1 and Y2 (64 columns each, two buffers by chunk parity), U (N columns)
+  static constexpr uint32_t kTG = 0, kTY1 = 128, kTY2 = 256, kTU = 384;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -117,11 +131,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* full = bars;                // [kNS] a chunk's tiles landed
   uint64_t* empty = bars + kNS;         // [kNS] the math warps are done with a stage
-  uint64_t* g_done = bars + 2 * kNS;    // G of the chunk is in TMEM
-  uint64_t* y_done = g_done + 1;        // [2] Y1 and Y2 of chunk k (barrier k & 1) are in TMEM
+  uint64_t* g_done = bars + 2 * kNS;    // [2] G of chunk k (barrier k & 1) is in TMEM
+  uint64_t* y_done = g_done + 2;        // [2] Y1 and Y2 of chunk k (barrier k & 1) are in TMEM
   uint64_t* u_done = y_done + 2;        // U of the chunk is in TMEM
-  uint64_t* mg_ready = u_done + 1;      // the masked G planes and w o x are in shared memory
-  uint64_t* h_ready = mg_ready + 1;     // the hi/lo planes of the state entering a chunk
+  uint64_t* mg_ready = u_done + 1;      // the masked G and w o x are in shared memory
+  uint64_t* h_ready = mg_ready + 1;     // the bf16 planes of the state entering a chunk
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kNBar);
   float* cs_all = reinterpret_cast<float*>(smem + S::kCs);
   float* dl_all = reinterpret_cast<float*>(smem + S::kDl);
@@ -143,7 +157,8 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       mm::mbar_init(&full[i], 1);
       mm::mbar_init(&empty[i], kMathWarps);
     }
-    mm::mbar_init(g_done, 1);
+    mm::mbar_init(&g_done[0], 1);
+    mm::mbar_init(&g_done[1], 1);
     mm::mbar_init(&y_done[0], 1);
     mm::mbar_init(&y_done[1], 1);
     mm::mbar_init(u_done, 1);
@@ -178,67 +193,85 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       }
       mm::tma_load_4d(st + S::kX, &tm_x, &full[s], 0, h, t0, int(b), 1024, 2, status);
     };
+    // G of chunk k into its parity buffer (the buffer's previous G, chunk k - 2, was masked
+    // before mg_ready of chunk k - 1, which this warp waited for)
+    auto issue_g = [&](int k) -> bool {
+      const int s = k % kNS;
+      const uint32_t st = sb + uint32_t(s * S::kStage);
+      if (!__all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status)))
+        return false;
+      if (lane == 0) {
+        mm::tc_fence_after();
+        constexpr uint32_t idG = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 0>();
+        const uint32_t dc = mm::umma_desc_lo(st + S::kC, 16), db = mm::umma_desc_lo(st + S::kB, 16);
+#pragma unroll
+        for (int kk = 0; kk < N / 16; ++kk) {
+          const uint32_t o = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
+          mm::umma_bf16_lo(tbase + S::kTG + uint32_t(k & 1) * 64u, dc + o, db + o, idG,
+                           kk > 0 ? 1u : 0u);
+        }
+        mm::umma_commit(&g_done[k & 1]);
+        last_bar = &g_done[k & 1];
+        last_par = uint32_t(k >> 1) & 1u;
+      }
+      __syncwarp();
+      return true;
+    };
     if (lane == 0)
       for (int k = 0; k < nck && k < kNS; ++k) issue(k);
     issued = nck < kNS ? nck : kNS;
     __syncwarp();
+    if (nck > 0) good = issue_g(0);
     for (int k = 0; good && k < nck; ++k) {
       const int s = k % kNS;
       const uint32_t st = sb + uint32_t(s * S::kStage);
       const uint32_t ty1 = S::kTY1 + uint32_t(k & 1) * 64u, ty2 = S::kTY2 + uint32_t(k & 1) * 64u;
-      good = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status));
-      if (!good) break;
-      // G of this chunk as soon as its tiles are in (the math warps read the previous G before
-      // they signalled mg_ready, which this warp waited for)
-      if (lane == 0) {
-        mm::tc_fence_after();
-        constexpr uint32_t idG = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 0>();
-        for (int kk = 0; kk < N / 16; ++kk) {
-          const uint32_t o = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
-          mm::umma_bf16(tbase + S::kTG, mm::umma_desc_sw128(st + S::kC + o),
-                        mm::umma_desc_sw128(st + S::kB + o), idG, kk > 0 ? 1u : 0u);
-        }
-        mm::umma_commit(g_done);
-        last_bar = g_done;
-        last_par = uint32_t(k) & 1u;
-      }
-      __syncwarp();
-      // C H^T takes the state entering this chunk (hi, then lo), into this chunk's Y1 buffer
+      // C H^T takes the state entering this chunk, into this chunk's Y1 buffer
       good = __all_sync(0xffffffffu, mm::mbar_wait(h_ready, uint32_t(k) & 1u, status));
       if (!good) break;
       if (lane == 0) {
         mm::tc_fence_after();
         constexpr uint32_t idY = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 0>();
-        int n = 0;
-        for (int pl = 0; pl < 2; ++pl)
-          for (int kk = 0; kk < N / 16; ++kk, ++n) {
-            const uint32_t o = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32);
-            mm::umma_bf16(tbase + ty1, mm::umma_desc_sw128(st + S::kC + o),
-                          mm::umma_desc_sw128(sb + uint32_t(pl ? S::kHl : S::kHh) + o), idY,
-                          n > 0 ? 1u : 0u);
+        const uint32_t dc = mm::umma_desc_lo(st + S::kC, 16), dh = mm::umma_desc_lo(sb + S::kH, 16);
+#pragma unroll
+        for (int pl = 0; pl < kHPl; ++pl)
+#pragma unroll
+          for (int kk = 0; kk < N / 16; ++kk) {
+            const uint32_t o = uint32_t((kk >> 2) * kPanel + (kk & 3) * 32) >> 4;
+            mm::umma_bf16_lo(tbase + ty1, dc + o, dh + uint32_t(pl * NP * kPanel >> 4) + o, idY,
+                             pl + kk > 0 ? 1u : 0u);
           }
       }
       __syncwarp();
+      // the next chunk's G runs while the math warps mask this chunk's
+      if (k + 1 < nck) {
+        good = issue_g(k + 1);
+        if (!good) break;
+      }
       good = __all_sync(0xffffffffu, mm::mbar_wait(mg_ready, uint32_t(k) & 1u, status));
       if (!good) break;
       if (lane == 0) {
         mm::tc_fence_after();
         constexpr uint32_t idY2 = mm::umma_idesc_bf16_f32_mj<64, 64, 0, 1>();
-        int n = 0;
-        for (int pl = 0; pl < 2; ++pl)
-          for (int kk = 0; kk < kQ / 16; ++kk, ++n)
-            mm::umma_bf16(tbase + ty2,
-                          mm::umma_desc_sw128(sb + uint32_t(pl ? S::kMGl : S::kMGh) + kk * 32),
-                          mm::umma_desc_mn_sw128(st + S::kX + kk * 2048, kPanel), idY2,
-                          n > 0 ? 1u : 0u);
+        const uint32_t dm = mm::umma_desc_lo(sb + S::kMG, 16);
+        const uint32_t dx = mm::umma_desc_lo(st + S::kX, kPanel);
+#pragma unroll
+        for (int pl = 0; pl < kMGPl; ++pl)
+#pragma unroll
+          for (int kk = 0; kk < kQ / 16; ++kk)
+            mm::umma_bf16_lo(tbase + ty2, dm + uint32_t((pl * kPanel + kk * 32) >> 4),
+                             dx + uint32_t(kk * 2048 >> 4), idY2, pl + kk > 0 ? 1u : 0u);
         mm::umma_commit(&y_done[k & 1]);
         constexpr uint32_t idU = mm::umma_idesc_bf16_f32_mj<64, N, 1, 1>();
+        const uint32_t dw = mm::umma_desc_lo(sb + S::kXw, kPanel);
+        const uint32_t dbm = mm::umma_desc_lo(st + S::kB, kPanel);
+#pragma unroll
         for (int kk = 0; kk < kQ / 16; ++kk)
-          mm::umma_bf16(tbase + S::kTU, mm::umma_desc_mn_sw128(sb + S::kXw + kk * 2048, kPanel),
-                        mm::umma_desc_mn_sw128(st + S::kB + kk * 2048, kPanel), idU,
-                        kk > 0 ? 1u : 0u);
+          mm::umma_bf16_lo(tbase + S::kTU, dw + uint32_t(kk * 2048 >> 4),
+                           dbm + uint32_t(kk * 2048 >> 4), idU, kk > 0 ? 1u : 0u);
         mm::umma_commit(u_done);
         last_bar = u_done;
+        last_par = uint32_t(k) & 1u;
       }
       __syncwarp();
       // the stage of chunk k - 1 takes chunk k + kNS - 1 once the math warps are done with it
@@ -305,19 +338,25 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       }
     }
   }
-  // the state's hi/lo planes (B operand of C H^T): row p = r, this lane's columns
+  // the state's bf16 planes (B operand of C H^T): row p = r, this lane's columns
   auto put_state = [&]() {
 #pragma unroll
     for (int i = 0; i < NH2; i += 8) {
       const int n = ncol0 + i;
       const uint32_t off = uint32_t((n >> 6) * kPanel) + pofs(r, n & 63);
-      uint4 vh, vl;
-      split_bf16(H[i], H[i + 1], vh.x, vl.x);
-      split_bf16(H[i + 2], H[i + 3], vh.y, vl.y);
-      split_bf16(H[i + 4], H[i + 5], vh.z, vl.z);
-      split_bf16(H[i + 6], H[i + 7], vh.w, vl.w);
-      sts_u128(sb + S::kHh + off, vh);
-      sts_u128(sb + S::kHl + off, vl);
+      if constexpr (kHPl == 2) {
+        uint4 vh, vl;
+        split_bf16(H[i], H[i + 1], vh.x, vl.x);
+        split_bf16(H[i + 2], H[i + 3], vh.y, vl.y);
+        split_bf16(H[i + 4], H[i + 5], vh.z, vl.z);
+        split_bf16(H[i + 6], H[i + 7], vh.w, vl.w);
+        sts_u128(sb + S::kH + off, vh);
+        sts_u128(sb + S::kH + uint32_t(NP * kPanel) + off, vl);
+      } else {
+        sts_u128(sb + S::kH + off,
+                 make_uint4(pack_bf16(H[i], H[i + 1]), pack_bf16(H[i + 2], H[i + 3]),
+                            pack_bf16(H[i + 4], H[i + 5]), pack_bf16(H[i + 6], H[i + 7])));
+      }
     }
     mm::fence_async_shared();
     mm::tc_fence_before();
@@ -334,7 +373,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     dtn0 = t < L ? __bfloat162float(a.dt[(b * L + t) * a.H + h]) : 0.f;
     dtn1 = t + 1 < L ? __bfloat162float(a.dt[(b * L + t + 1) * a.H + h]) : 0.f;
   };
-  auto chunk_cs = [&](int k) {   // warp 0; dt of chunk k loaded
+  auto chunk_cs = [&](int k) {   // warp kCsWarp; dt of chunk k loaded
     float* cs = cs_all + (k % 3) * kQ;
     float* dl = dl_all + (k % 3) * kQ;
     const int64_t t = (c_begin + k) * kQ + 2 * lane;
@@ -355,7 +394,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     dl[2 * lane] = d0;
     dl[2 * lane + 1] = d1;
   };
-  if (warp == 0 && nck > 0) {
+  if (warp == kCsWarp && nck > 0) {
     load_dt(c_begin);
     chunk_cs(0);
   }
@@ -421,14 +460,14 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     if (!ok) break;
     const float csl = cs[kQ - 1];
 
-    // ---- the mask of G: M[t, s] = G[t, s] 2^(cs_t - cs_s) Delta_s for s <= t, as hi/lo planes
+    // ---- the mask of G: M[t, s] = G[t, s] 2^(cs_t - cs_s) Delta_s for s <= t, in bf16
     ok = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status)) &&
-         __all_sync(0xffffffffu, mm::mbar_wait(g_done, uint32_t(k) & 1u, status));
+         __all_sync(0xffffffffu, mm::mbar_wait(&g_done[k & 1], uint32_t(k >> 1) & 1u, status));
     if (!ok) continue;
     mm::tc_fence_after();
     {
       float g[kLW];
-      ld_half(tq + S::kTG + uint32_t(kCW * hf), g);
+      ld_half(tq + S::kTG + uint32_t(k & 1) * 64u + uint32_t(kCW * hf), g);
       mm::tmem_wait_ld();
       const int c0 = kCW * hf + kLW * part;        // this lane's kLW columns s
       float csv[kLW], dlv[kLW];
@@ -442,30 +481,31 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       const float ct = cs[r];
 #pragma unroll
       for (int j = 0; j < kLW / 8; ++j) {
-        uint4 vh, vl;
-        uint32_t* ph = &vh.x;
-        uint32_t* plo = &vl.x;
+        uint32_t pw[4];
+        [[maybe_unused]] uint32_t pl[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i0 = 8 * j + 2 * e;
           const float v0 = c0 + i0 <= r ? g[i0] * mm::ex2_approx(ct - csv[i0]) * dlv[i0] : 0.f;
           const float v1 = c0 + i0 + 1 <= r ? g[i0 + 1] * mm::ex2_approx(ct - csv[i0 + 1]) * dlv[i0 + 1] : 0.f;
-          split_bf16(v0, v1, ph[e], plo[e]);
+          if constexpr (kMGPl == 2) split_bf16(v0, v1, pw[e], pl[e]);
+          else pw[e] = pack_bf16(v0, v1);
         }
         const uint32_t off = pofs(r, c0 + 8 * j);
-        sts_u128(sb + S::kMGh + off, vh);
-        sts_u128(sb + S::kMGl + off, vl);
+        sts_u128(sb + S::kMG + off, make_uint4(pw[0], pw[1], pw[2], pw[3]));
+        if constexpr (kMGPl == 2)
+          sts_u128(sb + S::kMG + uint32_t(kPanel) + off, make_uint4(pl[0], pl[1], pl[2], pl[3]));
       }
     }
-    // w o x, w_s = 2^(cs_last - cs_s) Delta_s: thread i of the math warps takes kXE
-    // consecutive elements of row i / (64 / kXE)
-    {
-      constexpr int kXE = kQ * kP / (32 * kMathWarps);
-      const int row = tid / (kP / kXE), c0 = (tid % (kP / kXE)) * kXE;
-      const float w = mm::ex2_approx(csl - cs[row]) * dl[row];
-#pragma unroll
-      for (int j = 0; j < kXE / 8; ++j) {
-        const uint32_t off = pofs(row, c0 + 8 * j);
+    // w o x, w_s = 2^(cs_last - cs_s) Delta_s, in 8-element pieces (row pc / 8, columns
+    // 8 (pc mod 8) ..): the 192 threads of the math warps off sub-partition 0 take pieces
+    // u, u + 192, ...
+    if (q != 0) {
+      const int u = (warp - 1 - (warp >> 2)) * 32 + lane;
+      for (int pc = u; pc < kQ * kP / 8; pc += 6 * 32) {
+        const int row = pc >> 3;
+        const float w = mm::ex2_approx(csl - cs[row]) * dl[row];
+        const uint32_t off = pofs(row, (pc & 7) * 8);
         const uint4 v = lds_u128(st + S::kX + off);
         uint4 o;
         o.x = pack_bf16(w * bf16_lo(v.x), w * bf16_hi(v.x));
@@ -479,7 +519,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     mm::tc_fence_before();
     __syncwarp();
     if (lane == 0) mm::mbar_arrive(mg_ready);
-    if (warp == 0 && k + 1 < nck) chunk_cs(k + 1);   // read by all after the next barrier
+    if (warp == kCsWarp && k + 1 < nck) chunk_cs(k + 1);   // read by all after the next barrier
 
     // ---- the outputs of the previous chunk, while this chunk's (M o G) x and U run
     if (k > 0) {
@@ -487,7 +527,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       if (!ok) continue;
     }
 
-    // ---- the state: H <- 2^cs_last H + U, then its hi/lo planes for the next chunk (u_done
+    // ---- the state: H <- 2^cs_last H + U, then its bf16 planes for the next chunk (u_done
     // also means this chunk's C H^T and (M o G) x are complete)
     ok = __all_sync(0xffffffffu, mm::mbar_wait(u_done, uint32_t(k) & 1u, status));
     if (!ok) continue;
