@@ -14,9 +14,10 @@
 // (m mod 16) + 32 floor(m / 16)); the operand tiles in shared memory use the 128-byte
 // swizzle the TMA copies write (64-element rows, 8-row atoms of 1024 bytes).
 //
-// CTA = one (batch row, head, time segment), 9 warps:
-//   warp 8 (copy / MMA warp): lane 0 issues the TMA copies of each chunk's C, B and x tiles
-//     into a 3-deep ring and every tcgen05.mma, committing each group to an mbarrier;
+// CTA = one (batch row, head, time segment), 10 warps:
+//   warp 9 (copy warp): lane 0 issues the TMA copies of each chunk's C, B and x tiles into a
+//     3-deep ring, refilling a stage as soon as the math warps release it;
+//   warp 8 (MMA warp): lane 0 issues every tcgen05.mma, committing each group to an mbarrier;
 //   warps 0..7 (math warps, warp w reads TMEM lanes 32 (w mod 4) .. + 31, column half w / 4):
 //     Delta and cs (warp 3), the mask of G into a bf16 plane and w o x, the outputs from
 //     Y1 and Y2, and the state: H is held in registers (row p = 16 (w mod 4) + lane mod 16,
@@ -24,20 +25,20 @@
 //     bf16 planes that the next chunk's C H^T reads.  An M = 64 accumulator's rows sit in lanes
 //     0..15 of each quarter; the 16x32bx2 load shape hands lanes 16..31 of the warp the
 //     second half of the same rows' columns, so all lanes work.
-//   Per chunk k the math warps: mask G_k (warp 0 then forms chunk k + 1's cs), write the
+//   Per chunk k the math warps: mask G_k (warp 3 then forms chunk k + 1's cs), write the
 //   outputs of chunk k - 1 while (M o G_k) x and U_k run, update the state -- after which
-//   the copy/MMA warp can start C H^T of chunk k + 1.  The tensor pipe is the scarce unit (an
-//   M = 64, N = 64, K = 16 product takes about 47 clocks, N = 128 about 67), so the copy/MMA
-//   warp keeps it fed: G of chunk k + 1 is issued right behind C H^T of chunk k and runs
-//   while the math warps mask G_k.  G, Y1 and Y2 are double-buffered in TMEM, the tiles
-//   triple-buffered in shared memory.
+//   the MMA warp can start C H^T of chunk k + 1.  The tensor pipe is the scarce unit (an
+//   M = 64, N = 64, K = 16 product takes about 47 clocks, N = 128 about 67), so the MMA warp
+//   keeps it fed: G of chunk k + 1 is issued right behind C H^T of chunk k and runs while
+//   the math warps mask G_k, and the copies are left to their own warp.  G, Y1 and Y2 are
+//   double-buffered in TMEM, the tiles triple-buffered in shared memory.
 // Numerics: bf16 inputs enter exactly; the masked G and w o x are each rounded once to bf16
 // (round to nearest), the state used by C H^T enters as a hi + lo bf16 pair; accumulation
 // is fp32 and the carried state itself stays fp32 in registers.
 //
 // Every wait is bounded: a warp that gives up records MAMBA_ERR_TIMEOUT in *status and leaves
-// its loop; the copy/MMA warp waits (bounded) for its copies and products in flight before
-// it frees TMEM.
+// its loop; the copy warp waits (bounded) for its copies in flight and the MMA warp for its
+// products before the CTA leaves and TMEM is freed.
 #pragma once
 
 #include <cuda.h>
@@ -51,12 +52,14 @@ namespace ssd {
 namespace tc {
 
 constexpr int kMathWarps = 8;
-constexpr int kThreads = 32 * (kMathWarps + 1);
+constexpr int kMmaWarp = kMathWarps;      // issues every tcgen05.mma, owns TMEM
+constexpr int kCopyWarp = kMathWarps + 1; // issues the TMA copies
+constexpr int kThreads = 32 * (kMathWarps + 2);
 constexpr int kCS = kMathWarps / 4;  // math warps per TMEM lane quarter: each takes 1/kCS of the columns
 constexpr int kCW = 64 / kCS;        // columns of a 64-column accumulator per math warp
 constexpr int kLW = kCW / 2;         // ... per lane
 constexpr int kNS = 3;             // TMA ring depth (chunks in flight)
-// The copy/MMA warp (warp 8) shares sub-partition 0 with math warps 0 and 4, and its
+// The MMA warp (warp 8) shares sub-partition 0 with math warps 0 and 4, and its
 // tcgen05.mma issue slows to about half rate when they issue back to back; the math work
 // that is not tied to TMEM lane quarter 0 therefore runs on the other sub-partitions: the
 // cumulative sums on warp kCsWarp, w o x on the six math warps with warp % 4 != 0.
@@ -165,7 +168,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     mm::mbar_init(mg_ready, kMathWarps);
     mm::mbar_init(h_ready, kMathWarps);
   }
-  if (warp == kMathWarps) {
+  if (warp == kMmaWarp) {
     mm::tmem_alloc(tmem_slot, S::kTmemCols);
     mm::tmem_relinquish();
   }
@@ -174,12 +177,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
   mm::tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp == kMathWarps) {
-    // ============================================================== copy / MMA warp
-    bool good = true;
-    int issued = 0;
-    uint64_t* last_bar = nullptr;   // the barrier of the last commit, and its phase
-    uint32_t last_par = 0;
+  if (warp == kCopyWarp) {
+    // ================================================================== copy warp
+    // the stage of chunk k - kNS takes chunk k once the math warps are done with it (they
+    // finish a chunk's outputs during the next chunk, after its products completed)
     auto issue = [&](int k) {
       const int s = k % kNS;
       const int t0 = int((c_begin + k) * kQ);
@@ -193,6 +194,34 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       }
       mm::tma_load_4d(st + S::kX, &tm_x, &full[s], 0, h, t0, int(b), 1024, 2, status);
     };
+    bool good = true;
+    if (lane == 0)
+      for (int k = 0; k < nck && k < kNS; ++k) issue(k);
+    int issued = nck < kNS ? nck : kNS;
+    __syncwarp();
+    for (int k = kNS; good && k < nck; ++k) {
+      good = __all_sync(0xffffffffu, mm::mbar_wait(&empty[(k - kNS) % kNS],
+                                                   uint32_t((k - kNS) / kNS) & 1u, status));
+      if (!good) break;
+      if (lane == 0) issue(k);
+      __syncwarp();
+      issued = k + 1;
+    }
+    mm::named_bar_sync(0, kThreads);
+    // nothing may still write the stages when the CTA leaves (after a failure elsewhere the
+    // last copies may not have been waited for)
+    if (lane == 0)
+      for (int k = issued - kNS < 0 ? 0 : issued - kNS; k < issued; ++k)
+        mm::mbar_wait(&full[k % kNS], uint32_t(k / kNS) & 1u, nullptr);
+    __syncwarp();
+    return;
+  }
+
+  if (warp == kMmaWarp) {
+    // =================================================================== MMA warp
+    bool good = true;
+    uint64_t* last_bar = nullptr;   // the barrier of the last commit, and its phase
+    uint32_t last_par = 0;
     // G of chunk k into its parity buffer (the buffer's previous G, chunk k - 2, was masked
     // before mg_ready of chunk k - 1, which this warp waited for)
     auto issue_g = [&](int k) -> bool {
@@ -217,10 +246,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
       __syncwarp();
       return true;
     };
-    if (lane == 0)
-      for (int k = 0; k < nck && k < kNS; ++k) issue(k);
-    issued = nck < kNS ? nck : kNS;
-    __syncwarp();
     if (nck > 0) good = issue_g(0);
     for (int k = 0; good && k < nck; ++k) {
       const int s = k % kNS;
@@ -274,24 +299,10 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
         last_par = uint32_t(k) & 1u;
       }
       __syncwarp();
-      // the stage of chunk k - 1 takes chunk k + kNS - 1 once the math warps are done with it
-      // (they finish a chunk's outputs during the next chunk)
-      if (k >= 1 && k + kNS - 1 < nck) {
-        good = __all_sync(0xffffffffu, mm::mbar_wait(&empty[(k - 1) % kNS],
-                                                     uint32_t((k - 1) / kNS) & 1u, status));
-        if (!good) break;
-        if (lane == 0) issue(k + kNS - 1);
-        __syncwarp();
-        issued = k + kNS;
-      }
     }
     mm::named_bar_sync(0, kThreads);
-    if (lane == 0) {
-      // nothing may still write the stages or TMEM when the CTA leaves
-      for (int k = issued - kNS < 0 ? 0 : issued - kNS; !good && k < issued; ++k)
-        mm::mbar_wait(&full[k % kNS], uint32_t(k / kNS) & 1u, nullptr);
-      if (last_bar) mm::mbar_wait(last_bar, last_par, nullptr);
-    }
+    // nothing may still write TMEM when it is freed
+    if (lane == 0 && last_bar) mm::mbar_wait(last_bar, last_par, nullptr);
     __syncwarp();
     mm::tc_fence_after();
     mm::tmem_dealloc(tbase, S::kTmemCols);
@@ -547,7 +558,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
   if (ok && nck > 0) ok = epilogue(nck - 1);
 
   if (nck > 0) ok = bar_and(1, 32 * kMathWarps, ok);   // a failure in the last chunk counts
-  mm::named_bar_sync(0, kThreads);   // pairs with the copy / MMA warp's barrier
+  mm::named_bar_sync(0, kThreads);   // pairs with the copy and MMA warps' barriers
   // the last segment leaves the final state
   if (ok && seg == a.nseg - 1 && a.h_out) {
     float* ho = a.h_out + bh * int64_t(kP * N) + int64_t(r) * N + ncol0;
