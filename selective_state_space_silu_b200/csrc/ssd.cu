@@ -135,14 +135,31 @@ cudaError_t launch(const ssd::SsdArgs& a, int64_t batch, cudaStream_t st) {
   return launch_one<N, kGate, false, kSeq>(a, batch, a.nseg, st);
 }
 
-// The tensor-core main pass (no document resets), after the mma.sync state pass when the
-// rows are cut into segments.
+// The tensor-core passes (no document resets): the state pass when the rows are cut into
+// segments, then the main pass.
+template <int N>
+cudaError_t launch_tc_state(const ssd::SsdArgs& a, int64_t batch, const CUtensorMap* maps,
+                            int* status, cudaStream_t st) {
+  using S = ssd::tc::StateSmem<N>;
+  auto kern = ssd::tc::ssd_tc_state_kernel<N>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               S::kDynamic);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kern<<<dim3(unsigned(a.H), unsigned(batch), unsigned(a.nseg - 1)), ssd::tc::kThreads,
+         S::kDynamic, st>>>(maps[1], maps[2], a, status);
+  return cudaGetLastError();
+}
+
 template <int N, bool kGate>
 cudaError_t launch_tc(const ssd::SsdArgs& a, int64_t batch, const CUtensorMap* maps, int* status,
                       cudaStream_t st) {
   using S = ssd::tc::Smem<N>;
   if (a.nseg > 1) {
-    cudaError_t e = launch_one<N, false, true, false>(a, batch, a.nseg - 1, st);
+    cudaError_t e = launch_tc_state<N>(a, batch, maps, status, st);
     if (e != cudaSuccess) return e;
   }
   auto kern = ssd::tc::ssd_tc_kernel<N, kGate>;

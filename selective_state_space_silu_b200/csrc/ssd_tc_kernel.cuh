@@ -29,8 +29,9 @@
 //   outputs of chunk k - 1 while (M o G_k) x and U_k run, update the state -- after which
 //   the MMA warp can start C H^T of chunk k + 1.  The tensor pipe is the scarce unit (an
 //   M = 64, N = 64, K = 16 product takes about 47 clocks, N = 128 about 67), so the MMA warp
-//   keeps it fed: G of chunk k + 1 is issued right behind C H^T of chunk k and runs while
-//   the math warps mask G_k, and the copies are left to their own warp.  G, Y1 and Y2 are
+//   keeps it fed: G of chunk k + 1 is issued right behind U_k and runs while the math warps
+//   update the state, C H^T of chunk k + 1 runs while they mask G_{k+1}, and the copies are
+//   left to their own warp.  G, Y1 and Y2 are
 //   double-buffered in TMEM, the tiles triple-buffered in shared memory.
 // Numerics: bf16 inputs enter exactly; the masked G and w o x are each rounded once to bf16
 // (round to nearest), the state used by C H^T enters as a hi + lo bf16 pair; accumulation
@@ -64,6 +65,37 @@ constexpr int kNS = 3;             // TMA ring depth (chunks in flight)
 // that is not tied to TMEM lane quarter 0 therefore runs on the other sub-partitions: the
 // cumulative sums on warp kCsWarp, w o x on the six math warps with warp % 4 != 0.
 constexpr int kCsWarp = 3;
+
+// dt_raw of steps 2 lane and 2 lane + 1 of the next kDtAhead chunks, as raw bf16 bits (the
+// loads land in their registers without a consumer in between, so nothing waits for them
+// until the chunk's cumulative sum is formed kDtAhead chunks later).  Slot = chunk mod
+// kDtAhead, chosen by a switch so that the array stays in registers.
+constexpr int kDtAhead = 4;
+struct DtRing {
+  uint32_t v[2 * kDtAhead];
+  __device__ __forceinline__ void load(int slot, const __nv_bfloat16* dt, int64_t row0, int64_t L,
+                                       int H, int h, int64_t t) {
+    const unsigned short* p = reinterpret_cast<const unsigned short*>(dt) + (row0 + t) * H + h;
+    switch (slot) {
+      case 0: v[0] = 0u; v[1] = 0u; if (t < L) v[0] = __ldg(p); if (t + 1 < L) v[1] = __ldg(p + H); break;
+      case 1: v[2] = 0u; v[3] = 0u; if (t < L) v[2] = __ldg(p); if (t + 1 < L) v[3] = __ldg(p + H); break;
+      case 2: v[4] = 0u; v[5] = 0u; if (t < L) v[4] = __ldg(p); if (t + 1 < L) v[5] = __ldg(p + H); break;
+      default: v[6] = 0u; v[7] = 0u; if (t < L) v[6] = __ldg(p); if (t + 1 < L) v[7] = __ldg(p + H); break;
+    }
+  }
+  __device__ __forceinline__ void take(int slot, float& d0, float& d1) const {
+    uint32_t r0, r1;
+    switch (slot) {
+      case 0: r0 = v[0]; r1 = v[1]; break;
+      case 1: r0 = v[2]; r1 = v[3]; break;
+      case 2: r0 = v[4]; r1 = v[5]; break;
+      default: r0 = v[6]; r1 = v[7]; break;
+    }
+    d0 = __uint_as_float(r0 << 16);
+    d1 = __uint_as_float(r1 << 16);
+  }
+};
+static_assert(kDtAhead == 4, "DtRing has four slots");
 constexpr int kPanel = kQ * 128;   // 64 rows of 128 bytes: one swizzled operand panel
 // bf16 planes of the masked G and of the state that C H^T reads.  The state takes two
 // (hi = bf16(H), lo = bf16(H - hi)): rounded once, its inter-chunk term C H^T carries an
@@ -223,7 +255,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     uint64_t* last_bar = nullptr;   // the barrier of the last commit, and its phase
     uint32_t last_par = 0;
     // G of chunk k into its parity buffer (the buffer's previous G, chunk k - 2, was masked
-    // before mg_ready of chunk k - 1, which this warp waited for)
+    // before mg_ready of chunk k - 2, which this warp waited for)
     auto issue_g = [&](int k) -> bool {
       const int s = k % kNS;
       const uint32_t st = sb + uint32_t(s * S::kStage);
@@ -268,11 +300,6 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
           }
       }
       __syncwarp();
-      // the next chunk's G runs while the math warps mask this chunk's
-      if (k + 1 < nck) {
-        good = issue_g(k + 1);
-        if (!good) break;
-      }
       good = __all_sync(0xffffffffu, mm::mbar_wait(mg_ready, uint32_t(k) & 1u, status));
       if (!good) break;
       if (lane == 0) {
@@ -299,6 +326,11 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
         last_par = uint32_t(k) & 1u;
       }
       __syncwarp();
+      // the next chunk's G runs while the math warps update the state
+      if (k + 1 < nck) {
+        good = issue_g(k + 1);
+        if (!good) break;
+      }
     }
     mm::named_bar_sync(0, kThreads);
     // nothing may still write TMEM when it is freed
@@ -376,21 +408,22 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
   };
   put_state();
 
-  // warp 0: dt_raw of steps 2 lane, 2 lane + 1 of a chunk, then Delta and the inclusive
-  // cumulative sum of Delta A (log2 units) over it into the chunk's parity buffer
-  float dtn0 = 0.f, dtn1 = 0.f;
-  auto load_dt = [&](int64_t c) {
-    const int64_t t = c * kQ + 2 * lane;
-    dtn0 = t < L ? __bfloat162float(a.dt[(b * L + t) * a.H + h]) : 0.f;
-    dtn1 = t + 1 < L ? __bfloat162float(a.dt[(b * L + t + 1) * a.H + h]) : 0.f;
+  // warp kCsWarp: dt_raw of steps 2 lane, 2 lane + 1 of a chunk (loaded kDtAhead chunks
+  // ahead), then Delta and the inclusive cumulative sum of Delta A (log2 units) over it into
+  // the chunk's buffer (k mod 3)
+  DtRing dtr;
+  auto load_dt = [&](int k) {   // chunk k of the segment into slot k mod kDtAhead
+    dtr.load(k % kDtAhead, a.dt, b * L, L, a.H, h, (c_begin + k) * kQ + 2 * lane);
   };
   auto chunk_cs = [&](int k) {   // warp kCsWarp; dt of chunk k loaded
     float* cs = cs_all + (k % 3) * kQ;
     float* dl = dl_all + (k % 3) * kQ;
     const int64_t t = (c_begin + k) * kQ + 2 * lane;
-    const float d0 = t < L ? mm::Math<false>::softplus(dtn0 + bias) : 0.f;
-    const float d1 = t + 1 < L ? mm::Math<false>::softplus(dtn1 + bias) : 0.f;
-    if (k + 1 < nck) load_dt(c_begin + k + 1);
+    float r0, r1;
+    dtr.take(k % kDtAhead, r0, r1);
+    const float d0 = t < L ? mm::Math<false>::softplus(r0 + bias) : 0.f;
+    const float d1 = t + 1 < L ? mm::Math<false>::softplus(r1 + bias) : 0.f;
+    if (k + kDtAhead < nck) load_dt(k + kDtAhead);
     const float e0 = d0 * A2, e1 = d1 * A2;
     float sum = e0 + e1;
 #pragma unroll
@@ -406,7 +439,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     dl[2 * lane + 1] = d1;
   };
   if (warp == kCsWarp && nck > 0) {
-    load_dt(c_begin);
+    for (int k = 0; k < kDtAhead && k < nck; ++k) load_dt(k);
     chunk_cs(0);
   }
 
@@ -565,6 +598,264 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
 #pragma unroll
     for (int i = 0; i < NH2; i += 4)
       *reinterpret_cast<float4*>(ho + i) = make_float4(H[i], H[i + 1], H[i + 2], H[i + 3]);
+  }
+}
+
+
+// ---------------------------------------------------------------------------------------
+// The state pass on the tensor cores: CTA z < nseg - 1 of row b, head h leaves the end state
+// of its segment started from zero, sum_k 2^(cs_last,k ...) U_k, in ws_H slot z and the
+// segment's summed Delta A log2 e in ws_A; segment 0 also copies h_in into slot nseg - 1 (the
+// main pass reads the carried-in state from there, so that its last segment may write h_out
+// over h_in).  Per chunk only U = (w o x)^T B runs (B and x tiles, no C), and the state
+// update H <- 2^cs_last H + U.  Same warp roles as the main pass; 82 KB of shared memory and
+// N TMEM columns, so two CTAs share an SM.
+template <int N>
+struct StateSmem {
+  static constexpr int NP = N / 64;
+  static constexpr int kB = 0;                     // B [64 s][N n]
+  static constexpr int kX = NP * kPanel;           // x [64 s][64 p]
+  static constexpr int kStage = (NP + 1) * kPanel;
+  static constexpr int kXw = kNS * kStage;         // w o x [64 s][64 p]
+  static constexpr int kCs = kXw + kPanel;         // [3][kQ] cs (log2 units)
+  static constexpr int kDl = kCs + 3 * kQ * 4;     // [3][kQ] Delta
+  static constexpr int kBar = kDl + 3 * kQ * 4;
+  // full[kNS], empty[kNS], u_done, mg_ready
+  static constexpr int kNBar = 2 * kNS + 2;
+  static constexpr int kTotal = kBar + 8 * kNBar + 16;
+  static constexpr int kDynamic = kTotal + 1024;
+  static constexpr uint32_t kTmemCols = N;         // U
+};
+
+template <int N>
+__global__ void __launch_bounds__(kThreads, 2)
+ssd_tc_state_kernel(const __grid_constant__ CUtensorMap tm_B,
+                    const __grid_constant__ CUtensorMap tm_x, const SsdArgs a, int* status) {
+  using S = StateSmem<N>;
+  constexpr int NP = S::NP;
+  constexpr int NH = N / kCS;
+  constexpr int NH2 = NH / 2;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = mm::smem_addr(smem_raw);
+  unsigned char* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sb = mm::smem_addr(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kNS;
+  uint64_t* u_done = bars + 2 * kNS;
+  uint64_t* mg_ready = u_done + 1;     // w o x is in shared memory
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + S::kNBar);
+  float* cs_all = reinterpret_cast<float*>(smem + S::kCs);
+  float* dl_all = reinterpret_cast<float*>(smem + S::kDl);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.x;
+  const int64_t b = blockIdx.y;
+  const int seg = blockIdx.z;
+  const int grp = h / (a.H / a.G);
+  const int64_t L = a.L;
+  const int64_t nchunks = (L + kQ - 1) / kQ;
+  const int64_t c_begin = int64_t(seg) * a.cps;
+  const int64_t c_end = c_begin + a.cps < nchunks ? c_begin + a.cps : nchunks;
+  const int nck = c_end > c_begin ? int(c_end - c_begin) : 0;
+  const int64_t bh = b * a.H + h;
+
+  if (tid == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mm::mbar_init(&full[i], 1);
+      mm::mbar_init(&empty[i], kMathWarps);
+    }
+    mm::mbar_init(u_done, 1);
+    mm::mbar_init(mg_ready, kMathWarps);
+  }
+  if (warp == kMmaWarp) {
+    mm::tmem_alloc(tmem_slot, S::kTmemCols);
+    mm::tmem_relinquish();
+  }
+  mm::tc_fence_before();
+  __syncthreads();
+  mm::tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == kCopyWarp) {
+    // ================================================================== copy warp
+    auto issue = [&](int k) {
+      const int s = k % kNS;
+      const int t0 = int((c_begin + k) * kQ);
+      const uint32_t st = sb + uint32_t(s * S::kStage);
+      mm::mbar_arrive_expect_tx(&full[s], uint32_t(S::kStage));
+      for (int pn = 0; pn < NP; ++pn)
+        mm::tma_load_4d(st + S::kB + pn * kPanel, &tm_B, &full[s], pn * 64, grp, t0, int(b), 1024,
+                        2, status);
+      mm::tma_load_4d(st + S::kX, &tm_x, &full[s], 0, h, t0, int(b), 1024, 2, status);
+    };
+    bool good = true;
+    if (lane == 0)
+      for (int k = 0; k < nck && k < kNS; ++k) issue(k);
+    int issued = nck < kNS ? nck : kNS;
+    __syncwarp();
+    for (int k = kNS; good && k < nck; ++k) {
+      good = __all_sync(0xffffffffu, mm::mbar_wait(&empty[(k - kNS) % kNS],
+                                                   uint32_t((k - kNS) / kNS) & 1u, status));
+      if (!good) break;
+      if (lane == 0) issue(k);
+      __syncwarp();
+      issued = k + 1;
+    }
+    mm::named_bar_sync(0, kThreads);
+    if (lane == 0)
+      for (int k = issued - kNS < 0 ? 0 : issued - kNS; k < issued; ++k)
+        mm::mbar_wait(&full[k % kNS], uint32_t(k / kNS) & 1u, nullptr);
+    __syncwarp();
+    return;
+  }
+
+  if (warp == kMmaWarp) {
+    // =================================================================== MMA warp
+    bool good = true;
+    int last = -1;   // the chunk of the last commit
+    for (int k = 0; good && k < nck; ++k) {
+      const int s = k % kNS;
+      const uint32_t st = sb + uint32_t(s * S::kStage);
+      // U_k overwrites U_{k-1}: the math warps read it before they signalled mg_ready of k
+      good = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status)) &&
+             __all_sync(0xffffffffu, mm::mbar_wait(mg_ready, uint32_t(k) & 1u, status));
+      if (!good) break;
+      if (lane == 0) {
+        mm::tc_fence_after();
+        constexpr uint32_t idU = mm::umma_idesc_bf16_f32_mj<64, N, 1, 1>();
+        const uint32_t dw = mm::umma_desc_lo(sb + S::kXw, kPanel);
+        const uint32_t dbm = mm::umma_desc_lo(st + S::kB, kPanel);
+#pragma unroll
+        for (int kk = 0; kk < kQ / 16; ++kk)
+          mm::umma_bf16_lo(tbase, dw + uint32_t(kk * 2048 >> 4), dbm + uint32_t(kk * 2048 >> 4),
+                           idU, kk > 0 ? 1u : 0u);
+        mm::umma_commit(u_done);
+      }
+      __syncwarp();
+      last = k;
+    }
+    mm::named_bar_sync(0, kThreads);
+    // nothing may still write TMEM when it is freed
+    if (lane == 0 && last >= 0) mm::mbar_wait(u_done, uint32_t(last) & 1u, nullptr);
+    __syncwarp();
+    mm::tc_fence_after();
+    mm::tmem_dealloc(tbase, S::kTmemCols);
+    return;
+  }
+
+  // ================================================================== math warps
+  const int q = warp & 3, hf = warp >> 2;
+  const int part = lane >> 4;
+  const int r = 16 * q + (lane & 15);
+  const uint32_t tq = tbase + (uint32_t(32 * q) << 16);
+  const float A2 = -expf(a.A_log[h]) * mm::kLog2e;
+  const float bias = a.dt_bias[h];
+  const int ncol0 = hf * NH + part * NH2;
+  const int64_t col0 = int64_t(r) * N + ncol0;
+
+  if (seg == 0 && a.h_in) {   // the copy of h_in the main pass starts from
+    const float* hi = a.h_in + bh * int64_t(kP * N);
+    float* hc = a.ws_H + (bh * a.nseg + a.nseg - 1) * int64_t(kP * N);
+#pragma unroll
+    for (int i = 0; i < NH2; i += 4)
+      *reinterpret_cast<float4*>(hc + col0 + i) = *reinterpret_cast<const float4*>(hi + col0 + i);
+  }
+  float H[NH2];
+#pragma unroll
+  for (int i = 0; i < NH2; ++i) H[i] = 0.0f;
+  float seg_a = 0.0f;
+
+  DtRing dtr;
+  auto load_dt = [&](int k) {   // chunk k of the segment into slot k mod kDtAhead
+    dtr.load(k % kDtAhead, a.dt, b * L, L, a.H, h, (c_begin + k) * kQ + 2 * lane);
+  };
+  auto chunk_cs = [&](int k) {   // warp kCsWarp; dt of chunk k loaded
+    float* cs = cs_all + (k % 3) * kQ;
+    float* dl = dl_all + (k % 3) * kQ;
+    const int64_t t = (c_begin + k) * kQ + 2 * lane;
+    float r0, r1;
+    dtr.take(k % kDtAhead, r0, r1);
+    const float d0 = t < L ? mm::Math<false>::softplus(r0 + bias) : 0.f;
+    const float d1 = t + 1 < L ? mm::Math<false>::softplus(r1 + bias) : 0.f;
+    if (k + kDtAhead < nck) load_dt(k + kDtAhead);
+    const float e0 = d0 * A2, e1 = d1 * A2;
+    float sum = e0 + e1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const float v = __shfl_up_sync(0xffffffffu, sum, o);
+      if (lane >= o) sum += v;
+    }
+    float ex = __shfl_up_sync(0xffffffffu, sum, 1);
+    if (lane == 0) ex = 0.f;
+    cs[2 * lane] = ex + e0;
+    cs[2 * lane + 1] = ex + e0 + e1;
+    dl[2 * lane] = d0;
+    dl[2 * lane + 1] = d1;
+  };
+  if (warp == kCsWarp && nck > 0) {
+    for (int k = 0; k < kDtAhead && k < nck; ++k) load_dt(k);
+    chunk_cs(0);
+  }
+
+  bool ok = true;
+  for (int k = 0; k < nck; ++k) {
+    const int s = k % kNS;
+    const uint32_t st = sb + uint32_t(s * S::kStage);
+    const float* cs = cs_all + (k % 3) * kQ;
+    const float* dl = dl_all + (k % 3) * kQ;
+    ok = bar_and(1, 32 * kMathWarps, ok);      // this chunk's cs and Delta visible
+    if (!ok) break;
+    const float csl = cs[kQ - 1];
+    seg_a += csl;
+    ok = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status));
+    if (!ok) continue;
+    // w o x, w_s = 2^(cs_last - cs_s) Delta_s, in 8-element pieces: the 192 threads of the
+    // math warps off sub-partition 0 take pieces u, u + 192, ...
+    if (q != 0) {
+      const int u = (warp - 1 - (warp >> 2)) * 32 + lane;
+      for (int pc = u; pc < kQ * kP / 8; pc += 6 * 32) {
+        const int row = pc >> 3;
+        const float w = mm::ex2_approx(csl - cs[row]) * dl[row];
+        const uint32_t off = pofs(row, (pc & 7) * 8);
+        const uint4 v = lds_u128(st + S::kX + off);
+        uint4 o;
+        o.x = pack_bf16(w * bf16_lo(v.x), w * bf16_hi(v.x));
+        o.y = pack_bf16(w * bf16_lo(v.y), w * bf16_hi(v.y));
+        o.z = pack_bf16(w * bf16_lo(v.z), w * bf16_hi(v.z));
+        o.w = pack_bf16(w * bf16_lo(v.w), w * bf16_hi(v.w));
+        sts_u128(sb + S::kXw + off, o);
+      }
+    }
+    mm::fence_async_shared();
+    mm::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mm::mbar_arrive(mg_ready);
+    if (warp == kCsWarp && k + 1 < nck) chunk_cs(k + 1);   // read by all after the next barrier
+
+    ok = __all_sync(0xffffffffu, mm::mbar_wait(u_done, uint32_t(k) & 1u, status));
+    if (!ok) continue;
+    mm::tc_fence_after();
+    {
+      const float dec = mm::ex2_approx(csl);
+      float u[NH2];
+      ld_half(tq + uint32_t(hf * NH), u);
+      mm::tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < NH2; ++i) H[i] = fmaf(dec, H[i], u[i]);
+    }
+    mm::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mm::mbar_arrive(&empty[s]);   // the stage's tiles and U are read
+  }
+  if (nck > 0) ok = bar_and(1, 32 * kMathWarps, ok);
+  mm::named_bar_sync(0, kThreads);
+  if (ok && seg < a.nseg - 1) {
+    float* out = a.ws_H + (bh * a.nseg + seg) * int64_t(kP * N) + col0;
+#pragma unroll
+    for (int i = 0; i < NH2; i += 4)
+      *reinterpret_cast<float4*>(out + i) = make_float4(H[i], H[i + 1], H[i + 2], H[i + 3]);
+    if (tid == 0) a.ws_A[bh * (a.nseg - 1) + seg] = seg_a;
   }
 }
 
