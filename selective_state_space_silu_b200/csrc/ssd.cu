@@ -62,36 +62,38 @@ bool overlap(const Range& a, const Range& b) {
 
 // Time segments: with few (batch row, head) pairs, each pair's chunks are cut into
 // segments that run as separate CTAs (a state pass over segments 0 .. nseg - 2 first).
-// With fewer pairs than resident main-pass CTAs (2 per SM on the 148 SMs), the count
-// minimises (waves of main-pass CTAs) x (chunks per segment), the fewest segments on a tie
-// (each extra one adds state-pass and fold work).
-// Measured (B200, 24 heads x 64, d_state 128): 8 x 2048 steps -> 3 segments, 165 us (2: 204,
-// 6: 200); 2 x 8192 -> 6 segments, 189 us (12: 200, 16: 218).
+// Measured (B200, 24 heads x 64, d_state 128): 8 x 2048 steps -> 1 segment, 125 us (2: 131,
+// 3: 138); 2 x 8192 -> 6 segments, 129 us (3: 139, 8: 160).
 struct SegPlan {
   int nseg, cps;
 };
 
 constexpr int64_t kSms = 148;
 
-constexpr int64_t kMainSlots = 2 * kSms;  // main-pass CTAs resident at once (mma.sync pass)
-
-// Rows without document resets take the tensor-core main pass (one CTA per SM: 9 warps of
-// 168 registers; for d_state 128 also 138 KB of shared memory and 512 TMEM columns); both
-// passes use the same segment plan (at one CTA per SM its segments make about 2 waves more).
+// Rows without document resets take the tensor-core passes (main pass: one CTA per SM, 10
+// warps, 170 KB of shared memory for d_state 128 and 512 TMEM columns).
 bool use_tc(const int32_t* seq_idx) { return seq_idx == nullptr; }
 
+// Time segments.  One plan serves both passes (the workspace query does not know whether
+// document ids will be given); it is set by the tensor-core passes, which take every row
+// without document resets.  Their cost, measured on B200 (d_state 128, 64-step chunks): a
+// main-pass CTA (one per SM) takes about (5.3 + c) x 1.675 us for c chunks, a state-pass CTA
+// (two per SM) about c x 1.5 us.  The plan minimises the waves of both passes times those
+// costs over 1..16 segments, the fewest segments on a tie.
 SegPlan seg_plan(int64_t Bt, int64_t L, int64_t H) {
   const int64_t nchunks = (L + ssd::kQ - 1) / ssd::kQ;
   const int64_t pairs = Bt * H;
-  // pairs that fill the resident slots by themselves gain nothing from a split
-  if (nchunks <= 1 || pairs <= 0 || pairs >= kMainSlots) return {1, int(nchunks > 0 ? nchunks : 1)};
-  int64_t best_cost = -1, best_n = 1, best_cps = nchunks;
+  if (nchunks <= 1 || pairs <= 0) return {1, int(nchunks > 0 ? nchunks : 1)};
+  double best_cost = -1.0;
+  int64_t best_n = 1, best_cps = nchunks;
   for (int64_t n = 1; n <= 16 && n <= nchunks; ++n) {
     const int64_t cps = (nchunks + n - 1) / n;
     const int64_t n_eff = (nchunks + cps - 1) / cps;
-    const int64_t waves = (pairs * n_eff + kMainSlots - 1) / kMainSlots;
-    const int64_t cost = waves * cps;
-    if (best_cost < 0 || cost < best_cost) {
+    const int64_t main_waves = (pairs * n_eff + kSms - 1) / kSms;
+    const int64_t state_waves = n_eff > 1 ? (pairs * (n_eff - 1) + 2 * kSms - 1) / (2 * kSms) : 0;
+    const double cost = double(main_waves) * (5.3 + double(cps)) * 1.675 +
+                        double(state_waves) * double(cps) * 1.5;
+    if (best_cost < 0.0 || cost < best_cost - 1e-9) {
       best_cost = cost;
       best_n = n_eff;
       best_cps = cps;

@@ -122,9 +122,10 @@ def _nseg(lib, **kw):
 
 
 def test_segment_plan(lib):
-    # fewer (row, head) pairs than resident main-pass CTAs (2 per SM x 148): minimise
-    # waves x chunks per segment, fewest segments on a tie; otherwise no split
-    assert _nseg(lib, batch=8, seqlen=2048, nheads=24) == 3
+    # the plan minimises the modelled time of the tensor-core passes: main-pass waves (one CTA
+    # per SM, 148 SMs) x (5.3 + chunks per segment) x 1.675 us plus state-pass waves (two CTAs
+    # per SM) x chunks per segment x 1.5 us, fewest segments on a tie
+    assert _nseg(lib, batch=8, seqlen=2048, nheads=24) == 1       # 192 pairs: 2 waves, no state pass
     assert _nseg(lib, batch=2, seqlen=8192, nheads=24) == 6
     assert _nseg(lib, batch=1, seqlen=640, nheads=2) == 10        # 10 chunks, one each
     assert _nseg(lib, batch=1, seqlen=65536, nheads=2) == 16      # at most 16
