@@ -6,7 +6,7 @@
 // and H [headdim p x d_state n] the state entering the chunk:
 //   G  = C B^T                                   (M 64 t, N 64 s, K n)       K-major A and B
 //   Y1 = C H^T        (H as bf16 hi + lo planes)  (M 64 t, N 64 p, K n)       K-major A and B
-//   Y2 = (M o G) x    (M o G rounded to bf16)     (M 64 t, N 64 p, K 64 s)    x MN-major
+//   Y2 = (M o G) x    (M o G as hi + lo planes)   (M 64 t, N 64 p, K 64 s)    x MN-major
 //   U  = (w o x)^T B  (w o x rounded to bf16)     (M 64 p, N n, K 64 s)       both MN-major
 //   y_t = 2^cs_t Y1[t] + Y2[t] + D x_t (times SiLU(z_t)),   H <- 2^cs_last H + U
 // with M[t, s] = 2^(cs_t - cs_s) Delta_s for s <= t and w_s = 2^(cs_last - cs_s) Delta_s.
@@ -19,7 +19,7 @@
 //     3-deep ring, refilling a stage as soon as the math warps release it;
 //   warp 8 (MMA warp): lane 0 issues every tcgen05.mma, committing each group to an mbarrier;
 //   warps 0..7 (math warps, warp w reads TMEM lanes 32 (w mod 4) .. + 31, column half w / 4):
-//     Delta and cs (warp 3), the mask of G into a bf16 plane and w o x, the outputs from
+//     Delta and cs (warp 3), the mask of G into bf16 hi/lo planes and w o x, the outputs from
 //     Y1 and Y2, and the state: H is held in registers (row p = 16 (w mod 4) + lane mod 16,
 //     a quarter of the n columns per lane), updated from U and written back as the hi/lo
 //     bf16 planes that the next chunk's C H^T reads.  An M = 64 accumulator's rows sit in lanes
@@ -33,9 +33,9 @@
 //   update the state, C H^T of chunk k + 1 runs while they mask G_{k+1}, and the copies are
 //   left to their own warp.  G, Y1 and Y2 are
 //   double-buffered in TMEM, the tiles triple-buffered in shared memory.
-// Numerics: bf16 inputs enter exactly; the masked G and w o x are each rounded once to bf16
-// (round to nearest), the state used by C H^T enters as a hi + lo bf16 pair; accumulation
-// is fp32 and the carried state itself stays fp32 in registers.
+// Numerics: bf16 inputs enter exactly; the masked G and the state used by C H^T enter as
+// hi + lo bf16 pairs, w o x is rounded once to bf16 (round to nearest); accumulation is fp32
+// and the carried state itself stays fp32 in registers.
 //
 // Every wait is bounded: a warp that gives up records MAMBA_ERR_TIMEOUT in *status and leaves
 // its loop; the copy warp waits (bounded) for its copies in flight and the MMA warp for its
@@ -97,12 +97,12 @@ struct DtRing {
 };
 static_assert(kDtAhead == 4, "DtRing has four slots");
 constexpr int kPanel = kQ * 128;   // 64 rows of 128 bytes: one swizzled operand panel
-// bf16 planes of the masked G and of the state that C H^T reads.  The state takes two
-// (hi = bf16(H), lo = bf16(H - hi)): rounded once, its inter-chunk term C H^T carries an
-// error of 2^-9 times |C| |H| summed over d_state, which with a carried-in state of order one
-// and d_state 128 exceeds the output tolerance (measured: 1 element in 82k at 1.5x the bound).
-// The masked G takes one.
-constexpr int kMGPl = 1;
+// bf16 planes of the masked G and of the state that C H^T reads: two each (hi = bf16(v),
+// lo = bf16(v - hi)).  Rounded once, either term carries an error of 2^-9 times the sum of
+// its products' magnitudes, which with a carried-in state of order one and d_state 128
+// exceeds the output tolerance on rare elements (measured: one plane for the state, 1 element
+// in 82k at 1.5x the bound; one plane for the masked G, 1 in 422k at 1.2x).
+constexpr int kMGPl = 2;
 constexpr int kHPl = 2;
 
 template <int N>
@@ -504,7 +504,7 @@ ssd_tc_kernel(const __grid_constant__ CUtensorMap tm_C, const __grid_constant__ 
     if (!ok) break;
     const float csl = cs[kQ - 1];
 
-    // ---- the mask of G: M[t, s] = G[t, s] 2^(cs_t - cs_s) Delta_s for s <= t, in bf16
+    // ---- the mask of G: M[t, s] = G[t, s] 2^(cs_t - cs_s) Delta_s for s <= t, as hi/lo planes
     ok = __all_sync(0xffffffffu, mm::mbar_wait(&full[s], uint32_t(k / kNS) & 1u, status)) &&
          __all_sync(0xffffffffu, mm::mbar_wait(&g_done[k & 1], uint32_t(k >> 1) & 1u, status));
     if (!ok) continue;

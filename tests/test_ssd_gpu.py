@@ -51,6 +51,10 @@ CASES = [
     (1, 1, 2, 64, 1, True, True),
     (2, 200, 8, 128, 4, False, False),
     (1, 640, 2, 128, 1, True, True),
+    # time segments (state pass) at d_state 64 with a carried-in state
+    (1, 300, 2, 64, 1, False, True),
+    # segments over a ragged last chunk (1100 = 17 x 64 + 12), gated, carried-in state
+    (2, 1100, 3, 128, 1, True, True),
 ]
 
 
