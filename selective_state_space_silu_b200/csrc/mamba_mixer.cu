@@ -448,19 +448,47 @@ size_t bwd_workspace_for(const mamba_dims* d) { return bwd_layout(d, make_plan(d
 // out is recorded here (one word per context; mamba_mixer_step_check reads and clears it).
 static __device__ int g_step_status;
 
+// SMs of device `dev`, looked up once per device.
+int sm_count(int dev) {
+  static std::atomic<int> cache[64];
+  if (dev < 0 || dev >= 64) return 148;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+  }
+  return v;
+}
+
 template <int N, typename IO, bool P>
 cudaError_t launch_step(mm::StepArgs& a, cudaStream_t st) {
-  // short row runs over many CTAs (about 32 per SM over the whole grid) with a 2-deep ring
-  // measured fastest on 256 x 5120: 40.9 us, against 43.1 (16 per SM), 41.5 (64), 49.2
-  // (4 per SM, 4 stages) and 59.5 (4 per SM, 6 stages)
+  // About one wave: (channel block, row slice) CTAs of ceil(batch x blocks / resident CTAs)
+  // rows each, walking their rows through the 2-deep ring.  Measured on 256 x 5120 (10
+  // resident CTAs per SM, so 14 rows per CTA): 34.9 us, against 36.0 with 15 rows (a
+  // strict single wave, whose last slice holds one row), 35.4 at 7 rows, 36.7 at 5 rows
+  // (about 32 CTAs per SM, 2.8 waves), 41.4 at 12 rows (1.2 waves).
+  auto kern = mm::step_kernel<N, IO, P>;
+  constexpr int smem = mm::StepSmem<N, IO>::kTotal;
+  static std::atomic<int> per_sm{0};   // resident CTAs per SM of this instantiation
+  int occ = per_sm.load(std::memory_order_relaxed);
+  if (occ == 0) {
+    const cudaError_t e =
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, mm::kStepThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (occ < 1) occ = 1;
+    per_sm.store(occ, std::memory_order_relaxed);
+  }
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
   const int64_t nblk = (a.Di + mm::kStepCh - 1) / mm::kStepCh;
-  constexpr int64_t kCtasPerSm = 32;
-  int64_t rows = (a.batch * nblk + kCtasPerSm * 148 - 1) / (kCtasPerSm * 148);
+  const int64_t slots = int64_t(occ) * sm_count(dev);
+  int64_t rows = (a.batch * nblk + slots - 1) / slots;
   if (rows < 1) rows = 1;
   a.rows_per_cta = int(rows);
   const int64_t slices = (a.batch + rows - 1) / rows;
-  mm::step_kernel<N, IO, P><<<dim3(unsigned(nblk), unsigned(slices)), mm::kStepThreads,
-                              mm::StepSmem<N, IO>::kTotal, st>>>(a);
+  kern<<<dim3(unsigned(nblk), unsigned(slices)), mm::kStepThreads, smem, st>>>(a);
   return cudaGetLastError();
 }
 
