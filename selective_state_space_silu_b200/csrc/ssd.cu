@@ -489,8 +489,12 @@ extern "C" MAMBA_API int mamba2_gated_rmsnorm(const mamba2_dims* dims, const voi
   const int64_t items = rows * G;
   const int64_t grid = (items + ssd::kNormWarps - 1) / ssd::kNormWarps;
   if (grid > 0x7fffffff) return ssd_fail(MAMBA_ERR_UNSUPPORTED, "too many rows for one launch");
-  ssd::gated_rmsnorm_kernel<<<unsigned(grid), ssd::kNormWarps * 32, 0,
-                              static_cast<cudaStream_t>(cuda_stream)>>>(a);
+  if (a.gs <= 32 * 8 * ssd::kNormCachedUnits)
+    ssd::gated_rmsnorm_kernel<true><<<unsigned(grid), ssd::kNormWarps * 32, 0,
+                                      static_cast<cudaStream_t>(cuda_stream)>>>(a);
+  else
+    ssd::gated_rmsnorm_kernel<false><<<unsigned(grid), ssd::kNormWarps * 32, 0,
+                                       static_cast<cudaStream_t>(cuda_stream)>>>(a);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return ssd_fail(MAMBA_ERR_CUDA, "norm launch failed: %s", cudaGetErrorString(e));
   return ssd_ok();

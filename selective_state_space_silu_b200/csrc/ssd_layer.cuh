@@ -156,10 +156,14 @@ struct NormArgs {
 };
 
 constexpr int kNormWarps = 8;
+constexpr int kNormCachedUnits = 8;   // 16-byte units per lane kept in registers (gs <= 2048)
 
 // Grid ceil(rows * (D / gs) / kNormWarps) CTAs of kNormWarps warps; one warp per (row,
-// group): sum of (y SiLU(z))^2 over the group, then the scaled output (the second pass
-// re-reads the group's 4 gs bytes from cache).
+// group): sum of (y SiLU(z))^2 over the group, then the scaled output.  kCached (groups of
+// at most 32 kNormCachedUnits 8-channel units): every load of the group is issued up front
+// and y SiLU(z) stays in registers for the output; otherwise the second pass re-reads the
+// group's 4 gs bytes from cache.
+template <bool kCached>
 __global__ void __launch_bounds__(kNormWarps * 32) gated_rmsnorm_kernel(const NormArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t item = int64_t(blockIdx.x) * kNormWarps + (threadIdx.x >> 5);
@@ -171,6 +175,52 @@ __global__ void __launch_bounds__(kNormWarps * 32) gated_rmsnorm_kernel(const No
   const __nv_bfloat16* zr = a.z + row * a.D + c0;
   const int units = a.gs / 8;
   float ss = 0.f;
+  if constexpr (kCached) {
+    uint4 yc[kNormCachedUnits], zc[kNormCachedUnits];
+#pragma unroll
+    for (int i = 0; i < kNormCachedUnits; ++i) {
+      const int u = lane + 32 * i;
+      if (u < units) {
+        yc[i] = __ldg(reinterpret_cast<const uint4*>(yr) + u);
+        zc[i] = __ldg(reinterpret_cast<const uint4*>(zr) + u);
+      }
+    }
+    float g[kNormCachedUnits][8];
+#pragma unroll
+    for (int i = 0; i < kNormCachedUnits; ++i) {
+      const int u = lane + 32 * i;
+      if (u < units) {
+        float yv[8], zv[8];
+        bf16x8_to_f32(yc[i], yv);
+        bf16x8_to_f32(zc[i], zv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          g[i][e] = yv[e] * mm::Math<false>::silu(zv[e]);
+          ss = fmaf(g[i][e], g[i][e], ss);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = rsqrtf(ss / float(a.gs) + a.eps);
+#pragma unroll
+    for (int i = 0; i < kNormCachedUnits; ++i) {
+      const int u = lane + 32 * i;
+      if (u < units) {
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(a.w + c0) + 2 * u);
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(a.w + c0) + 2 * u + 1);
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __nv_bfloat162 pk = __floats2bfloat162_rn(g[i][2 * k] * r * wv[2 * k],
+                                                          g[i][2 * k + 1] * r * wv[2 * k + 1]);
+          o[k] = *reinterpret_cast<const uint32_t*>(&pk);
+        }
+        reinterpret_cast<uint4*>(a.out + row * a.D + c0)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  } else {
   for (int u = lane; u < units; u += 32) {
     float yv[8], zv[8];
     bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(yr) + u), yv);
@@ -200,6 +250,7 @@ __global__ void __launch_bounds__(kNormWarps * 32) gated_rmsnorm_kernel(const No
       o[k] = *reinterpret_cast<const uint32_t*>(&pk);
     }
     reinterpret_cast<uint4*>(a.out + row * a.D + c0)[u] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
   }
 }
 
