@@ -89,9 +89,14 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_kernel(const ConvArgs 
   else { dst = a.C; dstride = a.GN; dc = c0 - a.DI - a.GN; }
   dst += b * a.L * dstride + dc;
 
+  // step t + 1's input is requested before step t's math (one more load in flight per
+  // thread; two ahead cost registers and measured slower: 61.8 against 49.6 us)
+  uint4 nxt = t0 < t1 ? __ldg(reinterpret_cast<const uint4*>(xr + t0 * a.Cc)) : make_uint4(0, 0, 0, 0);
   for (int64_t t = t0; t < t1; ++t) {
     float cur[8];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(xr + t * a.Cc)), cur);
+    const uint4 raw = nxt;
+    if (t + 1 < t1) nxt = __ldg(reinterpret_cast<const uint4*>(xr + (t + 1) * a.Cc));
+    bf16x8_to_f32(raw, cur);
     float m0 = 1.f, m1 = 1.f, m2 = 1.f;  // live taps t-3, t-2, t-1
     if constexpr (kSeq) {
       if (t >= 1 && ids[t] != ids[t - 1]) lr = t;
